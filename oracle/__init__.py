@@ -1,0 +1,152 @@
+"""CKDA fp64 CPU oracle -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The
+product path (``delta_rule_linear_ckda_b200``) never imports it, and it never
+imports the product path: the two share no code.
+
+Contents
+--------
+``forward`` / ``decode_step``
+    Thin ctypes wrappers around ``ckda_oracle.c``: the sequential CKDA
+    recurrence in fp64, token by token,
+    ``S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T``,
+    ``o_t = S_t^T q_t`` ("Complex KDA ..." page, section "Complex KDA (CKDA)
+    Mimarisi ve Parametre Genislemesi"; "Gated DeltaNet-2" page, Methodology
+    section 1 with b_t = w_t = beta_t).
+``chunked`` (submodule)
+    A plain numpy fp64 restatement of the chunkwise WY form, used only to pin
+    the chunked algorithm against the sequential loop on tiny inputs.
+
+Inputs are upcast exactly to fp64 (bf16 and fp32 values are representable),
+so the oracle consumes bit-identical values to the CUDA path.  Parity
+status of every function is listed in the test-suite module docstrings; all
+functions here are pinned (no "parity unpinned" entries).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ckda_oracle.c")
+_LIB = os.path.join(_HERE, "libckda_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``ckda_oracle.c`` with gcc into ``libckda_oracle.so``."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lpthread"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            dp = ctypes.POINTER(ctypes.c_double)
+            i64 = ctypes.c_int64
+            lib.ckda_oracle_forward.argtypes = [
+                i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int64),
+                dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
+            ]
+            lib.ckda_oracle_forward.restype = ctypes.c_int
+            lib.ckda_oracle_decode_step.argtypes = [
+                i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
+            ]
+            lib.ckda_oracle_decode_step.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    """Exact upcast to a contiguous fp64 numpy array (torch or numpy input)."""
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().to("cpu")
+        import torch
+
+        x = x.to(torch.float64).numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def forward(q, k, v, alpha, beta, S0=None, cu_seqlens=None, n_threads=None):
+    """Sequential fp64 CKDA forward.
+
+    Fixed-length batch: q, k, alpha ``[B, T, H, dk]``, v ``[B, T, H, dv]``,
+    beta ``[B, T, H]``.  Packed batch: pass ``cu_seqlens`` (``[N+1]``) and
+    tensors ``[T_total, H, d]`` (a leading 1 is accepted).  ``S0`` is
+    ``[N, H, dk, dv]`` or None (zero state).
+
+    Returns ``(out, S_final)`` as fp64 numpy arrays, ``out`` shaped like ``v``.
+    """
+    qd, kd, vd, ad, bd = (_f64(t) for t in (q, k, v, alpha, beta))
+    out_shape = vd.shape
+    if cu_seqlens is None:
+        if qd.ndim != 4:
+            raise ValueError("fixed-length batch expects [B, T, H, d] tensors")
+        B, T, H, dk = qd.shape
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int64))
+        if qd.ndim == 4:
+            if qd.shape[0] != 1:
+                raise ValueError("packed batch expects a leading dimension of 1")
+            qd, kd, vd, ad, bd = qd[0], kd[0], vd[0], ad[0], bd[0]
+        H, dk = qd.shape[1], qd.shape[2]
+    N = len(cu) - 1
+    dv = vd.shape[-1]
+    T_total = int(cu[-1])
+    qd, kd, ad = (x.reshape(T_total, H, dk) for x in (qd, kd, ad))
+    vd = vd.reshape(T_total, H, dv)
+    bd = bd.reshape(T_total, H)
+    S0d = None if S0 is None else _f64(S0).reshape(N, H, dk, dv)
+    out = np.zeros((T_total, H, dv), dtype=np.float64)
+    S_final = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().ckda_oracle_forward(
+        N, H, dk, dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(qd), _ptr(kd), _ptr(vd), _ptr(ad), _ptr(bd), _ptr(S0d),
+        _ptr(out), _ptr(S_final), int(n_threads or default_threads()),
+    )
+    if rc != 0:
+        raise ValueError("ckda_oracle_forward rejected its arguments")
+    return out.reshape(out_shape), S_final
+
+
+def decode_step(q, k, v, alpha, beta, S, n_threads=None):
+    """One fp64 recurrent step: q, k, alpha ``[B, H, dk]``, v ``[B, H, dv]``,
+    beta ``[B, H]``, S ``[B, H, dk, dv]``.  Returns ``(out, S_new)``."""
+    qd, kd, vd, ad, bd = (_f64(t) for t in (q, k, v, alpha, beta))
+    Sd = _f64(S).copy()
+    B, H, dk = qd.shape
+    dv = vd.shape[-1]
+    out = np.zeros((B, H, dv), dtype=np.float64)
+    rc = _load().ckda_oracle_decode_step(
+        B, H, dk, dv, _ptr(qd), _ptr(kd), _ptr(vd), _ptr(ad), _ptr(bd), _ptr(Sd),
+        _ptr(out), int(n_threads or default_threads()),
+    )
+    if rc != 0:
+        raise ValueError("ckda_oracle_decode_step rejected its arguments")
+    return out, Sd

@@ -1,0 +1,171 @@
+/*
+ * CKDA fp64 CPU oracle -- TEST INFRASTRUCTURE ONLY.
+ *
+ * This file is the slow, obviously correct reference for the Complex Kimi
+ * Delta Attention (CKDA) recurrence.  Only the test suite, the package's
+ * smoke check and the CPU-baseline leg of the benchmark may load it.  It
+ * shares no code with the CUDA path and includes no CUDA header.
+ *
+ * What it computes (per sequence n and head h, all arithmetic in fp64):
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = S_t^T q_t                         (read-out after the update)
+ *
+ * Sources:
+ *  - "Complex KDA: Kimi Delta Attention Mimarisinin Ifade Gucunu Anlamak ve
+ *    Gelistirmek", section "Complex KDA (CKDA) Mimarisi ve Parametre
+ *    Genislemesi": per-channel gate alpha in [-1, 1], delta coefficient
+ *    beta in [0, 2], diagonal-plus-rank-one transition.
+ *  - "Gated DeltaNet-2" technical summary, Methodology section 1, the state
+ *    equation S_t = (I - k_t (b_t . k_t)^T) D_t S_{t-1} + k_t (w_t . v_t)^T
+ *    with D_t = Diag(alpha_t); tying b_t = w_t = beta_t gives the form above.
+ *  - "Semidirect Fourier Delta Attention (SFDA)" technical summary,
+ *    "Arquitectura Central" equation with zero phase (Lambda_t = diag(alpha_t)).
+ *  The read-out o_t = S_t^T q_t is not printed on those pages; the plainest
+ *  reading (post-update state, no query scale) is used.
+ *
+ * The per-token body is written exactly in the order of the equation:
+ *   1. S <- Diag(alpha) S            (scale row i by alpha_i)
+ *   2. r <- S^T k                    (read the current association of k)
+ *   3. S <- S + beta k (v - r)^T     ((I - beta k k^T) S' + beta k v^T)
+ *   4. o <- S^T q
+ *
+ * Layouts (row-major, contiguous):
+ *   q, k, alpha : [T_total, H, dk]     v, out : [T_total, H, dv]
+ *   beta        : [T_total, H]
+ *   S0, S_final : [N, H, dk, dv]       (S0 may be NULL: zero initial state)
+ *   cu_seqlens  : int64 [N + 1], sequence n spans tokens [cu[n], cu[n+1])
+ */
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef struct {
+    int64_t n_seqs, H, dk, dv;
+    const int64_t *cu;
+    const double *q, *k, *v, *alpha, *beta, *S0;
+    double *out, *S_final;
+    int64_t next_unit; /* shared work counter (guarded by lock) */
+    pthread_mutex_t lock;
+} oracle_job;
+
+/* One (sequence, head) unit: the sequential recurrence, token by token. */
+static void run_unit(const oracle_job *J, int64_t n, int64_t h, double *S,
+                     double *r) {
+    const int64_t H = J->H, dk = J->dk, dv = J->dv;
+    if (J->S0) {
+        memcpy(S, J->S0 + ((n * H + h) * dk) * dv, sizeof(double) * dk * dv);
+    } else {
+        memset(S, 0, sizeof(double) * dk * dv);
+    }
+    for (int64_t t = J->cu[n]; t < J->cu[n + 1]; ++t) {
+        const double *q = J->q + (t * H + h) * dk;
+        const double *k = J->k + (t * H + h) * dk;
+        const double *a = J->alpha + (t * H + h) * dk;
+        const double *v = J->v + (t * H + h) * dv;
+        const double b = J->beta[t * H + h];
+        double *o = J->out + (t * H + h) * dv;
+
+        /* 1. S <- Diag(alpha) S */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) S[i * dv + j] *= a[i];
+        /* 2. r <- S^T k */
+        for (int64_t j = 0; j < dv; ++j) r[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * k[i];
+        /* 3. S <- S + beta k (v - r)^T */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j)
+                S[i * dv + j] += b * k[i] * (v[j] - r[j]);
+        /* 4. o <- S^T q */
+        for (int64_t j = 0; j < dv; ++j) o[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) o[j] += S[i * dv + j] * q[i];
+    }
+    if (J->S_final)
+        memcpy(J->S_final + ((n * H + h) * dk) * dv, S,
+               sizeof(double) * dk * dv);
+}
+
+static void *worker(void *arg) {
+    oracle_job *J = (oracle_job *)arg;
+    double *S = (double *)malloc(sizeof(double) * J->dk * J->dv);
+    double *r = (double *)malloc(sizeof(double) * J->dv);
+    const int64_t n_units = J->n_seqs * J->H;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        int64_t u = J->next_unit++;
+        pthread_mutex_unlock(&J->lock);
+        if (u >= n_units) break;
+        run_unit(J, u / J->H, u % J->H, S, r);
+    }
+    free(S);
+    free(r);
+    return NULL;
+}
+
+/*
+ * Sequential CKDA forward over a packed batch.  Returns 0 on success, -1 on
+ * an argument error (bad sizes or offsets).  Units of (sequence, head) are
+ * independent and are shared out to `n_threads` host threads; the result
+ * does not depend on the thread count.
+ */
+int ckda_oracle_forward(int64_t n_seqs, int64_t H, int64_t dk, int64_t dv,
+                        const int64_t *cu_seqlens, const double *q,
+                        const double *k, const double *v, const double *alpha,
+                        const double *beta, const double *S0, double *out,
+                        double *S_final, int n_threads) {
+    if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens)
+        return -1;
+    if (cu_seqlens[0] != 0) return -1;
+    for (int64_t n = 0; n < n_seqs; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    oracle_job J;
+    J.n_seqs = n_seqs;
+    J.H = H;
+    J.dk = dk;
+    J.dv = dv;
+    J.cu = cu_seqlens;
+    J.q = q;
+    J.k = k;
+    J.v = v;
+    J.alpha = alpha;
+    J.beta = beta;
+    J.S0 = S0;
+    J.out = out;
+    J.S_final = S_final;
+    J.next_unit = 0;
+    pthread_mutex_init(&J.lock, NULL);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    pthread_t tid[256];
+    int started = 0;
+    for (int i = 1; i < n_threads; ++i)
+        if (pthread_create(&tid[started], NULL, worker, &J) == 0) ++started;
+    worker(&J);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    pthread_mutex_destroy(&J.lock);
+    return 0;
+}
+
+/*
+ * One recurrent decode step for B independent sequences: the same body as
+ * above applied to a single token, with the state updated in place.
+ * ("Complex KDA ...", section "Yazilim Gelistirme Acisindan Pratik
+ * Cikarimlar": constant-size state at inference.)
+ *   q, k, alpha : [B, H, dk]   v, out : [B, H, dv]   beta : [B, H]
+ *   S_inout     : [B, H, dk, dv]
+ */
+int ckda_oracle_decode_step(int64_t B, int64_t H, int64_t dk, int64_t dv,
+                            const double *q, const double *k, const double *v,
+                            const double *alpha, const double *beta,
+                            double *S_inout, double *out, int n_threads) {
+    if (B < 0 || H <= 0 || dk <= 0 || dv <= 0) return -1;
+    int64_t *cu = (int64_t *)malloc(sizeof(int64_t) * (B + 1));
+    for (int64_t b = 0; b <= B; ++b) cu[b] = b;
+    int rc = ckda_oracle_forward(B, H, dk, dv, cu, q, k, v, alpha, beta,
+                                 S_inout, out, S_inout, n_threads);
+    free(cu);
+    return rc;
+}
