@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Benchmark of the CKDA hot path on B200: prints ONE JSON line (rank 0).
+
+Default workload: the KDA-layer prefill -- B=4, H=16, T=4096, d_k=d_v=128,
+chunk 64, bf16 q/k/v, fp32 gates -- through ``ckda_fwd_chunked``.  A step is
+one chunked forward over that batch; ``value`` is whole-job tokens/s (tokens
+= B*T positions, each with all H heads).  The recurrent decode step (B=256,
+H=32, d=128, bf16, 1024 steps) is measured in the same run and reported under
+``decode``.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch under torchrun: every rank runs an independent replica on
+its own seeded batch (weak scaling; the path has no cross-unit exchange), the
+time is the max over ranks and ``value`` sums all ranks' tokens.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+# workload constants (KDA-layer prefill)
+B, T, H, D, CHUNK = 4, 4096, 16, 128, 64
+DEC_B, DEC_H, DEC_STEPS = 256, 32, 1024
+
+# algorithmic counts per token-head (d = 128, C = 64)
+BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 2          # q,k,v bf16 + alpha + beta + out
+STRICT_FLOPS_PER_TOKEN_HEAD = 6 * CHUNK * D + 6 * D * D + CHUNK * CHUNK // 3
+DENSE_FLOPS_PER_TOKEN_HEAD = 12 * CHUNK * D + 6 * D * D
+DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2
+
+SPEC_BF16_TFLOPS = 2250.0
+SPEC_HBM_GBS = 8000.0
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--json-out", default=None)
+    return ap.parse_args()
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _emit(obj, args, rank):
+    if rank != 0:
+        return
+    line = json.dumps(obj)
+    print(line, flush=True)
+    if args.json_out:
+        with open(args.json_out, "w") as f:
+            f.write(line + "\n")
+
+
+# ---------------------------------------------------------------- clocks ---
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.tmp.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.tmp.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ reference ---
+
+def _oracle_sample(n_units, seed=0):
+    """A bounded sample of the workload for the CPU oracle: n (b, h) units of
+    full length T, drawn exactly like the GPU inputs."""
+    from delta_rule_linear_ckda_b200 import inputs
+
+    nb = max(1, min(B, n_units))
+    case = inputs.kda_prefill(seed=seed, device="cpu", B=nb, T=T, H=H, d=D)
+    hsel = max(1, min(H, math.ceil(n_units / nb)))
+    return case, nb, hsel
+
+
+def _time_oracle(n_units, threads):
+    import oracle
+
+    case, nb, hsel = _oracle_sample(n_units)
+    q, k, v, a, b = (x[:, :, :hsel].contiguous() for x in (case.q, case.k, case.v, case.alpha, case.beta))
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, a, b, n_threads=threads)
+    dt = time.perf_counter() - t0
+    token_heads = nb * hsel * T
+    return dt, token_heads, nb * hsel
+
+
+def cpu_baseline(target_s=12.0):
+    import oracle
+
+    threads = oracle.default_threads()
+    dt1, th1, u1 = _time_oracle(1, 1)  # calibration: one unit, one thread
+    per_unit = dt1
+    n_units = int(max(1, min(B * H, target_s * threads / max(per_unit, 1e-6))))
+    n_units = max(threads, (n_units // threads) * threads) if n_units >= threads else n_units
+    n_units = min(n_units, B * H)
+    dt, th, u = _time_oracle(n_units, threads)
+    tokens_per_s = th / dt / H  # token-heads/s expressed per position with all H heads
+    return {"value": tokens_per_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{u} (b,h) units x T={T} of the kda_prefill workload "
+                      f"({th} token-heads, {dt:.1f} s wall, fp64 sequential loop)"}
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    import oracle
+
+    threads = oracle.default_threads()
+    dt1, _, _ = _time_oracle(1, 1)
+    # each step: a bounded sample sized to ~1 s of oracle work on all threads
+    n_units = int(max(1, min(B * H, 1.0 * threads / max(dt1, 1e-6))))
+    for _ in range(args.warmup):
+        _time_oracle(n_units, threads)
+    total_dt, total_th = 0.0, 0
+    for _ in range(args.steps):
+        dt, th, u = _time_oracle(n_units, threads)
+        total_dt += dt
+        total_th += th
+    value = total_th / total_dt / H
+    obj = {"metric": "CKDA fwd tokens/s (KDA-layer prefill T=4096, H=16, d=128)",
+           "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": 1000.0 * total_dt / args.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": {"workload": f"kda_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 inputs",
+                      "sample_units_per_step": n_units, "parallelism": "host threads"},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                            "sample": f"{n_units} (b,h) units x T={T} per step"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    _emit(obj, args, rank)
+
+
+# ------------------------------------------------------------------ ours ---
+
+def _kernel_src_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "delta_rule_linear_ckda_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_from_profile():
+    """DRAM bytes per launch from a committed ncu summary, if it matches the
+    current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("src_hash") != _kernel_src_hash():
+        return None, d.get("src_hash")
+    return d.get("fwd_dram_bytes_per_launch"), d.get("src_hash")
+
+
+def run_ours(args, ws, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import delta_rule_linear_ckda_b200 as ck
+    from delta_rule_linear_ckda_b200 import _lib, inputs
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if ws > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    hbm_peak, tc_peak, tc_peak_sus, peak_src = _peaks()
+
+    def barrier():
+        if ws > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if ws == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # two input sets (each ~0.4 GB > 126 MB L2), rotated so no step finds its
+    # inputs in L2
+    sets = [inputs.kda_prefill(seed=1000 * rank + i, device=dev) for i in range(2)]
+    out = torch.empty_like(sets[0].v)
+    S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        c = sets[i % 2]
+        ck.fwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, out=out, S_final=S_final)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert ck.device_status(dev) == 0
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id).start() if rank == 0 else None
+    time.sleep(0.3 if rank == 0 else 0.0)
+
+    K = args.steps
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    wall0 = time.perf_counter()
+    ev0.record(stream)
+    for i in range(K):
+        ks[i].record(stream)
+        step(i)
+        ke[i].record(stream)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(K))
+    kern_ms = max_over_ranks(kern_ms)
+    ms_per_step = elapsed_ms / K
+    tokens = B * T
+    value = ws * tokens / (ms_per_step / 1e3)
+
+    token_heads = B * T * H
+    alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + B * H * D * D * 4
+    strict_flops = token_heads * STRICT_FLOPS_PER_TOKEN_HEAD
+    dense_flops = token_heads * DENSE_FLOPS_PER_TOKEN_HEAD
+    achieved_gbs = alg_bytes / (kern_ms / 1e3) / 1e9
+    tflops_strict = strict_flops / (kern_ms / 1e3) / 1e12
+    tflops_dense = dense_flops / (kern_ms / 1e3) / 1e12
+    traffic, _ = _traffic_from_profile()
+
+    # ---- end to end: host (pinned) buffers through the public API --------
+    c = sets[0]
+    host = {n: getattr(c, n).cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
+    dbuf = {n: torch.empty_like(getattr(c, n)) for n in host}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    Sf_h = torch.empty(S_final.shape, dtype=S_final.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size() + Sf_h.numel() * Sf_h.element_size()
+
+    def e2e_step():
+        for n, t in host.items():
+            dbuf[n].copy_(t, non_blocking=True)
+        ck.fwd_chunked(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], chunk=CHUNK,
+                       out=out, S_final=S_final)
+        out_h.copy_(out, non_blocking=True)
+        Sf_h.copy_(S_final, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    E = max(1, args.e2e_steps)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1)) / E
+    e2e_value = ws * tokens / (e2e_ms / 1e3)
+    del dbuf, host
+
+    # ---- decode step (B=256, H=32, d=128, bf16), 1024 steps --------------
+    decode = None
+    if not args.no_decode:
+        dc = inputs.decode(seed=2000 + rank, device=dev, B=DEC_B, H=DEC_H, d=D, steps=DEC_STEPS)
+        S = dc.S0.clone()
+        dout = torch.empty((DEC_B, DEC_H, D), dtype=torch.bfloat16, device=dev)
+        for t in range(8):
+            ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ev0.record(stream)
+        for t in range(DEC_STEPS):
+            ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        dec_ms = max_over_ranks(ev0.elapsed_time(ev1)) / DEC_STEPS
+        dbytes = DEC_B * DEC_H * DEC_BYTES_PER_HEAD_STEP
+        dgbs = dbytes / (dec_ms / 1e3) / 1e9
+        decode = {"workload": f"decode B={DEC_B} H={DEC_H} d={D} bf16, {DEC_STEPS} steps",
+                  "ms_per_step": dec_ms, "tokens_per_s": ws * DEC_B / (dec_ms / 1e3),
+                  "achieved_gbs": dgbs, "hbm_frac_of_measured": dgbs / hbm_peak,
+                  "hbm_frac_of_spec_8tbs": dgbs / SPEC_HBM_GBS,
+                  "bytes_per_step": dbytes, "gpu_launches": DEC_STEPS}
+        del dc, S
+
+    lib_path = _lib.LIB_PATH
+    obj = {
+        "metric": "CKDA fwd tokens/s (KDA-layer prefill T=4096, H=16, d=128)",
+        "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"kda_prefill B={B} H={H} T={T} d_k=d_v={D} C={CHUNK} "
+                               "bf16 q/k/v, fp32 alpha/beta, S0=0, S_final stored",
+                   "global_batch": ws * B, "seq_len": T, "heads": H, "head_dim": D,
+                   "chunk": CHUNK, "parallelism": f"replicas x{ws} (no data-path collective)",
+                   "l2": "inputs larger than L2: two rotating 0.40 GB input sets"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} hbm_gbs (burst copy)",
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms},
+        "tensor": {"strict_tflops": tflops_strict, "dense_block_tflops": tflops_dense,
+                   "frac_strict_of_measured": tflops_strict / tc_peak,
+                   "frac_dense_of_measured": tflops_dense / tc_peak,
+                   "frac_strict_of_spec": tflops_strict / SPEC_BF16_TFLOPS,
+                   "frac_dense_of_spec": tflops_dense / SPEC_BF16_TFLOPS,
+                   "measured_bf16_tflops": tc_peak},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": K,
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+        "lib": os.path.relpath(lib_path, ROOT),
+    }
+    if decode is not None:
+        obj["decode"] = decode
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        obj["cpu_baseline"] = cpu_baseline()
+    _emit(obj, args, rank)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = _args()
+    ws, rank, local = _dist()
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        return
+    run_ours(args, ws, rank, local)
+
+
+if __name__ == "__main__":
+    main()

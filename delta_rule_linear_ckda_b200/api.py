@@ -1,0 +1,130 @@
+"""Torch-tensor front end of the C ABI (argument marshalling only).
+
+Every function checks dtypes, shapes and contiguity, passes ``data_ptr()``
+values and the current CUDA stream to ``libckda.so`` and raises ``CKDAError``
+on a non-zero status.  All arithmetic happens in the CUDA kernels.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import CKDAError
+
+_DT = {torch.float32: _lib.CKDA_F32, torch.bfloat16: _lib.CKDA_BF16}
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
+                out=None, S_final=None, return_final: bool = True, fp32core: bool = False
+                ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked CKDA forward.  Shapes as in ``ckda_fwd_chunked`` (include/ckda.h).
+
+    Fixed-length: q, k, alpha ``[B, T, H, dk]``; v ``[B, T, H, dv]``; beta ``[B, T, H]``.
+    Packed: ``cu_seqlens`` int32 ``[N+1]`` and tensors with a leading 1 or without it.
+    Returns ``(out, S_final)``; ``S_final`` is None when ``return_final`` is False.
+    """
+    dev = q.device
+    if q.dtype not in _DT:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(alpha, "alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    if cu_seqlens is None:
+        if q.dim() != 4:
+            raise ValueError("q must be [B, T, H, dk]")
+        B, T, H, dk = q.shape
+        N = B
+    else:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
+        if q.dim() == 4:
+            if q.shape[0] != 1:
+                raise ValueError("packed inputs take a leading dimension of 1")
+            T, H, dk = q.shape[1:]
+        else:
+            T, H, dk = q.shape
+        N = cu_seqlens.numel() - 1
+        B = N
+    dv = v.shape[-1]
+    if k.shape != q.shape or alpha.shape != q.shape or v.shape[:-1] != q.shape[:-1]:
+        raise ValueError("q, k, alpha must share a shape and v must match it but for the last dim")
+    if tuple(beta.shape) != tuple(q.shape[:-1]):
+        raise ValueError("beta must have q's shape without the last dim")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=dev)
+    else:
+        _need(out, "out", v.dtype, dev)
+    if return_final and S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, dev)
+    fn = _lib.load().ckda_fwd_chunked_fp32core if fp32core else _lib.load().ckda_fwd_chunked
+    with torch.cuda.device(dev):
+        rc = fn(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(out),
+                _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_fwd_chunked")
+    return out, S_final
+
+
+def decode_step(q, k, v, alpha, beta, S, out=None) -> torch.Tensor:
+    """One recurrent step, in place on ``S`` ``[B, H, dk, dv]`` (fp32).
+
+    q, k, alpha ``[B, H, dk]``; v ``[B, H, dv]``; beta ``[B, H]``.  Returns ``out``.
+    """
+    dev = q.device
+    if q.dtype not in _DT:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(alpha, "alpha", torch.float32, dev)
+    _need(beta, "beta", torch.float32, dev)
+    _need(S, "S", torch.float32, dev)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(S.shape) != (B, H, dk, dv) or tuple(beta.shape) != (B, H):
+        raise ValueError("shape mismatch")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=v.dtype, device=dev)
+    else:
+        _need(out, "out", v.dtype, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(out),
+                                          B, H, dk, dv, _DT[q.dtype], _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_decode_step")
+    return out
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return _lib.load().ckda_device_status(_stream_ptr(dev))

@@ -1,0 +1,162 @@
+// Host side of libckda.so: argument validation, the device status word and
+// dispatch to the kernels.  Every check happens before any CUDA call, so an
+// argument error launches nothing and touches no memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "ckda.h"
+
+namespace ckda {
+cudaError_t launch_decode(int dtype, int dk, int dv, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, float* S, void* out, int BH,
+                          cudaStream_t stream);
+cudaError_t launch_fwd_simt(int dtype, int dk, int dv, const void* q, const void* k,
+                            const void* v, const float* alpha, const float* beta, const float* S0,
+                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
+                            int C, int* status, cudaStream_t stream);
+// Returns cudaErrorNotSupported when the shape is not covered by the
+// tensor-core kernel (the caller then uses the CUDA-core kernel).
+cudaError_t launch_fwd_tc(int dtype, int dk, int dv, const void* q, const void* k, const void* v,
+                          const float* alpha, const float* beta, const float* S0,
+                          const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
+                          int C, int* status, cudaStream_t stream);
+}  // namespace ckda
+
+// First device-side error since the last ckda_device_status() call.
+__device__ int g_ckda_status = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int*> g_status_ptr[kMaxDevices];
+
+// Device address of the status word on the current device (looked up once
+// per device; cudaGetSymbolAddress needs that device to be current).
+int* status_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  int* p = g_status_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_ckda_status) != cudaSuccess) return nullptr;
+    p = static_cast<int*>(addr);
+    g_status_ptr[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+int validate_fwd(const void* q, const void* k, const void* v, const float* alpha,
+                 const float* beta, const float* S0, const int32_t* cu, const void* out,
+                 const float* S_final, int B, int T, int H, int d_k, int d_v, int* chunk,
+                 int dtype) {
+  if (B < 0 || T < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
+  if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (*chunk == 0) *chunk = 64;
+  if (*chunk != 16 && *chunk != 32 && *chunk != 64) return CKDA_ERR_UNSUPPORTED;
+  const int64_t tokens = (cu != nullptr) ? (int64_t)T : (int64_t)B * T;
+  if (tokens > 0 && (!q || !k || !v || !alpha || !beta || !out)) return CKDA_ERR_INVALID_ARG;
+  if (cu == nullptr && (int64_t)B * T * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
+  if (cu != nullptr && B == 0 && T != 0) return CKDA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, alpha, beta, S0, out, S_final, cu};
+  for (const void* p : ptrs)
+    if (p != nullptr && !aligned16(p) && p != cu) return CKDA_ERR_MISALIGNED;
+  if (cu != nullptr && (reinterpret_cast<uintptr_t>(cu) & 3u) != 0) return CKDA_ERR_MISALIGNED;
+  if (out != nullptr && (out == q || out == k || out == v || out == alpha || out == beta))
+    return CKDA_ERR_INVALID_ARG;
+  return CKDA_OK;
+}
+
+int fwd_impl(bool allow_tc, const void* q, const void* k, const void* v, const float* alpha,
+             const float* beta, const float* S0, const int32_t* cu, void* out, float* S_final,
+             int B, int T, int H, int d_k, int d_v, int chunk, int dtype, void* stream) {
+  int rc = validate_fwd(q, k, v, alpha, beta, S0, cu, out, S_final, B, T, H, d_k, d_v, &chunk,
+                        dtype);
+  if (rc != CKDA_OK) return rc;
+  const int n_seqs = B;
+  if (n_seqs == 0) return CKDA_OK;
+  int* status = status_ptr();
+  if (status == nullptr) return CKDA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaErrorNotSupported;
+  if (allow_tc)
+    e = ckda::launch_fwd_tc(dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs,
+                            T, H, chunk, status, st);
+  if (e == cudaErrorNotSupported)
+    e = ckda::launch_fwd_simt(dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final,
+                              n_seqs, T, H, chunk, status, st);
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int ckda_version(void) { return 100; }
+
+const char* ckda_status_string(int status) {
+  switch (status) {
+    case CKDA_OK: return "ok";
+    case CKDA_ERR_INVALID_ARG: return "invalid argument (NULL pointer or bad size)";
+    case CKDA_ERR_UNSUPPORTED: return "unsupported head size, chunk size or dtype";
+    case CKDA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case CKDA_ERR_CUDA: return "CUDA runtime or launch error";
+    case CKDA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    case CKDA_ERR_BAD_SEQLENS: return "cu_seqlens is not a valid offsets array";
+  }
+  return "unknown status";
+}
+
+int ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                     const float* beta, const float* S0, const int32_t* cu_seqlens, void* out,
+                     float* S_final, int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
+                     void* stream) {
+  return fwd_impl(true, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
+                  chunk, dtype, stream);
+}
+
+int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void* v, const float* alpha,
+                              const float* beta, const float* S0, const int32_t* cu_seqlens,
+                              void* out, float* S_final, int B, int T, int H, int d_k, int d_v,
+                              int chunk, int dtype, void* stream) {
+  return fwd_impl(false, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
+                  chunk, dtype, stream);
+}
+
+int ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                     const float* beta, float* S_inout, void* out, int B, int H, int d_k, int d_v,
+                     int dtype, void* stream) {
+  if (B < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
+  if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
+  if (B == 0) return CKDA_OK;
+  if (!q || !k || !v || !alpha || !beta || !S_inout || !out) return CKDA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, alpha, beta, S_inout, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return CKDA_ERR_MISALIGNED;
+  if (out == S_inout || out == q || out == k || out == v) return CKDA_ERR_INVALID_ARG;
+  cudaError_t e = ckda::launch_decode(dtype, d_k, d_v, q, k, v, alpha, beta, S_inout, out, B * H,
+                                      static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+int ckda_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return CKDA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_ckda_status, sizeof(int)) != cudaSuccess) return CKDA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_ckda_status, &zero, sizeof(int)) != cudaSuccess)
+      return CKDA_ERR_CUDA;
+  }
+  return v;
+}
+
+}  // extern "C"

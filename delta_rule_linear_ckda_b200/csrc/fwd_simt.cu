@@ -1,0 +1,429 @@
+// Chunkwise WY forward of CKDA on fp32 CUDA cores (every product and sum in
+// fp32; inputs widened from bf16 or fp32).  This is the fp32-faithful path:
+// any d_k, d_v in {16, 32, 64, 128} and chunk C in {16, 32, 64}.
+//
+// Chunk algebra (for one chunk of positions r = 0..C-1 with start state S0,
+// P(r, s) = alpha_{s+1} * ... * alpha_r channel-wise, P(r, r) = 1):
+//   Gamma_r = P(r, -1), rho_s = P(C-1, s), gamma = Gamma_{C-1}
+//   T[r, s] = beta_r sum_i k_ri k_si P_i(r, s)        (s < r)
+//   A[r, s] = sum_i q_ri k_si P_i(r, s)               (s <= r)
+//   [W | U~] = (I + T)^-1 diag(beta) [K * Gamma | V]
+//   U = U~ - W S0;   O = (Q * Gamma) S0 + A U;   S_C = Diag(gamma) S0 + (K * rho)^T U
+// Sources: "Semidirect Fourier Delta Attention" page, "El Teorema de
+// Chunk-WY Constructivo" and "Principales Contribuciones" item 3 (affine
+// block transfer); "Gated DeltaNet-2" page, Methodology section 3 (decay
+// absorbed into the WY factors, triangular solve (I + T)^-1).
+//
+// Every gate product is a running product of alphas: no division, no
+// logarithm, so zero and negative gates are exact and underflow goes to 0.
+// Positions past the end of a sequence are identity transitions
+// (alpha = 1, beta = 0, q = k = v = 0) and produce no output.
+//
+// One CTA owns one (sequence, head, d_v slice of width BV) and walks its
+// chunks in order; the slice of the state stays in shared memory in fp32.
+#include "common.cuh"
+
+namespace ckda {
+namespace simt {
+
+constexpr int kThreads = 256;
+constexpr int kMaxC = 64;
+
+template <int DK, int BV>
+struct Smem {
+  static constexpr int KS = DK + 4;  // row stride of [C][DK] tiles (floats)
+  static constexpr int VS = BV + 4;  // row stride of [C][BV] and [DK][BV] tiles
+  static constexpr int CS = kMaxC + 4;
+  static constexpr int kK = 0;
+  static constexpr int kQ = kK + kMaxC * KS;
+  static constexpr int kA = kQ + kMaxC * KS;
+  static constexpr int kW = kA + kMaxC * KS;
+  static constexpr int kV = kW + kMaxC * KS;
+  static constexpr int kT = kV + kMaxC * VS;
+  static constexpr int kAm = kT + kMaxC * CS;
+  static constexpr int kS = kAm + kMaxC * CS;
+  static constexpr int kBeta = kS + DK * VS;
+  static constexpr int kGam = kBeta + kMaxC;
+  static constexpr int kFloats = kGam + DK;
+  static constexpr size_t kBytes = sizeof(float) * kFloats;
+};
+
+// Channels held by each lane while building the score blocks.
+template <int DK>
+struct LaneChannels {
+  static constexpr int kPer = DK >= 32 ? DK / 32 : 1;
+  static __device__ __forceinline__ bool active(int lane) { return lane * kPer < DK; }
+};
+
+template <int N>
+__device__ __forceinline__ void lds(const float* p, float* x) {
+  if constexpr (N == 4) {
+    float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  } else if constexpr (N == 2) {
+    float2 a = *reinterpret_cast<const float2*>(p);
+    x[0] = a.x; x[1] = a.y;
+  } else {
+    x[0] = p[0];
+  }
+}
+
+// Sum an 8-vector over the 32 lanes of a warp and leave the total of
+// element e in every lane whose index satisfies (lane & 7) == e, in v[0].
+__device__ __forceinline__ void reduce_scatter8(float* v, int lane) {
+  {
+    const bool up = lane & 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float send = up ? v[i] : v[i + 4];
+      const float keep = up ? v[i + 4] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+    }
+  }
+  {
+    const bool up = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const float send = up ? v[i] : v[i + 2];
+      const float keep = up ? v[i + 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+  }
+  {
+    const bool up = lane & 1;
+    const float send = up ? v[0] : v[1];
+    const float keep = up ? v[1] : v[0];
+    v[0] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+  }
+  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 8);
+  v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+
+template <int DK, int BV, typename Tin>
+__global__ void __launch_bounds__(kThreads, 1)
+fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
+                const float* __restrict__ alpha, const float* __restrict__ beta,
+                const float* S0, const int32_t* __restrict__ cu, Tin* __restrict__ out,
+                float* S_final, int n_seqs, int T, int H, int DV, int C, int* status) {
+  using L = Smem<DK, BV>;
+  constexpr int KS = L::KS, VS = L::VS, CS = L::CS;
+  extern __shared__ __align__(16) float smem[];
+  float* Ks = smem + L::kK;   // k, then K * rho
+  float* Qs = smem + L::kQ;   // q, then Q * Gamma
+  float* As = smem + L::kA;   // alpha
+  float* Ws = smem + L::kW;   // beta K Gamma, then W
+  float* Vs = smem + L::kV;   // v, then beta v, then U~, then U
+  float* Tm = smem + L::kT;   // T (strictly lower)
+  float* Am = smem + L::kAm;  // A (lower incl. diagonal)
+  float* Ss = smem + L::kS;   // state slice [DK][BV]
+  float* bs = smem + L::kBeta;
+  float* gs = smem + L::kGam;
+
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int j0 = blockIdx.x * BV;
+  const int h = blockIdx.y;
+  const int n = blockIdx.z;
+
+  const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
+  if (!sr.ok) return;
+
+  const size_t sbase = ((size_t)n * H + h) * DK * DV + j0;
+  for (int e = tid; e < DK * BV / 4; e += kThreads) {
+    const int i = e / (BV / 4), c4 = e % (BV / 4);
+    float4 val = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (S0 != nullptr) val = *reinterpret_cast<const float4*>(S0 + sbase + (size_t)i * DV + 4 * c4);
+    *reinterpret_cast<float4*>(Ss + i * VS + 4 * c4) = val;
+  }
+
+  for (int64_t t0 = sr.begin; t0 < sr.end; t0 += C) {
+    const int Lc = (sr.end - t0 < (int64_t)C) ? (int)(sr.end - t0) : C;
+    __syncthreads();  // previous chunk finished with every buffer
+
+    // ---- stage inputs (fp32), identity transitions past the end ---------
+    for (int e = tid; e < C * DK / 4; e += kThreads) {
+      const int r = e / (DK / 4), c4 = e % (DK / 4);
+      float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk, aa = make_float4(1.f, 1.f, 1.f, 1.f);
+      if (r < Lc) {
+        const size_t off = ((size_t)(t0 + r) * H + h) * DK + 4 * c4;
+        kk = load4_f32(k + off);
+        qq = load4_f32(q + off);
+        aa = *reinterpret_cast<const float4*>(alpha + off);
+      }
+      *reinterpret_cast<float4*>(Ks + r * KS + 4 * c4) = kk;
+      *reinterpret_cast<float4*>(Qs + r * KS + 4 * c4) = qq;
+      *reinterpret_cast<float4*>(As + r * KS + 4 * c4) = aa;
+    }
+    for (int e = tid; e < C * BV / 4; e += kThreads) {
+      const int r = e / (BV / 4), c4 = e % (BV / 4);
+      float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < Lc) vv = load4_f32(v + ((size_t)(t0 + r) * H + h) * DV + j0 + 4 * c4);
+      *reinterpret_cast<float4*>(Vs + r * VS + 4 * c4) = vv;
+    }
+    for (int r = tid; r < C; r += kThreads)
+      bs[r] = (r < Lc) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    __syncthreads();
+
+    // ---- score blocks T and A: one warp per column s ------------------
+    // x = k_s * P(r, s) is carried down the rows r > s by multiplying with
+    // alpha_r; the dot products with k_r and q_r give T[r, s] / beta_r and
+    // A[r, s].  Lanes split the channels; eight rows are reduced at once.
+    {
+      using LC = LaneChannels<DK>;
+      constexpr int CPL = LC::kPer;
+      const bool act = LC::active(lane);
+      const int cb = lane * CPL;
+      for (int s = warp; s < C; s += kThreads / 32) {
+        float x[CPL];
+        float qs[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) { x[c] = 0.f; qs[c] = 0.f; }
+        if (act) { lds<CPL>(Ks + s * KS + cb, x); lds<CPL>(Qs + s * KS + cb, qs); }
+        float d = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) d = fmaf(qs[c], x[c], d);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+        if (lane == 0) { Am[s * CS + s] = d; Tm[s * CS + s] = 0.f; }
+        for (int r = lane; r < s; r += 32) { Tm[r * CS + s] = 0.f; Am[r * CS + s] = 0.f; }
+        for (int rb = s + 1; rb < C; rb += 8) {
+          float pk[8], pq[8];
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            pk[jj] = 0.f;
+            pq[jj] = 0.f;
+            const int r = rb + jj;
+            if (r < C) {
+              float a[CPL], kr[CPL], qr[CPL];
+#pragma unroll
+              for (int c = 0; c < CPL; ++c) { a[c] = 1.f; kr[c] = 0.f; qr[c] = 0.f; }
+              if (act) {
+                lds<CPL>(As + r * KS + cb, a);
+                lds<CPL>(Ks + r * KS + cb, kr);
+                lds<CPL>(Qs + r * KS + cb, qr);
+              }
+#pragma unroll
+              for (int c = 0; c < CPL; ++c) {
+                x[c] *= a[c];
+                pk[jj] = fmaf(kr[c], x[c], pk[jj]);
+                pq[jj] = fmaf(qr[c], x[c], pq[jj]);
+              }
+            }
+          }
+          reduce_scatter8(pk, lane);
+          reduce_scatter8(pq, lane);
+          const int r = rb + (lane & 7);
+          if (lane < 8 && r < C) {
+            Tm[r * CS + s] = bs[r] * pk[0];
+            Am[r * CS + s] = pq[0];
+          }
+        }
+      }
+    }
+    __syncthreads();
+
+    // ---- gate products: one thread per channel ------------------------
+    // forward: Gamma_r (inclusive prefix); W rhs = beta K Gamma; Q <- Q Gamma
+    // backward: rho_s (exclusive suffix); K <- K rho
+    if (tid < DK) {
+      const int i = tid;
+      float gmm = 1.f;
+      for (int r = 0; r < C; ++r) {
+        gmm *= As[r * KS + i];
+        Ws[r * KS + i] = bs[r] * Ks[r * KS + i] * gmm;
+        Qs[r * KS + i] *= gmm;
+      }
+      gs[i] = gmm;
+      float p = 1.f;
+      for (int s = C - 1; s >= 0; --s) {
+        Ks[s * KS + i] *= p;
+        p *= As[s * KS + i];
+      }
+    }
+    for (int e = tid; e < C * BV; e += kThreads) {
+      const int r = e / BV, c = e % BV;
+      Vs[r * VS + c] *= bs[r];
+    }
+    __syncthreads();
+
+    // ---- WY factors: [W | U~] = (I + T)^-1 [beta K Gamma | beta V] -----
+    // Forward substitution, one thread per column, 16 rows at a time in
+    // registers: rows of earlier blocks are final when a block starts.
+    if (tid < DK + BV) {
+      float* X = (tid < DK) ? (Ws + tid) : (Vs + (tid - DK));
+      const int xs = (tid < DK) ? KS : VS;
+      for (int rb = 0; rb < C; rb += 16) {
+        float acc[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) acc[m] = X[(rb + m) * xs];
+        for (int s = 0; s < rb; ++s) {
+          const float xv = X[s * xs];
+#pragma unroll
+          for (int m = 0; m < 16; ++m) acc[m] = fmaf(-Tm[(rb + m) * CS + s], xv, acc[m]);
+        }
+#pragma unroll
+        for (int m = 1; m < 16; ++m) {
+#pragma unroll
+          for (int m2 = 0; m2 < m; ++m2) acc[m] = fmaf(-Tm[(rb + m) * CS + rb + m2], acc[m2], acc[m]);
+        }
+#pragma unroll
+        for (int m = 0; m < 16; ++m) X[(rb + m) * xs] = acc[m];
+      }
+    }
+    __syncthreads();
+
+    // ---- state carry ----------------------------------------------------
+    // (a) U = U~ - W S  (C x BV), 4x4 register tiles
+    const int ntile = (C / 4) * (BV / 4);
+    const int tr = tid / (BV / 4), tc = tid % (BV / 4);
+    const int r0 = tr * 4, c0 = tc * 4;
+    if (tid < ntile) {
+      float4 acc[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m] = *reinterpret_cast<const float4*>(Vs + (r0 + m) * VS + c0);
+#pragma unroll 4
+      for (int i = 0; i < DK; ++i) {
+        const float4 s4 = *reinterpret_cast<const float4*>(Ss + i * VS + c0);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float w = Ws[(r0 + m) * KS + i];
+          acc[m].x = fmaf(-w, s4.x, acc[m].x); acc[m].y = fmaf(-w, s4.y, acc[m].y);
+          acc[m].z = fmaf(-w, s4.z, acc[m].z); acc[m].w = fmaf(-w, s4.w, acc[m].w);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) *reinterpret_cast<float4*>(Vs + (r0 + m) * VS + c0) = acc[m];
+    }
+    __syncthreads();
+
+    // (b) O = (Q Gamma) S + A U  -> out rows of real tokens
+    if (tid < ntile) {
+      float4 acc[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (int i = 0; i < DK; ++i) {
+        const float4 s4 = *reinterpret_cast<const float4*>(Ss + i * VS + c0);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float w = Qs[(r0 + m) * KS + i];
+          acc[m].x = fmaf(w, s4.x, acc[m].x); acc[m].y = fmaf(w, s4.y, acc[m].y);
+          acc[m].z = fmaf(w, s4.z, acc[m].z); acc[m].w = fmaf(w, s4.w, acc[m].w);
+        }
+      }
+      const int smax = min(C, r0 + 4);  // A is lower triangular
+      for (int s = 0; s < smax; ++s) {
+        const float4 u4 = *reinterpret_cast<const float4*>(Vs + s * VS + c0);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const float w = Am[(r0 + m) * CS + s];
+          acc[m].x = fmaf(w, u4.x, acc[m].x); acc[m].y = fmaf(w, u4.y, acc[m].y);
+          acc[m].z = fmaf(w, u4.z, acc[m].z); acc[m].w = fmaf(w, u4.w, acc[m].w);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = r0 + m;
+        if (r < Lc) store4(out + ((size_t)(t0 + r) * H + h) * DV + j0 + c0, acc[m]);
+      }
+    }
+    __syncthreads();
+
+    // (c) S <- Diag(gamma) S + (K rho)^T U   (DK x BV)
+    for (int tile = tid; tile < (DK / 4) * (BV / 4); tile += kThreads) {
+      const int i0 = (tile / (BV / 4)) * 4, cc = (tile % (BV / 4)) * 4;
+      float4 acc[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s = 0; s < C; ++s) {
+        const float4 kh = *reinterpret_cast<const float4*>(Ks + s * KS + i0);
+        const float4 u4 = *reinterpret_cast<const float4*>(Vs + s * VS + cc);
+        const float khv[4] = {kh.x, kh.y, kh.z, kh.w};
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          acc[m].x = fmaf(khv[m], u4.x, acc[m].x); acc[m].y = fmaf(khv[m], u4.y, acc[m].y);
+          acc[m].z = fmaf(khv[m], u4.z, acc[m].z); acc[m].w = fmaf(khv[m], u4.w, acc[m].w);
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        float4* sp = reinterpret_cast<float4*>(Ss + (i0 + m) * VS + cc);
+        float4 sv = *sp;
+        const float g = gs[i0 + m];
+        sv.x = fmaf(g, sv.x, acc[m].x); sv.y = fmaf(g, sv.y, acc[m].y);
+        sv.z = fmaf(g, sv.z, acc[m].z); sv.w = fmaf(g, sv.w, acc[m].w);
+        *sp = sv;
+      }
+    }
+  }
+  __syncthreads();
+  if (S_final != nullptr) {
+    for (int e = tid; e < DK * BV / 4; e += kThreads) {
+      const int i = e / (BV / 4), c4 = e % (BV / 4);
+      *reinterpret_cast<float4*>(S_final + sbase + (size_t)i * DV + 4 * c4) =
+          *reinterpret_cast<const float4*>(Ss + i * VS + 4 * c4);
+    }
+  }
+}
+
+template <int DK, int BV, typename Tin>
+static cudaError_t launch_t(const void* q, const void* k, const void* v, const float* alpha,
+                            const float* beta, const float* S0, const int32_t* cu, void* out,
+                            float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
+                            cudaStream_t stream) {
+  using L = Smem<DK, BV>;
+  auto kern = fwd_simt_kernel<DK, BV, Tin>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)L::kBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid(DV / BV, H, n_seqs);
+  kern<<<grid, kThreads, L::kBytes, stream>>>(
+      static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
+      beta, S0, cu, static_cast<Tin*>(out), S_final, n_seqs, T, H, DV, C, status);
+  return cudaGetLastError();
+}
+
+template <int DK, typename Tin>
+static cudaError_t launch_bv(const void* q, const void* k, const void* v, const float* alpha,
+                             const float* beta, const float* S0, const int32_t* cu, void* out,
+                             float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
+                             cudaStream_t stream) {
+  switch (DV) {
+    case 16:
+      return launch_t<DK, 16, Tin>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
+                                   C, status, stream);
+    case 32:
+      return launch_t<DK, 32, Tin>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
+                                   C, status, stream);
+    default:  // 64 and 128: slices of 64 columns
+      return launch_t<DK, 64, Tin>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
+                                   C, status, stream);
+  }
+}
+
+}  // namespace simt
+
+cudaError_t launch_fwd_simt(int dtype, int dk, int dv, const void* q, const void* k,
+                            const void* v, const float* alpha, const float* beta, const float* S0,
+                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
+                            int C, int* status, cudaStream_t stream) {
+#define CKDA_SIMT_DK(DKV)                                                                       \
+  case DKV:                                                                                     \
+    return (dtype == CKDA_BF16)                                                                 \
+               ? simt::launch_bv<DKV, __nv_bfloat16>(q, k, v, alpha, beta, S0, cu, out,        \
+                                                      S_final, n_seqs, T, H, dv, C, status,     \
+                                                      stream)                                   \
+               : simt::launch_bv<DKV, float>(q, k, v, alpha, beta, S0, cu, out, S_final,       \
+                                             n_seqs, T, H, dv, C, status, stream);
+  switch (dk) {
+    CKDA_SIMT_DK(16)
+    CKDA_SIMT_DK(32)
+    CKDA_SIMT_DK(64)
+    CKDA_SIMT_DK(128)
+  }
+#undef CKDA_SIMT_DK
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace ckda

@@ -1,0 +1,159 @@
+/*
+ * ckda.h -- C ABI of libckda.so: the Complex Kimi Delta Attention (CKDA)
+ * recurrence on one NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Complex KDA: Kimi Delta Attention Mimarisinin Ifade Gucunu
+ * Anlamak ve Gelistirmek", section "Complex KDA (CKDA) Mimarisi ve Parametre
+ * Genislemesi"; "Gated DeltaNet-2", Methodology section 1 with the erase and
+ * write gates tied to beta_t; "Semidirect Fourier Delta Attention",
+ * "Arquitectura Central" with zero phase):
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * with a per-channel gate alpha_t in [-1, 1]^{d_k}, a scalar delta
+ * coefficient beta_t in [0, 2] per (token, head), and a d_k x d_v fp32 state
+ * per (sequence, head).  The read-out uses the state after the update and no
+ * query scale.  The library does not normalise q or k.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA
+ *    memory) on the current CUDA device, row-major and contiguous, 16-byte
+ *    aligned.  The caller owns every buffer; the library allocates nothing
+ *    and keeps no state between calls except one device status word.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream and returns as soon
+ *    as the work is enqueued.
+ *  - dtype selects the element type of q, k, v and out: CKDA_F32 or
+ *    CKDA_BF16.  alpha, beta, S0, S_final and S_inout are always fp32.
+ *    Outputs are rounded to the output type with round-to-nearest-even from
+ *    fp32 accumulators; the state stays fp32.
+ *  - Return value: CKDA_OK (0) or a negative CKDA_ERR_* code.  On an
+ *    argument error nothing is launched and no memory is touched.  Errors
+ *    found on the device (a bad cu_seqlens array, a bounded wait that timed
+ *    out) are recorded in the device status word and reported by
+ *    ckda_device_status().
+ */
+#ifndef CKDA_H
+#define CKDA_H
+
+#include <stdint.h>
+
+/* Symbols of the C ABI are exported even when the library is compiled with
+   hidden default visibility. */
+#if defined(__GNUC__)
+#define CKDA_API __attribute__((visibility("default")))
+#else
+#define CKDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  CKDA_F32 = 0,
+  CKDA_BF16 = 1
+};
+
+enum {
+  CKDA_OK = 0,
+  CKDA_ERR_INVALID_ARG = -1,   /* NULL required pointer, negative or
+                                  inconsistent sizes */
+  CKDA_ERR_UNSUPPORTED = -2,   /* d_k or d_v not in {16,32,64,128}, chunk
+                                  not in {0,16,32,64}, unknown dtype */
+  CKDA_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned */
+  CKDA_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
+  CKDA_ERR_DEVICE_TIMEOUT = -5,/* a bounded device-side wait gave up */
+  CKDA_ERR_BAD_SEQLENS = -6    /* cu_seqlens not 0 = cu[0] <= ... <= cu[N] = T */
+};
+
+/*
+ * ckda_fwd_chunked -- chunkwise-parallel WY forward (prefill).
+ *
+ * Source of the chunk form: "Semidirect Fourier Delta Attention", sections
+ * "El Teorema de Chunk-WY Constructivo" (block products as a diagonal
+ * product minus a correction of rank <= chunk) and "Principales
+ * Contribuciones" item 3 (exact affine block transfer between chunks);
+ * "Gated DeltaNet-2", Methodology section 3 (decay absorbed into the WY
+ * factors, lower-triangular solve (I + T)^-1).  The result equals the
+ * token-by-token recurrence above up to rounding; the chunk size does not
+ * change it.
+ *
+ * Fixed-length batch (cu_seqlens == NULL):
+ *   q, k   [B, T, H, d_k]   (dtype)     v, out [B, T, H, d_v] (dtype)
+ *   alpha  [B, T, H, d_k]   fp32        beta   [B, T, H]       fp32
+ *   S0, S_final [B, H, d_k, d_v] fp32
+ * Packed variable-length batch (cu_seqlens != NULL):
+ *   B is the number of sequences N and T the total number of packed tokens;
+ *   q, k, alpha are [T, H, d_k], v and out [T, H, d_v], beta [T, H];
+ *   cu_seqlens is a DEVICE int32 array [N + 1] with cu[0] = 0,
+ *   cu[n] <= cu[n+1], cu[N] = T; sequence n owns tokens [cu[n], cu[n+1]).
+ *   S0 and S_final are [N, H, d_k, d_v].  The state restarts at every
+ *   sequence start.  The array is validated on the device: a violation sets
+ *   CKDA_ERR_BAD_SEQLENS in the status word and the affected sequences
+ *   produce no output.
+ *
+ *   S0       may be NULL (zero initial state).
+ *   S_final  may be NULL (final state not stored) and may equal S0 (each
+ *            unit reads its own S0 slice before it writes the same slice).
+ *   out      must not alias any input.
+ *   chunk    0 (default 64), 16, 32 or 64.
+ *   d_k, d_v each in {16, 32, 64, 128}.
+ * A zero-length sequence stores S_final = S0 and writes no output rows.
+ */
+CKDA_API int ckda_fwd_chunked(const void* q, const void* k, const void* v,
+                     const float* alpha, const float* beta, const float* S0,
+                     const int32_t* cu_seqlens, void* out, float* S_final,
+                     int B, int T, int H, int d_k, int d_v, int chunk,
+                     int dtype, void* stream);
+
+/*
+ * ckda_fwd_chunked_fp32core -- the same operation and arguments as
+ * ckda_fwd_chunked, forced onto the fp32 CUDA-core kernel (every product
+ * and sum in fp32 FFMA, no tensor-core rounding of intermediate operands).
+ * ckda_fwd_chunked itself routes here for fp32 inputs and for shapes the
+ * tensor-core kernel does not cover; this entry point exists so callers (and
+ * tests) can request the fp32-faithful path for bf16 inputs too.
+ */
+CKDA_API int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta,
+                              const float* S0, const int32_t* cu_seqlens,
+                              void* out, float* S_final, int B, int T, int H,
+                              int d_k, int d_v, int chunk, int dtype,
+                              void* stream);
+
+/*
+ * ckda_decode_step -- one recurrent token for B independent sequences,
+ * in place on the state ("Complex KDA ...", section "Yazilim Gelistirme
+ * Acisindan Pratik Cikarimlar": O(1) inference state).
+ *   q, k, alpha [B, H, d_k]    v, out [B, H, d_v]    beta [B, H]
+ *   S_inout     [B, H, d_k, d_v] fp32, read once and overwritten once.
+ * No pointer may alias another, except that nothing else aliases S_inout.
+ */
+CKDA_API int ckda_decode_step(const void* q, const void* k, const void* v,
+                     const float* alpha, const float* beta, float* S_inout,
+                     void* out, int B, int H, int d_k, int d_v, int dtype,
+                     void* stream);
+
+/* Human-readable text for a CKDA_* status code (static storage). */
+CKDA_API const char* ckda_status_string(int status);
+
+/*
+ * ckda_device_status -- synchronise `stream`, then read and clear the
+ * status word of the current device.  Returns CKDA_OK, the first device
+ * error recorded since the last call (CKDA_ERR_BAD_SEQLENS,
+ * CKDA_ERR_DEVICE_TIMEOUT), or CKDA_ERR_CUDA if the synchronisation itself
+ * failed.
+ */
+CKDA_API int ckda_device_status(void* stream);
+
+/* Library ABI version (major * 100 + minor). */
+CKDA_API int ckda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CKDA_H */

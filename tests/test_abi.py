@@ -1,0 +1,130 @@
+"""The C-ABI library loads and exports every symbol its header declares.
+
+CPU only: argument errors are rejected on the host before any CUDA call, so
+these calls launch nothing and need no GPU.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from delta_rule_linear_ckda_b200 import build as b
+
+    b.build()
+    from delta_rule_linear_ckda_b200 import _lib
+
+    return _lib.load()
+
+
+def declared_symbols():
+    names = []
+    for fn in sorted(os.listdir(HEADER_DIR)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(HEADER_DIR, fn)).read()
+            names += re.findall(r"CKDA_API\s+[\w\s\*]+?\b(ckda_\w+)\s*\(", text)
+    return names
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for required in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_status_string",
+                     "ckda_device_status"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    from delta_rule_linear_ckda_b200._lib import LIB_PATH, SIGNATURES
+
+    out = subprocess.run(["nm", "-D", "--defined-only", LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT\s+(ckda_\w+)", out))
+    for name in declared_symbols():
+        assert name in exported, name
+        assert hasattr(lib, name)
+        assert name in SIGNATURES, f"binding lacks a signature for {name}"
+
+
+def test_library_has_no_runtime_dependency_on_libcudart():
+    from delta_rule_linear_ckda_b200._lib import LIB_PATH
+
+    out = subprocess.run(["ldd", LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcudart" not in out
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        s = lib.ckda_status_string(code)
+        assert s and b"unknown" not in s
+    assert lib.ckda_status_string(-99) == b"unknown status"
+    assert lib.ckda_version() >= 100
+
+
+# Fake, never-dereferenced "device" addresses: validation rejects the call
+# before any CUDA call is made.
+P = 1 << 20          # 16-byte aligned
+MIS = (1 << 20) + 4  # misaligned
+
+
+def fwd(lib, **kw):
+    a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000, S0=None,
+             cu=None, out=P + 0x5000, S_final=None, B=1, T=8, H=1, dk=16, dv=16, chunk=16,
+             dtype=0, stream=None)
+    a.update(kw)
+    return lib.ckda_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S0"], a["cu"],
+                                a["out"], a["S_final"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
+                                a["chunk"], a["dtype"], a["stream"])
+
+
+def test_fwd_argument_errors(lib):
+    assert fwd(lib, q=None) == -1
+    assert fwd(lib, beta=None) == -1
+    assert fwd(lib, out=None) == -1
+    assert fwd(lib, B=-1) == -1
+    assert fwd(lib, H=0) == -1
+    assert fwd(lib, T=-3) == -1
+    assert fwd(lib, dk=48) == -2
+    assert fwd(lib, dv=256) == -2
+    assert fwd(lib, chunk=128) == -2
+    assert fwd(lib, chunk=8) == -2
+    assert fwd(lib, dtype=7) == -2
+    assert fwd(lib, q=MIS) == -3
+    assert fwd(lib, S_final=MIS) == -3
+    assert fwd(lib, out=P) == -1        # out aliases q
+    assert fwd(lib, cu=P + 0x9002) == -3  # cu_seqlens must be 4-byte aligned
+    # packed batch with no sequences but tokens
+    assert fwd(lib, cu=P + 0x9000, B=0, T=5) == -1
+
+
+def test_fwd_fp32core_shares_validation(lib):
+    r = lib.ckda_fwd_chunked_fp32core(None, P, P, P, P, None, None, P + 16, None, 1, 8, 1, 16, 16,
+                                      16, 0, None)
+    assert r == -1
+
+
+def test_decode_argument_errors(lib):
+    def dec(**kw):
+        a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000,
+                 S=P + 0x5000, out=P + 0x6000, B=2, H=2, dk=16, dv=16, dtype=1)
+        a.update(kw)
+        return lib.ckda_decode_step(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S"], a["out"],
+                                    a["B"], a["H"], a["dk"], a["dv"], a["dtype"], None)
+
+    assert dec(S=None) == -1
+    assert dec(H=0) == -1
+    assert dec(dk=24) == -2
+    assert dec(dtype=3) == -2
+    assert dec(alpha=MIS) == -3
+    assert dec(out=P + 0x5000) == -1   # out aliases the state
+    assert dec(B=0) == 0               # nothing to do, nothing launched
+
+
+def test_zero_sequences_is_a_no_op(lib):
+    assert fwd(lib, B=0) == 0
