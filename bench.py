@@ -38,10 +38,10 @@ B, T, H, D, CHUNK = 4, 4096, 16, 128, 64
 DEC_B, DEC_H, DEC_STEPS = 256, 32, 1024
 
 # algorithmic counts per token-head (d = 128, C = 64)
-BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 2          # q,k,v bf16 + alpha + beta + out
+BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4          # q,k,v bf16 + alpha + beta + out fp32
 STRICT_FLOPS_PER_TOKEN_HEAD = 6 * CHUNK * D + 6 * D * D + CHUNK * CHUNK // 3
 DENSE_FLOPS_PER_TOKEN_HEAD = 12 * CHUNK * D + 6 * D * D
-DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 2
+DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4
 
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
@@ -64,7 +64,9 @@ def _args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
+    ap.add_argument("--decode-steps", type=int, default=DEC_STEPS,
+                    help="decode steps timed (inputs for all of them are pre-generated)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -267,7 +269,7 @@ def run_ours(args, ws, rank, local):
     # two input sets (each ~0.4 GB > 126 MB L2), rotated so no step finds its
     # inputs in L2
     sets = [inputs.kda_prefill(seed=1000 * rank + i, device=dev) for i in range(2)]
-    out = torch.empty_like(sets[0].v)
+    out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -319,7 +321,27 @@ def run_ours(args, ws, rank, local):
     traffic, _ = _traffic_from_profile()
 
     # ---- end to end: host (pinned) buffers through the public API --------
-    c = sets[0]
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = _run_e2e(args, ck, torch, sets[0], out, S_final, stream, barrier, max_over_ranks,
+                       ws, tokens, dev)
+
+    # ---- decode step (B=256, H=32, d=128, bf16), 1024 steps --------------
+    decode = None
+    if not args.no_decode:
+        decode = _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ranks,
+                             ws, hbm_peak)
+    _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
+            peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
+            _lib.LIB_PATH)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_over_ranks, ws, tokens, dev):
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
     host = {n: getattr(c, n).cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
     dbuf = {n: torch.empty_like(getattr(c, n)) for n in host}
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -349,42 +371,50 @@ def run_ours(args, ws, rank, local):
     barrier()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1)) / E
     e2e_value = ws * tokens / (e2e_ms / 1e3)
-    del dbuf, host
+    return {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    # ---- decode step (B=256, H=32, d=128, bf16), 1024 steps --------------
-    decode = None
-    if not args.no_decode:
-        dc = inputs.decode(seed=2000 + rank, device=dev, B=DEC_B, H=DEC_H, d=D, steps=DEC_STEPS)
-        S = dc.S0.clone()
-        dout = torch.empty((DEC_B, DEC_H, D), dtype=torch.bfloat16, device=dev)
-        for t in range(8):
-            ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
-        torch.cuda.synchronize(dev)
-        barrier()
-        ev0.record(stream)
-        for t in range(DEC_STEPS):
-            ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        dec_ms = max_over_ranks(ev0.elapsed_time(ev1)) / DEC_STEPS
-        dbytes = DEC_B * DEC_H * DEC_BYTES_PER_HEAD_STEP
-        dgbs = dbytes / (dec_ms / 1e3) / 1e9
-        decode = {"workload": f"decode B={DEC_B} H={DEC_H} d={D} bf16, {DEC_STEPS} steps",
-                  "ms_per_step": dec_ms, "tokens_per_s": ws * DEC_B / (dec_ms / 1e3),
-                  "achieved_gbs": dgbs, "hbm_frac_of_measured": dgbs / hbm_peak,
-                  "hbm_frac_of_spec_8tbs": dgbs / SPEC_HBM_GBS,
-                  "bytes_per_step": dbytes, "gpu_launches": DEC_STEPS}
-        del dc, S
 
-    lib_path = _lib.LIB_PATH
+def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ranks, ws, hbm_peak):
+    steps = max(1, args.decode_steps)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    dc = inputs.decode(seed=2000 + rank, device=dev, B=DEC_B, H=DEC_H, d=D, steps=steps + 8)
+    S = dc.S0.clone()
+    dout = torch.empty((DEC_B, DEC_H, D), dtype=torch.float32, device=dev)
+    for t in range(8):
+        ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ev0.record(stream)
+    for t in range(8, 8 + steps):
+        ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    dec_ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
+    dbytes = DEC_B * DEC_H * DEC_BYTES_PER_HEAD_STEP
+    dgbs = dbytes / (dec_ms / 1e3) / 1e9
+    decode = {"workload": f"decode B={DEC_B} H={DEC_H} d={D} bf16 q/k/v, fp32 out, "
+                          f"{steps} steps",
+              "ms_per_step": dec_ms, "tokens_per_s": ws * DEC_B / (dec_ms / 1e3),
+              "achieved_gbs": dgbs, "hbm_frac_of_measured": dgbs / hbm_peak,
+              "hbm_frac_of_spec_8tbs": dgbs / SPEC_HBM_GBS,
+              "bytes_per_step": dbytes, "gpu_launches": steps}
+    del dc, S
+    return decode
+
+
+def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
+            peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
+            lib_path):
     obj = {
         "metric": "CKDA fwd tokens/s (KDA-layer prefill T=4096, H=16, d=128)",
         "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": f"kda_prefill B={B} H={H} T={T} d_k=d_v={D} C={CHUNK} "
-                               "bf16 q/k/v, fp32 alpha/beta, S0=0, S_final stored",
+                               "bf16 q/k/v, fp32 alpha/beta, fp32 out, S0=0, S_final stored",
                    "global_batch": ws * B, "seq_len": T, "heads": H, "head_dim": D,
                    "chunk": CHUNK, "parallelism": f"replicas x{ws} (no data-path collective)",
                    "l2": "inputs larger than L2: two rotating 0.40 GB input sets"},
@@ -398,8 +428,7 @@ def run_ours(args, ws, rank, local):
                    "frac_strict_of_spec": tflops_strict / SPEC_BF16_TFLOPS,
                    "frac_dense_of_spec": tflops_dense / SPEC_BF16_TFLOPS,
                    "measured_bf16_tflops": tc_peak},
-        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "e2e": e2e,
         "gpu_launches": K,
         "clocks": clocks,
         "wall_s_timed_region": wall,
@@ -410,9 +439,6 @@ def run_ours(args, ws, rank, local):
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         obj["cpu_baseline"] = cpu_baseline()
     _emit(obj, args, rank)
-    if ws > 1:
-        dist.barrier()
-        dist.destroy_process_group()
 
 
 def main():

@@ -38,12 +38,14 @@ def _p(t: Optional[torch.Tensor]):
 
 
 def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
-                out=None, S_final=None, return_final: bool = True, fp32core: bool = False
-                ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                out=None, S_final=None, return_final: bool = True, fp32core: bool = False,
+                out_dtype=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked CKDA forward.  Shapes as in ``ckda_fwd_chunked`` (include/ckda.h).
 
     Fixed-length: q, k, alpha ``[B, T, H, dk]``; v ``[B, T, H, dv]``; beta ``[B, T, H]``.
     Packed: ``cu_seqlens`` int32 ``[N+1]`` and tensors with a leading 1 or without it.
+    ``out_dtype`` (float32 or bfloat16) defaults to the dtype of ``out`` if given,
+    else to the input dtype.
     Returns ``(out, S_final)``; ``S_final`` is None when ``return_final`` is False.
     """
     dev = q.device
@@ -77,10 +79,16 @@ def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
         _need(S0, "S0", torch.float32, dev)
         if tuple(S0.shape) != (N, H, dk, dv):
             raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
     if out is None:
-        out = torch.empty(v.shape, dtype=v.dtype, device=dev)
+        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
     else:
-        _need(out, "out", v.dtype, dev)
+        _need(out, "out", out_dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must have v's shape")
     if return_final and S_final is None:
         S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if S_final is not None:
@@ -88,16 +96,18 @@ def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
     fn = _lib.load().ckda_fwd_chunked_fp32core if fp32core else _lib.load().ckda_fwd_chunked
     with torch.cuda.device(dev):
         rc = fn(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(out),
-                _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _stream_ptr(dev))
+                _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
+                _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_fwd_chunked")
     return out, S_final
 
 
-def decode_step(q, k, v, alpha, beta, S, out=None) -> torch.Tensor:
+def decode_step(q, k, v, alpha, beta, S, out=None, out_dtype=None) -> torch.Tensor:
     """One recurrent step, in place on ``S`` ``[B, H, dk, dv]`` (fp32).
 
-    q, k, alpha ``[B, H, dk]``; v ``[B, H, dv]``; beta ``[B, H]``.  Returns ``out``.
+    q, k, alpha ``[B, H, dk]``; v ``[B, H, dv]``; beta ``[B, H]``.  Returns ``out``
+    (``out_dtype`` defaults to the dtype of ``out`` if given, else the input dtype).
     """
     dev = q.device
     if q.dtype not in _DT:
@@ -111,13 +121,18 @@ def decode_step(q, k, v, alpha, beta, S, out=None) -> torch.Tensor:
     dv = v.shape[-1]
     if tuple(S.shape) != (B, H, dk, dv) or tuple(beta.shape) != (B, H):
         raise ValueError("shape mismatch")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
     if out is None:
-        out = torch.empty((B, H, dv), dtype=v.dtype, device=dev)
+        out = torch.empty((B, H, dv), dtype=out_dtype, device=dev)
     else:
-        _need(out, "out", v.dtype, dev)
+        _need(out, "out", out_dtype, dev)
     with torch.cuda.device(dev):
         rc = _lib.load().ckda_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(out),
-                                          B, H, dk, dv, _DT[q.dtype], _stream_ptr(dev))
+                                          B, H, dk, dv, _DT[q.dtype], _DT[out_dtype],
+                                          _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_decode_step")
     return out

@@ -9,16 +9,16 @@
 #include "ckda.h"
 
 namespace ckda {
-cudaError_t launch_decode(int dtype, int dk, int dv, const void* q, const void* k, const void* v,
-                          const float* alpha, const float* beta, float* S, void* out, int BH,
-                          cudaStream_t stream);
-cudaError_t launch_fwd_simt(int dtype, int dk, int dv, const void* q, const void* k,
-                            const void* v, const float* alpha, const float* beta, const float* S0,
-                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
-                            int C, int* status, cudaStream_t stream);
+cudaError_t launch_decode(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k,
+                          const void* v, const float* alpha, const float* beta, float* S, void* out,
+                          int BH, cudaStream_t stream);
+cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
+                            const void* k, const void* v, const float* alpha, const float* beta,
+                            const float* S0, const int32_t* cu, void* out, float* S_final,
+                            int n_seqs, int T, int H, int C, int* status, cudaStream_t stream);
 // Returns cudaErrorNotSupported when the shape is not covered by the
 // tensor-core kernel (the caller then uses the CUDA-core kernel).
-cudaError_t launch_fwd_tc(int dtype, int dk, int dv, const void* q, const void* k, const void* v,
+cudaError_t launch_fwd_tc(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k, const void* v,
                           const float* alpha, const float* beta, const float* S0,
                           const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
                           int C, int* status, cudaStream_t stream);
@@ -53,9 +53,10 @@ bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 int validate_fwd(const void* q, const void* k, const void* v, const float* alpha,
                  const float* beta, const float* S0, const int32_t* cu, const void* out,
                  const float* S_final, int B, int T, int H, int d_k, int d_v, int* chunk,
-                 int dtype) {
+                 int dtype, int out_dtype) {
   if (B < 0 || T < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
   if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (out_dtype != CKDA_F32 && out_dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
   if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
   if (*chunk == 0) *chunk = 64;
   if (*chunk != 16 && *chunk != 32 && *chunk != 64) return CKDA_ERR_UNSUPPORTED;
@@ -74,9 +75,10 @@ int validate_fwd(const void* q, const void* k, const void* v, const float* alpha
 
 int fwd_impl(bool allow_tc, const void* q, const void* k, const void* v, const float* alpha,
              const float* beta, const float* S0, const int32_t* cu, void* out, float* S_final,
-             int B, int T, int H, int d_k, int d_v, int chunk, int dtype, void* stream) {
+             int B, int T, int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
+             void* stream) {
   int rc = validate_fwd(q, k, v, alpha, beta, S0, cu, out, S_final, B, T, H, d_k, d_v, &chunk,
-                        dtype);
+                        dtype, out_dtype);
   if (rc != CKDA_OK) return rc;
   const int n_seqs = B;
   if (n_seqs == 0) return CKDA_OK;
@@ -85,10 +87,10 @@ int fwd_impl(bool allow_tc, const void* q, const void* k, const void* v, const f
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (allow_tc)
-    e = ckda::launch_fwd_tc(dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs,
+    e = ckda::launch_fwd_tc(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs,
                             T, H, chunk, status, st);
   if (e == cudaErrorNotSupported)
-    e = ckda::launch_fwd_simt(dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final,
+    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final,
                               n_seqs, T, H, chunk, status, st);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
@@ -115,24 +117,25 @@ const char* ckda_status_string(int status) {
 int ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, const float* S0, const int32_t* cu_seqlens, void* out,
                      float* S_final, int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
-                     void* stream) {
+                     int out_dtype, void* stream) {
   return fwd_impl(true, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
-                  chunk, dtype, stream);
+                  chunk, dtype, out_dtype, stream);
 }
 
 int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void* v, const float* alpha,
                               const float* beta, const float* S0, const int32_t* cu_seqlens,
                               void* out, float* S_final, int B, int T, int H, int d_k, int d_v,
-                              int chunk, int dtype, void* stream) {
+                              int chunk, int dtype, int out_dtype, void* stream) {
   return fwd_impl(false, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
-                  chunk, dtype, stream);
+                  chunk, dtype, out_dtype, stream);
 }
 
 int ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, float* S_inout, void* out, int B, int H, int d_k, int d_v,
-                     int dtype, void* stream) {
+                     int dtype, int out_dtype, void* stream) {
   if (B < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
   if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (out_dtype != CKDA_F32 && out_dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
   if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
   if ((int64_t)B * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
   if (B == 0) return CKDA_OK;
@@ -141,7 +144,7 @@ int ckda_decode_step(const void* q, const void* k, const void* v, const float* a
   for (const void* p : ptrs)
     if (!aligned16(p)) return CKDA_ERR_MISALIGNED;
   if (out == S_inout || out == q || out == k || out == v) return CKDA_ERR_INVALID_ARG;
-  cudaError_t e = ckda::launch_decode(dtype, d_k, d_v, q, k, v, alpha, beta, S_inout, out, B * H,
+  cudaError_t e = ckda::launch_decode(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S_inout, out, B * H,
                                       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }

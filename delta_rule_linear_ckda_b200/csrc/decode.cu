@@ -29,12 +29,12 @@ struct DecodeShape {
   static_assert(DK % kRpp == 0, "row split");
 };
 
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, typename Tout>
 __global__ void __launch_bounds__(DecodeShape<DK, DV>::kThreads, 2)
 decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                    const Tin* __restrict__ v, const float* __restrict__ alpha,
                    const float* __restrict__ beta, float* __restrict__ S,
-                   Tin* __restrict__ out) {
+                   Tout* __restrict__ out) {
   using Sh = DecodeShape<DK, DV>;
   constexpr int CPR = Sh::kCpr, RPP = Sh::kRpp, NR = Sh::kRows, NT = Sh::kThreads;
   __shared__ float4 red_r[RPP][CPR];
@@ -115,49 +115,55 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   }
 }
 
-template <int DK, int DV, typename Tin>
+template <int DK, int DV, typename Tin, typename Tout>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* alpha,
                                    const float* beta, float* S, void* out, int BH,
                                    cudaStream_t stream) {
   using Sh = DecodeShape<DK, DV>;
-  decode_step_kernel<DK, DV, Tin><<<BH, Sh::kThreads, 0, stream>>>(
+  decode_step_kernel<DK, DV, Tin, Tout><<<BH, Sh::kThreads, 0, stream>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
-      beta, S, static_cast<Tin*>(out));
+      beta, S, static_cast<Tout*>(out));
   return cudaGetLastError();
 }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename Tout>
 static cudaError_t launch_decode_dv(int dv, const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, float* S, void* out,
                                     int BH, cudaStream_t stream) {
   switch (dv) {
-    case 16: return launch_decode_t<DK, 16, Tin>(q, k, v, alpha, beta, S, out, BH, stream);
-    case 32: return launch_decode_t<DK, 32, Tin>(q, k, v, alpha, beta, S, out, BH, stream);
-    case 64: return launch_decode_t<DK, 64, Tin>(q, k, v, alpha, beta, S, out, BH, stream);
-    case 128: return launch_decode_t<DK, 128, Tin>(q, k, v, alpha, beta, S, out, BH, stream);
+    case 16: return launch_decode_t<DK, 16, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
+    case 32: return launch_decode_t<DK, 32, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
+    case 64: return launch_decode_t<DK, 64, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
+    case 128: return launch_decode_t<DK, 128, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
   }
   return cudaErrorInvalidValue;
 }
 
-template <typename Tin>
+template <typename Tin, typename Tout>
 static cudaError_t launch_decode_dk(int dk, int dv, const void* q, const void* k, const void* v,
                                     const float* alpha, const float* beta, float* S, void* out,
                                     int BH, cudaStream_t stream) {
   switch (dk) {
-    case 16: return launch_decode_dv<16, Tin>(dv, q, k, v, alpha, beta, S, out, BH, stream);
-    case 32: return launch_decode_dv<32, Tin>(dv, q, k, v, alpha, beta, S, out, BH, stream);
-    case 64: return launch_decode_dv<64, Tin>(dv, q, k, v, alpha, beta, S, out, BH, stream);
-    case 128: return launch_decode_dv<128, Tin>(dv, q, k, v, alpha, beta, S, out, BH, stream);
+    case 16: return launch_decode_dv<16, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
+    case 32: return launch_decode_dv<32, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
+    case 64: return launch_decode_dv<64, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
+    case 128: return launch_decode_dv<128, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
   }
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_decode(int dtype, int dk, int dv, const void* q, const void* k, const void* v,
-                          const float* alpha, const float* beta, float* S, void* out, int BH,
-                          cudaStream_t stream) {
-  if (dtype == CKDA_BF16)
-    return launch_decode_dk<__nv_bfloat16>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
-  return launch_decode_dk<float>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
+cudaError_t launch_decode(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k,
+                          const void* v, const float* alpha, const float* beta, float* S, void* out,
+                          int BH, cudaStream_t stream) {
+  if (dtype == CKDA_BF16) {
+    if (out_dtype == CKDA_BF16)
+      return launch_decode_dk<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, alpha, beta, S, out,
+                                                            BH, stream);
+    return launch_decode_dk<__nv_bfloat16, float>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
+  }
+  if (out_dtype == CKDA_BF16)
+    return launch_decode_dk<float, __nv_bfloat16>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
+  return launch_decode_dk<float, float>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
 }
 
 }  // namespace ckda

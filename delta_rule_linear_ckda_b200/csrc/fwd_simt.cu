@@ -99,11 +99,11 @@ __device__ __forceinline__ void reduce_scatter8(float* v, int lane) {
   v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
 }
 
-template <int DK, int BV, typename Tin>
+template <int DK, int BV, typename Tin, typename Tout>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta,
-                const float* S0, const int32_t* __restrict__ cu, Tin* __restrict__ out,
+                const float* S0, const int32_t* __restrict__ cu, Tout* __restrict__ out,
                 float* S_final, int n_seqs, int T, int H, int DV, int C, int* status) {
   using L = Smem<DK, BV>;
   constexpr int KS = L::KS, VS = L::VS, CS = L::CS;
@@ -367,55 +367,57 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
   }
 }
 
-template <int DK, int BV, typename Tin>
+template <int DK, int BV, typename Tin, typename Tout>
 static cudaError_t launch_t(const void* q, const void* k, const void* v, const float* alpha,
                             const float* beta, const float* S0, const int32_t* cu, void* out,
                             float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
                             cudaStream_t stream) {
   using L = Smem<DK, BV>;
-  auto kern = fwd_simt_kernel<DK, BV, Tin>;
+  auto kern = fwd_simt_kernel<DK, BV, Tin, Tout>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(DV / BV, H, n_seqs);
   kern<<<grid, kThreads, L::kBytes, stream>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
-      beta, S0, cu, static_cast<Tin*>(out), S_final, n_seqs, T, H, DV, C, status);
+      beta, S0, cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
   return cudaGetLastError();
 }
 
-template <int DK, typename Tin>
+template <int DK, typename Tin, typename Tout>
 static cudaError_t launch_bv(const void* q, const void* k, const void* v, const float* alpha,
                              const float* beta, const float* S0, const int32_t* cu, void* out,
                              float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
                              cudaStream_t stream) {
   switch (DV) {
     case 16:
-      return launch_t<DK, 16, Tin>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
+      return launch_t<DK, 16, Tin, Tout>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
                                    C, status, stream);
     case 32:
-      return launch_t<DK, 32, Tin>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
+      return launch_t<DK, 32, Tin, Tout>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
                                    C, status, stream);
     default:  // 64 and 128: slices of 64 columns
-      return launch_t<DK, 64, Tin>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
+      return launch_t<DK, 64, Tin, Tout>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
                                    C, status, stream);
   }
 }
 
 }  // namespace simt
 
-cudaError_t launch_fwd_simt(int dtype, int dk, int dv, const void* q, const void* k,
-                            const void* v, const float* alpha, const float* beta, const float* S0,
-                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
-                            int C, int* status, cudaStream_t stream) {
-#define CKDA_SIMT_DK(DKV)                                                                       \
-  case DKV:                                                                                     \
-    return (dtype == CKDA_BF16)                                                                 \
-               ? simt::launch_bv<DKV, __nv_bfloat16>(q, k, v, alpha, beta, S0, cu, out,        \
-                                                      S_final, n_seqs, T, H, dv, C, status,     \
-                                                      stream)                                   \
-               : simt::launch_bv<DKV, float>(q, k, v, alpha, beta, S0, cu, out, S_final,       \
-                                             n_seqs, T, H, dv, C, status, stream);
+cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
+                            const void* k, const void* v, const float* alpha, const float* beta,
+                            const float* S0, const int32_t* cu, void* out, float* S_final,
+                            int n_seqs, int T, int H, int C, int* status, cudaStream_t stream) {
+#define CKDA_SIMT_CALL(DKV, TI, TO)                                                           \
+  simt::launch_bv<DKV, TI, TO>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, dv, C, \
+                               status, stream)
+#define CKDA_SIMT_DK(DKV)                                                                  \
+  case DKV:                                                                                \
+    if (dtype == CKDA_BF16)                                                                \
+      return out_dtype == CKDA_BF16 ? CKDA_SIMT_CALL(DKV, __nv_bfloat16, __nv_bfloat16)    \
+                                    : CKDA_SIMT_CALL(DKV, __nv_bfloat16, float);           \
+    return out_dtype == CKDA_BF16 ? CKDA_SIMT_CALL(DKV, float, __nv_bfloat16)              \
+                                  : CKDA_SIMT_CALL(DKV, float, float);
   switch (dk) {
     CKDA_SIMT_DK(16)
     CKDA_SIMT_DK(32)
@@ -423,6 +425,7 @@ cudaError_t launch_fwd_simt(int dtype, int dk, int dv, const void* q, const void
     CKDA_SIMT_DK(128)
   }
 #undef CKDA_SIMT_DK
+#undef CKDA_SIMT_CALL
   return cudaErrorInvalidValue;
 }
 

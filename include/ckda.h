@@ -25,10 +25,12 @@
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call is asynchronous on that stream and returns as soon
  *    as the work is enqueued.
- *  - dtype selects the element type of q, k, v and out: CKDA_F32 or
- *    CKDA_BF16.  alpha, beta, S0, S_final and S_inout are always fp32.
- *    Outputs are rounded to the output type with round-to-nearest-even from
- *    fp32 accumulators; the state stays fp32.
+ *  - dtype selects the element type of q, k and v, out_dtype the element
+ *    type of out: each CKDA_F32 or CKDA_BF16.  alpha, beta, S0, S_final and
+ *    S_inout are always fp32.  Every output element is computed in fp32 and
+ *    stored as fp32, or rounded once to bf16 (round-to-nearest-even) when
+ *    out_dtype is CKDA_BF16, so a bf16 output is exactly the bf16 rounding
+ *    of the fp32 output of the same call.  The state stays fp32.
  *  - Return value: CKDA_OK (0) or a negative CKDA_ERR_* code.  On an
  *    argument error nothing is launched and no memory is touched.  Errors
  *    found on the device (a bad cu_seqlens array, a bounded wait that timed
@@ -62,7 +64,8 @@ enum {
   CKDA_ERR_INVALID_ARG = -1,   /* NULL required pointer, negative or
                                   inconsistent sizes */
   CKDA_ERR_UNSUPPORTED = -2,   /* d_k or d_v not in {16,32,64,128}, chunk
-                                  not in {0,16,32,64}, unknown dtype */
+                                  not in {0,16,32,64}, unknown dtype or
+                                  out_dtype */
   CKDA_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned */
   CKDA_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
   CKDA_ERR_DEVICE_TIMEOUT = -5,/* a bounded device-side wait gave up */
@@ -107,7 +110,7 @@ CKDA_API int ckda_fwd_chunked(const void* q, const void* k, const void* v,
                      const float* alpha, const float* beta, const float* S0,
                      const int32_t* cu_seqlens, void* out, float* S_final,
                      int B, int T, int H, int d_k, int d_v, int chunk,
-                     int dtype, void* stream);
+                     int dtype, int out_dtype, void* stream);
 
 /*
  * ckda_fwd_chunked_fp32core -- the same operation and arguments as
@@ -122,7 +125,7 @@ CKDA_API int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void*
                               const float* S0, const int32_t* cu_seqlens,
                               void* out, float* S_final, int B, int T, int H,
                               int d_k, int d_v, int chunk, int dtype,
-                              void* stream);
+                              int out_dtype, void* stream);
 
 /*
  * ckda_decode_step -- one recurrent token for B independent sequences,
@@ -135,7 +138,7 @@ CKDA_API int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void*
 CKDA_API int ckda_decode_step(const void* q, const void* k, const void* v,
                      const float* alpha, const float* beta, float* S_inout,
                      void* out, int B, int H, int d_k, int d_v, int dtype,
-                     void* stream);
+                     int out_dtype, void* stream);
 
 /* Human-readable text for a CKDA_* status code (static storage). */
 CKDA_API const char* ckda_status_string(int status);

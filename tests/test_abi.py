@@ -76,11 +76,11 @@ MIS = (1 << 20) + 4  # misaligned
 def fwd(lib, **kw):
     a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000, S0=None,
              cu=None, out=P + 0x5000, S_final=None, B=1, T=8, H=1, dk=16, dv=16, chunk=16,
-             dtype=0, stream=None)
+             dtype=0, out_dtype=0, stream=None)
     a.update(kw)
     return lib.ckda_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S0"], a["cu"],
                                 a["out"], a["S_final"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
-                                a["chunk"], a["dtype"], a["stream"])
+                                a["chunk"], a["dtype"], a["out_dtype"], a["stream"])
 
 
 def test_fwd_argument_errors(lib):
@@ -95,6 +95,7 @@ def test_fwd_argument_errors(lib):
     assert fwd(lib, chunk=128) == -2
     assert fwd(lib, chunk=8) == -2
     assert fwd(lib, dtype=7) == -2
+    assert fwd(lib, out_dtype=2) == -2
     assert fwd(lib, q=MIS) == -3
     assert fwd(lib, S_final=MIS) == -3
     assert fwd(lib, out=P) == -1        # out aliases q
@@ -105,22 +106,24 @@ def test_fwd_argument_errors(lib):
 
 def test_fwd_fp32core_shares_validation(lib):
     r = lib.ckda_fwd_chunked_fp32core(None, P, P, P, P, None, None, P + 16, None, 1, 8, 1, 16, 16,
-                                      16, 0, None)
+                                      16, 0, 0, None)
     assert r == -1
 
 
 def test_decode_argument_errors(lib):
     def dec(**kw):
         a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000,
-                 S=P + 0x5000, out=P + 0x6000, B=2, H=2, dk=16, dv=16, dtype=1)
+                 S=P + 0x5000, out=P + 0x6000, B=2, H=2, dk=16, dv=16, dtype=1, out_dtype=0)
         a.update(kw)
         return lib.ckda_decode_step(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S"], a["out"],
-                                    a["B"], a["H"], a["dk"], a["dv"], a["dtype"], None)
+                                    a["B"], a["H"], a["dk"], a["dv"], a["dtype"], a["out_dtype"],
+                                    None)
 
     assert dec(S=None) == -1
     assert dec(H=0) == -1
     assert dec(dk=24) == -2
     assert dec(dtype=3) == -2
+    assert dec(out_dtype=-1) == -2
     assert dec(alpha=MIS) == -3
     assert dec(out=P + 0x5000) == -1   # out aliases the state
     assert dec(B=0) == 0               # nothing to do, nothing launched

@@ -27,7 +27,7 @@ def ck():
 
 def _run_vs_oracle(ck, case, tol, fp32core=False):
     out, S = ck.fwd_chunked(case.q, case.k, case.v, case.alpha, case.beta, S0=case.S0,
-                            chunk=case.chunk, fp32core=fp32core)
+                            chunk=case.chunk, fp32core=fp32core, out_dtype=torch.float32)
     assert ck.device_status() == 0
     ro, rS, _, _ = oracle_fixed(case)
     eo, es = rel_max_err(out, ro), rel_max_err(S, rS)
@@ -129,17 +129,18 @@ def test_chunk_size_independence_and_resume(ck, dtype, tol):
     case = inputs.random_prefill(2, 300, 4, 128, 128, dtype=dtype, gates="kda", s0_std=0.02,
                                  chunk=64, seed=22, device=DEV)
     ref, Sref = ck.fwd_chunked(case.q, case.k, case.v, case.alpha, case.beta, S0=case.S0,
-                               chunk=64, fp32core=True)
+                               chunk=64, fp32core=True, out_dtype=torch.float32)
     for C in (16, 32, 64):
-        o, S = ck.fwd_chunked(case.q, case.k, case.v, case.alpha, case.beta, S0=case.S0, chunk=C)
+        o, S = ck.fwd_chunked(case.q, case.k, case.v, case.alpha, case.beta, S0=case.S0, chunk=C,
+                              out_dtype=torch.float32)
         assert rel_max_err(o, ref.double().cpu().numpy()) <= tol
         assert rel_max_err(S, Sref.double().cpu().numpy()) <= tol
     # split call at T1 = 100 (not a chunk multiple) and resume from S_final
     T1 = 100
     parts = [x[:, :T1].contiguous() for x in (case.q, case.k, case.v, case.alpha, case.beta)]
     rest = [x[:, T1:].contiguous() for x in (case.q, case.k, case.v, case.alpha, case.beta)]
-    o_a, S_mid = ck.fwd_chunked(*parts, S0=case.S0)
-    o_b, S_end = ck.fwd_chunked(*rest, S0=S_mid)
+    o_a, S_mid = ck.fwd_chunked(*parts, S0=case.S0, out_dtype=torch.float32)
+    o_b, S_end = ck.fwd_chunked(*rest, S0=S_mid, out_dtype=torch.float32)
     assert rel_max_err(torch.cat([o_a, o_b], 1), ref.double().cpu().numpy()) <= tol
     assert rel_max_err(S_end, Sref.double().cpu().numpy()) <= tol
 
