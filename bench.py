@@ -333,9 +333,10 @@ def run_ours(args, ws, rank, local):
     if not args.no_decode:
         decode = _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ranks,
                              ws, hbm_peak)
+    path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
     _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            _lib.LIB_PATH)
+            _lib.LIB_PATH, path)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -409,12 +410,17 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ra
 
 def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            lib_path):
+            lib_path, path):
+    # arithmetic of the forward: tcgen05 MMAs on fp16 operands with fp32
+    # accumulation and fp32 state, or fp32 FFMA on CUDA cores
+    dtype = "f16" if path == "tcgen05" else "f32"
     obj = {
         "metric": "CKDA fwd tokens/s (KDA-layer prefill T=4096, H=16, d=128)",
         "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "compute": {"kernel": path, "mma_operands": "f16" if path == "tcgen05" else None,
+                    "accumulate": "f32", "state": "f32", "inputs": "bf16 q/k/v, f32 gates"},
         "config": {"workload": f"kda_prefill B={B} H={H} T={T} d_k=d_v={D} C={CHUNK} "
                                "bf16 q/k/v, fp32 alpha/beta, fp32 out, S0=0, S_final stored",
                    "global_batch": ws * B, "seq_len": T, "heads": H, "head_dim": D,

@@ -30,6 +30,7 @@ _i = ctypes.c_int
 SIGNATURES = {
     "ckda_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_fwd_chunked_fp32core": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "ckda_fwd_chunked_path": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_device_status": (_i, [_vp]),

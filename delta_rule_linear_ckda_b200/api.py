@@ -103,6 +103,16 @@ def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
     return out, S_final
 
 
+def fwd_path(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, out_dtype=torch.float32,
+             varlen=False) -> str:
+    """Which kernel ``fwd_chunked`` runs for these sizes: "tcgen05" or "fp32core"."""
+    rc = _lib.load().ckda_fwd_chunked_path(B, T, H, dk, dv, chunk, _DT[dtype], _DT[out_dtype],
+                                           1 if varlen else 0)
+    if rc < 0:
+        raise CKDAError(rc, "ckda_fwd_chunked_path")
+    return "tcgen05" if rc == 1 else "fp32core"
+
+
 def decode_step(q, k, v, alpha, beta, S, out=None, out_dtype=None) -> torch.Tensor:
     """One recurrent step, in place on ``S`` ``[B, H, dk, dv]`` (fp32).
 

@@ -22,6 +22,7 @@ cudaError_t launch_fwd_tc(int dtype, int out_dtype, int dk, int dv, const void* 
                           const float* alpha, const float* beta, const float* S0,
                           const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
                           int C, int* status, cudaStream_t stream);
+bool fwd_tc_supported(int dtype, int dk, int dv, int C, uint64_t rows);
 }  // namespace ckda
 
 // First device-side error since the last ckda_device_status() call.
@@ -128,6 +129,20 @@ int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void* v, const
                               int chunk, int dtype, int out_dtype, void* stream) {
   return fwd_impl(false, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
                   chunk, dtype, out_dtype, stream);
+}
+
+int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
+                          int out_dtype, int varlen) {
+  // Sizes only: validate with stand-in aligned pointers that are never used.
+  const void* p = reinterpret_cast<const void*>(static_cast<uintptr_t>(1) << 20);
+  const int32_t* cu = varlen ? reinterpret_cast<const int32_t*>(static_cast<uintptr_t>(2) << 20)
+                             : nullptr;
+  int rc = validate_fwd(p, p, p, static_cast<const float*>(p), static_cast<const float*>(p),
+                        nullptr, cu, reinterpret_cast<const void*>(static_cast<uintptr_t>(3) << 20),
+                        nullptr, B, T, H, d_k, d_v, &chunk, dtype, out_dtype);
+  if (rc != CKDA_OK) return rc;
+  const uint64_t rows = varlen ? (uint64_t)T : (uint64_t)B * (uint64_t)T;
+  return ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, rows) ? 1 : 0;
 }
 
 int ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,

@@ -23,17 +23,25 @@
 // Division-free score blocks: every pair s < r is split at the anchor m of
 // the highest bit in which r and s differ ("level" h, block size b = 2^h):
 // P(r, s) = [alpha_m ... alpha_r] * [alpha_{s+1} ... alpha_{m-1}], two
-// running products that restart at the anchor.  Each level is one GEMM of
-// the anchored operands, so zero and negative gates are exact and underflow
-// goes to zero; no logarithm or division is taken.
+// running products that restart at the anchor.  Levels 2..5 (blocks of 4 to
+// 32) are one GEMM each on the anchored operands; levels 0..1 (pairs inside
+// aligned blocks of 4) are direct fp32 dot products.  Zero and negative
+// gates are exact and underflow goes to zero; no logarithm or division.
+//
+// All gate products of a chunk come from one pass over 8-position groups:
+// every thread owns 4 channels of one group, forms the running products of
+// its 8 positions, and combines them with the products of whole groups
+// (exchanged through shared memory) into the level operands and into
+// K * Gamma, Q * Gamma and K * rho.  The pass runs once per 64-channel half
+// of d_k, so the level GEMMs are split along K and the next chunk's inputs
+// stream in by TMA while the rest of the chunk runs.
 //
 // One CTA (256 threads) owns one (sequence, head, 64-column d_v slice) and
-// walks its chunks in order.  Inputs arrive by TMA; operands are fp16 tiles
-// in 128-byte-swizzled shared memory; accumulators live in tensor memory;
-// the state slice stays in fp32 registers (row i = tensor-memory lane i).
-// Every mbarrier wait is bounded: on time-out the kernel records
-// CKDA_ERR_DEVICE_TIMEOUT, waits once more (bounded) for its own copies,
-// frees its tensor memory and returns.
+// walks its chunks in order.  Operands are fp16 tiles in 128-byte-swizzled
+// shared memory; accumulators live in tensor memory; the state slice stays
+// in fp32 registers (row i = tensor-memory lane i).  Every mbarrier wait is
+// bounded: on time-out the kernel records CKDA_ERR_DEVICE_TIMEOUT, waits once
+// more (bounded) for its own copies, frees its tensor memory and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -47,60 +55,66 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int DK = 128;
+constexpr int HC = 64;  // channels per half of d_k
 constexpr int BV = 64;
 constexpr int NT = 256;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
 // ---- shared memory map (byte offsets from a 1024-aligned base) ----------
-// region X: TMA tiles of q, k (bf16 [64][128]) and alpha (fp32 [64][128]);
-// reused for the fp32 inverse workspace and the A / Inv / P operand tiles,
-// then for the [W; Q'] operand tile.
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = 16384;
-constexpr uint32_t OFF_A = 32768;
-constexpr uint32_t OFF_TF = 0;       // T, fp32 [64][64]
-constexpr uint32_t OFF_INV = 16384;  // (I + T)^-1, fp32 [64][64]
-constexpr uint32_t OFF_AQ = 32768;   // A, fp16 K-major [64 r][64 s]
-constexpr uint32_t OFF_IP = 40960;   // [Inv diag(beta); P], fp16 K-major [128][64]
-constexpr uint32_t OFF_YF = 57344;   // inverse scratch, fp32 [16][48]
-constexpr uint32_t OFF_WQ = 0;       // [W; Q'], fp16 K-major [128][128]
-// region Y: score operands of two levels, then K * Gamma and Q * Gamma.
-constexpr uint32_t OFF_LOP0 = 65536;  // [beta K L; Q L], fp16 K-major [64][128]
-constexpr uint32_t OFF_LOP1 = 81920;
-constexpr uint32_t OFF_ROP0 = 98304;  // K R, fp16 K-major [32][128]
-constexpr uint32_t OFF_ROP1 = 106496;
-constexpr uint32_t OFF_KG = 65536;   // K * Gamma, fp16 MN-major [64 s][128 i]
-constexpr uint32_t OFF_QG = 81920;   // Q * Gamma, fp16 row-major [64][QG_STRIDE]
-constexpr int QG_STRIDE = 136;
-// dedicated tiles
-constexpr uint32_t OFF_KH = 114688;  // K * rho, fp16 MN-major [64 s][128 i]
-constexpr uint32_t OFF_V = 131072;   // v slice (TMA, 128B swizzle), bf16 -> fp16 [64 s][64 j]
-constexpr uint32_t OFF_SB = 139264;  // state slice, fp16 MN-major [128 i][64 j]
-constexpr uint32_t OFF_UB = 155648;  // U, fp16 MN-major [64 s][64 j]
-constexpr uint32_t OFF_BETA = 163840;
-constexpr uint32_t OFF_GAMMA = 164096;
-constexpr uint32_t OFF_ADIAG = 164608;
-constexpr uint32_t OFF_BAR = 164864;  // mbarriers: tma, mma, level0, level1
-constexpr uint32_t OFF_TMEMPTR = 164896;
-constexpr uint32_t kSmemUsed = 164912;
+// Two input buffers, one per 64-channel half: q, k (bf16 [64 pos][64 ch])
+// and alpha (fp32 [64 pos][64 ch]), filled by TMA.
+constexpr uint32_t OFF_IN0 = 0;
+constexpr uint32_t OFF_IN1 = 32768;
+constexpr uint32_t IN_Q = 0, IN_K = 8192, IN_A = 16384, kInBytes = 32768;
+constexpr uint32_t OFF_V = 65536;  // v slice (TMA, 128B swizzle), bf16 -> fp16 [64 s][64 j]
+// Work region: level operands while the gate pass runs; then the fp32
+// inverse workspace and the A / [Inv; P] operands; then the U operand.
+constexpr uint32_t OFF_LVX = 73728;
+constexpr uint32_t kLvBytes = 12288;          // per level: LOP 8 KB + ROP 4 KB
+constexpr uint32_t LV_ROP = 8192;
+constexpr uint32_t OFF_TF = OFF_LVX;          // T, fp32 [64][64]
+constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A staging then (I + T)^-1, fp32 [64][64]
+constexpr uint32_t OFF_AQ = OFF_LVX + 32768;  // A, fp16 K-major [64 r][64 s]
+constexpr uint32_t OFF_IP = OFF_LVX + 40960;  // [Inv diag(beta); P], fp16 K-major [128][64]
+constexpr uint32_t OFF_YF = OFF_LVX + 57344;  // doubling scratch, fp32 (<= 1024 values)
+constexpr uint32_t OFF_UB = OFF_LVX;          // U, fp16 MN-major [64 s][64 j]
+constexpr uint32_t OFF_KG = 139264;  // K * Gamma, fp16 MN-major [64 s][128 i]
+constexpr uint32_t OFF_WQ = 155648;  // [W; Q'] fp16 K-major [128][128]; rows 64.. hold Q * Gamma first
+constexpr uint32_t OFF_KH = 188416;  // K * rho, fp16 MN-major [64 s][128 i]
+constexpr uint32_t OFF_SB = 204800;  // state slice, fp16 MN-major [128 i][64 j]
+constexpr uint32_t OFF_GT = 221184;  // products of whole 8-position groups, fp32 [8][64]
+constexpr uint32_t OFF_PR = 223232;  // direct pairs and diag(A), fp32 [8 groups][32]
+constexpr uint32_t OFF_BETA = 224256;
+constexpr uint32_t OFF_GAMMA = 224512;
+constexpr uint32_t OFF_BAR = 225024;  // mbarriers: in0, in1, v, mma, lv
+constexpr uint32_t OFF_TMEMPTR = 225088;
+constexpr uint32_t kSmemUsed = 225104;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 
-constexpr uint32_t kTmaBytes = 16384 + 16384 + 32768 + 8192;
-
 // ---- tensor memory columns ------------------------------------------------
-constexpr uint32_t TM_SCORE = 0;  // 6 levels x 32 columns (M = 64 layout)
-constexpr uint32_t TM_P = 192;    // P (M = 64 layout)
-constexpr uint32_t TM_W = 256;    // [W; A W]       (M = 128, 128 columns)
-constexpr uint32_t TM_U = 384;    // [U~; A U~]     (M = 128, 64 columns)
-constexpr uint32_t TM_X = 448;    // [W S; Q' S]    (M = 128, 64 columns)
-constexpr uint32_t TM_D = 0;      // (K rho)^T U    (M = 128, 64 columns)
-
-__device__ __forceinline__ float bf(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+constexpr uint32_t TM_LV = 0;    // levels 2..5, 32 columns each (M = 64 layout)
+constexpr uint32_t TM_P = 128;   // P (M = 64 layout)
+constexpr uint32_t TM_W = 192;   // [W; A W]       (M = 128, 128 columns)
+constexpr uint32_t TM_U = 320;   // [U~; A U~]     (M = 128, 64 columns)
+constexpr uint32_t TM_X = 384;   // [W S; Q' S]    (M = 128, 64 columns)
+constexpr uint32_t TM_D = 448;   // (K rho)^T U    (M = 128, 64 columns)
 
 #ifdef CKDA_TC_DEBUG
-// Intermediate dump of the first chunk of CTA (0, 0, 0) (diagnostic builds only).
+// Intermediate dump of the first chunk of CTA (0, 0, 0) and per-phase clock
+// counts (diagnostic builds only).
 __device__ float* g_tc_dbg = nullptr;
+__device__ unsigned long long* g_tc_time = nullptr;
+__device__ unsigned long long* g_tc_time2 = nullptr;
+#define GP_MARK(k)                                                                     \
+  do {                                                                                 \
+    if (g_tc_time2 != nullptr && (tid == 0 || tid == 32) && blockIdx.x == 0 &&         \
+        blockIdx.y == 0 && blockIdx.z == 0) {                                          \
+      const long long now = clock64();                                                 \
+      atomicAdd(g_tc_time2 + 4 * (tid >> 5) + (k), (unsigned long long)(now - gp_last)); \
+      gp_last = now;                                                                   \
+    }                                                                                  \
+  } while (0)
 #define TC_DBG(stmt)                                                                   \
   do {                                                                                 \
     if (g_tc_dbg != nullptr && c == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&         \
@@ -108,9 +122,24 @@ __device__ float* g_tc_dbg = nullptr;
       stmt;                                                                            \
     }                                                                                  \
   } while (0)
+#define TC_MARK(k)                                                                       \
+  do {                                                                                   \
+    if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&        \
+        blockIdx.z == 0) {                                                               \
+      const long long now = clock64();                                                   \
+      tmark[k] += now - tlast;                                                           \
+      tlast = now;                                                                       \
+    }                                                                                    \
+  } while (0)
 #else
+#define GP_MARK(k) \
+  do {             \
+  } while (0)
 #define TC_DBG(stmt) \
   do {               \
+  } while (0)
+#define TC_MARK(k) \
+  do {             \
   } while (0)
 #endif
 
@@ -120,8 +149,11 @@ __device__ float* g_tc_dbg = nullptr;
 // 2^-11 relative instead of bf16's 2^-9.  The values involved are bounded
 // (|k|, |q| <= 1 per element after normalisation, |gate products| <= 1), far
 // inside fp16's range.
-__device__ __forceinline__ void st_h(uint8_t* base, uint32_t off, float x) {
-  *reinterpret_cast<__half*>(base + off) = __float2half_rn(x);
+__device__ __forceinline__ void st_h4(uint8_t* base, uint32_t off, float4 v) {
+  uint2 pk;
+  pk.x = pack_f16x2(v.x, v.y);
+  pk.y = pack_f16x2(v.z, v.w);
+  *reinterpret_cast<uint2*>(base + off) = pk;
 }
 
 __device__ __forceinline__ void st_chunk8(uint8_t* base, uint32_t off, const float* v) {
@@ -133,8 +165,42 @@ __device__ __forceinline__ void st_chunk8(uint8_t* base, uint32_t off, const flo
   *reinterpret_cast<uint4*>(base + off) = pk;
 }
 
+__device__ __forceinline__ float4 mul4(float4 a, float4 b) {
+  return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
+}
+
+__device__ __forceinline__ float4 scale4(float s, float4 a) {
+  return make_float4(s * a.x, s * a.y, s * a.z, s * a.w);
+}
+
+__device__ __forceinline__ float dot4(float4 a, float4 b) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, a.w * b.w)));
+}
+
+__device__ __forceinline__ float4 ld_bf4(const uint8_t* p) {
+  const uint2 raw = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 __device__ __forceinline__ uint32_t taddr(uint32_t tmem, int lane_base, uint32_t col) {
   return tmem + ((uint32_t)lane_base << 16) + col;
+}
+
+// Sum a 16-vector over the 16 lanes of a half-warp; afterwards lane L of the
+// half holds the total of element (L & 15) in w[0].
+__device__ __forceinline__ void reduce_scatter16(float* w, int lane) {
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = up ? w[i] : w[i + o];
+      const float keep = up ? w[i + o] : w[i];
+      w[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
 }
 
 template <typename Tout>
@@ -162,6 +228,255 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
   }
 }
 
+// One gate pass over one 64-channel half (see the file comment).  Thread
+// (c4, g, role): channels 4*c4 .. 4*c4+3 of the half, positions 8g .. 8g+7.
+// Role 0 walks forward (prefix products: Gamma and the right halves of
+// levels 2..5); role 1 walks backward (suffix products: rho and the left
+// halves) and adds its channels' share of the direct pairs of levels 0..1
+// and of diag(A) into the pair buffer (stored by half 0, added by half 1).
+// The role is the warp's
+// parity, so the two warps sharing a scheduler (w and w + 4) run the same
+// code; one out-of-line copy serves both halves.
+__device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid) {
+  const int role = (tid >> 5) & 1;
+  const int rt = ((tid >> 6) << 5) | (tid & 31);  // index among the 128 threads of this role
+  const int c4 = rt & 15;
+  const int g = rt >> 4;
+  const int cl = 4 * c4;
+  const int ig = HC * hh + cl;
+  const float4 one = make_float4(1.f, 1.f, 1.f, 1.f);
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  auto bf4 = [](uint2 raw) -> float4 {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  };
+  auto h4 = [](float4 v) -> uint2 {
+    uint2 pk;
+    pk.x = pack_f16x2(v.x, v.y);
+    pk.y = pack_f16x2(v.z, v.w);
+    return pk;
+  };
+
+  // every input of this thread's 8 positions, loaded up front
+  float4 aa[8], ka[8], qa[8];
+  float bb[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int p = 8 * g + u;
+    const bool val = p < Lc;
+    aa[u] = val ? lds_f4(in + IN_A + p * 256 + cl * 4) : one;
+    ka[u] = val ? bf4(lds_u2(in + IN_K + p * 128 + cl * 2)) : zero;
+    qa[u] = val ? bf4(lds_u2(in + IN_Q + p * 128 + cl * 2)) : zero;
+    bb[u] = lds_f(sb + OFF_BETA + p * 4);
+  }
+#ifdef CKDA_TC_DEBUG
+  long long gp_last = clock64();
+#endif
+  // products of whole groups
+  const uint32_t gt = sb + OFF_GT + cl * 4;
+  if (role == 0) {
+    float4 t = aa[0];
+#pragma unroll
+    for (int u = 1; u < 8; ++u) t = mul4(t, aa[u]);
+    sts_f4(gt + g * HC * 4, t);
+  }
+  GP_MARK(0);
+  __syncthreads();
+  GP_MARK(1);
+  auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * HC * 4); };
+  const uint32_t LV = sb + OFF_LVX;
+  auto lop = [&](int lv, int row) -> uint32_t {
+    return LV + (lv - 2) * kLvBytes + sw128_elem(row, cl, 64);
+  };
+  auto rop = [&](int lv, int row) -> uint32_t {
+    return LV + (lv - 2) * kLvBytes + LV_ROP + sw128_elem(row, cl, 32);
+  };
+
+  if (role == 0) {
+    float4 pg = one;  // Gamma offset: product of the earlier groups
+    for (int gg = 0; gg < g; ++gg) pg = mul4(pg, gtot(gg));
+    float4 off4 = one, off5 = one;
+    if ((g & 3) == 3) off4 = gtot(g - 1);
+    for (int gg = 4; gg < g; ++gg) off5 = mul4(off5, gtot(gg));
+    float4 lp = one, l2 = one;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int p = 8 * g + u;
+      const float4 a = aa[u];
+      const float4 kf = ka[u];
+      const float4 qf = qa[u];
+      const float4 bk = scale4(bb[u], kf);
+      pg = mul4(pg, a);
+      lp = (u == 0) ? a : mul4(lp, a);
+      sts_u2(sb + OFF_KG + sw128_elem(p, ig, 64), h4(mul4(kf, pg)));
+      sts_u2(sb + OFF_WQ + sw128_elem(64 + p, ig, 128), h4(mul4(qf, pg)));
+      if (u >= 4) {  // level 2: right half of the group
+        l2 = (u == 4) ? a : mul4(l2, a);
+        const int rho = 4 * g + u - 4;
+        sts_u2(lop(2, rho), h4(mul4(bk, l2)));
+        sts_u2(lop(2, 32 + rho), h4(mul4(qf, l2)));
+      }
+      if (g & 1) {  // level 3: right half
+        const int rho = 8 * (g >> 1) + u;
+        sts_u2(lop(3, rho), h4(mul4(bk, lp)));
+        sts_u2(lop(3, 32 + rho), h4(mul4(qf, lp)));
+      }
+      if (g & 2) {  // level 4: right half
+        const float4 L = mul4(off4, lp);
+        const int rho = 16 * (g >> 2) + 8 * (g & 1) + u;
+        sts_u2(lop(4, rho), h4(mul4(bk, L)));
+        sts_u2(lop(4, 32 + rho), h4(mul4(qf, L)));
+      }
+      if (g & 4) {  // level 5: right half
+        const float4 L = mul4(off5, lp);
+        const int rho = 8 * (g - 4) + u;
+        sts_u2(lop(5, rho), h4(mul4(bk, L)));
+        sts_u2(lop(5, 32 + rho), h4(mul4(qf, L)));
+      }
+    }
+    if (g == 7) sts_f4(sb + OFF_GAMMA + ig * 4, pg);
+    GP_MARK(2);
+  } else {
+    float4 offr = one;  // rho offset: product of the later groups
+    for (int gg = g + 1; gg < 8; ++gg) offr = mul4(offr, gtot(gg));
+    const float4 off4 = (g & 1) ? one : gtot(g + 1);
+    float4 off5 = one;
+    for (int gg = g + 1; gg < 4; ++gg) off5 = mul4(off5, gtot(gg));
+    float4 ls = one, r2 = one;
+#pragma unroll
+    for (int u = 7; u >= 0; --u) {
+      const int p = 8 * g + u;
+      const float4 a = aa[u];
+      const float4 kf = ka[u];
+      sts_u2(sb + OFF_KH + sw128_elem(p, ig, 64), h4(mul4(kf, mul4(offr, ls))));
+      if (u < 4) {  // level 2: left half of the group
+        sts_u2(rop(2, 4 * g + u), h4(mul4(kf, r2)));
+        r2 = mul4(r2, a);
+      }
+      if (!(g & 1)) sts_u2(rop(3, 8 * (g >> 1) + u), h4(mul4(kf, ls)));
+      if (!(g & 2)) sts_u2(rop(4, 16 * (g >> 2) + 8 * (g & 1) + u), h4(mul4(kf, mul4(off4, ls))));
+      if (!(g & 4)) sts_u2(rop(5, 8 * g + u), h4(mul4(kf, mul4(off5, ls))));
+      ls = mul4(ls, a);
+    }
+    GP_MARK(3);
+    // direct pairs inside each aligned block of 4 (levels 0 and 1) and diag(A)
+    float acc[32];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const float4 k0 = ka[4 * m], k1 = ka[4 * m + 1], k2 = ka[4 * m + 2], k3 = ka[4 * m + 3];
+      const float4 a1 = aa[4 * m + 1], a2 = aa[4 * m + 2], a3 = aa[4 * m + 3];
+      const float4 q1 = qa[4 * m + 1], q2 = qa[4 * m + 2], q3 = qa[4 * m + 3];
+      const float4 e10 = mul4(a1, k0);
+      const float4 e20 = mul4(a2, e10);
+      const float4 e21 = mul4(a2, k1);
+      const float4 e30 = mul4(a3, e20);
+      const float4 e31 = mul4(a3, e21);
+      const float4 e32 = mul4(a3, k2);
+      float* o = acc + 12 * m;
+      o[0] = dot4(k1, e10);  o[1] = dot4(q1, e10);
+      o[2] = dot4(k2, e20);  o[3] = dot4(q2, e20);
+      o[4] = dot4(k2, e21);  o[5] = dot4(q2, e21);
+      o[6] = dot4(k3, e30);  o[7] = dot4(q3, e30);
+      o[8] = dot4(k3, e31);  o[9] = dot4(q3, e31);
+      o[10] = dot4(k3, e32); o[11] = dot4(q3, e32);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[24 + u] = dot4(qa[u], ka[u]);
+    // sum over the 16 threads (channels) of the group, then over the halves
+    const int lane = tid & 31;
+    reduce_scatter16(acc, lane);
+    reduce_scatter16(acc + 16, lane);
+    const uint32_t pr = sb + OFF_PR + 128 * g;
+    const uint32_t p0 = pr + 4 * (lane & 15), p1 = pr + 64 + 4 * (lane & 15);
+    if (hh == 0) {
+      sts_f(p0, acc[0]);
+      sts_f(p1, acc[16]);
+    } else {
+      sts_f(p0, lds_f(p0) + acc[0]);
+      sts_f(p1, lds_f(p1) + acc[16]);
+    }
+    GP_MARK(2);
+  }
+}
+
+// One step of the recursive-doubling inverse of the unit lower-triangular
+// (I + T): merge diagonal blocks of size M into blocks of size 2M,
+//   [[A, 0], [B, D]]^-1 = [[A^-1, 0], [-D^-1 B A^-1, D^-1]],  B = T block.
+// Inv holds the inverses of the M-blocks (zero above each block diagonal),
+// so the triangular limits of both products can be left to the zeros.
+template <int M>
+__device__ __forceinline__ void inv_merge(const float* Tf, float* Inv, float* Yf, int tid) {
+  constexpr int NMERGE = 64 / (2 * M);
+  if constexpr (M >= 4) {
+    constexpr int W4 = M / 4;                  // float4 groups per block row
+    constexpr int NOUT = NMERGE * M * W4;      // float4 outputs per phase
+    for (int e = tid; e < NOUT; e += NT) {
+      const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
+      const int r0 = 2 * M * qb;
+      const float* trow = Tf + (r0 + M + a) * 64 + r0;
+      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int t4 = 0; t4 < M / 4; ++t4) {
+        const float4 tv = *reinterpret_cast<const float4*>(trow + 4 * t4);
+        const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float4 iv =
+              *reinterpret_cast<const float4*>(Inv + (r0 + 4 * t4 + w) * 64 + r0 + 4 * c4);
+          y.x = fmaf(tt[w], iv.x, y.x); y.y = fmaf(tt[w], iv.y, y.y);
+          y.z = fmaf(tt[w], iv.z, y.z); y.w = fmaf(tt[w], iv.w, y.w);
+        }
+      }
+      *reinterpret_cast<float4*>(Yf + qb * M * M + a * M + 4 * c4) = y;
+    }
+    __syncthreads();
+    for (int e = tid; e < NOUT; e += NT) {
+      const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
+      const int r0 = 2 * M * qb;
+      const float* irow = Inv + (r0 + M + a) * 64 + r0 + M;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int t4 = 0; t4 < M / 4; ++t4) {
+        const float4 dv = *reinterpret_cast<const float4*>(irow + 4 * t4);
+        const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float4 yv =
+              *reinterpret_cast<const float4*>(Yf + qb * M * M + (4 * t4 + w) * M + 4 * c4);
+          x.x = fmaf(dd[w], yv.x, x.x); x.y = fmaf(dd[w], yv.y, x.y);
+          x.z = fmaf(dd[w], yv.z, x.z); x.w = fmaf(dd[w], yv.w, x.w);
+        }
+      }
+      *reinterpret_cast<float4*>(Inv + (r0 + M + a) * 64 + r0 + 4 * c4) =
+          make_float4(-x.x, -x.y, -x.z, -x.w);
+    }
+    __syncthreads();
+  } else {
+    constexpr int NOUT = NMERGE * M * M;
+    for (int e = tid; e < NOUT; e += NT) {
+      const int qb = e / (M * M), a = (e / M) % M, cc = e % M;
+      const int r0 = 2 * M * qb;
+      float y = 0.f;
+#pragma unroll
+      for (int t = 0; t < M; ++t)
+        y = fmaf(Tf[(r0 + M + a) * 64 + r0 + t], Inv[(r0 + t) * 64 + r0 + cc], y);
+      Yf[e] = y;
+    }
+    __syncthreads();
+    for (int e = tid; e < NOUT; e += NT) {
+      const int qb = e / (M * M), a = (e / M) % M, cc = e % M;
+      const int r0 = 2 * M * qb;
+      float x = 0.f;
+#pragma unroll
+      for (int t = 0; t < M; ++t)
+        x = fmaf(Inv[(r0 + M + a) * 64 + r0 + M + t], Yf[qb * M * M + t * M + cc], x);
+      Inv[(r0 + M + a) * 64 + r0 + cc] = -x;
+    }
+    __syncthreads();
+  }
+}
+
 template <typename Tout>
 __global__ void __launch_bounds__(NT, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -169,9 +484,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
               const float* __restrict__ beta, const float* S0, const int32_t* __restrict__ cu,
               Tout* __restrict__ out, float* S_final, int n_seqs, int T, int H, int DV,
               int* status) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                           ~static_cast<uintptr_t>(1023));
+  // Offsetting the __shared__ array itself (not a cast integer) keeps every
+  // access below in the shared state space.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -184,18 +500,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   if (!sr.ok) return;
 
   float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
-  float* gamma_s = reinterpret_cast<float*>(sm + OFF_GAMMA);
-  float* adiag_s = reinterpret_cast<float*>(sm + OFF_ADIAG);
-  const uint32_t bar_tma = sb + OFF_BAR;
-  const uint32_t bar_mma = sb + OFF_BAR + 8;
-  const uint32_t bar_lv0 = sb + OFF_BAR + 16;
-  const uint32_t bar_lv1 = sb + OFF_BAR + 24;
+  const float* gamma_s = reinterpret_cast<const float*>(sm + OFF_GAMMA);
+  const uint32_t bar_in0 = sb + OFF_BAR;
+  const uint32_t bar_in1 = sb + OFF_BAR + 8;
+  const uint32_t bar_v = sb + OFF_BAR + 16;
+  const uint32_t bar_mma = sb + OFF_BAR + 24;
+  const uint32_t bar_lv = sb + OFF_BAR + 32;
 
   if (tid == 0) {
-    mbar_init(bar_tma, 1);
+    mbar_init(bar_in0, 1);
+    mbar_init(bar_in1, 1);
+    mbar_init(bar_v, 1);
     mbar_init(bar_mma, 1);
-    mbar_init(bar_lv0, 1);
-    mbar_init(bar_lv1, 1);
+    mbar_init(bar_lv, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
@@ -210,6 +527,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF_TMEMPTR);
+#ifdef CKDA_TC_DEBUG
+  long long tmark[16] = {0};
+  long long tlast = clock64();
+#endif
 
   // State slice: row i = 32 * (warp % 4) + lane, columns [32 * (warp / 4), +32).
   const int q4 = warp & 3;
@@ -229,270 +550,216 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int64_t tok0 = sr.begin;
   const int64_t tok1 = sr.end;
   const int nchunks = (int)((tok1 - tok0 + C - 1) / C);
-  uint32_t ph_tma = 0, ph_mma = 0, ph_lv0 = 0, ph_lv1 = 0;
-  bool tma_pending = false;
+  uint32_t ph_in0 = 0, ph_in1 = 0, ph_v = 0, ph_mma = 0, ph_lv = 0;
+  int pend_in0 = 0, pend_in1 = 0, pend_v = 0;
   int ok = 1;
 
-  auto issue_tma = [&](int64_t t0) {
-    mbar_expect_tx(bar_tma, kTmaBytes);
-    tma_load_2d(sb + OFF_Q, &tm_q, h * DK, (int)t0, bar_tma);
-    tma_load_2d(sb + OFF_K, &tm_k, h * DK, (int)t0, bar_tma);
-    tma_load_2d(sb + OFF_A, &tm_a, h * DK, (int)t0, bar_tma);
-    tma_load_2d(sb + OFF_V, &tm_v, h * DV + j0, (int)t0, bar_tma);
+  auto issue_in = [&](int hh, int64_t t0) {
+    const uint32_t base = sb + (hh ? OFF_IN1 : OFF_IN0);
+    const uint32_t bar = hh ? bar_in1 : bar_in0;
+    mbar_expect_tx(bar, kInBytes);
+    tma_load_2d(base + IN_Q, &tm_q, h * DK + HC * hh, (int)t0, bar);
+    tma_load_2d(base + IN_K, &tm_k, h * DK + HC * hh, (int)t0, bar);
+    tma_load_2d(base + IN_A, &tm_a, h * DK + HC * hh, (int)t0, bar);
+  };
+  auto issue_v = [&](int64_t t0) {
+    mbar_expect_tx(bar_v, 8192);
+    tma_load_2d(sb + OFF_V, &tm_v, h * DV + j0, (int)t0, bar_v);
   };
   if (nchunks > 0) {
-    if (tid == 0) issue_tma(tok0);
-    tma_pending = true;
+    if (tid == 0) {
+      issue_in(0, tok0);
+      issue_in(1, tok0);
+      issue_v(tok0);
+    }
+    pend_in0 = pend_in1 = pend_v = 1;
   }
 
-  const int ich = tid & 127;
-  const bool upper = tid >= 128;
-  const __nv_bfloat16* Qs = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_Q);
-  const __nv_bfloat16* Ks = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_K);
-  const float* As = reinterpret_cast<const float*>(sm + OFF_A);
+  auto level_mmas = [&](int hh) {
+    constexpr uint32_t id = idesc_f16(64, 32, 0, 0);
+#pragma unroll
+    for (int lv = 2; lv < 6; ++lv) {
+      const uint32_t la = sb + OFF_LVX + (lv - 2) * kLvBytes;
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = smem_desc(la + kk * 32, 16, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(la + LV_ROP + kk * 32, 16, 1024, kSwizzle128);
+        mma_f16(tmem + TM_LV + 32 * (lv - 2), ad, bd, id, (hh > 0 || kk > 0) ? 1u : 0u);
+      }
+    }
+    mma_commit(bar_lv);
+  };
 
   for (int c = 0; c < nchunks; ++c) {
     const int64_t t0 = tok0 + (int64_t)c * C;
     const int Lc = (tok1 - t0 < (int64_t)C) ? (int)(tok1 - t0) : C;
+    const bool more = c + 1 < nchunks;
     if (tid < C) beta_s[tid] = (tid < Lc) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-    ok = mbar_wait_bounded(bar_tma, ph_tma, kWaitNs);
-    ph_tma ^= 1;
+    // ---- gate pass, half 0 ---------------------------------------------------
+    ok = mbar_wait_bounded(bar_in0, ph_in0, kWaitNs);
+    ph_in0 ^= 1;
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    tma_pending = false;
-
-    // ---- score blocks, one hierarchy level at a time ----------------------
-    for (int lv = 0; lv < 6; ++lv) {
-      const int b = 1 << lv;
-      const int buf = lv & 1;
-      if (lv >= 2) {
-        if (buf) {
-          ok = mbar_wait_bounded(bar_lv1, ph_lv1, kWaitNs);
-          ph_lv1 ^= 1;
-        } else {
-          ok = mbar_wait_bounded(bar_lv0, ph_lv0, kWaitNs);
-          ph_lv0 ^= 1;
-        }
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-      }
-      uint8_t* LOP = sm + (buf ? OFF_LOP1 : OFF_LOP0);
-      uint8_t* ROP = sm + (buf ? OFF_ROP1 : OFF_ROP0);
-      const int nseg = C / (2 * b);
-      if (upper) {
-        // right halves: L_r = alpha_m ... alpha_r; rows rho of [beta K L] and [Q L]
-        for (int j = 0; j < nseg; ++j) {
-          const int m = 2 * b * j + b;
-          float p = 1.f;
-          for (int u = 0; u < b; ++u) {
-            const int r = m + u;
-            const bool val = r < Lc;
-            p *= val ? As[r * DK + ich] : 1.f;
-            const float kv = val ? bf(Ks + r * DK + ich) : 0.f;
-            const float qv = val ? bf(Qs + r * DK + ich) : 0.f;
-            const int rho = j * b + u;
-            st_h(LOP, sw128_elem(rho, ich, 64), beta_s[r] * kv * p);
-            st_h(LOP, sw128_elem(32 + rho, ich, 64), qv * p);
-          }
-        }
-      } else {
-        // left halves: R_s = alpha_{s+1} ... alpha_{m-1}; rows sigma of [K R]
-        for (int j = 0; j < nseg; ++j) {
-          const int m = 2 * b * j + b;
-          float p = 1.f;
-          for (int u = b - 1; u >= 0; --u) {
-            const int s = m - b + u;
-            const bool val = s < Lc;
-            const float kv = val ? bf(Ks + s * DK + ich) : 0.f;
-            st_h(ROP, sw128_elem(j * b + u, ich, 32), kv * p);
-            p *= val ? As[s * DK + ich] : 1.f;
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t la = sb + (buf ? OFF_LOP1 : OFF_LOP0);
-        const uint32_t ra = sb + (buf ? OFF_ROP1 : OFF_ROP0);
-        constexpr uint32_t id = idesc_f16(64, 32, 0, 0);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = smem_desc(la + (kk >> 2) * (64 * 128) + (kk & 3) * 32, 16, 1024, kSwizzle128);
-          const uint64_t bd = smem_desc(ra + (kk >> 2) * (32 * 128) + (kk & 3) * 32, 16, 1024, kSwizzle128);
-          mma_f16(tmem + TM_SCORE + 32 * lv, ad, bd, id, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(buf ? bar_lv1 : bar_lv0);
-      }
-    }
-    if (!ok) break;
-    ok = mbar_wait_bounded(bar_lv0, ph_lv0, kWaitNs);
-    ph_lv0 ^= 1;
-    ok = mbar_wait_bounded(bar_lv1, ph_lv1, kWaitNs) && ok;
-    ph_lv1 ^= 1;
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-
-    // ---- Gamma (prefix), rho (suffix), gamma, diag(A), identity padding ----
-    {
-      uint8_t* KG = sm + OFF_KG;
-      __half* QG = reinterpret_cast<__half*>(sm + OFF_QG);
-      uint8_t* KH = sm + OFF_KH;
-      if (!upper) {
-        float g = 1.f;
-        for (int r = 0; r < C; ++r) {
-          const bool val = r < Lc;
-          g *= val ? As[r * DK + ich] : 1.f;
-          const float kv = val ? bf(Ks + r * DK + ich) : 0.f;
-          const float qv = val ? bf(Qs + r * DK + ich) : 0.f;
-          st_h(KG, sw128_elem(r, ich, 64), kv * g);
-          QG[r * QG_STRIDE + ich] = __float2half_rn(qv * g);
-        }
-        gamma_s[ich] = g;
-      } else {
-        float p = 1.f;
-        for (int s = C - 1; s >= 0; --s) {
-          const bool val = s < Lc;
-          const float kv = val ? bf(Ks + s * DK + ich) : 0.f;
-          st_h(KH, sw128_elem(s, ich, 64), kv * p);
-          p *= val ? As[s * DK + ich] : 1.f;
-        }
-      }
-      for (int rr = 0; rr < 8; ++rr) {
-        const int r = 8 * warp + rr;
-        float acc = 0.f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc = fmaf(bf(Qs + r * DK + 4 * lane + e), bf(Ks + r * DK + 4 * lane + e), acc);
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) adiag_s[r] = (r < Lc) ? acc : 0.f;
-      }
-      // v tile: bf16 (as loaded) -> fp16 in place; rows past the end -> 0.
-      // Each 16-byte chunk stays within its 128-byte row under the swizzle.
-      {
-        uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V);
-        for (int e = tid; e < C * 8; e += NT) {
-          uint4 raw = vt[e];
-          if ((e >> 3) < Lc) {
-            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-            float f[8];
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-              const float2 x2 = __bfloat1622float2(p2[t]);
-              f[2 * t] = x2.x;
-              f[2 * t + 1] = x2.y;
-            }
-            raw.x = pack_f16x2(f[0], f[1]);
-            raw.y = pack_f16x2(f[2], f[3]);
-            raw.z = pack_f16x2(f[4], f[5]);
-            raw.w = pack_f16x2(f[6], f[7]);
-          } else {
-            raw = make_uint4(0u, 0u, 0u, 0u);
-          }
-          vt[e] = raw;
-        }
-      }
-    }
+    pend_in0 = 0;
+    TC_MARK(0);
+    gate_pass(sb, sb + OFF_IN0, 0, Lc, tid);
+    fence_proxy_async_smem();
     __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      level_mmas(0);
+      if (more) issue_in(0, t0 + C);
+    }
+    if (more) pend_in0 = 1;
+    TC_MARK(1);
 
-    // ---- gather T (fp32) and A (fp16) from the level accumulators ---------
+    // ---- gate pass, half 1 (after the half-0 level GEMMs release the operands)
+    ok = mbar_wait_bounded(bar_in1, ph_in1, kWaitNs);
+    ph_in1 ^= 1;
+    ok = mbar_wait_bounded(bar_lv, ph_lv, kWaitNs) && ok;
+    ph_lv ^= 1;
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    pend_in1 = 0;
+    gate_pass(sb, sb + OFF_IN1, 1, Lc, tid);
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      level_mmas(1);
+      if (more) issue_in(1, t0 + C);
+    }
+    if (more) pend_in1 = 1;
+    TC_MARK(2);
+    ok = mbar_wait_bounded(bar_lv, ph_lv, kWaitNs);
+    ph_lv ^= 1;
+    ok = mbar_wait_bounded(bar_v, ph_v, kWaitNs) && ok;
+    ph_v ^= 1;
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    pend_v = 0;
+    tc_fence_after();
+    TC_MARK(3);
+
+    // ---- T and A (fp32) from levels 2..5, the direct pairs and diag(A) -------
     {
       uint4* z = reinterpret_cast<uint4*>(sm + OFF_TF);
-      for (int e = tid; e < (int)(40960 / 16); e += NT) z[e] = make_uint4(0u, 0u, 0u, 0u);
+      for (int e = tid; e < 2048; e += NT) z[e] = make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
-    tc_fence_after();
     {
       float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
-      uint8_t* AQ = sm + OFF_AQ;
+      float* Af = reinterpret_cast<float*>(sm + OFF_AF);
       if (warp < 4) {
         const int rho = 16 * warp + lane;
         const int rr = rho & 31;
-        for (int lv = 0; lv < 6; ++lv) {
+        float* dst = (rho < 32) ? Tf : Af;
+#pragma unroll
+        for (int lv = 2; lv < 6; ++lv) {
           float v[32];
-          tmem_ld32(taddr(tmem, 32 * warp, TM_SCORE + 32 * lv), v);
+          tmem_ld32(taddr(tmem, 32 * warp, TM_LV + 32 * (lv - 2)), v);
           tmem_ld_wait();
           if (lane < 16) {
             const int b = 1 << lv;
             const int j = rr >> lv;
             const int r = 2 * b * j + b + (rr & (b - 1));
+            float* row = dst + r * 64 + b * j;
 #pragma unroll
-            for (int sg = 0; sg < 32; ++sg) {
-              if ((sg >> lv) == j) {
-                const int s = 2 * b * j + (sg & (b - 1));
-                if (rho < 32)
-                  Tf[r * 64 + s] = v[sg];
-                else
-                  st_h(AQ, sw128_elem(r, s, 64), v[sg]);
-              }
+            for (int m4 = 0; m4 < 8; ++m4) {
+              if (((4 * m4) >> lv) == j)
+                *reinterpret_cast<float4*>(row + 4 * m4) =
+                    make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
             }
           }
         }
+      } else {
+        // direct pairs (r, s) inside aligned blocks of 4, and the diagonal of A
+        const float* pr = reinterpret_cast<const float*>(sm + OFF_PR);
+        for (int e = tid - 128; e < 8 * 32; e += 128) {
+          const int g = e >> 5, w = e & 31;
+          const float val = pr[e];
+          if (w < 24) {
+            const int m = w / 12, jj = (w % 12) >> 1;
+            // pair order inside the block: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+            const int rl = (jj == 0) ? 1 : (jj < 3 ? 2 : 3);
+            const int sl = (jj == 0 || jj == 1 || jj == 3) ? 0 : (jj == 2 || jj == 4 ? 1 : 2);
+            const int r = 8 * g + 4 * m + rl, s = 8 * g + 4 * m + sl;
+            if (w & 1)
+              Af[r * 64 + s] = val;
+            else
+              Tf[r * 64 + s] = beta_s[r] * val;
+          } else {
+            const int r = 8 * g + (w - 24);
+            Af[r * 64 + r] = val;
+          }
+        }
       }
-      if (tid < C) st_h(AQ, sw128_elem(tid, tid, 64), adiag_s[tid]);
+      // v tile: bf16 (as loaded) -> fp16 in place; rows past the end -> 0.
+      // Each 16-byte chunk stays within its 128-byte row under the swizzle.
+      uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V);
+      for (int e = tid; e < C * 8; e += NT) {
+        uint4 raw = vt[e];
+        if ((e >> 3) < Lc) {
+          float f[8];
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 x2 = __bfloat1622float2(p2[t]);
+            f[2 * t] = x2.x;
+            f[2 * t + 1] = x2.y;
+          }
+          raw.x = pack_f16x2(f[0], f[1]);
+          raw.y = pack_f16x2(f[2], f[3]);
+          raw.z = pack_f16x2(f[4], f[5]);
+          raw.w = pack_f16x2(f[6], f[7]);
+        } else {
+          raw = make_uint4(0u, 0u, 0u, 0u);
+        }
+        vt[e] = raw;
+      }
     }
     tc_fence_before();
     __syncthreads();
     TC_DBG(for (int e = tid; e < 4096; e += NT) {
       g_tc_dbg[e] = reinterpret_cast<const float*>(sm + OFF_TF)[e];
-      g_tc_dbg[4096 + e] = __half2float(*reinterpret_cast<const __half*>(sm + OFF_AQ + sw128_elem(e >> 6, e & 63, 64)));
+      g_tc_dbg[4096 + e] = reinterpret_cast<const float*>(sm + OFF_AF)[e];
     });
+    TC_MARK(4);
 
-    // ---- (I + T)^-1 in fp32, 16 x 16 blocks ---------------------------------
+    // ---- A -> fp16 operand; (I + T)^-1 by recursive doubling ------------------
+    {
+      const float* Af = reinterpret_cast<const float*>(sm + OFF_AF);
+      for (int e = tid; e < 64 * 8; e += NT) {
+        const int r = e >> 3, cg = e & 7;
+        st_chunk8(sm + OFF_AQ, sw128_chunk(r, 8 * cg, 64), Af + r * 64 + 8 * cg);
+      }
+    }
+    __syncthreads();
     {
       const float* Tf = reinterpret_cast<const float*>(sm + OFF_TF);
-      float* Inv = reinterpret_cast<float*>(sm + OFF_INV);
+      float* Inv = reinterpret_cast<float*>(sm + OFF_AF);
       float* Yf = reinterpret_cast<float*>(sm + OFF_YF);
-      if (tid < 64) {
-        const int base = 16 * (tid >> 4);
-        const int cc = tid & 15;
-        float x[16];
-#pragma unroll
-        for (int r2 = 0; r2 < 16; ++r2) {
-          float acc = (r2 == cc) ? 1.f : 0.f;
-#pragma unroll
-          for (int s2 = 0; s2 < r2; ++s2) acc = fmaf(-Tf[(base + r2) * 64 + base + s2], x[s2], acc);
-          x[r2] = (r2 < cc) ? 0.f : acc;
-        }
-#pragma unroll
-        for (int r2 = 0; r2 < 16; ++r2) Inv[(base + r2) * 64 + base + cc] = x[r2];
-      }
+      for (int e = tid; e < 4096; e += NT) Inv[e] = ((e >> 6) == (e & 63)) ? 1.f : 0.f;
       __syncthreads();
-      for (int I = 1; I < 4; ++I) {
-        for (int e = tid; e < 256 * I; e += NT) {
-          const int J = e >> 8, r2 = (e >> 4) & 15, cc = e & 15;
-          float acc = 0.f;
-          for (int K = J; K < I; ++K) {
-#pragma unroll
-            for (int kk = 0; kk < 16; ++kk)
-              acc = fmaf(Tf[(16 * I + r2) * 64 + 16 * K + kk], Inv[(16 * K + kk) * 64 + 16 * J + cc], acc);
-          }
-          Yf[r2 * 48 + 16 * J + cc] = acc;
-        }
-        __syncthreads();
-        for (int e = tid; e < 256 * I; e += NT) {
-          const int J = e >> 8, r2 = (e >> 4) & 15, cc = e & 15;
-          float acc = 0.f;
-#pragma unroll
-          for (int kk = 0; kk < 16; ++kk)
-            acc = fmaf(Inv[(16 * I + r2) * 64 + 16 * I + kk], Yf[kk * 48 + 16 * J + cc], acc);
-          Inv[(16 * I + r2) * 64 + 16 * J + cc] = -acc;
-        }
-        __syncthreads();
-      }
+      inv_merge<1>(Tf, Inv, Yf, tid);
+      inv_merge<2>(Tf, Inv, Yf, tid);
+      inv_merge<4>(Tf, Inv, Yf, tid);
+      inv_merge<8>(Tf, Inv, Yf, tid);
+      inv_merge<16>(Tf, Inv, Yf, tid);
+      inv_merge<32>(Tf, Inv, Yf, tid);
       TC_DBG(for (int e = tid; e < 4096; e += NT) g_tc_dbg[8192 + e] = Inv[e]);
       // Inv diag(beta) -> rows 0..63 of the stacked operand
-      uint8_t* IP = sm + OFF_IP;
       for (int e = tid; e < 64 * 8; e += NT) {
         const int r = e >> 3, cg = e & 7;
         float v[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) v[t] = Inv[r * 64 + 8 * cg + t] * beta_s[8 * cg + t];
-        st_chunk8(IP, sw128_chunk(r, 8 * cg, 128), v);
+        st_chunk8(sm + OFF_IP, sw128_chunk(r, 8 * cg, 128), v);
       }
     }
     fence_proxy_async_smem();
     __syncthreads();
+    TC_MARK(5);
 
     // ---- P = A Inv diag(beta) ---------------------------------------------------
     if (tid == 0) {
@@ -526,6 +793,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    TC_MARK(6);
 
     // ---- [W, U~; A W, A U~] = [Inv diag(beta); P] [K Gamma, V] ----------------
     if (tid == 0) {
@@ -548,9 +816,16 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
     ph_mma ^= 1;
+    fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
+    // the v tile is free: fetch the next chunk's
+    if (more) {
+      if (tid == 0) issue_v(t0 + C);
+      pend_v = 1;
+    }
+    TC_MARK(7);
 
     // ---- [W; Q' = Q Gamma - A W] -> carry operand -------------------------------
     {
@@ -561,16 +836,17 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_ld_wait();
       TC_DBG(for (int e = 0; e < 64; ++e) g_tc_dbg[16384 + L * 128 + 64 * half + e] = v[e]);
       if (L >= 64) {
-        const __half* qg = reinterpret_cast<const __half*>(sm + OFF_QG) + (L - 64) * QG_STRIDE + 64 * half;
+        // Q * Gamma sits in this row of the tile already (written by the gate pass)
 #pragma unroll
-        for (int e = 0; e < 64; e += 8) {
-          uint4 raw = *reinterpret_cast<const uint4*>(qg + e);
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 raw =
+              *reinterpret_cast<const uint4*>(sm + OFF_WQ + sw128_chunk(L, 64 * half + 8 * c8, 128));
           const __half2* p2 = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const float2 f = __half22float2(p2[t]);
-            v[e + 2 * t] = f.x - v[e + 2 * t];
-            v[e + 2 * t + 1] = f.y - v[e + 2 * t + 1];
+            v[8 * c8 + 2 * t] = f.x - v[8 * c8 + 2 * t];
+            v[8 * c8 + 2 * t + 1] = f.y - v[8 * c8 + 2 * t + 1];
           }
         }
       }
@@ -581,6 +857,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    TC_MARK(8);
 
     // ---- carry 1: X = [W; Q'] S ---------------------------------------------------
     if (tid == 0) {
@@ -597,15 +874,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
     ph_mma ^= 1;
-    fence_proxy_async_smem();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    // the input tiles are free: fetch the next chunk under the rest of the carry
-    if (c + 1 < nchunks) {
-      if (tid == 0) issue_tma(t0 + C);
-      tma_pending = true;
-    }
+    TC_MARK(9);
 
     // ---- U = U~ - X_top -> operand;  O = A U~ + X_bottom -> out ------------------
     {
@@ -633,6 +905,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    TC_MARK(10);
 
     // ---- carry 2: D = (K rho)^T U;  S <- Diag(gamma) S + D ----------------------
     if (tid == 0) {
@@ -655,9 +928,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       float d[32];
       tmem_ld32(taddr(tmem, 32 * q4, TM_D + 32 * half), d);
       tmem_ld_wait();
-      const float g = gamma_s[srow];
+      const float gm = gamma_s[srow];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) S[e] = fmaf(g, S[e], d[e]);
+      for (int e = 0; e < 32; ++e) S[e] = fmaf(gm, S[e], d[e]);
       TC_DBG(for (int e = 0; e < 32; ++e) {
         g_tc_dbg[49152 + srow * 64 + 32 * half + e] = d[e];
         g_tc_dbg[57344 + srow * 64 + 32 * half + e] = S[e];
@@ -669,7 +942,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    TC_MARK(11);
   }
+#ifdef CKDA_TC_DEBUG
+  if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    for (int k = 0; k < 16; ++k) g_tc_time[k] = tmark[k];
+#endif
 
   if (ok) {
     if (S_final != nullptr) {
@@ -681,7 +959,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) {
       set_status(status, CKDA_ERR_DEVICE_TIMEOUT);
       // wait (bounded) for copies and tensor-core work this CTA still has in flight
-      if (tma_pending) mbar_wait_bounded(bar_tma, ph_tma, kWaitNs);
+      if (pend_in0) mbar_wait_bounded(bar_in0, ph_in0, kWaitNs);
+      if (pend_in1) mbar_wait_bounded(bar_in1, ph_in1, kWaitNs);
+      if (pend_v) mbar_wait_bounded(bar_v, ph_v, kWaitNs);
       mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
     }
   }
@@ -729,13 +1009,13 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* a
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
   CUtensorMap mq, mk, mv, ma;
   const bool ok = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows,
-                           DK, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                           HC, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows,
-                           DK, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
+                           HC, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
                   make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows,
                            BV, C, CU_TENSOR_MAP_SWIZZLE_128B) &&
                   make_map(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)H * DK,
-                           rows, DK, C, CU_TENSOR_MAP_SWIZZLE_NONE);
+                           rows, HC, C, CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
   auto kern = fwd_tc_kernel<Tout>;
   static bool attr_set = false;
@@ -753,16 +1033,20 @@ cudaError_t launch_t(const void* q, const void* k, const void* v, const float* a
 
 }  // namespace tc
 
-// Shapes covered by the tensor-core kernel; everything else returns
+// Shapes covered by the tensor-core kernel (`rows` = packed or B*T tokens).
+bool fwd_tc_supported(int dtype, int dk, int dv, int C, uint64_t rows) {
+  return dtype == CKDA_BF16 && dk == tc::DK && (dv == 64 || dv == 128) && C == tc::C &&
+         rows > 0 && rows <= 0x7fffffffull;
+}
+
+// Everything the tensor-core kernel does not cover returns
 // cudaErrorNotSupported so the caller can use the CUDA-core kernel.
 cudaError_t launch_fwd_tc(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k,
                           const void* v, const float* alpha, const float* beta, const float* S0,
                           const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
                           int C, int* status, cudaStream_t stream) {
-  if (dtype != CKDA_BF16 || dk != tc::DK || (dv != 64 && dv != 128) || C != tc::C)
-    return cudaErrorNotSupported;
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
-  if (rows == 0 || rows > 0x7fffffffull) return cudaErrorNotSupported;
+  if (!fwd_tc_supported(dtype, dk, dv, C, rows)) return cudaErrorNotSupported;
   if (out_dtype == CKDA_BF16)
     return tc::launch_t<__nv_bfloat16>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H,
                                        dv, status, stream);

@@ -128,6 +128,18 @@ CKDA_API int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void*
                               int out_dtype, void* stream);
 
 /*
+ * ckda_fwd_chunked_path -- which kernel ckda_fwd_chunked runs for these
+ * parameters, without launching anything: 1 = the tcgen05 tensor-core
+ * kernel (bf16 inputs, d_k = 128, d_v in {64, 128}, chunk 64; fp16 operands
+ * with fp32 accumulation), 0 = the fp32 CUDA-core kernel, or the negative
+ * status an actual call with these sizes would return.  `varlen` is nonzero
+ * for a packed batch (cu_seqlens given); B and T have the same meaning as in
+ * ckda_fwd_chunked.  Pure host function: needs no GPU.
+ */
+CKDA_API int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
+                                   int out_dtype, int varlen);
+
+/*
  * ckda_decode_step -- one recurrent token for B independent sequences,
  * in place on the state ("Complex KDA ...", section "Yazilim Gelistirme
  * Acisindan Pratik Cikarimlar": O(1) inference state).

@@ -131,3 +131,17 @@ def test_decode_argument_errors(lib):
 
 def test_zero_sequences_is_a_no_op(lib):
     assert fwd(lib, B=0) == 0
+
+
+def test_path_query_needs_no_gpu(lib):
+    F32, BF16 = 0, 1
+    assert lib.ckda_fwd_chunked_path(4, 4096, 16, 128, 128, 64, BF16, F32, 0) == 1
+    assert lib.ckda_fwd_chunked_path(1, 65536, 32, 128, 128, 0, BF16, BF16, 0) == 1
+    assert lib.ckda_fwd_chunked_path(64, 135000, 16, 128, 128, 64, BF16, F32, 1) == 1
+    assert lib.ckda_fwd_chunked_path(4, 4096, 16, 128, 64, 64, BF16, F32, 0) == 1
+    assert lib.ckda_fwd_chunked_path(4, 4096, 16, 128, 128, 64, F32, F32, 0) == 0   # fp32 inputs
+    assert lib.ckda_fwd_chunked_path(4, 4096, 16, 128, 128, 32, BF16, F32, 0) == 0  # chunk 32
+    assert lib.ckda_fwd_chunked_path(4, 4096, 16, 64, 64, 64, BF16, F32, 0) == 0    # d_k 64
+    assert lib.ckda_fwd_chunked_path(4, 0, 16, 128, 128, 64, BF16, F32, 0) == 0     # no tokens
+    assert lib.ckda_fwd_chunked_path(4, 4096, 16, 128, 128, 48, BF16, F32, 0) == -2
+    assert lib.ckda_fwd_chunked_path(4, 4096, 0, 128, 128, 64, BF16, F32, 0) == -1

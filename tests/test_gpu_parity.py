@@ -55,6 +55,13 @@ def test_kda_prefill_small_ragged(ck, fp32core):
     _check_fixed(ck, case, TOL_BF16, fp32core=fp32core)
 
 
+def test_prefill_workloads_run_on_tensor_cores(ck):
+    assert ck.fwd_path(4, 4096, 16, 128, 128, 64, torch.bfloat16, torch.float32) == "tcgen05"
+    assert ck.fwd_path(1, 65536, 32, 128, 128, 64, torch.bfloat16, torch.float32) == "tcgen05"
+    assert ck.fwd_path(64, 135000, 16, 128, 128, 64, torch.float32, torch.float32,
+                       varlen=True) == "fp32core"
+
+
 def test_kda_prefill_full_size_sampled(ck):
     case = inputs.kda_prefill(seed=0, device=DEV)  # B=4, H=16, T=4096, d=128
     _check_fixed(ck, case, TOL_BF16, b_idx=[0, 3], h_idx=[0, 5, 15])
