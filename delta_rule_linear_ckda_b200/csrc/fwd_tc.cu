@@ -739,11 +739,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const float* Tf = reinterpret_cast<const float*>(sm + OFF_TF);
       float* Inv = reinterpret_cast<float*>(sm + OFF_AF);
       float* Yf = reinterpret_cast<float*>(sm + OFF_YF);
-      for (int e = tid; e < 4096; e += NT) Inv[e] = ((e >> 6) == (e & 63)) ? 1.f : 0.f;
+      {
+        uint4* z = reinterpret_cast<uint4*>(Inv);
+        for (int e = tid; e < 1024; e += NT) z[e] = make_uint4(0u, 0u, 0u, 0u);
+      }
       __syncthreads();
-      inv_merge<1>(Tf, Inv, Yf, tid);
-      inv_merge<2>(Tf, Inv, Yf, tid);
-      inv_merge<4>(Tf, Inv, Yf, tid);
+      // 8 x 8 diagonal blocks by forward substitution, one column per thread
+      if (tid < 64) {
+        const int base = 8 * (tid >> 3), cc = tid & 7;
+        float x[8];
+#pragma unroll
+        for (int r2 = 0; r2 < 8; ++r2) {
+          float acc = (r2 == cc) ? 1.f : 0.f;
+#pragma unroll
+          for (int s2 = 0; s2 < r2; ++s2) acc = fmaf(-Tf[(base + r2) * 64 + base + s2], x[s2], acc);
+          x[r2] = (r2 < cc) ? 0.f : acc;
+          Inv[(base + r2) * 64 + base + cc] = x[r2];
+        }
+      }
+      __syncthreads();
       inv_merge<8>(Tf, Inv, Yf, tid);
       inv_merge<16>(Tf, Inv, Yf, tid);
       inv_merge<32>(Tf, Inv, Yf, tid);
