@@ -78,6 +78,29 @@ def _dist():
     return ws, rank, local
 
 
+def rank_seeds(rank: int):
+    """Seeds of the two rotating input sets of a rank: every replica draws its
+    own batch (weak scaling, no shared data)."""
+    return [1000 * rank + i for i in range(2)]
+
+
+def max_over_ranks(x: float, ws: int, device="cpu") -> float:
+    """Max of a per-rank time over all ranks (the job is as slow as its slowest rank)."""
+    if ws == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, ws: int, seconds_per_step: float) -> float:
+    """Units all ranks processed per second, timed by the slowest rank."""
+    return ws * units_per_rank / seconds_per_step
+
+
 def _emit(obj, args, rank):
     if rank != 0:
         return
@@ -193,8 +216,10 @@ def run_reference(args, ws, rank):
 
     threads = oracle.default_threads()
     dt1, _, _ = _time_oracle(1, 1)
-    # each step: a bounded sample sized to ~1 s of oracle work on all threads
-    n_units = int(max(1, min(B * H, 1.0 * threads / max(dt1, 1e-6))))
+    # each step: a bounded sample of whole (b, h) units, sized so that the
+    # whole run stays near 100 s of oracle time (at most 1 s per step)
+    step_s = min(1.0, 100.0 / max(1, args.steps + args.warmup))
+    n_units = int(max(1, min(B * H, step_s * threads / max(dt1, 1e-6))))
     for _ in range(args.warmup):
         _time_oracle(n_units, threads)
     total_dt, total_th = 0.0, 0
@@ -261,16 +286,12 @@ def run_ours(args, ws, rank, local):
         if ws > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if ws == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x: float) -> float:
+        return max_over_ranks(x, ws, dev)
 
     # two input sets (each ~0.4 GB > 126 MB L2), rotated so no step finds its
     # inputs in L2
-    sets = [inputs.kda_prefill(seed=1000 * rank + i, device=dev) for i in range(2)]
+    sets = [inputs.kda_prefill(seed=sd, device=dev) for sd in rank_seeds(rank)]
     out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -306,12 +327,12 @@ def run_ours(args, ws, rank, local):
     barrier()
     wall = time.perf_counter() - wall0
     clocks = sampler.stop() if sampler else None
-    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    elapsed_ms = max_ranks(ev0.elapsed_time(ev1))
     kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(K))
-    kern_ms = max_over_ranks(kern_ms)
+    kern_ms = max_ranks(kern_ms)
     ms_per_step = elapsed_ms / K
     tokens = B * T
-    value = ws * tokens / (ms_per_step / 1e3)
+    value = whole_job_rate(tokens, ws, ms_per_step / 1e3)
 
     token_heads = B * T * H
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + B * H * D * D * 4
@@ -325,13 +346,13 @@ def run_ours(args, ws, rank, local):
     # ---- end to end: host (pinned) buffers through the public API --------
     e2e = None
     if args.e2e_steps > 0:
-        e2e = _run_e2e(args, ck, torch, sets[0], out, S_final, stream, barrier, max_over_ranks,
+        e2e = _run_e2e(args, ck, torch, sets[0], out, S_final, stream, barrier, max_ranks,
                        ws, tokens, dev)
 
     # ---- decode step (B=256, H=32, d=128, bf16), 1024 steps --------------
     decode = None
     if not args.no_decode:
-        decode = _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ranks,
+        decode = _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
                              ws, hbm_peak)
     path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
     _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
@@ -342,7 +363,7 @@ def run_ours(args, ws, rank, local):
         dist.destroy_process_group()
 
 
-def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_over_ranks, ws, tokens, dev):
+def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, tokens, dev):
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     host = {n: getattr(c, n).cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
@@ -372,13 +393,13 @@ def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_over_ranks, 
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1)) / E
+    e2e_ms = max_ranks(ev0.elapsed_time(ev1)) / E
     e2e_value = ws * tokens / (e2e_ms / 1e3)
     return {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
-def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ranks, ws, hbm_peak):
+def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak):
     steps = max(1, args.decode_steps)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
@@ -395,7 +416,7 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_over_ra
     ev1.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    dec_ms = max_over_ranks(ev0.elapsed_time(ev1)) / steps
+    dec_ms = max_ranks(ev0.elapsed_time(ev1)) / steps
     dbytes = DEC_B * DEC_H * DEC_BYTES_PER_HEAD_STEP
     dgbs = dbytes / (dec_ms / 1e3) / 1e9
     decode = {"workload": f"decode B={DEC_B} H={DEC_H} d={D} bf16 q/k/v, fp32 out, "

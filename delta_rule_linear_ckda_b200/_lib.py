@@ -34,6 +34,7 @@ SIGNATURES = {
     "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_device_status": (_i, [_vp]),
+    "ckda_selftest_bounded_wait": (_i, [_i, _vp]),
     "ckda_version": (_i, []),
 }
 

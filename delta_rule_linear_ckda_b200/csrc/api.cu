@@ -23,6 +23,8 @@ cudaError_t launch_fwd_tc(int dtype, int out_dtype, int dk, int dv, const void* 
                           const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
                           int C, int* status, cudaStream_t stream);
 bool fwd_tc_supported(int dtype, int dk, int dv, int C, uint64_t rows);
+cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
+                                      cudaStream_t stream);
 }  // namespace ckda
 
 // First device-side error since the last ckda_device_status() call.
@@ -161,6 +163,15 @@ int ckda_decode_step(const void* q, const void* k, const void* v, const float* a
   if (out == S_inout || out == q || out == k || out == v) return CKDA_ERR_INVALID_ARG;
   cudaError_t e = ckda::launch_decode(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S_inout, out, B * H,
                                       static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+int ckda_selftest_bounded_wait(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 10000000) return CKDA_ERR_INVALID_ARG;
+  int* status = status_ptr();
+  if (status == nullptr) return CKDA_ERR_CUDA;
+  cudaError_t e = ckda::launch_bounded_wait_probe(
+      status, 1000ull * (unsigned long long)limit_us, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 

@@ -164,6 +164,17 @@ CKDA_API const char* ckda_status_string(int status);
  */
 CKDA_API int ckda_device_status(void* stream);
 
+/*
+ * ckda_selftest_bounded_wait -- exercise the device-side time-out path.
+ * Launches one thread that waits, with the bounded wait every tensor-core
+ * kernel uses, on an mbarrier nothing completes; after about `limit_us`
+ * microseconds (1 .. 10,000,000) the wait gives up and records
+ * CKDA_ERR_DEVICE_TIMEOUT in the status word, which ckda_device_status()
+ * then returns.  Faults nothing and leaves the context usable.  Returns
+ * CKDA_OK once launched, CKDA_ERR_INVALID_ARG for a limit out of range.
+ */
+CKDA_API int ckda_selftest_bounded_wait(int limit_us, void* stream);
+
 /* Library ABI version (major * 100 + minor). */
 CKDA_API int ckda_version(void);
 

@@ -145,3 +145,8 @@ def test_path_query_needs_no_gpu(lib):
     assert lib.ckda_fwd_chunked_path(4, 0, 16, 128, 128, 64, BF16, F32, 0) == 0     # no tokens
     assert lib.ckda_fwd_chunked_path(4, 4096, 16, 128, 128, 48, BF16, F32, 0) == -2
     assert lib.ckda_fwd_chunked_path(4, 4096, 0, 128, 128, 64, BF16, F32, 0) == -1
+
+
+def test_selftest_rejects_bad_limits(lib):
+    assert lib.ckda_selftest_bounded_wait(0, None) == -1
+    assert lib.ckda_selftest_bounded_wait(20000000, None) == -1
