@@ -71,8 +71,11 @@ constexpr uint32_t OFF_V = 65536;  // v slice (TMA, 128B swizzle), bf16 -> fp16 
 // Work region: level operands while the gate pass runs; then the fp32
 // inverse workspace and the A / [Inv; P] operands; then the U operand.
 constexpr uint32_t OFF_LVX = 73728;
-constexpr uint32_t kLvBytes = 12288;          // per level: LOP 8 KB + ROP 4 KB
-constexpr uint32_t LV_ROP = 8192;
+// Levels are paired (2, 3) and (4, 5): one M=128 x N=64 GEMM per pair, of
+// which the two diagonal 64 x 32 blocks are used.  Per pair: the left
+// operand [levels a; b] (128 rows) and the right operand (64 rows).
+constexpr uint32_t kPairBytes = 24576;
+constexpr uint32_t PAIR_ROP = 16384;
 constexpr uint32_t OFF_TF = OFF_LVX;          // T, fp32 [64][64]
 constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A staging then (I + T)^-1, fp32 [64][64]
 constexpr uint32_t OFF_AQ = OFF_LVX + 32768;  // A, fp16 K-major [64 r][64 s]
@@ -93,7 +96,7 @@ constexpr uint32_t kSmemUsed = 225104;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 
 // ---- tensor memory columns ------------------------------------------------
-constexpr uint32_t TM_LV = 0;    // levels 2..5, 32 columns each (M = 64 layout)
+constexpr uint32_t TM_LV = 0;    // level pairs, 64 columns each (M = 128)
 constexpr uint32_t TM_P = 128;   // P (M = 64 layout)
 constexpr uint32_t TM_W = 192;   // [W; A W]       (M = 128, 128 columns)
 constexpr uint32_t TM_U = 320;   // [U~; A U~]     (M = 128, 64 columns)
@@ -287,10 +290,11 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
   auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * HC * 4); };
   const uint32_t LV = sb + OFF_LVX;
   auto lop = [&](int lv, int row) -> uint32_t {
-    return LV + (lv - 2) * kLvBytes + sw128_elem(row, cl, 64);
+    return LV + ((lv - 2) >> 1) * kPairBytes + sw128_elem(64 * ((lv - 2) & 1) + row, cl, 128);
   };
   auto rop = [&](int lv, int row) -> uint32_t {
-    return LV + (lv - 2) * kLvBytes + LV_ROP + sw128_elem(row, cl, 32);
+    return LV + ((lv - 2) >> 1) * kPairBytes + PAIR_ROP +
+           sw128_elem(32 * ((lv - 2) & 1) + row, cl, 64);
   };
 
   if (role == 0) {
@@ -576,15 +580,15 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   }
 
   auto level_mmas = [&](int hh) {
-    constexpr uint32_t id = idesc_f16(64, 32, 0, 0);
+    constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
 #pragma unroll
-    for (int lv = 2; lv < 6; ++lv) {
-      const uint32_t la = sb + OFF_LVX + (lv - 2) * kLvBytes;
+    for (int pr = 0; pr < 2; ++pr) {
+      const uint32_t la = sb + OFF_LVX + pr * kPairBytes;
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = smem_desc(la + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(la + LV_ROP + kk * 32, 16, 1024, kSwizzle128);
-        mma_f16(tmem + TM_LV + 32 * (lv - 2), ad, bd, id, (hh > 0 || kk > 0) ? 1u : 0u);
+        const uint64_t bd = smem_desc(la + PAIR_ROP + kk * 32, 16, 1024, kSwizzle128);
+        mma_f16(tmem + TM_LV + 64 * pr, ad, bd, id, (hh > 0 || kk > 0) ? 1u : 0u);
       }
     }
     mma_commit(bar_lv);
@@ -642,34 +646,31 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     TC_MARK(3);
 
     // ---- T and A (fp32) from levels 2..5, the direct pairs and diag(A) -------
-    {
-      uint4* z = reinterpret_cast<uint4*>(sm + OFF_TF);
-      for (int e = tid; e < 2048; e += NT) z[e] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    __syncthreads();
+    // Every strictly-lower entry of T and every lower entry of A is written
+    // exactly once; the rest is never read (T) or masked on conversion (A).
     {
       float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
       float* Af = reinterpret_cast<float*>(sm + OFF_AF);
       if (warp < 4) {
-        const int rho = 16 * warp + lane;
+        const int L = 32 * warp + lane;  // lane of the pair accumulators
+        const int rho = L & 63;
         const int rr = rho & 31;
         float* dst = (rho < 32) ? Tf : Af;
 #pragma unroll
-        for (int lv = 2; lv < 6; ++lv) {
+        for (int pr = 0; pr < 2; ++pr) {
+          const int lv = 2 + 2 * pr + (L >> 6);
           float v[32];
-          tmem_ld32(taddr(tmem, 32 * warp, TM_LV + 32 * (lv - 2)), v);
+          tmem_ld32(taddr(tmem, 32 * warp, TM_LV + 64 * pr + 32 * (warp >> 1)), v);
           tmem_ld_wait();
-          if (lane < 16) {
-            const int b = 1 << lv;
-            const int j = rr >> lv;
-            const int r = 2 * b * j + b + (rr & (b - 1));
-            float* row = dst + r * 64 + b * j;
+          const int b = 1 << lv;
+          const int j = rr >> lv;
+          const int r = 2 * b * j + b + (rr & (b - 1));
+          float* row = dst + r * 64 + b * j;
 #pragma unroll
-            for (int m4 = 0; m4 < 8; ++m4) {
-              if (((4 * m4) >> lv) == j)
-                *reinterpret_cast<float4*>(row + 4 * m4) =
-                    make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
-            }
+          for (int m4 = 0; m4 < 8; ++m4) {
+            if (((4 * m4) >> lv) == j)
+              *reinterpret_cast<float4*>(row + 4 * m4) =
+                  make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
           }
         }
       } else {
@@ -731,7 +732,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       const float* Af = reinterpret_cast<const float*>(sm + OFF_AF);
       for (int e = tid; e < 64 * 8; e += NT) {
         const int r = e >> 3, cg = e & 7;
-        st_chunk8(sm + OFF_AQ, sw128_chunk(r, 8 * cg, 64), Af + r * 64 + 8 * cg);
+        float v[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) v[t] = (8 * cg + t <= r) ? Af[r * 64 + 8 * cg + t] : 0.f;
+        st_chunk8(sm + OFF_AQ, sw128_chunk(r, 8 * cg, 64), v);
       }
     }
     __syncthreads();
@@ -747,15 +751,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // 8 x 8 diagonal blocks by forward substitution, one column per thread
       if (tid < 64) {
         const int base = 8 * (tid >> 3), cc = tid & 7;
+        float tb[8][8];
+#pragma unroll
+        for (int r2 = 1; r2 < 8; ++r2) {
+          const float4 lo = *reinterpret_cast<const float4*>(Tf + (base + r2) * 64 + base);
+          const float4 hi = *reinterpret_cast<const float4*>(Tf + (base + r2) * 64 + base + 4);
+          tb[r2][0] = lo.x; tb[r2][1] = lo.y; tb[r2][2] = lo.z; tb[r2][3] = lo.w;
+          tb[r2][4] = hi.x; tb[r2][5] = hi.y; tb[r2][6] = hi.z; tb[r2][7] = hi.w;
+        }
         float x[8];
 #pragma unroll
         for (int r2 = 0; r2 < 8; ++r2) {
           float acc = (r2 == cc) ? 1.f : 0.f;
 #pragma unroll
-          for (int s2 = 0; s2 < r2; ++s2) acc = fmaf(-Tf[(base + r2) * 64 + base + s2], x[s2], acc);
+          for (int s2 = 0; s2 < r2; ++s2) acc = fmaf(-tb[r2][s2], x[s2], acc);
           x[r2] = (r2 < cc) ? 0.f : acc;
-          Inv[(base + r2) * 64 + base + cc] = x[r2];
         }
+#pragma unroll
+        for (int r2 = 0; r2 < 8; ++r2) Inv[(base + r2) * 64 + base + cc] = x[r2];
       }
       __syncthreads();
       inv_merge<8>(Tf, Inv, Yf, tid);
