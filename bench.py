@@ -295,10 +295,23 @@ def run_ours(args, ws, rank, local):
     out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+    path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
+    wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
+                        device=dev)
+    two_phase = path == "tcgen05"
 
-    def step(i):
+    def step(i, mid=None):
+        # One forward over the batch.  On the tensor-core path it is the factor
+        # kernel then the carry kernel (what ckda_fwd_chunked runs), issued as
+        # the two ABI phases so an event between them times each kernel.
         c = sets[i % 2]
-        ck.fwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, out=out, S_final=S_final)
+        if two_phase:
+            ck.fwd_factors(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, workspace=wsbuf)
+            if mid is not None:
+                mid.record(stream)
+            ck.fwd_carry(wsbuf, B, T, H, D, D, chunk=CHUNK, out=out, S_final=S_final)
+        else:
+            ck.fwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, out=out, S_final=S_final)
 
     for i in range(args.warmup):
         step(i)
@@ -313,6 +326,7 @@ def run_ours(args, ws, rank, local):
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     ks = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    km = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     barrier()
     torch.cuda.synchronize(dev)
@@ -320,7 +334,7 @@ def run_ours(args, ws, rank, local):
     ev0.record(stream)
     for i in range(K):
         ks[i].record(stream)
-        step(i)
+        step(i, km[i])
         ke[i].record(stream)
     ev1.record(stream)
     torch.cuda.synchronize(dev)
@@ -330,6 +344,13 @@ def run_ours(args, ws, rank, local):
     elapsed_ms = max_ranks(ev0.elapsed_time(ev1))
     kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(K))
     kern_ms = max_ranks(kern_ms)
+    kernels = None
+    if two_phase:
+        f_ms = max_ranks(statistics.mean(ks[i].elapsed_time(km[i]) for i in range(K)))
+        c_ms = max_ranks(statistics.mean(km[i].elapsed_time(ke[i]) for i in range(K)))
+        kernels = {"factor_kernel": {"ms": f_ms, "share": f_ms / (f_ms + c_ms),
+                                     "workspace_bytes_written": wsbuf.numel()},
+                   "carry_kernel": {"ms": c_ms, "share": c_ms / (f_ms + c_ms)}}
     ms_per_step = elapsed_ms / K
     tokens = B * T
     value = whole_job_rate(tokens, ws, ms_per_step / 1e3)
@@ -347,23 +368,22 @@ def run_ours(args, ws, rank, local):
     e2e = None
     if args.e2e_steps > 0:
         e2e = _run_e2e(args, ck, torch, sets[0], out, S_final, stream, barrier, max_ranks,
-                       ws, tokens, dev)
+                       ws, tokens, dev, wsbuf)
 
     # ---- decode step (B=256, H=32, d=128, bf16), 1024 steps --------------
     decode = None
     if not args.no_decode:
         decode = _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
                              ws, hbm_peak)
-    path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
     _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            _lib.LIB_PATH, path)
+            _lib.LIB_PATH, path, kernels)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, tokens, dev):
+def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, tokens, dev, wsbuf):
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     host = {n: getattr(c, n).cpu().pin_memory() for n in ("q", "k", "v", "alpha", "beta")}
@@ -377,7 +397,7 @@ def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, t
         for n, t in host.items():
             dbuf[n].copy_(t, non_blocking=True)
         ck.fwd_chunked(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["alpha"], dbuf["beta"], chunk=CHUNK,
-                       out=out, S_final=S_final)
+                       out=out, S_final=S_final, workspace=wsbuf)
         out_h.copy_(out, non_blocking=True)
         Sf_h.copy_(S_final, non_blocking=True)
 
@@ -431,7 +451,7 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, 
 
 def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            lib_path, path):
+            lib_path, path, kernels=None):
     # arithmetic of the forward: tcgen05 MMAs on fp16 operands with fp32
     # accumulation and fp32 state, or fp32 FFMA on CUDA cores
     dtype = "f16" if path == "tcgen05" else "f32"
@@ -450,7 +470,10 @@ def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                      "peak_source": f"{peak_src} hbm_gbs (burst copy)",
-                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms},
+                     "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms,
+                     "scope": "the chunked forward: factor kernel + carry kernel, one pair per "
+                              "step; bytes are the forward's algorithmic bytes"},
+        "kernels": kernels,
         "tensor": {"strict_tflops": tflops_strict, "dense_block_tflops": tflops_dense,
                    "frac_strict_of_measured": tflops_strict / tc_peak,
                    "frac_dense_of_measured": tflops_dense / tc_peak,
@@ -458,7 +481,7 @@ def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_
                    "frac_dense_of_spec": tflops_dense / SPEC_BF16_TFLOPS,
                    "measured_bf16_tflops": tc_peak},
         "e2e": e2e,
-        "gpu_launches": K,
+        "gpu_launches": 2 * K if path == "tcgen05" else K,
         "clocks": clocks,
         "wall_s_timed_region": wall,
         "lib": os.path.relpath(lib_path, ROOT),

@@ -22,13 +22,20 @@ STATUS = {
     -4: "CKDA_ERR_CUDA",
     -5: "CKDA_ERR_DEVICE_TIMEOUT",
     -6: "CKDA_ERR_BAD_SEQLENS",
+    -7: "CKDA_ERR_WORKSPACE",
 }
 
 # name -> (restype, argtypes), mirroring include/ckda.h
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
 SIGNATURES = {
-    "ckda_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
+    "ckda_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+                              _vp, ctypes.c_size_t, _vp]),
+    "ckda_fwd_chunked_workspace_bytes": (ctypes.c_int64, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ckda_fwd_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
+                              ctypes.c_size_t, _vp]),
+    "ckda_fwd_carry": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+                            ctypes.c_size_t, _vp]),
     "ckda_fwd_chunked_fp32core": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_fwd_chunked_path": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),

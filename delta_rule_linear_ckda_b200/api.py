@@ -6,6 +6,7 @@ on a non-zero status.  All arithmetic happens in the CUDA kernels.
 """
 from __future__ import annotations
 
+import math
 from typing import Optional, Tuple
 
 import torch
@@ -39,15 +40,62 @@ def _p(t: Optional[torch.Tensor]):
 
 def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
                 out=None, S_final=None, return_final: bool = True, fp32core: bool = False,
-                out_dtype=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+                out_dtype=None, workspace=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
     """Chunked CKDA forward.  Shapes as in ``ckda_fwd_chunked`` (include/ckda.h).
 
     Fixed-length: q, k, alpha ``[B, T, H, dk]``; v ``[B, T, H, dv]``; beta ``[B, T, H]``.
     Packed: ``cu_seqlens`` int32 ``[N+1]`` and tensors with a leading 1 or without it.
     ``out_dtype`` (float32 or bfloat16) defaults to the dtype of ``out`` if given,
-    else to the input dtype.
+    else to the input dtype.  ``workspace`` is an optional uint8 CUDA tensor of at
+    least ``workspace_bytes(...)`` bytes; without it one is taken from torch's
+    caching allocator for the call.
     Returns ``(out, S_final)``; ``S_final`` is None when ``return_final`` is False.
     """
+    dev = q.device
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, cu_seqlens)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must have v's shape")
+    if return_final and S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, dev)
+    lib = _lib.load()
+    with torch.cuda.device(dev):
+        if fp32core:
+            rc = lib.ckda_fwd_chunked_fp32core(
+                _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(out),
+                _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
+                _stream_ptr(dev))
+        else:
+            need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, out_dtype,
+                                   cu_seqlens is not None)
+            if workspace is None and need > 0:
+                workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+            if workspace is not None:
+                _need(workspace, "workspace", torch.uint8, dev)
+            rc = lib.ckda_fwd_chunked(
+                _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(out),
+                _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
+                _p(workspace), 0 if workspace is None else workspace.numel(), _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_fwd_chunked")
+    return out, S_final
+
+
+def _inputs_shape(q, k, v, alpha, beta, cu_seqlens):
+    """Checks the forward inputs; returns (B, T, H, dk, dv, N) as passed to the ABI."""
     dev = q.device
     if q.dtype not in _DT:
         raise TypeError("q, k, v must be float32 or bfloat16")
@@ -75,32 +123,73 @@ def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
         raise ValueError("q, k, alpha must share a shape and v must match it but for the last dim")
     if tuple(beta.shape) != tuple(q.shape[:-1]):
         raise ValueError("beta must have q's shape without the last dim")
+    return B, T, H, dk, dv, N
+
+
+def fwd_factors(q, k, v, alpha, beta, cu_seqlens=None, chunk: int = 64, workspace=None):
+    """Phase 1 of the tensor-core forward: the S0-independent WY factors of every
+    chunk, written to ``workspace`` (uint8 CUDA tensor; allocated if None).
+    Returns the workspace, to be passed to ``fwd_carry`` with the same sizes."""
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, cu_seqlens)
+    dev = q.device
+    need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, torch.float32, cu_seqlens is not None)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_fwd_factors(
+            _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(cu_seqlens), B, T, H, dk, dv, chunk,
+            _DT[q.dtype], _p(workspace), workspace.numel(), _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_fwd_factors")
+    return workspace
+
+
+def fwd_carry(workspace, B, T, H, dk, dv, S0=None, cu_seqlens=None, chunk: int = 64,
+              dtype=torch.bfloat16, out=None, S_final=None, out_dtype=torch.float32,
+              return_final: bool = True):
+    """Phase 2: apply the factors in ``workspace`` from ``S0``.  Sizes (B, T, H as in
+    ``ckda_fwd_chunked``) and ``dtype`` must be those of the ``fwd_factors`` call.
+    Returns ``(out, S_final)``."""
+    dev = workspace.device
+    _need(workspace, "workspace", torch.uint8, dev)
+    N = B
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    shape = (B, T, H, dv) if cu_seqlens is None else (T, H, dv)
+    if out is None:
+        out = torch.empty(shape, dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+        if out.numel() != math.prod(shape):
+            raise ValueError(f"out must hold {shape}")
     if S0 is not None:
         _need(S0, "S0", torch.float32, dev)
         if tuple(S0.shape) != (N, H, dk, dv):
             raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
-    if out_dtype is None:
-        out_dtype = out.dtype if out is not None else q.dtype
-    if out_dtype not in _DT:
-        raise TypeError("out_dtype must be float32 or bfloat16")
-    if out is None:
-        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
-    else:
-        _need(out, "out", out_dtype, dev)
-        if out.shape != v.shape:
-            raise ValueError("out must have v's shape")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, dev)
     if return_final and S_final is None:
         S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if S_final is not None:
         _need(S_final, "S_final", torch.float32, dev)
-    fn = _lib.load().ckda_fwd_chunked_fp32core if fp32core else _lib.load().ckda_fwd_chunked
     with torch.cuda.device(dev):
-        rc = fn(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(out),
-                _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
-                _stream_ptr(dev))
+        rc = _lib.load().ckda_fwd_carry(
+            _p(S0), _p(cu_seqlens), _p(out), _p(S_final), B, T, H, dk, dv, chunk, _DT[dtype],
+            _DT[out_dtype], _p(workspace), workspace.numel(), _stream_ptr(dev))
     if rc != 0:
-        raise CKDAError(rc, "ckda_fwd_chunked")
+        raise CKDAError(rc, "ckda_fwd_carry")
     return out, S_final
+
+
+def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, out_dtype=torch.float32,
+                    varlen=False) -> int:
+    """Scratch bytes ``fwd_chunked`` needs for these sizes (0 on the fp32 CUDA-core path)."""
+    rc = _lib.load().ckda_fwd_chunked_workspace_bytes(B, T, H, dk, dv, chunk, _DT[dtype],
+                                                      _DT[out_dtype], 1 if varlen else 0)
+    if rc < 0:
+        raise CKDAError(int(rc), "ckda_fwd_chunked_workspace_bytes")
+    return int(rc)
 
 
 def fwd_path(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, out_dtype=torch.float32,

@@ -17,12 +17,15 @@ cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void
                             const float* S0, const int32_t* cu, void* out, float* S_final,
                             int n_seqs, int T, int H, int C, int* status, cudaStream_t stream);
 // Returns cudaErrorNotSupported when the shape is not covered by the
-// tensor-core kernel (the caller then uses the CUDA-core kernel).
-cudaError_t launch_fwd_tc(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k, const void* v,
-                          const float* alpha, const float* beta, const float* S0,
-                          const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
-                          int C, int* status, cudaStream_t stream);
-bool fwd_tc_supported(int dtype, int dk, int dv, int C, uint64_t rows);
+// tensor-core kernels (the caller then uses the CUDA-core kernel).
+cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
+                          const void* k, const void* v, const float* alpha, const float* beta,
+                          const float* S0, const int32_t* cu, void* out, float* S_final,
+                          int n_seqs, int T, int H, int C, void* ws, int* status,
+                          cudaStream_t stream);
+bool fwd_tc_supported(int dtype, int dk, int dv, int C, int n_seqs, int T, int H, bool varlen);
+size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int T, int H,
+                              bool varlen);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
                                       cudaStream_t stream);
 }  // namespace ckda
@@ -53,10 +56,14 @@ int* status_ptr() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
+// Forward phases: the inputs are read by the factor phase, out is written by
+// the carry phase; the one-call forward runs both.
+constexpr int kFactors = 1, kCarry = 2, kBoth = 3;
+
 int validate_fwd(const void* q, const void* k, const void* v, const float* alpha,
                  const float* beta, const float* S0, const int32_t* cu, const void* out,
                  const float* S_final, int B, int T, int H, int d_k, int d_v, int* chunk,
-                 int dtype, int out_dtype) {
+                 int dtype, int out_dtype, int phases = kBoth) {
   if (B < 0 || T < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
   if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
   if (out_dtype != CKDA_F32 && out_dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
@@ -64,7 +71,9 @@ int validate_fwd(const void* q, const void* k, const void* v, const float* alpha
   if (*chunk == 0) *chunk = 64;
   if (*chunk != 16 && *chunk != 32 && *chunk != 64) return CKDA_ERR_UNSUPPORTED;
   const int64_t tokens = (cu != nullptr) ? (int64_t)T : (int64_t)B * T;
-  if (tokens > 0 && (!q || !k || !v || !alpha || !beta || !out)) return CKDA_ERR_INVALID_ARG;
+  if (tokens > 0 && (phases & kFactors) && (!q || !k || !v || !alpha || !beta))
+    return CKDA_ERR_INVALID_ARG;
+  if (tokens > 0 && (phases & kCarry) && !out) return CKDA_ERR_INVALID_ARG;
   if (cu == nullptr && (int64_t)B * T * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
   if (cu != nullptr && B == 0 && T != 0) return CKDA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, alpha, beta, S0, out, S_final, cu};
@@ -76,26 +85,52 @@ int validate_fwd(const void* q, const void* k, const void* v, const float* alpha
   return CKDA_OK;
 }
 
-int fwd_impl(bool allow_tc, const void* q, const void* k, const void* v, const float* alpha,
-             const float* beta, const float* S0, const int32_t* cu, void* out, float* S_final,
-             int B, int T, int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
-             void* stream) {
+int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void* v,
+             const float* alpha, const float* beta, const float* S0, const int32_t* cu,
+             void* out, float* S_final, int B, int T, int H, int d_k, int d_v, int chunk,
+             int dtype, int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = validate_fwd(q, k, v, alpha, beta, S0, cu, out, S_final, B, T, H, d_k, d_v, &chunk,
-                        dtype, out_dtype);
+                        dtype, out_dtype, phases);
   if (rc != CKDA_OK) return rc;
   const int n_seqs = B;
+  const bool tc = allow_tc && n_seqs > 0 &&
+                  ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, n_seqs, T, H, cu != nullptr);
+  // the two-phase calls exist only on the tensor-core path
+  if (phases != kBoth && !tc && n_seqs > 0) return CKDA_ERR_UNSUPPORTED;
   if (n_seqs == 0) return CKDA_OK;
+  if (tc) {
+    const size_t need =
+        ckda::fwd_tc_workspace_bytes(dtype, d_k, d_v, chunk, n_seqs, T, H, cu != nullptr);
+    if (workspace == nullptr || workspace_bytes < need ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+      return CKDA_ERR_WORKSPACE;
+    const void* ws_end = static_cast<const uint8_t*>(workspace) + need;
+    const void* ptrs[] = {q, k, v, alpha, beta, S0, out, S_final, cu};
+    for (const void* p : ptrs)
+      if (p != nullptr && p >= workspace && p < ws_end) return CKDA_ERR_WORKSPACE;
+  }
   int* status = status_ptr();
   if (status == nullptr) return CKDA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
-  if (allow_tc)
-    e = ckda::launch_fwd_tc(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs,
-                            T, H, chunk, status, st);
+  if (tc)
+    e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu,
+                            out, S_final, n_seqs, T, H, chunk, workspace, status, st);
   if (e == cudaErrorNotSupported)
     e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final,
                               n_seqs, T, H, chunk, status, st);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
+
+// Sizes only: validate with stand-in aligned pointers that are never used.
+int validate_sizes(int B, int T, int H, int d_k, int d_v, int* chunk, int dtype, int out_dtype,
+                   int varlen) {
+  const void* p = reinterpret_cast<const void*>(static_cast<uintptr_t>(1) << 20);
+  const int32_t* cu = varlen ? reinterpret_cast<const int32_t*>(static_cast<uintptr_t>(2) << 20)
+                             : nullptr;
+  return validate_fwd(p, p, p, static_cast<const float*>(p), static_cast<const float*>(p),
+                      nullptr, cu, reinterpret_cast<const void*>(static_cast<uintptr_t>(3) << 20),
+                      nullptr, B, T, H, d_k, d_v, chunk, dtype, out_dtype);
 }
 
 }  // namespace
@@ -113,6 +148,7 @@ const char* ckda_status_string(int status) {
     case CKDA_ERR_CUDA: return "CUDA runtime or launch error";
     case CKDA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
     case CKDA_ERR_BAD_SEQLENS: return "cu_seqlens is not a valid offsets array";
+    case CKDA_ERR_WORKSPACE: return "workspace missing, too small, misaligned or overlapping";
   }
   return "unknown status";
 }
@@ -120,31 +156,47 @@ const char* ckda_status_string(int status) {
 int ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, const float* S0, const int32_t* cu_seqlens, void* out,
                      float* S_final, int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
-                     int out_dtype, void* stream) {
-  return fwd_impl(true, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
-                  chunk, dtype, out_dtype, stream);
+                     int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(true, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
+                  d_v, chunk, dtype, out_dtype, workspace, workspace_bytes, stream);
+}
+
+int ckda_fwd_factors(const void* q, const void* k, const void* v, const float* alpha,
+                     const float* beta, const int32_t* cu_seqlens, int B, int T, int H, int d_k,
+                     int d_v, int chunk, int dtype, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  return fwd_impl(true, kFactors, q, k, v, alpha, beta, nullptr, cu_seqlens, nullptr, nullptr, B,
+                  T, H, d_k, d_v, chunk, dtype, CKDA_F32, workspace, workspace_bytes, stream);
+}
+
+int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* out, float* S_final, int B,
+                   int T, int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(true, kCarry, nullptr, nullptr, nullptr, nullptr, nullptr, S0, cu_seqlens, out,
+                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, workspace,
+                  workspace_bytes, stream);
 }
 
 int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void* v, const float* alpha,
                               const float* beta, const float* S0, const int32_t* cu_seqlens,
                               void* out, float* S_final, int B, int T, int H, int d_k, int d_v,
                               int chunk, int dtype, int out_dtype, void* stream) {
-  return fwd_impl(false, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
-                  chunk, dtype, out_dtype, stream);
+  return fwd_impl(false, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
+                  d_v, chunk, dtype, out_dtype, nullptr, 0, stream);
 }
 
 int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
                           int out_dtype, int varlen) {
-  // Sizes only: validate with stand-in aligned pointers that are never used.
-  const void* p = reinterpret_cast<const void*>(static_cast<uintptr_t>(1) << 20);
-  const int32_t* cu = varlen ? reinterpret_cast<const int32_t*>(static_cast<uintptr_t>(2) << 20)
-                             : nullptr;
-  int rc = validate_fwd(p, p, p, static_cast<const float*>(p), static_cast<const float*>(p),
-                        nullptr, cu, reinterpret_cast<const void*>(static_cast<uintptr_t>(3) << 20),
-                        nullptr, B, T, H, d_k, d_v, &chunk, dtype, out_dtype);
+  int rc = validate_sizes(B, T, H, d_k, d_v, &chunk, dtype, out_dtype, varlen);
   if (rc != CKDA_OK) return rc;
-  const uint64_t rows = varlen ? (uint64_t)T : (uint64_t)B * (uint64_t)T;
-  return ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, rows) ? 1 : 0;
+  return ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, B, T, H, varlen != 0) ? 1 : 0;
+}
+
+int64_t ckda_fwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v, int chunk,
+                                         int dtype, int out_dtype, int varlen) {
+  int rc = validate_sizes(B, T, H, d_k, d_v, &chunk, dtype, out_dtype, varlen);
+  if (rc != CKDA_OK) return rc;
+  return (int64_t)ckda::fwd_tc_workspace_bytes(dtype, d_k, d_v, chunk, B, T, H, varlen != 0);
 }
 
 int ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,

@@ -11,14 +11,22 @@
 // Contribuciones" item 3; "Gated DeltaNet-2" page, Methodology section 3:
 // decay absorbed into the WY factors and the triangular solve (I + T)^-1.)
 //
-// The form used here groups the S0-independent work so that the carry is
-// two dependent tensor-core products per chunk:
-//   P  = A Inv diag(beta)
-//   [W, U~; A W, A U~] = [Inv diag(beta); P] [K * Gamma, V]      (one M=128 MMA)
-//   Q' = Q * Gamma - A W
-//   X  = [W; Q'] S0                                             (carry MMA 1)
-//   U  = U~ - X_top,   O = A U~ + X_bottom
-//   D  = (K * rho)^T U,  S_C = Diag(gamma) S0 + D               (carry MMA 2)
+// Everything except the last two lines is independent of S0, so the forward
+// runs as two kernels:
+//
+//  1. factor_kernel -- one work unit per (chunk, head), all units in
+//     parallel (a persistent grid of one CTA per SM walks them).  It forms
+//       P  = A Inv diag(beta)
+//       [W, U~; A W, A U~] = [Inv diag(beta); P] [K * Gamma, V]   (one M=128 MMA)
+//       Q' = Q * Gamma - A W
+//     and writes [W; Q'] (fp16), K * rho (fp16), [U~; A U~] (fp32) and
+//     gamma (fp32) of the unit to a workspace.
+//  2. carry_kernel -- one CTA per (sequence, head, 64-column d_v slice)
+//     walks its chunks in order with two dependent tensor-core products each:
+//       X  = [W; Q'] S0                                 (carry MMA 1)
+//       U  = U~ - X_top,   O = A U~ + X_bottom
+//       D  = (K * rho)^T U,  S_C = Diag(gamma) S0 + D   (carry MMA 2)
+//     while TMA streams the next chunk's factors in.
 //
 // Division-free score blocks: every pair s < r is split at the anchor m of
 // the highest bit in which r and s differ ("level" h, block size b = 2^h):
@@ -33,15 +41,15 @@
 // its 8 positions, and combines them with the products of whole groups
 // (exchanged through shared memory) into the level operands and into
 // K * Gamma, Q * Gamma and K * rho.  The pass runs once per 64-channel half
-// of d_k, so the level GEMMs are split along K and the next chunk's inputs
-// stream in by TMA while the rest of the chunk runs.
+// of d_k, so the level GEMMs are split along K and the next unit's inputs
+// stream in by TMA while the rest of the unit runs.
 //
-// One CTA (256 threads) owns one (sequence, head, 64-column d_v slice) and
-// walks its chunks in order.  Operands are fp16 tiles in 128-byte-swizzled
-// shared memory; accumulators live in tensor memory; the state slice stays
-// in fp32 registers (row i = tensor-memory lane i).  Every mbarrier wait is
-// bounded: on time-out the kernel records CKDA_ERR_DEVICE_TIMEOUT, waits once
-// more (bounded) for its own copies, frees its tensor memory and returns.
+// Operands are fp16 tiles in 128-byte-swizzled shared memory; accumulators
+// live in tensor memory; the carry kernel keeps its state slice in fp32
+// registers (row i = tensor-memory lane i).  Every mbarrier wait is
+// bounded: on time-out the kernel records CKDA_ERR_DEVICE_TIMEOUT, waits
+// once more (bounded) for its own copies, frees its tensor memory and
+// returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -56,21 +64,27 @@ using namespace sm100;
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int HC = 64;  // channels per half of d_k
-constexpr int BV = 64;
+constexpr int BV = 64;  // d_v columns of one carry CTA
 constexpr int NT = 256;
-constexpr uint32_t kTmemCols = 512;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
-// ---- shared memory map (byte offsets from a 1024-aligned base) ----------
+// ---- workspace: per unit (one chunk of one head), four arrays -------------
+constexpr size_t kWsWQ = (size_t)2 * C * DK * 2;  // [W; Q'] fp16 [128][128]
+constexpr size_t kWsKH = (size_t)C * DK * 2;      // K * rho fp16 [64][128]
+constexpr size_t kWsG = (size_t)DK * 4;           // gamma fp32 [128]
+// [U~; A U~] fp32 [128][d_v]: 2 * C * d_v * 4 bytes
+
+// ---- factor kernel: shared memory map (byte offsets, 1024-aligned base) ---
 // Two input buffers, one per 64-channel half: q, k (bf16 [64 pos][64 ch])
 // and alpha (fp32 [64 pos][64 ch]), filled by TMA.
 constexpr uint32_t OFF_IN0 = 0;
 constexpr uint32_t OFF_IN1 = 32768;
 constexpr uint32_t IN_Q = 0, IN_K = 8192, IN_A = 16384, kInBytes = 32768;
-constexpr uint32_t OFF_V = 65536;  // v slice (TMA, 128B swizzle), bf16 -> fp16 [64 s][64 j]
+// v tile (TMA, 128B swizzle), bf16 -> fp16 [64 s][d_v] as 64-column atoms
+constexpr uint32_t OFF_V = 65536;
 // Work region: level operands while the gate pass runs; then the fp32
-// inverse workspace and the A / [Inv; P] operands; then the U operand.
-constexpr uint32_t OFF_LVX = 73728;
+// inverse workspace and the A / [Inv; P] operands.
+constexpr uint32_t OFF_LVX = 81920;
 // Levels are paired (2, 3) and (4, 5): one M=128 x N=64 GEMM per pair, of
 // which the two diagonal 64 x 32 blocks are used.  Per pair: the left
 // operand [levels a; b] (128 rows) and the right operand (64 rows).
@@ -81,31 +95,52 @@ constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A staging then (I + T)^-1, fp32
 constexpr uint32_t OFF_AQ = OFF_LVX + 32768;  // A, fp16 K-major [64 r][64 s]
 constexpr uint32_t OFF_IP = OFF_LVX + 40960;  // [Inv diag(beta); P], fp16 K-major [128][64]
 constexpr uint32_t OFF_YF = OFF_LVX + 57344;  // doubling scratch, fp32 (<= 1024 values)
-constexpr uint32_t OFF_UB = OFF_LVX;          // U, fp16 MN-major [64 s][64 j]
-constexpr uint32_t OFF_KG = 139264;  // K * Gamma, fp16 MN-major [64 s][128 i]
-constexpr uint32_t OFF_WQ = 155648;  // [W; Q'] fp16 K-major [128][128]; rows 64.. hold Q * Gamma first
-constexpr uint32_t OFF_KH = 188416;  // K * rho, fp16 MN-major [64 s][128 i]
-constexpr uint32_t OFF_SB = 204800;  // state slice, fp16 MN-major [128 i][64 j]
-constexpr uint32_t OFF_GT = 221184;  // products of whole 8-position groups, fp32 [8][64]
-constexpr uint32_t OFF_PR = 223232;  // direct pairs and diag(A), fp32 [8 groups][32]
-constexpr uint32_t OFF_BETA = 224256;
-constexpr uint32_t OFF_GAMMA = 224512;
-constexpr uint32_t OFF_BAR = 225024;  // mbarriers: in0, in1, v, mma, lv
-constexpr uint32_t OFF_TMEMPTR = 225088;
-constexpr uint32_t kSmemUsed = 225104;
+constexpr uint32_t OFF_KG = 143360;  // K * Gamma, fp16 MN-major [64 s][128 i]
+constexpr uint32_t OFF_QG = 159744;  // Q * Gamma, then Q', fp16 [64 r][128 i] (128B swizzle)
+constexpr uint32_t OFF_KH = 176128;  // K * rho, then W, fp16 [64][128 i] (128B swizzle)
+constexpr uint32_t OFF_GT = 192512;  // products of whole 8-position groups, fp32 [8][64]
+constexpr uint32_t OFF_PR = 194560;  // direct pairs and diag(A), fp32 [8 groups][32]
+constexpr uint32_t OFF_BETA = 195584;
+constexpr uint32_t OFF_GAMMA = 195840;
+constexpr uint32_t OFF_BAR = 196352;  // mbarriers: in0, in1, v, mma, lv
+constexpr uint32_t OFF_TMEMPTR = 196416;
+constexpr uint32_t kSmemUsed = 196432;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
+// Staging of the workspace tiles for their TMA stores: [U~; A U~] as
+// [128][32] fp32 atoms over the dead work region and K * Gamma (up to 4
+// atoms), W over K * rho (stored to the workspace after the gate passes),
+// Q' in place of Q * Gamma.
+constexpr uint32_t OFF_UUST = OFF_LVX;
 
-// ---- tensor memory columns ------------------------------------------------
+// factor kernel tensor-memory columns
+constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t TM_LV = 0;    // level pairs, 64 columns each (M = 128)
 constexpr uint32_t TM_P = 128;   // P (M = 64 layout)
 constexpr uint32_t TM_W = 192;   // [W; A W]       (M = 128, 128 columns)
-constexpr uint32_t TM_U = 320;   // [U~; A U~]     (M = 128, 64 columns)
-constexpr uint32_t TM_X = 384;   // [W S; Q' S]    (M = 128, 64 columns)
-constexpr uint32_t TM_D = 448;   // (K rho)^T U    (M = 128, 64 columns)
+constexpr uint32_t TM_U = 320;   // [U~; A U~]     (M = 128, d_v columns)
+
+// ---- carry kernel: shared memory map ---------------------------------------
+// Two stages of one chunk's factors, each filled by one TMA transaction.
+constexpr uint32_t CS_WQ = 0;      // [W; Q'] fp16 K-major [128][128] (two 64-column atoms)
+constexpr uint32_t CS_KH = 32768;  // K * rho fp16 MN-major [64 s][128 i]
+constexpr uint32_t CS_UU = 49152;  // [U~; A U~] fp32 [128][64 of d_v] as two [128][32] atoms
+constexpr uint32_t kStageBytes = 81920;
+constexpr uint32_t OFF2_SB = 2 * kStageBytes;  // state slice, fp16 MN-major [128 i][64 j]
+constexpr uint32_t OFF2_UB = OFF2_SB + 16384;  // U, fp16 MN-major [64 s][64 j]
+constexpr uint32_t OFF2_OB = OFF2_UB + 8192;  // O staging for its TMA store: fp32 [64][32] x 2 or bf16 [64][64]
+constexpr uint32_t OFF2_BAR = OFF2_OB + 16384;  // mbarriers: stage 0, stage 1, mma
+constexpr uint32_t OFF2_TMEMPTR = OFF2_BAR + 32;
+constexpr uint32_t kSmem2Used = OFF2_TMEMPTR + 16;
+constexpr size_t kSmem2Bytes = kSmem2Used + 1024;
+
+// carry kernel tensor-memory columns
+constexpr uint32_t kTmem2Cols = 128;
+constexpr uint32_t TM2_X = 0;    // [W S; Q' S]    (M = 128, 64 columns)
+constexpr uint32_t TM2_D = 64;   // (K rho)^T U    (M = 128, 64 columns)
 
 #ifdef CKDA_TC_DEBUG
-// Intermediate dump of the first chunk of CTA (0, 0, 0) and per-phase clock
-// counts (diagnostic builds only).
+// Intermediate dump of the first unit of CTA 0 and of the first chunk of
+// carry CTA (0, 0, 0), and per-phase clock counts (diagnostic builds only).
 __device__ float* g_tc_dbg = nullptr;
 __device__ unsigned long long* g_tc_time = nullptr;
 __device__ unsigned long long* g_tc_time2 = nullptr;
@@ -231,6 +266,41 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
   }
 }
 
+// Row r (0..63) of the output tile, columns [32 * half, +32), as a + x into
+// the 128B-swizzled staging of the TMA store: fp32 as two [64][32] atoms,
+// bf16 as one [64][64] atom.
+template <typename Tout>
+__device__ __forceinline__ void stage_row32(uint32_t ob, int r, int half, const float* a,
+                                            const float* x);
+
+template <>
+__device__ __forceinline__ void stage_row32<float>(uint32_t ob, int r, int half, const float* a,
+                                                   const float* x) {
+  const uint32_t row = ob + 8192 * half + 128 * r;
+#pragma unroll
+  for (int c4 = 0; c4 < 8; ++c4) {
+    const int e = 4 * c4;
+    sts_f4(row + ((c4 ^ (r & 7)) << 4),
+           make_float4(a[e] + x[e], a[e + 1] + x[e + 1], a[e + 2] + x[e + 2], a[e + 3] + x[e + 3]));
+  }
+}
+
+template <>
+__device__ __forceinline__ void stage_row32<__nv_bfloat16>(uint32_t ob, int r, int half,
+                                                           const float* a, const float* x) {
+  const uint32_t row = ob + 128 * r;
+#pragma unroll
+  for (int c8 = 0; c8 < 4; ++c8) {
+    const int e = 8 * c8;
+    uint32_t w[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(a[e + 2 * t] + x[e + 2 * t], a[e + 2 * t + 1] + x[e + 2 * t + 1]);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (((4 * half + c8) ^ (r & 7)) << 4)),
+                 "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+                 : "memory");
+  }
+}
+
 // One gate pass over one 64-channel half (see the file comment).  Thread
 // (c4, g, role): channels 4*c4 .. 4*c4+3 of the half, positions 8g .. 8g+7.
 // Role 0 walks forward (prefix products: Gamma and the right halves of
@@ -314,7 +384,7 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
       pg = mul4(pg, a);
       lp = (u == 0) ? a : mul4(lp, a);
       sts_u2(sb + OFF_KG + sw128_elem(p, ig, 64), h4(mul4(kf, pg)));
-      sts_u2(sb + OFF_WQ + sw128_elem(64 + p, ig, 128), h4(mul4(qf, pg)));
+      sts_u2(sb + OFF_QG + sw128_elem(p, ig, 64), h4(mul4(qf, pg)));
       if (u >= 4) {  // level 2: right half of the group
         l2 = (u == 4) ? a : mul4(l2, a);
         const int rho = 4 * g + u - 4;
@@ -481,13 +551,82 @@ __device__ __forceinline__ void inv_merge(const float* Tf, float* Inv, float* Yf
   }
 }
 
-template <typename Tout>
+// ---- work units ----------------------------------------------------------------
+//
+// A unit is one chunk of one head.  Units are numbered slot * H + head, and a
+// sequence's chunks occupy consecutive slots:
+//   fixed-length batch:  slot = n * nch + c                   (nch = ceil(T / C))
+//   packed batch:        slot = floor(cu[n] / C) + n + c
+// For a packed batch the slots of sequence n end before those of n + 1
+// (floor(cu[n] / C) + ceil(len_n / C) <= floor(cu[n+1] / C) + 1), so every
+// slot is owned by at most one sequence and all lie below floor(T / C) + N.
+
+struct Unit {
+  int64_t idx;  // unit number; -1 = none left
+  int64_t t0;   // first token row of the chunk
+  int Lc;       // tokens in the chunk (1..C)
+  int h;        // head
+};
+
+__device__ __forceinline__ int64_t slot_base(const int32_t* cu, int n, int nch) {
+  return cu ? (int64_t)(cu[n] / C) + n : (int64_t)n * nch;
+}
+
+// The first unit at or after `ui` (stepping by `stride`) that holds tokens.
+__device__ Unit find_unit(int64_t ui, int64_t stride, int64_t n_units, const int32_t* cu,
+                          int n_seqs, int T, int H, int nch) {
+  for (; ui < n_units; ui += stride) {
+    const int64_t slot = ui / H;
+    const int h = (int)(ui - slot * H);
+    int64_t b, e, c;
+    if (cu == nullptr) {
+      if (nch <= 0) break;
+      const int n = (int)(slot / nch);
+      c = slot - (int64_t)n * nch;
+      b = (int64_t)n * T;
+      e = b + T;
+    } else {
+      // last sequence n with floor(cu[n] / C) + n <= slot
+      int lo = 0, hi = n_seqs - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)(cu[mid] / C) + mid <= slot)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      b = cu[lo];
+      e = cu[lo + 1];
+      c = slot - ((int64_t)(b / C) + lo);
+      if (b < 0 || e < b || e > T || c < 0) continue;
+    }
+    const int64_t t0 = b + c * C;
+    if (t0 >= e) continue;
+    Unit u;
+    u.idx = ui;
+    u.t0 = t0;
+    u.Lc = (e - t0 < (int64_t)C) ? (int)(e - t0) : C;
+    u.h = h;
+    return u;
+  }
+  Unit none;
+  none.idx = -1;
+  none.t0 = 0;
+  none.Lc = 0;
+  none.h = 0;
+  return none;
+}
+
+// ---- kernel 1: per-unit WY factors ----------------------------------------------
+
+template <int DV>
 __global__ void __launch_bounds__(NT, 1)
-fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-              const float* __restrict__ beta, const float* S0, const int32_t* __restrict__ cu,
-              Tout* __restrict__ out, float* S_final, int n_seqs, int T, int H, int DV,
-              int* status) {
+              const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
+              const __grid_constant__ CUtensorMap tm_uu, const float* __restrict__ beta,
+              const int32_t* __restrict__ cu, int n_seqs, int T, int H, int nch, int64_t n_units,
+              float* __restrict__ ws_g, int* status) {
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
   // access below in the shared state space.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -496,12 +635,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int j0 = blockIdx.x * BV;
-  const int h = blockIdx.y;
-  const int n = blockIdx.z;
-
-  const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
-  if (!sr.ok) return;
+  const int q4 = warp & 3;
+  const int half = warp >> 2;
 
   float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
   const float* gamma_s = reinterpret_cast<const float*>(sm + OFF_GAMMA);
@@ -522,6 +657,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_wq);
+    prefetch_tmap(&tm_kh);
+    prefetch_tmap(&tm_uu);
   }
   if (warp == 0) {
     tmem_alloc(sb + OFF_TMEMPTR, kTmemCols);
@@ -536,49 +674,35 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   long long tlast = clock64();
 #endif
 
-  // State slice: row i = 32 * (warp % 4) + lane, columns [32 * (warp / 4), +32).
-  const int q4 = warp & 3;
-  const int half = warp >> 2;
-  const int srow = 32 * q4 + lane;
-  const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + 32 * half;
-  float S[32];
-#pragma unroll
-  for (int e = 0; e < 32; e += 4) {
-    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (S0 != nullptr) v4 = *reinterpret_cast<const float4*>(S0 + s_off + e);
-    S[e] = v4.x; S[e + 1] = v4.y; S[e + 2] = v4.z; S[e + 3] = v4.w;
-  }
-#pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4) st_chunk8(sm + OFF_SB, sw128_chunk(srow, 32 * half + 8 * c4, 128), S + 8 * c4);
-
-  const int64_t tok0 = sr.begin;
-  const int64_t tok1 = sr.end;
-  const int nchunks = (int)((tok1 - tok0 + C - 1) / C);
+  // A phase bit advances only when its wait succeeds, and a barrier stays
+  // "pending" from its issue to that wait, so the time-out path below knows
+  // exactly which copies and products may still be in flight.
   uint32_t ph_in0 = 0, ph_in1 = 0, ph_v = 0, ph_mma = 0, ph_lv = 0;
-  int pend_in0 = 0, pend_in1 = 0, pend_v = 0;
+  int pend_in0 = 0, pend_in1 = 0, pend_v = 0, pend_mma = 0, pend_lv = 0;
   int ok = 1;
+  auto wait = [&](uint32_t bar, uint32_t& ph, int& pend) -> bool {
+    const bool r = mbar_wait_bounded(bar, ph, kWaitNs);
+    if (r) {
+      ph ^= 1;
+      pend = 0;
+    }
+    return r;
+  };
 
-  auto issue_in = [&](int hh, int64_t t0) {
+  auto issue_in = [&](int hh, const Unit& u) {
     const uint32_t base = sb + (hh ? OFF_IN1 : OFF_IN0);
     const uint32_t bar = hh ? bar_in1 : bar_in0;
     mbar_expect_tx(bar, kInBytes);
-    tma_load_2d(base + IN_Q, &tm_q, h * DK + HC * hh, (int)t0, bar);
-    tma_load_2d(base + IN_K, &tm_k, h * DK + HC * hh, (int)t0, bar);
-    tma_load_2d(base + IN_A, &tm_a, h * DK + HC * hh, (int)t0, bar);
+    tma_load_2d(base + IN_Q, &tm_q, u.h * DK + HC * hh, (int)u.t0, bar);
+    tma_load_2d(base + IN_K, &tm_k, u.h * DK + HC * hh, (int)u.t0, bar);
+    tma_load_2d(base + IN_A, &tm_a, u.h * DK + HC * hh, (int)u.t0, bar);
   };
-  auto issue_v = [&](int64_t t0) {
-    mbar_expect_tx(bar_v, 8192);
-    tma_load_2d(sb + OFF_V, &tm_v, h * DV + j0, (int)t0, bar_v);
+  auto issue_v = [&](const Unit& u) {
+    mbar_expect_tx(bar_v, 8192 * (DV / 64));
+#pragma unroll
+    for (int a = 0; a < DV / 64; ++a)
+      tma_load_2d(sb + OFF_V + 8192 * a, &tm_v, u.h * DV + 64 * a, (int)u.t0, bar_v);
   };
-  if (nchunks > 0) {
-    if (tid == 0) {
-      issue_in(0, tok0);
-      issue_in(1, tok0);
-      issue_v(tok0);
-    }
-    pend_in0 = pend_in1 = pend_v = 1;
-  }
-
   auto level_mmas = [&](int hh) {
     constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
 #pragma unroll
@@ -594,17 +718,34 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mma_commit(bar_lv);
   };
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int64_t t0 = tok0 + (int64_t)c * C;
-    const int Lc = (tok1 - t0 < (int64_t)C) ? (int)(tok1 - t0) : C;
-    const bool more = c + 1 < nchunks;
-    if (tid < C) beta_s[tid] = (tid < Lc) ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+  // beta of a unit, one value per thread tid < C (0 past the end)
+  auto load_beta = [&](const Unit& uu) -> float {
+    return (uu.idx >= 0 && tid < uu.Lc) ? beta[(size_t)(uu.t0 + tid) * H + uu.h] : 0.f;
+  };
+  Unit cur = find_unit(blockIdx.x, gridDim.x, n_units, cu, n_seqs, T, H, nch);
+  float beta_next = 0.f;
+  if (cur.idx >= 0) {
+    if (tid == 0) {
+      issue_in(0, cur);
+      issue_in(1, cur);
+      issue_v(cur);
+    }
+    pend_in0 = pend_in1 = pend_v = 1;
+    if (tid < C) beta_next = load_beta(cur);
+  }
+
+  for (int c = 0; cur.idx >= 0; ++c) {
+    const Unit nxt = find_unit(cur.idx + gridDim.x, gridDim.x, n_units, cu, n_seqs, T, H, nch);
+    const bool more = nxt.idx >= 0;
+    const int Lc = cur.Lc;
+    const size_t u = (size_t)cur.idx;
+    if (tid < C) beta_s[tid] = beta_next;
     // ---- gate pass, half 0 ---------------------------------------------------
-    ok = mbar_wait_bounded(bar_in0, ph_in0, kWaitNs);
-    ph_in0 ^= 1;
+    ok = wait(bar_in0, ph_in0, pend_in0);
+    // the previous unit's workspace stores must have read their staging
+    if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    pend_in0 = 0;
     TC_MARK(0);
     gate_pass(sb, sb + OFF_IN0, 0, Lc, tid);
     fence_proxy_async_smem();
@@ -612,36 +753,37 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) {
       tc_fence_after();
       level_mmas(0);
-      if (more) issue_in(0, t0 + C);
+      if (more) issue_in(0, nxt);
     }
+    pend_lv = 1;
     if (more) pend_in0 = 1;
+    if (tid < C) beta_next = load_beta(nxt);
     TC_MARK(1);
 
     // ---- gate pass, half 1 (after the half-0 level GEMMs release the operands)
-    ok = mbar_wait_bounded(bar_in1, ph_in1, kWaitNs);
-    ph_in1 ^= 1;
-    ok = mbar_wait_bounded(bar_lv, ph_lv, kWaitNs) && ok;
-    ph_lv ^= 1;
+    ok = wait(bar_in1, ph_in1, pend_in1);
+    ok = wait(bar_lv, ph_lv, pend_lv) && ok;
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    pend_in1 = 0;
     gate_pass(sb, sb + OFF_IN1, 1, Lc, tid);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
       level_mmas(1);
-      if (more) issue_in(1, t0 + C);
+      if (more) issue_in(1, nxt);
+      // K * rho is complete: store it to the workspace
+      tma_store_2d(&tm_kh, sb + OFF_KH, 0, (int)(u * C));
+      tma_store_2d(&tm_kh, sb + OFF_KH + 8192, 64, (int)(u * C));
+      bulk_commit();
     }
+    pend_lv = 1;
     if (more) pend_in1 = 1;
     TC_MARK(2);
-    ok = mbar_wait_bounded(bar_lv, ph_lv, kWaitNs);
-    ph_lv ^= 1;
-    ok = mbar_wait_bounded(bar_v, ph_v, kWaitNs) && ok;
-    ph_v ^= 1;
+    ok = wait(bar_lv, ph_lv, pend_lv);
+    ok = wait(bar_v, ph_v, pend_v) && ok;
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    pend_v = 0;
     tc_fence_after();
     TC_MARK(3);
 
@@ -698,9 +840,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       // v tile: bf16 (as loaded) -> fp16 in place; rows past the end -> 0.
       // Each 16-byte chunk stays within its 128-byte row under the swizzle.
       uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V);
-      for (int e = tid; e < C * 8; e += NT) {
+      for (int e = tid; e < C * 8 * (DV / 64); e += NT) {
         uint4 raw = vt[e];
-        if ((e >> 3) < Lc) {
+        if (((e >> 3) & 63) < Lc) {
           float f[8];
           const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
@@ -800,8 +942,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       mma_commit(bar_mma);
     }
-    ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
-    ph_mma ^= 1;
+    pend_mma = 1;
+    ok = wait(bar_mma, ph_mma, pend_mma);
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
@@ -826,7 +968,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id1 = idesc_f16(128, 128, 0, 1);
-      constexpr uint32_t id2 = idesc_f16(128, 64, 0, 1);
+      constexpr uint32_t id2 = idesc_f16(128, DV, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = smem_desc(sb + OFF_IP + kk * 32, 16, 1024, kSwizzle128);
@@ -841,20 +983,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       }
       mma_commit(bar_mma);
     }
-    ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
-    ph_mma ^= 1;
+    pend_mma = 1;
+    ok = wait(bar_mma, ph_mma, pend_mma);
     fence_proxy_async_smem();
+    // K * rho has been read out: its tile takes W next
+    if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    // the v tile is free: fetch the next chunk's
+    // the v tile is free: fetch the next unit's
     if (more) {
-      if (tid == 0) issue_v(t0 + C);
+      if (tid == 0) issue_v(nxt);
       pend_v = 1;
     }
     TC_MARK(7);
 
-    // ---- [W; Q' = Q Gamma - A W] -> carry operand -------------------------------
+    // ---- [W; Q' = Q Gamma - A W], [U~; A U~] and gamma -> workspace -------------
+    // Each thread holds one tensor-memory row; the rows go to 128B-swizzled
+    // staging tiles (conflict-free), which TMA stores to the workspace.
     {
       const int L = 32 * q4 + lane;
       float v[64];
@@ -862,29 +1008,193 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tmem_ld32(taddr(tmem, 32 * q4, TM_W + 64 * half + 32), v + 32);
       tmem_ld_wait();
       TC_DBG(for (int e = 0; e < 64; ++e) g_tc_dbg[16384 + L * 128 + 64 * half + e] = v[e]);
-      if (L >= 64) {
-        // Q * Gamma sits in this row of the tile already (written by the gate pass)
+      // W rows -> the K * rho tile; Q' rows replace Q * Gamma in place
+      const int r = L & 63;
+      const uint32_t dst = sb + ((L < 64) ? OFF_KH : OFF_QG);
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const uint4 raw =
-              *reinterpret_cast<const uint4*>(sm + OFF_WQ + sw128_chunk(L, 64 * half + 8 * c8, 128));
+      for (int c8 = 0; c8 < 8; ++c8) {
+        const uint32_t off = dst + sw128_chunk(r, 64 * half + 8 * c8, 64);
+        float w8[8];
+        if (L >= 64) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(sm + (off - sb));
           const __half2* p2 = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
             const float2 f = __half22float2(p2[t]);
-            v[8 * c8 + 2 * t] = f.x - v[8 * c8 + 2 * t];
-            v[8 * c8 + 2 * t + 1] = f.y - v[8 * c8 + 2 * t + 1];
+            w8[2 * t] = f.x - v[8 * c8 + 2 * t];
+            w8[2 * t + 1] = f.y - v[8 * c8 + 2 * t + 1];
           }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) w8[t] = v[8 * c8 + t];
         }
+        st_chunk8(sm, off - sb, w8);
       }
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        st_chunk8(sm + OFF_WQ, sw128_chunk(L, 64 * half + 8 * c8, 128), v + 8 * c8);
+      for (int a = 0; a < DV / 64; ++a) {
+        float w[32];
+        tmem_ld32(taddr(tmem, 32 * q4, TM_U + (DV / 2) * half + 32 * a), w);
+        tmem_ld_wait();
+        const uint32_t row = sb + OFF_UUST + 16384 * ((DV / 64) * half + a) + 128 * L;
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4)
+          sts_f4(row + ((c4 ^ (L & 7)) << 4),
+                 make_float4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]));
+      }
+      if (tid < DK) ws_g[u * DK + tid] = gamma_s[tid];
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+      const int y = (int)(u * 2 * C);
+      tma_store_2d(&tm_wq, sb + OFF_KH, 0, y);
+      tma_store_2d(&tm_wq, sb + OFF_KH + 8192, 64, y);
+      tma_store_2d(&tm_wq, sb + OFF_QG, 0, y + C);
+      tma_store_2d(&tm_wq, sb + OFF_QG + 8192, 64, y + C);
+#pragma unroll
+      for (int a = 0; a < DV / 32; ++a) tma_store_2d(&tm_uu, sb + OFF_UUST + 16384 * a, 32 * a, y);
+      bulk_commit();
+    }
     TC_MARK(8);
+    cur = nxt;
+  }
+#ifdef CKDA_TC_DEBUG
+  if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+    for (int k = 0; k < 9; ++k) g_tc_time[k] = tmark[k];
+#endif
+  if (tid == 0) bulk_wait_all();
+
+  if (!ok) {
+    if (tid == 0) {
+      set_status(status, CKDA_ERR_DEVICE_TIMEOUT);
+      // wait (bounded) for copies and tensor-core work this CTA still has in flight
+      if (pend_in0) mbar_wait_bounded(bar_in0, ph_in0, kWaitNs);
+      if (pend_in1) mbar_wait_bounded(bar_in1, ph_in1, kWaitNs);
+      if (pend_v) mbar_wait_bounded(bar_v, ph_v, kWaitNs);
+      if (pend_mma) mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
+      if (pend_lv) mbar_wait_bounded(bar_lv, ph_lv, kWaitNs);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---- kernel 2: the chunk-to-chunk carry ---------------------------------------------
+
+template <typename Tout>
+__global__ void __launch_bounds__(NT, 1)
+carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
+             const __grid_constant__ CUtensorMap tm_uu, const __grid_constant__ CUtensorMap tm_out,
+             const float* __restrict__ ws_g,
+             const float* S0, const int32_t* __restrict__ cu, Tout* __restrict__ out,
+             float* S_final, int n_seqs, int T, int H, int DV, int nch, int* status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t sb = smem_u32(sm);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int j0 = blockIdx.x * BV;
+  const int h = blockIdx.y;
+  const int n = blockIdx.z;
+
+  const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
+  if (!sr.ok) return;
+
+  const uint32_t bar_full0 = sb + OFF2_BAR;
+  const uint32_t bar_mma = sb + OFF2_BAR + 16;
+  if (tid == 0) {
+    mbar_init(bar_full0, 1);
+    mbar_init(bar_full0 + 8, 1);
+    mbar_init(bar_mma, 1);
+    fence_mbar_init();
+    prefetch_tmap(&tm_wq);
+    prefetch_tmap(&tm_kh);
+    prefetch_tmap(&tm_uu);
+    prefetch_tmap(&tm_out);
+  }
+  if (warp == 0) {
+    tmem_alloc(sb + OFF2_TMEMPTR, kTmem2Cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF2_TMEMPTR);
+#ifdef CKDA_TC_DEBUG
+  long long tmark[16] = {0};
+  long long tlast = clock64();
+#endif
+
+  // State slice: row i = 32 * (warp % 4) + lane, columns [32 * (warp / 4), +32).
+  const int q4 = warp & 3;
+  const int half = warp >> 2;
+  const int srow = 32 * q4 + lane;
+  const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + 32 * half;
+  float S[32];
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (S0 != nullptr) v4 = *reinterpret_cast<const float4*>(S0 + s_off + e);
+    S[e] = v4.x; S[e + 1] = v4.y; S[e + 2] = v4.z; S[e + 3] = v4.w;
+  }
+#pragma unroll
+  for (int c4 = 0; c4 < 4; ++c4)
+    st_chunk8(sm + OFF2_SB, sw128_chunk(srow, 32 * half + 8 * c4, 128), S + 8 * c4);
+  fence_proxy_async_smem();
+
+  const int64_t tok0 = sr.begin;
+  const int64_t tok1 = sr.end;
+  const int nchunks = (int)((tok1 - tok0 + C - 1) / C);
+  const int64_t slot0 = slot_base(cu, n, nch);
+  auto unit_of = [&](int c) -> int64_t { return (slot0 + c) * H + h; };
+  // phase bits advance only on a successful wait (see the factor kernel)
+  uint32_t ph0 = 0, ph1 = 0, ph_mma = 0;
+  int pend0 = 0, pend1 = 0, pend_mma = 0;
+  int ok = 1;
+  auto wait = [&](uint32_t bar, uint32_t& phase, int& pending) -> bool {
+    const bool r = mbar_wait_bounded(bar, phase, kWaitNs);
+    if (r) {
+      phase ^= 1;
+      pending = 0;
+    }
+    return r;
+  };
+
+  auto issue = [&](int c, int st) {
+    const uint32_t bar = bar_full0 + 8 * st;
+    const uint32_t base = sb + st * kStageBytes;
+    const int64_t uidx = unit_of(c);
+    mbar_expect_tx(bar, kStageBytes);
+    tma_load_2d(base + CS_WQ, &tm_wq, 0, (int)(uidx * 2 * C), bar);
+    tma_load_2d(base + CS_WQ + 16384, &tm_wq, 64, (int)(uidx * 2 * C), bar);
+    tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), bar);
+    tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), bar);
+    tma_load_2d(base + CS_UU, &tm_uu, j0, (int)(uidx * 2 * C), bar);
+    tma_load_2d(base + CS_UU + 16384, &tm_uu, j0 + 32, (int)(uidx * 2 * C), bar);
+  };
+  if (tid == 0) {
+    if (nchunks > 0) issue(0, 0);
+    if (nchunks > 1) issue(1, 1);
+  }
+  pend0 = nchunks > 0;
+  pend1 = nchunks > 1;
+  float gm = (nchunks > 0) ? ws_g[unit_of(0) * DK + srow] : 1.f;
+  __syncthreads();
+
+  for (int c = 0; c < nchunks; ++c) {
+    const int st = c & 1;
+    const int64_t t0 = tok0 + (int64_t)c * C;
+    const int Lc = (tok1 - t0 < (int64_t)C) ? (int)(tok1 - t0) : C;
+    const uint32_t stage = sb + st * kStageBytes;
+    const bool tma_out = (cu == nullptr) || Lc == C;
+    ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
+    const float gm_next = (c + 1 < nchunks) ? ws_g[unit_of(c + 1) * DK + srow] : 1.f;
+    TC_MARK(9);
 
     // ---- carry 1: X = [W; Q'] S ---------------------------------------------------
     if (tid == 0) {
@@ -893,46 +1203,76 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint64_t ad =
-            smem_desc(sb + OFF_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF_SB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM_X, ad, bd, id, kk > 0 ? 1u : 0u);
+            smem_desc(stage + CS_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(sb + OFF2_SB + kk * 2048, 8192, 1024, kSwizzle128);
+        mma_f16(tmem + TM2_X, ad, bd, id, kk > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
     }
-    ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
-    ph_mma ^= 1;
+    pend_mma = 1;
+    ok = wait(bar_mma, ph_mma, pend_mma);
+    // the previous chunk's output store must have read its staging
+    if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    TC_MARK(9);
+    TC_MARK(10);
 
     // ---- U = U~ - X_top -> operand;  O = A U~ + X_bottom -> out ------------------
     {
       float a[32], x[32];
-      tmem_ld32(taddr(tmem, 32 * q4, TM_U + 32 * half), a);
-      tmem_ld32(taddr(tmem, 32 * q4, TM_X + 32 * half), x);
+      tmem_ld32(taddr(tmem, 32 * q4, TM2_X + 32 * half), x);
+      const uint32_t arow = stage + CS_UU + 16384 * half + 128 * srow;
+#pragma unroll
+      for (int c4 = 0; c4 < 8; ++c4) {
+        const float4 f = lds_f4(arow + ((c4 ^ (srow & 7)) << 4));
+        a[4 * c4] = f.x; a[4 * c4 + 1] = f.y; a[4 * c4 + 2] = f.z; a[4 * c4 + 3] = f.w;
+      }
       tmem_ld_wait();
       TC_DBG(for (int e = 0; e < 32; ++e) {
-        g_tc_dbg[32768 + (32 * q4 + lane) * 64 + 32 * half + e] = a[e];
-        g_tc_dbg[40960 + (32 * q4 + lane) * 64 + 32 * half + e] = x[e];
+        g_tc_dbg[32768 + srow * 64 + 32 * half + e] = a[e];
+        g_tc_dbg[40960 + srow * 64 + 32 * half + e] = x[e];
       });
       if (q4 < 2) {
-        const int r = 32 * q4 + lane;
-        float u[32];
+        float uv[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) u[e] = a[e] - x[e];
+        for (int e = 0; e < 32; ++e) uv[e] = a[e] - x[e];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
-          st_chunk8(sm + OFF_UB, sw128_chunk(r, 32 * half + 8 * c4, 64), u + 8 * c4);
+          st_chunk8(sm + OFF2_UB, sw128_chunk(srow, 32 * half + 8 * c4, 64), uv + 8 * c4);
       } else {
-        const int r = 32 * (q4 - 2) + lane;
-        if (r < Lc) store_row32<Tout>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + 32 * half, a, x);
+        const int r = srow - 64;
+        if (tma_out)
+          stage_row32<Tout>(sb + OFF2_OB, r, half, a, x);
+        else if (r < Lc)
+          store_row32<Tout>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + 32 * half, a, x);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    TC_MARK(10);
+    if (tma_out && tid == 0) {
+      // fixed-length batch: [T, H * d_v] per sequence, rows past T are clipped;
+      // packed batch: only whole chunks go through TMA
+      const int x0 = h * DV + j0;
+      if (cu == nullptr) {
+        if (sizeof(Tout) == 4) {
+          tma_store_3d(&tm_out, sb + OFF2_OB, x0, c * C, n);
+          tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, c * C, n);
+        } else {
+          tma_store_3d(&tm_out, sb + OFF2_OB, x0, c * C, n);
+        }
+      } else {
+        if (sizeof(Tout) == 4) {
+          tma_store_2d(&tm_out, sb + OFF2_OB, x0, (int)t0);
+          tma_store_2d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, (int)t0);
+        } else {
+          tma_store_2d(&tm_out, sb + OFF2_OB, x0, (int)t0);
+        }
+      }
+      bulk_commit();
+    }
+    TC_MARK(11);
 
     // ---- carry 2: D = (K rho)^T U;  S <- Diag(gamma) S + D ----------------------
     if (tid == 0) {
@@ -940,22 +1280,29 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       constexpr uint32_t id = idesc_f16(128, 64, 1, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(sb + OFF_KH + kk * 2048, 8192, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF_UB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM_D, ad, bd, id, kk > 0 ? 1u : 0u);
+        const uint64_t ad = smem_desc(stage + CS_KH + kk * 2048, 8192, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(sb + OFF2_UB + kk * 2048, 8192, 1024, kSwizzle128);
+        mma_f16(tmem + TM2_D, ad, bd, id, kk > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
     }
-    ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
-    ph_mma ^= 1;
+    pend_mma = 1;
+    ok = wait(bar_mma, ph_mma, pend_mma);
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
+    // this stage is consumed: fetch chunk c + 2 into it
+    if (c + 2 < nchunks) {
+      if (tid == 0) issue(c + 2, st);
+      if (st)
+        pend1 = 1;
+      else
+        pend0 = 1;
+    }
     {
       float d[32];
-      tmem_ld32(taddr(tmem, 32 * q4, TM_D + 32 * half), d);
+      tmem_ld32(taddr(tmem, 32 * q4, TM2_D + 32 * half), d);
       tmem_ld_wait();
-      const float gm = gamma_s[srow];
 #pragma unroll
       for (int e = 0; e < 32; ++e) S[e] = fmaf(gm, S[e], d[e]);
       TC_DBG(for (int e = 0; e < 32; ++e) {
@@ -964,17 +1311,19 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       });
 #pragma unroll
       for (int c4 = 0; c4 < 4; ++c4)
-        st_chunk8(sm + OFF_SB, sw128_chunk(srow, 32 * half + 8 * c4, 128), S + 8 * c4);
+        st_chunk8(sm + OFF2_SB, sw128_chunk(srow, 32 * half + 8 * c4, 128), S + 8 * c4);
     }
+    gm = gm_next;
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    TC_MARK(11);
+    TC_MARK(12);
   }
 #ifdef CKDA_TC_DEBUG
   if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-    for (int k = 0; k < 16; ++k) g_tc_time[k] = tmark[k];
+    for (int k = 9; k < 13; ++k) g_tc_time[k] = tmark[k];
 #endif
+  if (tid == 0) bulk_wait_all();
 
   if (ok) {
     if (S_final != nullptr) {
@@ -985,16 +1334,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   } else {
     if (tid == 0) {
       set_status(status, CKDA_ERR_DEVICE_TIMEOUT);
-      // wait (bounded) for copies and tensor-core work this CTA still has in flight
-      if (pend_in0) mbar_wait_bounded(bar_in0, ph_in0, kWaitNs);
-      if (pend_in1) mbar_wait_bounded(bar_in1, ph_in1, kWaitNs);
-      if (pend_v) mbar_wait_bounded(bar_v, ph_v, kWaitNs);
-      mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
+      if (pend0) mbar_wait_bounded(bar_full0, ph0, kWaitNs);
+      if (pend1) mbar_wait_bounded(bar_full0 + 8, ph1, kWaitNs);
+      if (pend_mma) mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, kTmem2Cols);
 }
 
 // ---- host side ------------------------------------------------------------------
@@ -1028,57 +1375,169 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, size_t es
   return r == CUDA_SUCCESS;
 }
 
-template <typename Tout>
-cudaError_t launch_t(const void* q, const void* k, const void* v, const float* alpha,
+bool make_map3(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, size_t esize,
+               uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1,
+               CUtensorMapSwizzle swz) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {d0 * esize, d0 * d1 * esize};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Work units of a call (at least one, so the workspace maps are never empty).
+int64_t n_units(bool varlen, int n_seqs, int T, int H) {
+  const int64_t nch = ((int64_t)T + C - 1) / C;
+  const int64_t slots = varlen ? (int64_t)T / C + n_seqs : (int64_t)n_seqs * nch;
+  const int64_t u = slots * H;
+  return u > 0 ? u : 1;
+}
+
+size_t unit_bytes(int DV) { return kWsWQ + kWsKH + kWsG + (size_t)2 * C * DV * 4; }
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    return 148;
+  return n;
+}
+
+template <typename K>
+cudaError_t set_smem(K kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// phases: kFactors runs kernel 1 (inputs -> workspace), kCarry kernel 2
+// (workspace, S0 -> out, S_final); a full forward runs both, in order, on
+// `stream`.
+constexpr int kFactors = 1, kCarry = 2;
+
+template <int DV, typename Tout>
+cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, const float* S0, const int32_t* cu, void* out,
-                     float* S_final, int n_seqs, int T, int H, int DV, int* status,
+                     float* S_final, int n_seqs, int T, int H, void* ws, int* status,
                      cudaStream_t stream) {
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
-  CUtensorMap mq, mk, mv, ma;
-  const bool ok = make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows,
-                           HC, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                  make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows,
-                           HC, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
-                  make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows,
-                           BV, C, CU_TENSOR_MAP_SWIZZLE_128B) &&
-                  make_map(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)H * DK,
-                           rows, HC, C, CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (!ok) return cudaErrorInvalidValue;
-  auto kern = fwd_tc_kernel<Tout>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  const int nch = (int)(((int64_t)T + C - 1) / C);
+  const int64_t nu = n_units(cu != nullptr, n_seqs, T, H);
+  // workspace arrays, in this order: [W; Q'], K rho, [U~; A U~], gamma
+  uint8_t* w8 = static_cast<uint8_t*>(ws);
+  __half* ws_wq = reinterpret_cast<__half*>(w8);
+  __half* ws_kh = reinterpret_cast<__half*>(w8 + nu * kWsWQ);
+  float* ws_uu = reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH));
+  float* ws_g = reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH + (size_t)2 * C * DV * 4));
+
+  CUtensorMap mkh, muu;
+  if (!make_map(&mkh, ws_kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * C, 64, C,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&muu, ws_uu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DV, (uint64_t)nu * 2 * C, 32,
+                2 * C, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+
+  if (phases & kFactors) {
+    CUtensorMap mq, mk, mv, ma, mwq64;
+    const bool ok =
+        make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HC, C,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HC, C,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows, 64, C,
+                 CU_TENSOR_MAP_SWIZZLE_128B) &&
+        make_map(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)H * DK, rows, HC, C,
+                 CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        make_map(&mwq64, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
+                 C, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    auto k1 = factor_kernel<DV>;
+    static bool attr1 = false;
+    if (!attr1) {
+      cudaError_t e = set_smem(k1, kSmemBytes);
+      if (e != cudaSuccess) return e;
+      attr1 = true;
+    }
+    const int64_t g1 = nu < (int64_t)sm_count() ? nu : (int64_t)sm_count();
+    k1<<<(unsigned)g1, NT, kSmemBytes, stream>>>(mq, mk, mv, ma, mwq64, mkh, muu, beta, cu,
+                                                 n_seqs, T, H, nch, nu, ws_g, status);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
-  dim3 grid(DV / BV, H, n_seqs);
-  kern<<<grid, NT, kSmemBytes, stream>>>(mq, mk, mv, ma, beta, S0, cu, static_cast<Tout*>(out),
-                                         S_final, n_seqs, T, H, DV, status);
-  return cudaGetLastError();
+
+  if (phases & kCarry) {
+    constexpr bool kF32 = sizeof(Tout) == 4;
+    const CUtensorMapDataType tout =
+        kF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint32_t ob_cols = kF32 ? 32 : 64;
+    CUtensorMap mwq, mout;
+    const bool ok =
+        make_map(&mwq, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
+                 2 * C, CU_TENSOR_MAP_SWIZZLE_128B) &&
+        (cu ? make_map(&mout, out, tout, sizeof(Tout), (uint64_t)H * DV, rows, ob_cols, C,
+                       CU_TENSOR_MAP_SWIZZLE_128B)
+            : make_map3(&mout, out, tout, sizeof(Tout), (uint64_t)H * DV, (uint64_t)T,
+                        (uint64_t)n_seqs, ob_cols, C, CU_TENSOR_MAP_SWIZZLE_128B));
+    if (!ok) return cudaErrorInvalidValue;
+    auto k2 = carry_kernel<Tout>;
+    static bool attr2 = false;
+    if (!attr2) {
+      cudaError_t e = set_smem(k2, kSmem2Bytes);
+      if (e != cudaSuccess) return e;
+      attr2 = true;
+    }
+    dim3 grid(DV / BV, H, n_seqs);
+    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, muu, mout, ws_g, S0, cu,
+                                          static_cast<Tout*>(out), S_final, n_seqs, T, H, DV,
+                                          nch, status);
+    return cudaGetLastError();
+  }
+  return cudaSuccess;
 }
 
 }  // namespace tc
 
-// Shapes covered by the tensor-core kernel (`rows` = packed or B*T tokens).
-bool fwd_tc_supported(int dtype, int dk, int dv, int C, uint64_t rows) {
-  return dtype == CKDA_BF16 && dk == tc::DK && (dv == 64 || dv == 128) && C == tc::C &&
-         rows > 0 && rows <= 0x7fffffffull;
+// Shapes covered by the tensor-core kernels: bf16 inputs, d_k = 128,
+// d_v in {64, 128}, chunk 64, and every TMA row coordinate (token rows and
+// workspace rows, 2 C per unit) within int32.
+bool fwd_tc_supported(int dtype, int dk, int dv, int C, int n_seqs, int T, int H, bool varlen) {
+  const uint64_t rows = varlen ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
+  if (dtype != CKDA_BF16 || dk != tc::DK || (dv != 64 && dv != 128) || C != tc::C) return false;
+  if (n_seqs <= 0 || H <= 0 || rows == 0 || rows > 0x7fffffffull) return false;
+  return (uint64_t)tc::n_units(varlen, n_seqs, T, H) * 2 * tc::C <= 0x7fffffffull;
 }
 
-// Everything the tensor-core kernel does not cover returns
+// Workspace bytes the tensor-core path needs (0 when it does not apply).
+size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int T, int H,
+                              bool varlen) {
+  if (!fwd_tc_supported(dtype, dk, dv, C, n_seqs, T, H, varlen)) return 0;
+  const int64_t nu = tc::n_units(varlen, n_seqs, T, H);
+  return (size_t)nu * tc::unit_bytes(dv);
+}
+
+// Everything the tensor-core kernels do not cover returns
 // cudaErrorNotSupported so the caller can use the CUDA-core kernel.
-cudaError_t launch_fwd_tc(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k,
-                          const void* v, const float* alpha, const float* beta, const float* S0,
-                          const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
-                          int C, int* status, cudaStream_t stream) {
-  const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
-  if (!fwd_tc_supported(dtype, dk, dv, C, rows)) return cudaErrorNotSupported;
-  if (out_dtype == CKDA_BF16)
-    return tc::launch_t<__nv_bfloat16>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H,
-                                       dv, status, stream);
-  return tc::launch_t<float>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, dv, status,
-                             stream);
+// `phases`: 1 = factors only, 2 = carry only, 3 = the whole forward.
+cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
+                          const void* k, const void* v, const float* alpha, const float* beta,
+                          const float* S0, const int32_t* cu, void* out, float* S_final,
+                          int n_seqs, int T, int H, int C, void* ws, int* status,
+                          cudaStream_t stream) {
+  if (!fwd_tc_supported(dtype, dk, dv, C, n_seqs, T, H, cu != nullptr))
+    return cudaErrorNotSupported;
+  const bool bf = out_dtype == CKDA_BF16;
+  if (dv == 128)
+    return bf ? tc::launch_t<128, __nv_bfloat16>(phases, q, k, v, alpha, beta, S0, cu, out,
+                                                 S_final, n_seqs, T, H, ws, status, stream)
+              : tc::launch_t<128, float>(phases, q, k, v, alpha, beta, S0, cu, out, S_final,
+                                         n_seqs, T, H, ws, status, stream);
+  return bf ? tc::launch_t<64, __nv_bfloat16>(phases, q, k, v, alpha, beta, S0, cu, out, S_final,
+                                              n_seqs, T, H, ws, status, stream)
+            : tc::launch_t<64, float>(phases, q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs,
+                                      T, H, ws, status, stream);
 }
 
 }  // namespace ckda

@@ -20,8 +20,9 @@
  * ---------------------------------------
  *  - All tensor pointers are DEVICE pointers (cudaMalloc / torch CUDA
  *    memory) on the current CUDA device, row-major and contiguous, 16-byte
- *    aligned.  The caller owns every buffer; the library allocates nothing
- *    and keeps no state between calls except one device status word.
+ *    aligned.  The caller owns every buffer, scratch workspace included;
+ *    the library allocates nothing and keeps no state between calls except
+ *    one device status word.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call is asynchronous on that stream and returns as soon
  *    as the work is enqueued.
@@ -40,6 +41,7 @@
 #ifndef CKDA_H
 #define CKDA_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 /* Symbols of the C ABI are exported even when the library is compiled with
@@ -69,7 +71,10 @@ enum {
   CKDA_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned */
   CKDA_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
   CKDA_ERR_DEVICE_TIMEOUT = -5,/* a bounded device-side wait gave up */
-  CKDA_ERR_BAD_SEQLENS = -6    /* cu_seqlens not 0 = cu[0] <= ... <= cu[N] = T */
+  CKDA_ERR_BAD_SEQLENS = -6,   /* cu_seqlens not 0 = cu[0] <= ... <= cu[N] = T */
+  CKDA_ERR_WORKSPACE = -7      /* workspace NULL, smaller than
+                                  ckda_fwd_chunked_workspace_bytes(), not
+                                  256-byte aligned, or overlapping a tensor */
 };
 
 /*
@@ -104,13 +109,75 @@ enum {
  *   out      must not alias any input.
  *   chunk    0 (default 64), 16, 32 or 64.
  *   d_k, d_v each in {16, 32, 64, 128}.
+ *   workspace, workspace_bytes
+ *            device scratch owned by the caller, at least
+ *            ckda_fwd_chunked_workspace_bytes() bytes for these sizes,
+ *            256-byte aligned, overlapping no tensor argument; its contents
+ *            on entry do not matter and on return are unspecified.  Only
+ *            the tensor-core path uses it (per chunk and head: the WY
+ *            factors [W; Q'] and K * rho in fp16, [U~; A U~] and gamma in
+ *            fp32, about 115 KB at d_v = 128); when the size query returns 0
+ *            both may be NULL / 0.  Calls that run concurrently (other
+ *            streams) need separate workspaces; calls ordered on one stream
+ *            may share one.  A workspace that is missing or too small
+ *            returns CKDA_ERR_WORKSPACE and launches nothing.
  * A zero-length sequence stores S_final = S0 and writes no output rows.
  */
 CKDA_API int ckda_fwd_chunked(const void* q, const void* k, const void* v,
                      const float* alpha, const float* beta, const float* S0,
                      const int32_t* cu_seqlens, void* out, float* S_final,
                      int B, int T, int H, int d_k, int d_v, int chunk,
-                     int dtype, int out_dtype, void* stream);
+                     int dtype, int out_dtype, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
+ * ckda_fwd_factors, ckda_fwd_carry -- ckda_fwd_chunked in its two phases,
+ * for the tensor-core path only (sizes for which ckda_fwd_chunked_path
+ * returns 1; otherwise CKDA_ERR_UNSUPPORTED).
+ *
+ * ckda_fwd_factors reads q, k, v, alpha and beta (layouts as in
+ * ckda_fwd_chunked) and writes, for every chunk of every head, the
+ * S0-independent WY factors into `workspace`: [W; Q'] and K * rho (fp16),
+ * [U~; A U~] and gamma (fp32) ("Gated DeltaNet-2", Methodology section 3:
+ * the decay absorbed into the WY factors; "Semidirect Fourier Delta
+ * Attention", "Principales Contribuciones" item 3: each chunk is an affine
+ * map of the state, S_end = (Diag(gamma) - (K*rho)^T W) S + (K*rho)^T U~).
+ * ckda_fwd_carry applies those maps chunk after chunk from S0 and writes
+ * out and S_final.
+ *
+ * Because the factors do not depend on S0, one factor call can serve
+ * several carry calls with different initial states.  ckda_fwd_carry must
+ * see the workspace of a completed ckda_fwd_factors call with the same B,
+ * T, H, d_k, d_v, chunk, dtype and cu_seqlens (stream order or an event
+ * makes it complete); the library cannot check this.  Running the two on
+ * one stream equals one ckda_fwd_chunked call, bit for bit.  Arguments,
+ * ownership and errors are those of ckda_fwd_chunked; out_dtype is only
+ * meaningful to the carry.
+ */
+CKDA_API int ckda_fwd_factors(const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta,
+                              const int32_t* cu_seqlens, int B, int T, int H,
+                              int d_k, int d_v, int chunk, int dtype,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+CKDA_API int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* out,
+                            float* S_final, int B, int T, int H, int d_k, int d_v,
+                            int chunk, int dtype, int out_dtype, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * ckda_fwd_chunked_workspace_bytes -- scratch bytes ckda_fwd_chunked needs
+ * for these sizes (same meaning of B, T and `varlen` as in
+ * ckda_fwd_chunked_path), 0 when the call runs the fp32 CUDA-core kernel,
+ * or the negative status an actual call with these sizes would return.
+ * Pure host function: needs no GPU.  The tensor-core path takes
+ * (B * ceil(T / 64)) * H work units for a fixed-length batch and
+ * (floor(T / 64) + N) * H for a packed one, each 2*64*128*2 + 64*128*2 +
+ * 128*4 + 2*64*d_v*4 bytes.
+ */
+CKDA_API int64_t ckda_fwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v,
+                                                  int chunk, int dtype, int out_dtype,
+                                                  int varlen);
 
 /*
  * ckda_fwd_chunked_fp32core -- the same operation and arguments as
@@ -130,8 +197,10 @@ CKDA_API int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void*
 /*
  * ckda_fwd_chunked_path -- which kernel ckda_fwd_chunked runs for these
  * parameters, without launching anything: 1 = the tcgen05 tensor-core
- * kernel (bf16 inputs, d_k = 128, d_v in {64, 128}, chunk 64; fp16 operands
- * with fp32 accumulation), 0 = the fp32 CUDA-core kernel, or the negative
+ * kernels (bf16 inputs, d_k = 128, d_v in {64, 128}, chunk 64; fp16 operands
+ * with fp32 accumulation; a per-chunk factor kernel over all chunks in
+ * parallel, then a carry kernel per sequence, head and 64 columns of d_v),
+ * 0 = the fp32 CUDA-core kernel, or the negative
  * status an actual call with these sizes would return.  `varlen` is nonzero
  * for a packed batch (cu_seqlens given); B and T have the same meaning as in
  * ckda_fwd_chunked.  Pure host function: needs no GPU.

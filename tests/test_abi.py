@@ -35,7 +35,8 @@ def declared_symbols():
 
 def test_header_declares_entry_points():
     names = declared_symbols()
-    for required in ("ckda_fwd_chunked", "ckda_decode_step", "ckda_status_string",
+    for required in ("ckda_fwd_chunked", "ckda_fwd_chunked_workspace_bytes", "ckda_fwd_factors",
+                     "ckda_fwd_carry", "ckda_decode_step", "ckda_status_string",
                      "ckda_device_status"):
         assert required in names
 
@@ -60,7 +61,7 @@ def test_library_has_no_runtime_dependency_on_libcudart():
 
 
 def test_status_strings(lib):
-    for code in (0, -1, -2, -3, -4, -5, -6):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         s = lib.ckda_status_string(code)
         assert s and b"unknown" not in s
     assert lib.ckda_status_string(-99) == b"unknown status"
@@ -76,11 +77,12 @@ MIS = (1 << 20) + 4  # misaligned
 def fwd(lib, **kw):
     a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000, S0=None,
              cu=None, out=P + 0x5000, S_final=None, B=1, T=8, H=1, dk=16, dv=16, chunk=16,
-             dtype=0, out_dtype=0, stream=None)
+             dtype=0, out_dtype=0, ws=None, ws_bytes=0, stream=None)
     a.update(kw)
     return lib.ckda_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S0"], a["cu"],
                                 a["out"], a["S_final"], a["B"], a["T"], a["H"], a["dk"], a["dv"],
-                                a["chunk"], a["dtype"], a["out_dtype"], a["stream"])
+                                a["chunk"], a["dtype"], a["out_dtype"], a["ws"], a["ws_bytes"],
+                                a["stream"])
 
 
 def test_fwd_argument_errors(lib):
@@ -150,3 +152,74 @@ def test_path_query_needs_no_gpu(lib):
 def test_selftest_rejects_bad_limits(lib):
     assert lib.ckda_selftest_bounded_wait(0, None) == -1
     assert lib.ckda_selftest_bounded_wait(20000000, None) == -1
+
+
+UNIT_BYTES_DV128 = 2 * 64 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 2 * 64 * 128 * 4
+
+
+def test_workspace_size_query_needs_no_gpu(lib):
+    F32, BF16 = 0, 1
+    q = lib.ckda_fwd_chunked_workspace_bytes
+    # fixed-length: B * ceil(T / 64) * H units
+    assert q(4, 4096, 16, 128, 128, 64, BF16, F32, 0) == 4 * 64 * 16 * UNIT_BYTES_DV128
+    assert q(2, 100, 3, 128, 128, 64, BF16, F32, 0) == 2 * 2 * 3 * UNIT_BYTES_DV128
+    assert q(1, 64, 1, 128, 64, 0, BF16, BF16, 0) == 2 * 64 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 2 * 64 * 64 * 4
+    # packed: (floor(T / 64) + N) * H units
+    assert q(5, 1000, 2, 128, 128, 64, BF16, F32, 1) == (1000 // 64 + 5) * 2 * UNIT_BYTES_DV128
+    # the CUDA-core path needs none
+    assert q(4, 4096, 16, 128, 128, 64, F32, F32, 0) == 0
+    assert q(4, 4096, 16, 64, 64, 64, BF16, F32, 0) == 0
+    assert q(4, 4096, 16, 128, 128, 32, BF16, F32, 0) == 0
+    # and argument errors come back as the call's status
+    assert q(4, 4096, 0, 128, 128, 64, BF16, F32, 0) == -1
+    assert q(4, 4096, 16, 128, 256, 64, BF16, F32, 0) == -2
+
+
+def test_workspace_errors_launch_nothing(lib):
+    tc = dict(dtype=1, out_dtype=0, dk=128, dv=128, chunk=64, T=128, B=1, H=1)
+    need = lib.ckda_fwd_chunked_workspace_bytes(1, 128, 1, 128, 128, 64, 1, 0, 0)
+    assert need == 2 * UNIT_BYTES_DV128
+    WS = 1 << 32  # 256-byte aligned, never dereferenced
+    assert fwd(lib, **tc) == -7                                   # missing
+    assert fwd(lib, ws=WS, ws_bytes=need - 1, **tc) == -7         # too small
+    assert fwd(lib, ws=WS + 16, ws_bytes=need, **tc) == -7        # not 256-byte aligned
+    assert fwd(lib, ws=P, ws_bytes=need, **tc) == -7              # overlaps q
+    # argument errors are reported before the workspace
+    assert fwd(lib, q=None, **tc) == -1
+
+
+def test_two_phase_calls_validate_without_a_gpu(lib):
+    F32, BF16 = 0, 1
+    WS = 1 << 32
+    need = lib.ckda_fwd_chunked_workspace_bytes(1, 128, 1, 128, 128, 64, BF16, F32, 0)
+
+    def factors(**kw):
+        a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000, cu=None,
+                 B=1, T=128, H=1, dk=128, dv=128, chunk=64, dtype=BF16, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.ckda_fwd_factors(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["cu"], a["B"],
+                                    a["T"], a["H"], a["dk"], a["dv"], a["chunk"], a["dtype"],
+                                    a["ws"], a["ws_bytes"], None)
+
+    def carry(**kw):
+        a = dict(S0=None, cu=None, out=P + 0x5000, S_final=None, B=1, T=128, H=1, dk=128, dv=128,
+                 chunk=64, dtype=BF16, out_dtype=F32, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.ckda_fwd_carry(a["S0"], a["cu"], a["out"], a["S_final"], a["B"], a["T"], a["H"],
+                                  a["dk"], a["dv"], a["chunk"], a["dtype"], a["out_dtype"], a["ws"],
+                                  a["ws_bytes"], None)
+
+    # the two phases exist only on the tensor-core path
+    assert factors(dtype=F32) == -2
+    assert factors(dk=64) == -2
+    assert carry(chunk=32) == -2
+    # each phase needs only its own tensors, and the workspace
+    assert factors(q=None) == -1
+    assert carry(out=None) == -1
+    assert factors() == -7
+    assert carry() == -7
+    assert factors(ws=WS, ws_bytes=need - 256) == -7
+    assert carry(ws=WS + 64, ws_bytes=need) == -7
+    # nothing to do for an empty batch
+    assert factors(B=0) == 0
+    assert carry(B=0) == 0
