@@ -13,6 +13,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libckda.so"
 
 CKDA_F32 = 0
 CKDA_BF16 = 1
+# capacity of the library's static device scratch (ckda_fwd_chunked_static)
+CKDA_STATIC_SCRATCH_BYTES = 64 * 1024 * 1024
 
 STATUS = {
     0: "CKDA_OK",
@@ -32,6 +34,8 @@ SIGNATURES = {
     "ckda_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
                               _vp, ctypes.c_size_t, _vp]),
     "ckda_fwd_chunked_workspace_bytes": (ctypes.c_int64, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ckda_fwd_chunked_static": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+                                     _i, _i, _i, _vp]),
     "ckda_fwd_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
                               ctypes.c_size_t, _vp]),
     "ckda_fwd_carry": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,

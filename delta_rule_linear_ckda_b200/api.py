@@ -94,6 +94,40 @@ def fwd_chunked(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
     return out, S_final
 
 
+def fwd_chunked_static(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: int = 64,
+                       out=None, S_final=None, return_final: bool = True, out_dtype=None):
+    """``fwd_chunked`` through ``ckda_fwd_chunked_static``: no workspace is passed or
+    allocated; the library's fixed device scratch (``CKDA_STATIC_SCRATCH_BYTES``)
+    is used.  Calls that may run concurrently on one device race on that scratch."""
+    dev = q.device
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, cu_seqlens)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must have v's shape")
+    if return_final and S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_fwd_chunked_static(
+            _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(out),
+            _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype], _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_fwd_chunked_static")
+    return out, S_final
+
+
 def _inputs_shape(q, k, v, alpha, beta, cu_seqlens):
     """Checks the forward inputs; returns (B, T, H, dk, dv, N) as passed to the ABI."""
     dev = q.device

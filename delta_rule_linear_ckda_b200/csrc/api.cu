@@ -33,6 +33,10 @@ cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
 // First device-side error since the last ckda_device_status() call.
 __device__ int g_ckda_status = 0;
 
+// Scratch of ckda_fwd_chunked_static: one fixed array per device, allocated
+// with the module, never by a call.  Nothing in it needs to start at zero.
+static __device__ __align__(256) uint8_t g_ckda_scratch[CKDA_STATIC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -49,6 +53,22 @@ int* status_ptr() {
     if (cudaGetSymbolAddress(&addr, g_ckda_status) != cudaSuccess) return nullptr;
     p = static_cast<int*>(addr);
     g_status_ptr[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
+
+std::atomic<void*> g_scratch_ptr[kMaxDevices];
+
+// Device address of the static scratch on the current device, looked up
+// once per device (the first call on a device must not be inside a stream
+// capture: the lookup is not a stream operation).
+void* scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    if (cudaGetSymbolAddress(&p, g_ckda_scratch) != cudaSuccess) return nullptr;
+    g_scratch_ptr[dev].store(p, std::memory_order_release);
   }
   return p;
 }
@@ -159,6 +179,24 @@ int ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* a
                      int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
   return fwd_impl(true, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
                   d_v, chunk, dtype, out_dtype, workspace, workspace_bytes, stream);
+}
+
+int ckda_fwd_chunked_static(const void* q, const void* k, const void* v, const float* alpha,
+                            const float* beta, const float* S0, const int32_t* cu_seqlens,
+                            void* out, float* S_final, int B, int T, int H, int d_k, int d_v,
+                            int chunk, int dtype, int out_dtype, void* stream) {
+  int rc = validate_fwd(q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
+                        &chunk, dtype, out_dtype);
+  if (rc != CKDA_OK) return rc;
+  const size_t need =
+      B > 0 ? ckda::fwd_tc_workspace_bytes(dtype, d_k, d_v, chunk, B, T, H, cu_seqlens != nullptr)
+            : 0;
+  if (need > (size_t)CKDA_STATIC_SCRATCH_BYTES) return CKDA_ERR_UNSUPPORTED;
+  void* ws = nullptr;
+  if (need > 0 && (ws = scratch_ptr()) == nullptr) return CKDA_ERR_CUDA;
+  return fwd_impl(true, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
+                  d_v, chunk, dtype, out_dtype, ws, need > 0 ? (size_t)CKDA_STATIC_SCRATCH_BYTES : 0,
+                  stream);
 }
 
 int ckda_fwd_factors(const void* q, const void* k, const void* v, const float* alpha,

@@ -131,6 +131,41 @@ CKDA_API int ckda_fwd_chunked(const void* q, const void* k, const void* v,
                      size_t workspace_bytes, void* stream);
 
 /*
+ * ckda_fwd_chunked_static -- ckda_fwd_chunked without a caller workspace:
+ * the tensor-core path uses a fixed scratch array that the library holds in
+ * device memory (CKDA_STATIC_SCRATCH_BYTES per device, reserved when the
+ * library's module is loaded).  No call allocates or frees memory.  This
+ * entry point is an interface convenience of this library; the pages
+ * describe no counterpart of it.
+ *
+ *  - Arguments, layouts and results are those of ckda_fwd_chunked; the
+ *    output is bit-identical to ckda_fwd_chunked with any valid workspace.
+ *  - Sizes whose workspace (ckda_fwd_chunked_workspace_bytes) exceeds
+ *    CKDA_STATIC_SCRATCH_BYTES return CKDA_ERR_UNSUPPORTED and launch
+ *    nothing: at d_v = 128 that is more than 582 units of
+ *    ceil(T / 64) * B * H (fixed-length) or (floor(T / 64) + N) * H
+ *    (packed), e.g. B = 1, T = 2048, H = 16 fits (512 units).  Sizes on the
+ *    fp32 CUDA-core path need no scratch and are always accepted.
+ *  - Nothing in the scratch has to start at zero: every byte the carry
+ *    kernel reads is written by the factor kernel of the same call.
+ *  - The scratch is shared by every call on a device: two calls that may
+ *    run at the same time (different streams, or threads without stream
+ *    order) race on it and give wrong results.  Calls ordered on one stream
+ *    are safe.
+ *  - The first call on each device looks the scratch address up with
+ *    cudaGetSymbolAddress and caches it; make that first call outside any
+ *    stream capture.
+ */
+#define CKDA_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+CKDA_API int ckda_fwd_chunked_static(const void* q, const void* k, const void* v,
+                                     const float* alpha, const float* beta,
+                                     const float* S0, const int32_t* cu_seqlens,
+                                     void* out, float* S_final, int B, int T, int H,
+                                     int d_k, int d_v, int chunk, int dtype,
+                                     int out_dtype, void* stream);
+
+/*
  * ckda_fwd_factors, ckda_fwd_carry -- ckda_fwd_chunked in its two phases,
  * for the tensor-core path only (sizes for which ckda_fwd_chunked_path
  * returns 1; otherwise CKDA_ERR_UNSUPPORTED).

@@ -223,3 +223,21 @@ def test_two_phase_calls_validate_without_a_gpu(lib):
     # nothing to do for an empty batch
     assert factors(B=0) == 0
     assert carry(B=0) == 0
+
+
+def test_static_scratch_entry_rejects_oversized_calls_without_a_gpu(lib):
+    from delta_rule_linear_ckda_b200._lib import CKDA_STATIC_SCRATCH_BYTES
+
+    F32, BF16 = 0, 1
+    # 4 x 64 x 16 units at d_v = 128 need 472 MB > the 64 MiB scratch
+    assert lib.ckda_fwd_chunked_workspace_bytes(4, 4096, 16, 128, 128, 64, BF16, F32, 0) > \
+        CKDA_STATIC_SCRATCH_BYTES
+    r = lib.ckda_fwd_chunked_static(P, P + 0x1000, P + 0x2000, P + 0x3000, P + 0x4000, None, None,
+                                    P + 0x5000, None, 4, 4096, 16, 128, 128, 64, BF16, F32, None)
+    assert r == -2
+    # argument errors come first, as in ckda_fwd_chunked
+    r = lib.ckda_fwd_chunked_static(None, P, P, P, P, None, None, P + 0x5000, None, 1, 64, 1, 128,
+                                    128, 64, BF16, F32, None)
+    assert r == -1
+    assert lib.ckda_fwd_chunked_static(P, P, P, P, P, None, None, P + 0x5000, None, 0, 64, 1, 128,
+                                       128, 64, BF16, F32, None) == 0
