@@ -65,14 +65,16 @@ constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int HC = 64;  // channels per half of d_k
 constexpr int BV = 64;  // d_v columns of one carry CTA
-constexpr int NT = 256;
+constexpr int NT = 256;   // carry kernel threads
+constexpr int NT1 = 512;  // factor kernel threads
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
-// ---- workspace: per unit (one chunk of one head), four arrays -------------
-constexpr size_t kWsWQ = (size_t)2 * C * DK * 2;  // [W; Q'] fp16 [128][128]
+// ---- workspace: per unit (one chunk of one head), five arrays -------------
+constexpr size_t kWsWQ = (size_t)2 * C * DK * 2;  // [-W; Q'] fp16 [128][128]
 constexpr size_t kWsKH = (size_t)C * DK * 2;      // K * rho fp16 [64][128]
+constexpr size_t kWsIP = (size_t)2 * C * C * 2;   // [Inv diag(beta); P] fp16 [128][64]
 constexpr size_t kWsG = (size_t)DK * 4;           // gamma fp32 [128]
-// [U~; A U~] fp32 [128][d_v]: 2 * C * d_v * 4 bytes
+// V as fp16 [64][d_v]: C * d_v * 2 bytes
 
 // ---- factor kernel: shared memory map (byte offsets, 1024-aligned base) ---
 // Two input buffers, one per 64-channel half: q, k (bf16 [64 pos][64 ch])
@@ -90,41 +92,41 @@ constexpr uint32_t OFF_LVX = 81920;
 // operand [levels a; b] (128 rows) and the right operand (64 rows).
 constexpr uint32_t kPairBytes = 24576;
 constexpr uint32_t PAIR_ROP = 16384;
-constexpr uint32_t OFF_TF = OFF_LVX;          // T, fp32 [64][64]
-constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A staging then (I + T)^-1, fp32 [64][64]
+constexpr uint32_t OFF_TF = OFF_LVX;          // T, fp32 [64][64] (swizzled, see fsw)
+constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A staging then (I + T)^-1, fp32 [64][64] (swizzled)
 constexpr uint32_t OFF_AQ = OFF_LVX + 32768;  // A, fp16 K-major [64 r][64 s]
 constexpr uint32_t OFF_IP = OFF_LVX + 40960;  // [Inv diag(beta); P], fp16 K-major [128][64]
 constexpr uint32_t OFF_YF = OFF_LVX + 57344;  // doubling scratch, fp32 (<= 1024 values)
 constexpr uint32_t OFF_KG = 143360;  // K * Gamma, fp16 MN-major [64 s][128 i]
 constexpr uint32_t OFF_QG = 159744;  // Q * Gamma, then Q', fp16 [64 r][128 i] (128B swizzle)
 constexpr uint32_t OFF_KH = 176128;  // K * rho, then W, fp16 [64][128 i] (128B swizzle)
-constexpr uint32_t OFF_GT = 192512;  // products of whole 8-position groups, fp32 [8][64]
-constexpr uint32_t OFF_PR = 194560;  // direct pairs and diag(A), fp32 [8 groups][32]
-constexpr uint32_t OFF_BETA = 195584;
-constexpr uint32_t OFF_GAMMA = 195840;
-constexpr uint32_t OFF_BAR = 196352;  // mbarriers: in0, in1, v, mma, lv
-constexpr uint32_t OFF_TMEMPTR = 196416;
-constexpr uint32_t kSmemUsed = 196432;
+constexpr uint32_t OFF_GT = 192512;  // products of whole 4-position groups, fp32 [16][64]
+constexpr uint32_t OFF_T4 = 196608;  // products of aligned runs of 4 groups, fp32 [4][64]
+constexpr uint32_t OFF_T8 = 197632;  // products of aligned runs of 8 groups, fp32 [2][64]
+constexpr uint32_t OFF_PR = 198144;  // direct pairs and diag(A), fp32 [16 groups][16]
+constexpr uint32_t OFF_BETA = 199168;
+constexpr uint32_t OFF_GAMMA = 199424;
+constexpr uint32_t OFF_BAR = 199936;  // mbarriers: in0, in1, v, mma, lv
+constexpr uint32_t OFF_TMEMPTR = 200000;
+constexpr uint32_t kSmemUsed = 200016;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
-// Staging of the workspace tiles for their TMA stores: [U~; A U~] as
-// [128][32] fp32 atoms over the dead work region and K * Gamma (up to 4
-// atoms), W over K * rho (stored to the workspace after the gate passes),
-// Q' in place of Q * Gamma.
-constexpr uint32_t OFF_UUST = OFF_LVX;
+// The workspace tiles leave by TMA stores straight from their operand
+// tiles ([Inv diag(beta); P], the fp16 V tile, K * rho) or from staging:
+// -W over K * rho (already stored by then), Q' in place of Q * Gamma.
 
 // factor kernel tensor-memory columns
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t TM_LV = 0;    // level pairs, 64 columns each (M = 128)
 constexpr uint32_t TM_P = 128;   // P (M = 64 layout)
 constexpr uint32_t TM_W = 192;   // [W; A W]       (M = 128, 128 columns)
-constexpr uint32_t TM_U = 320;   // [U~; A U~]     (M = 128, d_v columns)
 
 // ---- carry kernel: shared memory map ---------------------------------------
 // Two stages of one chunk's factors, each filled by one TMA transaction.
-constexpr uint32_t CS_WQ = 0;      // [W; Q'] fp16 K-major [128][128] (two 64-column atoms)
+constexpr uint32_t CS_WQ = 0;      // [-W; Q'] fp16 K-major [128][128] (two 64-column atoms)
 constexpr uint32_t CS_KH = 32768;  // K * rho fp16 MN-major [64 s][128 i]
-constexpr uint32_t CS_UU = 49152;  // [U~; A U~] fp32 [128][64 of d_v] as two [128][32] atoms
-constexpr uint32_t kStageBytes = 81920;
+constexpr uint32_t CS_IP = 49152;  // [Inv diag(beta); P] fp16 K-major [128 r][64 s]
+constexpr uint32_t CS_V = 65536;   // V slice fp16 MN-major [64 s][64 j]
+constexpr uint32_t kStageBytes = 73728;
 constexpr uint32_t OFF2_SB = 2 * kStageBytes;  // state slice, fp16 MN-major [128 i][64 j]
 constexpr uint32_t OFF2_UB = OFF2_SB + 16384;  // U, fp16 MN-major [64 s][64 j]
 constexpr uint32_t OFF2_OB = OFF2_UB + 8192;  // O staging for its TMA store: fp32 [64][32] x 2 or bf16 [64][64]
@@ -135,7 +137,7 @@ constexpr size_t kSmem2Bytes = kSmem2Used + 1024;
 
 // carry kernel tensor-memory columns
 constexpr uint32_t kTmem2Cols = 128;
-constexpr uint32_t TM2_X = 0;    // [W S; Q' S]    (M = 128, 64 columns)
+constexpr uint32_t TM2_X = 0;    // [U; O] = [U~ - W S; A U~ + Q' S]  (M = 128, 64 columns)
 constexpr uint32_t TM2_D = 64;   // (K rho)^T U    (M = 128, 64 columns)
 
 #ifdef CKDA_TC_DEBUG
@@ -241,78 +243,90 @@ __device__ __forceinline__ void reduce_scatter16(float* w, int lane) {
   }
 }
 
+// 32 consecutive output values of one row, fp32 or rounded once to bf16.
 template <typename Tout>
-__device__ __forceinline__ void store_row32(Tout* dst, const float* a, const float* x);
+__device__ __forceinline__ void store_row32(Tout* dst, const float* o);
 
 template <>
-__device__ __forceinline__ void store_row32<float>(float* dst, const float* a, const float* x) {
+__device__ __forceinline__ void store_row32<float>(float* dst, const float* o) {
 #pragma unroll
   for (int e = 0; e < 32; e += 4)
-    *reinterpret_cast<float4*>(dst + e) = make_float4(a[e] + x[e], a[e + 1] + x[e + 1],
-                                                      a[e + 2] + x[e + 2], a[e + 3] + x[e + 3]);
+    *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
 }
 
 template <>
-__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, const float* a,
-                                                           const float* x) {
+__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, const float* o) {
 #pragma unroll
   for (int e = 0; e < 32; e += 8) {
     uint4 pk;
-    pk.x = pack_bf16x2(a[e] + x[e], a[e + 1] + x[e + 1]);
-    pk.y = pack_bf16x2(a[e + 2] + x[e + 2], a[e + 3] + x[e + 3]);
-    pk.z = pack_bf16x2(a[e + 4] + x[e + 4], a[e + 5] + x[e + 5]);
-    pk.w = pack_bf16x2(a[e + 6] + x[e + 6], a[e + 7] + x[e + 7]);
+    pk.x = pack_bf16x2(o[e], o[e + 1]);
+    pk.y = pack_bf16x2(o[e + 2], o[e + 3]);
+    pk.z = pack_bf16x2(o[e + 4], o[e + 5]);
+    pk.w = pack_bf16x2(o[e + 6], o[e + 7]);
     *reinterpret_cast<uint4*>(dst + e) = pk;
   }
 }
 
-// Row r (0..63) of the output tile, columns [32 * half, +32), as a + x into
-// the 128B-swizzled staging of the TMA store: fp32 as two [64][32] atoms,
-// bf16 as one [64][64] atom.
+// Row r (0..63) of the output tile, columns [32 * half, +32), into the
+// 128B-swizzled staging of the TMA store: fp32 as two [64][32] atoms, bf16
+// as one [64][64] atom.
 template <typename Tout>
-__device__ __forceinline__ void stage_row32(uint32_t ob, int r, int half, const float* a,
-                                            const float* x);
+__device__ __forceinline__ void stage_row32(uint32_t ob, int r, int half, const float* o);
 
 template <>
-__device__ __forceinline__ void stage_row32<float>(uint32_t ob, int r, int half, const float* a,
-                                                   const float* x) {
+__device__ __forceinline__ void stage_row32<float>(uint32_t ob, int r, int half, const float* o) {
   const uint32_t row = ob + 8192 * half + 128 * r;
 #pragma unroll
   for (int c4 = 0; c4 < 8; ++c4) {
     const int e = 4 * c4;
-    sts_f4(row + ((c4 ^ (r & 7)) << 4),
-           make_float4(a[e] + x[e], a[e + 1] + x[e + 1], a[e + 2] + x[e + 2], a[e + 3] + x[e + 3]));
+    sts_f4(row + ((c4 ^ (r & 7)) << 4), make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
   }
 }
 
 template <>
 __device__ __forceinline__ void stage_row32<__nv_bfloat16>(uint32_t ob, int r, int half,
-                                                           const float* a, const float* x) {
+                                                           const float* o) {
   const uint32_t row = ob + 128 * r;
 #pragma unroll
   for (int c8 = 0; c8 < 4; ++c8) {
     const int e = 8 * c8;
     uint32_t w[4];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(a[e + 2 * t] + x[e + 2 * t], a[e + 2 * t + 1] + x[e + 2 * t + 1]);
+    for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(o[e + 2 * t], o[e + 2 * t + 1]);
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (((4 * half + c8) ^ (r & 7)) << 4)),
                  "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                  : "memory");
   }
 }
 
-// One gate pass over one 64-channel half (see the file comment).  Thread
-// (c4, g, role): channels 4*c4 .. 4*c4+3 of the half, positions 8g .. 8g+7.
-// Role 0 walks forward (prefix products: Gamma and the right halves of
-// levels 2..5); role 1 walks backward (suffix products: rho and the left
-// halves) and adds its channels' share of the direct pairs of levels 0..1
-// and of diag(A) into the pair buffer (stored by half 0, added by half 1).
-// The role is the warp's
-// parity, so the two warps sharing a scheduler (w and w + 4) run the same
-// code; one out-of-line copy serves both halves.
+// Word offset of element (r, c) in a 64 x 64 fp32 tile whose 16-byte groups
+// are XOR-swizzled by the row: a float4 column block read or written by
+// threads of different rows, or a row block by threads of different column
+// blocks, spreads over the banks.
+__device__ __forceinline__ int fsw(int r, int c) {
+  return r * 64 + ((((c >> 2) ^ r) & 15) << 2) + (c & 3);
+}
+
+// Row of position p among the 32 operand rows of level lv: the positions
+// whose bit lv is set (right halves) or clear (left halves), in order.
+__device__ __forceinline__ int level_row(int lv, int p) {
+  return ((p >> (lv + 1)) << lv) | (p & ((1 << lv) - 1));
+}
+
+// One gate pass over one 64-channel half.  Thread (role, g, c4): channels
+// 4*c4 .. 4*c4+3 of the half, positions 4g .. 4g+3 (g = 0..15, one aligned
+// block of 4).  Role 0 walks forward (prefix products: Gamma and the right
+// halves of levels 2..5); role 1 walks backward (suffix products: rho and the
+// left halves) and adds its channels' share of the direct pairs of levels
+// 0..1 (inside its block of 4) and of diag(A) into the pair buffer (stored by
+// half 0, added by half 1).  The products of whole groups, and of aligned
+// runs of 4 and 8 groups, are formed once and exchanged through shared
+// memory, so every anchored offset costs at most five loads.  The role is the
+// warp's parity, so the warps sharing a scheduler run the same code; one
+// out-of-line copy serves both halves.
 __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid) {
   const int role = (tid >> 5) & 1;
-  const int rt = ((tid >> 6) << 5) | (tid & 31);  // index among the 128 threads of this role
+  const int rt = ((tid >> 6) << 5) | (tid & 31);  // index among the 256 threads of this role
   const int c4 = rt & 15;
   const int g = rt >> 4;
   const int cl = 4 * c4;
@@ -331,12 +345,12 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     return pk;
   };
 
-  // every input of this thread's 8 positions, loaded up front
-  float4 aa[8], ka[8], qa[8];
-  float bb[8];
+  // every input of this thread's 4 positions, loaded up front
+  float4 aa[4], ka[4], qa[4];
+  float bb[4];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int p = 8 * g + u;
+  for (int u = 0; u < 4; ++u) {
+    const int p = 4 * g + u;
     const bool val = p < Lc;
     aa[u] = val ? lds_f4(in + IN_A + p * 256 + cl * 4) : one;
     ka[u] = val ? bf4(lds_u2(in + IN_K + p * 128 + cl * 2)) : zero;
@@ -346,18 +360,33 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
 #ifdef CKDA_TC_DEBUG
   long long gp_last = clock64();
 #endif
-  // products of whole groups
+  // products of whole groups, then of aligned runs of 4 and 8 groups
   const uint32_t gt = sb + OFF_GT + cl * 4;
-  if (role == 0) {
-    float4 t = aa[0];
+  if (role == 0) sts_f4(gt + g * 256, mul4(mul4(aa[0], aa[1]), mul4(aa[2], aa[3])));
+  __syncthreads();
+  if (tid < 96) {
+    const int sc = tid & 15, seg = tid >> 4;
+    const uint32_t src = sb + OFF_GT + sc * 16;
+    if (seg < 4) {
+      const float4 x = mul4(mul4(lds_f4(src + (4 * seg) * 256), lds_f4(src + (4 * seg + 1) * 256)),
+                            mul4(lds_f4(src + (4 * seg + 2) * 256), lds_f4(src + (4 * seg + 3) * 256)));
+      sts_f4(sb + OFF_T4 + seg * 256 + sc * 16, x);
+    } else {
+      const int b8 = 8 * (seg - 4);
+      float4 x[8];
 #pragma unroll
-    for (int u = 1; u < 8; ++u) t = mul4(t, aa[u]);
-    sts_f4(gt + g * HC * 4, t);
+      for (int j = 0; j < 8; ++j) x[j] = lds_f4(src + (b8 + j) * 256);
+      const float4 y = mul4(mul4(mul4(x[0], x[1]), mul4(x[2], x[3])),
+                            mul4(mul4(x[4], x[5]), mul4(x[6], x[7])));
+      sts_f4(sb + OFF_T8 + (seg - 4) * 256 + sc * 16, y);
+    }
   }
   GP_MARK(0);
   __syncthreads();
   GP_MARK(1);
-  auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * HC * 4); };
+  auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * 256); };
+  auto run4 = [&](int s4) -> float4 { return lds_f4(sb + OFF_T4 + s4 * 256 + cl * 4); };
+  auto run8 = [&](int s8) -> float4 { return lds_f4(sb + OFF_T8 + s8 * 256 + cl * 4); };
   const uint32_t LV = sb + OFF_LVX;
   auto lop = [&](int lv, int row) -> uint32_t {
     return LV + ((lv - 2) >> 1) * kPairBytes + sw128_elem(64 * ((lv - 2) & 1) + row, cl, 128);
@@ -368,15 +397,21 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
   };
 
   if (role == 0) {
-    float4 pg = one;  // Gamma offset: product of the earlier groups
-    for (int gg = 0; gg < g; ++gg) pg = mul4(pg, gtot(gg));
-    float4 off4 = one, off5 = one;
-    if ((g & 3) == 3) off4 = gtot(g - 1);
-    for (int gg = 4; gg < g; ++gg) off5 = mul4(off5, gtot(gg));
-    float4 lp = one, l2 = one;
+    // Offsets: products of the whole groups from a level's anchor up to g.
+    // Level 2's anchor is this group; level 3's the start of the pair of
+    // groups, level 4's of the run of 4, level 5's of the run of 8.
+    const int g4 = g & ~3;
+    float4 off4 = one;
+    if (g - g4 >= 1) off4 = gtot(g4);
+    if (g - g4 >= 2) off4 = mul4(off4, gtot(g4 + 1));
+    if (g - g4 >= 3) off4 = mul4(off4, gtot(g4 + 2));
+    const float4 off3 = (g & 1) ? gtot(g - 1) : one;
+    const float4 off5 = (g & 4) ? mul4(run4((g >> 2) & ~1), off4) : off4;
+    float4 pg = (g & 8) ? mul4(run8(0), off5) : off5;  // Gamma offset: every earlier group
+    float4 lp = one;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int p = 8 * g + u;
+    for (int u = 0; u < 4; ++u) {
+      const int p = 4 * g + u;
       const float4 a = aa[u];
       const float4 kf = ka[u];
       const float4 qf = qa[u];
@@ -385,91 +420,82 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
       lp = (u == 0) ? a : mul4(lp, a);
       sts_u2(sb + OFF_KG + sw128_elem(p, ig, 64), h4(mul4(kf, pg)));
       sts_u2(sb + OFF_QG + sw128_elem(p, ig, 64), h4(mul4(qf, pg)));
-      if (u >= 4) {  // level 2: right half of the group
-        l2 = (u == 4) ? a : mul4(l2, a);
-        const int rho = 4 * g + u - 4;
-        sts_u2(lop(2, rho), h4(mul4(bk, l2)));
-        sts_u2(lop(2, 32 + rho), h4(mul4(qf, l2)));
+      if (g & 1) {  // level 2: right half
+        const int r = level_row(2, p);
+        sts_u2(lop(2, r), h4(mul4(bk, lp)));
+        sts_u2(lop(2, 32 + r), h4(mul4(qf, lp)));
       }
-      if (g & 1) {  // level 3: right half
-        const int rho = 8 * (g >> 1) + u;
-        sts_u2(lop(3, rho), h4(mul4(bk, lp)));
-        sts_u2(lop(3, 32 + rho), h4(mul4(qf, lp)));
+      if (g & 2) {  // level 3: right half
+        const float4 L = mul4(off3, lp);
+        const int r = level_row(3, p);
+        sts_u2(lop(3, r), h4(mul4(bk, L)));
+        sts_u2(lop(3, 32 + r), h4(mul4(qf, L)));
       }
-      if (g & 2) {  // level 4: right half
+      if (g & 4) {  // level 4: right half
         const float4 L = mul4(off4, lp);
-        const int rho = 16 * (g >> 2) + 8 * (g & 1) + u;
-        sts_u2(lop(4, rho), h4(mul4(bk, L)));
-        sts_u2(lop(4, 32 + rho), h4(mul4(qf, L)));
+        const int r = level_row(4, p);
+        sts_u2(lop(4, r), h4(mul4(bk, L)));
+        sts_u2(lop(4, 32 + r), h4(mul4(qf, L)));
       }
-      if (g & 4) {  // level 5: right half
+      if (g & 8) {  // level 5: right half
         const float4 L = mul4(off5, lp);
-        const int rho = 8 * (g - 4) + u;
-        sts_u2(lop(5, rho), h4(mul4(bk, L)));
-        sts_u2(lop(5, 32 + rho), h4(mul4(qf, L)));
+        const int r = level_row(5, p);
+        sts_u2(lop(5, r), h4(mul4(bk, L)));
+        sts_u2(lop(5, 32 + r), h4(mul4(qf, L)));
       }
     }
-    if (g == 7) sts_f4(sb + OFF_GAMMA + ig * 4, pg);
+    if (g == 15) sts_f4(sb + OFF_GAMMA + ig * 4, pg);
     GP_MARK(2);
   } else {
-    float4 offr = one;  // rho offset: product of the later groups
-    for (int gg = g + 1; gg < 8; ++gg) offr = mul4(offr, gtot(gg));
-    const float4 off4 = (g & 1) ? one : gtot(g + 1);
-    float4 off5 = one;
-    for (int gg = g + 1; gg < 4; ++gg) off5 = mul4(off5, gtot(gg));
-    float4 ls = one, r2 = one;
+    // Offsets: products of the whole groups after g up to a level's anchor.
+    float4 offr4 = one;
+    if ((g | 3) - g >= 1) offr4 = gtot(g + 1);
+    if ((g | 3) - g >= 2) offr4 = mul4(offr4, gtot(g + 2));
+    if ((g | 3) - g >= 3) offr4 = mul4(offr4, gtot(g + 3));
+    const float4 offr3 = (g & 1) ? one : gtot(g + 1);
+    const float4 offr5 = (g & 4) ? offr4 : mul4(offr4, run4((g >> 2) + 1));
+    const float4 offr = (g & 8) ? offr5 : mul4(offr5, run8(1));  // rho offset: every later group
+    float4 ls = one;
 #pragma unroll
-    for (int u = 7; u >= 0; --u) {
-      const int p = 8 * g + u;
-      const float4 a = aa[u];
+    for (int u = 3; u >= 0; --u) {
+      const int p = 4 * g + u;
       const float4 kf = ka[u];
       sts_u2(sb + OFF_KH + sw128_elem(p, ig, 64), h4(mul4(kf, mul4(offr, ls))));
-      if (u < 4) {  // level 2: left half of the group
-        sts_u2(rop(2, 4 * g + u), h4(mul4(kf, r2)));
-        r2 = mul4(r2, a);
-      }
-      if (!(g & 1)) sts_u2(rop(3, 8 * (g >> 1) + u), h4(mul4(kf, ls)));
-      if (!(g & 2)) sts_u2(rop(4, 16 * (g >> 2) + 8 * (g & 1) + u), h4(mul4(kf, mul4(off4, ls))));
-      if (!(g & 4)) sts_u2(rop(5, 8 * g + u), h4(mul4(kf, mul4(off5, ls))));
-      ls = mul4(ls, a);
+      if (!(g & 1)) sts_u2(rop(2, level_row(2, p)), h4(mul4(kf, ls)));
+      if (!(g & 2)) sts_u2(rop(3, level_row(3, p)), h4(mul4(kf, mul4(offr3, ls))));
+      if (!(g & 4)) sts_u2(rop(4, level_row(4, p)), h4(mul4(kf, mul4(offr4, ls))));
+      if (!(g & 8)) sts_u2(rop(5, level_row(5, p)), h4(mul4(kf, mul4(offr5, ls))));
+      ls = mul4(ls, aa[u]);
     }
     GP_MARK(3);
-    // direct pairs inside each aligned block of 4 (levels 0 and 1) and diag(A)
-    float acc[32];
+    // direct pairs inside this aligned block of 4 (levels 0 and 1) and diag(A)
+    float acc[16];
+    {
+      const float4 k0 = ka[0], k1 = ka[1], k2 = ka[2], k3 = ka[3];
+      const float4 q1 = qa[1], q2 = qa[2], q3 = qa[3];
+      const float4 e10 = mul4(aa[1], k0);
+      const float4 e20 = mul4(aa[2], e10);
+      const float4 e21 = mul4(aa[2], k1);
+      const float4 e30 = mul4(aa[3], e20);
+      const float4 e31 = mul4(aa[3], e21);
+      const float4 e32 = mul4(aa[3], k2);
+      acc[0] = dot4(k1, e10);  acc[1] = dot4(q1, e10);
+      acc[2] = dot4(k2, e20);  acc[3] = dot4(q2, e20);
+      acc[4] = dot4(k2, e21);  acc[5] = dot4(q2, e21);
+      acc[6] = dot4(k3, e30);  acc[7] = dot4(q3, e30);
+      acc[8] = dot4(k3, e31);  acc[9] = dot4(q3, e31);
+      acc[10] = dot4(k3, e32); acc[11] = dot4(q3, e32);
 #pragma unroll
-    for (int m = 0; m < 2; ++m) {
-      const float4 k0 = ka[4 * m], k1 = ka[4 * m + 1], k2 = ka[4 * m + 2], k3 = ka[4 * m + 3];
-      const float4 a1 = aa[4 * m + 1], a2 = aa[4 * m + 2], a3 = aa[4 * m + 3];
-      const float4 q1 = qa[4 * m + 1], q2 = qa[4 * m + 2], q3 = qa[4 * m + 3];
-      const float4 e10 = mul4(a1, k0);
-      const float4 e20 = mul4(a2, e10);
-      const float4 e21 = mul4(a2, k1);
-      const float4 e30 = mul4(a3, e20);
-      const float4 e31 = mul4(a3, e21);
-      const float4 e32 = mul4(a3, k2);
-      float* o = acc + 12 * m;
-      o[0] = dot4(k1, e10);  o[1] = dot4(q1, e10);
-      o[2] = dot4(k2, e20);  o[3] = dot4(q2, e20);
-      o[4] = dot4(k2, e21);  o[5] = dot4(q2, e21);
-      o[6] = dot4(k3, e30);  o[7] = dot4(q3, e30);
-      o[8] = dot4(k3, e31);  o[9] = dot4(q3, e31);
-      o[10] = dot4(k3, e32); o[11] = dot4(q3, e32);
+      for (int u = 0; u < 4; ++u) acc[12 + u] = dot4(qa[u], ka[u]);
     }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) acc[24 + u] = dot4(qa[u], ka[u]);
-    // sum over the 16 threads (channels) of the group, then over the halves
+    // sum over the 16 threads (channels) of the group
     const int lane = tid & 31;
     reduce_scatter16(acc, lane);
-    reduce_scatter16(acc + 16, lane);
-    const uint32_t pr = sb + OFF_PR + 128 * g;
-    const uint32_t p0 = pr + 4 * (lane & 15), p1 = pr + 64 + 4 * (lane & 15);
-    if (hh == 0) {
+    const uint32_t p0 = sb + OFF_PR + 64 * g + 4 * (lane & 15);
+    if (hh == 0)
       sts_f(p0, acc[0]);
-      sts_f(p1, acc[16]);
-    } else {
+    else
       sts_f(p0, lds_f(p0) + acc[0]);
-      sts_f(p1, lds_f(p1) + acc[16]);
-    }
     GP_MARK(2);
   }
 }
@@ -478,77 +504,54 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
 // (I + T): merge diagonal blocks of size M into blocks of size 2M,
 //   [[A, 0], [B, D]]^-1 = [[A^-1, 0], [-D^-1 B A^-1, D^-1]],  B = T block.
 // Inv holds the inverses of the M-blocks (zero above each block diagonal),
-// so the triangular limits of both products can be left to the zeros.
+// so the triangular limits of both products can be left to the zeros.  Both
+// tiles use the fsw layout.
 template <int M>
 __device__ __forceinline__ void inv_merge(const float* Tf, float* Inv, float* Yf, int tid) {
   constexpr int NMERGE = 64 / (2 * M);
-  if constexpr (M >= 4) {
-    constexpr int W4 = M / 4;                  // float4 groups per block row
-    constexpr int NOUT = NMERGE * M * W4;      // float4 outputs per phase
-    for (int e = tid; e < NOUT; e += NT) {
-      const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
-      const int r0 = 2 * M * qb;
-      const float* trow = Tf + (r0 + M + a) * 64 + r0;
-      float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+  constexpr int W4 = M / 4;                  // float4 groups per block row
+  constexpr int NOUT = NMERGE * M * W4;      // float4 outputs per phase
+  for (int e = tid; e < NOUT; e += NT1) {
+    const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
+    const int r0 = 2 * M * qb;
+    const int tr = r0 + M + a;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int t4 = 0; t4 < M / 4; ++t4) {
-        const float4 tv = *reinterpret_cast<const float4*>(trow + 4 * t4);
-        const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+    for (int t4 = 0; t4 < M / 4; ++t4) {
+      const float4 tv = *reinterpret_cast<const float4*>(Tf + fsw(tr, r0 + 4 * t4));
+      const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float4 iv =
-              *reinterpret_cast<const float4*>(Inv + (r0 + 4 * t4 + w) * 64 + r0 + 4 * c4);
-          y.x = fmaf(tt[w], iv.x, y.x); y.y = fmaf(tt[w], iv.y, y.y);
-          y.z = fmaf(tt[w], iv.z, y.z); y.w = fmaf(tt[w], iv.w, y.w);
-        }
+      for (int w = 0; w < 4; ++w) {
+        const float4 iv =
+            *reinterpret_cast<const float4*>(Inv + fsw(r0 + 4 * t4 + w, r0 + 4 * c4));
+        y.x = fmaf(tt[w], iv.x, y.x); y.y = fmaf(tt[w], iv.y, y.y);
+        y.z = fmaf(tt[w], iv.z, y.z); y.w = fmaf(tt[w], iv.w, y.w);
       }
-      *reinterpret_cast<float4*>(Yf + qb * M * M + a * M + 4 * c4) = y;
     }
-    __syncthreads();
-    for (int e = tid; e < NOUT; e += NT) {
-      const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
-      const int r0 = 2 * M * qb;
-      const float* irow = Inv + (r0 + M + a) * 64 + r0 + M;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int t4 = 0; t4 < M / 4; ++t4) {
-        const float4 dv = *reinterpret_cast<const float4*>(irow + 4 * t4);
-        const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-          const float4 yv =
-              *reinterpret_cast<const float4*>(Yf + qb * M * M + (4 * t4 + w) * M + 4 * c4);
-          x.x = fmaf(dd[w], yv.x, x.x); x.y = fmaf(dd[w], yv.y, x.y);
-          x.z = fmaf(dd[w], yv.z, x.z); x.w = fmaf(dd[w], yv.w, x.w);
-        }
-      }
-      *reinterpret_cast<float4*>(Inv + (r0 + M + a) * 64 + r0 + 4 * c4) =
-          make_float4(-x.x, -x.y, -x.z, -x.w);
-    }
-    __syncthreads();
-  } else {
-    constexpr int NOUT = NMERGE * M * M;
-    for (int e = tid; e < NOUT; e += NT) {
-      const int qb = e / (M * M), a = (e / M) % M, cc = e % M;
-      const int r0 = 2 * M * qb;
-      float y = 0.f;
-#pragma unroll
-      for (int t = 0; t < M; ++t)
-        y = fmaf(Tf[(r0 + M + a) * 64 + r0 + t], Inv[(r0 + t) * 64 + r0 + cc], y);
-      Yf[e] = y;
-    }
-    __syncthreads();
-    for (int e = tid; e < NOUT; e += NT) {
-      const int qb = e / (M * M), a = (e / M) % M, cc = e % M;
-      const int r0 = 2 * M * qb;
-      float x = 0.f;
-#pragma unroll
-      for (int t = 0; t < M; ++t)
-        x = fmaf(Inv[(r0 + M + a) * 64 + r0 + M + t], Yf[qb * M * M + t * M + cc], x);
-      Inv[(r0 + M + a) * 64 + r0 + cc] = -x;
-    }
-    __syncthreads();
+    *reinterpret_cast<float4*>(Yf + qb * M * M + a * M + 4 * c4) = y;
   }
+  __syncthreads();
+  for (int e = tid; e < NOUT; e += NT1) {
+    const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
+    const int r0 = 2 * M * qb;
+    const int ir = r0 + M + a;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int t4 = 0; t4 < M / 4; ++t4) {
+      const float4 dv = *reinterpret_cast<const float4*>(Inv + fsw(ir, r0 + M + 4 * t4));
+      const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 yv =
+            *reinterpret_cast<const float4*>(Yf + qb * M * M + (4 * t4 + w) * M + 4 * c4);
+        x.x = fmaf(dd[w], yv.x, x.x); x.y = fmaf(dd[w], yv.y, x.y);
+        x.z = fmaf(dd[w], yv.z, x.z); x.w = fmaf(dd[w], yv.w, x.w);
+      }
+    }
+    *reinterpret_cast<float4*>(Inv + fsw(ir, r0 + 4 * c4)) =
+        make_float4(-x.x, -x.y, -x.z, -x.w);
+  }
+  __syncthreads();
 }
 
 // ---- work units ----------------------------------------------------------------
@@ -620,11 +623,12 @@ __device__ Unit find_unit(int64_t ui, int64_t stride, int64_t n_units, const int
 // ---- kernel 1: per-unit WY factors ----------------------------------------------
 
 template <int DV>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT1, 1)
 factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
               const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
-              const __grid_constant__ CUtensorMap tm_uu, const float* __restrict__ beta,
+              const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
+              const float* __restrict__ beta,
               const int32_t* __restrict__ cu, int n_seqs, int T, int H, int nch, int64_t n_units,
               float* __restrict__ ws_g, int* status) {
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
@@ -635,8 +639,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int q4 = warp & 3;
-  const int half = warp >> 2;
+  const int q4 = warp & 3;     // tensor-memory lane quarter of this warp
+  const int quarter = warp >> 2;  // which quarter of a tile's columns this warp takes
 
   float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
   const float* gamma_s = reinterpret_cast<const float*>(sm + OFF_GAMMA);
@@ -659,7 +663,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     prefetch_tmap(&tm_a);
     prefetch_tmap(&tm_wq);
     prefetch_tmap(&tm_kh);
-    prefetch_tmap(&tm_uu);
+    prefetch_tmap(&tm_ip);
+    prefetch_tmap(&tm_v16);
   }
   if (warp == 0) {
     tmem_alloc(sb + OFF_TMEMPTR, kTmemCols);
@@ -741,15 +746,34 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const size_t u = (size_t)cur.idx;
     if (tid < C) beta_s[tid] = beta_next;
     // ---- gate pass, half 0 ---------------------------------------------------
+    // the previous unit's workspace stores must have read their tiles before
+    // the gate pass and the v load reuse them
+    if (c > 0) {
+      if (tid == 0) {
+        bulk_wait_read_all();
+        issue_v(cur);
+      }
+      pend_v = 1;
+    }
     ok = wait(bar_in0, ph_in0, pend_in0);
-    // the previous unit's workspace stores must have read their staging
-    if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     TC_MARK(0);
+#ifdef CKDA_TC_DEBUG
+    const long long t_gp0 = clock64();
+#endif
     gate_pass(sb, sb + OFF_IN0, 0, Lc, tid);
+#ifdef CKDA_TC_DEBUG
+    const long long t_gp1 = clock64();
+#endif
     fence_proxy_async_smem();
     __syncthreads();
+#ifdef CKDA_TC_DEBUG
+    if (g_tc_time2 != nullptr && lane == 0 && blockIdx.x == 0) {
+      atomicAdd(g_tc_time2 + 8 + warp, (unsigned long long)(t_gp1 - t_gp0));
+      atomicAdd(g_tc_time2 + 24 + warp, (unsigned long long)(clock64() - t_gp1));
+    }
+#endif
     if (tid == 0) {
       tc_fence_after();
       level_mmas(0);
@@ -793,54 +817,51 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     {
       float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
       float* Af = reinterpret_cast<float*>(sm + OFF_AF);
-      if (warp < 4) {
-        const int L = 32 * warp + lane;  // lane of the pair accumulators
+      if (warp < 8) {
+        // warp (lane quarter q4, pair warp/4): one 32-column block of a pair
+        const int pr = warp >> 2;
+        const int L = 32 * q4 + lane;  // lane of the pair accumulators
         const int rho = L & 63;
         const int rr = rho & 31;
         float* dst = (rho < 32) ? Tf : Af;
+        const int lv = 2 + 2 * pr + (L >> 6);
+        float v[32];
+        tmem_ld32(taddr(tmem, 32 * q4, TM_LV + 64 * pr + 32 * (q4 >> 1)), v);
+        tmem_ld_wait();
+        const int b = 1 << lv;
+        const int j = rr >> lv;
+        const int r = 2 * b * j + b + (rr & (b - 1));
 #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          const int lv = 2 + 2 * pr + (L >> 6);
-          float v[32];
-          tmem_ld32(taddr(tmem, 32 * warp, TM_LV + 64 * pr + 32 * (warp >> 1)), v);
-          tmem_ld_wait();
-          const int b = 1 << lv;
-          const int j = rr >> lv;
-          const int r = 2 * b * j + b + (rr & (b - 1));
-          float* row = dst + r * 64 + b * j;
-#pragma unroll
-          for (int m4 = 0; m4 < 8; ++m4) {
-            if (((4 * m4) >> lv) == j)
-              *reinterpret_cast<float4*>(row + 4 * m4) =
-                  make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
-          }
+        for (int m4 = 0; m4 < 8; ++m4) {
+          if (((4 * m4) >> lv) == j)
+            *reinterpret_cast<float4*>(dst + fsw(r, b * j + 4 * m4)) =
+                make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
         }
       } else {
         // direct pairs (r, s) inside aligned blocks of 4, and the diagonal of A
         const float* pr = reinterpret_cast<const float*>(sm + OFF_PR);
-        for (int e = tid - 128; e < 8 * 32; e += 128) {
-          const int g = e >> 5, w = e & 31;
-          const float val = pr[e];
-          if (w < 24) {
-            const int m = w / 12, jj = (w % 12) >> 1;
-            // pair order inside the block: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
-            const int rl = (jj == 0) ? 1 : (jj < 3 ? 2 : 3);
-            const int sl = (jj == 0 || jj == 1 || jj == 3) ? 0 : (jj == 2 || jj == 4 ? 1 : 2);
-            const int r = 8 * g + 4 * m + rl, s = 8 * g + 4 * m + sl;
-            if (w & 1)
-              Af[r * 64 + s] = val;
-            else
-              Tf[r * 64 + s] = beta_s[r] * val;
-          } else {
-            const int r = 8 * g + (w - 24);
-            Af[r * 64 + r] = val;
-          }
+        const int e = tid - 256;
+        const int g = e >> 4, w = e & 15;
+        const float val = pr[e];
+        if (w < 12) {
+          const int jj = w >> 1;
+          // pair order inside the block: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
+          const int rl = (jj == 0) ? 1 : (jj < 3 ? 2 : 3);
+          const int sl = (jj == 0 || jj == 1 || jj == 3) ? 0 : (jj == 2 || jj == 4 ? 1 : 2);
+          const int r = 4 * g + rl, s = 4 * g + sl;
+          if (w & 1)
+            Af[fsw(r, s)] = val;
+          else
+            Tf[fsw(r, s)] = beta_s[r] * val;
+        } else {
+          const int r = 4 * g + (w - 12);
+          Af[fsw(r, r)] = val;
         }
       }
       // v tile: bf16 (as loaded) -> fp16 in place; rows past the end -> 0.
       // Each 16-byte chunk stays within its 128-byte row under the swizzle.
       uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V);
-      for (int e = tid; e < C * 8 * (DV / 64); e += NT) {
+      for (int e = tid; e < C * 8 * (DV / 64); e += NT1) {
         uint4 raw = vt[e];
         if (((e >> 3) & 63) < Lc) {
           float f[8];
@@ -863,20 +884,23 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     tc_fence_before();
     __syncthreads();
-    TC_DBG(for (int e = tid; e < 4096; e += NT) {
-      g_tc_dbg[e] = reinterpret_cast<const float*>(sm + OFF_TF)[e];
-      g_tc_dbg[4096 + e] = reinterpret_cast<const float*>(sm + OFF_AF)[e];
+    TC_DBG(for (int e = tid; e < 4096; e += NT1) {
+      g_tc_dbg[e] = reinterpret_cast<const float*>(sm + OFF_TF)[fsw(e >> 6, e & 63)];
+      g_tc_dbg[4096 + e] = reinterpret_cast<const float*>(sm + OFF_AF)[fsw(e >> 6, e & 63)];
     });
     TC_MARK(4);
 
     // ---- A -> fp16 operand; (I + T)^-1 by recursive doubling ------------------
     {
       const float* Af = reinterpret_cast<const float*>(sm + OFF_AF);
-      for (int e = tid; e < 64 * 8; e += NT) {
-        const int r = e >> 3, cg = e & 7;
+      {
+        const int r = tid >> 3, cg = tid & 7;  // 512 threads: one 8-column chunk each
+        const float4 lo = *reinterpret_cast<const float4*>(Af + fsw(r, 8 * cg));
+        const float4 hi = *reinterpret_cast<const float4*>(Af + fsw(r, 8 * cg + 4));
+        const float a8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         float v[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) v[t] = (8 * cg + t <= r) ? Af[r * 64 + 8 * cg + t] : 0.f;
+        for (int t = 0; t < 8; ++t) v[t] = (8 * cg + t <= r) ? a8[t] : 0.f;
         st_chunk8(sm + OFF_AQ, sw128_chunk(r, 8 * cg, 64), v);
       }
     }
@@ -887,7 +911,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       float* Yf = reinterpret_cast<float*>(sm + OFF_YF);
       {
         uint4* z = reinterpret_cast<uint4*>(Inv);
-        for (int e = tid; e < 1024; e += NT) z[e] = make_uint4(0u, 0u, 0u, 0u);
+        for (int e = tid; e < 1024; e += NT1) z[e] = make_uint4(0u, 0u, 0u, 0u);
       }
       __syncthreads();
       // 8 x 8 diagonal blocks by forward substitution, one column per thread
@@ -896,8 +920,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         float tb[8][8];
 #pragma unroll
         for (int r2 = 1; r2 < 8; ++r2) {
-          const float4 lo = *reinterpret_cast<const float4*>(Tf + (base + r2) * 64 + base);
-          const float4 hi = *reinterpret_cast<const float4*>(Tf + (base + r2) * 64 + base + 4);
+          const float4 lo = *reinterpret_cast<const float4*>(Tf + fsw(base + r2, base));
+          const float4 hi = *reinterpret_cast<const float4*>(Tf + fsw(base + r2, base + 4));
           tb[r2][0] = lo.x; tb[r2][1] = lo.y; tb[r2][2] = lo.z; tb[r2][3] = lo.w;
           tb[r2][4] = hi.x; tb[r2][5] = hi.y; tb[r2][6] = hi.z; tb[r2][7] = hi.w;
         }
@@ -910,19 +934,22 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           x[r2] = (r2 < cc) ? 0.f : acc;
         }
 #pragma unroll
-        for (int r2 = 0; r2 < 8; ++r2) Inv[(base + r2) * 64 + base + cc] = x[r2];
+        for (int r2 = 0; r2 < 8; ++r2) Inv[fsw(base + r2, base + cc)] = x[r2];
       }
       __syncthreads();
       inv_merge<8>(Tf, Inv, Yf, tid);
       inv_merge<16>(Tf, Inv, Yf, tid);
       inv_merge<32>(Tf, Inv, Yf, tid);
-      TC_DBG(for (int e = tid; e < 4096; e += NT) g_tc_dbg[8192 + e] = Inv[e]);
+      TC_DBG(for (int e = tid; e < 4096; e += NT1) g_tc_dbg[8192 + e] = Inv[fsw(e >> 6, e & 63)]);
       // Inv diag(beta) -> rows 0..63 of the stacked operand
-      for (int e = tid; e < 64 * 8; e += NT) {
-        const int r = e >> 3, cg = e & 7;
+      {
+        const int r = tid >> 3, cg = tid & 7;
+        const float4 lo = *reinterpret_cast<const float4*>(Inv + fsw(r, 8 * cg));
+        const float4 hi = *reinterpret_cast<const float4*>(Inv + fsw(r, 8 * cg + 4));
+        const float i8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         float v[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) v[t] = Inv[r * 64 + 8 * cg + t] * beta_s[8 * cg + t];
+        for (int t = 0; t < 8; ++t) v[t] = i8[t] * beta_s[8 * cg + t];
         st_chunk8(sm + OFF_IP, sw128_chunk(r, 8 * cg, 128), v);
       }
     }
@@ -948,15 +975,16 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (!ok) break;
     tc_fence_after();
     {
-      float v[32];
-      tmem_ld32(taddr(tmem, 32 * q4, TM_P + 32 * half), v);
+      // M = 64 accumulator: row 16 * q4 + l sits in lane l (< 16) of quarter q4
+      float v[16];
+      tmem_ld16(taddr(tmem, 32 * q4, TM_P + 16 * quarter), v);
       tmem_ld_wait();
       if (lane < 16) {
         const int rho = 16 * q4 + lane;
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          st_chunk8(sm + OFF_IP, sw128_chunk(64 + rho, 32 * half + 8 * c4, 128), v + 8 * c4);
-        TC_DBG(for (int e = 0; e < 32; ++e) g_tc_dbg[12288 + rho * 64 + 32 * half + e] = v[e]);
+        for (int c8 = 0; c8 < 2; ++c8)
+          st_chunk8(sm + OFF_IP, sw128_chunk(64 + rho, 16 * quarter + 8 * c8, 128), v + 8 * c8);
+        TC_DBG(for (int e = 0; e < 16; ++e) g_tc_dbg[12288 + rho * 64 + 16 * quarter + e] = v[e]);
       }
     }
     fence_proxy_async_smem();
@@ -968,55 +996,50 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id1 = idesc_f16(128, 128, 0, 1);
-      constexpr uint32_t id2 = idesc_f16(128, DV, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = smem_desc(sb + OFF_IP + kk * 32, 16, 1024, kSwizzle128);
         const uint64_t bd = smem_desc(sb + OFF_KG + kk * 2048, 8192, 1024, kSwizzle128);
         mma_f16(tmem + TM_W, ad, bd, id1, kk > 0 ? 1u : 0u);
       }
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(sb + OFF_IP + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF_V + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM_U, ad, bd, id2, kk > 0 ? 1u : 0u);
-      }
       mma_commit(bar_mma);
+      // [Inv diag(beta); P] and the fp16 V tile are final: store them (the
+      // carry kernel forms [U~; A U~] from them)
+      const int yu = (int)(u * 2 * C);
+      tma_store_2d(&tm_ip, sb + OFF_IP, 0, yu);
+#pragma unroll
+      for (int a = 0; a < DV / 64; ++a)
+        tma_store_2d(&tm_v16, sb + OFF_V + 8192 * a, 64 * a, (int)(u * C));
+      bulk_commit();
     }
     pend_mma = 1;
     ok = wait(bar_mma, ph_mma, pend_mma);
-    fence_proxy_async_smem();
-    // K * rho has been read out: its tile takes W next
-    if (tid == 0) bulk_wait_read_all();
+    // K * rho has been read out (the stores just issued may still read):
+    // its tile takes -W next
+    if (tid == 0) bulk_wait_read_all_but_last();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    // the v tile is free: fetch the next unit's
-    if (more) {
-      if (tid == 0) issue_v(nxt);
-      pend_v = 1;
-    }
     TC_MARK(7);
 
-    // ---- [W; Q' = Q Gamma - A W], [U~; A U~] and gamma -> workspace -------------
-    // Each thread holds one tensor-memory row; the rows go to 128B-swizzled
-    // staging tiles (conflict-free), which TMA stores to the workspace.
+    // ---- [-W; Q' = Q Gamma - A W] and gamma -> workspace ------------------------
+    // Each thread holds 32 columns of one tensor-memory row of [W; A W]; the
+    // rows go to 128B-swizzled staging (conflict-free), which TMA stores.
     {
       const int L = 32 * q4 + lane;
-      float v[64];
-      tmem_ld32(taddr(tmem, 32 * q4, TM_W + 64 * half), v);
-      tmem_ld32(taddr(tmem, 32 * q4, TM_W + 64 * half + 32), v + 32);
+      float v[32];
+      tmem_ld32(taddr(tmem, 32 * q4, TM_W + 32 * quarter), v);
       tmem_ld_wait();
-      TC_DBG(for (int e = 0; e < 64; ++e) g_tc_dbg[16384 + L * 128 + 64 * half + e] = v[e]);
-      // W rows -> the K * rho tile; Q' rows replace Q * Gamma in place
+      TC_DBG(for (int e = 0; e < 32; ++e) g_tc_dbg[16384 + L * 128 + 32 * quarter + e] = v[e]);
+      // -W rows -> the K * rho tile; Q' rows replace Q * Gamma in place
       const int r = L & 63;
-      const uint32_t dst = sb + ((L < 64) ? OFF_KH : OFF_QG);
+      const uint32_t dst = (L < 64) ? OFF_KH : OFF_QG;
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        const uint32_t off = dst + sw128_chunk(r, 64 * half + 8 * c8, 64);
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const uint32_t off = dst + sw128_chunk(r, 32 * quarter + 8 * c8, 64);
         float w8[8];
         if (L >= 64) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(sm + (off - sb));
+          const uint4 raw = *reinterpret_cast<const uint4*>(sm + off);
           const __half2* p2 = reinterpret_cast<const __half2*>(&raw);
 #pragma unroll
           for (int t = 0; t < 4; ++t) {
@@ -1026,20 +1049,9 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           }
         } else {
 #pragma unroll
-          for (int t = 0; t < 8; ++t) w8[t] = v[8 * c8 + t];
+          for (int t = 0; t < 8; ++t) w8[t] = -v[8 * c8 + t];
         }
-        st_chunk8(sm, off - sb, w8);
-      }
-#pragma unroll
-      for (int a = 0; a < DV / 64; ++a) {
-        float w[32];
-        tmem_ld32(taddr(tmem, 32 * q4, TM_U + (DV / 2) * half + 32 * a), w);
-        tmem_ld_wait();
-        const uint32_t row = sb + OFF_UUST + 16384 * ((DV / 64) * half + a) + 128 * L;
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4)
-          sts_f4(row + ((c4 ^ (L & 7)) << 4),
-                 make_float4(w[4 * c4], w[4 * c4 + 1], w[4 * c4 + 2], w[4 * c4 + 3]));
+        st_chunk8(sm, off, w8);
       }
       if (tid < DK) ws_g[u * DK + tid] = gamma_s[tid];
     }
@@ -1052,8 +1064,6 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       tma_store_2d(&tm_wq, sb + OFF_KH + 8192, 64, y);
       tma_store_2d(&tm_wq, sb + OFF_QG, 0, y + C);
       tma_store_2d(&tm_wq, sb + OFF_QG + 8192, 64, y + C);
-#pragma unroll
-      for (int a = 0; a < DV / 32; ++a) tma_store_2d(&tm_uu, sb + OFF_UUST + 16384 * a, 32 * a, y);
       bulk_commit();
     }
     TC_MARK(8);
@@ -1086,7 +1096,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 template <typename Tout>
 __global__ void __launch_bounds__(NT, 1)
 carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
-             const __grid_constant__ CUtensorMap tm_uu, const __grid_constant__ CUtensorMap tm_out,
+             const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
+             const __grid_constant__ CUtensorMap tm_out,
              const float* __restrict__ ws_g,
              const float* S0, const int32_t* __restrict__ cu, Tout* __restrict__ out,
              float* S_final, int n_seqs, int T, int H, int DV, int nch, int* status) {
@@ -1112,7 +1123,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     fence_mbar_init();
     prefetch_tmap(&tm_wq);
     prefetch_tmap(&tm_kh);
-    prefetch_tmap(&tm_uu);
+    prefetch_tmap(&tm_ip);
+    prefetch_tmap(&tm_v16);
     prefetch_tmap(&tm_out);
   }
   if (warp == 0) {
@@ -1172,8 +1184,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     tma_load_2d(base + CS_WQ + 16384, &tm_wq, 64, (int)(uidx * 2 * C), bar);
     tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), bar);
     tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), bar);
-    tma_load_2d(base + CS_UU, &tm_uu, j0, (int)(uidx * 2 * C), bar);
-    tma_load_2d(base + CS_UU + 16384, &tm_uu, j0 + 32, (int)(uidx * 2 * C), bar);
+    tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), bar);
+    tma_load_2d(base + CS_V, &tm_v16, j0, (int)(uidx * C), bar);
   };
   if (tid == 0) {
     if (nchunks > 0) issue(0, 0);
@@ -1196,16 +1208,22 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     const float gm_next = (c + 1 < nchunks) ? ws_g[unit_of(c + 1) * DK + srow] : 1.f;
     TC_MARK(9);
 
-    // ---- carry 1: X = [W; Q'] S ---------------------------------------------------
+    // ---- carry 1: [U; O] = [Inv diag(beta); P] V + [-W; Q'] S -------------------
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, 0, 1);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = smem_desc(stage + CS_IP + kk * 32, 16, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(stage + CS_V + kk * 2048, 8192, 1024, kSwizzle128);
+        mma_f16(tmem + TM2_X, ad, bd, id, kk > 0 ? 1u : 0u);
+      }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint64_t ad =
             smem_desc(stage + CS_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
         const uint64_t bd = smem_desc(sb + OFF2_SB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_X, ad, bd, id, kk > 0 ? 1u : 0u);
+        mma_f16(tmem + TM2_X, ad, bd, id, 1u);
       }
       mma_commit(bar_mma);
     }
@@ -1218,34 +1236,22 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     tc_fence_after();
     TC_MARK(10);
 
-    // ---- U = U~ - X_top -> operand;  O = A U~ + X_bottom -> out ------------------
+    // ---- U -> operand;  O -> out ---------------------------------------------------
     {
-      float a[32], x[32];
+      float x[32];
       tmem_ld32(taddr(tmem, 32 * q4, TM2_X + 32 * half), x);
-      const uint32_t arow = stage + CS_UU + 16384 * half + 128 * srow;
-#pragma unroll
-      for (int c4 = 0; c4 < 8; ++c4) {
-        const float4 f = lds_f4(arow + ((c4 ^ (srow & 7)) << 4));
-        a[4 * c4] = f.x; a[4 * c4 + 1] = f.y; a[4 * c4 + 2] = f.z; a[4 * c4 + 3] = f.w;
-      }
       tmem_ld_wait();
-      TC_DBG(for (int e = 0; e < 32; ++e) {
-        g_tc_dbg[32768 + srow * 64 + 32 * half + e] = a[e];
-        g_tc_dbg[40960 + srow * 64 + 32 * half + e] = x[e];
-      });
+      TC_DBG(for (int e = 0; e < 32; ++e) g_tc_dbg[32768 + srow * 64 + 32 * half + e] = x[e]);
       if (q4 < 2) {
-        float uv[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) uv[e] = a[e] - x[e];
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
-          st_chunk8(sm + OFF2_UB, sw128_chunk(srow, 32 * half + 8 * c4, 64), uv + 8 * c4);
+          st_chunk8(sm + OFF2_UB, sw128_chunk(srow, 32 * half + 8 * c4, 64), x + 8 * c4);
       } else {
         const int r = srow - 64;
         if (tma_out)
-          stage_row32<Tout>(sb + OFF2_OB, r, half, a, x);
+          stage_row32<Tout>(sb + OFF2_OB, r, half, x);
         else if (r < Lc)
-          store_row32<Tout>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + 32 * half, a, x);
+          store_row32<Tout>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + 32 * half, x);
       }
     }
     fence_proxy_async_smem();
@@ -1398,7 +1404,7 @@ int64_t n_units(bool varlen, int n_seqs, int T, int H) {
   return u > 0 ? u : 1;
 }
 
-size_t unit_bytes(int DV) { return kWsWQ + kWsKH + kWsG + (size_t)2 * C * DV * 4; }
+size_t unit_bytes(int DV) { return kWsWQ + kWsKH + kWsIP + kWsG + (size_t)C * DV * 2; }
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -1426,18 +1432,23 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
   const int nch = (int)(((int64_t)T + C - 1) / C);
   const int64_t nu = n_units(cu != nullptr, n_seqs, T, H);
-  // workspace arrays, in this order: [W; Q'], K rho, [U~; A U~], gamma
+  // workspace arrays, in this order: [-W; Q'], K rho, [Inv diag(beta); P],
+  // V (fp16), gamma -- every one a multiple of 512 bytes per unit
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   __half* ws_wq = reinterpret_cast<__half*>(w8);
   __half* ws_kh = reinterpret_cast<__half*>(w8 + nu * kWsWQ);
-  float* ws_uu = reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH));
-  float* ws_g = reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH + (size_t)2 * C * DV * 4));
+  __half* ws_ip = reinterpret_cast<__half*>(w8 + nu * (kWsWQ + kWsKH));
+  __half* ws_v = reinterpret_cast<__half*>(w8 + nu * (kWsWQ + kWsKH + kWsIP));
+  float* ws_g =
+      reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH + kWsIP + (size_t)C * DV * 2));
 
-  CUtensorMap mkh, muu;
+  CUtensorMap mkh, mip, mv16;
   if (!make_map(&mkh, ws_kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * C, 64, C,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&muu, ws_uu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DV, (uint64_t)nu * 2 * C, 32,
-                2 * C, CU_TENSOR_MAP_SWIZZLE_128B))
+      !make_map(&mip, ws_ip, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, C, (uint64_t)nu * 2 * C, 64,
+                2 * C, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&mv16, ws_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DV, (uint64_t)nu * C, 64, C,
+                CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
 
   if (phases & kFactors) {
@@ -1462,8 +1473,8 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       attr1 = true;
     }
     const int64_t g1 = nu < (int64_t)sm_count() ? nu : (int64_t)sm_count();
-    k1<<<(unsigned)g1, NT, kSmemBytes, stream>>>(mq, mk, mv, ma, mwq64, mkh, muu, beta, cu,
-                                                 n_seqs, T, H, nch, nu, ws_g, status);
+    k1<<<(unsigned)g1, NT1, kSmemBytes, stream>>>(mq, mk, mv, ma, mwq64, mkh, mip, mv16, beta,
+                                                  cu, n_seqs, T, H, nch, nu, ws_g, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1490,7 +1501,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       attr2 = true;
     }
     dim3 grid(DV / BV, H, n_seqs);
-    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, muu, mout, ws_g, S0, cu,
+    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, mv16, mout, ws_g, S0, cu,
                                           static_cast<Tout*>(out), S_final, n_seqs, T, H, DV,
                                           nch, status);
     return cudaGetLastError();

@@ -114,9 +114,9 @@ enum {
  *            ckda_fwd_chunked_workspace_bytes() bytes for these sizes,
  *            256-byte aligned, overlapping no tensor argument; its contents
  *            on entry do not matter and on return are unspecified.  Only
- *            the tensor-core path uses it (per chunk and head: the WY
- *            factors [W; Q'] and K * rho in fp16, [U~; A U~] and gamma in
- *            fp32, about 115 KB at d_v = 128); when the size query returns 0
+ *            the tensor-core path uses it (per chunk and head: [-W; Q'],
+ *            K * rho, [Inv diag(beta); P] and V in fp16, gamma in fp32,
+ *            82,432 bytes at d_v = 128); when the size query returns 0
  *            both may be NULL / 0.  Calls that run concurrently (other
  *            streams) need separate workspaces; calls ordered on one stream
  *            may share one.  A workspace that is missing or too small
@@ -142,7 +142,7 @@ CKDA_API int ckda_fwd_chunked(const void* q, const void* k, const void* v,
  *    output is bit-identical to ckda_fwd_chunked with any valid workspace.
  *  - Sizes whose workspace (ckda_fwd_chunked_workspace_bytes) exceeds
  *    CKDA_STATIC_SCRATCH_BYTES return CKDA_ERR_UNSUPPORTED and launch
- *    nothing: at d_v = 128 that is more than 582 units of
+ *    nothing: at d_v = 128 that is more than 814 units of
  *    ceil(T / 64) * B * H (fixed-length) or (floor(T / 64) + N) * H
  *    (packed), e.g. B = 1, T = 2048, H = 16 fits (512 units).  Sizes on the
  *    fp32 CUDA-core path need no scratch and are always accepted.
@@ -172,8 +172,9 @@ CKDA_API int ckda_fwd_chunked_static(const void* q, const void* k, const void* v
  *
  * ckda_fwd_factors reads q, k, v, alpha and beta (layouts as in
  * ckda_fwd_chunked) and writes, for every chunk of every head, the
- * S0-independent WY factors into `workspace`: [W; Q'] and K * rho (fp16),
- * [U~; A U~] and gamma (fp32) ("Gated DeltaNet-2", Methodology section 3:
+ * S0-independent WY factors into `workspace`: [-W; Q'], K * rho,
+ * [Inv diag(beta); P] and V (fp16), gamma (fp32), from which the carry forms
+ * [U~; A U~] = [Inv diag(beta); P] V ("Gated DeltaNet-2", Methodology section 3:
  * the decay absorbed into the WY factors; "Semidirect Fourier Delta
  * Attention", "Principales Contribuciones" item 3: each chunk is an affine
  * map of the state, S_end = (Diag(gamma) - (K*rho)^T W) S + (K*rho)^T U~).
@@ -208,7 +209,7 @@ CKDA_API int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* ou
  * Pure host function: needs no GPU.  The tensor-core path takes
  * (B * ceil(T / 64)) * H work units for a fixed-length batch and
  * (floor(T / 64) + N) * H for a packed one, each 2*64*128*2 + 64*128*2 +
- * 128*4 + 2*64*d_v*4 bytes.
+ * 2*64*64*2 + 128*4 + 64*d_v*2 bytes.
  */
 CKDA_API int64_t ckda_fwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v,
                                                   int chunk, int dtype, int out_dtype,

@@ -154,7 +154,9 @@ def test_selftest_rejects_bad_limits(lib):
     assert lib.ckda_selftest_bounded_wait(20000000, None) == -1
 
 
-UNIT_BYTES_DV128 = 2 * 64 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 2 * 64 * 128 * 4
+# per (chunk, head) unit: [-W; Q'] and K*rho (fp16), [Inv diag(beta); P] (fp16), gamma (fp32),
+# V (fp16, [64][d_v])
+UNIT_BYTES_DV128 = 2 * 64 * 128 * 2 + 64 * 128 * 2 + 2 * 64 * 64 * 2 + 128 * 4 + 64 * 128 * 2
 
 
 def test_workspace_size_query_needs_no_gpu(lib):
@@ -163,7 +165,7 @@ def test_workspace_size_query_needs_no_gpu(lib):
     # fixed-length: B * ceil(T / 64) * H units
     assert q(4, 4096, 16, 128, 128, 64, BF16, F32, 0) == 4 * 64 * 16 * UNIT_BYTES_DV128
     assert q(2, 100, 3, 128, 128, 64, BF16, F32, 0) == 2 * 2 * 3 * UNIT_BYTES_DV128
-    assert q(1, 64, 1, 128, 64, 0, BF16, BF16, 0) == 2 * 64 * 128 * 2 + 64 * 128 * 2 + 128 * 4 + 2 * 64 * 64 * 4
+    assert q(1, 64, 1, 128, 64, 0, BF16, BF16, 0) == UNIT_BYTES_DV128 - 64 * 64 * 2
     # packed: (floor(T / 64) + N) * H units
     assert q(5, 1000, 2, 128, 128, 64, BF16, F32, 1) == (1000 // 64 + 5) * 2 * UNIT_BYTES_DV128
     # the CUDA-core path needs none
@@ -229,7 +231,7 @@ def test_static_scratch_entry_rejects_oversized_calls_without_a_gpu(lib):
     from delta_rule_linear_ckda_b200._lib import CKDA_STATIC_SCRATCH_BYTES
 
     F32, BF16 = 0, 1
-    # 4 x 64 x 16 units at d_v = 128 need 472 MB > the 64 MiB scratch
+    # 4 x 64 x 16 units at d_v = 128 need 338 MB > the 64 MiB scratch
     assert lib.ckda_fwd_chunked_workspace_bytes(4, 4096, 16, 128, 128, 64, BF16, F32, 0) > \
         CKDA_STATIC_SCRATCH_BYTES
     r = lib.ckda_fwd_chunked_static(P, P + 0x1000, P + 0x2000, P + 0x3000, P + 0x4000, None, None,
