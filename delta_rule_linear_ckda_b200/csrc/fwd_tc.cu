@@ -388,13 +388,22 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
   auto run4 = [&](int s4) -> float4 { return lds_f4(sb + OFF_T4 + s4 * 256 + cl * 4); };
   auto run8 = [&](int s8) -> float4 { return lds_f4(sb + OFF_T8 + s8 * 256 + cl * 4); };
   const uint32_t LV = sb + OFF_LVX;
-  auto lop = [&](int lv, int row) -> uint32_t {
-    return LV + ((lv - 2) >> 1) * kPairBytes + sw128_elem(64 * ((lv - 2) & 1) + row, cl, 128);
-  };
-  auto rop = [&](int lv, int row) -> uint32_t {
-    return LV + ((lv - 2) >> 1) * kPairBytes + PAIR_ROP +
-           sw128_elem(32 * ((lv - 2) & 1) + row, cl, 64);
-  };
+
+  // Store addresses: every tile written here has 128-byte rows (64 fp16 of
+  // one channel half) in 128B-swizzled atoms, and position p = 4g + u lands
+  // in row (tile row of 4g) + u.  The 16-byte chunk of this thread's 4
+  // channels is XOR-ed with the row's low three bits, which for position
+  // rows and levels 3..5 are 4 (g & 1) + u and for level 2 4 ((g >> 1) & 1) + u.
+  uint32_t xo[4], xo2[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    xo[u] = (uint32_t)((((c4 >> 1) ^ (4 * (g & 1) + u)) << 4) | ((c4 & 1) << 3));
+    xo2[u] = (uint32_t)((((c4 >> 1) ^ (4 * ((g >> 1) & 1) + u)) << 4) | ((c4 & 1) << 3));
+  }
+  const uint32_t rowg = (uint32_t)(4 * g) * 128 + (uint32_t)hh * 8192;  // row 4g of this half's atom
+  // row 4g's level-lv operand row, as a byte offset inside the pair tile
+  auto lrow = [&](int lv) -> uint32_t { return (uint32_t)level_row(lv, 4 * g) * 128; };
+  auto pair_base = [&](int lv) -> uint32_t { return LV + ((lv - 2) >> 1) * kPairBytes; };
 
   if (role == 0) {
     // Offsets: products of the whole groups from a level's anchor up to g.
@@ -408,40 +417,44 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     const float4 off3 = (g & 1) ? gtot(g - 1) : one;
     const float4 off5 = (g & 4) ? mul4(run4((g >> 2) & ~1), off4) : off4;
     float4 pg = (g & 8) ? mul4(run8(0), off5) : off5;  // Gamma offset: every earlier group
+    // left operands [beta k L; q L] of level lv: rows level_row, 32 + level_row
+    const uint32_t kg_b = sb + OFF_KG + rowg;
+    const uint32_t qg_b = sb + OFF_QG + rowg;
+    const uint32_t l2b = pair_base(2) + lrow(2);
+    const uint32_t l3b = pair_base(3) + 64 * 128 + lrow(3);
+    const uint32_t l4b = pair_base(4) + lrow(4);
+    const uint32_t l5b = pair_base(5) + 64 * 128 + lrow(5);
     float4 lp = one;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int p = 4 * g + u;
       const float4 a = aa[u];
       const float4 kf = ka[u];
       const float4 qf = qa[u];
-      const float4 bk = scale4(bb[u], kf);
       pg = mul4(pg, a);
       lp = (u == 0) ? a : mul4(lp, a);
-      sts_u2(sb + OFF_KG + sw128_elem(p, ig, 64), h4(mul4(kf, pg)));
-      sts_u2(sb + OFF_QG + sw128_elem(p, ig, 64), h4(mul4(qf, pg)));
-      if (g & 1) {  // level 2: right half
-        const int r = level_row(2, p);
-        sts_u2(lop(2, r), h4(mul4(bk, lp)));
-        sts_u2(lop(2, 32 + r), h4(mul4(qf, lp)));
-      }
-      if (g & 2) {  // level 3: right half
-        const float4 L = mul4(off3, lp);
-        const int r = level_row(3, p);
-        sts_u2(lop(3, r), h4(mul4(bk, L)));
-        sts_u2(lop(3, 32 + r), h4(mul4(qf, L)));
-      }
-      if (g & 4) {  // level 4: right half
-        const float4 L = mul4(off4, lp);
-        const int r = level_row(4, p);
-        sts_u2(lop(4, r), h4(mul4(bk, L)));
-        sts_u2(lop(4, 32 + r), h4(mul4(qf, L)));
-      }
-      if (g & 8) {  // level 5: right half
-        const float4 L = mul4(off5, lp);
-        const int r = level_row(5, p);
-        sts_u2(lop(5, r), h4(mul4(bk, L)));
-        sts_u2(lop(5, 32 + r), h4(mul4(qf, L)));
+      const uint32_t ro = 128 * u + xo[u];
+      sts_u2(kg_b + ro, h4(mul4(kf, pg)));
+      sts_u2(qg_b + ro, h4(mul4(qf, pg)));
+      if (g & 15) {
+        const float4 qlp = mul4(qf, lp);
+        const float4 blp = scale4(bb[u], mul4(kf, lp));
+        if (g & 1) {  // level 2: right half
+          const uint32_t o2 = l2b + 128 * u + xo2[u];
+          sts_u2(o2, h4(blp));
+          sts_u2(o2 + 32 * 128, h4(qlp));
+        }
+        if (g & 2) {  // level 3: right half
+          sts_u2(l3b + ro, h4(mul4(blp, off3)));
+          sts_u2(l3b + 32 * 128 + ro, h4(mul4(qlp, off3)));
+        }
+        if (g & 4) {  // level 4: right half
+          sts_u2(l4b + ro, h4(mul4(blp, off4)));
+          sts_u2(l4b + 32 * 128 + ro, h4(mul4(qlp, off4)));
+        }
+        if (g & 8) {  // level 5: right half
+          sts_u2(l5b + ro, h4(mul4(blp, off5)));
+          sts_u2(l5b + 32 * 128 + ro, h4(mul4(qlp, off5)));
+        }
       }
     }
     if (g == 15) sts_f4(sb + OFF_GAMMA + ig * 4, pg);
@@ -455,16 +468,22 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     const float4 offr3 = (g & 1) ? one : gtot(g + 1);
     const float4 offr5 = (g & 4) ? offr4 : mul4(offr4, run4((g >> 2) + 1));
     const float4 offr = (g & 8) ? offr5 : mul4(offr5, run8(1));  // rho offset: every later group
+    // right operands k R of level lv: rows level_row of the level's 32
+    const uint32_t kh_b = sb + OFF_KH + rowg;
+    const uint32_t r2b = pair_base(2) + PAIR_ROP + lrow(2);
+    const uint32_t r3b = pair_base(3) + PAIR_ROP + 32 * 128 + lrow(3);
+    const uint32_t r4b = pair_base(4) + PAIR_ROP + lrow(4);
+    const uint32_t r5b = pair_base(5) + PAIR_ROP + 32 * 128 + lrow(5);
     float4 ls = one;
 #pragma unroll
     for (int u = 3; u >= 0; --u) {
-      const int p = 4 * g + u;
-      const float4 kf = ka[u];
-      sts_u2(sb + OFF_KH + sw128_elem(p, ig, 64), h4(mul4(kf, mul4(offr, ls))));
-      if (!(g & 1)) sts_u2(rop(2, level_row(2, p)), h4(mul4(kf, ls)));
-      if (!(g & 2)) sts_u2(rop(3, level_row(3, p)), h4(mul4(kf, mul4(offr3, ls))));
-      if (!(g & 4)) sts_u2(rop(4, level_row(4, p)), h4(mul4(kf, mul4(offr4, ls))));
-      if (!(g & 8)) sts_u2(rop(5, level_row(5, p)), h4(mul4(kf, mul4(offr5, ls))));
+      const float4 kls = mul4(ka[u], ls);
+      const uint32_t ro = 128 * u + xo[u];
+      sts_u2(kh_b + ro, h4(mul4(kls, offr)));
+      if (!(g & 1)) sts_u2(r2b + 128 * u + xo2[u], h4(kls));
+      if (!(g & 2)) sts_u2(r3b + ro, h4(mul4(kls, offr3)));
+      if (!(g & 4)) sts_u2(r4b + ro, h4(mul4(kls, offr4)));
+      if (!(g & 8)) sts_u2(r5b + ro, h4(mul4(kls, offr5)));
       ls = mul4(ls, aa[u]);
     }
     GP_MARK(3);
@@ -746,11 +765,12 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const size_t u = (size_t)cur.idx;
     if (tid < C) beta_s[tid] = beta_next;
     // ---- gate pass, half 0 ---------------------------------------------------
-    // the previous unit's workspace stores must have read their tiles before
-    // the gate pass and the v load reuse them
+    // the previous unit's workspace stores must have read the tiles the
+    // first gate pass and the v load reuse (all but the channel-64..127
+    // atoms of -W and Q', which the second gate pass waits for)
     if (c > 0) {
       if (tid == 0) {
-        bulk_wait_read_all();
+        bulk_wait_read_all_but_last();
         issue_v(cur);
       }
       pend_v = 1;
@@ -787,6 +807,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ---- gate pass, half 1 (after the half-0 level GEMMs release the operands)
     ok = wait(bar_in1, ph_in1, pend_in1);
     ok = wait(bar_lv, ph_lv, pend_lv) && ok;
+    if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     gate_pass(sb, sb + OFF_IN1, 1, Lc, tid);
@@ -1059,10 +1080,13 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
+      // channels 0..63 first: the next unit's first gate pass reuses only
+      // those atoms and waits for this group alone
       const int y = (int)(u * 2 * C);
       tma_store_2d(&tm_wq, sb + OFF_KH, 0, y);
-      tma_store_2d(&tm_wq, sb + OFF_KH + 8192, 64, y);
       tma_store_2d(&tm_wq, sb + OFF_QG, 0, y + C);
+      bulk_commit();
+      tma_store_2d(&tm_wq, sb + OFF_KH + 8192, 64, y);
       tma_store_2d(&tm_wq, sb + OFF_QG + 8192, 64, y + C);
       bulk_commit();
     }
