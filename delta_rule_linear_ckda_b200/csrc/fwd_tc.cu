@@ -93,7 +93,7 @@ constexpr uint32_t OFF_LVX = 81920;
 constexpr uint32_t kPairBytes = 24576;
 constexpr uint32_t PAIR_ROP = 16384;
 constexpr uint32_t OFF_TF = OFF_LVX;          // T, fp32 [64][64] (swizzled, see fsw)
-constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A staging then (I + T)^-1, fp32 [64][64] (swizzled)
+constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A, fp32 [64][64] (swizzled)
 constexpr uint32_t OFF_AQ = OFF_LVX + 32768;  // A, fp16 K-major [64 r][64 s]
 constexpr uint32_t OFF_IP = OFF_LVX + 40960;  // [Inv diag(beta); P], fp16 K-major [128][64]
 constexpr uint32_t OFF_YF = OFF_LVX + 57344;  // doubling scratch, fp32 (<= 1024 values)
@@ -108,7 +108,8 @@ constexpr uint32_t OFF_BETA = 199168;
 constexpr uint32_t OFF_GAMMA = 199424;
 constexpr uint32_t OFF_BAR = 199936;  // mbarriers: in0, in1, v, mma, lv
 constexpr uint32_t OFF_TMEMPTR = 200000;
-constexpr uint32_t kSmemUsed = 200016;
+constexpr uint32_t OFF_INV = 200704;  // (I + T)^-1, fp32 [64][64] (swizzled)
+constexpr uint32_t kSmemUsed = OFF_INV + 16384;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
 // The workspace tiles leave by TMA stores straight from their operand
 // tiles ([Inv diag(beta); P], the fp16 V tile, K * rho) or from staging:
@@ -595,16 +596,17 @@ __device__ __forceinline__ int64_t slot_base(const int32_t* cu, int n, int nch) 
 }
 
 // The first unit at or after `ui` (stepping by `stride`) that holds tokens.
-__device__ Unit find_unit(int64_t ui, int64_t stride, int64_t n_units, const int32_t* cu,
-                          int n_seqs, int T, int H, int nch) {
+// Unit and slot numbers fit in 32 bits (the host caps units at 2^31 / 128).
+__device__ Unit find_unit(int ui, int stride, int n_units, const int32_t* cu, int n_seqs, int T,
+                          int H, int nch) {
   for (; ui < n_units; ui += stride) {
-    const int64_t slot = ui / H;
-    const int h = (int)(ui - slot * H);
+    const int slot = ui / H;
+    const int h = ui - slot * H;
     int64_t b, e, c;
     if (cu == nullptr) {
       if (nch <= 0) break;
-      const int n = (int)(slot / nch);
-      c = slot - (int64_t)n * nch;
+      const int n = slot / nch;
+      c = slot - n * nch;
       b = (int64_t)n * T;
       e = b + T;
     } else {
@@ -612,14 +614,14 @@ __device__ Unit find_unit(int64_t ui, int64_t stride, int64_t n_units, const int
       int lo = 0, hi = n_seqs - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if ((int64_t)(cu[mid] / C) + mid <= slot)
+        if (cu[mid] / C + mid <= slot)
           lo = mid;
         else
           hi = mid - 1;
       }
       b = cu[lo];
       e = cu[lo + 1];
-      c = slot - ((int64_t)(b / C) + lo);
+      c = slot - (b / C + lo);
       if (b < 0 || e < b || e > T || c < 0) continue;
     }
     const int64_t t0 = b + c * C;
@@ -746,7 +748,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   auto load_beta = [&](const Unit& uu) -> float {
     return (uu.idx >= 0 && tid < uu.Lc) ? beta[(size_t)(uu.t0 + tid) * H + uu.h] : 0.f;
   };
-  Unit cur = find_unit(blockIdx.x, gridDim.x, n_units, cu, n_seqs, T, H, nch);
+  Unit cur = find_unit(blockIdx.x, gridDim.x, (int)n_units, cu, n_seqs, T, H, nch);
   float beta_next = 0.f;
   if (cur.idx >= 0) {
     if (tid == 0) {
@@ -759,7 +761,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
   }
 
   for (int c = 0; cur.idx >= 0; ++c) {
-    const Unit nxt = find_unit(cur.idx + gridDim.x, gridDim.x, n_units, cu, n_seqs, T, H, nch);
+    const Unit nxt =
+        find_unit((int)cur.idx + gridDim.x, gridDim.x, (int)n_units, cu, n_seqs, T, H, nch);
     const bool more = nxt.idx >= 0;
     const int Lc = cur.Lc;
     const size_t u = (size_t)cur.idx;
@@ -914,8 +917,15 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     // ---- A -> fp16 operand; (I + T)^-1 by recursive doubling ------------------
     {
       const float* Af = reinterpret_cast<const float*>(sm + OFF_AF);
+      const float* Tf = reinterpret_cast<const float*>(sm + OFF_TF);
+      float* Inv = reinterpret_cast<float*>(sm + OFF_INV);
+      float* Yf = reinterpret_cast<float*>(sm + OFF_YF);
+      // One phase: A to its fp16 operand (one 8-column chunk per thread);
+      // zeros above the 8 x 8 block diagonal of Inv (what the merges read
+      // before they write it); the 8 x 8 diagonal blocks by forward
+      // substitution, one column per thread.
       {
-        const int r = tid >> 3, cg = tid & 7;  // 512 threads: one 8-column chunk each
+        const int r = tid >> 3, cg = tid & 7;
         const float4 lo = *reinterpret_cast<const float4*>(Af + fsw(r, 8 * cg));
         const float4 hi = *reinterpret_cast<const float4*>(Af + fsw(r, 8 * cg + 4));
         const float a8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
@@ -924,18 +934,11 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int t = 0; t < 8; ++t) v[t] = (8 * cg + t <= r) ? a8[t] : 0.f;
         st_chunk8(sm + OFF_AQ, sw128_chunk(r, 8 * cg, 64), v);
       }
-    }
-    __syncthreads();
-    {
-      const float* Tf = reinterpret_cast<const float*>(sm + OFF_TF);
-      float* Inv = reinterpret_cast<float*>(sm + OFF_AF);
-      float* Yf = reinterpret_cast<float*>(sm + OFF_YF);
-      {
-        uint4* z = reinterpret_cast<uint4*>(Inv);
-        for (int e = tid; e < 1024; e += NT1) z[e] = make_uint4(0u, 0u, 0u, 0u);
+      for (int e = tid; e < 64 * 16; e += NT1) {
+        const int r = e >> 4, c4 = e & 15;
+        if (c4 >= 2 * (r >> 3) + 2)
+          *reinterpret_cast<float4*>(Inv + fsw(r, 4 * c4)) = make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      __syncthreads();
-      // 8 x 8 diagonal blocks by forward substitution, one column per thread
       if (tid < 64) {
         const int base = 8 * (tid >> 3), cc = tid & 7;
         float tb[8][8];
