@@ -101,13 +101,12 @@ constexpr uint32_t OFF_KG = 143360;  // K * Gamma, fp16 MN-major [64 s][128 i]
 constexpr uint32_t OFF_QG = 159744;  // Q * Gamma, then Q', fp16 [64 r][128 i] (128B swizzle)
 constexpr uint32_t OFF_KH = 176128;  // K * rho, then W, fp16 [64][128 i] (128B swizzle)
 constexpr uint32_t OFF_GT = 192512;  // products of whole 4-position groups, fp32 [16][64]
-constexpr uint32_t OFF_T4 = 196608;  // products of aligned runs of 4 groups, fp32 [4][64]
-constexpr uint32_t OFF_T8 = 197632;  // products of aligned runs of 8 groups, fp32 [2][64]
-constexpr uint32_t OFF_PR = 198144;  // direct pairs and diag(A), fp32 [16 groups][16]
-constexpr uint32_t OFF_BETA = 199168;
-constexpr uint32_t OFF_GAMMA = 199424;
-constexpr uint32_t OFF_BAR = 199936;  // mbarriers: in0, in1, v, mma, lv
-constexpr uint32_t OFF_TMEMPTR = 200000;
+constexpr uint32_t OFF_T2 = 196608;  // products of aligned pairs of groups, fp32 [8][64]
+constexpr uint32_t OFF_PR = 198656;  // direct pairs and diag(A), fp32 [16 groups][16]
+constexpr uint32_t OFF_BETA = 199680;
+constexpr uint32_t OFF_GAMMA = 199936;
+constexpr uint32_t OFF_BAR = 200448;  // mbarriers: in0, in1, v, mma, lv
+constexpr uint32_t OFF_TMEMPTR = 200512;
 constexpr uint32_t OFF_INV = 200704;  // (I + T)^-1, fp32 [64][64] (swizzled)
 constexpr uint32_t kSmemUsed = OFF_INV + 16384;
 constexpr size_t kSmemBytes = kSmemUsed + 1024;
@@ -320,14 +319,18 @@ __device__ __forceinline__ int level_row(int lv, int p) {
 // halves of levels 2..5); role 1 walks backward (suffix products: rho and the
 // left halves) and adds its channels' share of the direct pairs of levels
 // 0..1 (inside its block of 4) and of diag(A) into the pair buffer (stored by
-// half 0, added by half 1).  The products of whole groups, and of aligned
-// runs of 4 and 8 groups, are formed once and exchanged through shared
-// memory, so every anchored offset costs at most five loads.  The role is the
-// warp's parity, so the warps sharing a scheduler run the same code; one
-// out-of-line copy serves both halves.
+// half 0, added by half 1).  The products of whole groups and of aligned
+// pairs of groups are formed once and exchanged through shared memory, so
+// every anchored offset costs a handful of loads.  A warp holds groups 2k and
+// 2k + 1 of one role; each scheduler (warps w, w + 4, w + 8, w + 12) gets
+// both roles and the complementary pairs k and 7 - k, whose level work adds
+// up to the same amount on every scheduler.  One out-of-line copy serves
+// both halves.
 __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid) {
-  const int role = (tid >> 5) & 1;
-  const int rt = ((tid >> 6) << 5) | (tid & 31);  // index among the 256 threads of this role
+  const int w = tid >> 5;
+  const int role = (w >> 2) & 1;
+  const int kk = (w < 8) ? (w & 3) : 7 - (w & 3);
+  const int rt = (kk << 5) | (tid & 31);  // index among the 256 threads of this role
   const int c4 = rt & 15;
   const int g = rt >> 4;
   const int cl = 4 * c4;
@@ -361,33 +364,28 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
 #ifdef CKDA_TC_DEBUG
   long long gp_last = clock64();
 #endif
-  // products of whole groups, then of aligned runs of 4 and 8 groups
+  // products of whole groups, and (one shuffle across the two groups of a
+  // warp) of aligned pairs of groups
   const uint32_t gt = sb + OFF_GT + cl * 4;
-  if (role == 0) sts_f4(gt + g * 256, mul4(mul4(aa[0], aa[1]), mul4(aa[2], aa[3])));
-  __syncthreads();
-  if (tid < 96) {
-    const int sc = tid & 15, seg = tid >> 4;
-    const uint32_t src = sb + OFF_GT + sc * 16;
-    if (seg < 4) {
-      const float4 x = mul4(mul4(lds_f4(src + (4 * seg) * 256), lds_f4(src + (4 * seg + 1) * 256)),
-                            mul4(lds_f4(src + (4 * seg + 2) * 256), lds_f4(src + (4 * seg + 3) * 256)));
-      sts_f4(sb + OFF_T4 + seg * 256 + sc * 16, x);
-    } else {
-      const int b8 = 8 * (seg - 4);
-      float4 x[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = lds_f4(src + (b8 + j) * 256);
-      const float4 y = mul4(mul4(mul4(x[0], x[1]), mul4(x[2], x[3])),
-                            mul4(mul4(x[4], x[5]), mul4(x[6], x[7])));
-      sts_f4(sb + OFF_T8 + (seg - 4) * 256 + sc * 16, y);
-    }
+  if (role == 0) {
+    const float4 t = mul4(mul4(aa[0], aa[1]), mul4(aa[2], aa[3]));
+    sts_f4(gt + g * 256, t);
+    float4 o;
+    o.x = __shfl_xor_sync(0xffffffffu, t.x, 16);
+    o.y = __shfl_xor_sync(0xffffffffu, t.y, 16);
+    o.z = __shfl_xor_sync(0xffffffffu, t.z, 16);
+    o.w = __shfl_xor_sync(0xffffffffu, t.w, 16);
+    if (!(g & 1)) sts_f4(sb + OFF_T2 + (g >> 1) * 256 + cl * 4, mul4(t, o));
   }
   GP_MARK(0);
   __syncthreads();
   GP_MARK(1);
   auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * 256); };
-  auto run4 = [&](int s4) -> float4 { return lds_f4(sb + OFF_T4 + s4 * 256 + cl * 4); };
-  auto run8 = [&](int s8) -> float4 { return lds_f4(sb + OFF_T8 + s8 * 256 + cl * 4); };
+  auto run2 = [&](int s2) -> float4 { return lds_f4(sb + OFF_T2 + s2 * 256 + cl * 4); };
+  auto run4 = [&](int s4) -> float4 { return mul4(run2(2 * s4), run2(2 * s4 + 1)); };
+  auto run8 = [&](int s8) -> float4 {
+    return mul4(mul4(run2(4 * s8), run2(4 * s8 + 1)), mul4(run2(4 * s8 + 2), run2(4 * s8 + 3)));
+  };
   const uint32_t LV = sb + OFF_LVX;
 
   // Store addresses: every tile written here has 128-byte rows (64 fp16 of
