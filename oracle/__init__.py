@@ -14,6 +14,12 @@ Contents
     ``o_t = S_t^T q_t`` ("Complex KDA ..." page, section "Complex KDA (CKDA)
     Mimarisi ve Parametre Genislemesi"; "Gated DeltaNet-2" page, Methodology
     section 1 with b_t = w_t = beta_t).
+``forward_gdn2``
+    The Gated DeltaNet-2 recurrence ("Gated DeltaNet-2" page, Methodology
+    section 1): the same loop with an erase gate b_t (key side) and a write
+    gate w_t (value side) in place of beta_t,
+    ``S_t = (I - k_t (b_t . k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T``;
+    pinned by ``tests/pinlib_gdn2.py`` (G-1..G-7).
 ``chunked`` (submodule)
     A plain numpy fp64 restatement of the chunkwise WY form, used only to pin
     the chunked algorithm against the sequential loop on tiny inputs.
@@ -62,6 +68,11 @@ def _load():
                 dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
             ]
             lib.ckda_oracle_forward.restype = ctypes.c_int
+            lib.ckda_oracle_gdn2_forward.argtypes = [
+                i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int64),
+                dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
+            ]
+            lib.ckda_oracle_gdn2_forward.restype = ctypes.c_int
             lib.ckda_oracle_decode_step.argtypes = [
                 i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
             ]
@@ -132,6 +143,45 @@ def forward(q, k, v, alpha, beta, S0=None, cu_seqlens=None, n_threads=None):
     )
     if rc != 0:
         raise ValueError("ckda_oracle_forward rejected its arguments")
+    return out.reshape(out_shape), S_final
+
+
+def forward_gdn2(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, n_threads=None):
+    """Sequential fp64 Gated DeltaNet-2 forward ("Gated DeltaNet-2" summary,
+    Methodology section 1): the CKDA recurrence with the scalar beta replaced
+    by an erase gate ``b`` (shaped like ``k``) and a write gate ``w`` (shaped
+    like ``v``).  Other arguments and the result as in ``forward``."""
+    qd, kd, vd, ad, bgd, wgd = (_f64(t) for t in (q, k, v, alpha, b, w))
+    out_shape = vd.shape
+    if cu_seqlens is None:
+        if qd.ndim != 4:
+            raise ValueError("fixed-length batch expects [B, T, H, d] tensors")
+        B, T, H, dk = qd.shape
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int64))
+        if qd.ndim == 4:
+            if qd.shape[0] != 1:
+                raise ValueError("packed batch expects a leading dimension of 1")
+            qd, kd, vd, ad, bgd, wgd = qd[0], kd[0], vd[0], ad[0], bgd[0], wgd[0]
+        H, dk = qd.shape[1], qd.shape[2]
+    N = len(cu) - 1
+    dv = vd.shape[-1]
+    T_total = int(cu[-1])
+    qd, kd, ad, bgd = (x.reshape(T_total, H, dk) for x in (qd, kd, ad, bgd))
+    vd, wgd = (x.reshape(T_total, H, dv) for x in (vd, wgd))
+    S0d = None if S0 is None else _f64(S0).reshape(N, H, dk, dv)
+    out = np.zeros((T_total, H, dv), dtype=np.float64)
+    S_final = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().ckda_oracle_gdn2_forward(
+        N, H, dk, dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(qd), _ptr(kd), _ptr(vd), _ptr(ad), _ptr(bgd), _ptr(wgd), _ptr(S0d),
+        _ptr(out), _ptr(S_final), int(n_threads or default_threads()),
+    )
+    if rc != 0:
+        raise ValueError("ckda_oracle_gdn2_forward rejected its arguments")
     return out.reshape(out_shape), S_final
 
 

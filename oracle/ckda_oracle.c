@@ -35,6 +35,20 @@
  *   beta        : [T_total, H]
  *   S0, S_final : [N, H, dk, dv]       (S0 may be NULL: zero initial state)
  *   cu_seqlens  : int64 [N + 1], sequence n spans tokens [cu[n], cu[n+1])
+ *
+ * The Gated DeltaNet-2 form (ckda_oracle_gdn2_forward) replaces the scalar
+ * beta_t by an erase gate b_t in [0, 1]^dk on the key side and a write gate
+ * w_t in [0, 1]^dv on the value side ("Gated DeltaNet-2" technical summary,
+ * Methodology section 1):
+ *
+ *   S_t = (I - k_t (b_t . k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T
+ *
+ * with the same read-out; its body, in the order of that equation:
+ *   1. S <- Diag(alpha) S
+ *   2. r <- S^T e,  e = b . k         (the erased read)
+ *   3. S <- S + k (z - r)^T,  z = w . v
+ *   4. o <- S^T q
+ *   b : [T_total, H, dk]   w : [T_total, H, dv]
  */
 #include <pthread.h>
 #include <stdint.h>
@@ -45,6 +59,7 @@ typedef struct {
     int64_t n_seqs, H, dk, dv;
     const int64_t *cu;
     const double *q, *k, *v, *alpha, *beta, *S0;
+    const double *eg, *wg; /* Gated DeltaNet-2 gates (NULL for the beta form) */
     double *out, *S_final;
     int64_t next_unit; /* shared work counter (guarded by lock) */
     pthread_mutex_t lock;
@@ -88,6 +103,45 @@ static void run_unit(const oracle_job *J, int64_t n, int64_t h, double *S,
                sizeof(double) * dk * dv);
 }
 
+/* One (sequence, head) unit of the Gated DeltaNet-2 recurrence. */
+static void run_unit_gdn2(const oracle_job *J, int64_t n, int64_t h, double *S,
+                          double *r) {
+    const int64_t H = J->H, dk = J->dk, dv = J->dv;
+    if (J->S0) {
+        memcpy(S, J->S0 + ((n * H + h) * dk) * dv, sizeof(double) * dk * dv);
+    } else {
+        memset(S, 0, sizeof(double) * dk * dv);
+    }
+    for (int64_t t = J->cu[n]; t < J->cu[n + 1]; ++t) {
+        const double *q = J->q + (t * H + h) * dk;
+        const double *k = J->k + (t * H + h) * dk;
+        const double *a = J->alpha + (t * H + h) * dk;
+        const double *b = J->eg + (t * H + h) * dk;
+        const double *v = J->v + (t * H + h) * dv;
+        const double *w = J->wg + (t * H + h) * dv;
+        double *o = J->out + (t * H + h) * dv;
+
+        /* 1. S <- Diag(alpha) S */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) S[i * dv + j] *= a[i];
+        /* 2. r <- S^T (b . k) */
+        for (int64_t j = 0; j < dv; ++j) r[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * (b[i] * k[i]);
+        /* 3. S <- S + k (w . v - r)^T */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j)
+                S[i * dv + j] += k[i] * (w[j] * v[j] - r[j]);
+        /* 4. o <- S^T q */
+        for (int64_t j = 0; j < dv; ++j) o[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) o[j] += S[i * dv + j] * q[i];
+    }
+    if (J->S_final)
+        memcpy(J->S_final + ((n * H + h) * dk) * dv, S,
+               sizeof(double) * dk * dv);
+}
+
 static void *worker(void *arg) {
     oracle_job *J = (oracle_job *)arg;
     double *S = (double *)malloc(sizeof(double) * J->dk * J->dv);
@@ -98,11 +152,29 @@ static void *worker(void *arg) {
         int64_t u = J->next_unit++;
         pthread_mutex_unlock(&J->lock);
         if (u >= n_units) break;
-        run_unit(J, u / J->H, u % J->H, S, r);
+        if (J->eg)
+            run_unit_gdn2(J, u / J->H, u % J->H, S, r);
+        else
+            run_unit(J, u / J->H, u % J->H, S, r);
     }
     free(S);
     free(r);
     return NULL;
+}
+
+/* Share the (sequence, head) units of a job out to n_threads host threads. */
+static void run_job(oracle_job *J, int n_threads) {
+    J->next_unit = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    if (n_threads < 1) n_threads = 1;
+    if (n_threads > 256) n_threads = 256;
+    pthread_t tid[256];
+    int started = 0;
+    for (int i = 1; i < n_threads; ++i)
+        if (pthread_create(&tid[started], NULL, worker, J) == 0) ++started;
+    worker(J);
+    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
+    pthread_mutex_destroy(&J->lock);
 }
 
 /*
@@ -132,20 +204,48 @@ int ckda_oracle_forward(int64_t n_seqs, int64_t H, int64_t dk, int64_t dv,
     J.v = v;
     J.alpha = alpha;
     J.beta = beta;
+    J.eg = NULL;
+    J.wg = NULL;
     J.S0 = S0;
     J.out = out;
     J.S_final = S_final;
-    J.next_unit = 0;
-    pthread_mutex_init(&J.lock, NULL);
-    if (n_threads < 1) n_threads = 1;
-    if (n_threads > 256) n_threads = 256;
-    pthread_t tid[256];
-    int started = 0;
-    for (int i = 1; i < n_threads; ++i)
-        if (pthread_create(&tid[started], NULL, worker, &J) == 0) ++started;
-    worker(&J);
-    for (int i = 0; i < started; ++i) pthread_join(tid[i], NULL);
-    pthread_mutex_destroy(&J.lock);
+    run_job(&J, n_threads);
+    return 0;
+}
+
+/*
+ * Sequential Gated DeltaNet-2 forward over a packed batch (layouts as
+ * above, with the gates b [T_total, H, dk] and w [T_total, H, dv] in place
+ * of beta).  Returns 0 on success, -1 on an argument error.
+ */
+int ckda_oracle_gdn2_forward(int64_t n_seqs, int64_t H, int64_t dk, int64_t dv,
+                             const int64_t *cu_seqlens, const double *q,
+                             const double *k, const double *v,
+                             const double *alpha, const double *b,
+                             const double *w, const double *S0, double *out,
+                             double *S_final, int n_threads) {
+    if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens || !b || !w)
+        return -1;
+    if (cu_seqlens[0] != 0) return -1;
+    for (int64_t n = 0; n < n_seqs; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    oracle_job J;
+    J.n_seqs = n_seqs;
+    J.H = H;
+    J.dk = dk;
+    J.dv = dv;
+    J.cu = cu_seqlens;
+    J.q = q;
+    J.k = k;
+    J.v = v;
+    J.alpha = alpha;
+    J.beta = NULL;
+    J.eg = b;
+    J.wg = w;
+    J.S0 = S0;
+    J.out = out;
+    J.S_final = S_final;
+    run_job(&J, n_threads);
     return 0;
 }
 
