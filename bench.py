@@ -42,6 +42,8 @@ BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4          # q,k,v bf16 + alp
 STRICT_FLOPS_PER_TOKEN_HEAD = 6 * CHUNK * D + 6 * D * D + CHUNK * CHUNK // 3
 DENSE_FLOPS_PER_TOKEN_HEAD = 12 * CHUNK * D + 6 * D * D
 DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4
+# Gated DeltaNet-2 forward: q, k, v bf16 + alpha, b (d_k) and w (d_v) fp32 + out fp32
+GDN2_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + D * 4 + D * 4 + D * 4
 
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
@@ -67,6 +69,8 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS,
                     help="decode steps timed (inputs for all of them are pre-generated)")
+    ap.add_argument("--no-gdn2", action="store_true",
+                    help="skip the Gated DeltaNet-2 forward measurement")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -301,6 +305,9 @@ def run_ours(args, ws, rank, local):
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
+    gdn2 = None
+    if not args.no_gdn2:
+        gdn2 = _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak)
     wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
                         device=dev)
     two_phase = path == "tcgen05"
@@ -382,7 +389,7 @@ def run_ours(args, ws, rank, local):
                              ws, hbm_peak)
     _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            _lib.LIB_PATH, path, kernels)
+            _lib.LIB_PATH, path, kernels, gdn2)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -424,6 +431,44 @@ def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, t
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
+def _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=20):
+    """Gated DeltaNet-2 forward at the bench sizes (bf16 q/k/v, fp32 gates and
+    output), on the fp32 CUDA-core kernel; two rotating input sets."""
+    sets = [inputs.gdn2_prefill(B, T, H, D, D, dtype=torch.bfloat16, chunk=CHUNK,
+                                seed=3000 + 10 * rank + i, device=dev) for i in range(2)]
+    out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
+    S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+
+    def step(i):
+        c = sets[i % 2]
+        ck.gdn2_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], chunk=CHUNK,
+                            out=out, S_final=S_final)
+
+    for i in range(3):
+        step(i)
+    torch.cuda.synchronize(dev)
+    assert ck.device_status(dev) == 0
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for i in range(steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_ranks(ev0.elapsed_time(ev1)) / steps
+    nbytes = B * T * H * GDN2_BYTES_PER_TOKEN_HEAD + B * H * D * D * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del sets
+    return {"workload": f"gdn2_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 "
+                        "alpha/b/w, fp32 out (fp32 CUDA-core kernel)",
+            "ms_per_step": ms, "tokens_per_s": ws * B * T / (ms / 1e3),
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+            "hbm_frac_of_measured": gbs / hbm_peak, "gpu_launches": steps}
+
+
 def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak):
     steps = max(1, args.decode_steps)
     ev0 = torch.cuda.Event(enable_timing=True)
@@ -456,7 +501,7 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, 
 
 def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            lib_path, path, kernels=None):
+            lib_path, path, kernels=None, gdn2=None):
     # arithmetic of the forward: tcgen05 MMAs on fp16 operands with fp32
     # accumulation and fp32 state, or fp32 FFMA on CUDA cores
     dtype = "f16" if path == "tcgen05" else "f32"
@@ -493,6 +538,8 @@ def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_
     }
     if decode is not None:
         obj["decode"] = decode
+    if gdn2 is not None:
+        obj["gdn2"] = gdn2
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         obj["cpu_baseline"] = cpu_baseline()
     _emit(obj, args, rank)

@@ -8,12 +8,12 @@ without the native library.
 """
 from __future__ import annotations
 
-__all__ = ["fwd_chunked", "fwd_chunked_static", "fwd_factors", "fwd_carry", "fwd_path", "workspace_bytes", "decode_step",
+__all__ = ["fwd_chunked", "fwd_chunked_static", "gdn2_fwd_chunked", "fwd_factors", "fwd_carry", "fwd_path", "workspace_bytes", "decode_step",
            "device_status", "CKDAError", "lib_path"]
 
 
 def __getattr__(name):
-    if name in ("fwd_chunked", "fwd_chunked_static", "fwd_factors", "fwd_carry", "fwd_path", "workspace_bytes",
+    if name in ("fwd_chunked", "fwd_chunked_static", "gdn2_fwd_chunked", "fwd_factors", "fwd_carry", "fwd_path", "workspace_bytes",
                 "decode_step", "device_status"):
         from . import api
 

@@ -216,6 +216,46 @@ def fwd_carry(workspace, B, T, H, dk, dv, S0=None, cu_seqlens=None, chunk: int =
     return out, S_final
 
 
+def gdn2_fwd_chunked(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk: int = 64,
+                     out=None, S_final=None, return_final: bool = True, out_dtype=None):
+    """Chunked Gated DeltaNet-2 forward (``ckda_gdn2_fwd_chunked``): CKDA with an
+    erase gate ``b`` (fp32, shaped like ``k``) and a write gate ``w`` (fp32, shaped
+    like ``v``) in place of beta.  Other arguments and the result as in
+    ``fwd_chunked``."""
+    dev = q.device
+    _need(b, "b", torch.float32, dev)
+    _need(w, "w", torch.float32, dev)
+    if b.shape != k.shape or w.shape != v.shape:
+        raise ValueError("b must have k's shape and w v's shape")
+    beta_like = b[..., 0]  # shape check only: [B, T, H] or [T, H]
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta_like.contiguous(), cu_seqlens)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must have v's shape")
+    if return_final and S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_gdn2_fwd_chunked(
+            _p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), _p(S0), _p(cu_seqlens), _p(out),
+            _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype], _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_gdn2_fwd_chunked")
+    return out, S_final
+
+
 def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, out_dtype=torch.float32,
                     varlen=False) -> int:
     """Scratch bytes ``fwd_chunked`` needs for these sizes (0 on the fp32 CUDA-core path)."""

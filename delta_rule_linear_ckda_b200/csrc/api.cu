@@ -14,8 +14,9 @@ cudaError_t launch_decode(int dtype, int out_dtype, int dk, int dv, const void* 
                           int BH, cudaStream_t stream);
 cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
                             const void* k, const void* v, const float* alpha, const float* beta,
-                            const float* S0, const int32_t* cu, void* out, float* S_final,
-                            int n_seqs, int T, int H, int C, int* status, cudaStream_t stream);
+                            const float* bg, const float* wg, const float* S0,
+                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T,
+                            int H, int C, int* status, cudaStream_t stream);
 // Returns cudaErrorNotSupported when the shape is not covered by the
 // tensor-core kernels (the caller then uses the CUDA-core kernel).
 cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
@@ -137,8 +138,8 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
     e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu,
                             out, S_final, n_seqs, T, H, chunk, workspace, status, st);
   if (e == cudaErrorNotSupported)
-    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu, out, S_final,
-                              n_seqs, T, H, chunk, status, st);
+    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, nullptr, nullptr,
+                              S0, cu, out, S_final, n_seqs, T, H, chunk, status, st);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
@@ -197,6 +198,27 @@ int ckda_fwd_chunked_static(const void* q, const void* k, const void* v, const f
   return fwd_impl(true, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
                   d_v, chunk, dtype, out_dtype, ws, need > 0 ? (size_t)CKDA_STATIC_SCRATCH_BYTES : 0,
                   stream);
+}
+
+int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* b, const float* w, const float* S0,
+                          const int32_t* cu_seqlens, void* out, float* S_final, int B, int T, int H,
+                          int d_k, int d_v, int chunk, int dtype, int out_dtype, void* stream) {
+  // the erase gate takes beta's place in the shared checks; the write gate is checked here
+  int rc = validate_fwd(q, k, v, alpha, b, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
+                        &chunk, dtype, out_dtype);
+  if (rc != CKDA_OK) return rc;
+  const int64_t tokens = (cu_seqlens != nullptr) ? (int64_t)T : (int64_t)B * T;
+  if (tokens > 0 && w == nullptr) return CKDA_ERR_INVALID_ARG;
+  if (w != nullptr && !aligned16(w)) return CKDA_ERR_MISALIGNED;
+  if (out != nullptr && out == w) return CKDA_ERR_INVALID_ARG;
+  if (B == 0) return CKDA_OK;  // (zero-length sequences still store S_final = S0)
+  int* status = status_ptr();
+  if (status == nullptr) return CKDA_ERR_CUDA;
+  cudaError_t e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, nullptr, b, w,
+                                        S0, cu_seqlens, out, S_final, B, T, H, chunk, status,
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
 int ckda_fwd_factors(const void* q, const void* k, const void* v, const float* alpha,

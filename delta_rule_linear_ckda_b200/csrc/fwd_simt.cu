@@ -19,6 +19,13 @@
 // Positions past the end of a sequence are identity transitions
 // (alpha = 1, beta = 0, q = k = v = 0) and produce no output.
 //
+// Gated DeltaNet-2 ("Gated DeltaNet-2" page, Methodology section 1) replaces
+// beta_r by an erase gate b_r in [0, 1]^d_k on the key side and a write gate
+// w_r in [0, 1]^d_v on the value side.  The same derivation then gives, with
+// E = B * K and Z = W_g * V (rows e_r = b_r * k_r, z_r = w_r * v_r):
+//   T[r, s] = sum_i e_ri k_si P_i(r, s),   [W | U~] = (I + T)^-1 [E * Gamma | Z]
+// and everything else unchanged; the G2 instantiation computes that form.
+//
 // One CTA owns one (sequence, head, d_v slice of width BV) and walks its
 // chunks in order; the slice of the state stays in shared memory in fp32.
 #include "common.cuh"
@@ -99,20 +106,21 @@ __device__ __forceinline__ void reduce_scatter8(float* v, int lane) {
   v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
 }
 
-template <int DK, int BV, typename Tin, typename Tout>
+template <int DK, int BV, typename Tin, typename Tout, bool G2>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta,
-                const float* S0, const int32_t* __restrict__ cu, Tout* __restrict__ out,
-                float* S_final, int n_seqs, int T, int H, int DV, int C, int* status) {
+                const float* __restrict__ bg, const float* __restrict__ wg, const float* S0,
+                const int32_t* __restrict__ cu, Tout* __restrict__ out, float* S_final,
+                int n_seqs, int T, int H, int DV, int C, int* status) {
   using L = Smem<DK, BV>;
   constexpr int KS = L::KS, VS = L::VS, CS = L::CS;
   extern __shared__ __align__(16) float smem[];
   float* Ks = smem + L::kK;   // k, then K * rho
   float* Qs = smem + L::kQ;   // q, then Q * Gamma
   float* As = smem + L::kA;   // alpha
-  float* Ws = smem + L::kW;   // beta K Gamma, then W
-  float* Vs = smem + L::kV;   // v, then beta v, then U~, then U
+  float* Ws = smem + L::kW;   // beta K Gamma, then W (G2: E = b * k, then E * Gamma, then W)
+  float* Vs = smem + L::kV;   // v, then beta v (G2: w * v), then U~, then U
   float* Tm = smem + L::kT;   // T (strictly lower)
   float* Am = smem + L::kAm;  // A (lower incl. diagonal)
   float* Ss = smem + L::kS;   // state slice [DK][BV]
@@ -145,12 +153,18 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     for (int e = tid; e < C * DK / 4; e += kThreads) {
       const int r = e / (DK / 4), c4 = e % (DK / 4);
       float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk, aa = make_float4(1.f, 1.f, 1.f, 1.f);
+      float4 ee = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < Lc) {
         const size_t off = ((size_t)(t0 + r) * H + h) * DK + 4 * c4;
         kk = load4_f32(k + off);
         qq = load4_f32(q + off);
         aa = *reinterpret_cast<const float4*>(alpha + off);
+        if constexpr (G2) {
+          const float4 bb = *reinterpret_cast<const float4*>(bg + off);
+          ee = make_float4(bb.x * kk.x, bb.y * kk.y, bb.z * kk.z, bb.w * kk.w);
+        }
       }
+      if constexpr (G2) *reinterpret_cast<float4*>(Ws + r * KS + 4 * c4) = ee;
       *reinterpret_cast<float4*>(Ks + r * KS + 4 * c4) = kk;
       *reinterpret_cast<float4*>(Qs + r * KS + 4 * c4) = qq;
       *reinterpret_cast<float4*>(As + r * KS + 4 * c4) = aa;
@@ -158,17 +172,27 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     for (int e = tid; e < C * BV / 4; e += kThreads) {
       const int r = e / (BV / 4), c4 = e % (BV / 4);
       float4 vv = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < Lc) vv = load4_f32(v + ((size_t)(t0 + r) * H + h) * DV + j0 + 4 * c4);
+      if (r < Lc) {
+        const size_t voff = ((size_t)(t0 + r) * H + h) * DV + j0 + 4 * c4;
+        vv = load4_f32(v + voff);
+        if constexpr (G2) {
+          const float4 ww = *reinterpret_cast<const float4*>(wg + voff);
+          vv = make_float4(ww.x * vv.x, ww.y * vv.y, ww.z * vv.z, ww.w * vv.w);
+        }
+      }
       *reinterpret_cast<float4*>(Vs + r * VS + 4 * c4) = vv;
     }
-    for (int r = tid; r < C; r += kThreads)
-      bs[r] = (r < Lc) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    if constexpr (!G2) {
+      for (int r = tid; r < C; r += kThreads)
+        bs[r] = (r < Lc) ? beta[(size_t)(t0 + r) * H + h] : 0.f;
+    }
     __syncthreads();
 
     // ---- score blocks T and A: one warp per column s ------------------
     // x = k_s * P(r, s) is carried down the rows r > s by multiplying with
-    // alpha_r; the dot products with k_r and q_r give T[r, s] / beta_r and
-    // A[r, s].  Lanes split the channels; eight rows are reduced at once.
+    // alpha_r; the dot products with k_r (G2: e_r) and q_r give T[r, s] /
+    // beta_r (G2: T[r, s]) and A[r, s].  Lanes split the channels; eight rows
+    // are reduced at once.
     {
       using LC = LaneChannels<DK>;
       constexpr int CPL = LC::kPer;
@@ -200,7 +224,7 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
               for (int c = 0; c < CPL; ++c) { a[c] = 1.f; kr[c] = 0.f; qr[c] = 0.f; }
               if (act) {
                 lds<CPL>(As + r * KS + cb, a);
-                lds<CPL>(Ks + r * KS + cb, kr);
+                lds<CPL>((G2 ? Ws : Ks) + r * KS + cb, kr);
                 lds<CPL>(Qs + r * KS + cb, qr);
               }
 #pragma unroll
@@ -215,7 +239,7 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
           reduce_scatter8(pq, lane);
           const int r = rb + (lane & 7);
           if (lane < 8 && r < C) {
-            Tm[r * CS + s] = bs[r] * pk[0];
+            Tm[r * CS + s] = G2 ? pk[0] : bs[r] * pk[0];
             Am[r * CS + s] = pq[0];
           }
         }
@@ -224,14 +248,18 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     __syncthreads();
 
     // ---- gate products: one thread per channel ------------------------
-    // forward: Gamma_r (inclusive prefix); W rhs = beta K Gamma; Q <- Q Gamma
+    // forward: Gamma_r (inclusive prefix); W rhs = beta K Gamma (G2: E Gamma);
+    // Q <- Q Gamma
     // backward: rho_s (exclusive suffix); K <- K rho
     if (tid < DK) {
       const int i = tid;
       float gmm = 1.f;
       for (int r = 0; r < C; ++r) {
         gmm *= As[r * KS + i];
-        Ws[r * KS + i] = bs[r] * Ks[r * KS + i] * gmm;
+        if constexpr (G2)
+          Ws[r * KS + i] *= gmm;
+        else
+          Ws[r * KS + i] = bs[r] * Ks[r * KS + i] * gmm;
         Qs[r * KS + i] *= gmm;
       }
       gs[i] = gmm;
@@ -241,13 +269,16 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
         p *= As[s * KS + i];
       }
     }
-    for (int e = tid; e < C * BV; e += kThreads) {
-      const int r = e / BV, c = e % BV;
-      Vs[r * VS + c] *= bs[r];
+    if constexpr (!G2) {
+      for (int e = tid; e < C * BV; e += kThreads) {
+        const int r = e / BV, c = e % BV;
+        Vs[r * VS + c] *= bs[r];
+      }
     }
     __syncthreads();
 
     // ---- WY factors: [W | U~] = (I + T)^-1 [beta K Gamma | beta V] -----
+    // (G2: (I + T)^-1 [E Gamma | Z])
     // Forward substitution, one thread per column, 16 rows at a time in
     // registers: rows of earlier blocks are final when a block starts.
     if (tid < DK + BV) {
@@ -367,50 +398,63 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
   }
 }
 
-template <int DK, int BV, typename Tin, typename Tout>
+// Gates of a call: beta (CKDA) or the erase and write gates (G2).
+struct Gates {
+  const float* beta;
+  const float* b;
+  const float* w;
+};
+
+template <int DK, int BV, typename Tin, typename Tout, bool G2>
 static cudaError_t launch_t(const void* q, const void* k, const void* v, const float* alpha,
-                            const float* beta, const float* S0, const int32_t* cu, void* out,
+                            Gates gt, const float* S0, const int32_t* cu, void* out,
                             float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
                             cudaStream_t stream) {
   using L = Smem<DK, BV>;
-  auto kern = fwd_simt_kernel<DK, BV, Tin, Tout>;
+  auto kern = fwd_simt_kernel<DK, BV, Tin, Tout, G2>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(DV / BV, H, n_seqs);
   kern<<<grid, kThreads, L::kBytes, stream>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
-      beta, S0, cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
+      gt.beta, gt.b, gt.w, S0, cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
   return cudaGetLastError();
 }
 
-template <int DK, typename Tin, typename Tout>
+template <int DK, typename Tin, typename Tout, bool G2>
 static cudaError_t launch_bv(const void* q, const void* k, const void* v, const float* alpha,
-                             const float* beta, const float* S0, const int32_t* cu, void* out,
+                             Gates gt, const float* S0, const int32_t* cu, void* out,
                              float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
                              cudaStream_t stream) {
   switch (DV) {
     case 16:
-      return launch_t<DK, 16, Tin, Tout>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
-                                   C, status, stream);
+      return launch_t<DK, 16, Tin, Tout, G2>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
+                                             DV, C, status, stream);
     case 32:
-      return launch_t<DK, 32, Tin, Tout>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
-                                   C, status, stream);
+      return launch_t<DK, 32, Tin, Tout, G2>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
+                                             DV, C, status, stream);
     default:  // 64 and 128: slices of 64 columns
-      return launch_t<DK, 64, Tin, Tout>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, DV,
-                                   C, status, stream);
+      return launch_t<DK, 64, Tin, Tout, G2>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
+                                             DV, C, status, stream);
   }
 }
 
 }  // namespace simt
 
+// `bg` and `wg` non-NULL select the Gated DeltaNet-2 form (beta unused).
 cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
                             const void* k, const void* v, const float* alpha, const float* beta,
-                            const float* S0, const int32_t* cu, void* out, float* S_final,
-                            int n_seqs, int T, int H, int C, int* status, cudaStream_t stream) {
-#define CKDA_SIMT_CALL(DKV, TI, TO)                                                           \
-  simt::launch_bv<DKV, TI, TO>(q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs, T, H, dv, C, \
-                               status, stream)
+                            const float* bg, const float* wg, const float* S0,
+                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T,
+                            int H, int C, int* status, cudaStream_t stream) {
+  const simt::Gates gt{beta, bg, wg};
+  const bool g2 = bg != nullptr;
+#define CKDA_SIMT_CALL(DKV, TI, TO)                                                            \
+  (g2 ? simt::launch_bv<DKV, TI, TO, true>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, \
+                                           H, dv, C, status, stream)                           \
+      : simt::launch_bv<DKV, TI, TO, false>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs,   \
+                                            T, H, dv, C, status, stream))
 #define CKDA_SIMT_DK(DKV)                                                                  \
   case DKV:                                                                                \
     if (dtype == CKDA_BF16)                                                                \

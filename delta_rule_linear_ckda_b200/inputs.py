@@ -134,6 +134,28 @@ def random_prefill(B, T, H, dk, dv, *, dtype=F32, gates="uniform", s0_std=0.0,
     return PrefillCase(name, q, k, v, alpha.contiguous(), beta.contiguous(), S0, None, chunk)
 
 
+def gdn2_prefill(B, T, H, dk, dv, *, dtype=F32, s0_std=0.0, chunk=64, seed=0, device="cpu",
+                 name="gdn2") -> PrefillCase:
+    """Gated DeltaNet-2 batch: q, k normalised, v ~ N(0,1), alpha as the KDA
+    prefill recipe, erase gate b = sigmoid(x) per key channel and write gate
+    w = sigmoid(y) per value channel (both in [0, 1]), x, y ~ N(0,1).  The
+    gates go to ``extra["b"]`` and ``extra["w"]``; ``beta`` is unused (None)."""
+    g = _gen(device, seed)
+    q = _l2n(_normal((B, T, H, dk), g, device)).to(dtype)
+    k = _l2n(_normal((B, T, H, dk), g, device)).to(dtype)
+    v = _normal((B, T, H, dv), g, device).to(dtype)
+    alpha, _ = _kda_gates((B, T, H, dk), (B, T, H), g, device)
+    b = torch.sigmoid(_normal((B, T, H, dk), g, device)).to(F32).contiguous()
+    w = torch.sigmoid(_normal((B, T, H, dv), g, device)).to(F32).contiguous()
+    S0 = None
+    if s0_std > 0:
+        S0 = (_normal((B, H, dk, dv), g, device) * s0_std).contiguous()
+    case = PrefillCase(name, q, k, v, alpha.contiguous(), None, S0, None, chunk)
+    case.extra["b"] = b
+    case.extra["w"] = w
+    return case
+
+
 def tiny(seed=0, device="cpu") -> PrefillCase:
     return random_prefill(1, 64, 2, 16, 16, dtype=F32, gates="uniform", chunk=16,
                           seed=seed, device=device, name="tiny B=1 H=2 T=64 d=16 C=16 fp32")

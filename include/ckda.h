@@ -202,6 +202,34 @@ CKDA_API int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* ou
                             size_t workspace_bytes, void* stream);
 
 /*
+ * ckda_gdn2_fwd_chunked -- chunkwise forward of the Gated DeltaNet-2
+ * recurrence ("Gated DeltaNet-2" technical summary, Methodology section 1):
+ *
+ *     S_t = (I - k_t (b_t . k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T,
+ *     o_t = S_t^T q_t,
+ *
+ * i.e. CKDA with the scalar beta_t replaced by an erase gate b_t (per key
+ * channel) and a write gate w_t (per value channel); b_t = w_t = beta_t
+ * gives back ckda_fwd_chunked's recurrence.  In the chunk form T[r, s] uses
+ * b_r . k_r on its row side and the WY right-hand sides are
+ * [(B . K) * Gamma | W . V] (Methodology section 3).
+ *
+ *   b   fp32, shaped like k:  [B, T, H, d_k] (packed: [T, H, d_k])
+ *   w   fp32, shaped like v:  [B, T, H, d_v] (packed: [T, H, d_v])
+ * The gates are applied as given (the pages take them in [0, 1]).  Every
+ * other argument, layout, ownership and error rule is that of
+ * ckda_fwd_chunked (b takes beta's place in the checks; w must be non-NULL
+ * when there are tokens, 16-byte aligned and not aliased by out).  Runs on
+ * the fp32 CUDA-core kernel (any d_k, d_v in {16, 32, 64, 128}, chunk 16,
+ * 32 or 64; fp32 or bf16 q, k, v); it needs no workspace.
+ */
+CKDA_API int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* b, const float* w,
+                                   const float* S0, const int32_t* cu_seqlens, void* out,
+                                   float* S_final, int B, int T, int H, int d_k, int d_v,
+                                   int chunk, int dtype, int out_dtype, void* stream);
+
+/*
  * ckda_fwd_chunked_workspace_bytes -- scratch bytes ckda_fwd_chunked needs
  * for these sizes (same meaning of B, T and `varlen` as in
  * ckda_fwd_chunked_path), 0 when the call runs the fp32 CUDA-core kernel,

@@ -243,3 +243,22 @@ def test_static_scratch_entry_rejects_oversized_calls_without_a_gpu(lib):
     assert r == -1
     assert lib.ckda_fwd_chunked_static(P, P, P, P, P, None, None, P + 0x5000, None, 0, 64, 1, 128,
                                        128, 64, BF16, F32, None) == 0
+
+
+def test_gdn2_entry_validates_its_gates(lib):
+    def g2(**kw):
+        a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, b=P + 0x4000, w=P + 0x6000,
+                 S0=None, cu=None, out=P + 0x5000, S_final=None, B=1, T=8, H=1, dk=16, dv=16,
+                 chunk=16, dtype=0, out_dtype=0)
+        a.update(kw)
+        return lib.ckda_gdn2_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["b"], a["w"], a["S0"],
+                                         a["cu"], a["out"], a["S_final"], a["B"], a["T"], a["H"],
+                                         a["dk"], a["dv"], a["chunk"], a["dtype"], a["out_dtype"],
+                                         None)
+
+    assert g2(b=None) == -1
+    assert g2(w=None) == -1
+    assert g2(w=MIS) == -3
+    assert g2(out=P + 0x6000) == -1   # out aliases w
+    assert g2(dk=48) == -2
+    assert g2(B=0) == 0
