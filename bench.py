@@ -433,16 +433,18 @@ def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, t
 
 def _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=20):
     """Gated DeltaNet-2 forward at the bench sizes (bf16 q/k/v, fp32 gates and
-    output), on the fp32 CUDA-core kernel; two rotating input sets."""
+    output); two rotating input sets."""
     sets = [inputs.gdn2_prefill(B, T, H, D, D, dtype=torch.bfloat16, chunk=CHUNK,
                                 seed=3000 + 10 * rank + i, device=dev) for i in range(2)]
     out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
+    wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
+                        device=dev)
 
     def step(i):
         c = sets[i % 2]
         ck.gdn2_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], chunk=CHUNK,
-                            out=out, S_final=S_final)
+                            out=out, S_final=S_final, workspace=wsbuf)
 
     for i in range(3):
         step(i)
@@ -462,8 +464,9 @@ def _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
     nbytes = B * T * H * GDN2_BYTES_PER_TOKEN_HEAD + B * H * D * D * 4
     gbs = nbytes / (ms / 1e3) / 1e9
     del sets
+    path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
     return {"workload": f"gdn2_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 "
-                        "alpha/b/w, fp32 out (fp32 CUDA-core kernel)",
+                        f"alpha/b/w, fp32 out ({path} kernels)",
             "ms_per_step": ms, "tokens_per_s": ws * B * T / (ms / 1e3),
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_frac_of_measured": gbs / hbm_peak, "gpu_launches": steps}

@@ -37,7 +37,7 @@ SIGNATURES = {
     "ckda_fwd_chunked_static": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
                                      _i, _i, _i, _vp]),
     "ckda_gdn2_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
-                                   _i, _i, _i, _i, _vp]),
+                                   _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp]),
     "ckda_fwd_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
                               ctypes.c_size_t, _vp]),
     "ckda_fwd_carry": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,

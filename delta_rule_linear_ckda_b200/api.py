@@ -217,11 +217,12 @@ def fwd_carry(workspace, B, T, H, dk, dv, S0=None, cu_seqlens=None, chunk: int =
 
 
 def gdn2_fwd_chunked(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk: int = 64,
-                     out=None, S_final=None, return_final: bool = True, out_dtype=None):
+                     out=None, S_final=None, return_final: bool = True, out_dtype=None,
+                     workspace=None):
     """Chunked Gated DeltaNet-2 forward (``ckda_gdn2_fwd_chunked``): CKDA with an
     erase gate ``b`` (fp32, shaped like ``k``) and a write gate ``w`` (fp32, shaped
-    like ``v``) in place of beta.  Other arguments and the result as in
-    ``fwd_chunked``."""
+    like ``v``) in place of beta.  Other arguments, the workspace and the result
+    as in ``fwd_chunked``."""
     dev = q.device
     _need(b, "b", torch.float32, dev)
     _need(w, "w", torch.float32, dev)
@@ -247,10 +248,16 @@ def gdn2_fwd_chunked(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk: int 
         S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if S_final is not None:
         _need(S_final, "S_final", torch.float32, dev)
+    need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, out_dtype, cu_seqlens is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, dev)
     with torch.cuda.device(dev):
         rc = _lib.load().ckda_gdn2_fwd_chunked(
             _p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w), _p(S0), _p(cu_seqlens), _p(out),
-            _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype], _stream_ptr(dev))
+            _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype], _p(workspace),
+            0 if workspace is None else workspace.numel(), _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_gdn2_fwd_chunked")
     return out, S_final

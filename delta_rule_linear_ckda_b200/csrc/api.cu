@@ -21,9 +21,9 @@ cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void
 // tensor-core kernels (the caller then uses the CUDA-core kernel).
 cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
                           const void* k, const void* v, const float* alpha, const float* beta,
-                          const float* S0, const int32_t* cu, void* out, float* S_final,
-                          int n_seqs, int T, int H, int C, void* ws, int* status,
-                          cudaStream_t stream);
+                          const float* bg, const float* wg, const float* S0, const int32_t* cu,
+                          void* out, float* S_final, int n_seqs, int T, int H, int C, void* ws,
+                          int* status, cudaStream_t stream);
 bool fwd_tc_supported(int dtype, int dk, int dv, int C, int n_seqs, int T, int H, bool varlen);
 size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int T, int H,
                               bool varlen);
@@ -106,13 +106,23 @@ int validate_fwd(const void* q, const void* k, const void* v, const float* alpha
   return CKDA_OK;
 }
 
+// `bg` and `wg` non-NULL select the Gated DeltaNet-2 form: `bg` takes beta's
+// place in the shared checks, `wg` is checked here.
 int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void* v,
-             const float* alpha, const float* beta, const float* S0, const int32_t* cu,
-             void* out, float* S_final, int B, int T, int H, int d_k, int d_v, int chunk,
-             int dtype, int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
-  int rc = validate_fwd(q, k, v, alpha, beta, S0, cu, out, S_final, B, T, H, d_k, d_v, &chunk,
-                        dtype, out_dtype, phases);
+             const float* alpha, const float* beta, const float* bg, const float* wg,
+             const float* S0, const int32_t* cu, void* out, float* S_final, int B, int T, int H,
+             int d_k, int d_v, int chunk, int dtype, int out_dtype, void* workspace,
+             size_t workspace_bytes, void* stream) {
+  const bool gdn2 = bg != nullptr || wg != nullptr;
+  int rc = validate_fwd(q, k, v, alpha, gdn2 ? bg : beta, S0, cu, out, S_final, B, T, H, d_k,
+                        d_v, &chunk, dtype, out_dtype, phases);
   if (rc != CKDA_OK) return rc;
+  if (gdn2) {
+    const int64_t tokens = (cu != nullptr) ? (int64_t)T : (int64_t)B * T;
+    if (tokens > 0 && (bg == nullptr || wg == nullptr)) return CKDA_ERR_INVALID_ARG;
+    if (wg != nullptr && !aligned16(wg)) return CKDA_ERR_MISALIGNED;
+    if (out != nullptr && out == wg) return CKDA_ERR_INVALID_ARG;
+  }
   const int n_seqs = B;
   const bool tc = allow_tc && n_seqs > 0 &&
                   ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, n_seqs, T, H, cu != nullptr);
@@ -126,7 +136,7 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
       return CKDA_ERR_WORKSPACE;
     const void* ws_end = static_cast<const uint8_t*>(workspace) + need;
-    const void* ptrs[] = {q, k, v, alpha, beta, S0, out, S_final, cu};
+    const void* ptrs[] = {q, k, v, alpha, beta, bg, wg, S0, out, S_final, cu};
     for (const void* p : ptrs)
       if (p != nullptr && p >= workspace && p < ws_end) return CKDA_ERR_WORKSPACE;
   }
@@ -135,11 +145,11 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (tc)
-    e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S0, cu,
-                            out, S_final, n_seqs, T, H, chunk, workspace, status, st);
+    e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg, S0,
+                            cu, out, S_final, n_seqs, T, H, chunk, workspace, status, st);
   if (e == cudaErrorNotSupported)
-    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, nullptr, nullptr,
-                              S0, cu, out, S_final, n_seqs, T, H, chunk, status, st);
+    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg, S0, cu,
+                              out, S_final, n_seqs, T, H, chunk, status, st);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
@@ -178,8 +188,9 @@ int ckda_fwd_chunked(const void* q, const void* k, const void* v, const float* a
                      const float* beta, const float* S0, const int32_t* cu_seqlens, void* out,
                      float* S_final, int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
                      int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
-  return fwd_impl(true, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
-                  d_v, chunk, dtype, out_dtype, workspace, workspace_bytes, stream);
+  return fwd_impl(true, kBoth, q, k, v, alpha, beta, nullptr, nullptr, S0, cu_seqlens, out,
+                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, workspace,
+                  workspace_bytes, stream);
 }
 
 int ckda_fwd_chunked_static(const void* q, const void* k, const void* v, const float* alpha,
@@ -195,54 +206,44 @@ int ckda_fwd_chunked_static(const void* q, const void* k, const void* v, const f
   if (need > (size_t)CKDA_STATIC_SCRATCH_BYTES) return CKDA_ERR_UNSUPPORTED;
   void* ws = nullptr;
   if (need > 0 && (ws = scratch_ptr()) == nullptr) return CKDA_ERR_CUDA;
-  return fwd_impl(true, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
-                  d_v, chunk, dtype, out_dtype, ws, need > 0 ? (size_t)CKDA_STATIC_SCRATCH_BYTES : 0,
-                  stream);
+  return fwd_impl(true, kBoth, q, k, v, alpha, beta, nullptr, nullptr, S0, cu_seqlens, out,
+                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, ws,
+                  need > 0 ? (size_t)CKDA_STATIC_SCRATCH_BYTES : 0, stream);
 }
 
 int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
                           const float* b, const float* w, const float* S0,
                           const int32_t* cu_seqlens, void* out, float* S_final, int B, int T, int H,
-                          int d_k, int d_v, int chunk, int dtype, int out_dtype, void* stream) {
-  // the erase gate takes beta's place in the shared checks; the write gate is checked here
-  int rc = validate_fwd(q, k, v, alpha, b, S0, cu_seqlens, out, S_final, B, T, H, d_k, d_v,
-                        &chunk, dtype, out_dtype);
-  if (rc != CKDA_OK) return rc;
-  const int64_t tokens = (cu_seqlens != nullptr) ? (int64_t)T : (int64_t)B * T;
-  if (tokens > 0 && w == nullptr) return CKDA_ERR_INVALID_ARG;
-  if (w != nullptr && !aligned16(w)) return CKDA_ERR_MISALIGNED;
-  if (out != nullptr && out == w) return CKDA_ERR_INVALID_ARG;
-  if (B == 0) return CKDA_OK;  // (zero-length sequences still store S_final = S0)
-  int* status = status_ptr();
-  if (status == nullptr) return CKDA_ERR_CUDA;
-  cudaError_t e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, nullptr, b, w,
-                                        S0, cu_seqlens, out, S_final, B, T, H, chunk, status,
-                                        static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+                          int d_k, int d_v, int chunk, int dtype, int out_dtype, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  // (both gates NULL: checked as the beta form with beta NULL)
+  return fwd_impl(true, kBoth, q, k, v, alpha, nullptr, b, w, S0, cu_seqlens, out, S_final, B,
+                  T, H, d_k, d_v, chunk, dtype, out_dtype, workspace, workspace_bytes, stream);
 }
 
 int ckda_fwd_factors(const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, const int32_t* cu_seqlens, int B, int T, int H, int d_k,
                      int d_v, int chunk, int dtype, void* workspace, size_t workspace_bytes,
                      void* stream) {
-  return fwd_impl(true, kFactors, q, k, v, alpha, beta, nullptr, cu_seqlens, nullptr, nullptr, B,
-                  T, H, d_k, d_v, chunk, dtype, CKDA_F32, workspace, workspace_bytes, stream);
+  return fwd_impl(true, kFactors, q, k, v, alpha, beta, nullptr, nullptr, nullptr, cu_seqlens,
+                  nullptr, nullptr, B, T, H, d_k, d_v, chunk, dtype, CKDA_F32, workspace,
+                  workspace_bytes, stream);
 }
 
 int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* out, float* S_final, int B,
                    int T, int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
                    void* workspace, size_t workspace_bytes, void* stream) {
-  return fwd_impl(true, kCarry, nullptr, nullptr, nullptr, nullptr, nullptr, S0, cu_seqlens, out,
-                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, workspace,
-                  workspace_bytes, stream);
+  return fwd_impl(true, kCarry, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S0,
+                  cu_seqlens, out, S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype,
+                  workspace, workspace_bytes, stream);
 }
 
 int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void* v, const float* alpha,
                               const float* beta, const float* S0, const int32_t* cu_seqlens,
                               void* out, float* S_final, int B, int T, int H, int d_k, int d_v,
                               int chunk, int dtype, int out_dtype, void* stream) {
-  return fwd_impl(false, kBoth, q, k, v, alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, d_k,
-                  d_v, chunk, dtype, out_dtype, nullptr, 0, stream);
+  return fwd_impl(false, kBoth, q, k, v, alpha, beta, nullptr, nullptr, S0, cu_seqlens, out,
+                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, nullptr, 0, stream);
 }
 
 int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int chunk, int dtype,

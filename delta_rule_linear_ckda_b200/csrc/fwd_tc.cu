@@ -326,7 +326,14 @@ __device__ __forceinline__ int level_row(int lv, int p) {
 // both roles and the complementary pairs k and 7 - k, whose level work adds
 // up to the same amount on every scheduler.  One out-of-line copy serves
 // both halves.
-__device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid) {
+//
+// G2 (Gated DeltaNet-2): the erase side uses e = b * k (b per key channel,
+// read from global memory at `bgp` + position * `bstride`, the channels of
+// this half) in place of beta * k: in the T rows of the level operands, in
+// the direct T pairs and in E * Gamma (stored where K * Gamma goes).
+template <bool G2>
+__device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid,
+                                       const float* __restrict__ bgp, int bstride) {
   const int w = tid >> 5;
   const int role = (w >> 2) & 1;
   const int kk = (w < 8) ? (w & 3) : 7 - (w & 3);
@@ -349,9 +356,17 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     return pk;
   };
 
-  // every input of this thread's 4 positions, loaded up front
-  float4 aa[4], ka[4], qa[4];
+  // every input of this thread's 4 positions, loaded up front (the erase
+  // gate first: it comes from global memory)
+  float4 aa[4], ka[4], qa[4], eg[4];
   float bb[4];
+  if constexpr (G2) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = 4 * g + u;
+      eg[u] = (p < Lc) ? __ldg(reinterpret_cast<const float4*>(bgp + (size_t)p * bstride + cl)) : zero;
+    }
+  }
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const int p = 4 * g + u;
@@ -359,7 +374,11 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     aa[u] = val ? lds_f4(in + IN_A + p * 256 + cl * 4) : one;
     ka[u] = val ? bf4(lds_u2(in + IN_K + p * 128 + cl * 2)) : zero;
     qa[u] = val ? bf4(lds_u2(in + IN_Q + p * 128 + cl * 2)) : zero;
-    bb[u] = lds_f(sb + OFF_BETA + p * 4);
+    if constexpr (!G2) bb[u] = lds_f(sb + OFF_BETA + p * 4);
+  }
+  if constexpr (G2) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) eg[u] = mul4(eg[u], ka[u]);  // e = b * k
   }
 #ifdef CKDA_TC_DEBUG
   long long gp_last = clock64();
@@ -432,11 +451,11 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
       pg = mul4(pg, a);
       lp = (u == 0) ? a : mul4(lp, a);
       const uint32_t ro = 128 * u + xo[u];
-      sts_u2(kg_b + ro, h4(mul4(kf, pg)));
+      sts_u2(kg_b + ro, h4(mul4(G2 ? eg[u] : kf, pg)));
       sts_u2(qg_b + ro, h4(mul4(qf, pg)));
       if (g & 15) {
         const float4 qlp = mul4(qf, lp);
-        const float4 blp = scale4(bb[u], mul4(kf, lp));
+        const float4 blp = G2 ? mul4(eg[u], lp) : scale4(bb[u], mul4(kf, lp));
         if (g & 1) {  // level 2: right half
           const uint32_t o2 = l2b + 128 * u + xo2[u];
           sts_u2(o2, h4(blp));
@@ -491,18 +510,20 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     {
       const float4 k0 = ka[0], k1 = ka[1], k2 = ka[2], k3 = ka[3];
       const float4 q1 = qa[1], q2 = qa[2], q3 = qa[3];
+      // row side of the T pairs: k_r (scaled by beta_r in the gather) or e_r
+      const float4 t1 = G2 ? eg[1] : k1, t2 = G2 ? eg[2] : k2, t3 = G2 ? eg[3] : k3;
       const float4 e10 = mul4(aa[1], k0);
       const float4 e20 = mul4(aa[2], e10);
       const float4 e21 = mul4(aa[2], k1);
       const float4 e30 = mul4(aa[3], e20);
       const float4 e31 = mul4(aa[3], e21);
       const float4 e32 = mul4(aa[3], k2);
-      acc[0] = dot4(k1, e10);  acc[1] = dot4(q1, e10);
-      acc[2] = dot4(k2, e20);  acc[3] = dot4(q2, e20);
-      acc[4] = dot4(k2, e21);  acc[5] = dot4(q2, e21);
-      acc[6] = dot4(k3, e30);  acc[7] = dot4(q3, e30);
-      acc[8] = dot4(k3, e31);  acc[9] = dot4(q3, e31);
-      acc[10] = dot4(k3, e32); acc[11] = dot4(q3, e32);
+      acc[0] = dot4(t1, e10);  acc[1] = dot4(q1, e10);
+      acc[2] = dot4(t2, e20);  acc[3] = dot4(q2, e20);
+      acc[4] = dot4(t2, e21);  acc[5] = dot4(q2, e21);
+      acc[6] = dot4(t3, e30);  acc[7] = dot4(q3, e30);
+      acc[8] = dot4(t3, e31);  acc[9] = dot4(q3, e31);
+      acc[10] = dot4(t3, e32); acc[11] = dot4(q3, e32);
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[12 + u] = dot4(qa[u], ka[u]);
     }
@@ -641,13 +662,18 @@ __device__ Unit find_unit(int ui, int stride, int n_units, const int32_t* cu, in
 
 // ---- kernel 1: per-unit WY factors ----------------------------------------------
 
-template <int DV>
+// G2: the Gated DeltaNet-2 form -- erase gate bg (shaped like k) and write
+// gate wg (shaped like v) in place of beta; the workspace then holds
+// [-W; Q'] with W = Inv (E * Gamma), [Inv; A Inv] and Z = wg * V, and the
+// carry kernel is unchanged.
+template <int DV, bool G2>
 __global__ void __launch_bounds__(NT1, 1)
 factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
               const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
               const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
-              const float* __restrict__ beta,
+              const float* __restrict__ beta, const float* __restrict__ bg,
+              const float* __restrict__ wg,
               const int32_t* __restrict__ cu, int n_seqs, int T, int H, int nch, int64_t n_units,
               float* __restrict__ ws_g, int* status) {
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
@@ -744,8 +770,10 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
   // beta of a unit, one value per thread tid < C (0 past the end)
   auto load_beta = [&](const Unit& uu) -> float {
+    if constexpr (G2) return 0.f;  // unused
     return (uu.idx >= 0 && tid < uu.Lc) ? beta[(size_t)(uu.t0 + tid) * H + uu.h] : 0.f;
   };
+
   Unit cur = find_unit(blockIdx.x, gridDim.x, (int)n_units, cu, n_seqs, T, H, nch);
   float beta_next = 0.f;
   if (cur.idx >= 0) {
@@ -783,7 +811,9 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #ifdef CKDA_TC_DEBUG
     const long long t_gp0 = clock64();
 #endif
-    gate_pass(sb, sb + OFF_IN0, 0, Lc, tid);
+    // (G2: the erase gate of this half starts at row t0, channel h * DK + 64 hh)
+    const float* bg_row = G2 ? bg + ((size_t)cur.t0 * H + cur.h) * DK : nullptr;
+    gate_pass<G2>(sb, sb + OFF_IN0, 0, Lc, tid, bg_row, H * DK);
 #ifdef CKDA_TC_DEBUG
     const long long t_gp1 = clock64();
 #endif
@@ -811,7 +841,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    gate_pass(sb, sb + OFF_IN1, 1, Lc, tid);
+    gate_pass<G2>(sb, sb + OFF_IN1, 1, Lc, tid, G2 ? bg_row + HC : nullptr, H * DK);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -874,18 +904,20 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
           if (w & 1)
             Af[fsw(r, s)] = val;
           else
-            Tf[fsw(r, s)] = beta_s[r] * val;
+            Tf[fsw(r, s)] = G2 ? val : beta_s[r] * val;
         } else {
           const int r = 4 * g + (w - 12);
           Af[fsw(r, r)] = val;
         }
       }
-      // v tile: bf16 (as loaded) -> fp16 in place; rows past the end -> 0.
-      // Each 16-byte chunk stays within its 128-byte row under the swizzle.
+      // v tile: bf16 (as loaded) -> fp16 in place (G2: Z = w * v); rows past
+      // the end -> 0.  Each 16-byte chunk stays within its 128-byte row under
+      // the swizzle.
       uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V);
       for (int e = tid; e < C * 8 * (DV / 64); e += NT1) {
         uint4 raw = vt[e];
-        if (((e >> 3) & 63) < Lc) {
+        const int row = (e >> 3) & 63;
+        if (row < Lc) {
           float f[8];
           const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
@@ -893,6 +925,15 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             const float2 x2 = __bfloat1622float2(p2[t]);
             f[2 * t] = x2.x;
             f[2 * t + 1] = x2.y;
+          }
+          if constexpr (G2) {
+            // logical columns of this chunk: atom * 64 + 8 * (chunk ^ (row % 8))
+            const int col = 64 * (e >> 9) + 8 * ((e & 7) ^ (row & 7));
+            const float* wp = wg + ((size_t)(cur.t0 + row) * H + cur.h) * DV + col;
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp + 4));
+            f[0] *= w0.x; f[1] *= w0.y; f[2] *= w0.z; f[3] *= w0.w;
+            f[4] *= w1.x; f[5] *= w1.y; f[6] *= w1.z; f[7] *= w1.w;
           }
           raw.x = pack_f16x2(f[0], f[1]);
           raw.y = pack_f16x2(f[2], f[3]);
@@ -963,7 +1004,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
       inv_merge<16>(Tf, Inv, Yf, tid);
       inv_merge<32>(Tf, Inv, Yf, tid);
       TC_DBG(for (int e = tid; e < 4096; e += NT1) g_tc_dbg[8192 + e] = Inv[fsw(e >> 6, e & 63)]);
-      // Inv diag(beta) -> rows 0..63 of the stacked operand
+      // Inv diag(beta) (G2: Inv) -> rows 0..63 of the stacked operand
       {
         const int r = tid >> 3, cg = tid & 7;
         const float4 lo = *reinterpret_cast<const float4*>(Inv + fsw(r, 8 * cg));
@@ -971,7 +1012,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const float i8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         float v[8];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) v[t] = i8[t] * beta_s[8 * cg + t];
+        for (int t = 0; t < 8; ++t) v[t] = G2 ? i8[t] : i8[t] * beta_s[8 * cg + t];
         st_chunk8(sm + OFF_IP, sw128_chunk(r, 8 * cg, 128), v);
       }
     }
@@ -1449,11 +1490,11 @@ cudaError_t set_smem(K kern, size_t bytes) {
 // `stream`.
 constexpr int kFactors = 1, kCarry = 2;
 
-template <int DV, typename Tout>
+template <int DV, typename Tout, bool G2>
 cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, const float* alpha,
-                     const float* beta, const float* S0, const int32_t* cu, void* out,
-                     float* S_final, int n_seqs, int T, int H, void* ws, int* status,
-                     cudaStream_t stream) {
+                     const float* beta, const float* bg, const float* wg, const float* S0,
+                     const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
+                     void* ws, int* status, cudaStream_t stream) {
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
   const int nch = (int)(((int64_t)T + C - 1) / C);
   const int64_t nu = n_units(cu != nullptr, n_seqs, T, H);
@@ -1490,7 +1531,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
         make_map(&mwq64, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
                  C, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    auto k1 = factor_kernel<DV>;
+    auto k1 = factor_kernel<DV, G2>;
     static bool attr1 = false;
     if (!attr1) {
       cudaError_t e = set_smem(k1, kSmemBytes);
@@ -1498,8 +1539,8 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       attr1 = true;
     }
     const int64_t g1 = nu < (int64_t)sm_count() ? nu : (int64_t)sm_count();
-    k1<<<(unsigned)g1, NT1, kSmemBytes, stream>>>(mq, mk, mv, ma, mwq64, mkh, mip, mv16, beta,
-                                                  cu, n_seqs, T, H, nch, nu, ws_g, status);
+    k1<<<(unsigned)g1, NT1, kSmemBytes, stream>>>(mq, mk, mv, ma, mwq64, mkh, mip, mv16, beta, bg,
+                                                  wg, cu, n_seqs, T, H, nch, nu, ws_g, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1557,23 +1598,26 @@ size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int 
 // Everything the tensor-core kernels do not cover returns
 // cudaErrorNotSupported so the caller can use the CUDA-core kernel.
 // `phases`: 1 = factors only, 2 = carry only, 3 = the whole forward.
+// `bg`, `wg` non-NULL select the Gated DeltaNet-2 form (beta unused).
 cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
                           const void* k, const void* v, const float* alpha, const float* beta,
-                          const float* S0, const int32_t* cu, void* out, float* S_final,
-                          int n_seqs, int T, int H, int C, void* ws, int* status,
-                          cudaStream_t stream) {
+                          const float* bg, const float* wg, const float* S0, const int32_t* cu,
+                          void* out, float* S_final, int n_seqs, int T, int H, int C, void* ws,
+                          int* status, cudaStream_t stream) {
   if (!fwd_tc_supported(dtype, dk, dv, C, n_seqs, T, H, cu != nullptr))
     return cudaErrorNotSupported;
   const bool bf = out_dtype == CKDA_BF16;
-  if (dv == 128)
-    return bf ? tc::launch_t<128, __nv_bfloat16>(phases, q, k, v, alpha, beta, S0, cu, out,
-                                                 S_final, n_seqs, T, H, ws, status, stream)
-              : tc::launch_t<128, float>(phases, q, k, v, alpha, beta, S0, cu, out, S_final,
-                                         n_seqs, T, H, ws, status, stream);
-  return bf ? tc::launch_t<64, __nv_bfloat16>(phases, q, k, v, alpha, beta, S0, cu, out, S_final,
-                                              n_seqs, T, H, ws, status, stream)
-            : tc::launch_t<64, float>(phases, q, k, v, alpha, beta, S0, cu, out, S_final, n_seqs,
-                                      T, H, ws, status, stream);
+  const bool g2 = bg != nullptr;
+#define CKDA_TC_CALL(DVV, TO, G)                                                            \
+  tc::launch_t<DVV, TO, G>(phases, q, k, v, alpha, beta, bg, wg, S0, cu, out, S_final, n_seqs, T, \
+                           H, ws, status, stream)
+  if (dv == 128) {
+    if (g2) return bf ? CKDA_TC_CALL(128, __nv_bfloat16, true) : CKDA_TC_CALL(128, float, true);
+    return bf ? CKDA_TC_CALL(128, __nv_bfloat16, false) : CKDA_TC_CALL(128, float, false);
+  }
+  if (g2) return bf ? CKDA_TC_CALL(64, __nv_bfloat16, true) : CKDA_TC_CALL(64, float, true);
+  return bf ? CKDA_TC_CALL(64, __nv_bfloat16, false) : CKDA_TC_CALL(64, float, false);
+#undef CKDA_TC_CALL
 }
 
 }  // namespace ckda

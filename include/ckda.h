@@ -218,16 +218,19 @@ CKDA_API int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* ou
  *   w   fp32, shaped like v:  [B, T, H, d_v] (packed: [T, H, d_v])
  * The gates are applied as given (the pages take them in [0, 1]).  Every
  * other argument, layout, ownership and error rule is that of
- * ckda_fwd_chunked (b takes beta's place in the checks; w must be non-NULL
- * when there are tokens, 16-byte aligned and not aliased by out).  Runs on
- * the fp32 CUDA-core kernel (any d_k, d_v in {16, 32, 64, 128}, chunk 16,
- * 32 or 64; fp32 or bf16 q, k, v); it needs no workspace.
+ * ckda_fwd_chunked, workspace included (b takes beta's place in the checks;
+ * w must be non-NULL when there are tokens, 16-byte aligned and not aliased
+ * by out).  The kernels are those of ckda_fwd_chunked for the same sizes
+ * (ckda_fwd_chunked_path, ckda_fwd_chunked_workspace_bytes): the tcgen05
+ * pair for bf16 inputs with d_k = 128, d_v in {64, 128}, chunk 64, the fp32
+ * CUDA-core kernel otherwise.
  */
 CKDA_API int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v,
                                    const float* alpha, const float* b, const float* w,
                                    const float* S0, const int32_t* cu_seqlens, void* out,
                                    float* S_final, int B, int T, int H, int d_k, int d_v,
-                                   int chunk, int dtype, int out_dtype, void* stream);
+                                   int chunk, int dtype, int out_dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream);
 
 /*
  * ckda_fwd_chunked_workspace_bytes -- scratch bytes ckda_fwd_chunked needs

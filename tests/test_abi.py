@@ -254,7 +254,7 @@ def test_gdn2_entry_validates_its_gates(lib):
         return lib.ckda_gdn2_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["b"], a["w"], a["S0"],
                                          a["cu"], a["out"], a["S_final"], a["B"], a["T"], a["H"],
                                          a["dk"], a["dv"], a["chunk"], a["dtype"], a["out_dtype"],
-                                         None)
+                                         None, 0, None)
 
     assert g2(b=None) == -1
     assert g2(w=None) == -1
@@ -262,3 +262,5 @@ def test_gdn2_entry_validates_its_gates(lib):
     assert g2(out=P + 0x6000) == -1   # out aliases w
     assert g2(dk=48) == -2
     assert g2(B=0) == 0
+    # the tensor-core shapes need the same workspace as ckda_fwd_chunked
+    assert g2(dtype=1, dk=128, dv=128, chunk=64, T=128) == -7

@@ -82,3 +82,44 @@ def test_tied_gates_reproduce_the_ckda_path(ck):
     assert ck.device_status() == 0
     assert rel_max_err(o1, o2.double().cpu().numpy()) <= 1e-5
     assert rel_max_err(S1, S2.double().cpu().numpy()) <= 1e-5
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("T", [64, 200])
+def test_tensor_core_path_matches_oracle(ck, dv, T):
+    assert ck.fwd_path(2, T, 3, 128, dv, 64, torch.bfloat16, torch.float32) == "tcgen05"
+    c = inputs.gdn2_prefill(2, T, 3, 128, dv, dtype=torch.bfloat16, s0_std=0.02, chunk=64,
+                            seed=T + dv, device=DEV)
+    out, S = _run(ck, c)
+    ro, rS = oracle.forward_gdn2(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], S0=c.S0)
+    assert rel_max_err(out, ro) <= TOL_BF16 and rel_max_err(S, rS) <= TOL_BF16
+
+
+def test_tensor_core_packed_batch(ck):
+    lens = [70, 0, 129, 1, 64]
+    total = int(sum(lens))
+    c = inputs.gdn2_prefill(1, total, 2, 128, 128, dtype=torch.bfloat16, chunk=64, seed=19,
+                            device=DEV)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(20)
+    S0 = 0.02 * torch.randn(len(lens), 2, 128, 128, generator=g, device=DEV)
+    out, S = ck.gdn2_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], S0=S0,
+                                 cu_seqlens=cu, chunk=64, out_dtype=torch.float32)
+    assert ck.device_status() == 0
+    ro, rS = oracle.forward_gdn2(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], S0=S0,
+                                 cu_seqlens=cu)
+    assert rel_max_err(out, ro) <= TOL_BF16 and rel_max_err(S, rS) <= TOL_BF16
+    assert torch.equal(S[1], S0[1])
+
+
+def test_tensor_core_agrees_with_the_fp32_kernel(ck):
+    """Same bf16 inputs through the tcgen05 pair and the fp32 CUDA-core kernel
+    (chunk 32 forces the latter)."""
+    c = inputs.gdn2_prefill(1, 256, 4, 128, 128, dtype=torch.bfloat16, s0_std=0.02, chunk=64,
+                            seed=21, device=DEV)
+    o_tc, S_tc = _run(ck, c)
+    o_32, S_32 = ck.gdn2_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], S0=c.S0,
+                                     chunk=32, out_dtype=torch.float32)
+    assert ck.device_status() == 0
+    assert rel_max_err(o_tc, o_32.double().cpu().numpy()) <= TOL_BF16
+    assert rel_max_err(S_tc, S_32.double().cpu().numpy()) <= TOL_BF16
