@@ -20,6 +20,13 @@ Contents
     gate w_t (value side) in place of beta_t,
     ``S_t = (I - k_t (b_t . k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t . v_t)^T``;
     pinned by ``tests/pinlib_gdn2.py`` (G-1..G-7).
+``forward_sfda``
+    The SFDA recurrence ("Semidirect Fourier Delta Attention (SFDA)" page,
+    "Arquitectura Central"): the real diagonal gate replaced by 2x2
+    rotation-decay blocks ``alpha_p R(theta_p)`` on the state rows
+    ``(2p, 2p+1)``,
+    ``S_t = (I - beta_t k_t k_t^T) Lambda_t S_{t-1} + beta_t k_t v_t^T``;
+    pinned by ``tests/pinlib_sfda.py`` (S-1..S-8).
 ``chunked`` (submodule)
     A plain numpy fp64 restatement of the chunkwise WY form, used only to pin
     the chunked algorithm against the sequential loop on tiny inputs.
@@ -50,7 +57,7 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
-            ["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lpthread"]
+            ["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC", "-o", tmp, _SRC, "-lpthread", "-lm"]
         )
         os.replace(tmp, _LIB)
     return _LIB
@@ -73,6 +80,11 @@ def _load():
                 dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
             ]
             lib.ckda_oracle_gdn2_forward.restype = ctypes.c_int
+            lib.ckda_oracle_sfda_forward.argtypes = [
+                i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int64),
+                dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
+            ]
+            lib.ckda_oracle_sfda_forward.restype = ctypes.c_int
             lib.ckda_oracle_decode_step.argtypes = [
                 i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
             ]
@@ -182,6 +194,52 @@ def forward_gdn2(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, n_threads=None)
     )
     if rc != 0:
         raise ValueError("ckda_oracle_gdn2_forward rejected its arguments")
+    return out.reshape(out_shape), S_final
+
+
+def forward_sfda(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, n_threads=None):
+    """Sequential fp64 SFDA forward ("Semidirect Fourier Delta Attention
+    (SFDA)" summary, "Arquitectura Central", real coordinates): the CKDA
+    recurrence with Diag(alpha_t) replaced by the block-diagonal
+    phase-decay gate whose block p is ``alpha_p R(theta_p)`` on state rows
+    ``(2p, 2p+1)``.  ``alpha`` and ``theta`` are shaped like ``k`` with the
+    last dimension halved; other arguments and the result as in
+    ``forward``."""
+    qd, kd, vd, ad, td, bd = (_f64(t) for t in (q, k, v, alpha, theta, beta))
+    out_shape = vd.shape
+    if cu_seqlens is None:
+        if qd.ndim != 4:
+            raise ValueError("fixed-length batch expects [B, T, H, d] tensors")
+        B, T, H, dk = qd.shape
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int64))
+        if qd.ndim == 4:
+            if qd.shape[0] != 1:
+                raise ValueError("packed batch expects a leading dimension of 1")
+            qd, kd, vd, ad, td, bd = qd[0], kd[0], vd[0], ad[0], td[0], bd[0]
+        H, dk = qd.shape[1], qd.shape[2]
+    if dk % 2:
+        raise ValueError("SFDA pairs the key channels: dk must be even")
+    N = len(cu) - 1
+    dv = vd.shape[-1]
+    T_total = int(cu[-1])
+    qd, kd = (x.reshape(T_total, H, dk) for x in (qd, kd))
+    ad, td = (x.reshape(T_total, H, dk // 2) for x in (ad, td))
+    vd = vd.reshape(T_total, H, dv)
+    bd = bd.reshape(T_total, H)
+    S0d = None if S0 is None else _f64(S0).reshape(N, H, dk, dv)
+    out = np.zeros((T_total, H, dv), dtype=np.float64)
+    S_final = np.zeros((N, H, dk, dv), dtype=np.float64)
+    rc = _load().ckda_oracle_sfda_forward(
+        N, H, dk, dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(qd), _ptr(kd), _ptr(vd), _ptr(ad), _ptr(td), _ptr(bd), _ptr(S0d),
+        _ptr(out), _ptr(S_final), int(n_threads or default_threads()),
+    )
+    if rc != 0:
+        raise ValueError("ckda_oracle_sfda_forward rejected its arguments")
     return out.reshape(out_shape), S_final
 
 

@@ -49,7 +49,30 @@
  *   3. S <- S + k (z - r)^T,  z = w . v
  *   4. o <- S^T q
  *   b : [T_total, H, dk]   w : [T_total, H, dv]
+ *
+ * The SFDA form (ckda_oracle_sfda_forward) replaces the real diagonal gate by
+ * a phase-decay gate ("Semidirect Fourier Delta Attention (SFDA)" technical
+ * summary, "Arquitectura Central"): in complex coordinates
+ * Lambda_t = diag(alpha_t . e^{i theta_t}); in real coordinates, the form
+ * used here, Lambda_t is the direct sum of 2x2 rotation-decay blocks, block
+ * p acting on the state rows (2p, 2p+1) as
+ *
+ *   alpha_p * [[cos theta_p, -sin theta_p], [sin theta_p, cos theta_p]]
+ *
+ * (row 2p is the real part, row 2p+1 the imaginary part of channel p), and
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Lambda_t S_{t-1} + beta_t k_t v_t^T,
+ *
+ * i.e. the transition Lambda_t - u_t r_t^T with u_t = beta_t k_t and
+ * r_t = Lambda_t^T k_t ("El Teorema de Chunk-WY Constructivo").  Keys,
+ * queries, values and the state are real.  Its body:
+ *   1. S <- Lambda S                  (rotate and scale each row pair)
+ *   2. r <- S^T k
+ *   3. S <- S + beta k (v - r)^T
+ *   4. o <- S^T q
+ *   alpha, theta : [T_total, H, dk / 2]   (dk even)
  */
+#include <math.h>
 #include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
@@ -60,6 +83,7 @@ typedef struct {
     const int64_t *cu;
     const double *q, *k, *v, *alpha, *beta, *S0;
     const double *eg, *wg; /* Gated DeltaNet-2 gates (NULL for the beta form) */
+    const double *theta;   /* SFDA phases (NULL unless the SFDA form) */
     double *out, *S_final;
     int64_t next_unit; /* shared work counter (guarded by lock) */
     pthread_mutex_t lock;
@@ -142,6 +166,52 @@ static void run_unit_gdn2(const oracle_job *J, int64_t n, int64_t h, double *S,
                sizeof(double) * dk * dv);
 }
 
+/* One (sequence, head) unit of the SFDA recurrence (phase-decay blocks). */
+static void run_unit_sfda(const oracle_job *J, int64_t n, int64_t h, double *S,
+                          double *r) {
+    const int64_t H = J->H, dk = J->dk, dv = J->dv, np = dk / 2;
+    if (J->S0) {
+        memcpy(S, J->S0 + ((n * H + h) * dk) * dv, sizeof(double) * dk * dv);
+    } else {
+        memset(S, 0, sizeof(double) * dk * dv);
+    }
+    for (int64_t t = J->cu[n]; t < J->cu[n + 1]; ++t) {
+        const double *q = J->q + (t * H + h) * dk;
+        const double *k = J->k + (t * H + h) * dk;
+        const double *a = J->alpha + (t * H + h) * np;
+        const double *th = J->theta + (t * H + h) * np;
+        const double *v = J->v + (t * H + h) * dv;
+        const double b = J->beta[t * H + h];
+        double *o = J->out + (t * H + h) * dv;
+
+        /* 1. S <- Lambda S: rows (2p, 2p+1) times alpha_p R(theta_p) */
+        for (int64_t p = 0; p < np; ++p) {
+            const double c = a[p] * cos(th[p]), sn = a[p] * sin(th[p]);
+            double *x = S + (2 * p) * dv, *y = S + (2 * p + 1) * dv;
+            for (int64_t j = 0; j < dv; ++j) {
+                const double xr = x[j], yr = y[j];
+                x[j] = c * xr - sn * yr;
+                y[j] = sn * xr + c * yr;
+            }
+        }
+        /* 2. r <- S^T k */
+        for (int64_t j = 0; j < dv; ++j) r[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) r[j] += S[i * dv + j] * k[i];
+        /* 3. S <- S + beta k (v - r)^T */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j)
+                S[i * dv + j] += b * k[i] * (v[j] - r[j]);
+        /* 4. o <- S^T q */
+        for (int64_t j = 0; j < dv; ++j) o[j] = 0.0;
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dv; ++j) o[j] += S[i * dv + j] * q[i];
+    }
+    if (J->S_final)
+        memcpy(J->S_final + ((n * H + h) * dk) * dv, S,
+               sizeof(double) * dk * dv);
+}
+
 static void *worker(void *arg) {
     oracle_job *J = (oracle_job *)arg;
     double *S = (double *)malloc(sizeof(double) * J->dk * J->dv);
@@ -152,7 +222,9 @@ static void *worker(void *arg) {
         int64_t u = J->next_unit++;
         pthread_mutex_unlock(&J->lock);
         if (u >= n_units) break;
-        if (J->eg)
+        if (J->theta)
+            run_unit_sfda(J, u / J->H, u % J->H, S, r);
+        else if (J->eg)
             run_unit_gdn2(J, u / J->H, u % J->H, S, r);
         else
             run_unit(J, u / J->H, u % J->H, S, r);
@@ -206,6 +278,7 @@ int ckda_oracle_forward(int64_t n_seqs, int64_t H, int64_t dk, int64_t dv,
     J.beta = beta;
     J.eg = NULL;
     J.wg = NULL;
+    J.theta = NULL;
     J.S0 = S0;
     J.out = out;
     J.S_final = S_final;
@@ -242,6 +315,45 @@ int ckda_oracle_gdn2_forward(int64_t n_seqs, int64_t H, int64_t dk, int64_t dv,
     J.beta = NULL;
     J.eg = b;
     J.wg = w;
+    J.theta = NULL;
+    J.S0 = S0;
+    J.out = out;
+    J.S_final = S_final;
+    run_job(&J, n_threads);
+    return 0;
+}
+
+/*
+ * Sequential SFDA forward over a packed batch (layouts as above, with the
+ * decays alpha and phases theta both [T_total, H, dk / 2] and dk even).
+ * Returns 0 on success, -1 on an argument error.
+ */
+int ckda_oracle_sfda_forward(int64_t n_seqs, int64_t H, int64_t dk, int64_t dv,
+                             const int64_t *cu_seqlens, const double *q,
+                             const double *k, const double *v,
+                             const double *alpha, const double *theta,
+                             const double *beta, const double *S0, double *out,
+                             double *S_final, int n_threads) {
+    if (n_seqs < 0 || H <= 0 || dk <= 0 || dv <= 0 || (dk & 1) || !cu_seqlens ||
+        !theta)
+        return -1;
+    if (cu_seqlens[0] != 0) return -1;
+    for (int64_t n = 0; n < n_seqs; ++n)
+        if (cu_seqlens[n + 1] < cu_seqlens[n]) return -1;
+    oracle_job J;
+    J.n_seqs = n_seqs;
+    J.H = H;
+    J.dk = dk;
+    J.dv = dv;
+    J.cu = cu_seqlens;
+    J.q = q;
+    J.k = k;
+    J.v = v;
+    J.alpha = alpha;
+    J.beta = beta;
+    J.eg = NULL;
+    J.wg = NULL;
+    J.theta = theta;
     J.S0 = S0;
     J.out = out;
     J.S_final = S_final;
