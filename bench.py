@@ -44,6 +44,8 @@ DENSE_FLOPS_PER_TOKEN_HEAD = 12 * CHUNK * D + 6 * D * D
 DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4
 # Gated DeltaNet-2 forward: q, k, v bf16 + alpha, b (d_k) and w (d_v) fp32 + out fp32
 GDN2_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + D * 4 + D * 4 + D * 4
+# SFDA forward: q, k, v bf16 + alpha and theta (d_k / 2 each) fp32 + beta + out fp32
+SFDA_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + 2 * (D // 2) * 4 + 4 + D * 4
 
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
@@ -69,6 +71,8 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS,
                     help="decode steps timed (inputs for all of them are pre-generated)")
+    ap.add_argument("--no-sfda", action="store_true",
+                    help="skip the SFDA (phase-decay gates) sub-measure")
     ap.add_argument("--no-gdn2", action="store_true",
                     help="skip the Gated DeltaNet-2 forward measurement")
     ap.add_argument("--json-out", default=None)
@@ -305,9 +309,12 @@ def run_ours(args, ws, rank, local):
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
     path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
-    gdn2 = None
-    if not args.no_gdn2:
-        gdn2 = _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak)
+    variants = {}
+    for kind, off in (("gdn2", args.no_gdn2), ("sfda", args.no_sfda)):
+        if not off:
+            variants[kind] = _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier,
+                                          max_ranks, ws, hbm_peak, steps=20 if kind == "gdn2"
+                                          else 10)
     wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
                         device=dev)
     two_phase = path == "tcgen05"
@@ -389,7 +396,7 @@ def run_ours(args, ws, rank, local):
                              ws, hbm_peak)
     _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            _lib.LIB_PATH, path, kernels, gdn2)
+            _lib.LIB_PATH, path, kernels, variants)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -431,11 +438,17 @@ def _run_e2e(args, ck, torch, c, out, S_final, stream, barrier, max_ranks, ws, t
             "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
 
-def _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=20):
-    """Gated DeltaNet-2 forward at the bench sizes (bf16 q/k/v, fp32 gates and
-    output); two rotating input sets."""
-    sets = [inputs.gdn2_prefill(B, T, H, D, D, dtype=torch.bfloat16, chunk=CHUNK,
-                                seed=3000 + 10 * rank + i, device=dev) for i in range(2)]
+def _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak,
+                 steps=20):
+    """A variant's forward at the bench sizes (bf16 q/k/v, fp32 gates and
+    output); two rotating input sets.  kind "gdn2": Gated DeltaNet-2 (erase and
+    write gates); kind "sfda": SFDA (phase-decay gates)."""
+    if kind == "gdn2":
+        sets = [inputs.gdn2_prefill(B, T, H, D, D, dtype=torch.bfloat16, chunk=CHUNK,
+                                    seed=3000 + 10 * rank + i, device=dev) for i in range(2)]
+    else:
+        sets = [inputs.sfda_prefill(B, T, H, D, D, dtype=torch.bfloat16, chunk=CHUNK,
+                                    seed=4000 + 10 * rank + i, device=dev) for i in range(2)]
     out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
@@ -443,8 +456,12 @@ def _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
 
     def step(i):
         c = sets[i % 2]
-        ck.gdn2_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], chunk=CHUNK,
-                            out=out, S_final=S_final, workspace=wsbuf)
+        if kind == "gdn2":
+            ck.gdn2_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], chunk=CHUNK,
+                                out=out, S_final=S_final, workspace=wsbuf)
+        else:
+            ck.sfda_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["theta"], c.beta, chunk=CHUNK,
+                                out=out, S_final=S_final)
 
     for i in range(3):
         step(i)
@@ -461,12 +478,18 @@ def _run_gdn2(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
     torch.cuda.synchronize(dev)
     barrier()
     ms = max_ranks(ev0.elapsed_time(ev1)) / steps
-    nbytes = B * T * H * GDN2_BYTES_PER_TOKEN_HEAD + B * H * D * D * 4
+    per_th = GDN2_BYTES_PER_TOKEN_HEAD if kind == "gdn2" else SFDA_BYTES_PER_TOKEN_HEAD
+    nbytes = B * T * H * per_th + B * H * D * D * 4
     gbs = nbytes / (ms / 1e3) / 1e9
     del sets
-    path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
-    return {"workload": f"gdn2_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 "
-                        f"alpha/b/w, fp32 out ({path} kernels)",
+    if kind == "gdn2":
+        path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
+        what = f"gdn2_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 alpha/b/w"
+    else:
+        path = "fp32core"
+        what = (f"sfda_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 "
+                f"alpha/theta (d/2 pairs)/beta")
+    return {"workload": f"{what}, fp32 out ({path} kernels)",
             "ms_per_step": ms, "tokens_per_s": ws * B * T / (ms / 1e3),
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_frac_of_measured": gbs / hbm_peak, "gpu_launches": steps}
@@ -504,7 +527,7 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, 
 
 def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            lib_path, path, kernels=None, gdn2=None):
+            lib_path, path, kernels=None, variants=None):
     # arithmetic of the forward: tcgen05 MMAs on fp16 operands with fp32
     # accumulation and fp32 state, or fp32 FFMA on CUDA cores
     dtype = "f16" if path == "tcgen05" else "f32"
@@ -541,8 +564,8 @@ def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_
     }
     if decode is not None:
         obj["decode"] = decode
-    if gdn2 is not None:
-        obj["gdn2"] = gdn2
+    for kind, res in (variants or {}).items():
+        obj[kind] = res
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         obj["cpu_baseline"] = cpu_baseline()
     _emit(obj, args, rank)

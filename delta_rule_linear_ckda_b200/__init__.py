@@ -8,13 +8,13 @@ without the native library.
 """
 from __future__ import annotations
 
-__all__ = ["fwd_chunked", "fwd_chunked_static", "gdn2_fwd_chunked", "fwd_factors", "fwd_carry", "fwd_path", "workspace_bytes", "decode_step",
-           "device_status", "CKDAError", "lib_path"]
+_API = ("fwd_chunked", "fwd_chunked_static", "gdn2_fwd_chunked", "sfda_fwd_chunked", "fwd_factors",
+        "fwd_carry", "fwd_path", "workspace_bytes", "decode_step", "device_status")
+__all__ = list(_API) + ["CKDAError", "lib_path"]
 
 
 def __getattr__(name):
-    if name in ("fwd_chunked", "fwd_chunked_static", "gdn2_fwd_chunked", "fwd_factors", "fwd_carry", "fwd_path", "workspace_bytes",
-                "decode_step", "device_status"):
+    if name in _API:
         from . import api
 
         api._lib.load()

@@ -128,8 +128,9 @@ def fwd_chunked_static(q, k, v, alpha, beta, S0=None, cu_seqlens=None, chunk: in
     return out, S_final
 
 
-def _inputs_shape(q, k, v, alpha, beta, cu_seqlens):
-    """Checks the forward inputs; returns (B, T, H, dk, dv, N) as passed to the ABI."""
+def _inputs_shape(q, k, v, alpha, beta, cu_seqlens, pair_gates=False):
+    """Checks the forward inputs; returns (B, T, H, dk, dv, N) as passed to the ABI.
+    ``pair_gates``: alpha holds one decay per channel pair (last dim dk / 2)."""
     dev = q.device
     if q.dtype not in _DT:
         raise TypeError("q, k, v must be float32 or bfloat16")
@@ -153,8 +154,12 @@ def _inputs_shape(q, k, v, alpha, beta, cu_seqlens):
         N = cu_seqlens.numel() - 1
         B = N
     dv = v.shape[-1]
-    if k.shape != q.shape or alpha.shape != q.shape or v.shape[:-1] != q.shape[:-1]:
-        raise ValueError("q, k, alpha must share a shape and v must match it but for the last dim")
+    a_shape = q.shape[:-1] + (dk // 2,) if pair_gates else q.shape
+    if pair_gates and dk % 2:
+        raise ValueError("the phase-decay gates pair the key channels: dk must be even")
+    if k.shape != q.shape or alpha.shape != a_shape or v.shape[:-1] != q.shape[:-1]:
+        raise ValueError("q, k, alpha must share a shape (alpha: last dim dk / 2 for paired "
+                         "gates) and v must match it but for the last dim")
     if tuple(beta.shape) != tuple(q.shape[:-1]):
         raise ValueError("beta must have q's shape without the last dim")
     return B, T, H, dk, dv, N
@@ -260,6 +265,46 @@ def gdn2_fwd_chunked(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk: int 
             0 if workspace is None else workspace.numel(), _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_gdn2_fwd_chunked")
+    return out, S_final
+
+
+def sfda_fwd_chunked(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, chunk: int = 64,
+                     out=None, S_final=None, return_final: bool = True, out_dtype=None):
+    """Chunked SFDA forward (``ckda_sfda_fwd_chunked``): the CKDA recurrence with
+    Diag(alpha) replaced by phase-decay blocks ``alpha_p R(theta_p)`` on the key
+    channel pairs ``(2p, 2p+1)``.  ``alpha`` and ``theta`` are fp32 shaped like
+    ``k`` with the last dim halved; beta and the other arguments as in
+    ``fwd_chunked`` (no workspace: this form runs on the fp32 CUDA-core kernel)."""
+    dev = q.device
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, cu_seqlens, pair_gates=True)
+    _need(theta, "theta", torch.float32, dev)
+    if theta.shape != alpha.shape:
+        raise ValueError("theta must have alpha's shape")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must have v's shape")
+    if return_final and S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_sfda_fwd_chunked(
+            _p(q), _p(k), _p(v), _p(alpha), _p(theta), _p(beta), _p(S0), _p(cu_seqlens),
+            _p(out), _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
+            _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_sfda_fwd_chunked")
     return out, S_final
 
 

@@ -14,9 +14,9 @@ cudaError_t launch_decode(int dtype, int out_dtype, int dk, int dv, const void* 
                           int BH, cudaStream_t stream);
 cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
                             const void* k, const void* v, const float* alpha, const float* beta,
-                            const float* bg, const float* wg, const float* S0,
-                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T,
-                            int H, int C, int* status, cudaStream_t stream);
+                            const float* bg, const float* wg, const float* theta,
+                            const float* S0, const int32_t* cu, void* out, float* S_final,
+                            int n_seqs, int T, int H, int C, int* status, cudaStream_t stream);
 // Returns cudaErrorNotSupported when the shape is not covered by the
 // tensor-core kernels (the caller then uses the CUDA-core kernel).
 cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
@@ -107,24 +107,31 @@ int validate_fwd(const void* q, const void* k, const void* v, const float* alpha
 }
 
 // `bg` and `wg` non-NULL select the Gated DeltaNet-2 form: `bg` takes beta's
-// place in the shared checks, `wg` is checked here.
+// place in the shared checks, `wg` is checked here.  `sfda` selects the SFDA
+// form: `theta` (required when there are tokens) is checked here.
 int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void* v,
              const float* alpha, const float* beta, const float* bg, const float* wg,
              const float* S0, const int32_t* cu, void* out, float* S_final, int B, int T, int H,
              int d_k, int d_v, int chunk, int dtype, int out_dtype, void* workspace,
-             size_t workspace_bytes, void* stream) {
+             size_t workspace_bytes, void* stream, bool sfda = false,
+             const float* theta = nullptr) {
   const bool gdn2 = bg != nullptr || wg != nullptr;
   int rc = validate_fwd(q, k, v, alpha, gdn2 ? bg : beta, S0, cu, out, S_final, B, T, H, d_k,
                         d_v, &chunk, dtype, out_dtype, phases);
   if (rc != CKDA_OK) return rc;
+  const int64_t tokens = (cu != nullptr) ? (int64_t)T : (int64_t)B * T;
   if (gdn2) {
-    const int64_t tokens = (cu != nullptr) ? (int64_t)T : (int64_t)B * T;
     if (tokens > 0 && (bg == nullptr || wg == nullptr)) return CKDA_ERR_INVALID_ARG;
     if (wg != nullptr && !aligned16(wg)) return CKDA_ERR_MISALIGNED;
     if (out != nullptr && out == wg) return CKDA_ERR_INVALID_ARG;
   }
+  if (sfda) {
+    if (tokens > 0 && theta == nullptr) return CKDA_ERR_INVALID_ARG;
+    if (theta != nullptr && !aligned16(theta)) return CKDA_ERR_MISALIGNED;
+    if (out != nullptr && out == theta) return CKDA_ERR_INVALID_ARG;
+  }
   const int n_seqs = B;
-  const bool tc = allow_tc && n_seqs > 0 &&
+  const bool tc = allow_tc && !sfda && n_seqs > 0 &&
                   ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, n_seqs, T, H, cu != nullptr);
   // the two-phase calls exist only on the tensor-core path
   if (phases != kBoth && !tc && n_seqs > 0) return CKDA_ERR_UNSUPPORTED;
@@ -148,8 +155,9 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
     e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg, S0,
                             cu, out, S_final, n_seqs, T, H, chunk, workspace, status, st);
   if (e == cudaErrorNotSupported)
-    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg, S0, cu,
-                              out, S_final, n_seqs, T, H, chunk, status, st);
+    e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg,
+                              sfda ? theta : nullptr, S0, cu, out, S_final, n_seqs, T, H, chunk,
+                              status, st);
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
@@ -219,6 +227,16 @@ int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v, const flo
   // (both gates NULL: checked as the beta form with beta NULL)
   return fwd_impl(true, kBoth, q, k, v, alpha, nullptr, b, w, S0, cu_seqlens, out, S_final, B,
                   T, H, d_k, d_v, chunk, dtype, out_dtype, workspace, workspace_bytes, stream);
+}
+
+int ckda_sfda_fwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* theta, const float* beta, const float* S0,
+                          const int32_t* cu_seqlens, void* out, float* S_final, int B, int T,
+                          int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
+                          void* stream) {
+  return fwd_impl(false, kBoth, q, k, v, alpha, beta, nullptr, nullptr, S0, cu_seqlens, out,
+                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, nullptr, 0, stream,
+                  /*sfda=*/true, theta);
 }
 
 int ckda_fwd_factors(const void* q, const void* k, const void* v, const float* alpha,

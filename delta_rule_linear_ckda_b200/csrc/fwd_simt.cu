@@ -26,6 +26,18 @@
 //   T[r, s] = sum_i e_ri k_si P_i(r, s),   [W | U~] = (I + T)^-1 [E * Gamma | Z]
 // and everything else unchanged; the G2 instantiation computes that form.
 //
+// SFDA ("Semidirect Fourier Delta Attention (SFDA)" page, "Arquitectura
+// Central") replaces Diag(alpha_r) by the phase-decay gate Lambda_r, block
+// diagonal with 2x2 blocks lambda_rp = alpha_rp (cos theta_rp, sin theta_rp)
+// read as complex scalars acting on the channel pairs (2p, 2p+1).  Gate
+// products stay products of those complex scalars (still division-free), and
+// with P(r, s) = Lambda_r ... Lambda_{s+1}:
+//   T[r, s] = beta_r k_r^T P(r, s) k_s,   A[r, s] = q_r^T P(r, s) k_s
+//   W rows beta_r Gamma_r^T k_r, Q' rows Gamma_r^T q_r  (conjugate products)
+//   K-hat rows P(C-1, s) k_s,   S_C = Gamma S0 + K-hat^T U  (Gamma on row pairs)
+// which the SFDA instantiation computes.  Zero phases reproduce the CKDA
+// instantiation bit for bit when the decays of a pair are equal.
+//
 // One CTA owns one (sequence, head, d_v slice of width BV) and walks its
 // chunks in order; the slice of the state stays in shared memory in fp32.
 #include "common.cuh"
@@ -35,6 +47,11 @@ namespace simt {
 
 constexpr int kThreads = 256;
 constexpr int kMaxC = 64;
+
+// Gate families of the kernel.
+constexpr int kKda = 0;   // beta_r, Diag(alpha_r)
+constexpr int kGdn2 = 1;  // erase gate b_r, write gate w_r, Diag(alpha_r)
+constexpr int kSfda = 2;  // beta_r, phase-decay blocks alpha_rp e^{i theta_rp}
 
 template <int DK, int BV>
 struct Smem {
@@ -106,26 +123,38 @@ __device__ __forceinline__ void reduce_scatter8(float* v, int lane) {
   v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
 }
 
-template <int DK, int BV, typename Tin, typename Tout, bool G2>
+// (a + ib)(x + iy), real and imaginary parts; with b = 0 the results are
+// exactly a x and a y.
+__device__ __forceinline__ float cmul_re(float a, float b, float x, float y) {
+  return fmaf(-b, y, a * x);
+}
+__device__ __forceinline__ float cmul_im(float a, float b, float x, float y) {
+  return fmaf(b, x, a * y);
+}
+
+template <int DK, int BV, typename Tin, typename Tout, int GK>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __restrict__ v,
                 const float* __restrict__ alpha, const float* __restrict__ beta,
-                const float* __restrict__ bg, const float* __restrict__ wg, const float* S0,
+                const float* __restrict__ bg, const float* __restrict__ wg,
+                const float* __restrict__ theta, const float* S0,
                 const int32_t* __restrict__ cu, Tout* __restrict__ out, float* S_final,
                 int n_seqs, int T, int H, int DV, int C, int* status) {
+  constexpr bool G2 = GK == kGdn2;
+  constexpr bool SF = GK == kSfda;
   using L = Smem<DK, BV>;
   constexpr int KS = L::KS, VS = L::VS, CS = L::CS;
   extern __shared__ __align__(16) float smem[];
   float* Ks = smem + L::kK;   // k, then K * rho
   float* Qs = smem + L::kQ;   // q, then Q * Gamma
-  float* As = smem + L::kA;   // alpha
+  float* As = smem + L::kA;   // alpha (SFDA: lambda pairs, real then imaginary part)
   float* Ws = smem + L::kW;   // beta K Gamma, then W (G2: E = b * k, then E * Gamma, then W)
   float* Vs = smem + L::kV;   // v, then beta v (G2: w * v), then U~, then U
   float* Tm = smem + L::kT;   // T (strictly lower)
   float* Am = smem + L::kAm;  // A (lower incl. diagonal)
   float* Ss = smem + L::kS;   // state slice [DK][BV]
   float* bs = smem + L::kBeta;
-  float* gs = smem + L::kGam;
+  float* gs = smem + L::kGam;  // gamma (SFDA: complex pairs)
 
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -152,13 +181,25 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     // ---- stage inputs (fp32), identity transitions past the end ---------
     for (int e = tid; e < C * DK / 4; e += kThreads) {
       const int r = e / (DK / 4), c4 = e % (DK / 4);
-      float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk, aa = make_float4(1.f, 1.f, 1.f, 1.f);
+      float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), qq = kk;
+      float4 aa = SF ? make_float4(1.f, 0.f, 1.f, 0.f) : make_float4(1.f, 1.f, 1.f, 1.f);
       float4 ee = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < Lc) {
         const size_t off = ((size_t)(t0 + r) * H + h) * DK + 4 * c4;
         kk = load4_f32(k + off);
         qq = load4_f32(q + off);
-        aa = *reinterpret_cast<const float4*>(alpha + off);
+        if constexpr (SF) {
+          // channels 4 c4 .. 4 c4 + 3 are the pairs 2 c4 and 2 c4 + 1
+          const size_t goff = ((size_t)(t0 + r) * H + h) * (DK / 2) + 2 * c4;
+          const float2 a2 = *reinterpret_cast<const float2*>(alpha + goff);
+          const float2 t2 = *reinterpret_cast<const float2*>(theta + goff);
+          float s0, c0, s1, c1;
+          sincosf(t2.x, &s0, &c0);
+          sincosf(t2.y, &s1, &c1);
+          aa = make_float4(a2.x * c0, a2.x * s0, a2.y * c1, a2.y * s1);
+        } else {
+          aa = *reinterpret_cast<const float4*>(alpha + off);
+        }
         if constexpr (G2) {
           const float4 bb = *reinterpret_cast<const float4*>(bg + off);
           ee = make_float4(bb.x * kk.x, bb.y * kk.y, bb.z * kk.z, bb.w * kk.w);
@@ -227,9 +268,29 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
                 lds<CPL>((G2 ? Ws : Ks) + r * KS + cb, kr);
                 lds<CPL>(Qs + r * KS + cb, qr);
               }
+              if constexpr (SF) {
+                // x <- lambda_r x on every channel pair
+                if constexpr (CPL >= 2) {
+#pragma unroll
+                  for (int c = 0; c < CPL; c += 2) {
+                    const float xr = x[c], xi = x[c + 1];
+                    x[c] = cmul_re(a[c], a[c + 1], xr, xi);
+                    x[c + 1] = cmul_im(a[c], a[c + 1], xr, xi);
+                  }
+                } else {
+                  // one channel per lane: the pair partner is the neighbouring lane
+                  const float xo = __shfl_xor_sync(0xffffffffu, x[0], 1);
+                  const float lo = __shfl_xor_sync(0xffffffffu, a[0], 1);
+                  const bool odd = lane & 1;
+                  const float lre = odd ? lo : a[0], lim = odd ? a[0] : lo;
+                  x[0] = odd ? cmul_im(lre, lim, xo, x[0]) : cmul_re(lre, lim, x[0], xo);
+                }
+              } else {
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) x[c] *= a[c];
+              }
 #pragma unroll
               for (int c = 0; c < CPL; ++c) {
-                x[c] *= a[c];
                 pk[jj] = fmaf(kr[c], x[c], pk[jj]);
                 pq[jj] = fmaf(qr[c], x[c], pq[jj]);
               }
@@ -251,7 +312,38 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     // forward: Gamma_r (inclusive prefix); W rhs = beta K Gamma (G2: E Gamma);
     // Q <- Q Gamma
     // backward: rho_s (exclusive suffix); K <- K rho
-    if (tid < DK) {
+    if constexpr (SF) {
+      // one thread per channel pair p: complex running products
+      if (tid < DK / 2) {
+        const int e = 2 * tid, o = e + 1;
+        float gr = 1.f, gi = 0.f;
+        for (int r = 0; r < C; ++r) {
+          const float lr = As[r * KS + e], li = As[r * KS + o];
+          const float nr = cmul_re(gr, gi, lr, li), ni = cmul_im(gr, gi, lr, li);
+          gr = nr;
+          gi = ni;
+          // beta_r Gamma_r^T k_r and Gamma_r^T q_r: multiply by conj(gamma)
+          const float ke = bs[r] * Ks[r * KS + e], ko = bs[r] * Ks[r * KS + o];
+          Ws[r * KS + e] = cmul_re(gr, -gi, ke, ko);
+          Ws[r * KS + o] = cmul_im(gr, -gi, ke, ko);
+          const float qe = Qs[r * KS + e], qo = Qs[r * KS + o];
+          Qs[r * KS + e] = cmul_re(gr, -gi, qe, qo);
+          Qs[r * KS + o] = cmul_im(gr, -gi, qe, qo);
+        }
+        gs[e] = gr;
+        gs[o] = gi;
+        float pr = 1.f, pi = 0.f;
+        for (int s = C - 1; s >= 0; --s) {
+          const float ke = Ks[s * KS + e], ko = Ks[s * KS + o];
+          Ks[s * KS + e] = cmul_re(pr, pi, ke, ko);
+          Ks[s * KS + o] = cmul_im(pr, pi, ke, ko);
+          const float lr = As[s * KS + e], li = As[s * KS + o];
+          const float nr = cmul_re(pr, pi, lr, li), ni = cmul_im(pr, pi, lr, li);
+          pr = nr;
+          pi = ni;
+        }
+      }
+    } else if (tid < DK) {
       const int i = tid;
       float gmm = 1.f;
       for (int r = 0; r < C; ++r) {
@@ -377,14 +469,30 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
           acc[m].z = fmaf(khv[m], u4.z, acc[m].z); acc[m].w = fmaf(khv[m], u4.w, acc[m].w);
         }
       }
+      if constexpr (SF) {
+        // rows (i0, i0 + 1) and (i0 + 2, i0 + 3) are channel pairs
 #pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        float4* sp = reinterpret_cast<float4*>(Ss + (i0 + m) * VS + cc);
-        float4 sv = *sp;
-        const float g = gs[i0 + m];
-        sv.x = fmaf(g, sv.x, acc[m].x); sv.y = fmaf(g, sv.y, acc[m].y);
-        sv.z = fmaf(g, sv.z, acc[m].z); sv.w = fmaf(g, sv.w, acc[m].w);
-        *sp = sv;
+        for (int m = 0; m < 4; m += 2) {
+          float4* pe = reinterpret_cast<float4*>(Ss + (i0 + m) * VS + cc);
+          float4* po = reinterpret_cast<float4*>(Ss + (i0 + m + 1) * VS + cc);
+          const float4 se = *pe, so = *po;
+          const float gr = gs[i0 + m], gi = gs[i0 + m + 1];
+          const float4 ae = acc[m], ao = acc[m + 1];
+          *pe = make_float4(fmaf(gr, se.x, fmaf(-gi, so.x, ae.x)), fmaf(gr, se.y, fmaf(-gi, so.y, ae.y)),
+                            fmaf(gr, se.z, fmaf(-gi, so.z, ae.z)), fmaf(gr, se.w, fmaf(-gi, so.w, ae.w)));
+          *po = make_float4(fmaf(gr, so.x, fmaf(gi, se.x, ao.x)), fmaf(gr, so.y, fmaf(gi, se.y, ao.y)),
+                            fmaf(gr, so.z, fmaf(gi, se.z, ao.z)), fmaf(gr, so.w, fmaf(gi, se.w, ao.w)));
+        }
+      } else {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          float4* sp = reinterpret_cast<float4*>(Ss + (i0 + m) * VS + cc);
+          float4 sv = *sp;
+          const float g = gs[i0 + m];
+          sv.x = fmaf(g, sv.x, acc[m].x); sv.y = fmaf(g, sv.y, acc[m].y);
+          sv.z = fmaf(g, sv.z, acc[m].z); sv.w = fmaf(g, sv.w, acc[m].w);
+          *sp = sv;
+        }
       }
     }
   }
@@ -398,63 +506,68 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
   }
 }
 
-// Gates of a call: beta (CKDA) or the erase and write gates (G2).
+// Gates of a call: beta (CKDA), the erase and write gates (Gated DeltaNet-2)
+// or beta with the phases (SFDA).
 struct Gates {
   const float* beta;
   const float* b;
   const float* w;
+  const float* theta;
 };
 
-template <int DK, int BV, typename Tin, typename Tout, bool G2>
+template <int DK, int BV, typename Tin, typename Tout, int GK>
 static cudaError_t launch_t(const void* q, const void* k, const void* v, const float* alpha,
                             Gates gt, const float* S0, const int32_t* cu, void* out,
                             float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
                             cudaStream_t stream) {
   using L = Smem<DK, BV>;
-  auto kern = fwd_simt_kernel<DK, BV, Tin, Tout, G2>;
+  auto kern = fwd_simt_kernel<DK, BV, Tin, Tout, GK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L::kBytes);
   if (e != cudaSuccess) return e;
   dim3 grid(DV / BV, H, n_seqs);
   kern<<<grid, kThreads, L::kBytes, stream>>>(
       static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
-      gt.beta, gt.b, gt.w, S0, cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
+      gt.beta, gt.b, gt.w, gt.theta, S0, cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
   return cudaGetLastError();
 }
 
-template <int DK, typename Tin, typename Tout, bool G2>
+template <int DK, typename Tin, typename Tout, int GK>
 static cudaError_t launch_bv(const void* q, const void* k, const void* v, const float* alpha,
                              Gates gt, const float* S0, const int32_t* cu, void* out,
                              float* S_final, int n_seqs, int T, int H, int DV, int C, int* status,
                              cudaStream_t stream) {
   switch (DV) {
     case 16:
-      return launch_t<DK, 16, Tin, Tout, G2>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
+      return launch_t<DK, 16, Tin, Tout, GK>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
                                              DV, C, status, stream);
     case 32:
-      return launch_t<DK, 32, Tin, Tout, G2>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
+      return launch_t<DK, 32, Tin, Tout, GK>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
                                              DV, C, status, stream);
     default:  // 64 and 128: slices of 64 columns
-      return launch_t<DK, 64, Tin, Tout, G2>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
+      return launch_t<DK, 64, Tin, Tout, GK>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H,
                                              DV, C, status, stream);
   }
 }
 
 }  // namespace simt
 
-// `bg` and `wg` non-NULL select the Gated DeltaNet-2 form (beta unused).
+// `bg` and `wg` non-NULL select the Gated DeltaNet-2 form (beta unused);
+// `theta` non-NULL selects the SFDA form (alpha then holds dk / 2 decays).
 cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
                             const void* k, const void* v, const float* alpha, const float* beta,
-                            const float* bg, const float* wg, const float* S0,
-                            const int32_t* cu, void* out, float* S_final, int n_seqs, int T,
-                            int H, int C, int* status, cudaStream_t stream) {
-  const simt::Gates gt{beta, bg, wg};
-  const bool g2 = bg != nullptr;
-#define CKDA_SIMT_CALL(DKV, TI, TO)                                                            \
-  (g2 ? simt::launch_bv<DKV, TI, TO, true>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, \
-                                           H, dv, C, status, stream)                           \
-      : simt::launch_bv<DKV, TI, TO, false>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs,   \
-                                            T, H, dv, C, status, stream))
+                            const float* bg, const float* wg, const float* theta,
+                            const float* S0, const int32_t* cu, void* out, float* S_final,
+                            int n_seqs, int T, int H, int C, int* status, cudaStream_t stream) {
+  const simt::Gates gt{beta, bg, wg, theta};
+  const int gk = theta != nullptr ? simt::kSfda : (bg != nullptr ? simt::kGdn2 : simt::kKda);
+#define CKDA_SIMT_GK(DKV, TI, TO, GKV) \
+  simt::launch_bv<DKV, TI, TO, GKV>(q, k, v, alpha, gt, S0, cu, out, S_final, n_seqs, T, H, dv, C, \
+                                    status, stream)
+#define CKDA_SIMT_CALL(DKV, TI, TO)                                     \
+  (gk == simt::kSfda   ? CKDA_SIMT_GK(DKV, TI, TO, simt::kSfda)          \
+   : gk == simt::kGdn2 ? CKDA_SIMT_GK(DKV, TI, TO, simt::kGdn2)          \
+                       : CKDA_SIMT_GK(DKV, TI, TO, simt::kKda))
 #define CKDA_SIMT_DK(DKV)                                                                  \
   case DKV:                                                                                \
     if (dtype == CKDA_BF16)                                                                \
@@ -470,6 +583,7 @@ cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void
   }
 #undef CKDA_SIMT_DK
 #undef CKDA_SIMT_CALL
+#undef CKDA_SIMT_GK
   return cudaErrorInvalidValue;
 }
 

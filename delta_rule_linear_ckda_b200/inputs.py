@@ -31,6 +31,8 @@ from __future__ import annotations
 from dataclasses import dataclass, field
 from typing import Optional
 
+import math
+
 import torch
 
 F32 = torch.float32
@@ -153,6 +155,27 @@ def gdn2_prefill(B, T, H, dk, dv, *, dtype=F32, s0_std=0.0, chunk=64, seed=0, de
     case = PrefillCase(name, q, k, v, alpha.contiguous(), None, S0, None, chunk)
     case.extra["b"] = b
     case.extra["w"] = w
+    return case
+
+
+def sfda_prefill(B, T, H, dk, dv, *, dtype=F32, s0_std=0.0, chunk=64, seed=0, device="cpu",
+                 name="sfda") -> PrefillCase:
+    """SFDA batch: q, k normalised, v ~ N(0,1), beta = 2 sigmoid(z) as the KDA
+    prefill recipe; per channel pair a decay alpha = sigmoid(-x) in (0, 1) and
+    a phase theta ~ U[-pi, pi) (the phase carries the sign), x, z ~ N(0,1).
+    ``alpha`` is [B, T, H, dk / 2]; the phases go to ``extra["theta"]``."""
+    g = _gen(device, seed)
+    q = _l2n(_normal((B, T, H, dk), g, device)).to(dtype)
+    k = _l2n(_normal((B, T, H, dk), g, device)).to(dtype)
+    v = _normal((B, T, H, dv), g, device).to(dtype)
+    alpha = torch.sigmoid(-_normal((B, T, H, dk // 2), g, device)).to(F32).contiguous()
+    theta = _uniform((B, T, H, dk // 2), -math.pi, math.pi, g, device).contiguous()
+    beta = (2.0 * torch.sigmoid(_normal((B, T, H), g, device))).to(F32).contiguous()
+    S0 = None
+    if s0_std > 0:
+        S0 = (_normal((B, H, dk, dv), g, device) * s0_std).contiguous()
+    case = PrefillCase(name, q, k, v, alpha, beta, S0, None, chunk)
+    case.extra["theta"] = theta
     return case
 
 

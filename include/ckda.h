@@ -233,6 +233,40 @@ CKDA_API int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v,
                                    size_t workspace_bytes, void* stream);
 
 /*
+ * ckda_sfda_fwd_chunked -- chunkwise forward of the SFDA (phase-controlled)
+ * recurrence ("Semidirect Fourier Delta Attention (SFDA)" technical summary,
+ * "Arquitectura Central"), in real coordinates:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Lambda_t S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,
+ *
+ * with Lambda_t block diagonal: block p (p = 0 .. d_k/2 - 1) acts on the
+ * state rows (2p, 2p+1) as
+ *     alpha_p * [[cos theta_p, -sin theta_p], [sin theta_p, cos theta_p]],
+ * the real form of the complex gate alpha_p e^{i theta_p} on a channel whose
+ * real part is row 2p and imaginary part row 2p+1.  Zero phases give back
+ * ckda_fwd_chunked's recurrence with each decay on both rows of its pair; a
+ * phase of pi is a negative real gate.  The chunk form is the same WY
+ * factorisation with the channel-wise gate products replaced by products of
+ * these complex scalars ("El Teorema de Chunk-WY Constructivo").
+ *
+ *   alpha  fp32 [B, T, H, d_k / 2]  (packed: [T, H, d_k / 2]) decays
+ *   theta  fp32 [B, T, H, d_k / 2]  (packed: [T, H, d_k / 2]) phases, radians
+ * Both are applied as given (|alpha| <= 1 keeps the transitions
+ * non-expansive).  Every other argument, layout, ownership and error rule is
+ * that of ckda_fwd_chunked, except that no workspace is taken: this form
+ * runs on the fp32 CUDA-core kernel for every shape (any d_k, d_v in
+ * {16, 32, 64, 128}, chunk 16, 32 or 64; fp32 or bf16 inputs), with cos and
+ * sin of each phase evaluated once per token in fp32.  theta must be
+ * non-NULL when there are tokens, 16-byte aligned and not aliased by out.
+ */
+CKDA_API int ckda_sfda_fwd_chunked(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* theta, const float* beta,
+                                   const float* S0, const int32_t* cu_seqlens, void* out,
+                                   float* S_final, int B, int T, int H, int d_k, int d_v,
+                                   int chunk, int dtype, int out_dtype, void* stream);
+
+/*
  * ckda_fwd_chunked_workspace_bytes -- scratch bytes ckda_fwd_chunked needs
  * for these sizes (same meaning of B, T and `varlen` as in
  * ckda_fwd_chunked_path), 0 when the call runs the fp32 CUDA-core kernel,

@@ -264,3 +264,24 @@ def test_gdn2_entry_validates_its_gates(lib):
     assert g2(B=0) == 0
     # the tensor-core shapes need the same workspace as ckda_fwd_chunked
     assert g2(dtype=1, dk=128, dv=128, chunk=64, T=128) == -7
+
+
+def test_sfda_entry_validates_its_gates(lib):
+    def sf(**kw):
+        a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, theta=P + 0x4000,
+                 beta=P + 0x6000, S0=None, cu=None, out=P + 0x5000, S_final=None, B=1, T=8, H=1,
+                 dk=16, dv=16, chunk=16, dtype=0, out_dtype=0)
+        a.update(kw)
+        return lib.ckda_sfda_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["theta"],
+                                         a["beta"], a["S0"], a["cu"], a["out"], a["S_final"],
+                                         a["B"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"],
+                                         a["dtype"], a["out_dtype"], None)
+
+    assert sf(theta=None) == -1
+    assert sf(alpha=None) == -1
+    assert sf(beta=None) == -1
+    assert sf(theta=MIS) == -3
+    assert sf(out=P + 0x4000) == -1   # out aliases theta
+    assert sf(dk=48) == -2
+    assert sf(chunk=128) == -2
+    assert sf(B=0) == 0
