@@ -313,8 +313,7 @@ def run_ours(args, ws, rank, local):
     for kind, off in (("gdn2", args.no_gdn2), ("sfda", args.no_sfda)):
         if not off:
             variants[kind] = _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier,
-                                          max_ranks, ws, hbm_peak, steps=20 if kind == "gdn2"
-                                          else 10)
+                                          max_ranks, ws, hbm_peak)
     wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
                         device=dev)
     two_phase = path == "tcgen05"
@@ -461,7 +460,7 @@ def _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
                                 out=out, S_final=S_final, workspace=wsbuf)
         else:
             ck.sfda_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["theta"], c.beta, chunk=CHUNK,
-                                out=out, S_final=S_final)
+                                out=out, S_final=S_final, workspace=wsbuf)
 
     for i in range(3):
         step(i)
@@ -486,13 +485,14 @@ def _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
         path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
         what = f"gdn2_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 alpha/b/w"
     else:
-        path = "fp32core"
+        path = ck.fwd_path(B, T, H, D, D, CHUNK, torch.bfloat16, torch.float32)
         what = (f"sfda_prefill B={B} H={H} T={T} d={D} C={CHUNK} bf16 q/k/v, fp32 "
                 f"alpha/theta (d/2 pairs)/beta")
     return {"workload": f"{what}, fp32 out ({path} kernels)",
             "ms_per_step": ms, "tokens_per_s": ws * B * T / (ms / 1e3),
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
-            "hbm_frac_of_measured": gbs / hbm_peak, "gpu_launches": steps}
+            "hbm_frac_of_measured": gbs / hbm_peak,
+            "gpu_launches": steps * (2 if path == "tcgen05" else 1)}
 
 
 def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak):

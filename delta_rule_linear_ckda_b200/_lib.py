@@ -39,7 +39,9 @@ SIGNATURES = {
     "ckda_gdn2_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
                                    _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp]),
     "ckda_sfda_fwd_chunked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i,
-                                   _i, _i, _i, _i, _vp]),
+                                   _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp]),
+    "ckda_sfda_fwd_chunked_fp32core": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
+                                            _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_fwd_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
                               ctypes.c_size_t, _vp]),
     "ckda_fwd_carry": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,

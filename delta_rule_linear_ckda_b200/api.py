@@ -269,12 +269,13 @@ def gdn2_fwd_chunked(q, k, v, alpha, b, w, S0=None, cu_seqlens=None, chunk: int 
 
 
 def sfda_fwd_chunked(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, chunk: int = 64,
-                     out=None, S_final=None, return_final: bool = True, out_dtype=None):
+                     out=None, S_final=None, return_final: bool = True, out_dtype=None,
+                     workspace=None, fp32core: bool = False):
     """Chunked SFDA forward (``ckda_sfda_fwd_chunked``): the CKDA recurrence with
     Diag(alpha) replaced by phase-decay blocks ``alpha_p R(theta_p)`` on the key
     channel pairs ``(2p, 2p+1)``.  ``alpha`` and ``theta`` are fp32 shaped like
-    ``k`` with the last dim halved; beta and the other arguments as in
-    ``fwd_chunked`` (no workspace: this form runs on the fp32 CUDA-core kernel)."""
+    ``k`` with the last dim halved; beta, the workspace and the other arguments
+    as in ``fwd_chunked`` (``fp32core`` forces the fp32 CUDA-core kernel)."""
     dev = q.device
     B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, cu_seqlens, pair_gates=True)
     _need(theta, "theta", torch.float32, dev)
@@ -298,11 +299,26 @@ def sfda_fwd_chunked(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, chun
         S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if S_final is not None:
         _need(S_final, "S_final", torch.float32, dev)
+    lib = _lib.load()
+    if fp32core:
+        with torch.cuda.device(dev):
+            rc = lib.ckda_sfda_fwd_chunked_fp32core(
+                _p(q), _p(k), _p(v), _p(alpha), _p(theta), _p(beta), _p(S0), _p(cu_seqlens),
+                _p(out), _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
+                _stream_ptr(dev))
+        if rc != 0:
+            raise CKDAError(rc, "ckda_sfda_fwd_chunked_fp32core")
+        return out, S_final
+    need = workspace_bytes(B, T, H, dk, dv, chunk, q.dtype, out_dtype, cu_seqlens is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, dev)
     with torch.cuda.device(dev):
-        rc = _lib.load().ckda_sfda_fwd_chunked(
+        rc = lib.ckda_sfda_fwd_chunked(
             _p(q), _p(k), _p(v), _p(alpha), _p(theta), _p(beta), _p(S0), _p(cu_seqlens),
             _p(out), _p(S_final), B, T, H, dk, dv, chunk, _DT[q.dtype], _DT[out_dtype],
-            _stream_ptr(dev))
+            _p(workspace), 0 if workspace is None else workspace.numel(), _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_sfda_fwd_chunked")
     return out, S_final

@@ -21,9 +21,9 @@ cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void
 // tensor-core kernels (the caller then uses the CUDA-core kernel).
 cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
                           const void* k, const void* v, const float* alpha, const float* beta,
-                          const float* bg, const float* wg, const float* S0, const int32_t* cu,
-                          void* out, float* S_final, int n_seqs, int T, int H, int C, void* ws,
-                          int* status, cudaStream_t stream);
+                          const float* bg, const float* wg, const float* theta, const float* S0,
+                          const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
+                          int C, void* ws, int* status, cudaStream_t stream);
 bool fwd_tc_supported(int dtype, int dk, int dv, int C, int n_seqs, int T, int H, bool varlen);
 size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int T, int H,
                               bool varlen);
@@ -131,7 +131,7 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
     if (out != nullptr && out == theta) return CKDA_ERR_INVALID_ARG;
   }
   const int n_seqs = B;
-  const bool tc = allow_tc && !sfda && n_seqs > 0 &&
+  const bool tc = allow_tc && n_seqs > 0 &&
                   ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, n_seqs, T, H, cu != nullptr);
   // the two-phase calls exist only on the tensor-core path
   if (phases != kBoth && !tc && n_seqs > 0) return CKDA_ERR_UNSUPPORTED;
@@ -143,7 +143,7 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
       return CKDA_ERR_WORKSPACE;
     const void* ws_end = static_cast<const uint8_t*>(workspace) + need;
-    const void* ptrs[] = {q, k, v, alpha, beta, bg, wg, S0, out, S_final, cu};
+    const void* ptrs[] = {q, k, v, alpha, beta, bg, wg, theta, S0, out, S_final, cu};
     for (const void* p : ptrs)
       if (p != nullptr && p >= workspace && p < ws_end) return CKDA_ERR_WORKSPACE;
   }
@@ -152,8 +152,9 @@ int fwd_impl(bool allow_tc, int phases, const void* q, const void* k, const void
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaErrorNotSupported;
   if (tc)
-    e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg, S0,
-                            cu, out, S_final, n_seqs, T, H, chunk, workspace, status, st);
+    e = ckda::launch_fwd_tc(phases, dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg,
+                            sfda ? theta : nullptr, S0, cu, out, S_final, n_seqs, T, H, chunk,
+                            workspace, status, st);
   if (e == cudaErrorNotSupported)
     e = ckda::launch_fwd_simt(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg,
                               sfda ? theta : nullptr, S0, cu, out, S_final, n_seqs, T, H, chunk,
@@ -233,7 +234,17 @@ int ckda_sfda_fwd_chunked(const void* q, const void* k, const void* v, const flo
                           const float* theta, const float* beta, const float* S0,
                           const int32_t* cu_seqlens, void* out, float* S_final, int B, int T,
                           int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
-                          void* stream) {
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(true, kBoth, q, k, v, alpha, beta, nullptr, nullptr, S0, cu_seqlens, out,
+                  S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, workspace,
+                  workspace_bytes, stream, /*sfda=*/true, theta);
+}
+
+int ckda_sfda_fwd_chunked_fp32core(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* theta, const float* beta,
+                                   const float* S0, const int32_t* cu_seqlens, void* out,
+                                   float* S_final, int B, int T, int H, int d_k, int d_v,
+                                   int chunk, int dtype, int out_dtype, void* stream) {
   return fwd_impl(false, kBoth, q, k, v, alpha, beta, nullptr, nullptr, S0, cu_seqlens, out,
                   S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype, nullptr, 0, stream,
                   /*sfda=*/true, theta);

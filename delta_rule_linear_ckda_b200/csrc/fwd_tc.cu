@@ -44,6 +44,16 @@
 // of d_k, so the level GEMMs are split along K and the next unit's inputs
 // stream in by TMA while the rest of the unit runs.
 //
+// SFDA ("Semidirect Fourier Delta Attention (SFDA)" page, "Arquitectura
+// Central"): the gate of channel pair (2p, 2p+1) is the complex scalar
+// lambda_p = alpha_p e^{i theta_p}, i.e. a 2x2 rotation-decay block.  Those
+// blocks commute, so every product above stays a running product, now of
+// complex scalars; the left (row) side of T and A and the factors K * Gamma
+// and Q * Gamma take the conjugate products (Gamma_r^T k_r, Gamma_r^T q_r),
+// the right side and K * rho the plain ones, and the carry applies Gamma_C
+// to the state's row pairs.  A conversion step turns the (alpha, theta)
+// tiles of each half into interleaved (re, im) gates before its gate pass.
+//
 // Operands are fp16 tiles in 128-byte-swizzled shared memory; accumulators
 // live in tensor memory; the carry kernel keeps its state slice in fp32
 // registers (row i = tensor-memory lane i).  Every mbarrier wait is
@@ -68,6 +78,11 @@ constexpr int BV = 64;  // d_v columns of one carry CTA
 constexpr int NT = 256;   // carry kernel threads
 constexpr int NT1 = 512;  // factor kernel threads
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
+
+// Gate families of the factor kernel.
+constexpr int kKda = 0;   // beta_r, Diag(alpha_r)
+constexpr int kGdn2 = 1;  // erase gate b_r, write gate w_r, Diag(alpha_r)
+constexpr int kSfda = 2;  // beta_r, phase-decay blocks alpha_p e^{i theta_p}
 
 // ---- workspace: per unit (one chunk of one head), five arrays -------------
 constexpr size_t kWsWQ = (size_t)2 * C * DK * 2;  // [-W; Q'] fp16 [128][128]
@@ -209,6 +224,15 @@ __device__ __forceinline__ float4 mul4(float4 a, float4 b) {
   return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w);
 }
 
+// Two complex products at once: (a.x + i a.y)(b.x + i b.y) and
+// (a.z + i a.w)(b.z + i b.w).
+__device__ __forceinline__ float4 cmul4(float4 a, float4 b) {
+  return make_float4(fmaf(-a.y, b.y, a.x * b.x), fmaf(a.y, b.x, a.x * b.y),
+                     fmaf(-a.w, b.w, a.z * b.z), fmaf(a.w, b.z, a.z * b.w));
+}
+
+__device__ __forceinline__ float4 conj4(float4 a) { return make_float4(a.x, -a.y, a.z, -a.w); }
+
 __device__ __forceinline__ float4 scale4(float s, float4 a) {
   return make_float4(s * a.x, s * a.y, s * a.z, s * a.w);
 }
@@ -327,13 +351,31 @@ __device__ __forceinline__ int level_row(int lv, int p) {
 // up to the same amount on every scheduler.  One out-of-line copy serves
 // both halves.
 //
-// G2 (Gated DeltaNet-2): the erase side uses e = b * k (b per key channel,
-// read from global memory at `bgp` + position * `bstride`, the channels of
-// this half) in place of beta * k: in the T rows of the level operands, in
-// the direct T pairs and in E * Gamma (stored where K * Gamma goes).
-template <bool G2>
+// kGdn2 (Gated DeltaNet-2): the erase side uses e = b * k (b per key
+// channel, read from global memory at `bgp` + position * `bstride`, the
+// channels of this half) in place of beta * k: in the T rows of the level
+// operands, in the direct T pairs and in E * Gamma (stored where K * Gamma
+// goes).  kSfda: the gate tile holds (re, im) pairs, every gate product is a
+// complex product, and the row-side operands (K * Gamma, Q * Gamma, the left
+// level operands) take the conjugate of their gate product.
+template <int GK>
 __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid,
                                        const float* __restrict__ bgp, int bstride) {
+  constexpr bool G2 = GK == kGdn2;
+  constexpr bool SF = GK == kSfda;
+  // gate product and conjugate (plain products and identity unless SF)
+  auto gm = [](float4 a, float4 b) -> float4 {
+    if constexpr (SF)
+      return cmul4(a, b);
+    else
+      return mul4(a, b);
+  };
+  auto gc = [](float4 a) -> float4 {
+    if constexpr (SF)
+      return conj4(a);
+    else
+      return a;
+  };
   const int w = tid >> 5;
   const int role = (w >> 2) & 1;
   const int kk = (w < 8) ? (w & 3) : 7 - (w & 3);
@@ -342,7 +384,8 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
   const int g = rt >> 4;
   const int cl = 4 * c4;
   const int ig = HC * hh + cl;
-  const float4 one = make_float4(1.f, 1.f, 1.f, 1.f);
+  // the identity gate (complex 1 on both pairs for SF)
+  const float4 one = SF ? make_float4(1.f, 0.f, 1.f, 0.f) : make_float4(1.f, 1.f, 1.f, 1.f);
   const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
   auto bf4 = [](uint2 raw) -> float4 {
     const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
@@ -387,23 +430,23 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
   // warp) of aligned pairs of groups
   const uint32_t gt = sb + OFF_GT + cl * 4;
   if (role == 0) {
-    const float4 t = mul4(mul4(aa[0], aa[1]), mul4(aa[2], aa[3]));
+    const float4 t = gm(gm(aa[0], aa[1]), gm(aa[2], aa[3]));
     sts_f4(gt + g * 256, t);
     float4 o;
     o.x = __shfl_xor_sync(0xffffffffu, t.x, 16);
     o.y = __shfl_xor_sync(0xffffffffu, t.y, 16);
     o.z = __shfl_xor_sync(0xffffffffu, t.z, 16);
     o.w = __shfl_xor_sync(0xffffffffu, t.w, 16);
-    if (!(g & 1)) sts_f4(sb + OFF_T2 + (g >> 1) * 256 + cl * 4, mul4(t, o));
+    if (!(g & 1)) sts_f4(sb + OFF_T2 + (g >> 1) * 256 + cl * 4, gm(t, o));
   }
   GP_MARK(0);
   __syncthreads();
   GP_MARK(1);
   auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * 256); };
   auto run2 = [&](int s2) -> float4 { return lds_f4(sb + OFF_T2 + s2 * 256 + cl * 4); };
-  auto run4 = [&](int s4) -> float4 { return mul4(run2(2 * s4), run2(2 * s4 + 1)); };
+  auto run4 = [&](int s4) -> float4 { return gm(run2(2 * s4), run2(2 * s4 + 1)); };
   auto run8 = [&](int s8) -> float4 {
-    return mul4(mul4(run2(4 * s8), run2(4 * s8 + 1)), mul4(run2(4 * s8 + 2), run2(4 * s8 + 3)));
+    return gm(gm(run2(4 * s8), run2(4 * s8 + 1)), gm(run2(4 * s8 + 2), run2(4 * s8 + 3)));
   };
   const uint32_t LV = sb + OFF_LVX;
 
@@ -430,11 +473,13 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     const int g4 = g & ~3;
     float4 off4 = one;
     if (g - g4 >= 1) off4 = gtot(g4);
-    if (g - g4 >= 2) off4 = mul4(off4, gtot(g4 + 1));
-    if (g - g4 >= 3) off4 = mul4(off4, gtot(g4 + 2));
+    if (g - g4 >= 2) off4 = gm(off4, gtot(g4 + 1));
+    if (g - g4 >= 3) off4 = gm(off4, gtot(g4 + 2));
     const float4 off3 = (g & 1) ? gtot(g - 1) : one;
-    const float4 off5 = (g & 4) ? mul4(run4((g >> 2) & ~1), off4) : off4;
-    float4 pg = (g & 8) ? mul4(run8(0), off5) : off5;  // Gamma offset: every earlier group
+    const float4 off5 = (g & 4) ? gm(run4((g >> 2) & ~1), off4) : off4;
+    float4 pg = (g & 8) ? gm(run8(0), off5) : off5;  // Gamma offset: every earlier group
+    // the row side takes the conjugate offsets (the same values unless SF)
+    const float4 off3c = gc(off3), off4c = gc(off4), off5c = gc(off5);
     // left operands [beta k L; q L] of level lv: rows level_row, 32 + level_row
     const uint32_t kg_b = sb + OFF_KG + rowg;
     const uint32_t qg_b = sb + OFF_QG + rowg;
@@ -448,30 +493,32 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
       const float4 a = aa[u];
       const float4 kf = ka[u];
       const float4 qf = qa[u];
-      pg = mul4(pg, a);
-      lp = (u == 0) ? a : mul4(lp, a);
+      pg = gm(pg, a);
+      lp = (u == 0) ? a : gm(lp, a);
       const uint32_t ro = 128 * u + xo[u];
-      sts_u2(kg_b + ro, h4(mul4(G2 ? eg[u] : kf, pg)));
-      sts_u2(qg_b + ro, h4(mul4(qf, pg)));
+      // data times the row-side gate: gc(gate) * data (conjugate for SF)
+      sts_u2(kg_b + ro, h4(gm(gc(pg), G2 ? eg[u] : kf)));
+      sts_u2(qg_b + ro, h4(gm(gc(pg), qf)));
       if (g & 15) {
-        const float4 qlp = mul4(qf, lp);
-        const float4 blp = G2 ? mul4(eg[u], lp) : scale4(bb[u], mul4(kf, lp));
+        const float4 lpc = gc(lp);
+        const float4 qlp = gm(lpc, qf);
+        const float4 blp = G2 ? mul4(eg[u], lp) : scale4(bb[u], gm(lpc, kf));
         if (g & 1) {  // level 2: right half
           const uint32_t o2 = l2b + 128 * u + xo2[u];
           sts_u2(o2, h4(blp));
           sts_u2(o2 + 32 * 128, h4(qlp));
         }
         if (g & 2) {  // level 3: right half
-          sts_u2(l3b + ro, h4(mul4(blp, off3)));
-          sts_u2(l3b + 32 * 128 + ro, h4(mul4(qlp, off3)));
+          sts_u2(l3b + ro, h4(gm(blp, off3c)));
+          sts_u2(l3b + 32 * 128 + ro, h4(gm(qlp, off3c)));
         }
         if (g & 4) {  // level 4: right half
-          sts_u2(l4b + ro, h4(mul4(blp, off4)));
-          sts_u2(l4b + 32 * 128 + ro, h4(mul4(qlp, off4)));
+          sts_u2(l4b + ro, h4(gm(blp, off4c)));
+          sts_u2(l4b + 32 * 128 + ro, h4(gm(qlp, off4c)));
         }
         if (g & 8) {  // level 5: right half
-          sts_u2(l5b + ro, h4(mul4(blp, off5)));
-          sts_u2(l5b + 32 * 128 + ro, h4(mul4(qlp, off5)));
+          sts_u2(l5b + ro, h4(gm(blp, off5c)));
+          sts_u2(l5b + 32 * 128 + ro, h4(gm(qlp, off5c)));
         }
       }
     }
@@ -481,11 +528,11 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     // Offsets: products of the whole groups after g up to a level's anchor.
     float4 offr4 = one;
     if ((g | 3) - g >= 1) offr4 = gtot(g + 1);
-    if ((g | 3) - g >= 2) offr4 = mul4(offr4, gtot(g + 2));
-    if ((g | 3) - g >= 3) offr4 = mul4(offr4, gtot(g + 3));
+    if ((g | 3) - g >= 2) offr4 = gm(offr4, gtot(g + 2));
+    if ((g | 3) - g >= 3) offr4 = gm(offr4, gtot(g + 3));
     const float4 offr3 = (g & 1) ? one : gtot(g + 1);
-    const float4 offr5 = (g & 4) ? offr4 : mul4(offr4, run4((g >> 2) + 1));
-    const float4 offr = (g & 8) ? offr5 : mul4(offr5, run8(1));  // rho offset: every later group
+    const float4 offr5 = (g & 4) ? offr4 : gm(offr4, run4((g >> 2) + 1));
+    const float4 offr = (g & 8) ? offr5 : gm(offr5, run8(1));  // rho offset: every later group
     // right operands k R of level lv: rows level_row of the level's 32
     const uint32_t kh_b = sb + OFF_KH + rowg;
     const uint32_t r2b = pair_base(2) + PAIR_ROP + lrow(2);
@@ -495,14 +542,14 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
     float4 ls = one;
 #pragma unroll
     for (int u = 3; u >= 0; --u) {
-      const float4 kls = mul4(ka[u], ls);
+      const float4 kls = gm(ka[u], ls);
       const uint32_t ro = 128 * u + xo[u];
-      sts_u2(kh_b + ro, h4(mul4(kls, offr)));
+      sts_u2(kh_b + ro, h4(gm(kls, offr)));
       if (!(g & 1)) sts_u2(r2b + 128 * u + xo2[u], h4(kls));
-      if (!(g & 2)) sts_u2(r3b + ro, h4(mul4(kls, offr3)));
-      if (!(g & 4)) sts_u2(r4b + ro, h4(mul4(kls, offr4)));
-      if (!(g & 8)) sts_u2(r5b + ro, h4(mul4(kls, offr5)));
-      ls = mul4(ls, aa[u]);
+      if (!(g & 2)) sts_u2(r3b + ro, h4(gm(kls, offr3)));
+      if (!(g & 4)) sts_u2(r4b + ro, h4(gm(kls, offr4)));
+      if (!(g & 8)) sts_u2(r5b + ro, h4(gm(kls, offr5)));
+      ls = gm(ls, aa[u]);
     }
     GP_MARK(3);
     // direct pairs inside this aligned block of 4 (levels 0 and 1) and diag(A)
@@ -512,12 +559,12 @@ __device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc,
       const float4 q1 = qa[1], q2 = qa[2], q3 = qa[3];
       // row side of the T pairs: k_r (scaled by beta_r in the gather) or e_r
       const float4 t1 = G2 ? eg[1] : k1, t2 = G2 ? eg[2] : k2, t3 = G2 ? eg[3] : k3;
-      const float4 e10 = mul4(aa[1], k0);
-      const float4 e20 = mul4(aa[2], e10);
-      const float4 e21 = mul4(aa[2], k1);
-      const float4 e30 = mul4(aa[3], e20);
-      const float4 e31 = mul4(aa[3], e21);
-      const float4 e32 = mul4(aa[3], k2);
+      const float4 e10 = gm(aa[1], k0);
+      const float4 e20 = gm(aa[2], e10);
+      const float4 e21 = gm(aa[2], k1);
+      const float4 e30 = gm(aa[3], e20);
+      const float4 e31 = gm(aa[3], e21);
+      const float4 e32 = gm(aa[3], k2);
       acc[0] = dot4(t1, e10);  acc[1] = dot4(q1, e10);
       acc[2] = dot4(t2, e20);  acc[3] = dot4(q2, e20);
       acc[4] = dot4(t2, e21);  acc[5] = dot4(q2, e21);
@@ -662,20 +709,46 @@ __device__ Unit find_unit(int ui, int stride, int n_units, const int32_t* cu, in
 
 // ---- kernel 1: per-unit WY factors ----------------------------------------------
 
-// G2: the Gated DeltaNet-2 form -- erase gate bg (shaped like k) and write
+// SFDA: turn the (alpha, theta) tiles of one 64-channel half (alpha at
+// IN_A, theta at IN_A + 8192, fp32 [64 pos][32 pairs] each) into the gate
+// tile the gate pass reads, fp32 [64 pos][64] with (re, im) =
+// alpha (cos theta, sin theta) per pair, in place.  Every thread converts 4
+// pairs of one position; the values are read before the barrier and written
+// after it.
+__device__ __forceinline__ void phase_to_gates(uint32_t in, int tid) {
+  const int p = tid >> 3, j = tid & 7;
+  const float4 a = lds_f4(in + IN_A + p * 128 + 16 * j);
+  const float4 th = lds_f4(in + IN_A + 8192 + p * 128 + 16 * j);
+  float s0, c0, s1, c1, s2, c2, s3, c3;
+  sincosf(th.x, &s0, &c0);
+  sincosf(th.y, &s1, &c1);
+  sincosf(th.z, &s2, &c2);
+  sincosf(th.w, &s3, &c3);
+  __syncthreads();
+  sts_f4(in + IN_A + p * 256 + 32 * j, make_float4(a.x * c0, a.x * s0, a.y * c1, a.y * s1));
+  sts_f4(in + IN_A + p * 256 + 32 * j + 16, make_float4(a.z * c2, a.z * s2, a.w * c3, a.w * s3));
+  __syncthreads();
+}
+
+// kGdn2: the Gated DeltaNet-2 form -- erase gate bg (shaped like k) and write
 // gate wg (shaped like v) in place of beta; the workspace then holds
 // [-W; Q'] with W = Inv (E * Gamma), [Inv; A Inv] and Z = wg * V, and the
-// carry kernel is unchanged.
-template <int DV, bool G2>
+// carry kernel is unchanged.  kSfda: the phase-decay gates, alpha and theta
+// fp32 [rows, H * DK / 2] (tm_a, tm_th); gamma is stored as (re, im) pairs
+// and the carry kernel applies it to row pairs.
+template <int DV, int GK>
 __global__ void __launch_bounds__(NT1, 1)
 factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+              const __grid_constant__ CUtensorMap tm_th,
               const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
               const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
               const float* __restrict__ beta, const float* __restrict__ bg,
               const float* __restrict__ wg,
               const int32_t* __restrict__ cu, int n_seqs, int T, int H, int nch, int64_t n_units,
               float* __restrict__ ws_g, int* status) {
+  constexpr bool G2 = GK == kGdn2;
+  constexpr bool SF = GK == kSfda;
   // Offsetting the __shared__ array itself (not a cast integer) keeps every
   // access below in the shared state space.
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -706,6 +779,7 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_a);
+    if (SF) prefetch_tmap(&tm_th);
     prefetch_tmap(&tm_wq);
     prefetch_tmap(&tm_kh);
     prefetch_tmap(&tm_ip);
@@ -745,7 +819,12 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     mbar_expect_tx(bar, kInBytes);
     tma_load_2d(base + IN_Q, &tm_q, u.h * DK + HC * hh, (int)u.t0, bar);
     tma_load_2d(base + IN_K, &tm_k, u.h * DK + HC * hh, (int)u.t0, bar);
-    tma_load_2d(base + IN_A, &tm_a, u.h * DK + HC * hh, (int)u.t0, bar);
+    if constexpr (SF) {
+      tma_load_2d(base + IN_A, &tm_a, u.h * (DK / 2) + (HC / 2) * hh, (int)u.t0, bar);
+      tma_load_2d(base + IN_A + 8192, &tm_th, u.h * (DK / 2) + (HC / 2) * hh, (int)u.t0, bar);
+    } else {
+      tma_load_2d(base + IN_A, &tm_a, u.h * DK + HC * hh, (int)u.t0, bar);
+    }
   };
   auto issue_v = [&](const Unit& u) {
     mbar_expect_tx(bar_v, 8192 * (DV / 64));
@@ -813,7 +892,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #endif
     // (G2: the erase gate of this half starts at row t0, channel h * DK + 64 hh)
     const float* bg_row = G2 ? bg + ((size_t)cur.t0 * H + cur.h) * DK : nullptr;
-    gate_pass<G2>(sb, sb + OFF_IN0, 0, Lc, tid, bg_row, H * DK);
+    if constexpr (SF) phase_to_gates(sb + OFF_IN0, tid);
+    gate_pass<GK>(sb, sb + OFF_IN0, 0, Lc, tid, bg_row, H * DK);
 #ifdef CKDA_TC_DEBUG
     const long long t_gp1 = clock64();
 #endif
@@ -841,7 +921,8 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (tid == 0) bulk_wait_read_all();
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    gate_pass<G2>(sb, sb + OFF_IN1, 1, Lc, tid, G2 ? bg_row + HC : nullptr, H * DK);
+    if constexpr (SF) phase_to_gates(sb + OFF_IN1, tid);
+    gate_pass<GK>(sb, sb + OFF_IN1, 1, Lc, tid, G2 ? bg_row + HC : nullptr, H * DK);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
@@ -1159,7 +1240,9 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
 // ---- kernel 2: the chunk-to-chunk carry ---------------------------------------------
 
-template <typename Tout>
+// SF: gamma holds (re, im) pairs and multiplies the state's row pairs
+// (2p, 2p+1) as a complex scalar; the partner row is the neighbouring lane.
+template <typename Tout, bool SF>
 __global__ void __launch_bounds__(NT, 1)
 carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
              const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
@@ -1259,7 +1342,14 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   }
   pend0 = nchunks > 0;
   pend1 = nchunks > 1;
-  float gm = (nchunks > 0) ? ws_g[unit_of(0) * DK + srow] : 1.f;
+  // gamma of this row (SF: of its row pair, real and imaginary part)
+  const int grow = SF ? (srow & ~1) : srow;
+  auto load_gamma = [&](int c) -> float2 {
+    if (c >= nchunks) return make_float2(1.f, 0.f);
+    const float* gp = ws_g + unit_of(c) * DK + grow;
+    return SF ? *reinterpret_cast<const float2*>(gp) : make_float2(*gp, 0.f);
+  };
+  float2 gm = load_gamma(0);
   __syncthreads();
 
   for (int c = 0; c < nchunks; ++c) {
@@ -1271,7 +1361,7 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
     ok = __syncthreads_and(ok);
     if (!ok) break;
-    const float gm_next = (c + 1 < nchunks) ? ws_g[unit_of(c + 1) * DK + srow] : 1.f;
+    const float2 gm_next = load_gamma(c + 1);
     TC_MARK(9);
 
     // ---- carry 1: [U; O] = [Inv diag(beta); P] V + [-W; Q'] S -------------------
@@ -1375,8 +1465,18 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       float d[32];
       tmem_ld32(taddr(tmem, 32 * q4, TM2_D + 32 * half), d);
       tmem_ld_wait();
+      if constexpr (SF) {
+        // even row: gr S_e - gi S_o + d;  odd row: gr S_o + gi S_e + d
+        const float gi = (lane & 1) ? gm.y : -gm.y;
 #pragma unroll
-      for (int e = 0; e < 32; ++e) S[e] = fmaf(gm, S[e], d[e]);
+        for (int e = 0; e < 32; ++e) {
+          const float po = __shfl_xor_sync(0xffffffffu, S[e], 1);
+          S[e] = fmaf(gm.x, S[e], fmaf(gi, po, d[e]));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) S[e] = fmaf(gm.x, S[e], d[e]);
+      }
       TC_DBG(for (int e = 0; e < 32; ++e) {
         g_tc_dbg[49152 + srow * 64 + 32 * half + e] = d[e];
         g_tc_dbg[57344 + srow * 64 + 32 * half + e] = S[e];
@@ -1490,11 +1590,12 @@ cudaError_t set_smem(K kern, size_t bytes) {
 // `stream`.
 constexpr int kFactors = 1, kCarry = 2;
 
-template <int DV, typename Tout, bool G2>
+template <int DV, typename Tout, int GK>
 cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, const float* alpha,
-                     const float* beta, const float* bg, const float* wg, const float* S0,
-                     const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
-                     void* ws, int* status, cudaStream_t stream) {
+                     const float* beta, const float* bg, const float* wg, const float* theta,
+                     const float* S0, const int32_t* cu, void* out, float* S_final, int n_seqs,
+                     int T, int H, void* ws, int* status, cudaStream_t stream) {
+  constexpr bool SF = GK == kSfda;
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
   const int nch = (int)(((int64_t)T + C - 1) / C);
   const int64_t nu = n_units(cu != nullptr, n_seqs, T, H);
@@ -1518,7 +1619,10 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
     return cudaErrorInvalidValue;
 
   if (phases & kFactors) {
-    CUtensorMap mq, mk, mv, ma, mwq64;
+    CUtensorMap mq, mk, mv, ma, mth, mwq64;
+    // SF: alpha and theta hold one value per channel pair (DK / 2 per head)
+    const uint64_t a_cols = SF ? (uint64_t)H * (DK / 2) : (uint64_t)H * DK;
+    const uint32_t a_box = SF ? HC / 2 : HC;
     const bool ok =
         make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HC, C,
                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
@@ -1526,12 +1630,14 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
         make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows, 64, C,
                  CU_TENSOR_MAP_SWIZZLE_128B) &&
-        make_map(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)H * DK, rows, HC, C,
+        make_map(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a_cols, rows, a_box, C,
                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
+        make_map(&mth, SF ? theta : alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a_cols, rows,
+                 a_box, C, CU_TENSOR_MAP_SWIZZLE_NONE) &&
         make_map(&mwq64, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
                  C, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    auto k1 = factor_kernel<DV, G2>;
+    auto k1 = factor_kernel<DV, GK>;
     static bool attr1 = false;
     if (!attr1) {
       cudaError_t e = set_smem(k1, kSmemBytes);
@@ -1539,8 +1645,9 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       attr1 = true;
     }
     const int64_t g1 = nu < (int64_t)sm_count() ? nu : (int64_t)sm_count();
-    k1<<<(unsigned)g1, NT1, kSmemBytes, stream>>>(mq, mk, mv, ma, mwq64, mkh, mip, mv16, beta, bg,
-                                                  wg, cu, n_seqs, T, H, nch, nu, ws_g, status);
+    k1<<<(unsigned)g1, NT1, kSmemBytes, stream>>>(mq, mk, mv, ma, mth, mwq64, mkh, mip, mv16,
+                                                  beta, bg, wg, cu, n_seqs, T, H, nch, nu, ws_g,
+                                                  status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1559,7 +1666,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
             : make_map3(&mout, out, tout, sizeof(Tout), (uint64_t)H * DV, (uint64_t)T,
                         (uint64_t)n_seqs, ob_cols, C, CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return cudaErrorInvalidValue;
-    auto k2 = carry_kernel<Tout>;
+    auto k2 = carry_kernel<Tout, SF>;
     static bool attr2 = false;
     if (!attr2) {
       cudaError_t e = set_smem(k2, kSmem2Bytes);
@@ -1598,25 +1705,27 @@ size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int 
 // Everything the tensor-core kernels do not cover returns
 // cudaErrorNotSupported so the caller can use the CUDA-core kernel.
 // `phases`: 1 = factors only, 2 = carry only, 3 = the whole forward.
-// `bg`, `wg` non-NULL select the Gated DeltaNet-2 form (beta unused).
+// `bg`, `wg` non-NULL select the Gated DeltaNet-2 form (beta unused);
+// `theta` non-NULL the SFDA form (alpha then holds d_k / 2 decays).
 cudaError_t launch_fwd_tc(int phases, int dtype, int out_dtype, int dk, int dv, const void* q,
                           const void* k, const void* v, const float* alpha, const float* beta,
-                          const float* bg, const float* wg, const float* S0, const int32_t* cu,
-                          void* out, float* S_final, int n_seqs, int T, int H, int C, void* ws,
-                          int* status, cudaStream_t stream) {
+                          const float* bg, const float* wg, const float* theta, const float* S0,
+                          const int32_t* cu, void* out, float* S_final, int n_seqs, int T, int H,
+                          int C, void* ws, int* status, cudaStream_t stream) {
   if (!fwd_tc_supported(dtype, dk, dv, C, n_seqs, T, H, cu != nullptr))
     return cudaErrorNotSupported;
   const bool bf = out_dtype == CKDA_BF16;
-  const bool g2 = bg != nullptr;
-#define CKDA_TC_CALL(DVV, TO, G)                                                            \
-  tc::launch_t<DVV, TO, G>(phases, q, k, v, alpha, beta, bg, wg, S0, cu, out, S_final, n_seqs, T, \
-                           H, ws, status, stream)
-  if (dv == 128) {
-    if (g2) return bf ? CKDA_TC_CALL(128, __nv_bfloat16, true) : CKDA_TC_CALL(128, float, true);
-    return bf ? CKDA_TC_CALL(128, __nv_bfloat16, false) : CKDA_TC_CALL(128, float, false);
-  }
-  if (g2) return bf ? CKDA_TC_CALL(64, __nv_bfloat16, true) : CKDA_TC_CALL(64, float, true);
-  return bf ? CKDA_TC_CALL(64, __nv_bfloat16, false) : CKDA_TC_CALL(64, float, false);
+  const int gk = theta != nullptr ? tc::kSfda : (bg != nullptr ? tc::kGdn2 : tc::kKda);
+#define CKDA_TC_CALL(DVV, TO, G)                                                               \
+  tc::launch_t<DVV, TO, G>(phases, q, k, v, alpha, beta, bg, wg, theta, S0, cu, out, S_final,   \
+                           n_seqs, T, H, ws, status, stream)
+#define CKDA_TC_GK(DVV, TO)                                                                    \
+  (gk == tc::kSfda ? CKDA_TC_CALL(DVV, TO, tc::kSfda)                                           \
+                   : (gk == tc::kGdn2 ? CKDA_TC_CALL(DVV, TO, tc::kGdn2)                        \
+                                      : CKDA_TC_CALL(DVV, TO, tc::kKda)))
+  if (dv == 128) return bf ? CKDA_TC_GK(128, __nv_bfloat16) : CKDA_TC_GK(128, float);
+  return bf ? CKDA_TC_GK(64, __nv_bfloat16) : CKDA_TC_GK(64, float);
+#undef CKDA_TC_GK
 #undef CKDA_TC_CALL
 }
 

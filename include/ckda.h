@@ -253,18 +253,35 @@ CKDA_API int ckda_gdn2_fwd_chunked(const void* q, const void* k, const void* v,
  *   alpha  fp32 [B, T, H, d_k / 2]  (packed: [T, H, d_k / 2]) decays
  *   theta  fp32 [B, T, H, d_k / 2]  (packed: [T, H, d_k / 2]) phases, radians
  * Both are applied as given (|alpha| <= 1 keeps the transitions
- * non-expansive).  Every other argument, layout, ownership and error rule is
- * that of ckda_fwd_chunked, except that no workspace is taken: this form
- * runs on the fp32 CUDA-core kernel for every shape (any d_k, d_v in
- * {16, 32, 64, 128}, chunk 16, 32 or 64; fp32 or bf16 inputs), with cos and
- * sin of each phase evaluated once per token in fp32.  theta must be
- * non-NULL when there are tokens, 16-byte aligned and not aliased by out.
+ * non-expansive); cos and sin of each phase are evaluated once per token in
+ * fp32.  Every other argument, layout, ownership and error rule is that of
+ * ckda_fwd_chunked, workspace included: the kernels are those of
+ * ckda_fwd_chunked for the same sizes (ckda_fwd_chunked_path,
+ * ckda_fwd_chunked_workspace_bytes) -- the tcgen05 pair for bf16 inputs
+ * with d_k = 128, d_v in {64, 128}, chunk 64, the fp32 CUDA-core kernel
+ * otherwise.  theta must be non-NULL when there are tokens, 16-byte aligned
+ * and not aliased by out.  The two-phase calls (ckda_fwd_factors /
+ * ckda_fwd_carry) carry the real-gate form only.
  */
 CKDA_API int ckda_sfda_fwd_chunked(const void* q, const void* k, const void* v,
                                    const float* alpha, const float* theta, const float* beta,
                                    const float* S0, const int32_t* cu_seqlens, void* out,
                                    float* S_final, int B, int T, int H, int d_k, int d_v,
-                                   int chunk, int dtype, int out_dtype, void* stream);
+                                   int chunk, int dtype, int out_dtype, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * ckda_sfda_fwd_chunked_fp32core -- the same operation as
+ * ckda_sfda_fwd_chunked, forced onto the fp32 CUDA-core kernel (takes no
+ * workspace), as ckda_fwd_chunked_fp32core is for ckda_fwd_chunked.
+ */
+CKDA_API int ckda_sfda_fwd_chunked_fp32core(const void* q, const void* k, const void* v,
+                                            const float* alpha, const float* theta,
+                                            const float* beta, const float* S0,
+                                            const int32_t* cu_seqlens, void* out,
+                                            float* S_final, int B, int T, int H, int d_k,
+                                            int d_v, int chunk, int dtype, int out_dtype,
+                                            void* stream);
 
 /*
  * ckda_fwd_chunked_workspace_bytes -- scratch bytes ckda_fwd_chunked needs

@@ -275,7 +275,7 @@ def test_sfda_entry_validates_its_gates(lib):
         return lib.ckda_sfda_fwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["theta"],
                                          a["beta"], a["S0"], a["cu"], a["out"], a["S_final"],
                                          a["B"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"],
-                                         a["dtype"], a["out_dtype"], None)
+                                         a["dtype"], a["out_dtype"], None, 0, None)
 
     assert sf(theta=None) == -1
     assert sf(alpha=None) == -1
@@ -285,3 +285,9 @@ def test_sfda_entry_validates_its_gates(lib):
     assert sf(dk=48) == -2
     assert sf(chunk=128) == -2
     assert sf(B=0) == 0
+    # the tensor-core shapes need the same workspace as ckda_fwd_chunked
+    assert sf(dtype=1, dk=128, dv=128, chunk=64, T=128) == -7
+    r = lib.ckda_sfda_fwd_chunked_fp32core(P, P + 0x1000, P + 0x2000, P + 0x3000, None,
+                                           P + 0x6000, None, None, P + 0x5000, None, 1, 8, 1, 16,
+                                           16, 16, 0, 0, None)
+    assert r == -1  # theta missing

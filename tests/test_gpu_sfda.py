@@ -2,14 +2,15 @@
 
 ``ckda_sfda_fwd_chunked`` runs the chunk form of the SFDA recurrence
 ("Semidirect Fourier Delta Attention (SFDA)" summary, "Arquitectura Central"
-and "El Teorema de Chunk-WY Constructivo") on the fp32 CUDA-core kernel, the
-gate products being products of the complex phase-decay scalars.  The oracle
-it is compared with is pinned by ``pinlib_sfda`` (S-1..S-8).  Shapes span
-several chunks with ragged tails, every supported head size (16 and 32 put
-one channel per lane, so the two halves of a pair sit in neighbouring lanes)
-and chunk size, packed batches with empty sequences, the full-size workload
-on sampled units, zero phases (bit-identical to the CKDA kernel) and the
-constructed mod-5 counter.
+and "El Teorema de Chunk-WY Constructivo"), the gate products being products
+of the complex phase-decay scalars: on the tcgen05 pair for bf16 inputs with
+d_k = 128, d_v in {64, 128}, chunk 64, on the fp32 CUDA-core kernel
+otherwise.  The oracle it is compared with is pinned by ``pinlib_sfda``
+(S-1..S-8).  Shapes span several chunks with ragged tails, every supported
+head size (16 and 32 put one channel per lane, so the two halves of a pair
+sit in neighbouring lanes) and chunk size, packed batches with empty
+sequences, the full-size workload on sampled units, zero phases
+(bit-identical to the CKDA kernels) and the constructed mod-5 counter.
 """
 import math
 
@@ -32,10 +33,11 @@ def ck():
     return ck
 
 
-def _run(ck, c, cu=None, out_dtype=torch.float32, S0="case"):
+def _run(ck, c, cu=None, out_dtype=torch.float32, S0="case", fp32core=False):
     S0 = c.S0 if isinstance(S0, str) else S0
     out, S = ck.sfda_fwd_chunked(c.q, c.k, c.v, c.alpha, c.extra["theta"], c.beta, S0=S0,
-                                 cu_seqlens=cu, chunk=c.chunk, out_dtype=out_dtype)
+                                 cu_seqlens=cu, chunk=c.chunk, out_dtype=out_dtype,
+                                 fp32core=fp32core)
     assert ck.device_status() == 0
     return out, S
 
@@ -109,12 +111,14 @@ def test_phase_pi_is_a_negative_gate(ck):
     assert rel_max_err(o1, ro) <= TOL_F32 and rel_max_err(S1, rS) <= TOL_F32
 
 
-def test_constructed_mod5_counter(ck):
+@pytest.mark.parametrize("dt,d,tol", [(torch.float32, 16, 1e-4), (torch.bfloat16, 128, 2e-2)])
+def test_constructed_mod5_counter(ck, dt, d, tol):
     """Phase-only counter in the first channel pair ("Resultados", constructed
     mod-5 counter): alpha = 1, beta = 0, theta = 2 pi x_t / 5 for input bits
     x_t; the read-out along e_0 is cos(2 pi count_t / 5) and the final state
-    decodes count mod 5 exactly for lengths 27 to 213 (fp32 kernel)."""
-    dk = dv = 16
+    decodes count mod 5 exactly for lengths 27 to 213 (fp32 kernel at d = 16,
+    tensor-core kernels at d = 128)."""
+    dk = dv = d
     gen = torch.Generator().manual_seed(34)
     for L in (27, 100, 213):
         x = torch.randint(0, 2, (L,), generator=gen)
@@ -125,13 +129,13 @@ def test_constructed_mod5_counter(ck):
         k[..., 0] = 1.0
         S0 = torch.zeros(1, 1, dk, dv)
         S0[0, 0, 0, 0] = 1.0
-        args = [t.to(DEV).contiguous() for t in (k, k, torch.zeros(1, L, 1, dv), alpha, theta,
-                                                  torch.zeros(1, L, 1), S0)]
+        args = [t.to(DEV).contiguous() for t in (k.to(dt), k.to(dt), torch.zeros(1, L, 1, dv).to(dt),
+                                                  alpha, theta, torch.zeros(1, L, 1), S0)]
         out, S = ck.sfda_fwd_chunked(*args[:6], S0=args[6], chunk=64, out_dtype=torch.float32)
         assert ck.device_status() == 0
         count = torch.cumsum(x, 0).double()
         o = out[0, :, 0, 0].double().cpu()
-        assert float((o - torch.cos(2 * math.pi / 5 * count)).abs().max()) < 1e-4
+        assert float((o - torch.cos(2 * math.pi / 5 * count)).abs().max()) < tol
         ang = math.atan2(float(S[0, 0, 1, 0]), float(S[0, 0, 0, 0]))
         assert round(ang / (2 * math.pi / 5)) % 5 == int(count[-1]) % 5
 
@@ -149,3 +153,59 @@ def test_full_size_workload_on_sampled_units(ck):
                                      sel(c.extra["theta"]), sel(c.beta))
         assert rel_max_err(out[b:b + 1, :, h:h + 1], ro) <= TOL_BF16, (b, h)
         assert rel_max_err(S[b:b + 1, h:h + 1], rS) <= TOL_BF16, (b, h)
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+@pytest.mark.parametrize("T", [64, 200])
+def test_tensor_core_path_matches_oracle(ck, dv, T):
+    assert ck.fwd_path(2, T, 3, 128, dv, 64, torch.bfloat16, torch.float32) == "tcgen05"
+    c = inputs.sfda_prefill(2, T, 3, 128, dv, dtype=torch.bfloat16, s0_std=0.02, chunk=64,
+                            seed=30 + T + dv, device=DEV)
+    out, S = _run(ck, c)
+    ro, rS = _oracle(c)
+    assert rel_max_err(out, ro) <= TOL_BF16 and rel_max_err(S, rS) <= TOL_BF16
+    o16, _ = _run(ck, c, out_dtype=torch.bfloat16)
+    assert torch.equal(o16, out.to(torch.bfloat16))
+
+
+def test_tensor_core_packed_batch(ck):
+    lens = [65, 0, 130, 1, 191, 64, 0]
+    total = int(sum(lens))
+    c = inputs.sfda_prefill(1, total, 3, 128, 128, dtype=torch.bfloat16, chunk=64, seed=41,
+                            device=DEV)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=DEV)
+    assert ck.fwd_path(len(lens), total, 3, 128, 128, varlen=True) == "tcgen05"
+    g = torch.Generator(device=DEV).manual_seed(42)
+    S0 = 0.02 * torch.randn(len(lens), 3, 128, 128, generator=g, device=DEV)
+    out, S = _run(ck, c, cu=cu, S0=S0)
+    ro, rS = _oracle(c, S0=S0, cu=cu)
+    assert rel_max_err(out, ro) <= TOL_BF16 and rel_max_err(S, rS) <= TOL_BF16
+    assert torch.equal(S[1], S0[1]) and torch.equal(S[6], S0[6])  # empty sequences
+
+
+@pytest.mark.parametrize("dv", [64, 128])
+def test_tensor_core_zero_phase_is_the_ckda_kernels_bit_for_bit(ck, dv):
+    """theta = 0 on the tcgen05 pair: the complex gate products have zero
+    imaginary parts and reduce to the CKDA kernels' products, operand for
+    operand, with each decay on both rows of its pair."""
+    c = inputs.sfda_prefill(2, 200, 3, 128, dv, dtype=torch.bfloat16, s0_std=0.02, chunk=64,
+                            seed=50 + dv, device=DEV)
+    zero = torch.zeros_like(c.extra["theta"])
+    o1, S1 = ck.sfda_fwd_chunked(c.q, c.k, c.v, c.alpha, zero, c.beta, S0=c.S0,
+                                 out_dtype=torch.float32)
+    a2 = c.alpha.repeat_interleave(2, dim=-1).contiguous()
+    o2, S2 = ck.fwd_chunked(c.q, c.k, c.v, a2, c.beta, S0=c.S0, out_dtype=torch.float32)
+    assert ck.device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_tensor_core_agrees_with_the_fp32_kernel(ck):
+    c = inputs.sfda_prefill(2, 300, 3, 128, 128, dtype=torch.bfloat16, s0_std=0.02, chunk=64,
+                            seed=61, device=DEV)
+    o1, S1 = _run(ck, c)
+    o2, S2 = _run(ck, c, fp32core=True)
+    ro, rS = _oracle(c)
+    # the fp32 kernel is the closer of the two to the oracle; both pass the bar
+    assert rel_max_err(o2, ro) <= TOL_F32 * 10 and rel_max_err(S2, rS) <= TOL_F32 * 10
+    assert rel_max_err(o1, ro) <= TOL_BF16 and rel_max_err(S1, rS) <= TOL_BF16
+    assert rel_max_err(o1, o2.double().cpu().numpy()) <= TOL_BF16
