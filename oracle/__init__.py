@@ -27,6 +27,12 @@ Contents
     ``(2p, 2p+1)``,
     ``S_t = (I - beta_t k_t k_t^T) Lambda_t S_{t-1} + beta_t k_t v_t^T``;
     pinned by ``tests/pinlib_sfda.py`` (S-1..S-8).
+``backward``
+    The gradient of a scalar loss through the CKDA forward: given dL/do_t
+    and dL/dS_final, dL/d(q, k, v, alpha, beta, S0), the adjoint of the
+    per-token body taken step by step in reverse (states recomputed from
+    checkpoints every 64 tokens); pinned by ``tests/pinlib_bwd.py`` (B-1..B-6:
+    finite differences of the pinned forward, closed forms, symmetries).
 ``chunked`` (submodule)
     A plain numpy fp64 restatement of the chunkwise WY form, used only to pin
     the chunked algorithm against the sequential loop on tiny inputs.
@@ -85,6 +91,11 @@ def _load():
                 dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
             ]
             lib.ckda_oracle_sfda_forward.restype = ctypes.c_int
+            lib.ckda_oracle_backward.argtypes = [
+                i64, i64, i64, i64, ctypes.POINTER(ctypes.c_int64),
+                dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
+            ]
+            lib.ckda_oracle_backward.restype = ctypes.c_int
             lib.ckda_oracle_decode_step.argtypes = [
                 i64, i64, i64, i64, dp, dp, dp, dp, dp, dp, dp, ctypes.c_int,
             ]
@@ -241,6 +252,55 @@ def forward_sfda(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, n_thread
     if rc != 0:
         raise ValueError("ckda_oracle_sfda_forward rejected its arguments")
     return out.reshape(out_shape), S_final
+
+
+def backward(q, k, v, alpha, beta, dO, S0=None, dS_final=None, cu_seqlens=None,
+             n_threads=None):
+    """fp64 gradients of the CKDA forward (see ``ckda_oracle_backward``).
+
+    Inputs as in ``forward``; ``dO`` is shaped like ``v`` (the gradient of the
+    loss with respect to the output), ``dS_final`` like the final state (or
+    None = 0).  Returns a dict of fp64 numpy arrays ``dq, dk, dv, dalpha,
+    dbeta, dS0`` shaped like ``q, k, v, alpha, beta`` and the state."""
+    qd, kd, vd, ad, bd, dod = (_f64(t) for t in (q, k, v, alpha, beta, dO))
+    shapes = {"dq": qd.shape, "dk": kd.shape, "dv": vd.shape, "dalpha": ad.shape,
+              "dbeta": bd.shape}
+    if cu_seqlens is None:
+        if qd.ndim != 4:
+            raise ValueError("fixed-length batch expects [B, T, H, d] tensors")
+        B, T, H, dk = qd.shape
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens,
+            dtype=np.int64))
+        if qd.ndim == 4:
+            if qd.shape[0] != 1:
+                raise ValueError("packed batch expects a leading dimension of 1")
+            qd, kd, vd, ad, bd, dod = qd[0], kd[0], vd[0], ad[0], bd[0], dod[0]
+        H, dk = qd.shape[1], qd.shape[2]
+    N = len(cu) - 1
+    dv = vd.shape[-1]
+    T_total = int(cu[-1])
+    qd, kd, ad = (x.reshape(T_total, H, dk) for x in (qd, kd, ad))
+    vd, dod = (x.reshape(T_total, H, dv) for x in (vd, dod))
+    bd = bd.reshape(T_total, H)
+    S0d = None if S0 is None else _f64(S0).reshape(N, H, dk, dv)
+    dSf = None if dS_final is None else _f64(dS_final).reshape(N, H, dk, dv)
+    g = {"dq": np.zeros((T_total, H, dk)), "dk": np.zeros((T_total, H, dk)),
+         "dv": np.zeros((T_total, H, dv)), "dalpha": np.zeros((T_total, H, dk)),
+         "dbeta": np.zeros((T_total, H)), "dS0": np.zeros((N, H, dk, dv))}
+    rc = _load().ckda_oracle_backward(
+        N, H, dk, dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+        _ptr(qd), _ptr(kd), _ptr(vd), _ptr(ad), _ptr(bd), _ptr(S0d), _ptr(dod), _ptr(dSf),
+        _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]), _ptr(g["dalpha"]), _ptr(g["dbeta"]),
+        _ptr(g["dS0"]), int(n_threads or default_threads()),
+    )
+    if rc != 0:
+        raise ValueError("ckda_oracle_backward rejected its arguments")
+    for name, shp in shapes.items():
+        g[name] = g[name].reshape(shp)
+    return g
 
 
 def decode_step(q, k, v, alpha, beta, S, n_threads=None):
