@@ -46,6 +46,8 @@ DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4
 GDN2_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + D * 4 + D * 4 + D * 4
 # SFDA forward: q, k, v bf16 + alpha and theta (d_k / 2 each) fp32 + beta + out fp32
 SFDA_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + 2 * (D // 2) * 4 + 4 + D * 4
+# backward: q, k, v bf16 + alpha, beta, dO fp32 in; dq, dk, dalpha, dv fp32 + dbeta out
+BWD_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4 + 3 * D * 4 + D * 4 + 4
 
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
@@ -71,6 +73,7 @@ def _args():
     ap.add_argument("--e2e-steps", type=int, default=10, help="0 skips the end-to-end leg")
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS,
                     help="decode steps timed (inputs for all of them are pre-generated)")
+    ap.add_argument("--no-bwd", action="store_true", help="skip the backward sub-measure")
     ap.add_argument("--no-sfda", action="store_true",
                     help="skip the SFDA (phase-decay gates) sub-measure")
     ap.add_argument("--no-gdn2", action="store_true",
@@ -314,6 +317,9 @@ def run_ours(args, ws, rank, local):
         if not off:
             variants[kind] = _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier,
                                           max_ranks, ws, hbm_peak)
+    if not args.no_bwd:
+        variants["bwd"] = _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws,
+                                   hbm_peak)
     wsbuf = torch.empty(max(1, ck.workspace_bytes(B, T, H, D, D, CHUNK)), dtype=torch.uint8,
                         device=dev)
     two_phase = path == "tcgen05"
@@ -493,6 +499,49 @@ def _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_frac_of_measured": gbs / hbm_peak,
             "gpu_launches": steps * (2 if path == "tcgen05" else 1)}
+
+
+def _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=5):
+    """Backward at the bench sizes (bf16 q/k/v, fp32 gates and dO, fp32
+    gradients, no S0 / dS_final); inputs larger than L2, one set."""
+    c = inputs.kda_prefill(seed=5000 + rank, device=dev)
+    g = torch.Generator(device=dev).manual_seed(5100 + rank)
+    dO = torch.randn(c.v.shape, generator=g, device=dev)
+    grads = {"dq": torch.empty(c.q.shape, dtype=torch.float32, device=dev),
+             "dk": torch.empty(c.k.shape, dtype=torch.float32, device=dev),
+             "dv": torch.empty(c.v.shape, dtype=torch.float32, device=dev),
+             "dalpha": torch.empty(c.alpha.shape, dtype=torch.float32, device=dev),
+             "dbeta": torch.empty(c.beta.shape, dtype=torch.float32, device=dev)}
+    wsb = torch.empty(ck.bwd_workspace_bytes(B, T, H, D, D), dtype=torch.uint8, device=dev)
+
+    def step():
+        ck.bwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, dO, grads=grads, want_dS0=False,
+                       workspace=wsb)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    assert ck.device_status(dev) == 0
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_ranks(ev0.elapsed_time(ev1)) / steps
+    nbytes = B * T * H * BWD_BYTES_PER_TOKEN_HEAD
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"kda_prefill backward B={B} H={H} T={T} d={D}: bf16 q/k/v, fp32 "
+                        "alpha/beta/dO, fp32 gradients (fp32 CUDA-core kernel, clusters of "
+                        f"{D // 32} CTAs per (sequence, head))",
+            "ms_per_step": ms, "tokens_per_s": ws * B * T / (ms / 1e3),
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+            "hbm_frac_of_measured": gbs / hbm_peak, "workspace_bytes": wsb.numel(),
+            "gpu_launches": steps}
 
 
 def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak):

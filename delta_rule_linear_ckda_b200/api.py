@@ -324,6 +324,67 @@ def sfda_fwd_chunked(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, chun
     return out, S_final
 
 
+def bwd_workspace_bytes(B, T, H, dk, dv, varlen=False) -> int:
+    """Scratch bytes ``bwd_chunked`` needs for these sizes."""
+    rc = _lib.load().ckda_bwd_chunked_workspace_bytes(B, T, H, dk, dv, 1 if varlen else 0)
+    if rc < 0:
+        raise CKDAError(int(rc), "ckda_bwd_chunked_workspace_bytes")
+    return int(rc)
+
+
+def bwd_chunked(q, k, v, alpha, beta, dO, S0=None, dS_final=None, cu_seqlens=None,
+                grads=None, want_dS0: bool = True, workspace=None):
+    """Backward of ``fwd_chunked`` (``ckda_bwd_chunked``): the gradients of a scalar
+    loss with respect to q, k, v, alpha, beta and S0, given ``dO`` (dL/dout, fp32 or
+    bf16, shaped like v) and ``dS_final`` (dL/dS_final, fp32, or None = 0).
+
+    Returns a dict of fp32 tensors ``dq, dk, dv, dalpha, dbeta`` (shaped like the
+    inputs) and ``dS0`` (``[N, H, dk, dv]``, or None when ``want_dS0`` is false).
+    ``grads`` may supply preallocated output tensors under the same names."""
+    dev = q.device
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, cu_seqlens)
+    if dO.dtype not in _DT:
+        raise TypeError("dO must be float32 or bfloat16")
+    _need(dO, "dO", dO.dtype, dev)
+    if dO.shape != v.shape:
+        raise ValueError("dO must have v's shape")
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if dS_final is not None:
+        _need(dS_final, "dS_final", torch.float32, dev)
+        if tuple(dS_final.shape) != (N, H, dk, dv):
+            raise ValueError(f"dS_final must be [{N}, {H}, {dk}, {dv}]")
+    want = {"dq": q.shape, "dk": k.shape, "dv": v.shape, "dalpha": alpha.shape,
+            "dbeta": beta.shape}
+    if want_dS0:
+        want["dS0"] = (N, H, dk, dv)
+    g = dict(grads or {})
+    for name, shp in want.items():
+        if g.get(name) is None:
+            g[name] = torch.empty(shp, dtype=torch.float32, device=dev)
+        _need(g[name], name, torch.float32, dev)
+        if tuple(g[name].shape) != tuple(shp):
+            raise ValueError(f"{name} must be {tuple(shp)}")
+    if not want_dS0:
+        g["dS0"] = None
+    need = bwd_workspace_bytes(B, T, H, dk, dv, cu_seqlens is not None)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_bwd_chunked(
+            _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(cu_seqlens), _p(dO),
+            _p(dS_final), _p(g["dq"]), _p(g["dk"]), _p(g["dv"]), _p(g["dalpha"]),
+            _p(g["dbeta"]), _p(g["dS0"]), B, T, H, dk, dv, _DT[q.dtype], _DT[dO.dtype],
+            _p(workspace), 0 if workspace is None else workspace.numel(), _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_bwd_chunked")
+    return g
+
+
 def workspace_bytes(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, out_dtype=torch.float32,
                     varlen=False) -> int:
     """Scratch bytes ``fwd_chunked`` needs for these sizes (0 on the fp32 CUDA-core path)."""

@@ -29,6 +29,12 @@ size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int 
                               bool varlen);
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
                                       cudaStream_t stream);
+size_t bwd_workspace_bytes(int dk, int dv, int n_seqs, int T, int H, bool varlen);
+cudaError_t launch_bwd(int dtype, int grad_dtype, int dk_, int dv_, const void* q, const void* k,
+                       const void* v, const float* alpha, const float* beta, const float* S0,
+                       const int32_t* cu, const void* dO, const float* dSf, float* dq, float* dk,
+                       float* dv, float* dalpha, float* dbeta, float* dS0, void* ws, int n_seqs,
+                       int T, int H, int* status, cudaStream_t stream);
 }  // namespace ckda
 
 // First device-side error since the last ckda_device_status() call.
@@ -287,6 +293,64 @@ int64_t ckda_fwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v, 
   int rc = validate_sizes(B, T, H, d_k, d_v, &chunk, dtype, out_dtype, varlen);
   if (rc != CKDA_OK) return rc;
   return (int64_t)ckda::fwd_tc_workspace_bytes(dtype, d_k, d_v, chunk, B, T, H, varlen != 0);
+}
+
+int64_t ckda_bwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v, int varlen) {
+  if (B < 0 || T < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
+  if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (varlen && B == 0 && T != 0) return CKDA_ERR_INVALID_ARG;
+  if (!varlen && (int64_t)B * T * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
+  if (B == 0) return 0;
+  return (int64_t)ckda::bwd_workspace_bytes(d_k, d_v, B, T, H, varlen != 0);
+}
+
+int ckda_bwd_chunked(const void* q, const void* k, const void* v, const float* alpha,
+                     const float* beta, const float* S0, const int32_t* cu_seqlens,
+                     const void* dO, const float* dS_final, float* dq, float* dk, float* dv,
+                     float* dalpha, float* dbeta, float* dS0, int B, int T, int H, int d_k,
+                     int d_v, int dtype, int grad_dtype, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (B < 0 || T < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
+  if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (grad_dtype != CKDA_F32 && grad_dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if (cu_seqlens == nullptr && (int64_t)B * T * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
+  if (cu_seqlens != nullptr && B == 0 && T != 0) return CKDA_ERR_INVALID_ARG;
+  const int64_t tokens = (cu_seqlens != nullptr) ? (int64_t)T : (int64_t)B * T;
+  if (tokens > 0 && (!q || !k || !v || !alpha || !beta || !dO || !dq || !dk || !dv || !dalpha ||
+                     !dbeta))
+    return CKDA_ERR_INVALID_ARG;
+  const void* ins[] = {q, k, v, alpha, beta, S0, dO, dS_final};
+  const void* outs[] = {dq, dk, dv, dalpha, dbeta, dS0};
+  for (const void* p : ins)
+    if (p != nullptr && !aligned16(p)) return CKDA_ERR_MISALIGNED;
+  for (const void* p : outs)
+    if (p != nullptr && !aligned16(p)) return CKDA_ERR_MISALIGNED;
+  if (cu_seqlens != nullptr && (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0)
+    return CKDA_ERR_MISALIGNED;
+  for (const void* o : outs) {
+    if (o == nullptr) continue;
+    for (const void* p : ins)
+      if (p != nullptr && o == p) return CKDA_ERR_INVALID_ARG;
+  }
+  if (B == 0) return CKDA_OK;
+  const size_t need = ckda::bwd_workspace_bytes(d_k, d_v, B, T, H, cu_seqlens != nullptr);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return CKDA_ERR_WORKSPACE;
+  {
+    const void* ws_end = static_cast<const uint8_t*>(workspace) + need;
+    for (const void* p : ins)
+      if (p != nullptr && p >= workspace && p < ws_end) return CKDA_ERR_WORKSPACE;
+    for (const void* p : outs)
+      if (p != nullptr && p >= workspace && p < ws_end) return CKDA_ERR_WORKSPACE;
+  }
+  int* status = status_ptr();
+  if (status == nullptr) return CKDA_ERR_CUDA;
+  cudaError_t e = ckda::launch_bwd(dtype, grad_dtype, d_k, d_v, q, k, v, alpha, beta, S0,
+                                   cu_seqlens, dO, dS_final, dq, dk, dv, dalpha, dbeta, dS0,
+                                   workspace, B, T, H, status, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
 int ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,

@@ -327,6 +327,60 @@ CKDA_API int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int ch
                                    int out_dtype, int varlen);
 
 /*
+ * ckda_bwd_chunked -- backward of ckda_fwd_chunked: the gradient of a
+ * scalar loss L with respect to q, k, v, alpha, beta and S0, given
+ * dO = dL/dout and dS_final = dL/dS_final.  It is the adjoint of the
+ * recurrence token by token, in reverse (the chain rule through
+ *   S' = Diag(alpha_t) S_{t-1},  r = S'^T k_t,  u = beta_t (v_t - r),
+ *   S_t = S' + k_t u^T,  o_t = S_t^T q_t;
+ * "Complex KDA ...", section "Complex KDA (CKDA) Mimarisi ve Parametre
+ * Genislemesi"; "Gated DeltaNet-2", Methodology section 1 with b = w =
+ * beta).  The pages give no backward; this is the exact gradient of the
+ * forward above, computed in fp32 on CUDA cores with the states recomputed
+ * from checkpoints (every 64th token, then every 4th) -- no division, so
+ * zero and negative gates are exact.
+ *
+ *   q, k, v, alpha, beta, S0, cu_seqlens, B, T, H, d_k, d_v, dtype:
+ *            the forward's inputs, layouts and rules (ckda_fwd_chunked).
+ *   dO       shaped like out, element type grad_dtype (CKDA_F32 or
+ *            CKDA_BF16); required when there are tokens.
+ *   dS_final [N, H, d_k, d_v] fp32, may be NULL (zero).
+ *   dq, dk, dalpha [.., H, d_k] fp32;  dv [.., H, d_v] fp32;
+ *   dbeta [.., H] fp32 -- shaped like q, k, alpha, v, beta; every element
+ *            written; required when there are tokens.
+ *   dS0      [N, H, d_k, d_v] fp32, may be NULL (not stored).  A
+ *            zero-length sequence gets dS0 = dS_final.
+ *   workspace, workspace_bytes
+ *            device scratch of at least ckda_bwd_chunked_workspace_bytes()
+ *            bytes, 256-byte aligned, overlapping no tensor argument; its
+ *            contents on entry do not matter.
+ * Gradients are overwritten, not accumulated.  No output may alias an
+ * input; every pointer must be 16-byte aligned.  Errors as for
+ * ckda_fwd_chunked (CKDA_ERR_WORKSPACE for a missing or small workspace).
+ * Each (sequence, head) runs as one thread-block cluster of d_v / 32 CTAs
+ * (d_v = 16: one CTA); within a CTA each warp owns 4 state columns.
+ */
+CKDA_API int ckda_bwd_chunked(const void* q, const void* k, const void* v,
+                              const float* alpha, const float* beta, const float* S0,
+                              const int32_t* cu_seqlens, const void* dO,
+                              const float* dS_final, float* dq, float* dk, float* dv,
+                              float* dalpha, float* dbeta, float* dS0, int B, int T, int H,
+                              int d_k, int d_v, int dtype, int grad_dtype, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
+ * ckda_bwd_chunked_workspace_bytes -- scratch bytes ckda_bwd_chunked needs
+ * (B, T and `varlen` as in ckda_fwd_chunked_path), or the negative status
+ * an actual call with these sizes would return.  Pure host function: one
+ * stored state of 4 max(d_k, 32) d_v bytes per 64-token chunk slot and head
+ * (B ceil(T / 64) slots for a fixed-length batch, floor(T / 64) + N packed)
+ * plus 21 such states per sequence and head (the 16 segment starts of a
+ * chunk and the 5 states of a 4-token segment).
+ */
+CKDA_API int64_t ckda_bwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v,
+                                                  int varlen);
+
+/*
  * ckda_decode_step -- one recurrent token for B independent sequences,
  * in place on the state ("Complex KDA ...", section "Yazilim Gelistirme
  * Acisindan Pratik Cikarimlar": O(1) inference state).

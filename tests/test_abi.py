@@ -291,3 +291,33 @@ def test_sfda_entry_validates_its_gates(lib):
                                            P + 0x6000, None, None, P + 0x5000, None, 1, 8, 1, 16,
                                            16, 16, 0, 0, None)
     assert r == -1  # theta missing
+
+
+def test_bwd_entry_validates_without_a_gpu(lib):
+    def bw(**kw):
+        a = dict(q=P, k=P + 0x1000, v=P + 0x2000, alpha=P + 0x3000, beta=P + 0x4000, S0=None,
+                 cu=None, dO=P + 0x5000, dSf=None, dq=P + 0x6000, dk=P + 0x7000, dv=P + 0x8000,
+                 da=P + 0x9000, db=P + 0xA000, dS0=None, B=1, T=8, H=1, dk_=16, dv_=16, dtype=0,
+                 gdt=0, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.ckda_bwd_chunked(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S0"],
+                                    a["cu"], a["dO"], a["dSf"], a["dq"], a["dk"], a["dv"],
+                                    a["da"], a["db"], a["dS0"], a["B"], a["T"], a["H"], a["dk_"],
+                                    a["dv_"], a["dtype"], a["gdt"], a["ws"], a["ws_bytes"], None)
+
+    assert bw(dO=None) == -1
+    assert bw(dq=None) == -1
+    assert bw(db=None) == -1
+    assert bw(dk_=48) == -2
+    assert bw(gdt=3) == -2
+    assert bw(dv=MIS) == -3
+    assert bw(dq=P) == -1          # an output aliases q
+    assert bw() == -7              # no workspace
+    assert bw(B=0) == 0
+    need = lib.ckda_bwd_chunked_workspace_bytes(1, 8, 1, 16, 16, 0)
+    assert need == (1 + 21) * 32 * 16 * 4       # d_k < 32 stores 32 rows per state
+    assert lib.ckda_bwd_chunked_workspace_bytes(2, 130, 3, 128, 64, 0) == \
+        (2 * 3 * 3 + 2 * 3 * 21) * 128 * 64 * 4
+    assert lib.ckda_bwd_chunked_workspace_bytes(2, 130, 3, 128, 48, 0) == -2
+    # a workspace that overlaps an input
+    assert bw(ws=P, ws_bytes=need) == -7
