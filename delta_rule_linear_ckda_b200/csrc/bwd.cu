@@ -2,9 +2,12 @@
 // a scalar loss with respect to q, k, v, alpha, beta and S0, given dL/do_t
 // and dL/dS_final.
 //
-// Per token the forward is (the CKDA recurrence, "Complex KDA ..." page,
-// section "Complex KDA (CKDA) Mimarisi ve Parametre Genislemesi"; "Gated
-// DeltaNet-2" page, Methodology section 1 with b = w = beta):
+// The "Gated DeltaNet-2" page, Methodology section 3 (gate-aware backward),
+// asks that the per-channel gates enter the gradient directly; here the gate
+// gradient is dalpha = rowsum(dS' . S_prev) per token.  Per token the
+// forward is (the CKDA recurrence, "Complex KDA ..." page, section "Complex
+// KDA (CKDA) Mimarisi ve Parametre Genislemesi"; "Gated DeltaNet-2" page,
+// Methodology section 1 with b = w = beta):
 //   S' = Diag(a) S_prev,  r = S'^T k,  u = b (v - r),  S = S' + k u^T,  o = S^T q
 // and its adjoint, walked in reverse with dS = dL/dS (after the token):
 //   dq = S do;  dS += q do^T;  du = dS^T k;  dk = dS u + S' dr;

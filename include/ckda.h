@@ -335,10 +335,12 @@ CKDA_API int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int ch
  *   S_t = S' + k_t u^T,  o_t = S_t^T q_t;
  * "Complex KDA ...", section "Complex KDA (CKDA) Mimarisi ve Parametre
  * Genislemesi"; "Gated DeltaNet-2", Methodology section 1 with b = w =
- * beta).  The pages give no backward; this is the exact gradient of the
- * forward above, computed in fp32 on CUDA cores with the states recomputed
- * from checkpoints (every 64th token, then every 4th) -- no division, so
- * zero and negative gates are exact.
+ * beta; the gate-aware backward of "Gated DeltaNet-2", Methodology section
+ * 3, names the per-channel gates entering the gradient directly but prints
+ * no formula).  This is the exact gradient of the forward above, computed
+ * token by token in fp32 on CUDA cores with the states recomputed from
+ * checkpoints (every 64th token, then every 4th) -- no division, so zero
+ * and negative gates are exact.
  *
  *   q, k, v, alpha, beta, S0, cu_seqlens, B, T, H, d_k, d_v, dtype:
  *            the forward's inputs, layouts and rules (ckda_fwd_chunked).
