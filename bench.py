@@ -74,6 +74,8 @@ def _args():
     ap.add_argument("--decode-steps", type=int, default=DEC_STEPS,
                     help="decode steps timed (inputs for all of them are pre-generated)")
     ap.add_argument("--no-bwd", action="store_true", help="skip the backward sub-measure")
+    ap.add_argument("--no-long", action="store_true",
+                    help="skip the long-context prefill sub-measure (B=1, T=65536, H=32)")
     ap.add_argument("--no-sfda", action="store_true",
                     help="skip the SFDA (phase-decay gates) sub-measure")
     ap.add_argument("--no-gdn2", action="store_true",
@@ -317,6 +319,9 @@ def run_ours(args, ws, rank, local):
         if not off:
             variants[kind] = _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier,
                                           max_ranks, ws, hbm_peak)
+    if not args.no_long:
+        variants["long_prefill"] = _run_long(ck, torch, inputs, rank, dev, stream, barrier,
+                                             max_ranks, ws, hbm_peak)
     if not args.no_bwd:
         variants["bwd"] = _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws,
                                    hbm_peak)
@@ -499,6 +504,76 @@ def _run_variant(kind, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_frac_of_measured": gbs / hbm_peak,
             "gpu_launches": steps * (2 if path == "tcgen05" else 1)}
+
+
+def _run_long(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=10):
+    """The long-context prefill (B=1, T=65536, H=32, d=128, bf16 q/k/v, S0 read,
+    S_final stored): the forward's two kernels timed apart, as in the main step."""
+    Bl, Tl, Hl = 1, 65536, 32
+    c = inputs.long_prefill(seed=6000 + rank, device=dev, T=Tl, H=Hl, d=D)
+    out = torch.empty(c.v.shape, dtype=torch.float32, device=dev)
+    S_final = torch.empty((Bl, Hl, D, D), dtype=torch.float32, device=dev)
+    wsb = torch.empty(ck.workspace_bytes(Bl, Tl, Hl, D, D, CHUNK), dtype=torch.uint8, device=dev)
+
+    def step(mid=None):
+        ck.fwd_factors(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, workspace=wsb)
+        if mid is not None:
+            mid.record(stream)
+        ck.fwd_carry(wsb, Bl, Tl, Hl, D, D, S0=c.S0, chunk=CHUNK, out=out, S_final=S_final)
+
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(dev)
+    assert ck.device_status(dev) == 0
+    ks = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    km = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ke = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    for i in range(steps):
+        ks[i].record(stream)
+        step(km[i])
+        ke[i].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    f_ms = max_ranks(statistics.mean(ks[i].elapsed_time(km[i]) for i in range(steps)))
+    c_ms = max_ranks(statistics.mean(km[i].elapsed_time(ke[i]) for i in range(steps)))
+    ms = f_ms + c_ms
+    # the same forward as a chunk-parallel scan over G segments per sequence
+    scan = {}
+    for G in (2, 4):
+        wss = torch.empty(ck.scan_workspace_bytes(Bl, Tl, Hl, D, D, G), dtype=torch.uint8,
+                          device=dev)
+        for _ in range(2):
+            ck.fwd_chunked_scan(c.q, c.k, c.v, c.alpha, c.beta, G, S0=c.S0, out=out,
+                                S_final=S_final, workspace=wss)
+        torch.cuda.synchronize(dev)
+        assert ck.device_status(dev) == 0
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(5):
+            ck.fwd_chunked_scan(c.q, c.k, c.v, c.alpha, c.beta, G, S0=c.S0, out=out,
+                                S_final=S_final, workspace=wss)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        scan[f"segments_{G}"] = {"ms_per_step": max_ranks(e0.elapsed_time(e1)) / 5,
+                                 "gpu_launches_per_step": 4}
+        del wss
+    th = Bl * Tl * Hl
+    nbytes = th * BYTES_PER_TOKEN_HEAD + 2 * Bl * Hl * D * D * 4  # + S0 read, S_final written
+    return {"workload": f"long_prefill B={Bl} H={Hl} T={Tl} d={D} C={CHUNK} bf16 q/k/v, fp32 "
+                        "gates and out, S0 read, S_final stored (tcgen05 kernels)",
+            "ms_per_step": ms, "tokens_per_s": ws * Bl * Tl / (ms / 1e3),
+            "kernels": {"factor_kernel_ms": f_ms, "carry_kernel_ms": c_ms,
+                        "carry_ctas": 2 * Hl * Bl},
+            "chunk_parallel_scan": scan,
+            "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
+            "hbm_frac_of_measured": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
+            "gpu_launches": 2 * steps}
 
 
 def _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=5):

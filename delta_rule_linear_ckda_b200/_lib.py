@@ -42,6 +42,8 @@ SIGNATURES = {
                                    _i, _i, _i, _i, _vp, ctypes.c_size_t, _vp]),
     "ckda_sfda_fwd_chunked_fp32core": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i,
                                             _i, _i, _i, _i, _i, _i, _vp]),
+    "ckda_fwd_chunked_scan": (_i, [_vp] * 8 + [_i] * 9 + [_vp, ctypes.c_size_t, _vp]),
+    "ckda_fwd_chunked_scan_workspace_bytes": (ctypes.c_int64, [_i] * 6),
     "ckda_bwd_chunked": (_i, [_vp] * 15 + [_i] * 7 + [_vp, ctypes.c_size_t, _vp]),
     "ckda_bwd_chunked_workspace_bytes": (ctypes.c_int64, [_i, _i, _i, _i, _i, _i]),
     "ckda_fwd_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,

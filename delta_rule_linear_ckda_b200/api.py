@@ -324,6 +324,52 @@ def sfda_fwd_chunked(q, k, v, alpha, theta, beta, S0=None, cu_seqlens=None, chun
     return out, S_final
 
 
+def scan_workspace_bytes(B, T, H, dk, dv, segments) -> int:
+    """Scratch bytes ``fwd_chunked_scan`` needs for these sizes."""
+    rc = _lib.load().ckda_fwd_chunked_scan_workspace_bytes(B, T, H, dk, dv, segments)
+    if rc < 0:
+        raise CKDAError(int(rc), "ckda_fwd_chunked_scan_workspace_bytes")
+    return int(rc)
+
+
+def fwd_chunked_scan(q, k, v, alpha, beta, segments: int, S0=None, chunk: int = 64, out=None,
+                     S_final=None, return_final: bool = True, out_dtype=None, workspace=None):
+    """``fwd_chunked`` for fixed-length batches as a chunk-parallel scan over
+    ``segments`` segments of each sequence (``ckda_fwd_chunked_scan``): segment
+    summaries [M | B] in parallel, a scan of the segment start states, then
+    every segment's carry in parallel.  Same result up to rounding."""
+    dev = q.device
+    B, T, H, dk, dv, N = _inputs_shape(q, k, v, alpha, beta, None)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, dev)
+        if tuple(S0.shape) != (N, H, dk, dv):
+            raise ValueError(f"S0 must be [{N}, {H}, {dk}, {dv}]")
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    if out is None:
+        out = torch.empty(v.shape, dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+    if return_final and S_final is None:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _need(S_final, "S_final", torch.float32, dev)
+    if workspace is None:
+        workspace = torch.empty(max(1, scan_workspace_bytes(B, T, H, dk, dv, segments)),
+                                dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_fwd_chunked_scan(
+            _p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S0), _p(out), _p(S_final), B, T, H, dk,
+            dv, chunk, _DT[q.dtype], _DT[out_dtype], segments, _p(workspace), workspace.numel(),
+            _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_fwd_chunked_scan")
+    return out, S_final
+
+
 def bwd_workspace_bytes(B, T, H, dk, dv, varlen=False) -> int:
     """Scratch bytes ``bwd_chunked`` needs for these sizes."""
     rc = _lib.load().ckda_bwd_chunked_workspace_bytes(B, T, H, dk, dv, 1 if varlen else 0)

@@ -30,6 +30,11 @@ size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int 
 cudaError_t launch_bounded_wait_probe(int* status, unsigned long long limit_ns,
                                       cudaStream_t stream);
 size_t bwd_workspace_bytes(int dk, int dv, int n_seqs, int T, int H, bool varlen);
+size_t fwd_tc_scan_workspace_bytes(int dk, int dv, int n_seqs, int T, int H, int G);
+cudaError_t launch_fwd_tc_scan(int out_dtype, int dv, const void* q, const void* k,
+                               const void* v, const float* alpha, const float* beta,
+                               const float* S0, void* out, float* S_final, int n_seqs, int T,
+                               int H, int G, void* ws, int* status, cudaStream_t stream);
 cudaError_t launch_bwd(int dtype, int grad_dtype, int dk_, int dv_, const void* q, const void* k,
                        const void* v, const float* alpha, const float* beta, const float* S0,
                        const int32_t* cu, const void* dO, const float* dSf, float* dq, float* dk,
@@ -293,6 +298,46 @@ int64_t ckda_fwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v, 
   int rc = validate_sizes(B, T, H, d_k, d_v, &chunk, dtype, out_dtype, varlen);
   if (rc != CKDA_OK) return rc;
   return (int64_t)ckda::fwd_tc_workspace_bytes(dtype, d_k, d_v, chunk, B, T, H, varlen != 0);
+}
+
+int64_t ckda_fwd_chunked_scan_workspace_bytes(int B, int T, int H, int d_k, int d_v,
+                                              int segments) {
+  int chunk = 64;
+  int rc = validate_sizes(B, T, H, d_k, d_v, &chunk, CKDA_BF16, CKDA_F32, 0);
+  if (rc != CKDA_OK) return rc;
+  if (segments < 1) return CKDA_ERR_INVALID_ARG;
+  if (B == 0) return 0;
+  if (!ckda::fwd_tc_supported(CKDA_BF16, d_k, d_v, 64, B, T, H, false)) return CKDA_ERR_UNSUPPORTED;
+  return (int64_t)ckda::fwd_tc_scan_workspace_bytes(d_k, d_v, B, T, H, segments);
+}
+
+int ckda_fwd_chunked_scan(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* beta, const float* S0, void* out, float* S_final, int B,
+                          int T, int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
+                          int segments, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = validate_fwd(q, k, v, alpha, beta, S0, nullptr, out, S_final, B, T, H, d_k, d_v,
+                        &chunk, dtype, out_dtype);
+  if (rc != CKDA_OK) return rc;
+  if (segments < 1) return CKDA_ERR_INVALID_ARG;
+  if (B == 0) return CKDA_OK;
+  if (!ckda::fwd_tc_supported(dtype, d_k, d_v, chunk, B, T, H, false)) return CKDA_ERR_UNSUPPORTED;
+  const size_t need = ckda::fwd_tc_scan_workspace_bytes(d_k, d_v, B, T, H, segments);
+  if (workspace == nullptr || workspace_bytes < need ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return CKDA_ERR_WORKSPACE;
+  {
+    const void* ws_end = static_cast<const uint8_t*>(workspace) + need;
+    const void* ptrs[] = {q, k, v, alpha, beta, S0, out, S_final};
+    for (const void* p : ptrs)
+      if (p != nullptr && p >= workspace && p < ws_end) return CKDA_ERR_WORKSPACE;
+  }
+  if (S_final != nullptr && S_final == S0 && segments > 1) return CKDA_ERR_INVALID_ARG;
+  int* status = status_ptr();
+  if (status == nullptr) return CKDA_ERR_CUDA;
+  cudaError_t e = ckda::launch_fwd_tc_scan(out_dtype, d_v, q, k, v, alpha, beta, S0, out, S_final,
+                                           B, T, H, segments, workspace, status,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
 int64_t ckda_bwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v, int varlen) {

@@ -1242,6 +1242,18 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
 // SF: gamma holds (re, im) pairs and multiplies the state's row pairs
 // (2p, 2p+1) as a complex scalar; the partner row is the neighbouring lane.
+//
+// Segments (the chunk-parallel scan): a sequence's chunks split into
+// `seg_n` contiguous segments, chunks [g nck / seg_n, (g + 1) nck / seg_n);
+// this launch runs `seg_launch` of them (blockIdx.z = n seg_launch + g).
+// With summ == NULL (outputs): segment 0 starts from S0, segment g > 0 from
+// seg_start[n, g] ([N, seg_n, H, DK, DV] fp32), and the last segment stores
+// S_final.  With summ != NULL (the affine summary of a segment, "Principales
+// Contribuciones" item 3): the launch's columns are [M | B], DK + DV of them;
+// the M columns start from the identity and take no V term (the segment's
+// transfer matrix), the B columns start from zero (the zero-start state);
+// nothing is output and the end state goes to summ[n, g] ([N, seg_launch, H,
+// DK, DK + DV] fp32).  seg_n = seg_launch = 1 is the plain forward.
 template <typename Tout, bool SF>
 __global__ void __launch_bounds__(NT, 1)
 carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
@@ -1249,7 +1261,9 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
              const __grid_constant__ CUtensorMap tm_out,
              const float* __restrict__ ws_g,
              const float* S0, const int32_t* __restrict__ cu, Tout* __restrict__ out,
-             float* S_final, int n_seqs, int T, int H, int DV, int nch, int* status) {
+             float* S_final, int n_seqs, int T, int H, int DV, int nch, int* status,
+             int seg_n, int seg_launch, const float* __restrict__ seg_start,
+             float* __restrict__ summ) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(sm);
@@ -1258,7 +1272,11 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   const int lane = tid & 31;
   const int j0 = blockIdx.x * BV;
   const int h = blockIdx.y;
-  const int n = blockIdx.z;
+  const int n = blockIdx.z / seg_launch;
+  const int seg = blockIdx.z % seg_launch;
+  const bool summary = summ != nullptr;
+  const bool mcols = summary && j0 < DK;  // transfer-matrix columns
+  const int jv = summary ? j0 - DK : j0;  // V and output column of this CTA
 
   const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
   if (!sr.ok) return;
@@ -1294,11 +1312,26 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   const int half = warp >> 2;
   const int srow = 32 * q4 + lane;
   const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + 32 * half;
+  // this thread's 32 start values (row srow, 32 columns)
+  const float* s_row = nullptr;
+  if (seg == 0) {
+    if (S0 != nullptr) s_row = S0 + s_off;
+  } else {
+    s_row = seg_start + ((((size_t)n * seg_n + seg) * H + h) * DK + srow) * DV + j0 + 32 * half;
+  }
   float S[32];
 #pragma unroll
   for (int e = 0; e < 32; e += 4) {
     float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (S0 != nullptr) v4 = *reinterpret_cast<const float4*>(S0 + s_off + e);
+    if (summary) {
+      if (mcols) {
+        const int c = j0 + 32 * half + e - srow;  // identity: 1 where column == row
+        v4 = make_float4(c == 0 ? 1.f : 0.f, c == -1 ? 1.f : 0.f, c == -2 ? 1.f : 0.f,
+                         c == -3 ? 1.f : 0.f);
+      }
+    } else if (s_row != nullptr) {
+      v4 = *reinterpret_cast<const float4*>(s_row + e);
+    }
     S[e] = v4.x; S[e + 1] = v4.y; S[e + 2] = v4.z; S[e + 3] = v4.w;
   }
 #pragma unroll
@@ -1308,9 +1341,12 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
   const int64_t tok0 = sr.begin;
   const int64_t tok1 = sr.end;
-  const int nchunks = (int)((tok1 - tok0 + C - 1) / C);
+  const int nck_all = (int)((tok1 - tok0 + C - 1) / C);
+  // this segment's chunks [cbeg, cbeg + nchunks)
+  const int cbeg = (int)((int64_t)seg * nck_all / seg_n);
+  const int nchunks = (int)((int64_t)(seg + 1) * nck_all / seg_n) - cbeg;
   const int64_t slot0 = slot_base(cu, n, nch);
-  auto unit_of = [&](int c) -> int64_t { return (slot0 + c) * H + h; };
+  auto unit_of = [&](int c) -> int64_t { return (slot0 + cbeg + c) * H + h; };
   // phase bits advance only on a successful wait (see the factor kernel)
   uint32_t ph0 = 0, ph1 = 0, ph_mma = 0;
   int pend0 = 0, pend1 = 0, pend_mma = 0;
@@ -1334,7 +1370,7 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), bar);
     tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), bar);
     tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), bar);
-    tma_load_2d(base + CS_V, &tm_v16, j0, (int)(uidx * C), bar);
+    tma_load_2d(base + CS_V, &tm_v16, mcols ? 0 : jv, (int)(uidx * C), bar);
   };
   if (tid == 0) {
     if (nchunks > 0) issue(0, 0);
@@ -1354,10 +1390,10 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
   for (int c = 0; c < nchunks; ++c) {
     const int st = c & 1;
-    const int64_t t0 = tok0 + (int64_t)c * C;
+    const int64_t t0 = tok0 + (int64_t)(cbeg + c) * C;
     const int Lc = (tok1 - t0 < (int64_t)C) ? (int)(tok1 - t0) : C;
     const uint32_t stage = sb + st * kStageBytes;
-    const bool tma_out = (cu == nullptr) || Lc == C;
+    const bool tma_out = !summary && ((cu == nullptr) || Lc == C);
     ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
     ok = __syncthreads_and(ok);
     if (!ok) break;
@@ -1368,18 +1404,20 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(128, 64, 0, 1);
+      if (!mcols) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(stage + CS_IP + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(stage + CS_V + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_X, ad, bd, id, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = smem_desc(stage + CS_IP + kk * 32, 16, 1024, kSwizzle128);
+          const uint64_t bd = smem_desc(stage + CS_V + kk * 2048, 8192, 1024, kSwizzle128);
+          mma_f16(tmem + TM2_X, ad, bd, id, kk > 0 ? 1u : 0u);
+        }
       }
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint64_t ad =
             smem_desc(stage + CS_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
         const uint64_t bd = smem_desc(sb + OFF2_SB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_X, ad, bd, id, 1u);
+        mma_f16(tmem + TM2_X, ad, bd, id, (mcols && kk == 0) ? 0u : 1u);
       }
       mma_commit(bar_mma);
     }
@@ -1402,7 +1440,7 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4)
           st_chunk8(sm + OFF2_UB, sw128_chunk(srow, 32 * half + 8 * c4, 64), x + 8 * c4);
-      } else {
+      } else if (!summary) {
         const int r = srow - 64;
         if (tma_out)
           stage_row32<Tout>(sb + OFF2_OB, r, half, x);
@@ -1418,11 +1456,12 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       // packed batch: only whole chunks go through TMA
       const int x0 = h * DV + j0;
       if (cu == nullptr) {
+        const int y0 = (cbeg + c) * C;
         if (sizeof(Tout) == 4) {
-          tma_store_3d(&tm_out, sb + OFF2_OB, x0, c * C, n);
-          tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, c * C, n);
+          tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
+          tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, y0, n);
         } else {
-          tma_store_3d(&tm_out, sb + OFF2_OB, x0, c * C, n);
+          tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
         }
       } else {
         if (sizeof(Tout) == 4) {
@@ -1498,7 +1537,13 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   if (tid == 0) bulk_wait_all();
 
   if (ok) {
-    if (S_final != nullptr) {
+    if (summary) {
+      float* dst = summ + (((size_t)n * seg_launch + seg) * H + h) * DK * (DK + DV) +
+                   (size_t)srow * (DK + DV) + j0 + 32 * half;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    } else if (S_final != nullptr && seg == seg_n - 1) {
 #pragma unroll
       for (int e = 0; e < 32; e += 4)
         *reinterpret_cast<float4*>(S_final + s_off + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
@@ -1514,6 +1559,67 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, kTmem2Cols);
+}
+
+// ---- the scan over segment summaries ----------------------------------------------
+//
+// For one (sequence, head): S_start(0) = S0 (or 0) and
+//   S_start(g + 1) = M_g S_start(g) + B_g,   g = 0 .. seg_n - 2,
+// the exact affine transfer of a block of chunks ("Semidirect Fourier Delta
+// Attention" page, "Principales Contribuciones" item 3), with [M_g | B_g]
+// from the summary carry.  fp32 on CUDA cores: 256 threads, each an 8 x 8
+// block of the DK x DV product (DV = 128; DV = 64 uses half of them).
+constexpr int kScanThreads = 256;
+constexpr size_t kScanSmem = (size_t)(DK * DK + DK * 128) * 4;
+
+__global__ void __launch_bounds__(kScanThreads, 1)
+scan_kernel(const float* __restrict__ summ, const float* __restrict__ S0, float* __restrict__ seg_start,
+            int H, int DV, int seg_n) {
+  extern __shared__ __align__(16) float sm_scan[];
+  float* Ms = sm_scan;            // M_g [DK][DK]
+  float* Ss = sm_scan + DK * DK;  // S_start(g) [DK][DV]
+  const int tid = threadIdx.x;
+  const int h = blockIdx.x, n = blockIdx.y;
+  const int W = DK + DV;
+  for (int e = tid; e < DK * DV; e += kScanThreads)
+    Ss[e] = (S0 != nullptr) ? S0[(((size_t)n * H + h) * DK) * DV + e] : 0.f;
+  const int i0 = 8 * (tid / 16), jb = 8 * (tid % 16);
+  const bool act = jb < DV;
+  for (int g = 0; g + 1 < seg_n; ++g) {
+    const float* sg = summ + (((size_t)n * (seg_n - 1) + g) * H + h) * DK * W;
+    __syncthreads();  // Ss holds S_start(g); Ms is free
+    for (int e = tid; e < DK * DK; e += kScanThreads) Ms[e] = sg[(size_t)(e / DK) * W + e % DK];
+    __syncthreads();
+    float acc[8][8];
+    if (act) {
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = sg[(size_t)(i0 + a) * W + DK + jb + b];
+      for (int kx = 0; kx < DK; ++kx) {
+        float m[8], x[8];
+#pragma unroll
+        for (int a = 0; a < 8; ++a) m[a] = Ms[(i0 + a) * DK + kx];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) x[b] = Ss[kx * DV + jb + b];
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+          for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(m[a], x[b], acc[a][b]);
+      }
+    }
+    __syncthreads();  // every thread is done reading Ss
+    if (act) {
+      float* dst = seg_start + ((((size_t)n * seg_n + g + 1) * H + h) * DK) * DV;
+#pragma unroll
+      for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          Ss[(i0 + a) * DV + jb + b] = acc[a][b];
+          dst[(size_t)(i0 + a) * DV + jb + b] = acc[a][b];
+        }
+    }
+  }
 }
 
 // ---- host side ------------------------------------------------------------------
@@ -1590,11 +1696,21 @@ cudaError_t set_smem(K kern, size_t bytes) {
 // `stream`.
 constexpr int kFactors = 1, kCarry = 2;
 
+// Segments of the carry phase (the chunk-parallel scan); the default is the
+// plain forward (one segment).
+struct Segs {
+  int n = 1;                      // segments per sequence
+  int launch = 1;                 // segments this carry launch runs
+  const float* start = nullptr;   // start states of the segments
+  float* summ = nullptr;          // non-NULL: summary launch ([M | B] per segment)
+};
+
 template <int DV, typename Tout, int GK>
 cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, const float* bg, const float* wg, const float* theta,
                      const float* S0, const int32_t* cu, void* out, float* S_final, int n_seqs,
-                     int T, int H, void* ws, int* status, cudaStream_t stream) {
+                     int T, int H, void* ws, int* status, cudaStream_t stream,
+                     Segs segs = Segs()) {
   constexpr bool SF = GK == kSfda;
   const uint64_t rows = cu ? (uint64_t)T : (uint64_t)n_seqs * (uint64_t)T;
   const int nch = (int)(((int64_t)T + C - 1) / C);
@@ -1673,10 +1789,12 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       if (e != cudaSuccess) return e;
       attr2 = true;
     }
-    dim3 grid(DV / BV, H, n_seqs);
+    const int cols = segs.summ != nullptr ? DK + DV : DV;
+    dim3 grid(cols / BV, H, n_seqs * segs.launch);
     k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, mv16, mout, ws_g, S0, cu,
                                           static_cast<Tout*>(out), S_final, n_seqs, T, H, DV,
-                                          nch, status);
+                                          nch, status, segs.n, segs.launch, segs.start,
+                                          segs.summ);
     return cudaGetLastError();
   }
   return cudaSuccess;
@@ -1700,6 +1818,64 @@ size_t fwd_tc_workspace_bytes(int dtype, int dk, int dv, int C, int n_seqs, int 
   if (!fwd_tc_supported(dtype, dk, dv, C, n_seqs, T, H, varlen)) return 0;
   const int64_t nu = tc::n_units(varlen, n_seqs, T, H);
   return (size_t)nu * tc::unit_bytes(dv);
+}
+
+// ---- the chunk-parallel scan forward ------------------------------------------
+// Workspace: the factor workspace, then the segment summaries [N, G - 1, H,
+// DK, DK + DV] and the segment start states [N, G, H, DK, DV] (fp32).
+size_t fwd_tc_scan_workspace_bytes(int dk, int dv, int n_seqs, int T, int H, int G) {
+  if (!fwd_tc_supported(CKDA_BF16, dk, dv, tc::C, n_seqs, T, H, false) || G < 1) return 0;
+  const size_t fw = (size_t)tc::n_units(false, n_seqs, T, H) * tc::unit_bytes(dv);
+  const size_t sm = (size_t)n_seqs * (G - 1) * H * dk * (dk + dv) * 4;
+  const size_t ss = (size_t)n_seqs * G * H * dk * dv * 4;
+  return fw + sm + ss;
+}
+
+// The forward as G segments per sequence: factors of every chunk; the affine
+// summary [M_g | B_g] of segments 0 .. G - 2 (all in parallel); the scan of
+// the segments' start states; the carry of every segment from its start
+// state (all in parallel).  Same result as the plain forward up to rounding.
+cudaError_t launch_fwd_tc_scan(int out_dtype, int dv, const void* q, const void* k,
+                               const void* v, const float* alpha, const float* beta,
+                               const float* S0, void* out, float* S_final, int n_seqs, int T,
+                               int H, int G, void* ws, int* status, cudaStream_t stream) {
+  const size_t fw = (size_t)tc::n_units(false, n_seqs, T, H) * tc::unit_bytes(dv);
+  float* summ = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + fw);
+  float* starts = summ + (size_t)n_seqs * (G - 1) * H * tc::DK * (tc::DK + dv);
+  const bool bf = out_dtype == CKDA_BF16;
+  auto run = [&](int phases, tc::Segs sg, float* sfin) -> cudaError_t {
+#define CKDA_TC_SCAN(DVV, TO)                                                                  \
+  tc::launch_t<DVV, TO, tc::kKda>(phases, q, k, v, alpha, beta, nullptr, nullptr, nullptr, S0, \
+                                  nullptr, out, sfin, n_seqs, T, H, ws, status, stream, sg)
+    if (dv == 128) return bf ? CKDA_TC_SCAN(128, __nv_bfloat16) : CKDA_TC_SCAN(128, float);
+    return bf ? CKDA_TC_SCAN(64, __nv_bfloat16) : CKDA_TC_SCAN(64, float);
+#undef CKDA_TC_SCAN
+  };
+  cudaError_t e = run(tc::kFactors, tc::Segs(), S_final);
+  if (e != cudaSuccess || G == 1) {
+    if (e != cudaSuccess) return e;
+    return run(tc::kCarry, tc::Segs(), S_final);
+  }
+  tc::Segs sum;
+  sum.n = G;
+  sum.launch = G - 1;
+  sum.summ = summ;
+  if ((e = run(tc::kCarry, sum, nullptr)) != cudaSuccess) return e;
+  static bool attr = false;
+  if (!attr) {
+    if ((e = cudaFuncSetAttribute(tc::scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)tc::kScanSmem)) != cudaSuccess)
+      return e;
+    attr = true;
+  }
+  tc::scan_kernel<<<dim3(H, n_seqs), tc::kScanThreads, tc::kScanSmem, stream>>>(summ, S0, starts, H,
+                                                                                 dv, G);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  tc::Segs fin;
+  fin.n = G;
+  fin.launch = G;
+  fin.start = starts;
+  return run(tc::kCarry, fin, S_final);
 }
 
 // Everything the tensor-core kernels do not cover returns

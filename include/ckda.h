@@ -284,6 +284,47 @@ CKDA_API int ckda_sfda_fwd_chunked_fp32core(const void* q, const void* k, const 
                                             void* stream);
 
 /*
+ * ckda_fwd_chunked_scan -- ckda_fwd_chunked (fixed-length batches) as a
+ * chunk-parallel scan over `segments` contiguous segments of each sequence's
+ * chunks ("Semidirect Fourier Delta Attention", "Principales Contribuciones"
+ * item 3: a block of chunks acts on its start state as the exact affine map
+ * S_end = M S_start + B, with B the block's zero-start state):
+ *   1. the per-chunk factors of every chunk (as ckda_fwd_chunked);
+ *   2. for segments 0 .. segments - 2, all in parallel, the summary
+ *      [M_g | B_g]: the carry from [I | 0] with the V term on the B columns
+ *      only;
+ *   3. the scan S_start(g + 1) = M_g S_start(g) + B_g (fp32, S_start(0) = S0);
+ *   4. the carry of every segment from its start state, all in parallel,
+ *      writing out (and S_final from the last segment).
+ * The result equals ckda_fwd_chunked's up to rounding (the summaries go
+ * through the same fp16 tensor-core operands as the state).  segments = 1 is
+ * the plain forward.  Shapes: the tensor-core ones only (bf16 inputs,
+ * d_k = 128, d_v in {64, 128}, chunk 64), cu_seqlens not supported; other
+ * shapes return CKDA_ERR_UNSUPPORTED.  S_final may not alias S0 when
+ * segments > 1 (segments run concurrently).  Every other argument and rule
+ * is that of ckda_fwd_chunked; the workspace is
+ * ckda_fwd_chunked_scan_workspace_bytes().  On B200 this does not beat the
+ * plain forward at the sizes measured (the carry is latency-bound per chunk
+ * and the scan triples its work); it is the single-GPU form of splitting one
+ * sequence across GPUs.
+ */
+CKDA_API int ckda_fwd_chunked_scan(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* beta, const float* S0,
+                                   void* out, float* S_final, int B, int T, int H, int d_k,
+                                   int d_v, int chunk, int dtype, int out_dtype, int segments,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * ckda_fwd_chunked_scan_workspace_bytes -- scratch bytes of
+ * ckda_fwd_chunked_scan: ckda_fwd_chunked's workspace plus
+ * 4 N (segments - 1) H d_k (d_k + d_v) bytes of summaries and
+ * 4 N segments H d_k d_v bytes of segment start states; or the negative
+ * status a call with these sizes would return.  Pure host function.
+ */
+CKDA_API int64_t ckda_fwd_chunked_scan_workspace_bytes(int B, int T, int H, int d_k, int d_v,
+                                                       int segments);
+
+/*
  * ckda_fwd_chunked_workspace_bytes -- scratch bytes ckda_fwd_chunked needs
  * for these sizes (same meaning of B, T and `varlen` as in
  * ckda_fwd_chunked_path), 0 when the call runs the fp32 CUDA-core kernel,

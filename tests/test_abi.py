@@ -321,3 +321,25 @@ def test_bwd_entry_validates_without_a_gpu(lib):
     assert lib.ckda_bwd_chunked_workspace_bytes(2, 130, 3, 128, 48, 0) == -2
     # a workspace that overlaps an input
     assert bw(ws=P, ws_bytes=need) == -7
+
+
+def test_scan_entry_validates_without_a_gpu(lib):
+    def sc(**kw):
+        a = dict(q=P, k=P + 0x100000, v=P + 0x200000, alpha=P + 0x300000, beta=P + 0x400000,
+                 S0=None, out=P + 0x500000, S_final=None, B=1, T=128, H=1, dk_=128, dv_=128,
+                 chunk=64, dtype=1, odt=0, G=2, ws=None, ws_bytes=0)
+        a.update(kw)
+        return lib.ckda_fwd_chunked_scan(a["q"], a["k"], a["v"], a["alpha"], a["beta"], a["S0"],
+                                         a["out"], a["S_final"], a["B"], a["T"], a["H"], a["dk_"],
+                                         a["dv_"], a["chunk"], a["dtype"], a["odt"], a["G"],
+                                         a["ws"], a["ws_bytes"], None)
+
+    assert sc(G=0) == -1
+    assert sc(dtype=0) == -2              # fp32 inputs: not a tensor-core shape
+    assert sc(dk_=64) == -2
+    assert sc() == -7                     # no workspace
+    assert sc(B=0) == 0
+    need1 = lib.ckda_fwd_chunked_workspace_bytes(2, 300, 3, 128, 128, 64, 1, 0, 0)
+    need = lib.ckda_fwd_chunked_scan_workspace_bytes(2, 300, 3, 128, 128, 4)
+    assert need == need1 + 2 * 3 * 3 * 128 * 256 * 4 + 2 * 4 * 3 * 128 * 128 * 4
+    assert lib.ckda_fwd_chunked_scan_workspace_bytes(2, 300, 3, 128, 128, 0) == -1
