@@ -15,10 +15,9 @@
 //   dalpha = rowsum(dS' . S_prev);  dS <- Diag(a) dS'
 // with dS0 the final dS.  Every step needs the state before the token, so
 // the states are recomputed: a first forward pass stores the state at every
-// 64th token (workspace), the reverse pass re-runs each 64-token chunk from
-// its checkpoint storing the state at every 4th token (workspace, L2-sized),
-// and re-runs each 4-token segment into shared memory before walking it
-// backwards.  No division: zero and negative gates are exact.
+// 16th token (workspace), and the reverse pass re-runs each 16-token segment
+// from its checkpoint, storing its 17 states (workspace, L2-resident), before
+// walking it backwards.  No division: zero and negative gates are exact.
 //
 // One CTA owns one (sequence, head, d_v slice of BV <= 32 columns) and each
 // of its warps 4 columns of the slice over all d_k rows (lane l holds rows
@@ -39,9 +38,9 @@ namespace bwd {
 
 namespace cg = cooperative_groups;
 
-constexpr int kC = 64;  // checkpoint interval of the first pass (tokens)
-constexpr int kG = 4;   // recompute segment (tokens)
-constexpr int kSub = kC / kG;
+constexpr int kC = 16;  // checkpoint interval of the first pass = segment (tokens)
+constexpr int kG = 4;   // tokens per staged input block
+constexpr int kNB = kC / kG;
 
 template <int DK, int BV>
 struct Cfg {
@@ -53,10 +52,10 @@ struct Cfg {
   static constexpr int PW = 3 * DK + 1;             // partial sums per token: dq, dk, dalpha, dbeta
   // shared memory, in floats
   static constexpr int kWp = 0;                     // [2][NW][PW] the warps' partial sums of a token
-  static constexpr int kPbuf = kWp + 2 * NW * PW;   // [2][kG][PW] the CTA's partial sums of a segment
-  static constexpr int kR = kPbuf + 2 * kG * PW;    // [kG][BV] r of each token of the segment
-  static constexpr int kU = kR + kG * BV;           // [kG][BV] u of each token of the segment
-  static constexpr int kFloats = kU + kG * BV;
+  static constexpr int kPbuf = kWp + 2 * NW * PW;   // [2][kC][PW] the CTA's partial sums of a segment
+  static constexpr int kR = kPbuf + 2 * kC * PW;    // [kC][BV] r of each token of the segment
+  static constexpr int kU = kR + kC * BV;           // [kC][BV] u of each token of the segment
+  static constexpr int kFloats = kU + kC * BV;
 };
 
 // Inputs of one block of kG tokens, staged in shared memory by cp.async
@@ -86,10 +85,10 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 // The order in which the kernel consumes blocks of (up to) kG tokens:
-//   kind 0  first pass, chunk c (< nck - 1), block g of 16
-//   kind 1  second pass, chunk c, forward block g (< nsub - 1) to the segment states
-//   kind 2  second pass, chunk c, segment g, from nsub - 1 down to 0
-// Chunks of the second pass run from nck - 1 down to 0.
+//   kind 0  first pass, segment c (< nck - 1), block g of kNB (forward)
+//   kind 1  second pass, segment c, block g ascending (recompute the states)
+//   kind 2  second pass, segment c, block g descending (backward)
+// Segments of the second pass run from nck - 1 down to 0.
 struct Blk {
   int kind;  // -1: none left
   int c;
@@ -99,28 +98,25 @@ struct Blk {
 struct Sched {
   int Ls, nck;
   __device__ int lc(int c) const { return min(kC, Ls - c * kC); }
-  __device__ int nsub(int c) const { return (lc(c) + kG - 1) / kG; }
-  __device__ Blk pass2(int c) const {
-    if (c < 0) return Blk{-1, 0, 0};
-    return nsub(c) >= 2 ? Blk{1, c, 0} : Blk{2, c, nsub(c) - 1};
-  }
+  __device__ int nb(int c) const { return (lc(c) + kG - 1) / kG; }
+  __device__ Blk pass2(int c) const { return c < 0 ? Blk{-1, 0, 0} : Blk{1, c, 0}; }
   __device__ Blk first() const { return nck >= 2 ? Blk{0, 0, 0} : pass2(nck - 1); }
   __device__ Blk next(Blk b) const {
     if (b.kind == 0) {
-      if (b.g + 1 < kSub) return Blk{0, b.c, b.g + 1};
+      if (b.g + 1 < kNB) return Blk{0, b.c, b.g + 1};
       if (b.c + 1 < nck - 1) return Blk{0, b.c + 1, 0};
       return pass2(nck - 1);
     }
     if (b.kind == 1) {
-      if (b.g + 1 < nsub(b.c) - 1) return Blk{1, b.c, b.g + 1};
-      return Blk{2, b.c, nsub(b.c) - 1};
+      if (b.g + 1 < nb(b.c)) return Blk{1, b.c, b.g + 1};
+      return Blk{2, b.c, nb(b.c) - 1};
     }
     if (b.g > 0) return Blk{2, b.c, b.g - 1};
     return pass2(b.c - 1);
   }
   // tokens of a block (relative to the sequence start)
   __device__ int t0(Blk b) const { return b.c * kC + b.g * kG; }
-  __device__ int nt(Blk b) const { return b.kind == 2 ? min(kG, lc(b.c) - b.g * kG) : kG; }
+  __device__ int nt(Blk b) const { return b.kind == 0 ? kG : min(kG, lc(b.c) - b.g * kG); }
 };
 
 // Column sums of a warp's 4 columns over all rows: p[c] holds this lane's
@@ -214,9 +210,8 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   auto ck_ptr = [&](int c) -> float* {
     return ws_ck + (((size_t)(slot0 + c) * H + h) * nsl + srank) * tile + (size_t)tid * E;
   };
-  float* area = ws_sub + (((size_t)n * H + h) * nsl + srank) * (kSub + kG + 1) * tile;
-  auto sub_ptr = [&](int g) -> float* { return area + (size_t)g * tile + (size_t)tid * E; };
-  auto st_ptr = [&](int m) -> float* { return area + (size_t)(kSub + m) * tile + (size_t)tid * E; };
+  float* area = ws_sub + (((size_t)n * H + h) * nsl + srank) * (kC + 1) * tile;
+  auto st_ptr = [&](int m) -> float* { return area + (size_t)m * tile + (size_t)tid * E; };
 
   auto ld_st = [](const float* p, float* x) {
 #pragma unroll
@@ -337,6 +332,7 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
 
   float S[E];
   float dS[E];
+  float Sc[E];  // the state after the token the backward walk is at
   if (S0 != nullptr) {
     ld_glob(S0 + ((size_t)n * H + h) * DK * DV, S);
   } else {
@@ -360,128 +356,130 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
     issue(nx, sbuf ^ 1);  // the next block streams in meanwhile
     const uint8_t* sg = stage0 + sbuf * SG::kBytes;
     if (b.kind == 0) {
-      // ---- first pass: the state at the start of every chunk --------------------
+      // ---- first pass: the state at the start of every segment ------------------
       if (b.g == 0) st_st(ck_ptr(b.c), S);
       for (int m = 0; m < kG; ++m) fwd_step(S, sg, m, -1);
-    } else {
-      // ---- second pass, chunk b.c (the last chunk's start state is S already)
-      const int nsub = sch.nsub(b.c);
-      const bool chunk_start = (b.kind == 1 && b.g == 0) || (b.kind == 2 && b.g == nsub - 1 && nsub == 1);
-      if (chunk_start && b.c != nck - 1) ld_st(ck_ptr(b.c), S);
-      if (b.kind == 1) {
-        st_st(sub_ptr(b.g), S);
-        for (int m = 0; m < kG; ++m) fwd_step(S, sg, m, -1);
-      } else {
-        if (b.g == nsub - 1) st_st(sub_ptr(b.g), S);
-        const int64_t ts = L0 + sch.t0(b);
-        const int Lg = sch.nt(b);
-        ld_st(sub_ptr(b.g), S);
+    } else if (b.kind == 1) {
+      // ---- second pass, segment b.c: recompute its states (the last segment's
+      // start state is S already)
+      if (b.g == 0) {
+        if (b.c != nck - 1) ld_st(ck_ptr(b.c), S);
         st_st(st_ptr(0), S);
-        for (int m = 0; m < Lg; ++m) {
-          fwd_step(S, sg, m, m);
-          st_st(st_ptr(m + 1), S);
-        }
+      }
+      const int nt = sch.nt(b);
+      for (int m = 0; m < nt; ++m) {
+        const int j = b.g * kG + m;
+        fwd_step(S, sg, m, j);
+        st_st(st_ptr(j + 1), S);
+      }
+      if (b.g == sch.nb(b.c) - 1) {
         __syncwarp();
-        float* pb = pbuf + buf * kG * PW;
-        float Sc[E];
 #pragma unroll
-        for (int c = 0; c < E; ++c) Sc[c] = S[c];  // the state after the last token
-        for (int m = Lg - 1; m >= 0; --m) {
-          const size_t ti = (size_t)(ts + m) * H + h;
-          float qv[RPL], kv[RPL], av[RPL], go[4], vv[4];
-          rows(sg, SG::Q, m, qv, false);
-          rows(sg, SG::K, m, kv, false);
-          rows(sg, SG::A, m, av, true);
-          cols4(sg, SG::D, true, m, go);
-          cols4(sg, SG::V, false, m, vv);
-          const float bt = reinterpret_cast<const float*>(sg + SG::B)[m];
-          const float4 r4 = *reinterpret_cast<const float4*>(rr + m * BV + c0);
-          const float4 u4 = *reinterpret_cast<const float4*>(uu + m * BV + c0);
-          const float rv[4] = {r4.x, r4.y, r4.z, r4.w};
-          const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
-          float Sp[E];
-          ld_st(st_ptr(m), Sp);
-          // o = S^T q: dq (this warp's columns) and dS += q dO^T
-          float dqp[RPL], p[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int c = 0; c < E; ++c) Sc[c] = S[c];  // the state after the segment's last token
+      }
+    } else {
+      // ---- second pass, segment b.c: walk block b.g backwards -------------------
+      const int64_t ts = L0 + sch.t0(b);
+      const int Lg = sch.nt(b);
+      float* pb = pbuf + buf * kC * PW;
+      for (int m = Lg - 1; m >= 0; --m) {
+        const int j = b.g * kG + m;  // token index within the segment
+        const size_t ti = (size_t)(ts + m) * H + h;
+        float qv[RPL], kv[RPL], av[RPL], go[4], vv[4];
+        rows(sg, SG::Q, m, qv, false);
+        rows(sg, SG::K, m, kv, false);
+        rows(sg, SG::A, m, av, true);
+        cols4(sg, SG::D, true, m, go);
+        cols4(sg, SG::V, false, m, vv);
+        const float bt = reinterpret_cast<const float*>(sg + SG::B)[m];
+        const float4 r4 = *reinterpret_cast<const float4*>(rr + j * BV + c0);
+        const float4 u4 = *reinterpret_cast<const float4*>(uu + j * BV + c0);
+        const float rv[4] = {r4.x, r4.y, r4.z, r4.w};
+        const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
+        float Sp[E];
+        ld_st(st_ptr(j), Sp);
+        // o = S^T q: dq (this warp's columns) and dS += q dO^T
+        float dqp[RPL], p[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int r = 0; r < RPL; ++r) {
-            dqp[r] = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              dqp[r] = fmaf(Sc[4 * r + c], go[c], dqp[r]);
-              dS[4 * r + c] = fmaf(qv[r], go[c], dS[4 * r + c]);
-              p[c] = fmaf(dS[4 * r + c], kv[r], p[c]);
-            }
-          }
-          // S = S' + k u^T: du = dS^T k
-          float du[4];
-          col4_sums(p, du, lane);
-          float dbp = 0.f, dr[4];
+        for (int r = 0; r < RPL; ++r) {
+          dqp[r] = 0.f;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            dbp = fmaf(du[c], vv[c] - rv[c], dbp);
-            dr[c] = -bt * du[c];
+            dqp[r] = fmaf(Sc[4 * r + c], go[c], dqp[r]);
+            dS[4 * r + c] = fmaf(qv[r], go[c], dS[4 * r + c]);
+            p[c] = fmaf(dS[4 * r + c], kv[r], p[c]);
           }
-          if (lane < 4) {
-            const float d1 = (lane & 1) ? du[1] : du[0], d3 = (lane & 1) ? du[3] : du[2];
-            dv[ti * DV + j0 + c0 + lane] = bt * ((lane & 2) ? d3 : d1);
+        }
+        // S = S' + k u^T: du = dS^T k
+        float du[4];
+        col4_sums(p, du, lane);
+        float dbp = 0.f, dr[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          dbp = fmaf(du[c], vv[c] - rv[c], dbp);
+          dr[c] = -bt * du[c];
+        }
+        if (lane < 4) {
+          const float d1 = (lane & 1) ? du[1] : du[0], d3 = (lane & 1) ? du[3] : du[2];
+          dv[ti * DV + j0 + c0 + lane] = bt * ((lane & 2) ? d3 : d1);
+        }
+        float dkp[RPL], dap[RPL];
+#pragma unroll
+        for (int r = 0; r < RPL; ++r) {
+          float x = 0.f, y = 0.f, z = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            x = fmaf(dS[4 * r + c], uv[c], x);
+            y = fmaf(Sp[4 * r + c], dr[c], y);
+            const float dsp = fmaf(kv[r], dr[c], dS[4 * r + c]);  // dS' = dS + k dr^T
+            z = fmaf(dsp, Sp[4 * r + c], z);
+            dS[4 * r + c] = av[r] * dsp;
           }
-          float dkp[RPL], dap[RPL];
+          dkp[r] = fmaf(av[r], y, x);  // dS u + S' dr, S' = Diag(a) S_prev
+          dap[r] = z;
+        }
+        // the warps' partial sums meet in shared memory
+        float* w = wp + wbuf * L::NW * PW + warp * PW;
+        if (act) {
 #pragma unroll
           for (int r = 0; r < RPL; ++r) {
-            float x = 0.f, y = 0.f, z = 0.f;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              x = fmaf(dS[4 * r + c], uv[c], x);
-              y = fmaf(Sp[4 * r + c], dr[c], y);
-              const float dsp = fmaf(kv[r], dr[c], dS[4 * r + c]);  // dS' = dS + k dr^T
-              z = fmaf(dsp, Sp[4 * r + c], z);
-              dS[4 * r + c] = av[r] * dsp;
-            }
-            dkp[r] = fmaf(av[r], y, x);  // dS u + S' dr, S' = Diag(a) S_prev
-            dap[r] = z;
+            w[r0 + r] = dqp[r];
+            w[DK + r0 + r] = dkp[r];
+            w[2 * DK + r0 + r] = dap[r];
           }
-          // the warps' partial sums meet in shared memory
-          float* w = wp + wbuf * L::NW * PW + warp * PW;
-          if (act) {
-#pragma unroll
-            for (int r = 0; r < RPL; ++r) {
-              w[r0 + r] = dqp[r];
-              w[DK + r0 + r] = dkp[r];
-              w[2 * DK + r0 + r] = dap[r];
-            }
-          }
-          if (lane == 0) w[3 * DK] = dbp;
-          __syncthreads();
-          for (int e = tid; e < PW; e += NT) {
-            float sum = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < L::NW; ++ww) sum += wp[wbuf * L::NW * PW + ww * PW + e];
-            pb[m * PW + e] = sum;
-          }
-          wbuf ^= 1;
-#pragma unroll
-          for (int c = 0; c < E; ++c) Sc[c] = Sp[c];
         }
+        if (lane == 0) w[3 * DK] = dbp;
+        __syncthreads();
+        for (int e = tid; e < PW; e += NT) {
+          float sum = 0.f;
+#pragma unroll
+          for (int ww = 0; ww < L::NW; ++ww) sum += wp[wbuf * L::NW * PW + ww * PW + e];
+          pb[j * PW + e] = sum;
+        }
+        wbuf ^= 1;
+#pragma unroll
+        for (int c = 0; c < E; ++c) Sc[c] = Sp[c];
+      }
+      if (b.g == 0) {
         // the slices' partial sums of this segment: add across the cluster
+        const int64_t tseg = L0 + (int64_t)b.c * kC;
+        const int Lc = sch.lc(b.c);
         cluster.sync();
-        {
-          const int EE = Lg * PW;
-          const int e0 = (int)((int64_t)EE * srank / nsl), e1 = (int)((int64_t)EE * (srank + 1) / nsl);
-          for (int e = e0 + tid; e < e1; e += NT) {
-            float sum = 0.f;
-            for (int r = 0; r < nsl; ++r) sum += cluster.map_shared_rank(pb, r)[e];
-            const int m = e / PW, w = e % PW;
-            const size_t ti = (size_t)(ts + m) * H + h;
-            if (w < DK)
-              dq[ti * DK + w] = sum;
-            else if (w < 2 * DK)
-              dk[ti * DK + (w - DK)] = sum;
-            else if (w < 3 * DK)
-              dalpha[ti * DK + (w - 2 * DK)] = sum;
-            else
-              dbeta[ti] = sum;
-          }
+        const int EE = Lc * PW;
+        const int e0 = (int)((int64_t)EE * srank / nsl), e1 = (int)((int64_t)EE * (srank + 1) / nsl);
+        for (int e = e0 + tid; e < e1; e += NT) {
+          float sum = 0.f;
+          for (int r = 0; r < nsl; ++r) sum += cluster.map_shared_rank(pb, r)[e];
+          const int m = e / PW, w = e % PW;
+          const size_t ti = (size_t)(tseg + m) * H + h;
+          if (w < DK)
+            dq[ti * DK + w] = sum;
+          else if (w < 2 * DK)
+            dk[ti * DK + (w - DK)] = sum;
+          else if (w < 3 * DK)
+            dalpha[ti * DK + (w - 2 * DK)] = sum;
+          else
+            dbeta[ti] = sum;
         }
         buf ^= 1;
       }
@@ -549,15 +547,15 @@ static cudaError_t launch_dk(int dv_, const void* q, const void* k, const void* 
 
 }  // namespace bwd
 
-// Workspace of the backward: the chunk checkpoints (one d_k x d_v fp32 state
-// per 64-token chunk slot and head) and, per sequence and head, the 16
-// segment starts of a chunk and the kG + 1 states of a segment.
+// Workspace of the backward: the checkpoints (one d_k x d_v fp32 state per
+// 16-token segment slot and head) and, per sequence and head, the kC + 1
+// states of a segment.
 size_t bwd_workspace_bytes(int dk, int dv, int n_seqs, int T, int H, bool varlen) {
   const int64_t nch = ((int64_t)T + bwd::kC - 1) / bwd::kC;
   const int64_t slots = varlen ? (int64_t)T / bwd::kC + n_seqs : (int64_t)n_seqs * nch;
   // a stored state keeps each thread's values contiguous: max(d_k, 32) x d_v floats
   const size_t tile = (size_t)(dk > 32 ? dk : 32) * dv * sizeof(float);
-  return (size_t)slots * H * tile + (size_t)n_seqs * H * (bwd::kSub + bwd::kG + 1) * tile;
+  return (size_t)slots * H * tile + (size_t)n_seqs * H * (bwd::kC + 1) * tile;
 }
 
 cudaError_t launch_bwd(int dtype, int grad_dtype, int dk_, int dv_, const void* q, const void* k,

@@ -379,9 +379,9 @@ CKDA_API int ckda_fwd_chunked_path(int B, int T, int H, int d_k, int d_v, int ch
  * beta; the gate-aware backward of "Gated DeltaNet-2", Methodology section
  * 3, names the per-channel gates entering the gradient directly but prints
  * no formula).  This is the exact gradient of the forward above, computed
- * token by token in fp32 on CUDA cores with the states recomputed from
- * checkpoints (every 64th token, then every 4th) -- no division, so zero
- * and negative gates are exact.
+ * token by token in fp32 on CUDA cores with the states recomputed from a
+ * checkpoint at every 16th token -- no division, so zero and negative gates
+ * are exact.
  *
  *   q, k, v, alpha, beta, S0, cu_seqlens, B, T, H, d_k, d_v, dtype:
  *            the forward's inputs, layouts and rules (ckda_fwd_chunked).
@@ -415,10 +415,10 @@ CKDA_API int ckda_bwd_chunked(const void* q, const void* k, const void* v,
  * ckda_bwd_chunked_workspace_bytes -- scratch bytes ckda_bwd_chunked needs
  * (B, T and `varlen` as in ckda_fwd_chunked_path), or the negative status
  * an actual call with these sizes would return.  Pure host function: one
- * stored state of 4 max(d_k, 32) d_v bytes per 64-token chunk slot and head
- * (B ceil(T / 64) slots for a fixed-length batch, floor(T / 64) + N packed)
- * plus 21 such states per sequence and head (the 16 segment starts of a
- * chunk and the 5 states of a 4-token segment).
+ * stored state of 4 max(d_k, 32) d_v bytes per 16-token segment slot and
+ * head (B ceil(T / 16) slots for a fixed-length batch, floor(T / 16) + N
+ * packed) plus 17 such states per sequence and head (the states of one
+ * segment).
  */
 CKDA_API int64_t ckda_bwd_chunked_workspace_bytes(int B, int T, int H, int d_k, int d_v,
                                                   int varlen);

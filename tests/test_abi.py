@@ -315,9 +315,9 @@ def test_bwd_entry_validates_without_a_gpu(lib):
     assert bw() == -7              # no workspace
     assert bw(B=0) == 0
     need = lib.ckda_bwd_chunked_workspace_bytes(1, 8, 1, 16, 16, 0)
-    assert need == (1 + 21) * 32 * 16 * 4       # d_k < 32 stores 32 rows per state
+    assert need == (1 + 17) * 32 * 16 * 4       # d_k < 32 stores 32 rows per state
     assert lib.ckda_bwd_chunked_workspace_bytes(2, 130, 3, 128, 64, 0) == \
-        (2 * 3 * 3 + 2 * 3 * 21) * 128 * 64 * 4
+        (2 * 9 * 3 + 2 * 3 * 17) * 128 * 64 * 4     # 9 16-token slots per sequence
     assert lib.ckda_bwd_chunked_workspace_bytes(2, 130, 3, 128, 48, 0) == -2
     # a workspace that overlaps an input
     assert bw(ws=P, ws_bytes=need) == -7
