@@ -913,6 +913,19 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     pend_lv = 1;
     if (more) pend_in0 = 1;
     if (tid < C) beta_next = load_beta(nxt);
+    if constexpr (G2) {
+      // the next unit's erase and write gates are read with plain loads (in
+      // its gate passes and V conversion): pull their rows into L2 now, one
+      // 128-byte line per thread (64 rows x 4 lines of b, 4 of w)
+      const int r = tid >> 3, part = tid & 7;
+      if (more && r < nxt.Lc) {
+        const size_t row = (size_t)(nxt.t0 + r) * H + nxt.h;
+        if (part < 4)
+          prefetch_l2(bg + row * DK + 32 * part);
+        else if (32 * (part - 4) < DV)
+          prefetch_l2(wg + row * DV + 32 * (part - 4));
+      }
+    }
     TC_MARK(1);
 
     // ---- gate pass, half 1 (after the half-0 level GEMMs release the operands)
