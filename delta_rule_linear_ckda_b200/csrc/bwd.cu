@@ -202,9 +202,10 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
   const int nck = sch.nck;
 
   // workspace: every stored state keeps each thread's E values contiguous.
-  // Checkpoints are indexed by chunk slot (as the forward numbers its
-  // units); the segment starts and the segment's token states sit in a
-  // per-(sequence, head, slice) area.
+  // Checkpoints are indexed by 16-token segment slot (numbered as the
+  // forward numbers its chunks: a packed sequence n starts at slot
+  // floor(cu[n] / kC) + n); the kC + 1 states of the segment being walked sit
+  // in a per-(sequence, head, slice) area.
   const int64_t slot0 = (cu != nullptr) ? (int64_t)(sr.begin / kC) + n : (int64_t)n * nch_fixed;
   const size_t tile = (size_t)L::TS;
   auto ck_ptr = [&](int c) -> float* {
