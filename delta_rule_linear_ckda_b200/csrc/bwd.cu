@@ -153,11 +153,28 @@ __device__ __forceinline__ float ldf(const T* p) {
   return Elem<T>::to_f32(*p);
 }
 
-// RPL consecutive values of type T from shared memory, widened to fp32.
+// RPL consecutive values of type T from shared memory, widened to fp32
+// (one vector load when RPL is 2 or 4; p is aligned to RPL elements).
 template <int RPL, typename T>
 __device__ __forceinline__ void lds_rows(const T* p, float* x) {
+  if constexpr (RPL == 4 && sizeof(T) == 4) {
+    const float4 a = *reinterpret_cast<const float4*>(p);
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  } else if constexpr (RPL == 4 && sizeof(T) == 2) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(p);
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+  } else if constexpr (RPL == 2 && sizeof(T) == 4) {
+    const float2 a = *reinterpret_cast<const float2*>(p);
+    x[0] = a.x; x[1] = a.y;
+  } else if constexpr (RPL == 2 && sizeof(T) == 2) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    x[0] = a.x; x[1] = a.y;
+  } else {
 #pragma unroll
-  for (int r = 0; r < RPL; ++r) x[r] = Elem<T>::to_f32(p[r]);
+    for (int r = 0; r < RPL; ++r) x[r] = Elem<T>::to_f32(p[r]);
+  }
 }
 
 template <int DK, int BV, typename Tin, typename Tg>
@@ -279,15 +296,10 @@ bwd_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin* __re
 
   // the 4 values of this warp's columns of token m, widened to fp32
   auto cols4 = [&](const uint8_t* sg, int off, bool grad, int m, float* x) {
-    if (grad) {
-      const Tg* p = reinterpret_cast<const Tg*>(sg + off) + m * BV + c0;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) x[c] = Elem<Tg>::to_f32(p[c]);
-    } else {
-      const Tin* p = reinterpret_cast<const Tin*>(sg + off) + m * BV + c0;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) x[c] = Elem<Tin>::to_f32(p[c]);
-    }
+    if (grad)
+      lds_rows<4>(reinterpret_cast<const Tg*>(sg + off) + m * BV + c0, x);
+    else
+      lds_rows<4>(reinterpret_cast<const Tin*>(sg + off) + m * BV + c0, x);
   };
   auto rows = [&](const uint8_t* sg, int off, int m, float* x, bool f32) {
     if (!act) {
