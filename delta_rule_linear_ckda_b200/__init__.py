@@ -11,7 +11,7 @@ from __future__ import annotations
 _API = ("fwd_chunked", "fwd_chunked_static", "gdn2_fwd_chunked", "sfda_fwd_chunked", "fwd_factors",
         "fwd_carry", "fwd_path", "workspace_bytes", "bwd_chunked", "bwd_workspace_bytes",
         "fwd_chunked_scan", "scan_workspace_bytes",
-        "decode_step", "device_status")
+        "decode_step", "gdn2_decode_step", "sfda_decode_step", "device_status")
 __all__ = list(_API) + ["CKDAError", "lib_path"]
 
 

@@ -52,6 +52,8 @@ SIGNATURES = {
                             ctypes.c_size_t, _vp]),
     "ckda_fwd_chunked_fp32core": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_fwd_chunked_path": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
+    "ckda_gdn2_decode_step": (_i, [_vp] * 8 + [_i] * 6 + [_vp]),
+    "ckda_sfda_decode_step": (_i, [_vp] * 8 + [_i] * 6 + [_vp]),
     "ckda_decode_step": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_status_string": (ctypes.c_char_p, [_i]),
     "ckda_device_status": (_i, [_vp]),

@@ -451,38 +451,89 @@ def fwd_path(B, T, H, dk, dv, chunk=64, dtype=torch.bfloat16, out_dtype=torch.fl
     return "tcgen05" if rc == 1 else "fp32core"
 
 
+def _decode_out(q, v, out, out_dtype, dev):
+    if out_dtype is None:
+        out_dtype = out.dtype if out is not None else q.dtype
+    if out_dtype not in _DT:
+        raise TypeError("out_dtype must be float32 or bfloat16")
+    B, H, _ = q.shape
+    if out is None:
+        out = torch.empty((B, H, v.shape[-1]), dtype=out_dtype, device=dev)
+    else:
+        _need(out, "out", out_dtype, dev)
+    return out, out_dtype
+
+
+def _decode_checks(q, k, v, S, gates):
+    dev = q.device
+    if q.dtype not in _DT:
+        raise TypeError("q, k, v must be float32 or bfloat16")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, q.dtype, dev)
+    _need(S, "S", torch.float32, dev)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if tuple(S.shape) != (B, H, dk, dv) or k.shape != q.shape or tuple(v.shape[:2]) != (B, H):
+        raise ValueError("shape mismatch")
+    for name, t, shape in gates:
+        _need(t, name, torch.float32, dev)
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must be {tuple(shape)}")
+    return dev, B, H, dk, dv
+
+
 def decode_step(q, k, v, alpha, beta, S, out=None, out_dtype=None) -> torch.Tensor:
     """One recurrent step, in place on ``S`` ``[B, H, dk, dv]`` (fp32).
 
     q, k, alpha ``[B, H, dk]``; v ``[B, H, dv]``; beta ``[B, H]``.  Returns ``out``
     (``out_dtype`` defaults to the dtype of ``out`` if given, else the input dtype).
     """
-    dev = q.device
-    if q.dtype not in _DT:
-        raise TypeError("q, k, v must be float32 or bfloat16")
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, name, q.dtype, dev)
-    _need(alpha, "alpha", torch.float32, dev)
-    _need(beta, "beta", torch.float32, dev)
-    _need(S, "S", torch.float32, dev)
     B, H, dk = q.shape
-    dv = v.shape[-1]
-    if tuple(S.shape) != (B, H, dk, dv) or tuple(beta.shape) != (B, H):
-        raise ValueError("shape mismatch")
-    if out_dtype is None:
-        out_dtype = out.dtype if out is not None else q.dtype
-    if out_dtype not in _DT:
-        raise TypeError("out_dtype must be float32 or bfloat16")
-    if out is None:
-        out = torch.empty((B, H, dv), dtype=out_dtype, device=dev)
-    else:
-        _need(out, "out", out_dtype, dev)
+    dev, B, H, dk, dv = _decode_checks(q, k, v, S, (("alpha", alpha, (B, H, dk)),
+                                                    ("beta", beta, (B, H))))
+    out, out_dtype = _decode_out(q, v, out, out_dtype, dev)
     with torch.cuda.device(dev):
         rc = _lib.load().ckda_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(beta), _p(S), _p(out),
                                           B, H, dk, dv, _DT[q.dtype], _DT[out_dtype],
                                           _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_decode_step")
+    return out
+
+
+def gdn2_decode_step(q, k, v, alpha, b, w, S, out=None, out_dtype=None) -> torch.Tensor:
+    """One Gated DeltaNet-2 step in place on ``S`` (``ckda_gdn2_decode_step``):
+    erase gate ``b`` ``[B, H, dk]`` and write gate ``w`` ``[B, H, dv]`` (fp32) in
+    place of beta; otherwise as ``decode_step``."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, B, H, dk, dv = _decode_checks(q, k, v, S, (("alpha", alpha, (B, H, dk)),
+                                                    ("b", b, (B, H, dk)), ("w", w, (B, H, dv))))
+    out, out_dtype = _decode_out(q, v, out, out_dtype, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_gdn2_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(b), _p(w),
+                                               _p(S), _p(out), B, H, dk, dv, _DT[q.dtype],
+                                               _DT[out_dtype], _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_gdn2_decode_step")
+    return out
+
+
+def sfda_decode_step(q, k, v, alpha, theta, beta, S, out=None, out_dtype=None) -> torch.Tensor:
+    """One SFDA step in place on ``S`` (``ckda_sfda_decode_step``): decays
+    ``alpha`` and phases ``theta`` ``[B, H, dk / 2]`` (fp32) per channel pair,
+    ``beta`` ``[B, H]``; otherwise as ``decode_step``."""
+    B, H, dk = q.shape
+    dev, B, H, dk, dv = _decode_checks(q, k, v, S, (("alpha", alpha, (B, H, dk // 2)),
+                                                    ("theta", theta, (B, H, dk // 2)),
+                                                    ("beta", beta, (B, H))))
+    out, out_dtype = _decode_out(q, v, out, out_dtype, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.load().ckda_sfda_decode_step(_p(q), _p(k), _p(v), _p(alpha), _p(theta),
+                                               _p(beta), _p(S), _p(out), B, H, dk, dv,
+                                               _DT[q.dtype], _DT[out_dtype], _stream_ptr(dev))
+    if rc != 0:
+        raise CKDAError(rc, "ckda_sfda_decode_step")
     return out
 
 

@@ -10,8 +10,9 @@
 
 namespace ckda {
 cudaError_t launch_decode(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k,
-                          const void* v, const float* alpha, const float* beta, float* S, void* out,
-                          int BH, cudaStream_t stream);
+                          const void* v, const float* alpha, const float* beta, const float* bg,
+                          const float* wg, const float* theta, float* S, void* out, int BH,
+                          cudaStream_t stream);
 cudaError_t launch_fwd_simt(int dtype, int out_dtype, int dk, int dv, const void* q,
                             const void* k, const void* v, const float* alpha, const float* beta,
                             const float* bg, const float* wg, const float* theta,
@@ -184,6 +185,29 @@ int validate_sizes(int B, int T, int H, int d_k, int d_v, int* chunk, int dtype,
                       nullptr, B, T, H, d_k, d_v, chunk, dtype, out_dtype);
 }
 
+// The decode steps: `bg`, `wg` non-NULL select Gated DeltaNet-2 (b takes
+// beta's place in the checks), `theta` non-NULL SFDA.
+int decode_impl(const void* q, const void* k, const void* v, const float* alpha,
+                const float* beta, const float* bg, const float* wg, const float* theta,
+                float* S_inout, void* out, int B, int H, int d_k, int d_v, int dtype,
+                int out_dtype, void* stream) {
+  if (B < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
+  if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (out_dtype != CKDA_F32 && out_dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
+  if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
+  if ((int64_t)B * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
+  if (B == 0) return CKDA_OK;
+  const bool g2 = bg != nullptr || wg != nullptr;
+  if (!q || !k || !v || !alpha || !S_inout || !out) return CKDA_ERR_INVALID_ARG;
+  if (g2 ? (!bg || !wg) : !beta) return CKDA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, alpha, g2 ? bg : beta, wg, theta, S_inout, out};
+  for (const void* p : ptrs)
+    if (p != nullptr && !aligned16(p)) return CKDA_ERR_MISALIGNED;
+  if (out == S_inout || out == q || out == k || out == v) return CKDA_ERR_INVALID_ARG;
+  cudaError_t e = ckda::launch_decode(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, bg, wg,
+                                      theta, S_inout, out, B * H, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+}
 }  // namespace
 
 extern "C" {
@@ -398,23 +422,28 @@ int ckda_bwd_chunked(const void* q, const void* k, const void* v, const float* a
   return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
 }
 
+
 int ckda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
                      const float* beta, float* S_inout, void* out, int B, int H, int d_k, int d_v,
                      int dtype, int out_dtype, void* stream) {
-  if (B < 0 || H <= 0) return CKDA_ERR_INVALID_ARG;
-  if (dtype != CKDA_F32 && dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
-  if (out_dtype != CKDA_F32 && out_dtype != CKDA_BF16) return CKDA_ERR_UNSUPPORTED;
-  if (!supported_d(d_k) || !supported_d(d_v)) return CKDA_ERR_UNSUPPORTED;
-  if ((int64_t)B * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
-  if (B == 0) return CKDA_OK;
-  if (!q || !k || !v || !alpha || !beta || !S_inout || !out) return CKDA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, alpha, beta, S_inout, out};
-  for (const void* p : ptrs)
-    if (!aligned16(p)) return CKDA_ERR_MISALIGNED;
-  if (out == S_inout || out == q || out == k || out == v) return CKDA_ERR_INVALID_ARG;
-  cudaError_t e = ckda::launch_decode(dtype, out_dtype, d_k, d_v, q, k, v, alpha, beta, S_inout, out, B * H,
-                                      static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? CKDA_OK : CKDA_ERR_CUDA;
+  return decode_impl(q, k, v, alpha, beta, nullptr, nullptr, nullptr, S_inout, out, B, H, d_k,
+                     d_v, dtype, out_dtype, stream);
+}
+
+int ckda_gdn2_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* b, const float* w, float* S_inout, void* out, int B, int H,
+                          int d_k, int d_v, int dtype, int out_dtype, void* stream) {
+  if (B > 0 && (!b || !w)) return CKDA_ERR_INVALID_ARG;
+  return decode_impl(q, k, v, alpha, nullptr, b, w, nullptr, S_inout, out, B, H, d_k, d_v, dtype,
+                     out_dtype, stream);
+}
+
+int ckda_sfda_decode_step(const void* q, const void* k, const void* v, const float* alpha,
+                          const float* theta, const float* beta, float* S_inout, void* out, int B,
+                          int H, int d_k, int d_v, int dtype, int out_dtype, void* stream) {
+  if (B > 0 && !theta) return CKDA_ERR_INVALID_ARG;
+  return decode_impl(q, k, v, alpha, beta, nullptr, nullptr, theta, S_inout, out, B, H, d_k, d_v,
+                     dtype, out_dtype, stream);
 }
 
 int ckda_selftest_bounded_wait(int limit_us, void* stream) {

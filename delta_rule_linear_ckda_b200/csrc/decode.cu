@@ -8,6 +8,13 @@
 // which is S_t = (I - beta k k^T) Diag(alpha) S_{t-1} + beta k v^T and
 // o_t = S_t^T q_t rearranged so that S is read once and written once.
 //
+// Gated DeltaNet-2 ("Gated DeltaNet-2" page, Methodology section 1): the read
+// uses e = b . k and u = w . v - r (no beta).  SFDA ("Semidirect Fourier Delta
+// Attention (SFDA)" page, "Arquitectura Central"): S' = Lambda S, each pair of
+// rows (2p, 2p+1) turned by alpha_p (cos theta_p, sin theta_p); a thread then
+// holds whole row pairs, and the pairs' (cos, sin) are computed once per
+// (b, h) into shared memory.
+//
 // The step moves 2 * d_k * d_v * 4 bytes of state per head and does ~6
 // flops per state element: it is bound by HBM bandwidth.  Each CTA owns
 // one (b, h); each thread owns 4 adjacent columns (one 16-byte vector) of
@@ -19,27 +26,38 @@
 
 namespace ckda {
 
-template <int DK, int DV>
+// Gate families of the decode step.
+constexpr int kDecKda = 0, kDecGdn2 = 1, kDecSfda = 2;
+
+template <int DK, int DV, bool SF = false>
 struct DecodeShape {
   static constexpr int kCpr = DV / 4;  // threads across one row (float4 each)
-  static constexpr int kThreads = (DK * DV / 4 < 256) ? DK * DV / 4 : 256;
+  static constexpr int kThreads0 = (DK * DV / 4 < 256) ? DK * DV / 4 : 256;
+  // SFDA: at least two rows per thread (a whole row pair)
+  static constexpr int kThreads = (SF && DK * kCpr / kThreads0 < 2) ? kThreads0 / 2 : kThreads0;
   static constexpr int kRpp = kThreads / kCpr;  // rows covered per pass
   static constexpr int kRows = DK / kRpp;       // rows per thread
   static_assert(kThreads % 32 == 0 || kThreads < 32, "block size");
   static_assert(DK % kRpp == 0, "row split");
+  static_assert(!SF || kRows % 2 == 0, "row pairs");
 };
 
-template <int DK, int DV, typename Tin, typename Tout>
-__global__ void __launch_bounds__(DecodeShape<DK, DV>::kThreads, 2)
+// bg, wg: the Gated DeltaNet-2 gates ([BH, d_k], [BH, d_v]); theta: the SFDA
+// phases ([BH, d_k / 2], alpha then holds d_k / 2 decays); unused otherwise.
+template <int DK, int DV, typename Tin, typename Tout, int GK>
+__global__ void __launch_bounds__(DecodeShape<DK, DV, GK == kDecSfda>::kThreads, 2)
 decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
                    const Tin* __restrict__ v, const float* __restrict__ alpha,
-                   const float* __restrict__ beta, float* __restrict__ S,
-                   Tout* __restrict__ out) {
-  using Sh = DecodeShape<DK, DV>;
+                   const float* __restrict__ beta, const float* __restrict__ bg,
+                   const float* __restrict__ wg, const float* __restrict__ theta,
+                   float* __restrict__ S, Tout* __restrict__ out) {
+  constexpr bool G2 = GK == kDecGdn2, SF = GK == kDecSfda;
+  using Sh = DecodeShape<DK, DV, SF>;
   constexpr int CPR = Sh::kCpr, RPP = Sh::kRpp, NR = Sh::kRows, NT = Sh::kThreads;
   __shared__ float4 red_r[RPP][CPR];
   __shared__ float4 red_p[RPP][CPR];
   __shared__ float kq_part[(NT + 31) / 32];
+  __shared__ float2 lam[SF ? DK / 2 : 1];
 
   const int bh = blockIdx.x;
   const int t = threadIdx.x;
@@ -47,27 +65,53 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   const int g = t / CPR;
   const size_t kvec = (size_t)bh * DK;
   float4* Sb = reinterpret_cast<float4*>(S + (size_t)bh * DK * DV);
+  // the rows of this thread: g + RPP m (SFDA: 2 (g + RPP (m / 2)) + m % 2, so
+  // both rows of a pair are held by the same thread)
+  auto row_of = [&](int m) -> int { return SF ? 2 * (g + RPP * (m >> 1)) + (m & 1) : g + RPP * m; };
 
   // Issue every state load first (16 bytes each, streaming).
   float4 s[NR];
 #pragma unroll
-  for (int m = 0; m < NR; ++m) {
-    const int i = g + RPP * m;
-    s[m] = __ldcs(Sb + (size_t)i * CPR + c);
+  for (int m = 0; m < NR; ++m) s[m] = __ldcs(Sb + (size_t)row_of(m) * CPR + c);
+  if constexpr (SF) {
+    // the pairs' rotation-decay gates, once per (b, h)
+    for (int pp = t; pp < DK / 2; pp += NT) {
+      float sn, cs;
+      sincosf(__ldg(theta + (size_t)bh * (DK / 2) + pp), &sn, &cs);
+      const float a = __ldg(alpha + (size_t)bh * (DK / 2) + pp);
+      lam[pp] = make_float2(a * cs, a * sn);
+    }
+    __syncthreads();
   }
   float kr[NR];
   float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
+  if constexpr (SF) {
+    // S' = Lambda S on every row pair, then the column sums
+#pragma unroll
+    for (int m = 0; m < NR; m += 2) {
+      const int i = row_of(m);  // rows (i, i + 1) = (real, imaginary) of pair i / 2
+      const float2 l = lam[i >> 1];
+      const float4 e = s[m], o = s[m + 1];
+      s[m] = make_float4(fmaf(-l.y, o.x, l.x * e.x), fmaf(-l.y, o.y, l.x * e.y),
+                         fmaf(-l.y, o.z, l.x * e.z), fmaf(-l.y, o.w, l.x * e.w));
+      s[m + 1] = make_float4(fmaf(l.y, e.x, l.x * o.x), fmaf(l.y, e.y, l.x * o.y),
+                             fmaf(l.y, e.z, l.x * o.z), fmaf(l.y, e.w, l.x * o.w));
+    }
+  }
 #pragma unroll
   for (int m = 0; m < NR; ++m) {
-    const int i = g + RPP * m;
-    const float a = __ldg(alpha + kvec + i);
+    const int i = row_of(m);
     const float kk = Elem<Tin>::to_f32(k[kvec + i]);
     const float qq = Elem<Tin>::to_f32(q[kvec + i]);
     kr[m] = kk;
-    s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;
-    r.x = fmaf(s[m].x, kk, r.x); r.y = fmaf(s[m].y, kk, r.y);
-    r.z = fmaf(s[m].z, kk, r.z); r.w = fmaf(s[m].w, kk, r.w);
+    if constexpr (!SF) {
+      const float a = __ldg(alpha + kvec + i);
+      s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;
+    }
+    const float ek = G2 ? kk * __ldg(bg + kvec + i) : kk;  // the read direction
+    r.x = fmaf(s[m].x, ek, r.x); r.y = fmaf(s[m].y, ek, r.y);
+    r.z = fmaf(s[m].z, ek, r.z); r.w = fmaf(s[m].w, ek, r.w);
     p.x = fmaf(s[m].x, qq, p.x); p.y = fmaf(s[m].y, qq, p.y);
     p.z = fmaf(s[m].z, qq, p.z); p.w = fmaf(s[m].w, qq, p.w);
   }
@@ -94,11 +138,18 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 #pragma unroll
   for (int w = 0; w < (NT + 31) / 32; ++w) kqt += kq_part[w];
 
-  const float bt = __ldg(beta + bh);
   const float4 vv = load4_f32(v + (size_t)bh * DV + 4 * c);
   float4 u;
-  u.x = bt * (vv.x - R.x); u.y = bt * (vv.y - R.y);
-  u.z = bt * (vv.z - R.z); u.w = bt * (vv.w - R.w);
+  if constexpr (G2) {
+    // u = w . v - r
+    const float4 ww = *reinterpret_cast<const float4*>(wg + (size_t)bh * DV + 4 * c);
+    u.x = fmaf(ww.x, vv.x, -R.x); u.y = fmaf(ww.y, vv.y, -R.y);
+    u.z = fmaf(ww.z, vv.z, -R.z); u.w = fmaf(ww.w, vv.w, -R.w);
+  } else {
+    const float bt = __ldg(beta + bh);
+    u.x = bt * (vv.x - R.x); u.y = bt * (vv.y - R.y);
+    u.z = bt * (vv.z - R.z); u.w = bt * (vv.w - R.w);
+  }
   if (g == 0) {
     float4 o;
     o.x = fmaf(kqt, u.x, P.x); o.y = fmaf(kqt, u.y, P.y);
@@ -107,7 +158,7 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   }
 #pragma unroll
   for (int m = 0; m < NR; ++m) {
-    const int i = g + RPP * m;
+    const int i = row_of(m);
     float4 o = s[m];
     o.x = fmaf(kr[m], u.x, o.x); o.y = fmaf(kr[m], u.y, o.y);
     o.z = fmaf(kr[m], u.z, o.z); o.w = fmaf(kr[m], u.w, o.w);
@@ -115,55 +166,75 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   }
 }
 
+// Gates of a decode call: beta (CKDA), b and w (Gated DeltaNet-2), or beta
+// with the phases (SFDA).
+struct DecGates {
+  const float* beta;
+  const float* b;
+  const float* w;
+  const float* theta;
+};
+
 template <int DK, int DV, typename Tin, typename Tout>
 static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* alpha,
-                                   const float* beta, float* S, void* out, int BH,
-                                   cudaStream_t stream) {
-  using Sh = DecodeShape<DK, DV>;
-  decode_step_kernel<DK, DV, Tin, Tout><<<BH, Sh::kThreads, 0, stream>>>(
-      static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
-      beta, S, static_cast<Tout*>(out));
+                                   DecGates gt, float* S, void* out, int BH, cudaStream_t stream) {
+#define CKDA_DEC(GKV)                                                                          \
+  decode_step_kernel<DK, DV, Tin, Tout, GKV>                                                   \
+      <<<BH, DecodeShape<DK, DV, GKV == kDecSfda>::kThreads, 0, stream>>>(                      \
+          static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v),   \
+          alpha, gt.beta, gt.b, gt.w, gt.theta, S, static_cast<Tout*>(out))
+  if (gt.theta != nullptr)
+    CKDA_DEC(kDecSfda);
+  else if (gt.b != nullptr)
+    CKDA_DEC(kDecGdn2);
+  else
+    CKDA_DEC(kDecKda);
+#undef CKDA_DEC
   return cudaGetLastError();
 }
 
 template <int DK, typename Tin, typename Tout>
 static cudaError_t launch_decode_dv(int dv, const void* q, const void* k, const void* v,
-                                    const float* alpha, const float* beta, float* S, void* out,
-                                    int BH, cudaStream_t stream) {
+                                    const float* alpha, DecGates gt, float* S, void* out, int BH,
+                                    cudaStream_t stream) {
   switch (dv) {
-    case 16: return launch_decode_t<DK, 16, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
-    case 32: return launch_decode_t<DK, 32, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
-    case 64: return launch_decode_t<DK, 64, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
-    case 128: return launch_decode_t<DK, 128, Tin, Tout>(q, k, v, alpha, beta, S, out, BH, stream);
+    case 16: return launch_decode_t<DK, 16, Tin, Tout>(q, k, v, alpha, gt, S, out, BH, stream);
+    case 32: return launch_decode_t<DK, 32, Tin, Tout>(q, k, v, alpha, gt, S, out, BH, stream);
+    case 64: return launch_decode_t<DK, 64, Tin, Tout>(q, k, v, alpha, gt, S, out, BH, stream);
+    case 128: return launch_decode_t<DK, 128, Tin, Tout>(q, k, v, alpha, gt, S, out, BH, stream);
   }
   return cudaErrorInvalidValue;
 }
 
 template <typename Tin, typename Tout>
 static cudaError_t launch_decode_dk(int dk, int dv, const void* q, const void* k, const void* v,
-                                    const float* alpha, const float* beta, float* S, void* out,
-                                    int BH, cudaStream_t stream) {
+                                    const float* alpha, DecGates gt, float* S, void* out, int BH,
+                                    cudaStream_t stream) {
   switch (dk) {
-    case 16: return launch_decode_dv<16, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
-    case 32: return launch_decode_dv<32, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
-    case 64: return launch_decode_dv<64, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
-    case 128: return launch_decode_dv<128, Tin, Tout>(dv, q, k, v, alpha, beta, S, out, BH, stream);
+    case 16: return launch_decode_dv<16, Tin, Tout>(dv, q, k, v, alpha, gt, S, out, BH, stream);
+    case 32: return launch_decode_dv<32, Tin, Tout>(dv, q, k, v, alpha, gt, S, out, BH, stream);
+    case 64: return launch_decode_dv<64, Tin, Tout>(dv, q, k, v, alpha, gt, S, out, BH, stream);
+    case 128: return launch_decode_dv<128, Tin, Tout>(dv, q, k, v, alpha, gt, S, out, BH, stream);
   }
   return cudaErrorInvalidValue;
 }
 
+// bg and wg non-NULL: the Gated DeltaNet-2 form (beta unused); theta
+// non-NULL: the SFDA form (alpha holds d_k / 2 decays).
 cudaError_t launch_decode(int dtype, int out_dtype, int dk, int dv, const void* q, const void* k,
-                          const void* v, const float* alpha, const float* beta, float* S, void* out,
-                          int BH, cudaStream_t stream) {
+                          const void* v, const float* alpha, const float* beta, const float* bg,
+                          const float* wg, const float* theta, float* S, void* out, int BH,
+                          cudaStream_t stream) {
+  const DecGates gt{beta, bg, wg, theta};
   if (dtype == CKDA_BF16) {
     if (out_dtype == CKDA_BF16)
-      return launch_decode_dk<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, alpha, beta, S, out,
+      return launch_decode_dk<__nv_bfloat16, __nv_bfloat16>(dk, dv, q, k, v, alpha, gt, S, out,
                                                             BH, stream);
-    return launch_decode_dk<__nv_bfloat16, float>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
+    return launch_decode_dk<__nv_bfloat16, float>(dk, dv, q, k, v, alpha, gt, S, out, BH, stream);
   }
   if (out_dtype == CKDA_BF16)
-    return launch_decode_dk<float, __nv_bfloat16>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
-  return launch_decode_dk<float, float>(dk, dv, q, k, v, alpha, beta, S, out, BH, stream);
+    return launch_decode_dk<float, __nv_bfloat16>(dk, dv, q, k, v, alpha, gt, S, out, BH, stream);
+  return launch_decode_dk<float, float>(dk, dv, q, k, v, alpha, gt, S, out, BH, stream);
 }
 
 }  // namespace ckda

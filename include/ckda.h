@@ -436,6 +436,31 @@ CKDA_API int ckda_decode_step(const void* q, const void* k, const void* v,
                      void* out, int B, int H, int d_k, int d_v, int dtype,
                      int out_dtype, void* stream);
 
+/*
+ * ckda_gdn2_decode_step -- one recurrent token of the Gated DeltaNet-2
+ * recurrence ("Gated DeltaNet-2", Methodology section 1), in place on the
+ * state: S' = Diag(alpha) S, u = w . v - S'^T (b . k), S = S' + k u^T,
+ * o = S^T q.  b [B, H, d_k] and w [B, H, d_v] fp32 take beta's place; every
+ * other argument and rule is that of ckda_decode_step.
+ */
+CKDA_API int ckda_gdn2_decode_step(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* b, const float* w,
+                                   float* S_inout, void* out, int B, int H, int d_k, int d_v,
+                                   int dtype, int out_dtype, void* stream);
+
+/*
+ * ckda_sfda_decode_step -- one recurrent token of the SFDA recurrence
+ * ("Semidirect Fourier Delta Attention (SFDA)", "Arquitectura Central"), in
+ * place on the state: the gate of ckda_sfda_fwd_chunked (row pairs
+ * (2p, 2p+1) turned by alpha_p (cos theta_p, sin theta_p)), then the delta
+ * update with beta.  alpha and theta are fp32 [B, H, d_k / 2]; every other
+ * argument and rule is that of ckda_decode_step.
+ */
+CKDA_API int ckda_sfda_decode_step(const void* q, const void* k, const void* v,
+                                   const float* alpha, const float* theta, const float* beta,
+                                   float* S_inout, void* out, int B, int H, int d_k, int d_v,
+                                   int dtype, int out_dtype, void* stream);
+
 /* Human-readable text for a CKDA_* status code (static storage). */
 CKDA_API const char* ckda_status_string(int status);
 

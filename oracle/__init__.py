@@ -303,6 +303,30 @@ def backward(q, k, v, alpha, beta, dO, S0=None, dS_final=None, cu_seqlens=None,
     return g
 
 
+def _one_token(x):
+    """[B, H, ...] -> [B, 1, H, ...] (one token per sequence)."""
+    x = _f64(x)
+    return x.reshape(x.shape[0], 1, *x.shape[1:])
+
+
+def decode_step_gdn2(q, k, v, alpha, b, w, S, n_threads=None):
+    """One fp64 Gated DeltaNet-2 step (``forward_gdn2`` on one token per
+    sequence): q, k, alpha, b ``[B, H, dk]``, v, w ``[B, H, dv]``, S
+    ``[B, H, dk, dv]``.  Returns ``(out, S_new)``."""
+    out, Sn = forward_gdn2(*(_one_token(t) for t in (q, k, v, alpha, b, w)), S0=_f64(S),
+                           n_threads=n_threads)
+    return out[:, 0], Sn
+
+
+def decode_step_sfda(q, k, v, alpha, theta, beta, S, n_threads=None):
+    """One fp64 SFDA step (``forward_sfda`` on one token per sequence): q, k
+    ``[B, H, dk]``, v ``[B, H, dv]``, alpha, theta ``[B, H, dk / 2]``, beta
+    ``[B, H]``, S ``[B, H, dk, dv]``.  Returns ``(out, S_new)``."""
+    out, Sn = forward_sfda(*(_one_token(t) for t in (q, k, v, alpha, theta, beta)), S0=_f64(S),
+                           n_threads=n_threads)
+    return out[:, 0], Sn
+
+
 def decode_step(q, k, v, alpha, beta, S, n_threads=None):
     """One fp64 recurrent step: q, k, alpha ``[B, H, dk]``, v ``[B, H, dv]``,
     beta ``[B, H]``, S ``[B, H, dk, dv]``.  Returns ``(out, S_new)``."""

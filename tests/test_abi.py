@@ -343,3 +343,21 @@ def test_scan_entry_validates_without_a_gpu(lib):
     need = lib.ckda_fwd_chunked_scan_workspace_bytes(2, 300, 3, 128, 128, 4)
     assert need == need1 + 2 * 3 * 3 * 128 * 256 * 4 + 2 * 4 * 3 * 128 * 128 * 4
     assert lib.ckda_fwd_chunked_scan_workspace_bytes(2, 300, 3, 128, 128, 0) == -1
+
+
+def test_variant_decode_entries_validate_without_a_gpu(lib):
+    args = (P, P + 0x1000, P + 0x2000, P + 0x3000)
+    # Gated DeltaNet-2: b, w required
+    assert lib.ckda_gdn2_decode_step(*args, None, P + 0x5000, P + 0x6000, P + 0x7000, 1, 1, 16,
+                                     16, 0, 0, None) == -1
+    assert lib.ckda_gdn2_decode_step(*args, P + 0x4000, MIS, P + 0x6000, P + 0x7000, 1, 1, 16,
+                                     16, 0, 0, None) == -3
+    assert lib.ckda_gdn2_decode_step(*args, P + 0x4000, P + 0x5000, P + 0x6000, P + 0x7000, 0, 1,
+                                     16, 16, 0, 0, None) == 0
+    # SFDA: theta required
+    assert lib.ckda_sfda_decode_step(*args, None, P + 0x5000, P + 0x6000, P + 0x7000, 1, 1, 16,
+                                     16, 0, 0, None) == -1
+    assert lib.ckda_sfda_decode_step(*args, P + 0x4000, P + 0x5000, P + 0x6000, P + 0x7000, 1, 1,
+                                     48, 16, 0, 0, None) == -2
+    assert lib.ckda_sfda_decode_step(*args, P + 0x4000, P + 0x5000, P + 0x6000, P + 0x6000, 1, 1,
+                                     16, 16, 0, 0, None) == -1   # out aliases the state
