@@ -674,7 +674,41 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, 
               "achieved_gbs": dgbs, "hbm_frac_of_measured": dgbs / hbm_peak,
               "hbm_frac_of_spec_8tbs": dgbs / SPEC_HBM_GBS,
               "bytes_per_step": dbytes, "gpu_launches": steps}
-    del dc, S
+    # the two gate variants' decode steps on the same tokens and state size,
+    # 64 steps each after 4 warm-up steps
+    vs = min(64, steps)
+    g = torch.Generator(device=dev).manual_seed(2100 + rank)
+    u = lambda *shape: torch.rand(*shape, generator=g, device=dev)  # noqa: E731
+    bvar = {"gdn2": (u(vs + 4, DEC_B, DEC_H, D), u(vs + 4, DEC_B, DEC_H, D)),
+            "sfda": (u(vs + 4, DEC_B, DEC_H, D // 2),
+                     (2 * u(vs + 4, DEC_B, DEC_H, D // 2) - 1) * 3.141592653589793)}
+    # bytes per head-step beyond the state: q, k, v bf16, out fp32, and the gates
+    gate_bytes = {"gdn2": D * 4 + D * 4 + D * 4, "sfda": 2 * (D // 2) * 4 + 4}
+    for kind, (g1, g2) in bvar.items():
+        def one(t):
+            if kind == "gdn2":
+                ck.gdn2_decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], g1[t], g2[t], S,
+                                    out=dout)
+            else:
+                ck.sfda_decode_step(dc.q[t], dc.k[t], dc.v[t], g1[t], g2[t], dc.beta[t], S,
+                                    out=dout)
+        for t in range(4):
+            one(t)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ev0.record(stream)
+        for t in range(4, 4 + vs):
+            one(t)
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ms = max_ranks(ev0.elapsed_time(ev1)) / vs
+        nb = DEC_B * DEC_H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + gate_bytes[kind])
+        decode[kind] = {"ms_per_step": ms, "tokens_per_s": ws * DEC_B / (ms / 1e3),
+                        "achieved_gbs": nb / (ms / 1e3) / 1e9,
+                        "hbm_frac_of_measured": nb / (ms / 1e3) / 1e9 / hbm_peak,
+                        "bytes_per_step": nb, "steps": vs, "gpu_launches": vs}
+    del dc, S, bvar
     return decode
 
 
