@@ -352,10 +352,14 @@ def fwd_chunked_scan(q, k, v, alpha, beta, segments: int, S0=None, chunk: int = 
         out = torch.empty(v.shape, dtype=out_dtype, device=dev)
     else:
         _need(out, "out", out_dtype, dev)
+        if out.shape != v.shape:
+            raise ValueError("out must have v's shape")
     if return_final and S_final is None:
         S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     if S_final is not None:
         _need(S_final, "S_final", torch.float32, dev)
+        if tuple(S_final.shape) != (N, H, dk, dv):
+            raise ValueError(f"S_final must be [{N}, {H}, {dk}, {dv}]")
     if workspace is None:
         workspace = torch.empty(max(1, scan_workspace_bytes(B, T, H, dk, dv, segments)),
                                 dtype=torch.uint8, device=dev)
