@@ -5,7 +5,8 @@ recurrence ("Gated DeltaNet-2" summary, Methodology sections 1 and 3) on the
 fp32 CUDA-core kernel.  The oracle it is compared with is pinned by
 ``pinlib_gdn2`` (G-1..G-7).  Shapes span several chunks with ragged tails,
 every supported head size and chunk size, packed batches with empty
-sequences, and the reduction b = w = beta, which must reproduce the CKDA path.
+sequences, the full-size workload on sampled units, and the reduction
+b = w = beta, which must reproduce the CKDA path.
 """
 import numpy as np
 import pytest
@@ -123,3 +124,18 @@ def test_tensor_core_agrees_with_the_fp32_kernel(ck):
     assert ck.device_status() == 0
     assert rel_max_err(o_tc, o_32.double().cpu().numpy()) <= TOL_BF16
     assert rel_max_err(S_tc, S_32.double().cpu().numpy()) <= TOL_BF16
+
+
+def test_full_size_workload_on_sampled_units(ck):
+    """The bench workload (B=4, T=4096, H=16, d=128, bf16, tensor-core pair),
+    checked on four sampled (sequence, head) units against the oracle."""
+    assert ck.fwd_path(4, 4096, 16, 128, 128, 64, torch.bfloat16, torch.float32) == "tcgen05"
+    c = inputs.gdn2_prefill(4, 4096, 16, 128, 128, dtype=torch.bfloat16, chunk=64, seed=0,
+                            device=DEV)
+    out, S = _run(ck, c)
+    for b, h in [(0, 0), (1, 7), (2, 15), (3, 3)]:
+        sel = lambda x: x[b:b + 1, :, h:h + 1].cpu()  # noqa: E731
+        ro, rS = oracle.forward_gdn2(sel(c.q), sel(c.k), sel(c.v), sel(c.alpha),
+                                     sel(c.extra["b"]), sel(c.extra["w"]))
+        assert rel_max_err(out[b:b + 1, :, h:h + 1], ro) <= TOL_BF16, (b, h)
+        assert rel_max_err(S[b:b + 1, h:h + 1], rS) <= TOL_BF16, (b, h)
