@@ -8,7 +8,8 @@ gates on channel pairs: "Semidirect Fourier Delta Attention (SFDA)" summary,
 state.  They are compared step by step with the pinned fp64 oracles
 (``forward_gdn2`` / ``forward_sfda`` on one token per sequence), with their
 reductions to the CKDA step (b = w = beta; theta = 0), and with the chunked
-forward over the same tokens.
+forward over the same tokens; at the decode workload's size on sampled
+(sequence, head) units.
 """
 import math
 
@@ -124,3 +125,26 @@ def test_steps_equal_the_chunked_forward(ck, kind):
     assert ck.device_status() == 0
     assert rel_max_err(o_dec, o_fwd.double().cpu().numpy()) <= 1e-5
     assert rel_max_err(S, S_fwd.double().cpu().numpy()) <= 1e-5
+
+
+@pytest.mark.parametrize("kind", ["gdn2", "sfda"])
+def test_bench_size_steps_sampled(ck, kind):
+    """The decode workload's size (B=256, H=32, d=128, bf16 q/k/v, fp32 out):
+    64 steps of every head, checked on sampled (sequence, head) units against
+    the oracle run over the same 64 tokens."""
+    steps, B, H, d = 64, 256, 32, 128
+    q, k, v, gates, S0 = _inputs(B, H, d, d, steps, torch.bfloat16, 77, kind)
+    S = S0.clone()
+    outs = torch.stack([_run(ck, kind, q, k, v, gates, S, t) for t in range(steps)])
+    assert ck.device_status() == 0
+    b_idx = torch.tensor([0, 17, 128, 255], device=DEV)
+    h_idx = torch.tensor([0, 9, 31], device=DEV)
+
+    def sel(x):  # [steps, B, H, ...] -> [B', steps, H', ...] on the host
+        return x[:, b_idx][:, :, h_idx].transpose(0, 1).cpu()
+
+    f = oracle.forward_gdn2 if kind == "gdn2" else oracle.forward_sfda
+    ro, rS = f(sel(q), sel(k), sel(v), *(sel(g) for g in gates), S0=S0[b_idx][:, h_idx].cpu())
+    eo = rel_max_err(sel(outs), ro)
+    es = rel_max_err(S[b_idx][:, h_idx], rS)
+    assert eo <= TOL_BF16 and es <= TOL_BF16, (eo, es)
