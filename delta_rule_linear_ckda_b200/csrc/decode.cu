@@ -12,8 +12,8 @@
 // uses e = b . k and u = w . v - r (no beta).  SFDA ("Semidirect Fourier Delta
 // Attention (SFDA)" page, "Arquitectura Central"): S' = Lambda S, each pair of
 // rows (2p, 2p+1) turned by alpha_p (cos theta_p, sin theta_p); a thread then
-// holds whole row pairs, and the pairs' (cos, sin) are computed once per
-// (b, h) into shared memory.
+// holds whole row pairs, and each pair's (cos, sin) is computed once per row
+// group and passed to the group's lanes by warp shuffles.
 //
 // The step moves 2 * d_k * d_v * 4 bytes of state per head and does ~6
 // flops per state element: it is bound by HBM bandwidth.  Each CTA owns
@@ -21,7 +21,10 @@
 // d_k * d_v / (4 * blockDim) rows, held in registers between the read and
 // the write.  Column reductions over d_k combine register partials through
 // shared memory.  State traffic uses streaming cache hints (each element is
-// touched once per step).
+// touched once per step).  Every global load of the step (state, q, k, v and
+// the gates) comes before the one block barrier (the column reduction),
+// across which the compiler does not move loads: a CTA waits for one DRAM
+// round trip, not one per barrier.
 #include "common.cuh"
 
 namespace ckda {
@@ -40,6 +43,9 @@ struct DecodeShape {
   static_assert(kThreads % 32 == 0 || kThreads < 32, "block size");
   static_assert(DK % kRpp == 0, "row split");
   static_assert(!SF || kRows % 2 == 0, "row pairs");
+  // SFDA: a row group's pairs are evaluated by its own lanes (one each) and
+  // a group lies within one warp
+  static_assert(!SF || (kRows / 2 <= kCpr && 32 % kCpr == 0 && kThreads % 32 == 0), "pair lanes");
 };
 
 // bg, wg: the Gated DeltaNet-2 gates ([BH, d_k], [BH, d_v]); theta: the SFDA
@@ -57,7 +63,6 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   __shared__ float4 red_r[RPP][CPR];
   __shared__ float4 red_p[RPP][CPR];
   __shared__ float kq_part[(NT + 31) / 32];
-  __shared__ float2 lam[SF ? DK / 2 : 1];
 
   const int bh = blockIdx.x;
   const int t = threadIdx.x;
@@ -73,25 +78,36 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   float4 s[NR];
 #pragma unroll
   for (int m = 0; m < NR; ++m) s[m] = __ldcs(Sb + (size_t)row_of(m) * CPR + c);
-  if constexpr (SF) {
-    // the pairs' rotation-decay gates, once per (b, h)
-    for (int pp = t; pp < DK / 2; pp += NT) {
-      float sn, cs;
-      sincosf(__ldg(theta + (size_t)bh * (DK / 2) + pp), &sn, &cs);
-      const float a = __ldg(alpha + (size_t)bh * (DK / 2) + pp);
-      lam[pp] = make_float2(a * cs, a * sn);
-    }
-    __syncthreads();
-  }
+  // this thread's v columns and write-side gate (read after the reduction)
+  const float4 vv = load4_f32(v + (size_t)bh * DV + 4 * c);
+  float4 ww = make_float4(0.f, 0.f, 0.f, 0.f);
+  float bt = 0.f;
+  if constexpr (G2)
+    ww = *reinterpret_cast<const float4*>(wg + (size_t)bh * DV + 4 * c);
+  else
+    bt = __ldg(beta + bh);
   float kr[NR];
   float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
   if constexpr (SF) {
+    // The pairs' rotation-decay gates: the thread at column j < NR / 2 of a
+    // row group evaluates pair g + RPP j (rows 2 (g + RPP j) and the next),
+    // which every thread of the group holds; a group is CPR consecutive
+    // lanes of one warp, so the others read the value by a shuffle.
+    float2 mine = make_float2(0.f, 0.f);
+    if (c < NR / 2) {
+      const int pp = g + RPP * c;
+      float sn, cs;
+      sincosf(__ldg(theta + (size_t)bh * (DK / 2) + pp), &sn, &cs);
+      const float a = __ldg(alpha + (size_t)bh * (DK / 2) + pp);
+      mine = make_float2(a * cs, a * sn);
+    }
+    const int lane0 = (t & 31) & ~(CPR - 1);
     // S' = Lambda S on every row pair, then the column sums
 #pragma unroll
     for (int m = 0; m < NR; m += 2) {
-      const int i = row_of(m);  // rows (i, i + 1) = (real, imaginary) of pair i / 2
-      const float2 l = lam[i >> 1];
+      const float2 l = make_float2(__shfl_sync(0xffffffffu, mine.x, lane0 + (m >> 1)),
+                                   __shfl_sync(0xffffffffu, mine.y, lane0 + (m >> 1)));
       const float4 e = s[m], o = s[m + 1];
       s[m] = make_float4(fmaf(-l.y, o.x, l.x * e.x), fmaf(-l.y, o.y, l.x * e.y),
                          fmaf(-l.y, o.z, l.x * e.z), fmaf(-l.y, o.w, l.x * e.w));
@@ -138,15 +154,12 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 #pragma unroll
   for (int w = 0; w < (NT + 31) / 32; ++w) kqt += kq_part[w];
 
-  const float4 vv = load4_f32(v + (size_t)bh * DV + 4 * c);
   float4 u;
   if constexpr (G2) {
     // u = w . v - r
-    const float4 ww = *reinterpret_cast<const float4*>(wg + (size_t)bh * DV + 4 * c);
     u.x = fmaf(ww.x, vv.x, -R.x); u.y = fmaf(ww.y, vv.y, -R.y);
     u.z = fmaf(ww.z, vv.z, -R.z); u.w = fmaf(ww.w, vv.w, -R.w);
   } else {
-    const float bt = __ldg(beta + bh);
     u.x = bt * (vv.x - R.x); u.y = bt * (vv.y - R.y);
     u.z = bt * (vv.z - R.z); u.w = bt * (vv.w - R.w);
   }
