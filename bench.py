@@ -127,7 +127,14 @@ def _emit(obj, args, rank):
 # ---------------------------------------------------------------- clocks ---
 
 class ClockSampler:
-    """Samples SM clock and throttle reasons with nvidia-smi while running."""
+    """Samples SM clock and throttle reasons with nvidia-smi while running.
+
+    ``start`` returns once the first sample has been written (nvidia-smi can
+    take a second to come up), ``mark`` notes where the timed region begins,
+    and ``stop`` reports the samples taken from that mark on.  ``count``
+    gives how many there are so far, so that a timed region too short for
+    several samples can be followed by untimed repetitions of the same work
+    until there are enough (``soak_steps`` in the record)."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -137,6 +144,22 @@ class ClockSampler:
         self.gpu_id = gpu_id
         self.proc = None
         self.tmp = None
+        self.first = 0
+        self.soak_steps = 0
+
+    def _lines(self):
+        try:
+            with open(self.tmp.name) as f:
+                return [ln for ln in f.read().splitlines() if ln.count(",") >= 7]
+        except OSError:
+            return []
+
+    def count(self) -> int:
+        return max(0, len(self._lines()) - self.first) if self.proc is not None else 0
+
+    def mark(self):
+        if self.proc is not None:
+            self.first = len(self._lines())
 
     def start(self):
         try:
@@ -147,6 +170,10 @@ class ClockSampler:
                 stdout=self.tmp, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return self
+        t0 = time.perf_counter()
+        while not self._lines() and time.perf_counter() - t0 < 10.0 and self.proc.poll() is None:
+            time.sleep(0.05)
         return self
 
     def stop(self):
@@ -158,10 +185,10 @@ class ClockSampler:
         except Exception:
             self.proc.kill()
         self.tmp.flush()
-        self.tmp.seek(0)
+        lines = self._lines()[self.first:]
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.tmp.read().splitlines():
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
                 continue
@@ -176,7 +203,8 @@ class ClockSampler:
         os.unlink(self.tmp.name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "reasons": sorted(reasons),
+                "soak_steps": self.soak_steps}
 
 
 # ------------------------------------------------------------ reference ---
@@ -349,7 +377,6 @@ def run_ours(args, ws, rank, local):
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id).start() if rank == 0 else None
-    time.sleep(0.3 if rank == 0 else 0.0)
 
     K = args.steps
     ev0 = torch.cuda.Event(enable_timing=True)
@@ -359,6 +386,8 @@ def run_ours(args, ws, rank, local):
     ke = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     barrier()
     torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.mark()
     wall0 = time.perf_counter()
     ev0.record(stream)
     for i in range(K):
@@ -369,6 +398,16 @@ def run_ours(args, ws, rank, local):
     torch.cuda.synchronize(dev)
     barrier()
     wall = time.perf_counter() - wall0
+    if sampler:
+        # a region too short for 5 samples: the same steps again, untimed,
+        # until the sampler has seen 5 (at most 3 s)
+        t_soak = time.perf_counter()
+        while (sampler.count() < 5 and sampler.proc is not None
+               and time.perf_counter() - t_soak < 3.0):
+            for j in range(8):
+                step(j)
+            sampler.soak_steps += 8
+            torch.cuda.synchronize(dev)
     clocks = sampler.stop() if sampler else None
     elapsed_ms = max_ranks(ev0.elapsed_time(ev1))
     kern_ms = statistics.mean(ks[i].elapsed_time(ke[i]) for i in range(K))
@@ -649,28 +688,60 @@ def _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_p
 
 
 def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak):
+    """Decode steps through the public API, timed twice over the same steps:
+    eagerly (one Python call per step, as a plain loop issues them) and as a
+    CUDA graph of those calls replayed once (the kernels back to back, as a
+    serving loop under graphs runs them).  ``ms_per_step`` is the graph
+    figure; ``ms_per_step_eager`` the eager one."""
     steps = max(1, args.decode_steps)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     dc = inputs.decode(seed=2000 + rank, device=dev, B=DEC_B, H=DEC_H, d=D, steps=steps + 8)
     S = dc.S0.clone()
     dout = torch.empty((DEC_B, DEC_H, D), dtype=torch.float32, device=dev)
+
+    def timed(issue, n):
+        torch.cuda.synchronize(dev)
+        barrier()
+        ev0.record(stream)
+        issue()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        eager = max_ranks(ev0.elapsed_time(ev1)) / n
+        gr = torch.cuda.CUDAGraph()
+        try:
+            with torch.cuda.graph(gr):
+                issue()
+            ok = 1.0
+        except Exception:
+            ok = 0.0
+        torch.cuda.synchronize(dev)
+        ok = -max_ranks(-ok)  # every rank's capture succeeded
+        barrier()
+        ev0.record(stream)
+        if ok:
+            gr.replay()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        graph = max_ranks(ev0.elapsed_time(ev1)) / n
+        del gr
+        return (graph if ok else eager), eager, ("cuda_graph" if ok else "eager")
+
+    def kda_steps():
+        for t in range(8, 8 + steps):
+            ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
+
     for t in range(8):
         ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
-    torch.cuda.synchronize(dev)
-    barrier()
-    ev0.record(stream)
-    for t in range(8, 8 + steps):
-        ck.decode_step(dc.q[t], dc.k[t], dc.v[t], dc.alpha[t], dc.beta[t], S, out=dout)
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    dec_ms = max_ranks(ev0.elapsed_time(ev1)) / steps
+    dec_ms, dec_eager, how = timed(kda_steps, steps)
     dbytes = DEC_B * DEC_H * DEC_BYTES_PER_HEAD_STEP
     dgbs = dbytes / (dec_ms / 1e3) / 1e9
     decode = {"workload": f"decode B={DEC_B} H={DEC_H} d={D} bf16 q/k/v, fp32 out, "
                           f"{steps} steps",
-              "ms_per_step": dec_ms, "tokens_per_s": ws * DEC_B / (dec_ms / 1e3),
+              "ms_per_step": dec_ms, "ms_per_step_eager": dec_eager, "timing": how,
+              "tokens_per_s": ws * DEC_B / (dec_ms / 1e3),
               "achieved_gbs": dgbs, "hbm_frac_of_measured": dgbs / hbm_peak,
               "hbm_frac_of_spec_8tbs": dgbs / SPEC_HBM_GBS,
               "bytes_per_step": dbytes, "gpu_launches": steps}
@@ -692,19 +763,16 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, 
             else:
                 ck.sfda_decode_step(dc.q[t], dc.k[t], dc.v[t], g1[t], g2[t], dc.beta[t], S,
                                     out=dout)
+
+        def var_steps():
+            for t in range(4, 4 + vs):
+                one(t)
         for t in range(4):
             one(t)
-        torch.cuda.synchronize(dev)
-        barrier()
-        ev0.record(stream)
-        for t in range(4, 4 + vs):
-            one(t)
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        ms = max_ranks(ev0.elapsed_time(ev1)) / vs
+        ms, eager, how = timed(var_steps, vs)
         nb = DEC_B * DEC_H * (2 * D * D * 4 + 3 * D * 2 + D * 4 + gate_bytes[kind])
-        decode[kind] = {"ms_per_step": ms, "tokens_per_s": ws * DEC_B / (ms / 1e3),
+        decode[kind] = {"ms_per_step": ms, "ms_per_step_eager": eager, "timing": how,
+                        "tokens_per_s": ws * DEC_B / (ms / 1e3),
                         "achieved_gbs": nb / (ms / 1e3) / 1e9,
                         "hbm_frac_of_measured": nb / (ms / 1e3) / 1e9 / hbm_peak,
                         "bytes_per_step": nb, "steps": vs, "gpu_launches": vs}

@@ -21,10 +21,12 @@
 // d_k * d_v / (4 * blockDim) rows, held in registers between the read and
 // the write.  Column reductions over d_k combine register partials through
 // shared memory.  State traffic uses streaming cache hints (each element is
-// touched once per step).  Every global load of the step (state, q, k, v and
-// the gates) comes before the one block barrier (the column reduction),
-// across which the compiler does not move loads: a CTA waits for one DRAM
-// round trip, not one per barrier.
+// touched once per step).  The per-row vectors (k, q, the decay or the
+// erase gate: one value per state row, shared by all the threads of a row)
+// are requested first, one entry per thread, and staged in shared memory;
+// then the state; then v and the write-side gate.  Every global load thus
+// precedes the block barriers, which the compiler does not move loads
+// across: a CTA waits for one DRAM round trip, not one per barrier.
 #include "common.cuh"
 
 namespace ckda {
@@ -43,6 +45,8 @@ struct DecodeShape {
   static_assert(kThreads % 32 == 0 || kThreads < 32, "block size");
   static_assert(DK % kRpp == 0, "row split");
   static_assert(!SF || kRows % 2 == 0, "row pairs");
+  // the per-row vectors take one entry per thread
+  static_assert(kThreads >= DK, "vector staging");
   // SFDA: a row group's pairs are evaluated by its own lanes (one each) and
   // a group lies within one warp
   static_assert(!SF || (kRows / 2 <= kCpr && 32 % kCpr == 0 && kThreads % 32 == 0), "pair lanes");
@@ -63,6 +67,9 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   __shared__ float4 red_r[RPP][CPR];
   __shared__ float4 red_p[RPP][CPR];
   __shared__ float kq_part[(NT + 31) / 32];
+  // the per-row vectors: k, q, the decay (not SFDA) and the erase direction
+  // b . k (GDN-2)
+  __shared__ float vk[DK], vq[DK], va[SF ? 1 : DK], vb[G2 ? DK : 1];
 
   const int bh = blockIdx.x;
   const int t = threadIdx.x;
@@ -74,10 +81,33 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   // both rows of a pair are held by the same thread)
   auto row_of = [&](int m) -> int { return SF ? 2 * (g + RPP * (m >> 1)) + (m & 1) : g + RPP * m; };
 
-  // Issue every state load first (16 bytes each, streaming).
+  // SFDA: the phase and decay of the pair this thread evaluates (below),
+  // requested before the state so that they arrive first
+  float th_in = 0.f, al_in = 0.f;
+  if constexpr (SF) {
+    if (c < NR / 2) {
+      th_in = __ldg(theta + (size_t)bh * (DK / 2) + g + RPP * c);
+      al_in = __ldg(alpha + (size_t)bh * (DK / 2) + g + RPP * c);
+    }
+  }
+  // the per-row vectors, one entry per thread t < d_k (blockDim >= d_k)
+  float lk = 0.f, lq = 0.f, la = 0.f, lb = 0.f;
+  if (t < DK) {
+    lk = Elem<Tin>::to_f32(k[kvec + t]);
+    lq = Elem<Tin>::to_f32(q[kvec + t]);
+    if constexpr (!SF) la = __ldg(alpha + kvec + t);
+    if constexpr (G2) lb = __ldg(bg + kvec + t);
+  }
+  // Then every state load (16 bytes each, streaming).
   float4 s[NR];
 #pragma unroll
   for (int m = 0; m < NR; ++m) s[m] = __ldcs(Sb + (size_t)row_of(m) * CPR + c);
+  if (t < DK) {
+    vk[t] = lk;
+    vq[t] = lq;
+    if constexpr (!SF) va[t] = la;
+    if constexpr (G2) vb[t] = lk * lb;
+  }
   // this thread's v columns and write-side gate (read after the reduction)
   const float4 vv = load4_f32(v + (size_t)bh * DV + 4 * c);
   float4 ww = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -86,7 +116,7 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     ww = *reinterpret_cast<const float4*>(wg + (size_t)bh * DV + 4 * c);
   else
     bt = __ldg(beta + bh);
-  float kr[NR];
+  __syncthreads();
   float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
   float4 p = make_float4(0.f, 0.f, 0.f, 0.f);
   if constexpr (SF) {
@@ -96,11 +126,9 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
     // lanes of one warp, so the others read the value by a shuffle.
     float2 mine = make_float2(0.f, 0.f);
     if (c < NR / 2) {
-      const int pp = g + RPP * c;
       float sn, cs;
-      sincosf(__ldg(theta + (size_t)bh * (DK / 2) + pp), &sn, &cs);
-      const float a = __ldg(alpha + (size_t)bh * (DK / 2) + pp);
-      mine = make_float2(a * cs, a * sn);
+      sincosf(th_in, &sn, &cs);
+      mine = make_float2(al_in * cs, al_in * sn);
     }
     const int lane0 = (t & 31) & ~(CPR - 1);
     // S' = Lambda S on every row pair, then the column sums
@@ -118,14 +146,13 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
 #pragma unroll
   for (int m = 0; m < NR; ++m) {
     const int i = row_of(m);
-    const float kk = Elem<Tin>::to_f32(k[kvec + i]);
-    const float qq = Elem<Tin>::to_f32(q[kvec + i]);
-    kr[m] = kk;
+    const float kk = vk[i];
+    const float qq = vq[i];
     if constexpr (!SF) {
-      const float a = __ldg(alpha + kvec + i);
+      const float a = va[i];
       s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;
     }
-    const float ek = G2 ? kk * __ldg(bg + kvec + i) : kk;  // the read direction
+    const float ek = G2 ? vb[i] : kk;  // the read direction
     r.x = fmaf(s[m].x, ek, r.x); r.y = fmaf(s[m].y, ek, r.y);
     r.z = fmaf(s[m].z, ek, r.z); r.w = fmaf(s[m].w, ek, r.w);
     p.x = fmaf(s[m].x, qq, p.x); p.y = fmaf(s[m].y, qq, p.y);
@@ -135,9 +162,7 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   red_p[g][c] = p;
 
   // k . q over d_k: one partial per warp, summed below.
-  float kq = 0.f;
-  for (int i = t; i < DK; i += NT)
-    kq = fmaf(Elem<Tin>::to_f32(k[kvec + i]), Elem<Tin>::to_f32(q[kvec + i]), kq);
+  float kq = lk * lq;
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
   if ((t & 31) == 0) kq_part[t >> 5] = kq;
@@ -173,8 +198,9 @@ decode_step_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k,
   for (int m = 0; m < NR; ++m) {
     const int i = row_of(m);
     float4 o = s[m];
-    o.x = fmaf(kr[m], u.x, o.x); o.y = fmaf(kr[m], u.y, o.y);
-    o.z = fmaf(kr[m], u.z, o.z); o.w = fmaf(kr[m], u.w, o.w);
+    const float kk = vk[i];
+    o.x = fmaf(kk, u.x, o.x); o.y = fmaf(kk, u.y, o.y);
+    o.z = fmaf(kk, u.z, o.z); o.w = fmaf(kk, u.w, o.w);
     __stcs(Sb + (size_t)i * CPR + c, o);
   }
 }
