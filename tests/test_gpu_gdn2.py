@@ -51,7 +51,7 @@ def test_bf16_inputs_match_oracle(ck):
     ro, rS = oracle.forward_gdn2(c.q, c.k, c.v, c.alpha, c.extra["b"], c.extra["w"], S0=c.S0)
     assert rel_max_err(out, ro) <= TOL_BF16 and rel_max_err(S, rS) <= TOL_BF16
     # a bf16 output is exactly the bf16 rounding of the fp32 result (parity is
-    # judged on the fp32 output: the rounding alone can exceed the tolerance)
+    # checked on the fp32 output: the rounding alone can exceed the tolerance)
     o16, _ = _run(ck, c, out_dtype=torch.bfloat16)
     assert torch.equal(o16, out.to(torch.bfloat16))
 
