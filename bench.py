@@ -37,8 +37,15 @@ if ROOT not in sys.path:
 B, T, H, D, CHUNK = 4, 4096, 16, 128, 64
 DEC_B, DEC_H, DEC_STEPS = 256, 32, 1024
 
-# algorithmic counts per token-head (d = 128, C = 64)
-BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4          # q,k,v bf16 + alpha + beta + out fp32
+# algorithmic counts per token-head (d = 128, C = 64).  The scope table's
+# figure counts o in the input precision (bf16): q, k, v, o bf16 + alpha fp32 +
+# beta fp32 = 1540 B.  The bench stores o in fp32 (the precision the parity
+# bounds are checked at), which moves 256 B more per token-head: both are
+# reported, the first as the roofline's `achieved`.
+BYTES_PER_TOKEN_HEAD = 4 * D * 2 + D * 4 + 4                  # 1540: q,k,v,o bf16 + alpha + beta
+BYTES_PER_TOKEN_HEAD_F32_OUT = 3 * D * 2 + D * 4 + 4 + D * 4  # 1796: o in fp32
+# gate-extreme packed workload (fp32 q, k, v, alpha, out; beta)
+VARLEN_BYTES_PER_TOKEN_HEAD = 4 * D * 4 + 4 + D * 4           # 2564
 STRICT_FLOPS_PER_TOKEN_HEAD = 6 * CHUNK * D + 6 * D * D + CHUNK * CHUNK // 3
 DENSE_FLOPS_PER_TOKEN_HEAD = 12 * CHUNK * D + 6 * D * D
 DEC_BYTES_PER_HEAD_STEP = 2 * D * D * 4 + 3 * D * 2 + D * 4 + 4 + D * 4
@@ -80,6 +87,10 @@ def _args():
                     help="skip the SFDA (phase-decay gates) sub-measure")
     ap.add_argument("--no-gdn2", action="store_true",
                     help="skip the Gated DeltaNet-2 forward measurement")
+    ap.add_argument("--no-tiny", action="store_true",
+                    help="skip the tiny fp32 workload's latency sub-measure")
+    ap.add_argument("--no-varlen", action="store_true",
+                    help="skip the gate-extreme packed fp32 workload's sub-measure")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -425,9 +436,11 @@ def run_ours(args, ws, rank, local):
 
     token_heads = B * T * H
     alg_bytes = token_heads * BYTES_PER_TOKEN_HEAD + B * H * D * D * 4
+    alg_bytes_f32_out = token_heads * BYTES_PER_TOKEN_HEAD_F32_OUT + B * H * D * D * 4
     strict_flops = token_heads * STRICT_FLOPS_PER_TOKEN_HEAD
     dense_flops = token_heads * DENSE_FLOPS_PER_TOKEN_HEAD
     achieved_gbs = alg_bytes / (kern_ms / 1e3) / 1e9
+    achieved_gbs_f32_out = alg_bytes_f32_out / (kern_ms / 1e3) / 1e9
     tflops_strict = strict_flops / (kern_ms / 1e3) / 1e12
     tflops_dense = dense_flops / (kern_ms / 1e3) / 1e12
     traffic, _ = _traffic_from_profile()
@@ -443,9 +456,18 @@ def run_ours(args, ws, rank, local):
     if not args.no_decode:
         decode = _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks,
                              ws, hbm_peak)
+    # ---- the two fp32 workloads: tiny (latency) and gate-extreme varlen --
+    if not args.no_tiny:
+        variants["tiny"] = _run_tiny(ck, torch, inputs, rank, dev, stream, barrier, max_ranks)
+    if not args.no_varlen:
+        variants["varlen"] = _run_varlen(ck, torch, inputs, rank, dev, stream, barrier,
+                                         max_ranks, ws, hbm_peak)
+    extra_roof = {"achieved_fp32_out_bytes": achieved_gbs_f32_out,
+                  "frac_fp32_out_bytes": achieved_gbs_f32_out / hbm_peak,
+                  "algorithmic_bytes_fp32_out": alg_bytes_f32_out}
     _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            _lib.LIB_PATH, path, kernels, variants)
+            _lib.LIB_PATH, path, kernels, variants, extra_roof)
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -633,15 +655,105 @@ def _run_long(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
         del wss
     th = Bl * Tl * Hl
     nbytes = th * BYTES_PER_TOKEN_HEAD + 2 * Bl * Hl * D * D * 4  # + S0 read, S_final written
+    nbytes32 = th * BYTES_PER_TOKEN_HEAD_F32_OUT + 2 * Bl * Hl * D * D * 4
     return {"workload": f"long_prefill B={Bl} H={Hl} T={Tl} d={D} C={CHUNK} bf16 q/k/v, fp32 "
                         "gates and out, S0 read, S_final stored (tcgen05 kernels)",
             "ms_per_step": ms, "tokens_per_s": ws * Bl * Tl / (ms / 1e3),
+            "achieved_gbs_fp32_out_bytes": nbytes32 / (ms / 1e3) / 1e9,
             "kernels": {"factor_kernel_ms": f_ms, "carry_kernel_ms": c_ms,
                         "carry_ctas": 2 * Hl * Bl},
             "chunk_parallel_scan": scan,
             "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
             "hbm_frac_of_measured": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
             "gpu_launches": 2 * steps}
+
+
+def _run_tiny(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, calls=200):
+    """Latency of the tiny fp32 workload (B=1, H=2, T=64, d=16, C=16): one
+    forward call per step, timed eagerly through the Python API and replayed
+    from a CUDA graph of the same calls."""
+    c = inputs.tiny(seed=rank, device=dev)
+    out = torch.empty(c.v.shape, dtype=torch.float32, device=dev)
+    S_final = torch.empty((1, 2, 16, 16), dtype=torch.float32, device=dev)
+
+    def call():
+        ck.fwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, chunk=c.chunk, out=out, S_final=S_final)
+
+    for _ in range(5):
+        call()
+    torch.cuda.synchronize(dev)
+    assert ck.device_status(dev) == 0
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(calls):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    eager_us = 1e3 * max_ranks(e0.elapsed_time(e1)) / calls
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        for _ in range(calls):
+            call()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0.record(stream)
+    gr.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    graph_us = 1e3 * max_ranks(e0.elapsed_time(e1)) / calls
+    del gr
+    return {"workload": "tiny B=1 H=2 T=64 d=16 C=16 fp32 (alpha ~ U[-1,1], beta ~ U[0,2])",
+            "kernel": ck.fwd_path(1, 64, 2, 16, 16, 16, torch.float32, torch.float32),
+            "us_per_call_eager": eager_us, "us_per_call_graph": graph_us,
+            "tokens_per_s_graph": 64 / (graph_us / 1e6), "bound": "launch latency",
+            "gpu_launches_per_call": 1}
+
+
+def _run_varlen(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak,
+                steps=10):
+    """The gate-extreme packed workload (64 sequences, L ~ U[128, 4096], H=16,
+    d=128, fp32 q/k/v; near-zero gates then orthogonal transitions; S0 = 0,
+    S_final stored): ms per forward and GB/s of its algorithmic bytes (2564
+    B per token-head plus S_final), inputs larger than L2."""
+    c = inputs.varlen(seed=rank, device=dev)
+    Tt = c.q.shape[1]
+    N = c.n_seqs
+    out = torch.empty(c.v.shape, dtype=torch.float32, device=dev)
+    S_final = torch.empty((N, H, D, D), dtype=torch.float32, device=dev)
+
+    def call():
+        ck.fwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, cu_seqlens=c.cu_seqlens, chunk=CHUNK,
+                       out=out, S_final=S_final)
+
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize(dev)
+    assert ck.device_status(dev) == 0
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_ranks(e0.elapsed_time(e1)) / steps
+    nbytes = Tt * H * VARLEN_BYTES_PER_TOKEN_HEAD + N * H * D * D * 4
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"varlen N={N} L~U[128,4096] (T_total={Tt}) H={H} d={D} C={CHUNK} fp32, "
+                        "gate extremes, S0=0, S_final stored",
+            "kernel": ck.fwd_path(N, Tt, H, D, D, CHUNK, torch.float32, torch.float32,
+                                  varlen=True),
+            "ms_per_step": ms, "tokens_per_s": ws * Tt / (ms / 1e3),
+            "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
+            "hbm_frac_of_measured": gbs / hbm_peak,
+            "hbm_floor_ms_at_measured": nbytes / (hbm_peak * 1e9) * 1e3,
+            "steps": steps, "gpu_launches": steps}
 
 
 def _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=5):
@@ -782,10 +894,11 @@ def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, 
 
 def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_peak, traffic,
             peak_src, kern_ms, tflops_strict, tflops_dense, tc_peak, e2e, clocks, wall, decode,
-            lib_path, path, kernels=None, variants=None):
-    # arithmetic of the forward: tcgen05 MMAs on fp16 operands with fp32
+            lib_path, path, kernels=None, variants=None, extra_roof=None):
+    # `dtype` names the workload's input precision (bf16 q/k/v); the
+    # arithmetic is in `compute`: tcgen05 MMAs on fp16 operands with fp32
     # accumulation and fp32 state, or fp32 FFMA on CUDA cores
-    dtype = "f16" if path == "tcgen05" else "f32"
+    dtype = "bf16"
     obj = {
         "metric": "CKDA fwd tokens/s (KDA-layer prefill T=4096, H=16, d=128)",
         "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
@@ -802,8 +915,12 @@ def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_
                      "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                      "peak_source": f"{peak_src} hbm_gbs (burst copy)",
                      "algorithmic_bytes_per_launch": alg_bytes, "kernel_ms": kern_ms,
+                     "bytes_per_token_head": BYTES_PER_TOKEN_HEAD,
                      "scope": "the chunked forward: factor kernel + carry kernel, one pair per "
-                              "step; bytes are the forward's algorithmic bytes"},
+                              "step; bytes are the scope table's algorithmic bytes (q, k, v, o "
+                              "bf16, alpha, beta fp32, S_final); the fp32-output accounting "
+                              "(the output the bench actually stores) is beside it",
+                     **(extra_roof or {})},
         "kernels": kernels,
         "tensor": {"strict_tflops": tflops_strict, "dense_block_tflops": tflops_dense,
                    "frac_strict_of_measured": tflops_strict / tc_peak,

@@ -255,3 +255,56 @@ def first_halves(case: PrefillCase) -> PrefillCase:
                       cu_h.to(torch.int32).to(case.q.device), case.chunk)
     sub.extra["lengths"] = halves
     return sub
+
+
+def gate_extremes(B, T, H, d, *, kind, dtype=BF16, s0_std=0.0, chunk=64, seed=0,
+                  device="cpu") -> PrefillCase:
+    """Fixed-length batch whose gates sit at the ends of the CKDA ranges
+    (alpha in [-1, 1], beta in [0, 2]); q, k ~ N(0,1) normalised, v ~ N(0,1).
+
+    kind="zero":       alpha = 0 everywhere, beta ~ U[0, 2]
+    kind="orthogonal": alpha_i = +-1 uniformly, beta = 2, v = 0
+    kind="reflect":    alpha_i = +-1 uniformly, beta = 2, v ~ N(0,1)
+    kind="uniform":    alpha ~ U[-1, 1], beta ~ U[0, 2]
+    kind="tiny":       alpha ~ U[-0.05, 0.05], beta ~ U[0, 2]
+    kind="underflow":  per (token, head) with probability 0.15 alpha ~ U[-1e-3, 1e-3]
+                       per channel, else alpha = +-U[0.9, 1]; beta ~ U[0, 2]
+    kind="halves":     the first floor(T/2) tokens as "tiny", the rest as "orthogonal"
+
+    Draw order: q, k, v, a uniform tensor, a sign tensor, a selector, beta, S0.
+    """
+    g = _gen(device, seed)
+    q = _l2n(_normal((B, T, H, d), g, device)).to(dtype)
+    k = _l2n(_normal((B, T, H, d), g, device)).to(dtype)
+    v = _normal((B, T, H, d), g, device)
+    u = _uniform((B, T, H, d), 0.0, 1.0, g, device)
+    sgn = torch.where(torch.rand((B, T, H, d), generator=g, device=device) < 0.5, -1.0, 1.0)
+    sel = torch.rand((B, T, H, 1), generator=g, device=device)
+    bu = _uniform((B, T, H), 0.0, 2.0, g, device)
+    two = torch.full_like(bu, 2.0)
+    if kind == "zero":
+        alpha, beta = torch.zeros_like(u), bu
+    elif kind in ("orthogonal", "reflect"):
+        alpha, beta = sgn, two
+        if kind == "orthogonal":
+            v = torch.zeros_like(v)
+    elif kind == "uniform":
+        alpha, beta = 2.0 * u - 1.0, bu
+    elif kind == "tiny":
+        alpha, beta = 0.1 * u - 0.05, bu
+    elif kind == "underflow":
+        alpha = torch.where(sel < 0.15, 2e-3 * u - 1e-3, sgn * (0.9 + 0.1 * u))
+        beta = bu
+    elif kind == "halves":
+        first = (torch.arange(T, device=device) < T // 2).view(1, T, 1)
+        alpha = torch.where(first.unsqueeze(-1), 0.1 * u - 0.05, sgn)
+        beta = torch.where(first, bu, two)
+        v = torch.where(first.unsqueeze(-1), v, torch.zeros_like(v))
+    else:
+        raise ValueError(kind)
+    S0 = None
+    if s0_std > 0:
+        S0 = (_normal((B, H, d, d), g, device) * s0_std).contiguous()
+    return PrefillCase(f"gate_extremes[{kind}] B={B} T={T} H={H} d={d} C={chunk}",
+                       q.contiguous(), k.contiguous(), v.to(dtype).contiguous(),
+                       alpha.to(F32).contiguous(), beta.to(F32).contiguous(), S0, None, chunk)
