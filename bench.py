@@ -91,6 +91,9 @@ def _args():
                     help="skip the tiny fp32 workload's latency sub-measure")
     ap.add_argument("--no-varlen", action="store_true",
                     help="skip the gate-extreme packed fp32 workload's sub-measure")
+    ap.add_argument("--batch", type=int, default=B,
+                    help="sequences of the prefill workload (smaller values make a case small "
+                         "enough for a full ncu capture; the bench line is quoted at 4)")
     ap.add_argument("--json-out", default=None)
     return ap.parse_args()
 
@@ -348,7 +351,7 @@ def run_ours(args, ws, rank, local):
 
     # two input sets (each ~0.4 GB > 126 MB L2), rotated so no step finds its
     # inputs in L2
-    sets = [inputs.kda_prefill(seed=sd, device=dev) for sd in rank_seeds(rank)]
+    sets = [inputs.kda_prefill(seed=sd, device=dev, B=B) for sd in rank_seeds(rank)]
     out = torch.empty(sets[0].v.shape, dtype=torch.float32, device=dev)
     S_final = torch.empty((B, H, D, D), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -377,7 +380,7 @@ def run_ours(args, ws, rank, local):
             ck.fwd_factors(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, workspace=wsbuf)
             if mid is not None:
                 mid.record(stream)
-            ck.fwd_carry(wsbuf, B, T, H, D, D, chunk=CHUNK, out=out, S_final=S_final)
+            ck.fwd_carry(wsbuf, c.v, B, T, H, D, D, chunk=CHUNK, out=out, S_final=S_final)
         else:
             ck.fwd_chunked(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, out=out, S_final=S_final)
 
@@ -609,7 +612,7 @@ def _run_long(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
         ck.fwd_factors(c.q, c.k, c.v, c.alpha, c.beta, chunk=CHUNK, workspace=wsb)
         if mid is not None:
             mid.record(stream)
-        ck.fwd_carry(wsb, Bl, Tl, Hl, D, D, S0=c.S0, chunk=CHUNK, out=out, S_final=S_final)
+        ck.fwd_carry(wsb, c.v, Bl, Tl, Hl, D, D, S0=c.S0, chunk=CHUNK, out=out, S_final=S_final)
 
     for _ in range(2):
         step()
@@ -654,6 +657,7 @@ def _run_long(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
                                  "gpu_launches_per_step": 4}
         del wss
     th = Bl * Tl * Hl
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
     nbytes = th * BYTES_PER_TOKEN_HEAD + 2 * Bl * Hl * D * D * 4  # + S0 read, S_final written
     nbytes32 = th * BYTES_PER_TOKEN_HEAD_F32_OUT + 2 * Bl * Hl * D * D * 4
     return {"workload": f"long_prefill B={Bl} H={Hl} T={Tl} d={D} C={CHUNK} bf16 q/k/v, fp32 "
@@ -661,7 +665,8 @@ def _run_long(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_
             "ms_per_step": ms, "tokens_per_s": ws * Bl * Tl / (ms / 1e3),
             "achieved_gbs_fp32_out_bytes": nbytes32 / (ms / 1e3) / 1e9,
             "kernels": {"factor_kernel_ms": f_ms, "carry_kernel_ms": c_ms,
-                        "carry_ctas": 2 * Hl * Bl},
+                        "carry_ctas": Hl * Bl * (4 if 2 * (2 * Hl * Bl) <= n_sm else 2),
+                        "carry_columns_per_cta": 32 if 2 * (2 * Hl * Bl) <= n_sm else 64},
             "chunk_parallel_scan": scan,
             "algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (ms / 1e3) / 1e9,
             "hbm_frac_of_measured": nbytes / (ms / 1e3) / 1e9 / hbm_peak,
@@ -759,7 +764,7 @@ def _run_varlen(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hb
 def _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak, steps=5):
     """Backward at the bench sizes (bf16 q/k/v, fp32 gates and dO, fp32
     gradients, no S0 / dS_final); inputs larger than L2, one set."""
-    c = inputs.kda_prefill(seed=5000 + rank, device=dev)
+    c = inputs.kda_prefill(seed=5000 + rank, device=dev, B=B)
     g = torch.Generator(device=dev).manual_seed(5100 + rank)
     dO = torch.randn(c.v.shape, generator=g, device=dev)
     grads = {"dq": torch.empty(c.q.shape, dtype=torch.float32, device=dev),
@@ -944,7 +949,9 @@ def _finish(args, ws, rank, value, K, ms_per_step, alg_bytes, achieved_gbs, hbm_
 
 
 def main():
+    global B
     args = _args()
+    B = args.batch
     ws, rank, local = _dist()
     if args.impl == "reference":
         run_reference(args, ws, rank)

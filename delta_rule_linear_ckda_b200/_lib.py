@@ -48,7 +48,7 @@ SIGNATURES = {
     "ckda_bwd_chunked_workspace_bytes": (ctypes.c_int64, [_i, _i, _i, _i, _i, _i]),
     "ckda_fwd_factors": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp,
                               ctypes.c_size_t, _vp]),
-    "ckda_fwd_carry": (_i, [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
+    "ckda_fwd_carry": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp,
                             ctypes.c_size_t, _vp]),
     "ckda_fwd_chunked_fp32core": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp]),
     "ckda_fwd_chunked_path": (_i, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),

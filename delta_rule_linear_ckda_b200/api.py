@@ -184,14 +184,16 @@ def fwd_factors(q, k, v, alpha, beta, cu_seqlens=None, chunk: int = 64, workspac
     return workspace
 
 
-def fwd_carry(workspace, B, T, H, dk, dv, S0=None, cu_seqlens=None, chunk: int = 64,
+def fwd_carry(workspace, v, B, T, H, dk, dv, S0=None, cu_seqlens=None, chunk: int = 64,
               dtype=torch.bfloat16, out=None, S_final=None, out_dtype=torch.float32,
               return_final: bool = True):
-    """Phase 2: apply the factors in ``workspace`` from ``S0``.  Sizes (B, T, H as in
-    ``ckda_fwd_chunked``) and ``dtype`` must be those of the ``fwd_factors`` call.
+    """Phase 2: apply the factors in ``workspace`` from ``S0``.  ``v`` is the value
+    tensor of the ``fwd_factors`` call (the carry reads it); sizes (B, T, H as in
+    ``ckda_fwd_chunked``) and ``dtype`` must be those of that call.
     Returns ``(out, S_final)``."""
     dev = workspace.device
     _need(workspace, "workspace", torch.uint8, dev)
+    _need(v, "v", dtype, dev)
     N = B
     if out_dtype not in _DT:
         raise TypeError("out_dtype must be float32 or bfloat16")
@@ -214,7 +216,7 @@ def fwd_carry(workspace, B, T, H, dk, dv, S0=None, cu_seqlens=None, chunk: int =
         _need(S_final, "S_final", torch.float32, dev)
     with torch.cuda.device(dev):
         rc = _lib.load().ckda_fwd_carry(
-            _p(S0), _p(cu_seqlens), _p(out), _p(S_final), B, T, H, dk, dv, chunk, _DT[dtype],
+            _p(v), _p(S0), _p(cu_seqlens), _p(out), _p(S_final), B, T, H, dk, dv, chunk, _DT[dtype],
             _DT[out_dtype], _p(workspace), workspace.numel(), _stream_ptr(dev))
     if rc != 0:
         raise CKDAError(rc, "ckda_fwd_carry")

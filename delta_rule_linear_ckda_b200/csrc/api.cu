@@ -106,7 +106,7 @@ int validate_fwd(const void* q, const void* k, const void* v, const float* alpha
   const int64_t tokens = (cu != nullptr) ? (int64_t)T : (int64_t)B * T;
   if (tokens > 0 && (phases & kFactors) && (!q || !k || !v || !alpha || !beta))
     return CKDA_ERR_INVALID_ARG;
-  if (tokens > 0 && (phases & kCarry) && !out) return CKDA_ERR_INVALID_ARG;
+  if (tokens > 0 && (phases & kCarry) && (!out || !v)) return CKDA_ERR_INVALID_ARG;
   if (cu == nullptr && (int64_t)B * T * H > (int64_t)INT32_MAX) return CKDA_ERR_UNSUPPORTED;
   if (cu != nullptr && B == 0 && T != 0) return CKDA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, alpha, beta, S0, out, S_final, cu};
@@ -294,10 +294,10 @@ int ckda_fwd_factors(const void* q, const void* k, const void* v, const float* a
                   workspace_bytes, stream);
 }
 
-int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* out, float* S_final, int B,
-                   int T, int H, int d_k, int d_v, int chunk, int dtype, int out_dtype,
-                   void* workspace, size_t workspace_bytes, void* stream) {
-  return fwd_impl(true, kCarry, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, S0,
+int ckda_fwd_carry(const void* v, const float* S0, const int32_t* cu_seqlens, void* out,
+                   float* S_final, int B, int T, int H, int d_k, int d_v, int chunk, int dtype,
+                   int out_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return fwd_impl(true, kCarry, nullptr, nullptr, v, nullptr, nullptr, nullptr, nullptr, S0,
                   cu_seqlens, out, S_final, B, T, H, d_k, d_v, chunk, dtype, out_dtype,
                   workspace, workspace_bytes, stream);
 }

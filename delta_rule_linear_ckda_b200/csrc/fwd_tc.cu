@@ -14,19 +14,20 @@
 // Everything except the last two lines is independent of S0, so the forward
 // runs as two kernels:
 //
-//  1. factor_kernel -- one work unit per (chunk, head), all units in
-//     parallel (a persistent grid of one CTA per SM walks them).  It forms
+//  1. factor2_kernel -- one work unit per (chunk, head), all units in
+//     parallel (a persistent grid of two CTAs per SM walks them).  It forms
 //       P  = A Inv diag(beta)
-//       [W, U~; A W, A U~] = [Inv diag(beta); P] [K * Gamma, V]   (one M=128 MMA)
+//       [W; A W] = [Inv diag(beta); P] (K * Gamma)     (one M=128 MMA)
 //       Q' = Q * Gamma - A W
-//     and writes [W; Q'] (fp16), K * rho (fp16), [U~; A U~] (fp32) and
-//     gamma (fp32) of the unit to a workspace.
+//     and writes [-W; Q'], K * rho, [Inv diag(beta); P] (fp16) and gamma
+//     (fp32) of the unit to a workspace.
 //  2. carry_kernel -- one CTA per (sequence, head, 64-column d_v slice)
 //     walks its chunks in order with two dependent tensor-core products each:
-//       X  = [W; Q'] S0                                 (carry MMA 1)
-//       U  = U~ - X_top,   O = A U~ + X_bottom
+//       [U; O] = [Inv diag(beta); P] V + [-W; Q'] S0    (carry MMA 1)
 //       D  = (K * rho)^T U,  S_C = Diag(gamma) S0 + D   (carry MMA 2)
-//     while TMA streams the next chunk's factors in.
+//     since U = U~ - W S0 and O = A U~ + Q' S0 with [U~; A U~] =
+//     [Inv diag(beta); P] V, while TMA streams the next chunk's factors (and
+//     its bf16 V tile) in.
 //
 // Division-free score blocks: every pair s < r is split at the anchor m of
 // the highest bit in which r and s differ ("level" h, block size b = 2^h):
@@ -36,13 +37,14 @@
 // aligned blocks of 4) are direct fp32 dot products.  Zero and negative
 // gates are exact and underflow goes to zero; no logarithm or division.
 //
-// All gate products of a chunk come from one pass over 8-position groups:
-// every thread owns 4 channels of one group, forms the running products of
-// its 8 positions, and combines them with the products of whole groups
-// (exchanged through shared memory) into the level operands and into
-// K * Gamma, Q * Gamma and K * rho.  The pass runs once per 64-channel half
-// of d_k, so the level GEMMs are split along K and the next unit's inputs
-// stream in by TMA while the rest of the unit runs.
+// All gate products of a chunk come from one pass over aligned 4-position
+// groups: every thread owns 4 channels of one group, forms the running
+// products of its positions, and combines them with the products of whole
+// groups and of aligned runs of them (exchanged through shared memory) into
+// the level operands and into K * Gamma, Q * Gamma and K * rho.  The pass
+// runs once per 32-channel quarter of d_k, so the level GEMMs are split
+// along K and the next quarter's inputs stream in by TMA while the rest of
+// the quarter runs.
 //
 // SFDA ("Semidirect Fourier Delta Attention (SFDA)" page, "Arquitectura
 // Central"): the gate of channel pair (2p, 2p+1) is the complex scalar
@@ -52,7 +54,7 @@
 // and Q * Gamma take the conjugate products (Gamma_r^T k_r, Gamma_r^T q_r),
 // the right side and K * rho the plain ones, and the carry applies Gamma_C
 // to the state's row pairs.  A conversion step turns the (alpha, theta)
-// tiles of each half into interleaved (re, im) gates before its gate pass.
+// tiles of each quarter into interleaved (re, im) gates before its gate pass.
 //
 // Operands are fp16 tiles in 128-byte-swizzled shared memory; accumulators
 // live in tensor memory; the carry kernel keeps its state slice in fp32
@@ -73,11 +75,16 @@ using namespace sm100;
 
 constexpr int C = 64;
 constexpr int DK = 128;
-constexpr int HC = 64;  // channels per half of d_k
 constexpr int BV = 64;  // d_v columns of one carry CTA
 constexpr int NT = 256;   // carry kernel threads
-constexpr int NT1 = 512;  // factor kernel threads
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
+
+// Level operands of the factor kernel: levels are paired (2, 3) and (4, 5),
+// one M = 128 x N = 64 GEMM per pair, of which the two diagonal 64 x 32
+// blocks are used.  Per pair: the left operand [levels a; b] (128 rows) and
+// the right operand (64 rows), rows of one 64-channel half of d_k.
+constexpr uint32_t kPairBytes = 24576;
+constexpr uint32_t PAIR_ROP = 16384;
 
 // Gate families of the factor kernel.
 constexpr int kKda = 0;   // beta_r, Diag(alpha_r)
@@ -90,50 +97,6 @@ constexpr size_t kWsKH = (size_t)C * DK * 2;      // K * rho fp16 [64][128]
 constexpr size_t kWsIP = (size_t)2 * C * C * 2;   // [Inv diag(beta); P] fp16 [128][64]
 constexpr size_t kWsG = (size_t)DK * 4;           // gamma fp32 [128]
 // V as fp16 [64][d_v]: C * d_v * 2 bytes
-
-// ---- factor kernel: shared memory map (byte offsets, 1024-aligned base) ---
-// Two input buffers, one per 64-channel half: q, k (bf16 [64 pos][64 ch])
-// and alpha (fp32 [64 pos][64 ch]), filled by TMA.
-constexpr uint32_t OFF_IN0 = 0;
-constexpr uint32_t OFF_IN1 = 32768;
-constexpr uint32_t IN_Q = 0, IN_K = 8192, IN_A = 16384, kInBytes = 32768;
-// v tile (TMA, 128B swizzle), bf16 -> fp16 [64 s][d_v] as 64-column atoms
-constexpr uint32_t OFF_V = 65536;
-// Work region: level operands while the gate pass runs; then the fp32
-// inverse workspace and the A / [Inv; P] operands.
-constexpr uint32_t OFF_LVX = 81920;
-// Levels are paired (2, 3) and (4, 5): one M=128 x N=64 GEMM per pair, of
-// which the two diagonal 64 x 32 blocks are used.  Per pair: the left
-// operand [levels a; b] (128 rows) and the right operand (64 rows).
-constexpr uint32_t kPairBytes = 24576;
-constexpr uint32_t PAIR_ROP = 16384;
-constexpr uint32_t OFF_TF = OFF_LVX;          // T, fp32 [64][64] (swizzled, see fsw)
-constexpr uint32_t OFF_AF = OFF_LVX + 16384;  // A, fp32 [64][64] (swizzled)
-constexpr uint32_t OFF_AQ = OFF_LVX + 32768;  // A, fp16 K-major [64 r][64 s]
-constexpr uint32_t OFF_IP = OFF_LVX + 40960;  // [Inv diag(beta); P], fp16 K-major [128][64]
-constexpr uint32_t OFF_YF = OFF_LVX + 57344;  // doubling scratch, fp32 (<= 1024 values)
-constexpr uint32_t OFF_KG = 143360;  // K * Gamma, fp16 MN-major [64 s][128 i]
-constexpr uint32_t OFF_QG = 159744;  // Q * Gamma, then Q', fp16 [64 r][128 i] (128B swizzle)
-constexpr uint32_t OFF_KH = 176128;  // K * rho, then W, fp16 [64][128 i] (128B swizzle)
-constexpr uint32_t OFF_GT = 192512;  // products of whole 4-position groups, fp32 [16][64]
-constexpr uint32_t OFF_T2 = 196608;  // products of aligned pairs of groups, fp32 [8][64]
-constexpr uint32_t OFF_PR = 198656;  // direct pairs and diag(A), fp32 [16 groups][16]
-constexpr uint32_t OFF_BETA = 199680;
-constexpr uint32_t OFF_GAMMA = 199936;
-constexpr uint32_t OFF_BAR = 200448;  // mbarriers: in0, in1, v, mma, lv
-constexpr uint32_t OFF_TMEMPTR = 200512;
-constexpr uint32_t OFF_INV = 200704;  // (I + T)^-1, fp32 [64][64] (swizzled)
-constexpr uint32_t kSmemUsed = OFF_INV + 16384;
-constexpr size_t kSmemBytes = kSmemUsed + 1024;
-// The workspace tiles leave by TMA stores straight from their operand
-// tiles ([Inv diag(beta); P], the fp16 V tile, K * rho) or from staging:
-// -W over K * rho (already stored by then), Q' in place of Q * Gamma.
-
-// factor kernel tensor-memory columns
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t TM_LV = 0;    // level pairs, 64 columns each (M = 128)
-constexpr uint32_t TM_P = 128;   // P (M = 64 layout)
-constexpr uint32_t TM_W = 192;   // [W; A W]       (M = 128, 128 columns)
 
 // ---- carry kernel: shared memory map ---------------------------------------
 // Two stages of one chunk's factors, each filled by one TMA transaction.
@@ -160,16 +123,6 @@ constexpr uint32_t TM2_D = 64;   // (K rho)^T U    (M = 128, 64 columns)
 // carry CTA (0, 0, 0), and per-phase clock counts (diagnostic builds only).
 __device__ float* g_tc_dbg = nullptr;
 __device__ unsigned long long* g_tc_time = nullptr;
-__device__ unsigned long long* g_tc_time2 = nullptr;
-#define GP_MARK(k)                                                                     \
-  do {                                                                                 \
-    if (g_tc_time2 != nullptr && (tid == 0 || tid == 32) && blockIdx.x == 0 &&         \
-        blockIdx.y == 0 && blockIdx.z == 0) {                                          \
-      const long long now = clock64();                                                 \
-      atomicAdd(g_tc_time2 + 4 * (tid >> 5) + (k), (unsigned long long)(now - gp_last)); \
-      gp_last = now;                                                                   \
-    }                                                                                  \
-  } while (0)
 #define TC_DBG(stmt)                                                                   \
   do {                                                                                 \
     if (g_tc_dbg != nullptr && c == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&         \
@@ -187,9 +140,6 @@ __device__ unsigned long long* g_tc_time2 = nullptr;
     }                                                                                    \
   } while (0)
 #else
-#define GP_MARK(k) \
-  do {             \
-  } while (0)
 #define TC_DBG(stmt) \
   do {               \
   } while (0)
@@ -267,21 +217,18 @@ __device__ __forceinline__ void reduce_scatter16(float* w, int lane) {
   }
 }
 
-// 32 consecutive output values of one row, fp32 or rounded once to bf16.
-template <typename Tout>
-__device__ __forceinline__ void store_row32(Tout* dst, const float* o);
-
-template <>
-__device__ __forceinline__ void store_row32<float>(float* dst, const float* o) {
+// N consecutive output values of one row, fp32 or rounded once to bf16.
+template <int N>
+__device__ __forceinline__ void store_row(float* dst, const float* o) {
 #pragma unroll
-  for (int e = 0; e < 32; e += 4)
+  for (int e = 0; e < N; e += 4)
     *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
 }
 
-template <>
-__device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, const float* o) {
+template <int N>
+__device__ __forceinline__ void store_row(__nv_bfloat16* dst, const float* o) {
 #pragma unroll
-  for (int e = 0; e < 32; e += 8) {
+  for (int e = 0; e < N; e += 8) {
     uint4 pk;
     pk.x = pack_bf16x2(o[e], o[e + 1]);
     pk.y = pack_bf16x2(o[e + 2], o[e + 3]);
@@ -291,33 +238,30 @@ __device__ __forceinline__ void store_row32<__nv_bfloat16>(__nv_bfloat16* dst, c
   }
 }
 
-// Row r (0..63) of the output tile, columns [32 * half, +32), into the
-// 128B-swizzled staging of the TMA store: fp32 as two [64][32] atoms, bf16
-// as one [64][64] atom.
-template <typename Tout>
-__device__ __forceinline__ void stage_row32(uint32_t ob, int r, int half, const float* o);
-
-template <>
-__device__ __forceinline__ void stage_row32<float>(uint32_t ob, int r, int half, const float* o) {
-  const uint32_t row = ob + 8192 * half + 128 * r;
+// Row r (0..63) of the output tile, N columns from column c0 of the CTA's
+// slice, into the 128B-swizzled staging of the TMA store: fp32 as [64][32]
+// atoms (one per 32 columns), bf16 as one [64][64] atom.
+template <int N>
+__device__ __forceinline__ void stage_row(uint32_t ob, int r, int c0, const float* o, float) {
 #pragma unroll
-  for (int c4 = 0; c4 < 8; ++c4) {
-    const int e = 4 * c4;
-    sts_f4(row + ((c4 ^ (r & 7)) << 4), make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
+  for (int e = 0; e < N; e += 4) {
+    const int col = c0 + e;
+    const uint32_t row = ob + 8192 * (col >> 5) + 128 * r;
+    sts_f4(row + (((((col & 31) >> 2)) ^ (r & 7)) << 4),
+           make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]));
   }
 }
 
-template <>
-__device__ __forceinline__ void stage_row32<__nv_bfloat16>(uint32_t ob, int r, int half,
-                                                           const float* o) {
+template <int N>
+__device__ __forceinline__ void stage_row(uint32_t ob, int r, int c0, const float* o,
+                                          __nv_bfloat16) {
   const uint32_t row = ob + 128 * r;
 #pragma unroll
-  for (int c8 = 0; c8 < 4; ++c8) {
-    const int e = 8 * c8;
+  for (int e = 0; e < N; e += 8) {
     uint32_t w[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) w[t] = pack_bf16x2(o[e + 2 * t], o[e + 2 * t + 1]);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + (((4 * half + c8) ^ (r & 7)) << 4)),
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row + ((((c0 + e) >> 3) ^ (r & 7)) << 4)),
                  "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
                  : "memory");
   }
@@ -335,309 +279,6 @@ __device__ __forceinline__ int fsw(int r, int c) {
 // whose bit lv is set (right halves) or clear (left halves), in order.
 __device__ __forceinline__ int level_row(int lv, int p) {
   return ((p >> (lv + 1)) << lv) | (p & ((1 << lv) - 1));
-}
-
-// One gate pass over one 64-channel half.  Thread (role, g, c4): channels
-// 4*c4 .. 4*c4+3 of the half, positions 4g .. 4g+3 (g = 0..15, one aligned
-// block of 4).  Role 0 walks forward (prefix products: Gamma and the right
-// halves of levels 2..5); role 1 walks backward (suffix products: rho and the
-// left halves) and adds its channels' share of the direct pairs of levels
-// 0..1 (inside its block of 4) and of diag(A) into the pair buffer (stored by
-// half 0, added by half 1).  The products of whole groups and of aligned
-// pairs of groups are formed once and exchanged through shared memory, so
-// every anchored offset costs a handful of loads.  A warp holds groups 2k and
-// 2k + 1 of one role; each scheduler (warps w, w + 4, w + 8, w + 12) gets
-// both roles and the complementary pairs k and 7 - k, whose level work adds
-// up to the same amount on every scheduler.  One out-of-line copy serves
-// both halves.
-//
-// kGdn2 (Gated DeltaNet-2): the erase side uses e = b * k (b per key
-// channel, read from global memory at `bgp` + position * `bstride`, the
-// channels of this half) in place of beta * k: in the T rows of the level
-// operands, in the direct T pairs and in E * Gamma (stored where K * Gamma
-// goes).  kSfda: the gate tile holds (re, im) pairs, every gate product is a
-// complex product, and the row-side operands (K * Gamma, Q * Gamma, the left
-// level operands) take the conjugate of their gate product.
-template <int GK>
-__device__ __noinline__ void gate_pass(uint32_t sb, uint32_t in, int hh, int Lc, int tid,
-                                       const float* __restrict__ bgp, int bstride) {
-  constexpr bool G2 = GK == kGdn2;
-  constexpr bool SF = GK == kSfda;
-  // gate product and conjugate (plain products and identity unless SF)
-  auto gm = [](float4 a, float4 b) -> float4 {
-    if constexpr (SF)
-      return cmul4(a, b);
-    else
-      return mul4(a, b);
-  };
-  auto gc = [](float4 a) -> float4 {
-    if constexpr (SF)
-      return conj4(a);
-    else
-      return a;
-  };
-  const int w = tid >> 5;
-  const int role = (w >> 2) & 1;
-  const int kk = (w < 8) ? (w & 3) : 7 - (w & 3);
-  const int rt = (kk << 5) | (tid & 31);  // index among the 256 threads of this role
-  const int c4 = rt & 15;
-  const int g = rt >> 4;
-  const int cl = 4 * c4;
-  const int ig = HC * hh + cl;
-  // the identity gate (complex 1 on both pairs for SF)
-  const float4 one = SF ? make_float4(1.f, 0.f, 1.f, 0.f) : make_float4(1.f, 1.f, 1.f, 1.f);
-  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
-  auto bf4 = [](uint2 raw) -> float4 {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
-    return make_float4(a.x, a.y, b.x, b.y);
-  };
-  auto h4 = [](float4 v) -> uint2 {
-    uint2 pk;
-    pk.x = pack_f16x2(v.x, v.y);
-    pk.y = pack_f16x2(v.z, v.w);
-    return pk;
-  };
-
-  // every input of this thread's 4 positions, loaded up front (the erase
-  // gate first: it comes from global memory)
-  float4 aa[4], ka[4], qa[4], eg[4];
-  float bb[4];
-  if constexpr (G2) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int p = 4 * g + u;
-      eg[u] = (p < Lc) ? __ldg(reinterpret_cast<const float4*>(bgp + (size_t)p * bstride + cl)) : zero;
-    }
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int p = 4 * g + u;
-    const bool val = p < Lc;
-    aa[u] = val ? lds_f4(in + IN_A + p * 256 + cl * 4) : one;
-    ka[u] = val ? bf4(lds_u2(in + IN_K + p * 128 + cl * 2)) : zero;
-    qa[u] = val ? bf4(lds_u2(in + IN_Q + p * 128 + cl * 2)) : zero;
-    if constexpr (!G2) bb[u] = lds_f(sb + OFF_BETA + p * 4);
-  }
-  if constexpr (G2) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) eg[u] = mul4(eg[u], ka[u]);  // e = b * k
-  }
-#ifdef CKDA_TC_DEBUG
-  long long gp_last = clock64();
-#endif
-  // products of whole groups, and (one shuffle across the two groups of a
-  // warp) of aligned pairs of groups
-  const uint32_t gt = sb + OFF_GT + cl * 4;
-  if (role == 0) {
-    const float4 t = gm(gm(aa[0], aa[1]), gm(aa[2], aa[3]));
-    sts_f4(gt + g * 256, t);
-    float4 o;
-    o.x = __shfl_xor_sync(0xffffffffu, t.x, 16);
-    o.y = __shfl_xor_sync(0xffffffffu, t.y, 16);
-    o.z = __shfl_xor_sync(0xffffffffu, t.z, 16);
-    o.w = __shfl_xor_sync(0xffffffffu, t.w, 16);
-    if (!(g & 1)) sts_f4(sb + OFF_T2 + (g >> 1) * 256 + cl * 4, gm(t, o));
-  }
-  GP_MARK(0);
-  __syncthreads();
-  GP_MARK(1);
-  auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * 256); };
-  auto run2 = [&](int s2) -> float4 { return lds_f4(sb + OFF_T2 + s2 * 256 + cl * 4); };
-  auto run4 = [&](int s4) -> float4 { return gm(run2(2 * s4), run2(2 * s4 + 1)); };
-  auto run8 = [&](int s8) -> float4 {
-    return gm(gm(run2(4 * s8), run2(4 * s8 + 1)), gm(run2(4 * s8 + 2), run2(4 * s8 + 3)));
-  };
-  const uint32_t LV = sb + OFF_LVX;
-
-  // Store addresses: every tile written here has 128-byte rows (64 fp16 of
-  // one channel half) in 128B-swizzled atoms, and position p = 4g + u lands
-  // in row (tile row of 4g) + u.  The 16-byte chunk of this thread's 4
-  // channels is XOR-ed with the row's low three bits, which for position
-  // rows and levels 3..5 are 4 (g & 1) + u and for level 2 4 ((g >> 1) & 1) + u.
-  uint32_t xo[4], xo2[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    xo[u] = (uint32_t)((((c4 >> 1) ^ (4 * (g & 1) + u)) << 4) | ((c4 & 1) << 3));
-    xo2[u] = (uint32_t)((((c4 >> 1) ^ (4 * ((g >> 1) & 1) + u)) << 4) | ((c4 & 1) << 3));
-  }
-  const uint32_t rowg = (uint32_t)(4 * g) * 128 + (uint32_t)hh * 8192;  // row 4g of this half's atom
-  // row 4g's level-lv operand row, as a byte offset inside the pair tile
-  auto lrow = [&](int lv) -> uint32_t { return (uint32_t)level_row(lv, 4 * g) * 128; };
-  auto pair_base = [&](int lv) -> uint32_t { return LV + ((lv - 2) >> 1) * kPairBytes; };
-
-  if (role == 0) {
-    // Offsets: products of the whole groups from a level's anchor up to g.
-    // Level 2's anchor is this group; level 3's the start of the pair of
-    // groups, level 4's of the run of 4, level 5's of the run of 8.
-    const int g4 = g & ~3;
-    float4 off4 = one;
-    if (g - g4 >= 1) off4 = gtot(g4);
-    if (g - g4 >= 2) off4 = gm(off4, gtot(g4 + 1));
-    if (g - g4 >= 3) off4 = gm(off4, gtot(g4 + 2));
-    const float4 off3 = (g & 1) ? gtot(g - 1) : one;
-    const float4 off5 = (g & 4) ? gm(run4((g >> 2) & ~1), off4) : off4;
-    float4 pg = (g & 8) ? gm(run8(0), off5) : off5;  // Gamma offset: every earlier group
-    // the row side takes the conjugate offsets (the same values unless SF)
-    const float4 off3c = gc(off3), off4c = gc(off4), off5c = gc(off5);
-    // left operands [beta k L; q L] of level lv: rows level_row, 32 + level_row
-    const uint32_t kg_b = sb + OFF_KG + rowg;
-    const uint32_t qg_b = sb + OFF_QG + rowg;
-    const uint32_t l2b = pair_base(2) + lrow(2);
-    const uint32_t l3b = pair_base(3) + 64 * 128 + lrow(3);
-    const uint32_t l4b = pair_base(4) + lrow(4);
-    const uint32_t l5b = pair_base(5) + 64 * 128 + lrow(5);
-    float4 lp = one;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float4 a = aa[u];
-      const float4 kf = ka[u];
-      const float4 qf = qa[u];
-      pg = gm(pg, a);
-      lp = (u == 0) ? a : gm(lp, a);
-      const uint32_t ro = 128 * u + xo[u];
-      // data times the row-side gate: gc(gate) * data (conjugate for SF)
-      sts_u2(kg_b + ro, h4(gm(gc(pg), G2 ? eg[u] : kf)));
-      sts_u2(qg_b + ro, h4(gm(gc(pg), qf)));
-      if (g & 15) {
-        const float4 lpc = gc(lp);
-        const float4 qlp = gm(lpc, qf);
-        const float4 blp = G2 ? mul4(eg[u], lp) : scale4(bb[u], gm(lpc, kf));
-        if (g & 1) {  // level 2: right half
-          const uint32_t o2 = l2b + 128 * u + xo2[u];
-          sts_u2(o2, h4(blp));
-          sts_u2(o2 + 32 * 128, h4(qlp));
-        }
-        if (g & 2) {  // level 3: right half
-          sts_u2(l3b + ro, h4(gm(blp, off3c)));
-          sts_u2(l3b + 32 * 128 + ro, h4(gm(qlp, off3c)));
-        }
-        if (g & 4) {  // level 4: right half
-          sts_u2(l4b + ro, h4(gm(blp, off4c)));
-          sts_u2(l4b + 32 * 128 + ro, h4(gm(qlp, off4c)));
-        }
-        if (g & 8) {  // level 5: right half
-          sts_u2(l5b + ro, h4(gm(blp, off5c)));
-          sts_u2(l5b + 32 * 128 + ro, h4(gm(qlp, off5c)));
-        }
-      }
-    }
-    if (g == 15) sts_f4(sb + OFF_GAMMA + ig * 4, pg);
-    GP_MARK(2);
-  } else {
-    // Offsets: products of the whole groups after g up to a level's anchor.
-    float4 offr4 = one;
-    if ((g | 3) - g >= 1) offr4 = gtot(g + 1);
-    if ((g | 3) - g >= 2) offr4 = gm(offr4, gtot(g + 2));
-    if ((g | 3) - g >= 3) offr4 = gm(offr4, gtot(g + 3));
-    const float4 offr3 = (g & 1) ? one : gtot(g + 1);
-    const float4 offr5 = (g & 4) ? offr4 : gm(offr4, run4((g >> 2) + 1));
-    const float4 offr = (g & 8) ? offr5 : gm(offr5, run8(1));  // rho offset: every later group
-    // right operands k R of level lv: rows level_row of the level's 32
-    const uint32_t kh_b = sb + OFF_KH + rowg;
-    const uint32_t r2b = pair_base(2) + PAIR_ROP + lrow(2);
-    const uint32_t r3b = pair_base(3) + PAIR_ROP + 32 * 128 + lrow(3);
-    const uint32_t r4b = pair_base(4) + PAIR_ROP + lrow(4);
-    const uint32_t r5b = pair_base(5) + PAIR_ROP + 32 * 128 + lrow(5);
-    float4 ls = one;
-#pragma unroll
-    for (int u = 3; u >= 0; --u) {
-      const float4 kls = gm(ka[u], ls);
-      const uint32_t ro = 128 * u + xo[u];
-      sts_u2(kh_b + ro, h4(gm(kls, offr)));
-      if (!(g & 1)) sts_u2(r2b + 128 * u + xo2[u], h4(kls));
-      if (!(g & 2)) sts_u2(r3b + ro, h4(gm(kls, offr3)));
-      if (!(g & 4)) sts_u2(r4b + ro, h4(gm(kls, offr4)));
-      if (!(g & 8)) sts_u2(r5b + ro, h4(gm(kls, offr5)));
-      ls = gm(ls, aa[u]);
-    }
-    GP_MARK(3);
-    // direct pairs inside this aligned block of 4 (levels 0 and 1) and diag(A)
-    float acc[16];
-    {
-      const float4 k0 = ka[0], k1 = ka[1], k2 = ka[2], k3 = ka[3];
-      const float4 q1 = qa[1], q2 = qa[2], q3 = qa[3];
-      // row side of the T pairs: k_r (scaled by beta_r in the gather) or e_r
-      const float4 t1 = G2 ? eg[1] : k1, t2 = G2 ? eg[2] : k2, t3 = G2 ? eg[3] : k3;
-      const float4 e10 = gm(aa[1], k0);
-      const float4 e20 = gm(aa[2], e10);
-      const float4 e21 = gm(aa[2], k1);
-      const float4 e30 = gm(aa[3], e20);
-      const float4 e31 = gm(aa[3], e21);
-      const float4 e32 = gm(aa[3], k2);
-      acc[0] = dot4(t1, e10);  acc[1] = dot4(q1, e10);
-      acc[2] = dot4(t2, e20);  acc[3] = dot4(q2, e20);
-      acc[4] = dot4(t2, e21);  acc[5] = dot4(q2, e21);
-      acc[6] = dot4(t3, e30);  acc[7] = dot4(q3, e30);
-      acc[8] = dot4(t3, e31);  acc[9] = dot4(q3, e31);
-      acc[10] = dot4(t3, e32); acc[11] = dot4(q3, e32);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) acc[12 + u] = dot4(qa[u], ka[u]);
-    }
-    // sum over the 16 threads (channels) of the group
-    const int lane = tid & 31;
-    reduce_scatter16(acc, lane);
-    const uint32_t p0 = sb + OFF_PR + 64 * g + 4 * (lane & 15);
-    if (hh == 0)
-      sts_f(p0, acc[0]);
-    else
-      sts_f(p0, lds_f(p0) + acc[0]);
-    GP_MARK(2);
-  }
-}
-
-// One step of the recursive-doubling inverse of the unit lower-triangular
-// (I + T): merge diagonal blocks of size M into blocks of size 2M,
-//   [[A, 0], [B, D]]^-1 = [[A^-1, 0], [-D^-1 B A^-1, D^-1]],  B = T block.
-// Inv holds the inverses of the M-blocks (zero above each block diagonal),
-// so the triangular limits of both products can be left to the zeros.  Both
-// tiles use the fsw layout.
-template <int M>
-__device__ __forceinline__ void inv_merge(const float* Tf, float* Inv, float* Yf, int tid) {
-  constexpr int NMERGE = 64 / (2 * M);
-  constexpr int W4 = M / 4;                  // float4 groups per block row
-  constexpr int NOUT = NMERGE * M * W4;      // float4 outputs per phase
-  for (int e = tid; e < NOUT; e += NT1) {
-    const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
-    const int r0 = 2 * M * qb;
-    const int tr = r0 + M + a;
-    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int t4 = 0; t4 < M / 4; ++t4) {
-      const float4 tv = *reinterpret_cast<const float4*>(Tf + fsw(tr, r0 + 4 * t4));
-      const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float4 iv =
-            *reinterpret_cast<const float4*>(Inv + fsw(r0 + 4 * t4 + w, r0 + 4 * c4));
-        y.x = fmaf(tt[w], iv.x, y.x); y.y = fmaf(tt[w], iv.y, y.y);
-        y.z = fmaf(tt[w], iv.z, y.z); y.w = fmaf(tt[w], iv.w, y.w);
-      }
-    }
-    *reinterpret_cast<float4*>(Yf + qb * M * M + a * M + 4 * c4) = y;
-  }
-  __syncthreads();
-  for (int e = tid; e < NOUT; e += NT1) {
-    const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
-    const int r0 = 2 * M * qb;
-    const int ir = r0 + M + a;
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int t4 = 0; t4 < M / 4; ++t4) {
-      const float4 dv = *reinterpret_cast<const float4*>(Inv + fsw(ir, r0 + M + 4 * t4));
-      const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float4 yv =
-            *reinterpret_cast<const float4*>(Yf + qb * M * M + (4 * t4 + w) * M + 4 * c4);
-        x.x = fmaf(dd[w], yv.x, x.x); x.y = fmaf(dd[w], yv.y, x.y);
-        x.z = fmaf(dd[w], yv.z, x.z); x.w = fmaf(dd[w], yv.w, x.w);
-      }
-    }
-    *reinterpret_cast<float4*>(Inv + fsw(ir, r0 + 4 * c4)) =
-        make_float4(-x.x, -x.y, -x.z, -x.w);
-  }
-  __syncthreads();
 }
 
 // ---- work units ----------------------------------------------------------------
@@ -707,102 +348,462 @@ __device__ Unit find_unit(int ui, int stride, int n_units, const int32_t* cu, in
   return none;
 }
 
-// ---- kernel 1: per-unit WY factors ----------------------------------------------
+// ---- kernel 1, two CTAs per SM: per-unit WY factors (real gates) ------------------
+//
+// The algebra of factor_kernel for the real per-channel gates, laid out so
+// that two CTAs share each SM: the barrier and shared-memory stalls of one
+// CTA's phases (gate passes, inverse merges, tensor-core waits) overlap the
+// other CTA's work.  256 threads and at most 105 KB of shared memory per
+// CTA:
+//  * the gate pass runs over 32-channel quarters of d_k (four per unit); the
+//    level GEMMs of a quarter are issued as soon as its operands are written
+//    (K = 32 per quarter, accumulated in tensor memory);
+//  * K * rho and gamma go from registers straight to the workspace;
+//  * V is not touched: the carry kernel loads the bf16 input tile itself;
+//  * once the level GEMMs have read their operands, that region holds T, the
+//    inverse, A (fp16), then [Inv diag(beta); P] and the -W staging.
+constexpr int NT3 = 256;
+constexpr int HQ = 32;  // channels of one gate sub-pass
+constexpr uint32_t F2_LV = 0;        // level operands, 2 pairs x kPairBytes
+constexpr uint32_t F2_TF = 0;        //   T fp32 [64][64] (fsw layout)
+constexpr uint32_t F2_INV = 16384;   //   (I + T)^-1 fp32 [64][64] (fsw layout)
+constexpr uint32_t F2_AQ = 32768;    //   A fp16 K-major [64 r][64 s], 128B swizzle
+constexpr uint32_t F2_YF = 40960;    //   doubling scratch fp32 (<= 1024 values)
+constexpr uint32_t F2_IP = 0;        //   [Inv diag(beta); P] fp16 K-major [128][64] (over T)
+constexpr uint32_t F2_WS = 16384;    //   -W staging fp16 [64][128] (over the inverse)
+constexpr uint32_t F2_KG = 49152;    // K * Gamma fp16 MN-major [64 s][128 i]
+constexpr uint32_t F2_QG = 65536;    // Q * Gamma, then Q' (same layout)
+constexpr uint32_t F2_GT = 81920;    // products of whole 4-position groups, fp32 [16][32]
+constexpr uint32_t F2_T2 = 83968;    // products of aligned pairs of groups, fp32 [8][32]
+constexpr uint32_t F2_PR = 84992;    // direct pairs and diag(A), fp32 [16 groups][16]
+constexpr uint32_t F2_BETA = 86016;  // beta of the unit, fp32 [64]
+constexpr uint32_t F2_IN = 87040;    // one sub-pass of inputs, filled by TMA:
+constexpr uint32_t F2_INQ = 0, F2_INK = 4096, F2_INA = 8192, kF2InBytes = 16384;
+//                                      q, k bf16 [64][32]; alpha fp32 [64][32]
+constexpr uint32_t F2_BAR = F2_IN + kF2InBytes;  // mbarriers: in, lv0, lv1, mma
+constexpr uint32_t F2_TMEMPTR = F2_BAR + 32;
+constexpr uint32_t kF2SmemUsed = F2_TMEMPTR + 16;
+constexpr size_t kF2SmemBytes = kF2SmemUsed + 1024;
+static_assert(2 * (kF2SmemBytes + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(F2_YF + 4096 <= F2_LV + 2 * kPairBytes, "inverse tiles inside the level region");
+constexpr uint32_t kF2TmemCols = 256;
+constexpr uint32_t TM3_LV = 0;    // level pairs (M = 128), 64 columns each; then P (M = 64)
+constexpr uint32_t TM3_P = 0;
+constexpr uint32_t TM3_W = 128;   // [W; A W] (M = 128, 128 columns)
 
-// SFDA: turn the (alpha, theta) tiles of one 64-channel half (alpha at
-// IN_A, theta at IN_A + 8192, fp32 [64 pos][32 pairs] each) into the gate
-// tile the gate pass reads, fp32 [64 pos][64] with (re, im) =
-// alpha (cos theta, sin theta) per pair, in place.  Every thread converts 4
-// pairs of one position; the values are read before the barrier and written
-// after it.
-__device__ __forceinline__ void phase_to_gates(uint32_t in, int tid) {
-  const int p = tid >> 3, j = tid & 7;
-  const float4 a = lds_f4(in + IN_A + p * 128 + 16 * j);
-  const float4 th = lds_f4(in + IN_A + 8192 + p * 128 + 16 * j);
+// Four products as two packed fp32x2 multiplies (sm_100a); each lane rounds
+// like a scalar fp32 multiply, so the results equal mul4's and scale4's.
+__device__ __forceinline__ float4 mul4x(float4 a, float4 b) {
+  const float2 lo = __fmul2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+  const float2 hi = __fmul2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+  return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+__device__ __forceinline__ float4 scale4x(float s, float4 a) {
+  return mul4x(make_float4(s, s, s, s), a);
+}
+
+// Sum 16 values over the 8 lanes of an aligned lane octet; afterwards lane L
+// of the octet holds the totals of elements 2 (L % 8) and 2 (L % 8) + 1 in
+// w[0], w[1].
+__device__ __forceinline__ void reduce_scatter8x2(float* w, int lane) {
+#pragma unroll
+  for (int o = 4; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < 2 * o; ++i) {
+      const float send = up ? w[i] : w[i + 2 * o];
+      const float keep = up ? w[i + 2 * o] : w[i];
+      w[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
+// Where the next sub-pass's inputs come from: unit `u` (idx < 0: none),
+// quarter `j` of d_k.  SFDA fetches alpha and theta per channel pair (16 of
+// each per quarter) in place of alpha per channel.
+struct NextIn {
+  const CUtensorMap* tq;
+  const CUtensorMap* tk;
+  const CUtensorMap* ta;
+  const CUtensorMap* tth;  // SFDA phases (NULL otherwise)
+  uint32_t dst;
+  uint32_t bar;
+  int x;      // first column (channel) of the quarter in the row of all heads
+  int xa;     // first column of the gate tiles (the channel pair for SFDA)
+  int y;      // first token row
+  int valid;  // 0: nothing to fetch
+};
+
+// SFDA: turn the (alpha, theta) tiles of one quarter (alpha at F2_INA,
+// theta at F2_INA + 4096, fp32 [64 pos][16 pairs] each) into the gate tile
+// the gate pass reads, fp32 [64 pos][32] with (re, im) = alpha (cos theta,
+// sin theta) per pair, in place.  Every thread converts 4 pairs of one
+// position; the values are read before the barrier and written after it.
+__device__ __forceinline__ void phase_to_gates_q(uint32_t in, int tid) {
+  const int p = tid >> 2, j = tid & 3;
+  const float4 a = lds_f4(in + F2_INA + p * 64 + 16 * j);
+  const float4 th = lds_f4(in + F2_INA + 4096 + p * 64 + 16 * j);
   float s0, c0, s1, c1, s2, c2, s3, c3;
   sincosf(th.x, &s0, &c0);
   sincosf(th.y, &s1, &c1);
   sincosf(th.z, &s2, &c2);
   sincosf(th.w, &s3, &c3);
   __syncthreads();
-  sts_f4(in + IN_A + p * 256 + 32 * j, make_float4(a.x * c0, a.x * s0, a.y * c1, a.y * s1));
-  sts_f4(in + IN_A + p * 256 + 32 * j + 16, make_float4(a.z * c2, a.z * s2, a.w * c3, a.w * s3));
+  sts_f4(in + F2_INA + p * 128 + 32 * j, make_float4(a.x * c0, a.x * s0, a.y * c1, a.y * s1));
+  sts_f4(in + F2_INA + p * 128 + 32 * j + 16, make_float4(a.z * c2, a.z * s2, a.w * c3, a.w * s3));
   __syncthreads();
 }
 
-// kGdn2: the Gated DeltaNet-2 form -- erase gate bg (shaped like k) and write
-// gate wg (shaped like v) in place of beta; the workspace then holds
-// [-W; Q'] with W = Inv (E * Gamma), [Inv; A Inv] and Z = wg * V, and the
-// carry kernel is unchanged.  kSfda: the phase-decay gates, alpha and theta
-// fp32 [rows, H * DK / 2] (tm_a, tm_th); gamma is stored as (re, im) pairs
-// and the carry kernel applies it to row pairs.
-template <int DV, int GK>
-__global__ void __launch_bounds__(NT1, 1)
-factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-              const __grid_constant__ CUtensorMap tm_th,
-              const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
-              const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
-              const float* __restrict__ beta, const float* __restrict__ bg,
-              const float* __restrict__ wg,
-              const int32_t* __restrict__ cu, int n_seqs, int T, int H, int nch, int64_t n_units,
-              float* __restrict__ ws_g, int* status) {
+// One gate pass over quarter `jq` (channels 32 jq .. 32 jq + 31 of d_k) with
+// 256 threads.  Thread (role, g, c4): warp w = 4 role + kk, g = 4 kk + lane / 8
+// (positions 4g .. 4g + 3, one aligned block of 4), c4 = lane % 8 (channels
+// 4 c4 .. 4 c4 + 3 of the quarter).  Each scheduler (warps kk and kk + 4)
+// gets both roles of the same four groups, whose level work adds up to the
+// same amount on every scheduler.  Role 0 walks forward (Gamma, K * Gamma,
+// Q * Gamma, the right halves of levels 2..5, gamma to the workspace); role 1
+// walks backward (K * rho straight to the workspace, the left halves) and
+// adds its channels' share of the direct pairs of levels 0..1 and of diag(A)
+// to the pair buffer.  The inputs are read into registers first; after the
+// barrier that follows, thread 0 requests the next sub-pass's inputs into the
+// same buffer (`nx`).  Operand tiles have 128-byte rows of one 64-channel
+// half; this quarter fills logical 16-byte chunks 4 (jq % 2) .. 4 (jq % 2) + 3.
+//
+// kGdn2: the erase side uses e = b * k (b read from global memory at `bgp` +
+// position * `bstride`, the quarter's channels) in place of beta * k, in the
+// T rows of the level operands, the direct T pairs and E * Gamma (stored
+// where K * Gamma goes).  kSfda: the gate tile holds (re, im) pairs, every
+// gate product is a complex product and the row-side operands (K * Gamma,
+// Q * Gamma, the left level operands) take the conjugate of their product.
+template <int GK>
+__device__ __noinline__ void gate_pass_q(uint32_t sb, int jq, int Lc, int tid,
+                                         __half* __restrict__ kh_row0,
+                                         float* __restrict__ g_dst, NextIn nx,
+                                         const float* __restrict__ bgp, int bstride) {
   constexpr bool G2 = GK == kGdn2;
   constexpr bool SF = GK == kSfda;
-  // Offsetting the __shared__ array itself (not a cast integer) keeps every
-  // access below in the shared state space.
+  auto gm = [](float4 a, float4 b) -> float4 {
+    if constexpr (SF)
+      return cmul4(a, b);
+    else
+      return mul4x(a, b);
+  };
+  auto gc = [](float4 a) -> float4 {
+    if constexpr (SF)
+      return conj4(a);
+    else
+      return a;
+  };
+  const int w = tid >> 5;
+  const int lane = tid & 31;
+  const int role = w >> 2;
+  const int kk = w & 3;
+  const int g = 4 * kk + (lane >> 3);
+  const int c4 = lane & 7;
+  const int cl = 4 * c4;               // channel within the quarter
+  const int hh = jq >> 1;              // half of d_k
+  const int cq = 32 * (jq & 1) + cl;   // channel within the half
+  const int ig = 64 * hh + cq;         // channel within d_k
+  const float4 one = SF ? make_float4(1.f, 0.f, 1.f, 0.f) : make_float4(1.f, 1.f, 1.f, 1.f);
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  const uint32_t in = sb + F2_IN;
+  auto bf4 = [](uint2 raw) -> float4 {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+  };
+  auto h4 = [](float4 v) -> uint2 {
+    uint2 pk;
+    pk.x = pack_f16x2(v.x, v.y);
+    pk.y = pack_f16x2(v.z, v.w);
+    return pk;
+  };
+
+  float4 aa[4], ka[4], qa[4], eg[4];
+  float bb[4];
+  if constexpr (G2) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int p = 4 * g + u;
+      eg[u] = (p < Lc) ? __ldg(reinterpret_cast<const float4*>(bgp + (size_t)p * bstride + cl))
+                       : zero;
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int p = 4 * g + u;
+    const bool val = p < Lc;
+    aa[u] = val ? lds_f4(in + F2_INA + p * 128 + cl * 4) : one;
+    ka[u] = val ? bf4(lds_u2(in + F2_INK + p * 64 + cl * 2)) : zero;
+    qa[u] = val ? bf4(lds_u2(in + F2_INQ + p * 64 + cl * 2)) : zero;
+    if constexpr (!G2) bb[u] = lds_f(sb + F2_BETA + p * 4);
+  }
+  if constexpr (G2) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) eg[u] = mul4x(eg[u], ka[u]);  // e = b * k
+  }
+  // products of whole groups, and (one shuffle across neighbouring groups,
+  // 8 lanes apart) of aligned pairs of groups
+  const uint32_t gt = sb + F2_GT + cl * 4;
+  if (role == 0) {
+    const float4 t = gm(gm(aa[0], aa[1]), gm(aa[2], aa[3]));
+    sts_f4(gt + g * 128, t);
+    float4 o;
+    o.x = __shfl_xor_sync(0xffffffffu, t.x, 8);
+    o.y = __shfl_xor_sync(0xffffffffu, t.y, 8);
+    o.z = __shfl_xor_sync(0xffffffffu, t.z, 8);
+    o.w = __shfl_xor_sync(0xffffffffu, t.w, 8);
+    if (!(g & 1)) sts_f4(sb + F2_T2 + (g >> 1) * 128 + cl * 4, gm(t, o));
+  }
+  __syncthreads();
+  // every input of this sub-pass is in registers: the buffer takes the next one
+  if (tid == 0 && nx.valid) {
+    fence_proxy_async_smem();
+    mbar_expect_tx(nx.bar, kF2InBytes);
+    tma_load_2d(nx.dst + F2_INQ, nx.tq, nx.x, nx.y, nx.bar);
+    tma_load_2d(nx.dst + F2_INK, nx.tk, nx.x, nx.y, nx.bar);
+    tma_load_2d(nx.dst + F2_INA, nx.ta, nx.xa, nx.y, nx.bar);
+    if constexpr (SF) tma_load_2d(nx.dst + F2_INA + 4096, nx.tth, nx.xa, nx.y, nx.bar);
+  }
+  auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * 128); };
+  auto run2 = [&](int s2) -> float4 { return lds_f4(sb + F2_T2 + s2 * 128 + cl * 4); };
+  auto run4 = [&](int s4) -> float4 { return gm(run2(2 * s4), run2(2 * s4 + 1)); };
+  auto run8 = [&](int s8) -> float4 {
+    return gm(gm(run2(4 * s8), run2(4 * s8 + 1)), gm(run2(4 * s8 + 2), run2(4 * s8 + 3)));
+  };
+  const uint32_t LV = sb + F2_LV;
+  // Store addresses in the 128B-swizzled operand tiles: this thread's 4
+  // channels are logical chunk 4 (jq % 2) + c4 / 2, half c4 % 2 of it; the
+  // chunk is XOR-ed with the row's low three bits, which for position rows
+  // and levels 3..5 are 4 (g & 1) + u and for level 2 4 ((g >> 1) & 1) + u.
+  const int lchunk = 4 * (jq & 1) + (c4 >> 1);
+  uint32_t xo[4], xo2[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    xo[u] = (uint32_t)(((lchunk ^ (4 * (g & 1) + u)) << 4) | ((c4 & 1) << 3));
+    xo2[u] = (uint32_t)(((lchunk ^ (4 * ((g >> 1) & 1) + u)) << 4) | ((c4 & 1) << 3));
+  }
+  const uint32_t rowg = (uint32_t)(4 * g) * 128 + (uint32_t)hh * 8192;
+  auto lrow = [&](int lv) -> uint32_t { return (uint32_t)level_row(lv, 4 * g) * 128; };
+  auto pair_base = [&](int lv) -> uint32_t { return LV + ((lv - 2) >> 1) * kPairBytes; };
+
+  if (role == 0) {
+    const int g4 = g & ~3;
+    float4 off4 = one;
+    if (g - g4 >= 1) off4 = gtot(g4);
+    if (g - g4 >= 2) off4 = gm(off4, gtot(g4 + 1));
+    if (g - g4 >= 3) off4 = gm(off4, gtot(g4 + 2));
+    const float4 off3 = (g & 1) ? gtot(g - 1) : one;
+    const float4 off5 = (g & 4) ? gm(run4((g >> 2) & ~1), off4) : off4;
+    float4 pg = (g & 8) ? gm(run8(0), off5) : off5;  // Gamma offset: every earlier group
+    // the row side takes the conjugate offsets (the same values unless SF)
+    const float4 off3c = gc(off3), off4c = gc(off4), off5c = gc(off5);
+    const uint32_t kg_b = sb + F2_KG + rowg;
+    const uint32_t qg_b = sb + F2_QG + rowg;
+    const uint32_t l2b = pair_base(2) + lrow(2);
+    const uint32_t l3b = pair_base(3) + 64 * 128 + lrow(3);
+    const uint32_t l4b = pair_base(4) + lrow(4);
+    const uint32_t l5b = pair_base(5) + 64 * 128 + lrow(5);
+    float4 lp = one;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float4 a = aa[u];
+      pg = gm(pg, a);
+      lp = (u == 0) ? a : gm(lp, a);
+      const uint32_t ro = 128 * u + xo[u];
+      // data times the row-side gate: gc(gate) * data (conjugate for SF)
+      sts_u2(kg_b + ro, h4(gm(gc(pg), G2 ? eg[u] : ka[u])));
+      sts_u2(qg_b + ro, h4(gm(gc(pg), qa[u])));
+      if (g & 15) {
+        const float4 lpc = gc(lp);
+        const float4 qlp = gm(lpc, qa[u]);
+        const float4 blp = G2 ? mul4x(eg[u], lp) : scale4x(bb[u], gm(lpc, ka[u]));
+        if (g & 1) {  // level 2: right half
+          const uint32_t o2 = l2b + 128 * u + xo2[u];
+          sts_u2(o2, h4(blp));
+          sts_u2(o2 + 32 * 128, h4(qlp));
+        }
+        if (g & 2) {  // level 3: right half
+          sts_u2(l3b + ro, h4(gm(blp, off3c)));
+          sts_u2(l3b + 32 * 128 + ro, h4(gm(qlp, off3c)));
+        }
+        if (g & 4) {  // level 4: right half
+          sts_u2(l4b + ro, h4(gm(blp, off4c)));
+          sts_u2(l4b + 32 * 128 + ro, h4(gm(qlp, off4c)));
+        }
+        if (g & 8) {  // level 5: right half
+          sts_u2(l5b + ro, h4(gm(blp, off5c)));
+          sts_u2(l5b + 32 * 128 + ro, h4(gm(qlp, off5c)));
+        }
+      }
+    }
+    if (g == 15) *reinterpret_cast<float4*>(g_dst + ig) = pg;
+  } else {
+    float4 offr4 = one;
+    if ((g | 3) - g >= 1) offr4 = gtot(g + 1);
+    if ((g | 3) - g >= 2) offr4 = gm(offr4, gtot(g + 2));
+    if ((g | 3) - g >= 3) offr4 = gm(offr4, gtot(g + 3));
+    const float4 offr3 = (g & 1) ? one : gtot(g + 1);
+    const float4 offr5 = (g & 4) ? offr4 : gm(offr4, run4((g >> 2) + 1));
+    const float4 offr = (g & 8) ? offr5 : gm(offr5, run8(1));  // rho offset: every later group
+    const uint32_t r2b = pair_base(2) + PAIR_ROP + lrow(2);
+    const uint32_t r3b = pair_base(3) + PAIR_ROP + 32 * 128 + lrow(3);
+    const uint32_t r4b = pair_base(4) + PAIR_ROP + lrow(4);
+    const uint32_t r5b = pair_base(5) + PAIR_ROP + 32 * 128 + lrow(5);
+    float4 ls = one;
+#pragma unroll
+    for (int u = 3; u >= 0; --u) {
+      const float4 kls = gm(ka[u], ls);
+      const uint32_t ro = 128 * u + xo[u];
+      // K * rho, fp16, straight to the workspace row of position 4g + u
+      *reinterpret_cast<uint2*>(kh_row0 + (size_t)(4 * g + u) * DK + ig) = h4(gm(kls, offr));
+      if (!(g & 1)) sts_u2(r2b + 128 * u + xo2[u], h4(kls));
+      if (!(g & 2)) sts_u2(r3b + ro, h4(gm(kls, offr3)));
+      if (!(g & 4)) sts_u2(r4b + ro, h4(gm(kls, offr4)));
+      if (!(g & 8)) sts_u2(r5b + ro, h4(gm(kls, offr5)));
+      ls = gm(ls, aa[u]);
+    }
+    // direct pairs inside this aligned block of 4 (levels 0 and 1) and diag(A)
+    float acc[16];
+    {
+      const float4 k0 = ka[0], k1 = ka[1], k2 = ka[2], k3 = ka[3];
+      const float4 q1 = qa[1], q2 = qa[2], q3 = qa[3];
+      // row side of the T pairs: k_r (scaled by beta_r in the gather) or e_r
+      const float4 t1 = G2 ? eg[1] : k1, t2 = G2 ? eg[2] : k2, t3 = G2 ? eg[3] : k3;
+      const float4 e10 = gm(aa[1], k0);
+      const float4 e20 = gm(aa[2], e10);
+      const float4 e21 = gm(aa[2], k1);
+      const float4 e30 = gm(aa[3], e20);
+      const float4 e31 = gm(aa[3], e21);
+      const float4 e32 = gm(aa[3], k2);
+      acc[0] = dot4(t1, e10);  acc[1] = dot4(q1, e10);
+      acc[2] = dot4(t2, e20);  acc[3] = dot4(q2, e20);
+      acc[4] = dot4(t2, e21);  acc[5] = dot4(q2, e21);
+      acc[6] = dot4(t3, e30);  acc[7] = dot4(q3, e30);
+      acc[8] = dot4(t3, e31);  acc[9] = dot4(q3, e31);
+      acc[10] = dot4(t3, e32); acc[11] = dot4(q3, e32);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[12 + u] = dot4(qa[u], ka[u]);
+    }
+    // sum over the 8 threads (channels) of the group
+    reduce_scatter8x2(acc, lane);
+    const uint32_t p0 = sb + F2_PR + 64 * g + 8 * (lane & 7);
+    if (jq == 0) {
+      sts_u2(p0, make_uint2(__float_as_uint(acc[0]), __float_as_uint(acc[1])));
+    } else {
+      const uint2 o = lds_u2(p0);
+      sts_u2(p0, make_uint2(__float_as_uint(__uint_as_float(o.x) + acc[0]),
+                            __float_as_uint(__uint_as_float(o.y) + acc[1])));
+    }
+  }
+}
+
+// Recursive-doubling merge of the inverse (as inv_merge) for NTH threads.
+template <int M, int NTH>
+__device__ __forceinline__ void inv_merge_n(const float* Tf, float* Inv, float* Yf, int tid) {
+  constexpr int NMERGE = 64 / (2 * M);
+  constexpr int W4 = M / 4;
+  constexpr int NOUT = NMERGE * M * W4;
+  for (int e = tid; e < NOUT; e += NTH) {
+    const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
+    const int r0 = 2 * M * qb;
+    const int tr = r0 + M + a;
+    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int t4 = 0; t4 < M / 4; ++t4) {
+      const float4 tv = *reinterpret_cast<const float4*>(Tf + fsw(tr, r0 + 4 * t4));
+      const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 iv =
+            *reinterpret_cast<const float4*>(Inv + fsw(r0 + 4 * t4 + w, r0 + 4 * c4));
+        y.x = fmaf(tt[w], iv.x, y.x); y.y = fmaf(tt[w], iv.y, y.y);
+        y.z = fmaf(tt[w], iv.z, y.z); y.w = fmaf(tt[w], iv.w, y.w);
+      }
+    }
+    *reinterpret_cast<float4*>(Yf + qb * M * M + a * M + 4 * c4) = y;
+  }
+  __syncthreads();
+  for (int e = tid; e < NOUT; e += NTH) {
+    const int qb = e / (M * W4), a = (e / W4) % M, c4 = e % W4;
+    const int r0 = 2 * M * qb;
+    const int ir = r0 + M + a;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int t4 = 0; t4 < M / 4; ++t4) {
+      const float4 dv = *reinterpret_cast<const float4*>(Inv + fsw(ir, r0 + M + 4 * t4));
+      const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 yv =
+            *reinterpret_cast<const float4*>(Yf + qb * M * M + (4 * t4 + w) * M + 4 * c4);
+        x.x = fmaf(dd[w], yv.x, x.x); x.y = fmaf(dd[w], yv.y, x.y);
+        x.z = fmaf(dd[w], yv.z, x.z); x.w = fmaf(dd[w], yv.w, x.w);
+      }
+    }
+    *reinterpret_cast<float4*>(Inv + fsw(ir, r0 + 4 * c4)) =
+        make_float4(-x.x, -x.y, -x.z, -x.w);
+  }
+  __syncthreads();
+}
+
+// ws_kh: K * rho fp16 [units * C][DK] (row-major), ws_g: gamma fp32 [units][DK].
+// kGdn2: erase gate bg (shaped like k) and write gate wg (shaped like v) in
+// place of beta; the factors are [-W; Q'] with W = Inv (E * Gamma) and
+// [Inv; A Inv], and Z = wg * V goes to ws_v (fp16 [units * C][DV]) for the
+// carry kernel.  kSfda: alpha and theta fp32 [rows, H * DK / 2] (tm_a,
+// tm_th); gamma is stored as (re, im) pairs.
+template <int DV, int GK>
+__global__ void __launch_bounds__(NT3, 2)
+factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_th,
+               const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_ip,
+               const float* __restrict__ beta, const float* __restrict__ bg,
+               const float* __restrict__ wg, const __nv_bfloat16* __restrict__ qg,
+               const __nv_bfloat16* __restrict__ kg, const float* __restrict__ ag,
+               const float* __restrict__ thg, const __nv_bfloat16* __restrict__ vg,
+               const int32_t* __restrict__ cu, int n_seqs,
+               int T, int H, int nch, int64_t n_units, __half* __restrict__ ws_kh,
+               __half* __restrict__ ws_v, float* __restrict__ ws_g, int* status) {
+  constexpr bool G2 = GK == kGdn2;
+  constexpr bool SF = GK == kSfda;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const uint32_t sb = smem_u32(sm);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int q4 = warp & 3;     // tensor-memory lane quarter of this warp
-  const int quarter = warp >> 2;  // which quarter of a tile's columns this warp takes
+  const int q4 = warp & 3;        // tensor-memory lane quarter of this warp
+  const int quarter = warp >> 2;  // which half of a tile's columns this warp takes
 
-  float* beta_s = reinterpret_cast<float*>(sm + OFF_BETA);
-  const float* gamma_s = reinterpret_cast<const float*>(sm + OFF_GAMMA);
-  const uint32_t bar_in0 = sb + OFF_BAR;
-  const uint32_t bar_in1 = sb + OFF_BAR + 8;
-  const uint32_t bar_v = sb + OFF_BAR + 16;
-  const uint32_t bar_mma = sb + OFF_BAR + 24;
-  const uint32_t bar_lv = sb + OFF_BAR + 32;
-
+  float* beta_s = reinterpret_cast<float*>(sm + F2_BETA);
+  const uint32_t bar_in = sb + F2_BAR;
+  const uint32_t bar_lv0 = sb + F2_BAR + 8;
+  const uint32_t bar_mma = sb + F2_BAR + 24;
   if (tid == 0) {
-    mbar_init(bar_in0, 1);
-    mbar_init(bar_in1, 1);
-    mbar_init(bar_v, 1);
+    mbar_init(bar_in, 1);
+    mbar_init(bar_lv0, 1);
+    mbar_init(bar_lv0 + 8, 1);
     mbar_init(bar_mma, 1);
-    mbar_init(bar_lv, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
-    prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_a);
     if (SF) prefetch_tmap(&tm_th);
     prefetch_tmap(&tm_wq);
-    prefetch_tmap(&tm_kh);
     prefetch_tmap(&tm_ip);
-    prefetch_tmap(&tm_v16);
   }
   if (warp == 0) {
-    tmem_alloc(sb + OFF_TMEMPTR, kTmemCols);
+    tmem_alloc(sb + F2_TMEMPTR, kF2TmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF_TMEMPTR);
-#ifdef CKDA_TC_DEBUG
-  long long tmark[16] = {0};
-  long long tlast = clock64();
-#endif
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + F2_TMEMPTR);
 
-  // A phase bit advances only when its wait succeeds, and a barrier stays
-  // "pending" from its issue to that wait, so the time-out path below knows
-  // exactly which copies and products may still be in flight.
-  uint32_t ph_in0 = 0, ph_in1 = 0, ph_v = 0, ph_mma = 0, ph_lv = 0;
-  int pend_in0 = 0, pend_in1 = 0, pend_v = 0, pend_mma = 0, pend_lv = 0;
+  uint32_t ph_in = 0, ph_lv[2] = {0, 0}, ph_mma = 0;
+  int pend_in = 0, pend_lv[2] = {0, 0}, pend_mma = 0;
   int ok = 1;
   auto wait = [&](uint32_t bar, uint32_t& ph, int& pend) -> bool {
     const bool r = mbar_wait_bounded(bar, ph, kWaitNs);
@@ -812,262 +813,220 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
     return r;
   };
-
-  auto issue_in = [&](int hh, const Unit& u) {
-    const uint32_t base = sb + (hh ? OFF_IN1 : OFF_IN0);
-    const uint32_t bar = hh ? bar_in1 : bar_in0;
-    mbar_expect_tx(bar, kInBytes);
-    tma_load_2d(base + IN_Q, &tm_q, u.h * DK + HC * hh, (int)u.t0, bar);
-    tma_load_2d(base + IN_K, &tm_k, u.h * DK + HC * hh, (int)u.t0, bar);
-    if constexpr (SF) {
-      tma_load_2d(base + IN_A, &tm_a, u.h * (DK / 2) + (HC / 2) * hh, (int)u.t0, bar);
-      tma_load_2d(base + IN_A + 8192, &tm_th, u.h * (DK / 2) + (HC / 2) * hh, (int)u.t0, bar);
-    } else {
-      tma_load_2d(base + IN_A, &tm_a, u.h * DK + HC * hh, (int)u.t0, bar);
-    }
+  auto next_in = [&](const Unit& uu, int jq) -> NextIn {
+    NextIn n;
+    n.tq = &tm_q;
+    n.tk = &tm_k;
+    n.ta = &tm_a;
+    n.tth = SF ? &tm_th : nullptr;
+    n.dst = sb + F2_IN;
+    n.bar = bar_in;
+    n.x = uu.h * DK + HQ * jq;
+    n.xa = SF ? uu.h * (DK / 2) + (HQ / 2) * jq : n.x;
+    n.y = (int)uu.t0;
+    n.valid = uu.idx >= 0;
+    return n;
   };
-  auto issue_v = [&](const Unit& u) {
-    mbar_expect_tx(bar_v, 8192 * (DV / 64));
-#pragma unroll
-    for (int a = 0; a < DV / 64; ++a)
-      tma_load_2d(sb + OFF_V + 8192 * a, &tm_v, u.h * DV + 64 * a, (int)u.t0, bar_v);
-  };
-  auto level_mmas = [&](int hh) {
+  auto level_mmas = [&](int jq) {
     constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
-      const uint32_t la = sb + OFF_LVX + pr * kPairBytes;
+      const uint32_t la = sb + F2_LV + pr * kPairBytes;
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
+      for (int k2 = 0; k2 < 2; ++k2) {
+        const int kk = 2 * (jq & 1) + k2;
         const uint64_t ad = smem_desc(la + kk * 32, 16, 1024, kSwizzle128);
         const uint64_t bd = smem_desc(la + PAIR_ROP + kk * 32, 16, 1024, kSwizzle128);
-        mma_f16(tmem + TM_LV + 64 * pr, ad, bd, id, (hh > 0 || kk > 0) ? 1u : 0u);
+        mma_f16(tmem + TM3_LV + 64 * pr, ad, bd, id, (jq > 0 || k2 > 0) ? 1u : 0u);
       }
     }
-    mma_commit(bar_lv);
+    mma_commit(bar_lv0 + 8 * (jq & 1));
   };
-
-  // beta of a unit, one value per thread tid < C (0 past the end)
   auto load_beta = [&](const Unit& uu) -> float {
     if constexpr (G2) return 0.f;  // unused
     return (uu.idx >= 0 && tid < uu.Lc) ? beta[(size_t)(uu.t0 + tid) * H + uu.h] : 0.f;
+  };
+  // Pull a unit's input rows into L2, one 128-byte line per thread and step:
+  // per token q, k (2 lines each), the gates (alpha: 4 lines; SFDA alpha and
+  // theta: 2 each), and for Gated DeltaNet-2 the erase gate (4), the write
+  // gate (DV / 32) and v (DV / 64), read with plain loads.
+  auto prefetch_unit = [&](const Unit& uu) {
+    constexpr int NL = G2 ? 12 + DV / 32 + DV / 64 : 8;
+    if (uu.idx < 0) return;
+    for (int e = tid; e < C * NL; e += NT3) {
+      const int r = e / NL, li = e % NL;
+      if (r >= uu.Lc) break;
+      const size_t row = (size_t)(uu.t0 + r) * H + uu.h;
+      const void* a;
+      if (li < 2) {
+        a = qg + row * DK + 64 * li;
+      } else if (li < 4) {
+        a = kg + row * DK + 64 * (li - 2);
+      } else if (li < 8) {
+        if constexpr (SF) {
+          const float* base = (li < 6) ? ag : thg;
+          a = base + row * (DK / 2) + 32 * ((li - 4) & 1);
+        } else {
+          a = ag + row * DK + 32 * (li - 4);
+        }
+      } else if (li < 12) {
+        a = bg + row * DK + 32 * (li - 8);
+      } else if (li < 12 + DV / 32) {
+        a = wg + row * DV + 32 * (li - 12);
+      } else {
+        a = vg + row * DV + 64 * (li - 12 - DV / 32);
+      }
+      prefetch_l2(a);
+    }
   };
 
   Unit cur = find_unit(blockIdx.x, gridDim.x, (int)n_units, cu, n_seqs, T, H, nch);
   float beta_next = 0.f;
   if (cur.idx >= 0) {
     if (tid == 0) {
-      issue_in(0, cur);
-      issue_in(1, cur);
-      issue_v(cur);
+      const NextIn n0 = next_in(cur, 0);
+      mbar_expect_tx(bar_in, kF2InBytes);
+      tma_load_2d(n0.dst + F2_INQ, &tm_q, n0.x, n0.y, bar_in);
+      tma_load_2d(n0.dst + F2_INK, &tm_k, n0.x, n0.y, bar_in);
+      tma_load_2d(n0.dst + F2_INA, &tm_a, n0.xa, n0.y, bar_in);
+      if (SF) tma_load_2d(n0.dst + F2_INA + 4096, &tm_th, n0.xa, n0.y, bar_in);
     }
-    pend_in0 = pend_in1 = pend_v = 1;
-    if (tid < C) beta_next = load_beta(cur);
+    pend_in = 1;
+    beta_next = load_beta(cur);
   }
 
-  for (int c = 0; cur.idx >= 0; ++c) {
+  for (; cur.idx >= 0;) {
     const Unit nxt =
         find_unit((int)cur.idx + gridDim.x, gridDim.x, (int)n_units, cu, n_seqs, T, H, nch);
-    const bool more = nxt.idx >= 0;
     const int Lc = cur.Lc;
     const size_t u = (size_t)cur.idx;
+    prefetch_unit(nxt);
+    // the previous unit's workspace stores read the level region and Q'
+    if (tid == 0) bulk_wait_read_all();
     if (tid < C) beta_s[tid] = beta_next;
-    // ---- gate pass, half 0 ---------------------------------------------------
-    // the previous unit's workspace stores must have read the tiles the
-    // first gate pass and the v load reuse (all but the channel-64..127
-    // atoms of -W and Q', which the second gate pass waits for)
-    if (c > 0) {
+    __half* kh_row0 = ws_kh + u * C * DK;
+    float* g_dst = ws_g + u * DK;
+
+    // ---- four gate sub-passes; the level GEMMs of each follow it -------------
+    for (int jq = 0; jq < 4; ++jq) {
+      ok = wait(bar_in, ph_in, pend_in);
+      // sub-pass jq overwrites the operand chunks the GEMMs of jq - 2 read
+      if (jq >= 2) ok = wait(bar_lv0 + 8 * (jq & 1), ph_lv[jq & 1], pend_lv[jq & 1]) && ok;
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+      const NextIn nx = (jq < 3) ? next_in(cur, jq + 1) : next_in(nxt, 0);
+      if constexpr (SF) phase_to_gates_q(sb + F2_IN, tid);
+      gate_pass_q<GK>(sb, jq, Lc, tid, kh_row0, g_dst, nx,
+                      G2 ? bg + ((size_t)cur.t0 * H + cur.h) * DK + HQ * jq : nullptr, H * DK);
+      if (nx.valid) pend_in = 1;
+      fence_proxy_async_smem();
+      __syncthreads();
       if (tid == 0) {
-        bulk_wait_read_all_but_last();
-        issue_v(cur);
+        tc_fence_after();
+        level_mmas(jq);
       }
-      pend_v = 1;
+      pend_lv[jq & 1] = 1;
     }
-    ok = wait(bar_in0, ph_in0, pend_in0);
-    ok = __syncthreads_and(ok);
     if (!ok) break;
-    TC_MARK(0);
-#ifdef CKDA_TC_DEBUG
-    const long long t_gp0 = clock64();
-#endif
-    // (G2: the erase gate of this half starts at row t0, channel h * DK + 64 hh)
-    const float* bg_row = G2 ? bg + ((size_t)cur.t0 * H + cur.h) * DK : nullptr;
-    if constexpr (SF) phase_to_gates(sb + OFF_IN0, tid);
-    gate_pass<GK>(sb, sb + OFF_IN0, 0, Lc, tid, bg_row, H * DK);
-#ifdef CKDA_TC_DEBUG
-    const long long t_gp1 = clock64();
-#endif
-    fence_proxy_async_smem();
-    __syncthreads();
-#ifdef CKDA_TC_DEBUG
-    if (g_tc_time2 != nullptr && lane == 0 && blockIdx.x == 0) {
-      atomicAdd(g_tc_time2 + 8 + warp, (unsigned long long)(t_gp1 - t_gp0));
-      atomicAdd(g_tc_time2 + 24 + warp, (unsigned long long)(clock64() - t_gp1));
-    }
-#endif
-    if (tid == 0) {
-      tc_fence_after();
-      level_mmas(0);
-      if (more) issue_in(0, nxt);
-    }
-    pend_lv = 1;
-    if (more) pend_in0 = 1;
     if (tid < C) beta_next = load_beta(nxt);
     if constexpr (G2) {
-      // the next unit's erase and write gates are read with plain loads (in
-      // its gate passes and V conversion): pull their rows into L2 now, one
-      // 128-byte line per thread (64 rows x 4 lines of b, 4 of w)
-      const int r = tid >> 3, part = tid & 7;
-      if (more && r < nxt.Lc) {
-        const size_t row = (size_t)(nxt.t0 + r) * H + nxt.h;
-        if (part < 4)
-          prefetch_l2(bg + row * DK + 32 * part);
-        else if (32 * (part - 4) < DV)
-          prefetch_l2(wg + row * DV + 32 * (part - 4));
+      // Z = w * V (fp16) for the carry kernel: row tid / 4, a quarter of d_v
+      // per thread; rows past the chunk's end are zero
+      constexpr int NC = DV / 4;
+      const int r = tid >> 2, c0 = NC * (tid & 3);
+      __half* dst = ws_v + (u * C + r) * DV + c0;
+      const size_t src = ((size_t)(cur.t0 + r) * H + cur.h) * DV + c0;
+#pragma unroll
+      for (int e = 0; e < NC; e += 8) {
+        uint4 pk = make_uint4(0u, 0u, 0u, 0u);
+        if (r < Lc) {
+          float f[8];
+          load8_f32(vg + src + e, f);
+          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wg + src + e));
+          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wg + src + e + 4));
+          pk.x = pack_f16x2(f[0] * w0.x, f[1] * w0.y);
+          pk.y = pack_f16x2(f[2] * w0.z, f[3] * w0.w);
+          pk.z = pack_f16x2(f[4] * w1.x, f[5] * w1.y);
+          pk.w = pack_f16x2(f[6] * w1.z, f[7] * w1.w);
+        }
+        *reinterpret_cast<uint4*>(dst + e) = pk;
       }
     }
-    TC_MARK(1);
 
-    // ---- gate pass, half 1 (after the half-0 level GEMMs release the operands)
-    ok = wait(bar_in1, ph_in1, pend_in1);
-    ok = wait(bar_lv, ph_lv, pend_lv) && ok;
-    if (tid == 0) bulk_wait_read_all();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    if constexpr (SF) phase_to_gates(sb + OFF_IN1, tid);
-    gate_pass<GK>(sb, sb + OFF_IN1, 1, Lc, tid, G2 ? bg_row + HC : nullptr, H * DK);
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tc_fence_after();
-      level_mmas(1);
-      if (more) issue_in(1, nxt);
-      // K * rho is complete: store it to the workspace
-      tma_store_2d(&tm_kh, sb + OFF_KH, 0, (int)(u * C));
-      tma_store_2d(&tm_kh, sb + OFF_KH + 8192, 64, (int)(u * C));
-      bulk_commit();
+    // ---- T (fp32) and A (fp16 operand) from levels 2..5, direct pairs, diag(A)
+    ok = wait(bar_lv0, ph_lv[0], pend_lv[0]);
+    ok = wait(bar_lv0 + 8, ph_lv[1], pend_lv[1]) && ok;
+    // A's operand tile lies over level operands the GEMMs have now read: zero
+    // it (entries above the diagonal stay zero)
+    {
+      uint4* aq = reinterpret_cast<uint4*>(sm + F2_AQ);
+      aq[tid] = make_uint4(0u, 0u, 0u, 0u);
+      aq[tid + NT3] = make_uint4(0u, 0u, 0u, 0u);
     }
-    pend_lv = 1;
-    if (more) pend_in1 = 1;
-    TC_MARK(2);
-    ok = wait(bar_lv, ph_lv, pend_lv);
-    ok = wait(bar_v, ph_v, pend_v) && ok;
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    TC_MARK(3);
-
-    // ---- T and A (fp32) from levels 2..5, the direct pairs and diag(A) -------
-    // Every strictly-lower entry of T and every lower entry of A is written
-    // exactly once; the rest is never read (T) or masked on conversion (A).
     {
-      float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
-      float* Af = reinterpret_cast<float*>(sm + OFF_AF);
-      if (warp < 8) {
-        // warp (lane quarter q4, pair warp/4): one 32-column block of a pair
+      float* Tf = reinterpret_cast<float*>(sm + F2_TF);
+      // warp (lane quarter q4, pair warp / 4): one 32-column block of a pair
+      {
         const int pr = warp >> 2;
-        const int L = 32 * q4 + lane;  // lane of the pair accumulators
+        const int L = 32 * q4 + lane;
         const int rho = L & 63;
         const int rr = rho & 31;
-        float* dst = (rho < 32) ? Tf : Af;
         const int lv = 2 + 2 * pr + (L >> 6);
         float v[32];
-        tmem_ld32(taddr(tmem, 32 * q4, TM_LV + 64 * pr + 32 * (q4 >> 1)), v);
+        tmem_ld32(taddr(tmem, 32 * q4, TM3_LV + 64 * pr + 32 * (q4 >> 1)), v);
         tmem_ld_wait();
         const int b = 1 << lv;
         const int j = rr >> lv;
         const int r = 2 * b * j + b + (rr & (b - 1));
 #pragma unroll
         for (int m4 = 0; m4 < 8; ++m4) {
-          if (((4 * m4) >> lv) == j)
-            *reinterpret_cast<float4*>(dst + fsw(r, b * j + 4 * m4)) =
-                make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
+          if (((4 * m4) >> lv) == j) {
+            const int s = b * j + 4 * m4;
+            if (rho < 32) {
+              *reinterpret_cast<float4*>(Tf + fsw(r, s)) =
+                  make_float4(v[4 * m4], v[4 * m4 + 1], v[4 * m4 + 2], v[4 * m4 + 3]);
+            } else {
+              uint2 pk;
+              pk.x = pack_f16x2(v[4 * m4], v[4 * m4 + 1]);
+              pk.y = pack_f16x2(v[4 * m4 + 2], v[4 * m4 + 3]);
+              *reinterpret_cast<uint2*>(sm + F2_AQ + sw128_elem(r, s, 64)) = pk;
+            }
+          }
         }
-      } else {
-        // direct pairs (r, s) inside aligned blocks of 4, and the diagonal of A
-        const float* pr = reinterpret_cast<const float*>(sm + OFF_PR);
-        const int e = tid - 256;
-        const int g = e >> 4, w = e & 15;
-        const float val = pr[e];
+      }
+      // direct pairs (r, s) inside aligned blocks of 4, and the diagonal of A
+      {
+        const float* prb = reinterpret_cast<const float*>(sm + F2_PR);
+        const int g = tid >> 4, w = tid & 15;
+        const float val = prb[tid];
+        int r, s;
         if (w < 12) {
           const int jj = w >> 1;
           // pair order inside the block: (1,0) (2,0) (2,1) (3,0) (3,1) (3,2)
-          const int rl = (jj == 0) ? 1 : (jj < 3 ? 2 : 3);
-          const int sl = (jj == 0 || jj == 1 || jj == 3) ? 0 : (jj == 2 || jj == 4 ? 1 : 2);
-          const int r = 4 * g + rl, s = 4 * g + sl;
-          if (w & 1)
-            Af[fsw(r, s)] = val;
-          else
-            Tf[fsw(r, s)] = G2 ? val : beta_s[r] * val;
+          r = 4 * g + ((jj == 0) ? 1 : (jj < 3 ? 2 : 3));
+          s = 4 * g + ((jj == 0 || jj == 1 || jj == 3) ? 0 : (jj == 2 || jj == 4 ? 1 : 2));
         } else {
-          const int r = 4 * g + (w - 12);
-          Af[fsw(r, r)] = val;
+          r = s = 4 * g + (w - 12);
         }
-      }
-      // v tile: bf16 (as loaded) -> fp16 in place (G2: Z = w * v); rows past
-      // the end -> 0.  Each 16-byte chunk stays within its 128-byte row under
-      // the swizzle.
-      uint4* vt = reinterpret_cast<uint4*>(sm + OFF_V);
-      for (int e = tid; e < C * 8 * (DV / 64); e += NT1) {
-        uint4 raw = vt[e];
-        const int row = (e >> 3) & 63;
-        if (row < Lc) {
-          float f[8];
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 x2 = __bfloat1622float2(p2[t]);
-            f[2 * t] = x2.x;
-            f[2 * t + 1] = x2.y;
-          }
-          if constexpr (G2) {
-            // logical columns of this chunk: atom * 64 + 8 * (chunk ^ (row % 8))
-            const int col = 64 * (e >> 9) + 8 * ((e & 7) ^ (row & 7));
-            const float* wp = wg + ((size_t)(cur.t0 + row) * H + cur.h) * DV + col;
-            const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
-            const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp + 4));
-            f[0] *= w0.x; f[1] *= w0.y; f[2] *= w0.z; f[3] *= w0.w;
-            f[4] *= w1.x; f[5] *= w1.y; f[6] *= w1.z; f[7] *= w1.w;
-          }
-          raw.x = pack_f16x2(f[0], f[1]);
-          raw.y = pack_f16x2(f[2], f[3]);
-          raw.z = pack_f16x2(f[4], f[5]);
-          raw.w = pack_f16x2(f[6], f[7]);
-        } else {
-          raw = make_uint4(0u, 0u, 0u, 0u);
-        }
-        vt[e] = raw;
+        if (w < 12 && !(w & 1))
+          Tf[fsw(r, s)] = G2 ? val : beta_s[r] * val;
+        else
+          *reinterpret_cast<__half*>(sm + F2_AQ + sw128_elem(r, s, 64)) = __float2half_rn(val);
       }
     }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    TC_DBG(for (int e = tid; e < 4096; e += NT1) {
-      g_tc_dbg[e] = reinterpret_cast<const float*>(sm + OFF_TF)[fsw(e >> 6, e & 63)];
-      g_tc_dbg[4096 + e] = reinterpret_cast<const float*>(sm + OFF_AF)[fsw(e >> 6, e & 63)];
-    });
-    TC_MARK(4);
 
-    // ---- A -> fp16 operand; (I + T)^-1 by recursive doubling ------------------
+    // ---- (I + T)^-1 by recursive doubling -------------------------------------------
     {
-      const float* Af = reinterpret_cast<const float*>(sm + OFF_AF);
-      const float* Tf = reinterpret_cast<const float*>(sm + OFF_TF);
-      float* Inv = reinterpret_cast<float*>(sm + OFF_INV);
-      float* Yf = reinterpret_cast<float*>(sm + OFF_YF);
-      // One phase: A to its fp16 operand (one 8-column chunk per thread);
-      // zeros above the 8 x 8 block diagonal of Inv (what the merges read
-      // before they write it); the 8 x 8 diagonal blocks by forward
-      // substitution, one column per thread.
-      {
-        const int r = tid >> 3, cg = tid & 7;
-        const float4 lo = *reinterpret_cast<const float4*>(Af + fsw(r, 8 * cg));
-        const float4 hi = *reinterpret_cast<const float4*>(Af + fsw(r, 8 * cg + 4));
-        const float a8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        float v[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) v[t] = (8 * cg + t <= r) ? a8[t] : 0.f;
-        st_chunk8(sm + OFF_AQ, sw128_chunk(r, 8 * cg, 64), v);
-      }
-      for (int e = tid; e < 64 * 16; e += NT1) {
+      const float* Tf = reinterpret_cast<const float*>(sm + F2_TF);
+      float* Inv = reinterpret_cast<float*>(sm + F2_INV);
+      float* Yf = reinterpret_cast<float*>(sm + F2_YF);
+      for (int e = tid; e < 64 * 16; e += NT3) {
         const int r = e >> 4, c4 = e & 15;
         if (c4 >= 2 * (r >> 3) + 2)
           *reinterpret_cast<float4*>(Inv + fsw(r, 4 * c4)) = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -1094,35 +1053,34 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         for (int r2 = 0; r2 < 8; ++r2) Inv[fsw(base + r2, base + cc)] = x[r2];
       }
       __syncthreads();
-      inv_merge<8>(Tf, Inv, Yf, tid);
-      inv_merge<16>(Tf, Inv, Yf, tid);
-      inv_merge<32>(Tf, Inv, Yf, tid);
-      TC_DBG(for (int e = tid; e < 4096; e += NT1) g_tc_dbg[8192 + e] = Inv[fsw(e >> 6, e & 63)]);
-      // Inv diag(beta) (G2: Inv) -> rows 0..63 of the stacked operand
-      {
-        const int r = tid >> 3, cg = tid & 7;
+      inv_merge_n<8, NT3>(Tf, Inv, Yf, tid);
+      inv_merge_n<16, NT3>(Tf, Inv, Yf, tid);
+      inv_merge_n<32, NT3>(Tf, Inv, Yf, tid);
+      // Inv diag(beta) -> rows 0..63 of the stacked operand (over T, now unused)
+#pragma unroll
+      for (int rep = 0; rep < 2; ++rep) {
+        const int r = 32 * rep + (tid >> 3), cg = tid & 7;
         const float4 lo = *reinterpret_cast<const float4*>(Inv + fsw(r, 8 * cg));
         const float4 hi = *reinterpret_cast<const float4*>(Inv + fsw(r, 8 * cg + 4));
         const float i8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
         float v[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) v[t] = G2 ? i8[t] : i8[t] * beta_s[8 * cg + t];
-        st_chunk8(sm + OFF_IP, sw128_chunk(r, 8 * cg, 128), v);
+        st_chunk8(sm + F2_IP, sw128_chunk(r, 8 * cg, 128), v);
       }
     }
     fence_proxy_async_smem();
     __syncthreads();
-    TC_MARK(5);
 
-    // ---- P = A Inv diag(beta) ---------------------------------------------------
+    // ---- P = A Inv diag(beta) ---------------------------------------------------------
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_f16(64, 64, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(sb + OFF_AQ + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF_IP + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM_P, ad, bd, id, kk > 0 ? 1u : 0u);
+        const uint64_t ad = smem_desc(sb + F2_AQ + kk * 32, 16, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(sb + F2_IP + kk * 2048, 8192, 1024, kSwizzle128);
+        mma_f16(tmem + TM3_P, ad, bd, id, kk > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
     }
@@ -1133,122 +1091,98 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     tc_fence_after();
     {
       // M = 64 accumulator: row 16 * q4 + l sits in lane l (< 16) of quarter q4
-      float v[16];
-      tmem_ld16(taddr(tmem, 32 * q4, TM_P + 16 * quarter), v);
+      float v[32];
+      tmem_ld32(taddr(tmem, 32 * q4, TM3_P + 32 * quarter), v);
       tmem_ld_wait();
       if (lane < 16) {
         const int rho = 16 * q4 + lane;
 #pragma unroll
-        for (int c8 = 0; c8 < 2; ++c8)
-          st_chunk8(sm + OFF_IP, sw128_chunk(64 + rho, 16 * quarter + 8 * c8, 128), v + 8 * c8);
-        TC_DBG(for (int e = 0; e < 16; ++e) g_tc_dbg[12288 + rho * 64 + 16 * quarter + e] = v[e]);
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk8(sm + F2_IP, sw128_chunk(64 + rho, 32 * quarter + 8 * c8, 128), v + 8 * c8);
       }
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-    TC_MARK(6);
 
-    // ---- [W, U~; A W, A U~] = [Inv diag(beta); P] [K Gamma, V] ----------------
+    // ---- [W; A W] = [Inv diag(beta); P] (K Gamma) ----------------------------------------
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t id1 = idesc_f16(128, 128, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(sb + OFF_IP + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF_KG + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM_W, ad, bd, id1, kk > 0 ? 1u : 0u);
+        const uint64_t ad = smem_desc(sb + F2_IP + kk * 32, 16, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(sb + F2_KG + kk * 2048, 8192, 1024, kSwizzle128);
+        mma_f16(tmem + TM3_W, ad, bd, id1, kk > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
-      // [Inv diag(beta); P] and the fp16 V tile are final: store them (the
-      // carry kernel forms [U~; A U~] from them)
-      const int yu = (int)(u * 2 * C);
-      tma_store_2d(&tm_ip, sb + OFF_IP, 0, yu);
-#pragma unroll
-      for (int a = 0; a < DV / 64; ++a)
-        tma_store_2d(&tm_v16, sb + OFF_V + 8192 * a, 64 * a, (int)(u * C));
+      tma_store_2d(&tm_ip, sb + F2_IP, 0, (int)(u * 2 * C));
       bulk_commit();
     }
     pend_mma = 1;
     ok = wait(bar_mma, ph_mma, pend_mma);
-    // K * rho has been read out (the stores just issued may still read):
-    // its tile takes -W next
-    if (tid == 0) bulk_wait_read_all_but_last();
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
-    TC_MARK(7);
 
-    // ---- [-W; Q' = Q Gamma - A W] and gamma -> workspace ------------------------
-    // Each thread holds 32 columns of one tensor-memory row of [W; A W]; the
-    // rows go to 128B-swizzled staging (conflict-free), which TMA stores.
+    // ---- [-W; Q' = Q Gamma - A W] -> workspace -------------------------------------------
     {
       const int L = 32 * q4 + lane;
-      float v[32];
-      tmem_ld32(taddr(tmem, 32 * q4, TM_W + 32 * quarter), v);
-      tmem_ld_wait();
-      TC_DBG(for (int e = 0; e < 32; ++e) g_tc_dbg[16384 + L * 128 + 32 * quarter + e] = v[e]);
-      // -W rows -> the K * rho tile; Q' rows replace Q * Gamma in place
       const int r = L & 63;
-      const uint32_t dst = (L < 64) ? OFF_KH : OFF_QG;
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        const uint32_t off = dst + sw128_chunk(r, 32 * quarter + 8 * c8, 64);
-        float w8[8];
-        if (L >= 64) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(sm + off);
-          const __half2* p2 = reinterpret_cast<const __half2*>(&raw);
+      for (int cb = 0; cb < 2; ++cb) {
+        const int col0 = 64 * quarter + 32 * cb;
+        float v[32];
+        tmem_ld32(taddr(tmem, 32 * q4, TM3_W + col0), v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 f = __half22float2(p2[t]);
-            w8[2 * t] = f.x - v[8 * c8 + 2 * t];
-            w8[2 * t + 1] = f.y - v[8 * c8 + 2 * t + 1];
+        for (int c8 = 0; c8 < 4; ++c8) {
+          float w8[8];
+          if (L >= 64) {
+            const uint32_t off = F2_QG + sw128_chunk(r, col0 + 8 * c8, 64);
+            const uint4 raw = *reinterpret_cast<const uint4*>(sm + off);
+            const __half2* p2 = reinterpret_cast<const __half2*>(&raw);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const float2 f = __half22float2(p2[t]);
+              w8[2 * t] = f.x - v[8 * c8 + 2 * t];
+              w8[2 * t + 1] = f.y - v[8 * c8 + 2 * t + 1];
+            }
+            st_chunk8(sm, off, w8);
+          } else {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) w8[t] = -v[8 * c8 + t];
+            st_chunk8(sm, F2_WS + sw128_chunk(r, col0 + 8 * c8, 64), w8);
           }
-        } else {
-#pragma unroll
-          for (int t = 0; t < 8; ++t) w8[t] = -v[8 * c8 + t];
         }
-        st_chunk8(sm, off, w8);
       }
-      if (tid < DK) ws_g[u * DK + tid] = gamma_s[tid];
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-      // channels 0..63 first: the next unit's first gate pass reuses only
-      // those atoms and waits for this group alone
       const int y = (int)(u * 2 * C);
-      tma_store_2d(&tm_wq, sb + OFF_KH, 0, y);
-      tma_store_2d(&tm_wq, sb + OFF_QG, 0, y + C);
-      bulk_commit();
-      tma_store_2d(&tm_wq, sb + OFF_KH + 8192, 64, y);
-      tma_store_2d(&tm_wq, sb + OFF_QG + 8192, 64, y + C);
+      tma_store_2d(&tm_wq, sb + F2_WS, 0, y);
+      tma_store_2d(&tm_wq, sb + F2_WS + 8192, 64, y);
+      tma_store_2d(&tm_wq, sb + F2_QG, 0, y + C);
+      tma_store_2d(&tm_wq, sb + F2_QG + 8192, 64, y + C);
       bulk_commit();
     }
-    TC_MARK(8);
     cur = nxt;
   }
-#ifdef CKDA_TC_DEBUG
-  if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-    for (int k = 0; k < 9; ++k) g_tc_time[k] = tmark[k];
-#endif
   if (tid == 0) bulk_wait_all();
-
   if (!ok) {
     if (tid == 0) {
       set_status(status, CKDA_ERR_DEVICE_TIMEOUT);
-      // wait (bounded) for copies and tensor-core work this CTA still has in flight
-      if (pend_in0) mbar_wait_bounded(bar_in0, ph_in0, kWaitNs);
-      if (pend_in1) mbar_wait_bounded(bar_in1, ph_in1, kWaitNs);
-      if (pend_v) mbar_wait_bounded(bar_v, ph_v, kWaitNs);
+      if (pend_in) mbar_wait_bounded(bar_in, ph_in, kWaitNs);
+      if (pend_lv[0]) mbar_wait_bounded(bar_lv0, ph_lv[0], kWaitNs);
+      if (pend_lv[1]) mbar_wait_bounded(bar_lv0 + 8, ph_lv[1], kWaitNs);
       if (pend_mma) mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
-      if (pend_lv) mbar_wait_bounded(bar_lv, ph_lv, kWaitNs);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, kF2TmemCols);
 }
 
 // ---- kernel 2: the chunk-to-chunk carry ---------------------------------------------
@@ -1267,7 +1201,16 @@ factor_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // transfer matrix), the B columns start from zero (the zero-start state);
 // nothing is output and the end state goes to summ[n, g] ([N, seg_launch, H,
 // DK, DK + DV] fp32).  seg_n = seg_launch = 1 is the plain forward.
-template <typename Tout, bool SF>
+//
+// VIN: V comes from the bf16 input itself (tm_v16 then maps the input v,
+// [rows, H * d_v]) and is converted to fp16 in the stage, rows past the
+// chunk's end set to zero; the [-W; Q'] S part of carry 1 runs meanwhile.
+// Otherwise V is the factor kernel's fp16 copy in the workspace.
+//
+// NBV: the d_v columns of one CTA, 64 or 32 (narrower slices put more CTAs
+// on the GPU when there are few (sequence, head) pairs, as in one long
+// sequence); each thread holds NBV / 2 columns of one state row.
+template <typename Tout, bool SF, bool VIN, int NBV>
 __global__ void __launch_bounds__(NT, 1)
 carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
              const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
@@ -1283,7 +1226,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int j0 = blockIdx.x * BV;
+  constexpr int CPT = NBV / 2;  // state columns per thread
+  const int j0 = blockIdx.x * NBV;
   const int h = blockIdx.y;
   const int n = blockIdx.z / seg_launch;
   const int seg = blockIdx.z % seg_launch;
@@ -1320,25 +1264,25 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   long long tlast = clock64();
 #endif
 
-  // State slice: row i = 32 * (warp % 4) + lane, columns [32 * (warp / 4), +32).
+  // State slice: row i = 32 * (warp % 4) + lane, columns [CPT * (warp / 4), +CPT).
   const int q4 = warp & 3;
   const int half = warp >> 2;
   const int srow = 32 * q4 + lane;
-  const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + 32 * half;
-  // this thread's 32 start values (row srow, 32 columns)
+  const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + CPT * half;
+  // this thread's CPT start values (row srow, CPT columns)
   const float* s_row = nullptr;
   if (seg == 0) {
     if (S0 != nullptr) s_row = S0 + s_off;
   } else {
-    s_row = seg_start + ((((size_t)n * seg_n + seg) * H + h) * DK + srow) * DV + j0 + 32 * half;
+    s_row = seg_start + ((((size_t)n * seg_n + seg) * H + h) * DK + srow) * DV + j0 + CPT * half;
   }
-  float S[32];
+  float S[CPT];
 #pragma unroll
-  for (int e = 0; e < 32; e += 4) {
+  for (int e = 0; e < CPT; e += 4) {
     float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (summary) {
       if (mcols) {
-        const int c = j0 + 32 * half + e - srow;  // identity: 1 where column == row
+        const int c = j0 + CPT * half + e - srow;  // identity: 1 where column == row
         v4 = make_float4(c == 0 ? 1.f : 0.f, c == -1 ? 1.f : 0.f, c == -2 ? 1.f : 0.f,
                          c == -3 ? 1.f : 0.f);
       }
@@ -1348,8 +1292,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     S[e] = v4.x; S[e + 1] = v4.y; S[e + 2] = v4.z; S[e + 3] = v4.w;
   }
 #pragma unroll
-  for (int c4 = 0; c4 < 4; ++c4)
-    st_chunk8(sm + OFF2_SB, sw128_chunk(srow, 32 * half + 8 * c4, 128), S + 8 * c4);
+  for (int c4 = 0; c4 < CPT / 8; ++c4)
+    st_chunk8(sm + OFF2_SB, sw128_chunk(srow, CPT * half + 8 * c4, 128), S + 8 * c4);
   fence_proxy_async_smem();
 
   const int64_t tok0 = sr.begin;
@@ -1383,7 +1327,11 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), bar);
     tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), bar);
     tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), bar);
-    tma_load_2d(base + CS_V, &tm_v16, mcols ? 0 : jv, (int)(uidx * C), bar);
+    if constexpr (VIN)
+      tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
+                  (int)(tok0 + (int64_t)(cbeg + c) * C), bar);
+    else
+      tma_load_2d(base + CS_V, &tm_v16, mcols ? 0 : jv, (int)(uidx * C), bar);
   };
   if (tid == 0) {
     if (nchunks > 0) issue(0, 0);
@@ -1399,39 +1347,79 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     return SF ? *reinterpret_cast<const float2*>(gp) : make_float2(*gp, 0.f);
   };
   float2 gm = load_gamma(0);
+  // VIN: bf16 V (as loaded) -> fp16 in place in stage `s`, rows past the
+  // chunk's `len` tokens -> 0.  Each 16-byte chunk stays within its 128-byte
+  // row under the swizzle.  The V of chunk c + 1 is converted while carry 2
+  // of chunk c runs (its stage wait moves there), so carry 1 finds it ready.
+  const bool v_early = VIN && !mcols;
+  auto chunk_len = [&](int c) -> int {
+    const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
+    return (tok1 - t0c < (int64_t)C) ? (int)(tok1 - t0c) : C;
+  };
+  auto convert_v = [&](int s, int len) {
+    uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
+    for (int e = tid; e < C * 8; e += NT) {
+      uint4 raw = vt[e];
+      if ((e >> 3) < len) {
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+        uint32_t o[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 x2 = __bfloat1622float2(p2[t]);
+          o[t] = pack_f16x2(x2.x, x2.y);
+        }
+        raw = make_uint4(o[0], o[1], o[2], o[3]);
+      } else {
+        raw = make_uint4(0u, 0u, 0u, 0u);
+      }
+      vt[e] = raw;
+    }
+  };
+  if (v_early && nchunks > 0) {
+    ok = wait(bar_full0, ph0, pend0);
+    if (ok) convert_v(0, chunk_len(0));
+    fence_proxy_async_smem();
+  }
   __syncthreads();
 
   for (int c = 0; c < nchunks; ++c) {
     const int st = c & 1;
     const int64_t t0 = tok0 + (int64_t)(cbeg + c) * C;
-    const int Lc = (tok1 - t0 < (int64_t)C) ? (int)(tok1 - t0) : C;
+    const int Lc = chunk_len(c);
     const uint32_t stage = sb + st * kStageBytes;
-    const bool tma_out = !summary && ((cu == nullptr) || Lc == C);
-    ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
+    // (the bf16 output map's box is 64 columns wide: a 32-column slice stores
+    // its rows with plain stores)
+    const bool tma_out =
+        !summary && ((cu == nullptr) || Lc == C) && (NBV == 64 || sizeof(Tout) == 4);
+    if (!v_early) ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
     ok = __syncthreads_and(ok);
     if (!ok) break;
     const float2 gm_next = load_gamma(c + 1);
     TC_MARK(9);
 
     // ---- carry 1: [U; O] = [Inv diag(beta); P] V + [-W; Q'] S -------------------
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, 64, 0, 1);
-      if (!mcols) {
+    constexpr uint32_t id_c1 = idesc_f16(128, NBV, 0, 1);
+    auto mma_v = [&](uint32_t acc0) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ad = smem_desc(stage + CS_IP + kk * 32, 16, 1024, kSwizzle128);
-          const uint64_t bd = smem_desc(stage + CS_V + kk * 2048, 8192, 1024, kSwizzle128);
-          mma_f16(tmem + TM2_X, ad, bd, id, kk > 0 ? 1u : 0u);
-        }
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t ad = smem_desc(stage + CS_IP + kk * 32, 16, 1024, kSwizzle128);
+        const uint64_t bd = smem_desc(stage + CS_V + kk * 2048, 8192, 1024, kSwizzle128);
+        mma_f16(tmem + TM2_X, ad, bd, id_c1, (kk > 0 || acc0) ? 1u : 0u);
       }
+    };
+    auto mma_s = [&](uint32_t acc0) {
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint64_t ad =
             smem_desc(stage + CS_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
         const uint64_t bd = smem_desc(sb + OFF2_SB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_X, ad, bd, id, (mcols && kk == 0) ? 0u : 1u);
+        mma_f16(tmem + TM2_X, ad, bd, id_c1, (kk > 0 || acc0) ? 1u : 0u);
       }
+    };
+    if (tid == 0) {
+      tc_fence_after();
+      if (!mcols) mma_v(0u);
+      mma_s(mcols ? 0u : 1u);
       mma_commit(bar_mma);
     }
     pend_mma = 1;
@@ -1445,20 +1433,23 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
     // ---- U -> operand;  O -> out ---------------------------------------------------
     {
-      float x[32];
-      tmem_ld32(taddr(tmem, 32 * q4, TM2_X + 32 * half), x);
+      float x[CPT];
+      if constexpr (CPT == 32)
+        tmem_ld32(taddr(tmem, 32 * q4, TM2_X + CPT * half), x);
+      else
+        tmem_ld16(taddr(tmem, 32 * q4, TM2_X + CPT * half), x);
       tmem_ld_wait();
-      TC_DBG(for (int e = 0; e < 32; ++e) g_tc_dbg[32768 + srow * 64 + 32 * half + e] = x[e]);
+      TC_DBG(for (int e = 0; e < CPT; ++e) g_tc_dbg[32768 + srow * 64 + CPT * half + e] = x[e]);
       if (q4 < 2) {
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          st_chunk8(sm + OFF2_UB, sw128_chunk(srow, 32 * half + 8 * c4, 64), x + 8 * c4);
+        for (int c4 = 0; c4 < CPT / 8; ++c4)
+          st_chunk8(sm + OFF2_UB, sw128_chunk(srow, CPT * half + 8 * c4, 64), x + 8 * c4);
       } else if (!summary) {
         const int r = srow - 64;
         if (tma_out)
-          stage_row32<Tout>(sb + OFF2_OB, r, half, x);
+          stage_row<CPT>(sb + OFF2_OB, r, CPT * half, x, Tout());
         else if (r < Lc)
-          store_row32<Tout>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + 32 * half, x);
+          store_row<CPT>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + CPT * half, x);
       }
     }
     fence_proxy_async_smem();
@@ -1472,14 +1463,14 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const int y0 = (cbeg + c) * C;
         if (sizeof(Tout) == 4) {
           tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
-          tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, y0, n);
+          if (NBV == 64) tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, y0, n);
         } else {
           tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
         }
       } else {
         if (sizeof(Tout) == 4) {
           tma_store_2d(&tm_out, sb + OFF2_OB, x0, (int)t0);
-          tma_store_2d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, (int)t0);
+          if (NBV == 64) tma_store_2d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, (int)t0);
         } else {
           tma_store_2d(&tm_out, sb + OFF2_OB, x0, (int)t0);
         }
@@ -1491,7 +1482,7 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     // ---- carry 2: D = (K rho)^T U;  S <- Diag(gamma) S + D ----------------------
     if (tid == 0) {
       tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, 64, 1, 1);
+      constexpr uint32_t id = idesc_f16(128, NBV, 1, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t ad = smem_desc(stage + CS_KH + kk * 2048, 8192, 1024, kSwizzle128);
@@ -1501,7 +1492,12 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       mma_commit(bar_mma);
     }
     pend_mma = 1;
-    ok = wait(bar_mma, ph_mma, pend_mma);
+    // while carry 2 runs: the next chunk's stage, its V converted to fp16
+    if (v_early && c + 1 < nchunks) {
+      ok = st ? wait(bar_full0, ph0, pend0) : wait(bar_full0 + 8, ph1, pend1);
+      if (ok) convert_v(st ^ 1, chunk_len(c + 1));
+    }
+    ok = wait(bar_mma, ph_mma, pend_mma) && ok;
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
@@ -1514,33 +1510,37 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         pend0 = 1;
     }
     {
-      float d[32];
-      tmem_ld32(taddr(tmem, 32 * q4, TM2_D + 32 * half), d);
+      float d[CPT];
+      if constexpr (CPT == 32)
+        tmem_ld32(taddr(tmem, 32 * q4, TM2_D + CPT * half), d);
+      else
+        tmem_ld16(taddr(tmem, 32 * q4, TM2_D + CPT * half), d);
       tmem_ld_wait();
       if constexpr (SF) {
         // even row: gr S_e - gi S_o + d;  odd row: gr S_o + gi S_e + d
         const float gi = (lane & 1) ? gm.y : -gm.y;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
+        for (int e = 0; e < CPT; ++e) {
           const float po = __shfl_xor_sync(0xffffffffu, S[e], 1);
           S[e] = fmaf(gm.x, S[e], fmaf(gi, po, d[e]));
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) S[e] = fmaf(gm.x, S[e], d[e]);
+        for (int e = 0; e < CPT; ++e) S[e] = fmaf(gm.x, S[e], d[e]);
       }
-      TC_DBG(for (int e = 0; e < 32; ++e) {
-        g_tc_dbg[49152 + srow * 64 + 32 * half + e] = d[e];
-        g_tc_dbg[57344 + srow * 64 + 32 * half + e] = S[e];
+      TC_DBG(for (int e = 0; e < CPT; ++e) {
+        g_tc_dbg[49152 + srow * 64 + CPT * half + e] = d[e];
+        g_tc_dbg[57344 + srow * 64 + CPT * half + e] = S[e];
       });
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        st_chunk8(sm + OFF2_SB, sw128_chunk(srow, 32 * half + 8 * c4, 128), S + 8 * c4);
+      for (int c4 = 0; c4 < CPT / 8; ++c4)
+        st_chunk8(sm + OFF2_SB, sw128_chunk(srow, CPT * half + 8 * c4, 128), S + 8 * c4);
     }
     gm = gm_next;
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    ok = __syncthreads_and(ok);
+    if (!ok) break;
     TC_MARK(12);
   }
 #ifdef CKDA_TC_DEBUG
@@ -1552,13 +1552,13 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   if (ok) {
     if (summary) {
       float* dst = summ + (((size_t)n * seg_launch + seg) * H + h) * DK * (DK + DV) +
-                   (size_t)srow * (DK + DV) + j0 + 32 * half;
+                   (size_t)srow * (DK + DV) + j0 + CPT * half;
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
+      for (int e = 0; e < CPT; e += 4)
         *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
     } else if (S_final != nullptr && seg == seg_n - 1) {
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
+      for (int e = 0; e < CPT; e += 4)
         *reinterpret_cast<float4*>(S_final + s_off + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
     }
   } else {
@@ -1747,18 +1747,20 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
 
+  // Gated DeltaNet-2 keeps Z = w * V in the workspace (its write gate is
+  // applied there); the other gate families leave V to the carry kernel,
+  // which reads the bf16 input itself, and their V array stays unused.
+  constexpr bool kVin = GK != kGdn2;
   if (phases & kFactors) {
-    CUtensorMap mq, mk, mv, ma, mth, mwq64;
+    CUtensorMap mq, mk, ma, mth, mwq64;
     // SF: alpha and theta hold one value per channel pair (DK / 2 per head)
     const uint64_t a_cols = SF ? (uint64_t)H * (DK / 2) : (uint64_t)H * DK;
-    const uint32_t a_box = SF ? HC / 2 : HC;
+    const uint32_t a_box = SF ? HQ / 2 : HQ;
     const bool ok =
-        make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HC, C,
+        make_map(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HQ, C,
                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HC, C,
+        make_map(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DK, rows, HQ, C,
                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
-        make_map(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows, 64, C,
-                 CU_TENSOR_MAP_SWIZZLE_128B) &&
         make_map(&ma, alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a_cols, rows, a_box, C,
                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
         make_map(&mth, SF ? theta : alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a_cols, rows,
@@ -1766,27 +1768,37 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
         make_map(&mwq64, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
                  C, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    auto k1 = factor_kernel<DV, GK>;
+    // Two CTAs per SM (the largest shared-memory carveout); the persistent
+    // grid has two CTAs for every SM.  Measured on B200: the same grid of one
+    // CTA per SM takes 43 % longer.
+    auto k1 = factor2_kernel<DV, GK>;
     static bool attr1 = false;
     if (!attr1) {
-      cudaError_t e = set_smem(k1, kSmemBytes);
+      cudaError_t e = set_smem(k1, kF2SmemBytes);
+      if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(k1, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return e;
       attr1 = true;
     }
-    const int64_t g1 = nu < (int64_t)sm_count() ? nu : (int64_t)sm_count();
-    k1<<<(unsigned)g1, NT1, kSmemBytes, stream>>>(mq, mk, mv, ma, mth, mwq64, mkh, mip, mv16,
-                                                  beta, bg, wg, cu, n_seqs, T, H, nch, nu, ws_g,
-                                                  status);
+    const int64_t cap = 2 * (int64_t)sm_count();
+    const int64_t g1 = nu < cap ? nu : cap;
+    k1<<<(unsigned)g1, NT3, kF2SmemBytes, stream>>>(
+        mq, mk, ma, mth, mwq64, mip, beta, bg, wg, static_cast<const __nv_bfloat16*>(q),
+        static_cast<const __nv_bfloat16*>(k), alpha, theta, static_cast<const __nv_bfloat16*>(v),
+        cu, n_seqs, T, H, nch, nu, ws_kh, ws_v, ws_g, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-
   if (phases & kCarry) {
     constexpr bool kF32 = sizeof(Tout) == 4;
     const CUtensorMapDataType tout =
         kF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint32_t ob_cols = kF32 ? 32 : 64;
-    CUtensorMap mwq, mout;
+    CUtensorMap mwq, mout, mvin = mv16;
+    if (kVin && !make_map(&mvin, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows,
+                          64, C, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
     const bool ok =
         make_map(&mwq, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
                  2 * C, CU_TENSOR_MAP_SWIZZLE_128B) &&
@@ -1795,16 +1807,20 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
             : make_map3(&mout, out, tout, sizeof(Tout), (uint64_t)H * DV, (uint64_t)T,
                         (uint64_t)n_seqs, ob_cols, C, CU_TENSOR_MAP_SWIZZLE_128B));
     if (!ok) return cudaErrorInvalidValue;
-    auto k2 = carry_kernel<Tout, SF>;
-    static bool attr2 = false;
-    if (!attr2) {
+    // 32-column slices when 64-column ones would leave more than half of the
+    // SMs without a carry CTA (few (sequence, head) pairs: a long sequence)
+    const int cols = segs.summ != nullptr ? DK + DV : DV;
+    const int64_t ctas64 = (int64_t)(cols / BV) * H * n_seqs * segs.launch;
+    const bool narrow = 2 * ctas64 <= (int64_t)sm_count();
+    auto k2 = narrow ? carry_kernel<Tout, SF, kVin, 32> : carry_kernel<Tout, SF, kVin, 64>;
+    static bool attr2[2] = {false, false};
+    if (!attr2[narrow]) {
       cudaError_t e = set_smem(k2, kSmem2Bytes);
       if (e != cudaSuccess) return e;
-      attr2 = true;
+      attr2[narrow] = true;
     }
-    const int cols = segs.summ != nullptr ? DK + DV : DV;
-    dim3 grid(cols / BV, H, n_seqs * segs.launch);
-    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, mv16, mout, ws_g, S0, cu,
+    dim3 grid(cols / (narrow ? 32 : BV), H, n_seqs * segs.launch);
+    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, kVin ? mvin : mv16, mout, ws_g, S0, cu,
                                           static_cast<Tout*>(out), S_final, n_seqs, T, H, DV,
                                           nch, status, segs.n, segs.launch, segs.start,
                                           segs.summ);

@@ -170,16 +170,18 @@ CKDA_API int ckda_fwd_chunked_static(const void* q, const void* k, const void* v
  * for the tensor-core path only (sizes for which ckda_fwd_chunked_path
  * returns 1; otherwise CKDA_ERR_UNSUPPORTED).
  *
- * ckda_fwd_factors reads q, k, v, alpha and beta (layouts as in
- * ckda_fwd_chunked) and writes, for every chunk of every head, the
- * S0-independent WY factors into `workspace`: [-W; Q'], K * rho,
- * [Inv diag(beta); P] and V (fp16), gamma (fp32), from which the carry forms
- * [U~; A U~] = [Inv diag(beta); P] V ("Gated DeltaNet-2", Methodology section 3:
+ * ckda_fwd_factors reads q, k, alpha and beta (layouts as in
+ * ckda_fwd_chunked; v is accepted and not read) and writes, for every chunk
+ * of every head, the S0-independent WY factors into `workspace`: [-W; Q'],
+ * K * rho, [Inv diag(beta); P] (fp16) and gamma (fp32).  ckda_fwd_carry
+ * reads v itself and forms [U~; A U~] = [Inv diag(beta); P] V
+ * ("Gated DeltaNet-2", Methodology section 3:
  * the decay absorbed into the WY factors; "Semidirect Fourier Delta
  * Attention", "Principales Contribuciones" item 3: each chunk is an affine
  * map of the state, S_end = (Diag(gamma) - (K*rho)^T W) S + (K*rho)^T U~).
  * ckda_fwd_carry applies those maps chunk after chunk from S0 and writes
- * out and S_final.
+ * out and S_final; it reads v (the same tensor as the factor call's, layout
+ * as in ckda_fwd_chunked) and needs it non-NULL whenever there are tokens.
  *
  * Because the factors do not depend on S0, one factor call can serve
  * several carry calls with different initial states.  ckda_fwd_carry must
@@ -196,7 +198,7 @@ CKDA_API int ckda_fwd_factors(const void* q, const void* k, const void* v,
                               int d_k, int d_v, int chunk, int dtype,
                               void* workspace, size_t workspace_bytes, void* stream);
 
-CKDA_API int ckda_fwd_carry(const float* S0, const int32_t* cu_seqlens, void* out,
+CKDA_API int ckda_fwd_carry(const void* v, const float* S0, const int32_t* cu_seqlens, void* out,
                             float* S_final, int B, int T, int H, int d_k, int d_v,
                             int chunk, int dtype, int out_dtype, void* workspace,
                             size_t workspace_bytes, void* stream);

@@ -204,10 +204,11 @@ def test_two_phase_calls_validate_without_a_gpu(lib):
                                     a["ws"], a["ws_bytes"], None)
 
     def carry(**kw):
-        a = dict(S0=None, cu=None, out=P + 0x5000, S_final=None, B=1, T=128, H=1, dk=128, dv=128,
+        a = dict(v=P + 0x2000, S0=None, cu=None, out=P + 0x5000, S_final=None, B=1, T=128, H=1,
+                 dk=128, dv=128,
                  chunk=64, dtype=BF16, out_dtype=F32, ws=None, ws_bytes=0)
         a.update(kw)
-        return lib.ckda_fwd_carry(a["S0"], a["cu"], a["out"], a["S_final"], a["B"], a["T"], a["H"],
+        return lib.ckda_fwd_carry(a["v"], a["S0"], a["cu"], a["out"], a["S_final"], a["B"], a["T"], a["H"],
                                   a["dk"], a["dv"], a["chunk"], a["dtype"], a["out_dtype"], a["ws"],
                                   a["ws_bytes"], None)
 
@@ -218,6 +219,7 @@ def test_two_phase_calls_validate_without_a_gpu(lib):
     # each phase needs only its own tensors, and the workspace
     assert factors(q=None) == -1
     assert carry(out=None) == -1
+    assert carry(v=None) == -1
     assert factors() == -7
     assert carry() == -7
     assert factors(ws=WS, ws_bytes=need - 256) == -7

@@ -57,7 +57,7 @@ def test_two_phases_equal_one_call(ck, out_dtype, packed):
     ws = ck.fwd_factors(case.q, case.k, case.v, case.alpha, case.beta, cu_seqlens=cu)
     B = case.n_seqs
     T = case.q.shape[1]
-    out2, S2 = ck.fwd_carry(ws, B, T, case.H, 128, 128, S0=case.S0, cu_seqlens=cu,
+    out2, S2 = ck.fwd_carry(ws, case.v, B, T, case.H, 128, 128, S0=case.S0, cu_seqlens=cu,
                             out_dtype=out_dtype)
     assert ck.device_status() == 0
     assert torch.equal(out1.view(-1), out2.view(-1))
@@ -72,7 +72,7 @@ def test_one_factor_pass_serves_several_initial_states(ck):
         S0 = scale * case.S0
         ref_o, ref_S = ck.fwd_chunked(case.q, case.k, case.v, case.alpha, case.beta, S0=S0,
                                       out_dtype=torch.float32)
-        o, S = ck.fwd_carry(ws, B, T, H, 128, 128, S0=S0)
+        o, S = ck.fwd_carry(ws, case.v, B, T, H, 128, 128, S0=S0)
         assert torch.equal(o, ref_o) and torch.equal(S, ref_S), scale
     assert ck.device_status() == 0
 
