@@ -91,12 +91,11 @@ constexpr int kKda = 0;   // beta_r, Diag(alpha_r)
 constexpr int kGdn2 = 1;  // erase gate b_r, write gate w_r, Diag(alpha_r)
 constexpr int kSfda = 2;  // beta_r, phase-decay blocks alpha_p e^{i theta_p}
 
-// ---- workspace: per unit (one chunk of one head), five arrays -------------
+// ---- workspace: per unit (one chunk of one head), four arrays -------------
 constexpr size_t kWsWQ = (size_t)2 * C * DK * 2;  // [-W; Q'] fp16 [128][128]
 constexpr size_t kWsKH = (size_t)C * DK * 2;      // K * rho fp16 [64][128]
 constexpr size_t kWsIP = (size_t)2 * C * C * 2;   // [Inv diag(beta); P] fp16 [128][64]
 constexpr size_t kWsG = (size_t)DK * 4;           // gamma fp32 [128]
-// V as fp16 [64][d_v]: C * d_v * 2 bytes
 
 // ---- carry kernel: shared memory map ---------------------------------------
 // Two stages of one chunk's factors, each filled by one TMA transaction.
@@ -538,10 +537,6 @@ __device__ __noinline__ void gate_pass_q(uint32_t sb, int jq, int Lc, int tid,
     qa[u] = val ? bf4(lds_u2(in + F2_INQ + p * 64 + cl * 2)) : zero;
     if constexpr (!G2) bb[u] = lds_f(sb + F2_BETA + p * 4);
   }
-  if constexpr (G2) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) eg[u] = mul4x(eg[u], ka[u]);  // e = b * k
-  }
   // products of whole groups, and (one shuffle across neighbouring groups,
   // 8 lanes apart) of aligned pairs of groups
   const uint32_t gt = sb + F2_GT + cl * 4;
@@ -564,6 +559,10 @@ __device__ __noinline__ void gate_pass_q(uint32_t sb, int jq, int Lc, int tid,
     tma_load_2d(nx.dst + F2_INK, nx.tk, nx.x, nx.y, nx.bar);
     tma_load_2d(nx.dst + F2_INA, nx.ta, nx.xa, nx.y, nx.bar);
     if constexpr (SF) tma_load_2d(nx.dst + F2_INA + 4096, nx.tth, nx.xa, nx.y, nx.bar);
+  }
+  if constexpr (G2) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) eg[u] = mul4x(eg[u], ka[u]);  // e = b * k
   }
   auto gtot = [&](int gg) -> float4 { return lds_f4(gt + gg * 128); };
   auto run2 = [&](int s2) -> float4 { return lds_f4(sb + F2_T2 + s2 * 128 + cl * 4); };
@@ -698,7 +697,14 @@ __device__ __noinline__ void gate_pass_q(uint32_t sb, int jq, int Lc, int tid,
   }
 }
 
-// Recursive-doubling merge of the inverse (as inv_merge) for NTH threads.
+// One step of the recursive-doubling inverse of the unit lower-triangular
+// (I + T) with NTH threads: merge diagonal blocks of size M into blocks of
+// size 2M,
+//   [[A, 0], [B, D]]^-1 = [[A^-1, 0], [-D^-1 B A^-1, D^-1]],  B = T block.
+// Inv holds the inverses of the M-blocks and zeros above the block diagonal
+// (fsw layout, as T).  A^-1 and D^-1 are lower triangular, so the first
+// product only runs over rows t >= c of A^-1 and the second over t <= a of
+// D^-1.
 template <int M, int NTH>
 __device__ __forceinline__ void inv_merge_n(const float* Tf, float* Inv, float* Yf, int tid) {
   constexpr int NMERGE = 64 / (2 * M);
@@ -709,8 +715,8 @@ __device__ __forceinline__ void inv_merge_n(const float* Tf, float* Inv, float* 
     const int r0 = 2 * M * qb;
     const int tr = r0 + M + a;
     float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int t4 = 0; t4 < M / 4; ++t4) {
+#pragma unroll 2
+    for (int t4 = c4; t4 < M / 4; ++t4) {
       const float4 tv = *reinterpret_cast<const float4*>(Tf + fsw(tr, r0 + 4 * t4));
       const float tt[4] = {tv.x, tv.y, tv.z, tv.w};
 #pragma unroll
@@ -729,8 +735,8 @@ __device__ __forceinline__ void inv_merge_n(const float* Tf, float* Inv, float* 
     const int r0 = 2 * M * qb;
     const int ir = r0 + M + a;
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int t4 = 0; t4 < M / 4; ++t4) {
+#pragma unroll 2
+    for (int t4 = 0; t4 <= (a >> 2); ++t4) {
       const float4 dv = *reinterpret_cast<const float4*>(Inv + fsw(ir, r0 + M + 4 * t4));
       const float dd[4] = {dv.x, dv.y, dv.z, dv.w};
 #pragma unroll
@@ -748,23 +754,21 @@ __device__ __forceinline__ void inv_merge_n(const float* Tf, float* Inv, float* 
 }
 
 // ws_kh: K * rho fp16 [units * C][DK] (row-major), ws_g: gamma fp32 [units][DK].
-// kGdn2: erase gate bg (shaped like k) and write gate wg (shaped like v) in
-// place of beta; the factors are [-W; Q'] with W = Inv (E * Gamma) and
-// [Inv; A Inv], and Z = wg * V goes to ws_v (fp16 [units * C][DV]) for the
-// carry kernel.  kSfda: alpha and theta fp32 [rows, H * DK / 2] (tm_a,
-// tm_th); gamma is stored as (re, im) pairs.
-template <int DV, int GK>
+// kGdn2: erase gate bg (shaped like k) in place of beta on the key side; the
+// factors are [-W; Q'] with W = Inv (E * Gamma) and [Inv; A Inv] (the write
+// gate is applied to V by the carry kernel).  kSfda: alpha and theta fp32
+// [rows, H * DK / 2] (tm_a, tm_th); gamma is stored as (re, im) pairs.
+template <int GK>
 __global__ void __launch_bounds__(NT3, 2)
 factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_th,
                const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_ip,
                const float* __restrict__ beta, const float* __restrict__ bg,
-               const float* __restrict__ wg, const __nv_bfloat16* __restrict__ qg,
-               const __nv_bfloat16* __restrict__ kg, const float* __restrict__ ag,
-               const float* __restrict__ thg, const __nv_bfloat16* __restrict__ vg,
-               const int32_t* __restrict__ cu, int n_seqs,
-               int T, int H, int nch, int64_t n_units, __half* __restrict__ ws_kh,
-               __half* __restrict__ ws_v, float* __restrict__ ws_g, int* status) {
+               const __nv_bfloat16* __restrict__ qg, const __nv_bfloat16* __restrict__ kg,
+               const float* __restrict__ ag, const float* __restrict__ thg,
+               const int32_t* __restrict__ cu, int n_seqs, int T, int H, int nch,
+               int64_t n_units, __half* __restrict__ ws_kh, float* __restrict__ ws_g,
+               int* status) {
   constexpr bool G2 = GK == kGdn2;
   constexpr bool SF = GK == kSfda;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -848,10 +852,10 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   };
   // Pull a unit's input rows into L2, one 128-byte line per thread and step:
   // per token q, k (2 lines each), the gates (alpha: 4 lines; SFDA alpha and
-  // theta: 2 each), and for Gated DeltaNet-2 the erase gate (4), the write
-  // gate (DV / 32) and v (DV / 64), read with plain loads.
+  // theta: 2 each), and for Gated DeltaNet-2 the erase gate (4 lines), read
+  // with plain loads.
   auto prefetch_unit = [&](const Unit& uu) {
-    constexpr int NL = G2 ? 12 + DV / 32 + DV / 64 : 8;
+    constexpr int NL = G2 ? 12 : 8;
     if (uu.idx < 0) return;
     for (int e = tid; e < C * NL; e += NT3) {
       const int r = e / NL, li = e % NL;
@@ -869,12 +873,8 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         } else {
           a = ag + row * DK + 32 * (li - 4);
         }
-      } else if (li < 12) {
-        a = bg + row * DK + 32 * (li - 8);
-      } else if (li < 12 + DV / 32) {
-        a = wg + row * DV + 32 * (li - 12);
       } else {
-        a = vg + row * DV + 64 * (li - 12 - DV / 32);
+        a = bg + row * DK + 32 * (li - 8);
       }
       prefetch_l2(a);
     }
@@ -929,29 +929,6 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     if (!ok) break;
     if (tid < C) beta_next = load_beta(nxt);
-    if constexpr (G2) {
-      // Z = w * V (fp16) for the carry kernel: row tid / 4, a quarter of d_v
-      // per thread; rows past the chunk's end are zero
-      constexpr int NC = DV / 4;
-      const int r = tid >> 2, c0 = NC * (tid & 3);
-      __half* dst = ws_v + (u * C + r) * DV + c0;
-      const size_t src = ((size_t)(cur.t0 + r) * H + cur.h) * DV + c0;
-#pragma unroll
-      for (int e = 0; e < NC; e += 8) {
-        uint4 pk = make_uint4(0u, 0u, 0u, 0u);
-        if (r < Lc) {
-          float f[8];
-          load8_f32(vg + src + e, f);
-          const float4 w0 = __ldg(reinterpret_cast<const float4*>(wg + src + e));
-          const float4 w1 = __ldg(reinterpret_cast<const float4*>(wg + src + e + 4));
-          pk.x = pack_f16x2(f[0] * w0.x, f[1] * w0.y);
-          pk.y = pack_f16x2(f[2] * w0.z, f[3] * w0.w);
-          pk.z = pack_f16x2(f[4] * w1.x, f[5] * w1.y);
-          pk.w = pack_f16x2(f[6] * w1.z, f[7] * w1.w);
-        }
-        *reinterpret_cast<uint4*>(dst + e) = pk;
-      }
-    }
 
     // ---- T (fp32) and A (fp16 operand) from levels 2..5, direct pairs, diag(A)
     ok = wait(bar_lv0, ph_lv[0], pend_lv[0]);
@@ -1202,20 +1179,20 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // nothing is output and the end state goes to summ[n, g] ([N, seg_launch, H,
 // DK, DK + DV] fp32).  seg_n = seg_launch = 1 is the plain forward.
 //
-// VIN: V comes from the bf16 input itself (tm_v16 then maps the input v,
-// [rows, H * d_v]) and is converted to fp16 in the stage, rows past the
-// chunk's end set to zero; the [-W; Q'] S part of carry 1 runs meanwhile.
-// Otherwise V is the factor kernel's fp16 copy in the workspace.
+// V comes from the bf16 input itself (tm_v16 maps the input v, [rows,
+// H * d_v]) and is converted to fp16 in the stage, rows past the chunk's
+// end set to zero.  WG (Gated DeltaNet-2): the conversion multiplies V by
+// the write gate wg ([rows, H * d_v] fp32), giving Z = w * V.
 //
 // NBV: the d_v columns of one CTA, 64 or 32 (narrower slices put more CTAs
 // on the GPU when there are few (sequence, head) pairs, as in one long
 // sequence); each thread holds NBV / 2 columns of one state row.
-template <typename Tout, bool SF, bool VIN, int NBV>
+template <typename Tout, bool SF, bool WG, int NBV>
 __global__ void __launch_bounds__(NT, 1)
 carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
              const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
              const __grid_constant__ CUtensorMap tm_out,
-             const float* __restrict__ ws_g,
+             const float* __restrict__ ws_g, const float* __restrict__ wg,
              const float* S0, const int32_t* __restrict__ cu, Tout* __restrict__ out,
              float* S_final, int n_seqs, int T, int H, int DV, int nch, int* status,
              int seg_n, int seg_launch, const float* __restrict__ seg_start,
@@ -1327,11 +1304,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), bar);
     tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), bar);
     tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), bar);
-    if constexpr (VIN)
-      tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
-                  (int)(tok0 + (int64_t)(cbeg + c) * C), bar);
-    else
-      tma_load_2d(base + CS_V, &tm_v16, mcols ? 0 : jv, (int)(uidx * C), bar);
+    tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
+                (int)(tok0 + (int64_t)(cbeg + c) * C), bar);
   };
   if (tid == 0) {
     if (nchunks > 0) issue(0, 0);
@@ -1347,37 +1321,67 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     return SF ? *reinterpret_cast<const float2*>(gp) : make_float2(*gp, 0.f);
   };
   float2 gm = load_gamma(0);
-  // VIN: bf16 V (as loaded) -> fp16 in place in stage `s`, rows past the
-  // chunk's `len` tokens -> 0.  Each 16-byte chunk stays within its 128-byte
-  // row under the swizzle.  The V of chunk c + 1 is converted while carry 2
-  // of chunk c runs (its stage wait moves there), so carry 1 finds it ready.
-  const bool v_early = VIN && !mcols;
+  // bf16 V (as loaded) -> fp16 in place in stage `s` (WG: times the write
+  // gate), rows past the chunk's `len` tokens -> 0.  Each 16-byte chunk stays
+  // within its 128-byte row under the swizzle.  The V of chunk c + 1 is
+  // converted while carry 2 of chunk c runs (its stage wait moves there), so
+  // carry 1 finds it ready.
+  const bool v_early = !mcols;
   auto chunk_len = [&](int c) -> int {
     const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
     return (tok1 - t0c < (int64_t)C) ? (int)(tok1 - t0c) : C;
   };
-  auto convert_v = [&](int s, int len) {
+  auto convert_v = [&](int s, int c) {
+    const int len = chunk_len(c);
+    const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
     uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
     for (int e = tid; e < C * 8; e += NT) {
       uint4 raw = vt[e];
-      if ((e >> 3) < len) {
+      const int row = e >> 3;
+      if (row < len) {
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        uint32_t o[4];
+        float f[8];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const float2 x2 = __bfloat1622float2(p2[t]);
-          o[t] = pack_f16x2(x2.x, x2.y);
+          f[2 * t] = x2.x;
+          f[2 * t + 1] = x2.y;
         }
-        raw = make_uint4(o[0], o[1], o[2], o[3]);
+        if constexpr (WG) {
+          // logical columns of this 16-byte chunk: 8 * (chunk ^ (row % 8));
+          // only the slice's own NBV columns are used (and read)
+          const int col = 8 * ((e & 7) ^ (row & 7));
+          if (col < NBV) {
+            const float* wp = wg + ((size_t)(t0c + row) * H + h) * DV + jv + col;
+            const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
+            const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp + 4));
+            f[0] *= w0.x; f[1] *= w0.y; f[2] *= w0.z; f[3] *= w0.w;
+            f[4] *= w1.x; f[5] *= w1.y; f[6] *= w1.z; f[7] *= w1.w;
+          }
+        }
+        raw = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]), pack_f16x2(f[4], f[5]),
+                         pack_f16x2(f[6], f[7]));
       } else {
         raw = make_uint4(0u, 0u, 0u, 0u);
       }
       vt[e] = raw;
     }
   };
+  // WG: the write-gate rows of chunk c pulled into L2 (one 128-byte line per
+  // thread) a chunk before its conversion reads them
+  auto prefetch_w = [&](int c) {
+    if constexpr (WG) {
+      constexpr int LPR = NBV / 32;  // 128-byte lines per row
+      const int r = tid / LPR;
+      if (!mcols && c < nchunks && r < chunk_len(c))
+        prefetch_l2(wg + ((size_t)(tok0 + (int64_t)(cbeg + c) * C + r) * H + h) * DV + jv +
+                    32 * (tid % LPR));
+    }
+  };
   if (v_early && nchunks > 0) {
+    prefetch_w(1);
     ok = wait(bar_full0, ph0, pend0);
-    if (ok) convert_v(0, chunk_len(0));
+    if (ok) convert_v(0, 0);
     fence_proxy_async_smem();
   }
   __syncthreads();
@@ -1494,8 +1498,9 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     pend_mma = 1;
     // while carry 2 runs: the next chunk's stage, its V converted to fp16
     if (v_early && c + 1 < nchunks) {
+      prefetch_w(c + 2);
       ok = st ? wait(bar_full0, ph0, pend0) : wait(bar_full0 + 8, ph1, pend1);
-      if (ok) convert_v(st ^ 1, chunk_len(c + 1));
+      if (ok) convert_v(st ^ 1, c + 1);
     }
     ok = wait(bar_mma, ph_mma, pend_mma) && ok;
     ok = __syncthreads_and(ok);
@@ -1689,7 +1694,8 @@ int64_t n_units(bool varlen, int n_seqs, int T, int H) {
   return u > 0 ? u : 1;
 }
 
-size_t unit_bytes(int DV) { return kWsWQ + kWsKH + kWsIP + kWsG + (size_t)C * DV * 2; }
+// (the same for every d_v: V is read from the input by the carry kernel)
+size_t unit_bytes(int) { return kWsWQ + kWsKH + kWsIP + kWsG; }
 
 int sm_count() {
   int dev = 0, n = 0;
@@ -1729,28 +1735,23 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
   const int nch = (int)(((int64_t)T + C - 1) / C);
   const int64_t nu = n_units(cu != nullptr, n_seqs, T, H);
   // workspace arrays, in this order: [-W; Q'], K rho, [Inv diag(beta); P],
-  // V (fp16), gamma -- every one a multiple of 512 bytes per unit
+  // gamma -- every one a multiple of 512 bytes per unit
   uint8_t* w8 = static_cast<uint8_t*>(ws);
   __half* ws_wq = reinterpret_cast<__half*>(w8);
   __half* ws_kh = reinterpret_cast<__half*>(w8 + nu * kWsWQ);
   __half* ws_ip = reinterpret_cast<__half*>(w8 + nu * (kWsWQ + kWsKH));
-  __half* ws_v = reinterpret_cast<__half*>(w8 + nu * (kWsWQ + kWsKH + kWsIP));
-  float* ws_g =
-      reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH + kWsIP + (size_t)C * DV * 2));
+  float* ws_g = reinterpret_cast<float*>(w8 + nu * (kWsWQ + kWsKH + kWsIP));
 
-  CUtensorMap mkh, mip, mv16;
+  CUtensorMap mkh, mip;
   if (!make_map(&mkh, ws_kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * C, 64, C,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&mip, ws_ip, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, C, (uint64_t)nu * 2 * C, 64,
-                2 * C, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !make_map(&mv16, ws_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DV, (uint64_t)nu * C, 64, C,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+                2 * C, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
 
-  // Gated DeltaNet-2 keeps Z = w * V in the workspace (its write gate is
-  // applied there); the other gate families leave V to the carry kernel,
-  // which reads the bf16 input itself, and their V array stays unused.
-  constexpr bool kVin = GK != kGdn2;
+  // V never enters the workspace: the carry kernel reads the bf16 input
+  // itself (and applies Gated DeltaNet-2's write gate there).
+  constexpr bool G2 = GK == kGdn2;
   if (phases & kFactors) {
     CUtensorMap mq, mk, ma, mth, mwq64;
     // SF: alpha and theta hold one value per channel pair (DK / 2 per head)
@@ -1771,7 +1772,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
     // Two CTAs per SM (the largest shared-memory carveout); the persistent
     // grid has two CTAs for every SM.  Measured on B200: the same grid of one
     // CTA per SM takes 43 % longer.
-    auto k1 = factor2_kernel<DV, GK>;
+    auto k1 = factor2_kernel<GK>;
     static bool attr1 = false;
     if (!attr1) {
       cudaError_t e = set_smem(k1, kF2SmemBytes);
@@ -1784,9 +1785,9 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
     const int64_t cap = 2 * (int64_t)sm_count();
     const int64_t g1 = nu < cap ? nu : cap;
     k1<<<(unsigned)g1, NT3, kF2SmemBytes, stream>>>(
-        mq, mk, ma, mth, mwq64, mip, beta, bg, wg, static_cast<const __nv_bfloat16*>(q),
-        static_cast<const __nv_bfloat16*>(k), alpha, theta, static_cast<const __nv_bfloat16*>(v),
-        cu, n_seqs, T, H, nch, nu, ws_kh, ws_v, ws_g, status);
+        mq, mk, ma, mth, mwq64, mip, beta, bg, static_cast<const __nv_bfloat16*>(q),
+        static_cast<const __nv_bfloat16*>(k), alpha, theta, cu, n_seqs, T, H, nch, nu, ws_kh,
+        ws_g, status);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -1795,9 +1796,9 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
     const CUtensorMapDataType tout =
         kF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     const uint32_t ob_cols = kF32 ? 32 : 64;
-    CUtensorMap mwq, mout, mvin = mv16;
-    if (kVin && !make_map(&mvin, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows,
-                          64, C, CU_TENSOR_MAP_SWIZZLE_128B))
+    CUtensorMap mwq, mout, mvin;
+    if (!make_map(&mvin, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)H * DV, rows, 64, C,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
     const bool ok =
         make_map(&mwq, ws_wq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, DK, (uint64_t)nu * 2 * C, 64,
@@ -1812,7 +1813,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
     const int cols = segs.summ != nullptr ? DK + DV : DV;
     const int64_t ctas64 = (int64_t)(cols / BV) * H * n_seqs * segs.launch;
     const bool narrow = 2 * ctas64 <= (int64_t)sm_count();
-    auto k2 = narrow ? carry_kernel<Tout, SF, kVin, 32> : carry_kernel<Tout, SF, kVin, 64>;
+    auto k2 = narrow ? carry_kernel<Tout, SF, G2, 32> : carry_kernel<Tout, SF, G2, 64>;
     static bool attr2[2] = {false, false};
     if (!attr2[narrow]) {
       cudaError_t e = set_smem(k2, kSmem2Bytes);
@@ -1820,7 +1821,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       attr2[narrow] = true;
     }
     dim3 grid(cols / (narrow ? 32 : BV), H, n_seqs * segs.launch);
-    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, kVin ? mvin : mv16, mout, ws_g, S0, cu,
+    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, mvin, mout, ws_g, wg, S0, cu,
                                           static_cast<Tout*>(out), S_final, n_seqs, T, H, DV,
                                           nch, status, segs.n, segs.launch, segs.start,
                                           segs.summ);

@@ -115,8 +115,8 @@ enum {
  *            256-byte aligned, overlapping no tensor argument; its contents
  *            on entry do not matter and on return are unspecified.  Only
  *            the tensor-core path uses it (per chunk and head: [-W; Q'],
- *            K * rho, [Inv diag(beta); P] and V in fp16, gamma in fp32,
- *            82,432 bytes at d_v = 128); when the size query returns 0
+ *            K * rho and [Inv diag(beta); P] in fp16, gamma in fp32,
+ *            66,048 bytes for either d_v); when the size query returns 0
  *            both may be NULL / 0.  Calls that run concurrently (other
  *            streams) need separate workspaces; calls ordered on one stream
  *            may share one.  A workspace that is missing or too small
@@ -142,9 +142,9 @@ CKDA_API int ckda_fwd_chunked(const void* q, const void* k, const void* v,
  *    output is bit-identical to ckda_fwd_chunked with any valid workspace.
  *  - Sizes whose workspace (ckda_fwd_chunked_workspace_bytes) exceeds
  *    CKDA_STATIC_SCRATCH_BYTES return CKDA_ERR_UNSUPPORTED and launch
- *    nothing: at d_v = 128 that is more than 814 units of
- *    ceil(T / 64) * B * H (fixed-length) or (floor(T / 64) + N) * H
- *    (packed), e.g. B = 1, T = 2048, H = 16 fits (512 units).  Sizes on the
+ *    nothing: that is more than 1016 units of ceil(T / 64) * B * H
+ *    (fixed-length) or (floor(T / 64) + N) * H (packed), e.g. B = 1,
+ *    T = 2048, H = 16 fits (512 units).  Sizes on the
  *    fp32 CUDA-core path need no scratch and are always accepted.
  *  - Nothing in the scratch has to start at zero: every byte the carry
  *    kernel reads is written by the factor kernel of the same call.

@@ -154,20 +154,20 @@ def test_selftest_rejects_bad_limits(lib):
     assert lib.ckda_selftest_bounded_wait(20000000, None) == -1
 
 
-# per (chunk, head) unit: [-W; Q'] and K*rho (fp16), [Inv diag(beta); P] (fp16), gamma (fp32),
-# V (fp16, [64][d_v])
-UNIT_BYTES_DV128 = 2 * 64 * 128 * 2 + 64 * 128 * 2 + 2 * 64 * 64 * 2 + 128 * 4 + 64 * 128 * 2
+# per (chunk, head) unit: [-W; Q'] and K*rho (fp16), [Inv diag(beta); P] (fp16), gamma (fp32);
+# the same for every d_v (V is read from the input by the carry kernel)
+UNIT_BYTES = 2 * 64 * 128 * 2 + 64 * 128 * 2 + 2 * 64 * 64 * 2 + 128 * 4
 
 
 def test_workspace_size_query_needs_no_gpu(lib):
     F32, BF16 = 0, 1
     q = lib.ckda_fwd_chunked_workspace_bytes
     # fixed-length: B * ceil(T / 64) * H units
-    assert q(4, 4096, 16, 128, 128, 64, BF16, F32, 0) == 4 * 64 * 16 * UNIT_BYTES_DV128
-    assert q(2, 100, 3, 128, 128, 64, BF16, F32, 0) == 2 * 2 * 3 * UNIT_BYTES_DV128
-    assert q(1, 64, 1, 128, 64, 0, BF16, BF16, 0) == UNIT_BYTES_DV128 - 64 * 64 * 2
+    assert q(4, 4096, 16, 128, 128, 64, BF16, F32, 0) == 4 * 64 * 16 * UNIT_BYTES
+    assert q(2, 100, 3, 128, 128, 64, BF16, F32, 0) == 2 * 2 * 3 * UNIT_BYTES
+    assert q(1, 64, 1, 128, 64, 0, BF16, BF16, 0) == UNIT_BYTES
     # packed: (floor(T / 64) + N) * H units
-    assert q(5, 1000, 2, 128, 128, 64, BF16, F32, 1) == (1000 // 64 + 5) * 2 * UNIT_BYTES_DV128
+    assert q(5, 1000, 2, 128, 128, 64, BF16, F32, 1) == (1000 // 64 + 5) * 2 * UNIT_BYTES
     # the CUDA-core path needs none
     assert q(4, 4096, 16, 128, 128, 64, F32, F32, 0) == 0
     assert q(4, 4096, 16, 64, 64, 64, BF16, F32, 0) == 0
@@ -180,7 +180,7 @@ def test_workspace_size_query_needs_no_gpu(lib):
 def test_workspace_errors_launch_nothing(lib):
     tc = dict(dtype=1, out_dtype=0, dk=128, dv=128, chunk=64, T=128, B=1, H=1)
     need = lib.ckda_fwd_chunked_workspace_bytes(1, 128, 1, 128, 128, 64, 1, 0, 0)
-    assert need == 2 * UNIT_BYTES_DV128
+    assert need == 2 * UNIT_BYTES
     WS = 1 << 32  # 256-byte aligned, never dereferenced
     assert fwd(lib, **tc) == -7                                   # missing
     assert fwd(lib, ws=WS, ws_bytes=need - 1, **tc) == -7         # too small
@@ -233,7 +233,7 @@ def test_static_scratch_entry_rejects_oversized_calls_without_a_gpu(lib):
     from delta_rule_linear_ckda_b200._lib import CKDA_STATIC_SCRATCH_BYTES
 
     F32, BF16 = 0, 1
-    # 4 x 64 x 16 units at d_v = 128 need 338 MB > the 64 MiB scratch
+    # 4 x 64 x 16 units need 271 MB > the 64 MiB scratch
     assert lib.ckda_fwd_chunked_workspace_bytes(4, 4096, 16, 128, 128, 64, BF16, F32, 0) > \
         CKDA_STATIC_SCRATCH_BYTES
     r = lib.ckda_fwd_chunked_static(P, P + 0x1000, P + 0x2000, P + 0x3000, P + 0x4000, None, None,

@@ -58,7 +58,7 @@ def test_packed_batch_and_d_v_64(ck):
 
 def test_sizes_beyond_the_scratch_are_rejected(ck):
     c = _case(1, 64, 1, seed=4)
-    # 4 * 64 * 16 units need 338 MB: refused before any launch
+    # 4 * 64 * 16 units need 271 MB: refused before any launch
     big_T = 4096
     assert ck.workspace_bytes(4, big_T, 16, 128, 128) > _lib.CKDA_STATIC_SCRATCH_BYTES
     rc = _lib.load().ckda_fwd_chunked_static(
