@@ -831,16 +831,22 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     n.valid = uu.idx >= 0;
     return n;
   };
+  // Shared-memory descriptors: each tile's base; a K step adds its byte
+  // offset / 16 to the low field.
+  const uint64_t d_lv = smem_desc(sb + F2_LV, 16, 1024, kSwizzle128);
+  const uint64_t d_aq = smem_desc(sb + F2_AQ, 16, 1024, kSwizzle128);
+  const uint64_t d_ipk = smem_desc(sb + F2_IP, 16, 1024, kSwizzle128);     // K-major (A)
+  const uint64_t d_ipm = smem_desc(sb + F2_IP, 8192, 1024, kSwizzle128);   // MN-major (B)
+  const uint64_t d_kg = smem_desc(sb + F2_KG, 8192, 1024, kSwizzle128);
   auto level_mmas = [&](int jq) {
     constexpr uint32_t id = idesc_f16(128, 64, 0, 0);
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
-      const uint32_t la = sb + F2_LV + pr * kPairBytes;
 #pragma unroll
       for (int k2 = 0; k2 < 2; ++k2) {
         const int kk = 2 * (jq & 1) + k2;
-        const uint64_t ad = smem_desc(la + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(la + PAIR_ROP + kk * 32, 16, 1024, kSwizzle128);
+        const uint64_t ad = d_lv + (pr * kPairBytes + kk * 32) / 16;
+        const uint64_t bd = d_lv + (pr * kPairBytes + PAIR_ROP + kk * 32) / 16;
         mma_f16(tmem + TM3_LV + 64 * pr, ad, bd, id, (jq > 0 || k2 > 0) ? 1u : 0u);
       }
     }
@@ -1055,9 +1061,7 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       constexpr uint32_t id = idesc_f16(64, 64, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(sb + F2_AQ + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + F2_IP + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM3_P, ad, bd, id, kk > 0 ? 1u : 0u);
+        mma_f16(tmem + TM3_P, d_aq + 2 * kk, d_ipm + 128 * kk, id, kk > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
     }
@@ -1088,8 +1092,8 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       constexpr uint32_t id1 = idesc_f16(128, 128, 0, 1);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(sb + F2_IP + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + F2_KG + kk * 2048, 8192, 1024, kSwizzle128);
+        const uint64_t ad = d_ipk + 2 * kk;
+        const uint64_t bd = d_kg + 128 * kk;
         mma_f16(tmem + TM3_W, ad, bd, id1, kk > 0 ? 1u : 0u);
       }
       mma_commit(bar_mma);
@@ -1378,52 +1382,69 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                     32 * (tid % LPR));
     }
   };
+  // Shared-memory descriptors of the carry's operands: the base of each
+  // tile; a K step adds its byte offset / 16 to the low field.
+  // (a stage's descriptors are stage 0's plus kStageBytes / 16)
+  const uint64_t d_ip0 = smem_desc(sb + CS_IP, 16, 1024, kSwizzle128);
+  const uint64_t d_v0 = smem_desc(sb + CS_V, 8192, 1024, kSwizzle128);
+  const uint64_t d_wq0 = smem_desc(sb + CS_WQ, 16, 1024, kSwizzle128);
+  const uint64_t d_kh0 = smem_desc(sb + CS_KH, 8192, 1024, kSwizzle128);
+  auto stg = [](int s2) -> uint64_t { return s2 ? (uint64_t)(kStageBytes >> 4) : 0ull; };
+  const uint64_t d_sb = smem_desc(sb + OFF2_SB, 8192, 1024, kSwizzle128);
+  const uint64_t d_ub = smem_desc(sb + OFF2_UB, 8192, 1024, kSwizzle128);
+  constexpr uint32_t id_c1 = idesc_f16(128, NBV, 0, 1);
+  constexpr uint32_t id_c2 = idesc_f16(128, NBV, 1, 1);
+  // carry 1 in two parts: the V term (independent of S) and the S term
+  auto mma_v = [&](int s2, uint32_t acc0) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_f16(tmem + TM2_X, d_ip0 + stg(s2) + 2 * kk, d_v0 + stg(s2) + 128 * kk, id_c1,
+              (kk > 0 || acc0) ? 1u : 0u);
+  };
+  auto mma_s = [&](int s2, uint32_t acc0) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_f16(tmem + TM2_X, d_wq0 + stg(s2) + 1024 * (kk >> 2) + 2 * (kk & 3), d_sb + 128 * kk,
+              id_c1,
+              (kk > 0 || acc0) ? 1u : 0u);
+  };
+  // With V: the V term of chunk c goes in as soon as chunk c's V tile is in
+  // fp16 (for c > 0 while carry 2 of chunk c - 1 finishes), so only the
+  // S term of carry 1 is left on the chunk-to-chunk path.
   if (v_early && nchunks > 0) {
     prefetch_w(1);
     ok = wait(bar_full0, ph0, pend0);
     if (ok) convert_v(0, 0);
     fence_proxy_async_smem();
   }
-  __syncthreads();
+  ok = __syncthreads_and(ok);
+  if (ok && v_early && nchunks > 0 && tid == 0) {
+    tc_fence_after();
+    mma_v(0, 0u);
+  }
 
-  for (int c = 0; c < nchunks; ++c) {
+  for (int c = 0; ok && c < nchunks; ++c) {
     const int st = c & 1;
     const int64_t t0 = tok0 + (int64_t)(cbeg + c) * C;
     const int Lc = chunk_len(c);
-    const uint32_t stage = sb + st * kStageBytes;
     // (the bf16 output map's box is 64 columns wide: a 32-column slice stores
     // its rows with plain stores)
     const bool tma_out =
         !summary && ((cu == nullptr) || Lc == C) && (NBV == 64 || sizeof(Tout) == 4);
-    if (!v_early) ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
+    if (!v_early) {
+      // (with V the previous chunk's last barrier already combined `ok`)
+      ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
+      ok = __syncthreads_and(ok);
+      if (!ok) break;
+    }
     const float2 gm_next = load_gamma(c + 1);
     TC_MARK(9);
 
     // ---- carry 1: [U; O] = [Inv diag(beta); P] V + [-W; Q'] S -------------------
-    constexpr uint32_t id_c1 = idesc_f16(128, NBV, 0, 1);
-    auto mma_v = [&](uint32_t acc0) {
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(stage + CS_IP + kk * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(stage + CS_V + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_X, ad, bd, id_c1, (kk > 0 || acc0) ? 1u : 0u);
-      }
-    };
-    auto mma_s = [&](uint32_t acc0) {
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint64_t ad =
-            smem_desc(stage + CS_WQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF2_SB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_X, ad, bd, id_c1, (kk > 0 || acc0) ? 1u : 0u);
-      }
-    };
     if (tid == 0) {
       tc_fence_after();
-      if (!mcols) mma_v(0u);
-      mma_s(mcols ? 0u : 1u);
+      if (!v_early && !mcols) mma_v(st, 0u);
+      mma_s(st, mcols ? 0u : 1u);
       mma_commit(bar_mma);
     }
     pend_mma = 1;
@@ -1459,6 +1480,18 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    TC_MARK(11);
+
+    // ---- carry 2: D = (K rho)^T U;  S <- Diag(gamma) S + D ----------------------
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f16(tmem + TM2_D, d_kh0 + stg(st) + 128 * kk, d_ub + 128 * kk, id_c2,
+                kk > 0 ? 1u : 0u);
+      mma_commit(bar_mma);
+    }
+    pend_mma = 1;
     if (tma_out && tid == 0) {
       // fixed-length batch: [T, H * d_v] per sequence, rows past T are clipped;
       // packed batch: only whole chunks go through TMA
@@ -1481,31 +1514,20 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       }
       bulk_commit();
     }
-    TC_MARK(11);
-
-    // ---- carry 2: D = (K rho)^T U;  S <- Diag(gamma) S + D ----------------------
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_f16(128, NBV, 1, 1);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = smem_desc(stage + CS_KH + kk * 2048, 8192, 1024, kSwizzle128);
-        const uint64_t bd = smem_desc(sb + OFF2_UB + kk * 2048, 8192, 1024, kSwizzle128);
-        mma_f16(tmem + TM2_D, ad, bd, id, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(bar_mma);
-    }
-    pend_mma = 1;
     // while carry 2 runs: the next chunk's stage, its V converted to fp16
     if (v_early && c + 1 < nchunks) {
       prefetch_w(c + 2);
       ok = st ? wait(bar_full0, ph0, pend0) : wait(bar_full0 + 8, ph1, pend1);
       if (ok) convert_v(st ^ 1, c + 1);
+      // the converted tile is read by carry 1's V term right after the barrier
+      fence_proxy_async_smem();
     }
     ok = wait(bar_mma, ph_mma, pend_mma) && ok;
     ok = __syncthreads_and(ok);
     if (!ok) break;
     tc_fence_after();
+    // carry 1's V term of the next chunk (its accumulator was read out above)
+    if (v_early && c + 1 < nchunks && tid == 0) mma_v(st ^ 1, 0u);
     // this stage is consumed: fetch chunk c + 2 into it
     if (c + 2 < nchunks) {
       if (tid == 0) issue(c + 2, st);
