@@ -229,35 +229,72 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
     }
     __syncthreads();
 
-    // ---- score blocks T and A: one warp per column s ------------------
-    // x = k_s * P(r, s) is carried down the rows r > s by multiplying with
-    // alpha_r; the dot products with k_r (G2: e_r) and q_r give T[r, s] /
-    // beta_r (G2: T[r, s]) and A[r, s].  Lanes split the channels; eight rows
-    // are reduced at once.
+    // ---- score blocks T and A: four columns per warp ------------------
+    // For column s, x = k_s * P(r, s) is carried down the rows r > s by
+    // multiplying with alpha_r; the dot products with k_r (G2: e_r) and q_r
+    // give T[r, s] / beta_r (G2: T[r, s]) and A[r, s].  Lanes split the
+    // channels; eight rows are reduced at once.  A warp takes the columns
+    // s0, s0 + 8, s0 + 16, s0 + 24 together (s0 = warp, then warp + 32): their
+    // rows run in the same blocks of eight, column m joining at block m, so
+    // each row's alpha, k and q are read once for up to four independent
+    // chains.
     {
       using LC = LaneChannels<DK>;
       constexpr int CPL = LC::kPer;
       const bool act = LC::active(lane);
       const int cb = lane * CPL;
-      for (int s = warp; s < C; s += kThreads / 32) {
-        float x[CPL];
-        float qs[CPL];
+      // x <- gate_r x on this lane's channels (SFDA: complex pairs)
+      auto step = [&](float* x, const float* a) {
+        if constexpr (SF) {
+          if constexpr (CPL >= 2) {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) { x[c] = 0.f; qs[c] = 0.f; }
-        if (act) { lds<CPL>(Ks + s * KS + cb, x); lds<CPL>(Qs + s * KS + cb, qs); }
-        float d = 0.f;
+            for (int c = 0; c < CPL; c += 2) {
+              const float xr = x[c], xi = x[c + 1];
+              x[c] = cmul_re(a[c], a[c + 1], xr, xi);
+              x[c + 1] = cmul_im(a[c], a[c + 1], xr, xi);
+            }
+          } else {
+            // one channel per lane: the pair partner is the neighbouring lane
+            const float xo = __shfl_xor_sync(0xffffffffu, x[0], 1);
+            const float lo = __shfl_xor_sync(0xffffffffu, a[0], 1);
+            const bool odd = lane & 1;
+            const float lre = odd ? lo : a[0], lim = odd ? a[0] : lo;
+            x[0] = odd ? cmul_im(lre, lim, xo, x[0]) : cmul_re(lre, lim, x[0], xo);
+          }
+        } else {
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) d = fmaf(qs[c], x[c], d);
+          for (int c = 0; c < CPL; ++c) x[c] *= a[c];
+        }
+      };
+      for (int s0 = warp; s0 < C; s0 += 32) {
+        float x[4][CPL];
+        // columns of this quad: diagonal of A, zeros above the diagonal
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-        if (lane == 0) { Am[s * CS + s] = d; Tm[s * CS + s] = 0.f; }
-        for (int r = lane; r < s; r += 32) { Tm[r * CS + s] = 0.f; Am[r * CS + s] = 0.f; }
-        for (int rb = s + 1; rb < C; rb += 8) {
-          float pk[8], pq[8];
+        for (int m = 0; m < 4; ++m) {
+          const int s = s0 + 8 * m;
+          float qs[CPL];
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) { x[m][c] = 0.f; qs[c] = 0.f; }
+          if (s < C) {
+            if (act) { lds<CPL>(Ks + s * KS + cb, x[m]); lds<CPL>(Qs + s * KS + cb, qs); }
+            float d = 0.f;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) d = fmaf(qs[c], x[m][c], d);
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
+            if (lane == 0) { Am[s * CS + s] = d; Tm[s * CS + s] = 0.f; }
+            for (int r = lane; r < s; r += 32) { Tm[r * CS + s] = 0.f; Am[r * CS + s] = 0.f; }
+          }
+        }
+        for (int blk = 0; s0 + 1 + 8 * blk < C; ++blk) {
+          const int rb = s0 + 1 + 8 * blk;
+          float pk[4][8], pq[4][8];
+#pragma unroll
+          for (int m = 0; m < 4; ++m)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) { pk[m][jj] = 0.f; pq[m][jj] = 0.f; }
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
-            pk[jj] = 0.f;
-            pq[jj] = 0.f;
             const int r = rb + jj;
             if (r < C) {
               float a[CPL], kr[CPL], qr[CPL];
@@ -268,40 +305,31 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
                 lds<CPL>((G2 ? Ws : Ks) + r * KS + cb, kr);
                 lds<CPL>(Qs + r * KS + cb, qr);
               }
-              if constexpr (SF) {
-                // x <- lambda_r x on every channel pair
-                if constexpr (CPL >= 2) {
 #pragma unroll
-                  for (int c = 0; c < CPL; c += 2) {
-                    const float xr = x[c], xi = x[c + 1];
-                    x[c] = cmul_re(a[c], a[c + 1], xr, xi);
-                    x[c + 1] = cmul_im(a[c], a[c + 1], xr, xi);
+              for (int m = 0; m < 4; ++m) {
+                if (m <= blk) {
+                  step(x[m], a);
+#pragma unroll
+                  for (int c = 0; c < CPL; ++c) {
+                    pk[m][jj] = fmaf(kr[c], x[m][c], pk[m][jj]);
+                    pq[m][jj] = fmaf(qr[c], x[m][c], pq[m][jj]);
                   }
-                } else {
-                  // one channel per lane: the pair partner is the neighbouring lane
-                  const float xo = __shfl_xor_sync(0xffffffffu, x[0], 1);
-                  const float lo = __shfl_xor_sync(0xffffffffu, a[0], 1);
-                  const bool odd = lane & 1;
-                  const float lre = odd ? lo : a[0], lim = odd ? a[0] : lo;
-                  x[0] = odd ? cmul_im(lre, lim, xo, x[0]) : cmul_re(lre, lim, x[0], xo);
                 }
-              } else {
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) x[c] *= a[c];
-              }
-#pragma unroll
-              for (int c = 0; c < CPL; ++c) {
-                pk[jj] = fmaf(kr[c], x[c], pk[jj]);
-                pq[jj] = fmaf(qr[c], x[c], pq[jj]);
               }
             }
           }
-          reduce_scatter8(pk, lane);
-          reduce_scatter8(pq, lane);
           const int r = rb + (lane & 7);
-          if (lane < 8 && r < C) {
-            Tm[r * CS + s] = G2 ? pk[0] : bs[r] * pk[0];
-            Am[r * CS + s] = pq[0];
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            if (m <= blk) {
+              reduce_scatter8(pk[m], lane);
+              reduce_scatter8(pq[m], lane);
+              const int s = s0 + 8 * m;
+              if (lane < 8 && r < C) {
+                Tm[r * CS + s] = G2 ? pk[m][0] : bs[r] * pk[m][0];
+                Am[r * CS + s] = pq[m][0];
+              }
+            }
           }
         }
       }
