@@ -58,6 +58,29 @@ BWD_BYTES_PER_TOKEN_HEAD = 3 * D * 2 + D * 4 + 4 + D * 4 + 3 * D * 4 + D * 4 + 4
 
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
+# fp32 CUDA-core roof of the kernels that run on FFMA (the fp32-faithful
+# forward, the backward): 128 fp32 lanes per SM, one FMA (2 flops) per lane
+# per clock, at the B200's maximum SM clock of 1965 MHz.
+FP32_LANES_PER_SM = 128
+SM_MAX_MHZ = 1965.0
+# backward: one recompute of the state step (S' = Diag(a) S, r = S'^T k,
+# S' + k u^T: 5 d^2) and the adjoint step (dq, q do^T, dS^T k, dS u + S' dr,
+# k dr^T, rowsum(dS' . S), Diag(a) dS': 15 d^2) per token-head
+BWD_FLOPS_PER_TOKEN_HEAD = 20 * D * D
+
+
+def fp32_alu_peak_tflops(torch, dev):
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    return sms * FP32_LANES_PER_SM * 2 * SM_MAX_MHZ * 1e6 / 1e12, sms
+
+
+def alu_roofline(flops, ms, peak, sms, what):
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "flops_per_launch": flops,
+            "peak_basis": f"{sms} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 flops x "
+                          f"{SM_MAX_MHZ:.0f} MHz (FFMA)",
+            "flops": what}
 
 
 def _peaks():
@@ -750,6 +773,9 @@ def _run_varlen(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hb
     ms = max_ranks(e0.elapsed_time(e1)) / steps
     nbytes = Tt * H * VARLEN_BYTES_PER_TOKEN_HEAD + N * H * D * D * 4
     gbs = nbytes / (ms / 1e3) / 1e9
+    peak, sms = fp32_alu_peak_tflops(torch, dev)
+    roof = alu_roofline(Tt * H * STRICT_FLOPS_PER_TOKEN_HEAD, ms, peak, sms,
+                        "strict chunk flops per token-head (6 C d + 6 d^2 + C^2 / 3) x token-heads")
     return {"workload": f"varlen N={N} L~U[128,4096] (T_total={Tt}) H={H} d={D} C={CHUNK} fp32, "
                         "gate extremes, S0=0, S_final stored",
             "kernel": ck.fwd_path(N, Tt, H, D, D, CHUNK, torch.float32, torch.float32,
@@ -758,6 +784,7 @@ def _run_varlen(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hb
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_frac_of_measured": gbs / hbm_peak,
             "hbm_floor_ms_at_measured": nbytes / (hbm_peak * 1e9) * 1e3,
+            "roofline": roof, "alu_floor_ms": roof["flops_per_launch"] / (peak * 1e12) * 1e3,
             "steps": steps, "gpu_launches": steps}
 
 
@@ -795,13 +822,16 @@ def _run_bwd(ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_p
     ms = max_ranks(ev0.elapsed_time(ev1)) / steps
     nbytes = B * T * H * BWD_BYTES_PER_TOKEN_HEAD
     gbs = nbytes / (ms / 1e3) / 1e9
+    peak, sms = fp32_alu_peak_tflops(torch, dev)
+    roof = alu_roofline(B * T * H * BWD_FLOPS_PER_TOKEN_HEAD, ms, peak, sms,
+                        "per-token adjoint with one state recompute, 20 d^2 per token-head")
     return {"workload": f"kda_prefill backward B={B} H={H} T={T} d={D}: bf16 q/k/v, fp32 "
                         "alpha/beta/dO, fp32 gradients (fp32 CUDA-core kernel, clusters of "
                         f"{D // 32} CTAs per (sequence, head))",
             "ms_per_step": ms, "tokens_per_s": ws * B * T / (ms / 1e3),
             "algorithmic_bytes": nbytes, "achieved_gbs": gbs,
             "hbm_frac_of_measured": gbs / hbm_peak, "workspace_bytes": wsb.numel(),
-            "gpu_launches": steps}
+            "roofline": roof, "gpu_launches": steps}
 
 
 def _run_decode(args, ck, torch, inputs, rank, dev, stream, barrier, max_ranks, ws, hbm_peak):

@@ -81,6 +81,33 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
   *reinterpret_cast<uint2*>(p) = raw;
 }
 
+// Packed batches whose CTAs each walk one whole sequence: the sequence the
+// CTA with grid index `z` takes is the one of rank z when the sequences are
+// ordered by decreasing length (ties by index), so the longest start first
+// and the last CTAs the block scheduler hands out are short ones (longest
+// processing time first).  The map is a bijection for any offsets array, a
+// malformed one included (seq_range still flags it).  Block-wide: every
+// thread of the CTA calls it once, before any other use of the barrier.
+// Fixed-length batches (cu == NULL) and very large batches keep z.
+constexpr int kLongestFirstMaxSeqs = 1024;
+__device__ __forceinline__ int seq_longest_first(const int32_t* cu, int n_seqs, int z) {
+  if (cu == nullptr || n_seqs > kLongestFirstMaxSeqs) return z;
+  __shared__ int pick;
+  if (threadIdx.x == 0) pick = z;
+  __syncthreads();
+  for (int n = threadIdx.x; n < n_seqs; n += blockDim.x) {
+    const int ln = cu[n + 1] - cu[n];
+    int rank = 0;
+    for (int m = 0; m < n_seqs; ++m) {
+      const int lm = cu[m + 1] - cu[m];
+      rank += (lm > ln || (lm == ln && m < n)) ? 1 : 0;
+    }
+    if (rank == z) pick = n;
+  }
+  __syncthreads();
+  return pick;
+}
+
 // Token range of sequence n: fixed-length batches use n*T .. (n+1)*T;
 // packed batches read (and validate) the offsets array.
 struct SeqRange {

@@ -161,7 +161,7 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
   const int warp = tid >> 5;
   const int j0 = blockIdx.x * BV;
   const int h = blockIdx.y;
-  const int n = blockIdx.z;
+  const int n = seq_longest_first(cu, n_seqs, blockIdx.z);
 
   const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
   if (!sr.ok) return;

@@ -1210,7 +1210,9 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   constexpr int CPT = NBV / 2;  // state columns per thread
   const int j0 = blockIdx.x * NBV;
   const int h = blockIdx.y;
-  const int n = blockIdx.z / seg_launch;
+  // (a plain packed forward walks its sequences longest first)
+  const int n = (seg_n == 1 && summ == nullptr) ? seq_longest_first(cu, n_seqs, blockIdx.z)
+                                                : blockIdx.z / seg_launch;
   const int seg = blockIdx.z % seg_launch;
   const bool summary = summ != nullptr;
   const bool mcols = summary && j0 < DK;  // transfer-matrix columns
