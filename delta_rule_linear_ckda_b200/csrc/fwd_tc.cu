@@ -107,8 +107,18 @@ constexpr uint32_t kStageBytes = 73728;
 constexpr uint32_t OFF2_SB = 2 * kStageBytes;  // state slice, fp16 MN-major [128 i][64 j]
 constexpr uint32_t OFF2_UB = OFF2_SB + 16384;  // U, fp16 MN-major [64 s][64 j]
 constexpr uint32_t OFF2_OB = OFF2_UB + 8192;  // O staging for its TMA store: fp32 [64][32] x 2 or bf16 [64][64]
-constexpr uint32_t OFF2_BAR = OFF2_OB + 16384;  // mbarriers: stage 0, stage 1, mma
-constexpr uint32_t OFF2_TMEMPTR = OFF2_BAR + 32;
+constexpr uint32_t OFF2_BAR = OFF2_OB + 16384;  // mbarriers (below)
+constexpr uint32_t OFF2_TMEMPTR = OFF2_BAR + 128;
+// carry mbarriers, byte offsets from OFF2_BAR
+constexpr uint32_t CB_FULL = 0;   // stage s loaded (TMA transaction), + 8 s
+constexpr uint32_t CB_VRDY = 16;  // stage s's V converted to fp16 (compute threads), + 8 s
+constexpr uint32_t CB_SRDY = 32;  // the state's fp16 operand written (compute threads)
+constexpr uint32_t CB_X = 40;     // carry 1 ([U; O]) complete (tensor-core commit)
+constexpr uint32_t CB_U = 48;     // U in its operand tile, O staged or stored (compute threads)
+constexpr uint32_t CB_D = 56;     // carry 2 (D) complete (tensor-core commit)
+constexpr uint32_t CB_OB = 64;    // the output staging free again (store warp)
+constexpr int kCarryCompute = 256;              // state / epilogue threads (8 warps)
+constexpr int kCarryThreads = kCarryCompute + 64;  // + one MMA warp, one copy warp
 constexpr uint32_t kSmem2Used = OFF2_TMEMPTR + 16;
 constexpr size_t kSmem2Bytes = kSmem2Used + 1024;
 
@@ -116,36 +126,6 @@ constexpr size_t kSmem2Bytes = kSmem2Used + 1024;
 constexpr uint32_t kTmem2Cols = 128;
 constexpr uint32_t TM2_X = 0;    // [U; O] = [U~ - W S; A U~ + Q' S]  (M = 128, 64 columns)
 constexpr uint32_t TM2_D = 64;   // (K rho)^T U    (M = 128, 64 columns)
-
-#ifdef CKDA_TC_DEBUG
-// Intermediate dump of the first unit of CTA 0 and of the first chunk of
-// carry CTA (0, 0, 0), and per-phase clock counts (diagnostic builds only).
-__device__ float* g_tc_dbg = nullptr;
-__device__ unsigned long long* g_tc_time = nullptr;
-#define TC_DBG(stmt)                                                                   \
-  do {                                                                                 \
-    if (g_tc_dbg != nullptr && c == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&         \
-        blockIdx.z == 0) {                                                             \
-      stmt;                                                                            \
-    }                                                                                  \
-  } while (0)
-#define TC_MARK(k)                                                                       \
-  do {                                                                                   \
-    if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 &&        \
-        blockIdx.z == 0) {                                                               \
-      const long long now = clock64();                                                   \
-      tmark[k] += now - tlast;                                                           \
-      tlast = now;                                                                       \
-    }                                                                                    \
-  } while (0)
-#else
-#define TC_DBG(stmt) \
-  do {               \
-  } while (0)
-#define TC_MARK(k) \
-  do {             \
-  } while (0)
-#endif
 
 // Tensor-core operands are fp16: the bf16 inputs convert to it exactly
 // (apart from subnormals), and its 10-bit mantissa keeps the rounding of the
@@ -1192,7 +1172,7 @@ factor2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 // on the GPU when there are few (sequence, head) pairs, as in one long
 // sequence); each thread holds NBV / 2 columns of one state row.
 template <typename Tout, bool SF, bool WG, int NBV>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(kCarryThreads, 1)
 carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ CUtensorMap tm_kh,
              const __grid_constant__ CUtensorMap tm_ip, const __grid_constant__ CUtensorMap tm_v16,
              const __grid_constant__ CUtensorMap tm_out,
@@ -1207,7 +1187,7 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  constexpr int CPT = NBV / 2;  // state columns per thread
+  constexpr int CPT = NBV / 2;  // state columns per compute thread
   const int j0 = blockIdx.x * NBV;
   const int h = blockIdx.y;
   // (a plain packed forward walks its sequences longest first)
@@ -1217,16 +1197,22 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   const bool summary = summ != nullptr;
   const bool mcols = summary && j0 < DK;  // transfer-matrix columns
   const int jv = summary ? j0 - DK : j0;  // V and output column of this CTA
+  const bool has_v = !mcols;              // the chunk's V term enters carry 1
 
   const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
   if (!sr.ok) return;
 
-  const uint32_t bar_full0 = sb + OFF2_BAR;
-  const uint32_t bar_mma = sb + OFF2_BAR + 16;
+  const uint32_t bar = sb + OFF2_BAR;
   if (tid == 0) {
-    mbar_init(bar_full0, 1);
-    mbar_init(bar_full0 + 8, 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(bar + CB_FULL, 1);
+    mbar_init(bar + CB_FULL + 8, 1);
+    mbar_init(bar + CB_VRDY, kCarryCompute);
+    mbar_init(bar + CB_VRDY + 8, kCarryCompute);
+    mbar_init(bar + CB_SRDY, kCarryCompute);
+    mbar_init(bar + CB_X, 1);
+    mbar_init(bar + CB_U, kCarryCompute);
+    mbar_init(bar + CB_D, 1);
+    mbar_init(bar + CB_OB, 1);
     fence_mbar_init();
     prefetch_tmap(&tm_wq);
     prefetch_tmap(&tm_kh);
@@ -1242,42 +1228,6 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(sm + OFF2_TMEMPTR);
-#ifdef CKDA_TC_DEBUG
-  long long tmark[16] = {0};
-  long long tlast = clock64();
-#endif
-
-  // State slice: row i = 32 * (warp % 4) + lane, columns [CPT * (warp / 4), +CPT).
-  const int q4 = warp & 3;
-  const int half = warp >> 2;
-  const int srow = 32 * q4 + lane;
-  const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + CPT * half;
-  // this thread's CPT start values (row srow, CPT columns)
-  const float* s_row = nullptr;
-  if (seg == 0) {
-    if (S0 != nullptr) s_row = S0 + s_off;
-  } else {
-    s_row = seg_start + ((((size_t)n * seg_n + seg) * H + h) * DK + srow) * DV + j0 + CPT * half;
-  }
-  float S[CPT];
-#pragma unroll
-  for (int e = 0; e < CPT; e += 4) {
-    float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (summary) {
-      if (mcols) {
-        const int c = j0 + CPT * half + e - srow;  // identity: 1 where column == row
-        v4 = make_float4(c == 0 ? 1.f : 0.f, c == -1 ? 1.f : 0.f, c == -2 ? 1.f : 0.f,
-                         c == -3 ? 1.f : 0.f);
-      }
-    } else if (s_row != nullptr) {
-      v4 = *reinterpret_cast<const float4*>(s_row + e);
-    }
-    S[e] = v4.x; S[e + 1] = v4.y; S[e + 2] = v4.z; S[e + 3] = v4.w;
-  }
-#pragma unroll
-  for (int c4 = 0; c4 < CPT / 8; ++c4)
-    st_chunk8(sm + OFF2_SB, sw128_chunk(srow, CPT * half + 8 * c4, 128), S + 8 * c4);
-  fence_proxy_async_smem();
 
   const int64_t tok0 = sr.begin;
   const int64_t tok1 = sr.end;
@@ -1287,315 +1237,348 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   const int nchunks = (int)((int64_t)(seg + 1) * nck_all / seg_n) - cbeg;
   const int64_t slot0 = slot_base(cu, n, nch);
   auto unit_of = [&](int c) -> int64_t { return (slot0 + cbeg + c) * H + h; };
-  // phase bits advance only on a successful wait (see the factor kernel)
-  uint32_t ph0 = 0, ph1 = 0, ph_mma = 0;
-  int pend0 = 0, pend1 = 0, pend_mma = 0;
-  int ok = 1;
-  auto wait = [&](uint32_t bar, uint32_t& phase, int& pending) -> bool {
-    const bool r = mbar_wait_bounded(bar, phase, kWaitNs);
-    if (r) {
-      phase ^= 1;
-      pending = 0;
-    }
-    return r;
-  };
-
-  auto issue = [&](int c, int st) {
-    const uint32_t bar = bar_full0 + 8 * st;
-    const uint32_t base = sb + st * kStageBytes;
-    const int64_t uidx = unit_of(c);
-    mbar_expect_tx(bar, kStageBytes);
-    tma_load_2d(base + CS_WQ, &tm_wq, 0, (int)(uidx * 2 * C), bar);
-    tma_load_2d(base + CS_WQ + 16384, &tm_wq, 64, (int)(uidx * 2 * C), bar);
-    tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), bar);
-    tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), bar);
-    tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), bar);
-    tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
-                (int)(tok0 + (int64_t)(cbeg + c) * C), bar);
-  };
-  if (tid == 0) {
-    if (nchunks > 0) issue(0, 0);
-    if (nchunks > 1) issue(1, 1);
-  }
-  pend0 = nchunks > 0;
-  pend1 = nchunks > 1;
-  // gamma of this row (SF: of its row pair, real and imaginary part)
-  const int grow = SF ? (srow & ~1) : srow;
-  auto load_gamma = [&](int c) -> float2 {
-    if (c >= nchunks) return make_float2(1.f, 0.f);
-    const float* gp = ws_g + unit_of(c) * DK + grow;
-    return SF ? *reinterpret_cast<const float2*>(gp) : make_float2(*gp, 0.f);
-  };
-  float2 gm = load_gamma(0);
-  // bf16 V (as loaded) -> fp16 in place in stage `s` (WG: times the write
-  // gate), rows past the chunk's `len` tokens -> 0.  Each 16-byte chunk stays
-  // within its 128-byte row under the swizzle.  The V of chunk c + 1 is
-  // converted while carry 2 of chunk c runs (its stage wait moves there), so
-  // carry 1 finds it ready.
-  const bool v_early = !mcols;
   auto chunk_len = [&](int c) -> int {
     const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
     return (tok1 - t0c < (int64_t)C) ? (int)(tok1 - t0c) : C;
   };
-  auto convert_v = [&](int s, int c) {
-    const int len = chunk_len(c);
-    const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
-    uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
-    for (int e = tid; e < C * 8; e += NT) {
-      uint4 raw = vt[e];
-      const int row = e >> 3;
-      if (row < len) {
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-        float f[8];
+  // whole chunks go out by TMA (the bf16 output map's box is 64 columns
+  // wide, so a 32-column bf16 slice stores its rows itself)
+  auto tma_out = [&](int c) -> bool {
+    return !summary && ((cu == nullptr) || chunk_len(c) == C) &&
+           (NBV == 64 || sizeof(Tout) == 4);
+  };
+  auto wait = [&](uint32_t b, uint32_t parity) -> bool {
+    return mbar_wait_bounded(b, parity, kWaitNs);
+  };
+  int ok = 1;
+
+  // Three roles hand each chunk to one another through mbarriers, so that
+  // no block-wide barrier stands between the steps of the chunk-to-chunk
+  // chain (S -> carry 1 -> U -> carry 2 -> S):
+  //  * warps 0..7 (compute): the state slice in registers, the read-outs of
+  //    both tensor-memory products, U into its operand tile, O staged or
+  //    stored, V of the next chunk converted to fp16;
+  //  * warp 8 (one thread): every tcgen05 MMA;
+  //  * warp 9 (one thread): the stage loads and the output stores by TMA.
+  // Each barrier completes once per chunk (the stage barriers once per two),
+  // so the parity waited for follows from the chunk index.
+  float S[CPT];
+  int mma_pend = 0;            // MMA thread: a commit not yet seen complete
+  uint32_t mma_bar = 0, mma_par = 0;
+  uint32_t ld_pend = 0;        // copy thread: bit s, a load into stage s not yet seen complete
+  uint32_t ld_par = 0;         //   bit s, the parity of that load's phase
+
+  if (warp < 8) {
+    // ---- compute warps ----------------------------------------------------------------
+    // State slice: row i = 32 * (warp % 4) + lane, columns [CPT * (warp / 4), +CPT).
+    const int q4 = warp & 3;
+    const int half = warp >> 2;
+    const int srow = 32 * q4 + lane;
+    const size_t s_off = (((size_t)n * H + h) * DK + srow) * DV + j0 + CPT * half;
+    const float* s_row = nullptr;
+    if (seg == 0) {
+      if (S0 != nullptr) s_row = S0 + s_off;
+    } else {
+      s_row = seg_start + ((((size_t)n * seg_n + seg) * H + h) * DK + srow) * DV + j0 +
+              CPT * half;
+    }
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const float2 x2 = __bfloat1622float2(p2[t]);
-          f[2 * t] = x2.x;
-          f[2 * t + 1] = x2.y;
+    for (int e = 0; e < CPT; e += 4) {
+      float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (summary) {
+        if (mcols) {
+          const int c = j0 + CPT * half + e - srow;  // identity: 1 where column == row
+          v4 = make_float4(c == 0 ? 1.f : 0.f, c == -1 ? 1.f : 0.f, c == -2 ? 1.f : 0.f,
+                           c == -3 ? 1.f : 0.f);
         }
-        if constexpr (WG) {
-          // logical columns of this 16-byte chunk: 8 * (chunk ^ (row % 8));
-          // only the slice's own NBV columns are used (and read)
-          const int col = 8 * ((e & 7) ^ (row & 7));
-          if (col < NBV) {
-            const float* wp = wg + ((size_t)(t0c + row) * H + h) * DV + jv + col;
-            const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
-            const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp + 4));
-            f[0] *= w0.x; f[1] *= w0.y; f[2] *= w0.z; f[3] *= w0.w;
-            f[4] *= w1.x; f[5] *= w1.y; f[6] *= w1.z; f[7] *= w1.w;
+      } else if (s_row != nullptr) {
+        v4 = *reinterpret_cast<const float4*>(s_row + e);
+      }
+      S[e] = v4.x; S[e + 1] = v4.y; S[e + 2] = v4.z; S[e + 3] = v4.w;
+    }
+#pragma unroll
+    for (int c4 = 0; c4 < CPT / 8; ++c4)
+      st_chunk8(sm + OFF2_SB, sw128_chunk(srow, CPT * half + 8 * c4, 128), S + 8 * c4);
+    fence_proxy_async_smem();
+    mbar_arrive(bar + CB_SRDY);
+
+    // gamma of this row (SF: of its row pair, real and imaginary part)
+    const int grow = SF ? (srow & ~1) : srow;
+    auto load_gamma = [&](int c) -> float2 {
+      if (c >= nchunks) return make_float2(1.f, 0.f);
+      const float* gp = ws_g + unit_of(c) * DK + grow;
+      return SF ? *reinterpret_cast<const float2*>(gp) : make_float2(*gp, 0.f);
+    };
+    // bf16 V (as loaded) -> fp16 in place in stage `s` (WG: times the write
+    // gate), rows past the chunk's `len` tokens -> 0.  Each 16-byte chunk
+    // stays within its 128-byte row under the swizzle.
+    auto convert_v = [&](int s, int c) {
+      const int len = chunk_len(c);
+      const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
+      uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
+      for (int e = tid; e < C * 8; e += kCarryCompute) {
+        uint4 raw = vt[e];
+        const int row = e >> 3;
+        if (row < len) {
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          float f[8];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 x2 = __bfloat1622float2(p2[t]);
+            f[2 * t] = x2.x;
+            f[2 * t + 1] = x2.y;
+          }
+          if constexpr (WG) {
+            // logical columns of this 16-byte chunk: 8 * (chunk ^ (row % 8));
+            // only the slice's own NBV columns are used (and read)
+            const int col = 8 * ((e & 7) ^ (row & 7));
+            if (col < NBV) {
+              const float* wp = wg + ((size_t)(t0c + row) * H + h) * DV + jv + col;
+              const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
+              const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp + 4));
+              f[0] *= w0.x; f[1] *= w0.y; f[2] *= w0.z; f[3] *= w0.w;
+              f[4] *= w1.x; f[5] *= w1.y; f[6] *= w1.z; f[7] *= w1.w;
+            }
+          }
+          raw = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]),
+                           pack_f16x2(f[4], f[5]), pack_f16x2(f[6], f[7]));
+        } else {
+          raw = make_uint4(0u, 0u, 0u, 0u);
+        }
+        vt[e] = raw;
+      }
+    };
+    // WG: the write-gate rows of chunk c pulled into L2 (one 128-byte line
+    // per thread) a chunk before its conversion reads them
+    auto prefetch_w = [&](int c) {
+      if constexpr (WG) {
+        constexpr int LPR = NBV / 32;  // 128-byte lines per row
+        const int r = tid / LPR;
+        if (has_v && c < nchunks && r < chunk_len(c))
+          prefetch_l2(wg + ((size_t)(tok0 + (int64_t)(cbeg + c) * C + r) * H + h) * DV + jv +
+                      32 * (tid % LPR));
+      }
+    };
+    // V of `c` into stage `s`, once the stage has landed; then tell the MMA thread
+    auto ready_v = [&](int s, int c) -> bool {
+      if (!wait(bar + CB_FULL + 8 * s, (uint32_t)(c >> 1) & 1u)) return false;
+      convert_v(s, c);
+      fence_proxy_async_smem();
+      mbar_arrive(bar + CB_VRDY + 8 * s);
+      return true;
+    };
+
+    if (has_v && nchunks > 0) {
+      prefetch_w(1);
+      ok = ready_v(0, 0);
+    }
+    float2 gm = load_gamma(0);
+    for (int c = 0; ok && c < nchunks; ++c) {
+      const int st = c & 1;
+      const uint32_t par = (uint32_t)c & 1u;
+      const int64_t t0 = tok0 + (int64_t)(cbeg + c) * C;
+      const int Lc = chunk_len(c);
+      const bool to = tma_out(c);
+      const float2 gm_next = load_gamma(c + 1);
+
+      // ---- carry 1 done: U -> operand tile, O -> out ----------------------------
+      if (!wait(bar + CB_X, par)) { ok = 0; break; }
+      tc_fence_after();
+      {
+        float x[CPT];
+        if constexpr (CPT == 32)
+          tmem_ld32(taddr(tmem, 32 * q4, TM2_X + CPT * half), x);
+        else
+          tmem_ld16(taddr(tmem, 32 * q4, TM2_X + CPT * half), x);
+        tmem_ld_wait();
+        if (q4 < 2) {
+#pragma unroll
+          for (int c4 = 0; c4 < CPT / 8; ++c4)
+            st_chunk8(sm + OFF2_UB, sw128_chunk(srow, CPT * half + 8 * c4, 64), x + 8 * c4);
+        } else if (!summary) {
+          const int r = srow - 64;
+          if (to) {
+            // the previous chunk's output store must have read its staging
+            if (c > 0 && !wait(bar + CB_OB, par ^ 1u)) { ok = 0; break; }
+            stage_row<CPT>(sb + OFF2_OB, r, CPT * half, x, Tout());
+          } else if (r < Lc) {
+            store_row<CPT>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + CPT * half, x);
           }
         }
-        raw = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]), pack_f16x2(f[4], f[5]),
-                         pack_f16x2(f[6], f[7]));
-      } else {
-        raw = make_uint4(0u, 0u, 0u, 0u);
       }
-      vt[e] = raw;
-    }
-  };
-  // WG: the write-gate rows of chunk c pulled into L2 (one 128-byte line per
-  // thread) a chunk before its conversion reads them
-  auto prefetch_w = [&](int c) {
-    if constexpr (WG) {
-      constexpr int LPR = NBV / 32;  // 128-byte lines per row
-      const int r = tid / LPR;
-      if (!mcols && c < nchunks && r < chunk_len(c))
-        prefetch_l2(wg + ((size_t)(tok0 + (int64_t)(cbeg + c) * C + r) * H + h) * DV + jv +
-                    32 * (tid % LPR));
-    }
-  };
-  // Shared-memory descriptors of the carry's operands: the base of each
-  // tile; a K step adds its byte offset / 16 to the low field.
-  // (a stage's descriptors are stage 0's plus kStageBytes / 16)
-  const uint64_t d_ip0 = smem_desc(sb + CS_IP, 16, 1024, kSwizzle128);
-  const uint64_t d_v0 = smem_desc(sb + CS_V, 8192, 1024, kSwizzle128);
-  const uint64_t d_wq0 = smem_desc(sb + CS_WQ, 16, 1024, kSwizzle128);
-  const uint64_t d_kh0 = smem_desc(sb + CS_KH, 8192, 1024, kSwizzle128);
-  auto stg = [](int s2) -> uint64_t { return s2 ? (uint64_t)(kStageBytes >> 4) : 0ull; };
-  const uint64_t d_sb = smem_desc(sb + OFF2_SB, 8192, 1024, kSwizzle128);
-  const uint64_t d_ub = smem_desc(sb + OFF2_UB, 8192, 1024, kSwizzle128);
-  constexpr uint32_t id_c1 = idesc_f16(128, NBV, 0, 1);
-  constexpr uint32_t id_c2 = idesc_f16(128, NBV, 1, 1);
-  // carry 1 in two parts: the V term (independent of S) and the S term
-  auto mma_v = [&](int s2, uint32_t acc0) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_f16(tmem + TM2_X, d_ip0 + stg(s2) + 2 * kk, d_v0 + stg(s2) + 128 * kk, id_c1,
-              (kk > 0 || acc0) ? 1u : 0u);
-  };
-  auto mma_s = [&](int s2, uint32_t acc0) {
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      mma_f16(tmem + TM2_X, d_wq0 + stg(s2) + 1024 * (kk >> 2) + 2 * (kk & 3), d_sb + 128 * kk,
-              id_c1,
-              (kk > 0 || acc0) ? 1u : 0u);
-  };
-  // With V: the V term of chunk c goes in as soon as chunk c's V tile is in
-  // fp16 (for c > 0 while carry 2 of chunk c - 1 finishes), so only the
-  // S term of carry 1 is left on the chunk-to-chunk path.
-  if (v_early && nchunks > 0) {
-    prefetch_w(1);
-    ok = wait(bar_full0, ph0, pend0);
-    if (ok) convert_v(0, 0);
-    fence_proxy_async_smem();
-  }
-  ok = __syncthreads_and(ok);
-  if (ok && v_early && nchunks > 0 && tid == 0) {
-    tc_fence_after();
-    mma_v(0, 0u);
-  }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar + CB_U);
 
-  for (int c = 0; ok && c < nchunks; ++c) {
-    const int st = c & 1;
-    const int64_t t0 = tok0 + (int64_t)(cbeg + c) * C;
-    const int Lc = chunk_len(c);
-    // (the bf16 output map's box is 64 columns wide: a 32-column slice stores
-    // its rows with plain stores)
-    const bool tma_out =
-        !summary && ((cu == nullptr) || Lc == C) && (NBV == 64 || sizeof(Tout) == 4);
-    if (!v_early) {
-      // (with V the previous chunk's last barrier already combined `ok`)
-      ok = st ? wait(bar_full0 + 8, ph1, pend1) : wait(bar_full0, ph0, pend0);
-      ok = __syncthreads_and(ok);
-      if (!ok) break;
-    }
-    const float2 gm_next = load_gamma(c + 1);
-    TC_MARK(9);
+      // ---- while carry 2 runs: the next chunk's V ---------------------------------
+      if (has_v && c + 1 < nchunks) {
+        prefetch_w(c + 2);
+        if (!ready_v(st ^ 1, c + 1)) { ok = 0; break; }
+      }
 
-    // ---- carry 1: [U; O] = [Inv diag(beta); P] V + [-W; Q'] S -------------------
-    if (tid == 0) {
+      // ---- carry 2 done: S <- Diag(gamma) S + D, its fp16 copy for the next chunk --
+      if (!wait(bar + CB_D, par)) { ok = 0; break; }
       tc_fence_after();
-      if (!v_early && !mcols) mma_v(st, 0u);
-      mma_s(st, mcols ? 0u : 1u);
-      mma_commit(bar_mma);
-    }
-    pend_mma = 1;
-    ok = wait(bar_mma, ph_mma, pend_mma);
-    // the previous chunk's output store must have read its staging
-    if (tid == 0) bulk_wait_read_all();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    tc_fence_after();
-    TC_MARK(10);
-
-    // ---- U -> operand;  O -> out ---------------------------------------------------
-    {
-      float x[CPT];
-      if constexpr (CPT == 32)
-        tmem_ld32(taddr(tmem, 32 * q4, TM2_X + CPT * half), x);
-      else
-        tmem_ld16(taddr(tmem, 32 * q4, TM2_X + CPT * half), x);
-      tmem_ld_wait();
-      TC_DBG(for (int e = 0; e < CPT; ++e) g_tc_dbg[32768 + srow * 64 + CPT * half + e] = x[e]);
-      if (q4 < 2) {
+      {
+        float d[CPT];
+        if constexpr (CPT == 32)
+          tmem_ld32(taddr(tmem, 32 * q4, TM2_D + CPT * half), d);
+        else
+          tmem_ld16(taddr(tmem, 32 * q4, TM2_D + CPT * half), d);
+        tmem_ld_wait();
+        if constexpr (SF) {
+          // even row: gr S_e - gi S_o + d;  odd row: gr S_o + gi S_e + d
+          const float gi = (lane & 1) ? gm.y : -gm.y;
+#pragma unroll
+          for (int e = 0; e < CPT; ++e) {
+            const float po = __shfl_xor_sync(0xffffffffu, S[e], 1);
+            S[e] = fmaf(gm.x, S[e], fmaf(gi, po, d[e]));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < CPT; ++e) S[e] = fmaf(gm.x, S[e], d[e]);
+        }
 #pragma unroll
         for (int c4 = 0; c4 < CPT / 8; ++c4)
-          st_chunk8(sm + OFF2_UB, sw128_chunk(srow, CPT * half + 8 * c4, 64), x + 8 * c4);
-      } else if (!summary) {
-        const int r = srow - 64;
-        if (tma_out)
-          stage_row<CPT>(sb + OFF2_OB, r, CPT * half, x, Tout());
-        else if (r < Lc)
-          store_row<CPT>(out + ((size_t)(t0 + r) * H + h) * DV + j0 + CPT * half, x);
+          st_chunk8(sm + OFF2_SB, sw128_chunk(srow, CPT * half + 8 * c4, 128), S + 8 * c4);
       }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    TC_MARK(11);
-
-    // ---- carry 2: D = (K rho)^T U;  S <- Diag(gamma) S + D ----------------------
-    if (tid == 0) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f16(tmem + TM2_D, d_kh0 + stg(st) + 128 * kk, d_ub + 128 * kk, id_c2,
-                kk > 0 ? 1u : 0u);
-      mma_commit(bar_mma);
-    }
-    pend_mma = 1;
-    if (tma_out && tid == 0) {
-      // fixed-length batch: [T, H * d_v] per sequence, rows past T are clipped;
-      // packed batch: only whole chunks go through TMA
-      const int x0 = h * DV + j0;
-      if (cu == nullptr) {
-        const int y0 = (cbeg + c) * C;
-        if (sizeof(Tout) == 4) {
-          tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
-          if (NBV == 64) tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, y0, n);
-        } else {
-          tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
-        }
-      } else {
-        if (sizeof(Tout) == 4) {
-          tma_store_2d(&tm_out, sb + OFF2_OB, x0, (int)t0);
-          if (NBV == 64) tma_store_2d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, (int)t0);
-        } else {
-          tma_store_2d(&tm_out, sb + OFF2_OB, x0, (int)t0);
-        }
-      }
-      bulk_commit();
-    }
-    // while carry 2 runs: the next chunk's stage, its V converted to fp16
-    if (v_early && c + 1 < nchunks) {
-      prefetch_w(c + 2);
-      ok = st ? wait(bar_full0, ph0, pend0) : wait(bar_full0 + 8, ph1, pend1);
-      if (ok) convert_v(st ^ 1, c + 1);
-      // the converted tile is read by carry 1's V term right after the barrier
+      gm = gm_next;
       fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar + CB_SRDY);
     }
-    ok = wait(bar_mma, ph_mma, pend_mma) && ok;
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    tc_fence_after();
-    // carry 1's V term of the next chunk (its accumulator was read out above)
-    if (v_early && c + 1 < nchunks && tid == 0) mma_v(st ^ 1, 0u);
-    // this stage is consumed: fetch chunk c + 2 into it
-    if (c + 2 < nchunks) {
-      if (tid == 0) issue(c + 2, st);
-      if (st)
-        pend1 = 1;
-      else
-        pend0 = 1;
-    }
-    {
-      float d[CPT];
-      if constexpr (CPT == 32)
-        tmem_ld32(taddr(tmem, 32 * q4, TM2_D + CPT * half), d);
-      else
-        tmem_ld16(taddr(tmem, 32 * q4, TM2_D + CPT * half), d);
-      tmem_ld_wait();
-      if constexpr (SF) {
-        // even row: gr S_e - gi S_o + d;  odd row: gr S_o + gi S_e + d
-        const float gi = (lane & 1) ? gm.y : -gm.y;
+  } else if (warp == 8) {
+    // ---- MMA thread ---------------------------------------------------------------------
+    if (lane == 0) {
+      // Shared-memory descriptors of the carry's operands: the base of each
+      // tile; a K step adds its byte offset / 16 to the low field (a stage's
+      // descriptors are stage 0's plus kStageBytes / 16).
+      const uint64_t d_ip0 = smem_desc(sb + CS_IP, 16, 1024, kSwizzle128);
+      const uint64_t d_v0 = smem_desc(sb + CS_V, 8192, 1024, kSwizzle128);
+      const uint64_t d_wq0 = smem_desc(sb + CS_WQ, 16, 1024, kSwizzle128);
+      const uint64_t d_kh0 = smem_desc(sb + CS_KH, 8192, 1024, kSwizzle128);
+      const uint64_t d_sb = smem_desc(sb + OFF2_SB, 8192, 1024, kSwizzle128);
+      const uint64_t d_ub = smem_desc(sb + OFF2_UB, 8192, 1024, kSwizzle128);
+      constexpr uint32_t id_c1 = idesc_f16(128, NBV, 0, 1);
+      constexpr uint32_t id_c2 = idesc_f16(128, NBV, 1, 1);
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c & 1;
+        const uint32_t par = (uint32_t)c & 1u;
+        const uint32_t spar = (uint32_t)(c >> 1) & 1u;
+        const uint64_t so = st ? (uint64_t)(kStageBytes >> 4) : 0ull;
+        // the stage's factors have landed
+        if (!wait(bar + CB_FULL + 8 * st, spar)) { ok = 0; break; }
+        if (has_v) {
+          // carry 1's V term, [Inv diag(beta); P] V: independent of S, in as
+          // soon as V is fp16 (the accumulator was read out before carry 2
+          // of the previous chunk was issued)
+          if (!wait(bar + CB_VRDY + 8 * st, spar)) { ok = 0; break; }
+          tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < CPT; ++e) {
-          const float po = __shfl_xor_sync(0xffffffffu, S[e], 1);
-          S[e] = fmaf(gm.x, S[e], fmaf(gi, po, d[e]));
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f16(tmem + TM2_X, d_ip0 + so + 2 * kk, d_v0 + so + 128 * kk, id_c1,
+                    kk > 0 ? 1u : 0u);
         }
-      } else {
+        // carry 1's S term, [-W; Q'] S
+        if (!wait(bar + CB_SRDY, par)) { ok = 0; break; }
+        tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < CPT; ++e) S[e] = fmaf(gm.x, S[e], d[e]);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_f16(tmem + TM2_X, d_wq0 + so + 1024 * (kk >> 2) + 2 * (kk & 3), d_sb + 128 * kk,
+                  id_c1, (kk > 0 || has_v) ? 1u : 0u);
+        mma_commit(bar + CB_X);
+        mma_pend = 1; mma_bar = bar + CB_X; mma_par = par;
+        // carry 2, D = (K rho)^T U, once U is in its tile
+        if (!wait(bar + CB_U, par)) { ok = 0; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f16(tmem + TM2_D, d_kh0 + so + 128 * kk, d_ub + 128 * kk, id_c2, kk > 0 ? 1u : 0u);
+        mma_commit(bar + CB_D);
+        mma_bar = bar + CB_D;
       }
-      TC_DBG(for (int e = 0; e < CPT; ++e) {
-        g_tc_dbg[49152 + srow * 64 + CPT * half + e] = d[e];
-        g_tc_dbg[57344 + srow * 64 + CPT * half + e] = S[e];
-      });
-#pragma unroll
-      for (int c4 = 0; c4 < CPT / 8; ++c4)
-        st_chunk8(sm + OFF2_SB, sw128_chunk(srow, CPT * half + 8 * c4, 128), S + 8 * c4);
-    }
-    gm = gm_next;
-    fence_proxy_async_smem();
-    tc_fence_before();
-    ok = __syncthreads_and(ok);
-    if (!ok) break;
-    TC_MARK(12);
-  }
-#ifdef CKDA_TC_DEBUG
-  if (g_tc_time != nullptr && tid == 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
-    for (int k = 9; k < 13; ++k) g_tc_time[k] = tmark[k];
-#endif
-  if (tid == 0) bulk_wait_all();
-
-  if (ok) {
-    if (summary) {
-      float* dst = summ + (((size_t)n * seg_launch + seg) * H + h) * DK * (DK + DV) +
-                   (size_t)srow * (DK + DV) + j0 + CPT * half;
-#pragma unroll
-      for (int e = 0; e < CPT; e += 4)
-        *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
-    } else if (S_final != nullptr && seg == seg_n - 1) {
-#pragma unroll
-      for (int e = 0; e < CPT; e += 4)
-        *reinterpret_cast<float4*>(S_final + s_off + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
     }
   } else {
-    if (tid == 0) {
-      set_status(status, CKDA_ERR_DEVICE_TIMEOUT);
-      if (pend0) mbar_wait_bounded(bar_full0, ph0, kWaitNs);
-      if (pend1) mbar_wait_bounded(bar_full0 + 8, ph1, kWaitNs);
-      if (pend_mma) mbar_wait_bounded(bar_mma, ph_mma, kWaitNs);
+    // ---- copy thread: stage loads and output stores by TMA ----------------------------
+    if (lane == 0) {
+      auto issue = [&](int c, int st) {
+        const uint32_t b = bar + CB_FULL + 8 * st;
+        const uint32_t base = sb + st * kStageBytes;
+        const int64_t uidx = unit_of(c);
+        mbar_expect_tx(b, kStageBytes);
+        tma_load_2d(base + CS_WQ, &tm_wq, 0, (int)(uidx * 2 * C), b);
+        tma_load_2d(base + CS_WQ + 16384, &tm_wq, 64, (int)(uidx * 2 * C), b);
+        tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), b);
+        tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), b);
+        tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), b);
+        tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
+                    (int)(tok0 + (int64_t)(cbeg + c) * C), b);
+        ld_pend |= 1u << st;
+        ld_par = (ld_par & ~(1u << st)) | (((uint32_t)(c >> 1) & 1u) << st);
+      };
+      if (nchunks > 0) issue(0, 0);
+      if (nchunks > 1) issue(1, 1);
+      for (int c = 0; c < nchunks; ++c) {
+        const int st = c & 1;
+        const uint32_t par = (uint32_t)c & 1u;
+        const bool to = tma_out(c);
+        // O of the chunk staged: store it
+        if (!wait(bar + CB_U, par)) { ok = 0; break; }
+        if (to) {
+          // fixed-length batch: [T, H * d_v] per sequence, rows past T are
+          // clipped; packed batch: only whole chunks come here
+          const int x0 = h * DV + j0;
+          if (cu == nullptr) {
+            const int y0 = (cbeg + c) * C;
+            tma_store_3d(&tm_out, sb + OFF2_OB, x0, y0, n);
+            if (sizeof(Tout) == 4 && NBV == 64)
+              tma_store_3d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, y0, n);
+          } else {
+            const int t0 = (int)(tok0 + (int64_t)(cbeg + c) * C);
+            tma_store_2d(&tm_out, sb + OFF2_OB, x0, t0);
+            if (sizeof(Tout) == 4 && NBV == 64)
+              tma_store_2d(&tm_out, sb + OFF2_OB + 8192, x0 + 32, t0);
+          }
+          bulk_commit();
+        }
+        // both products of the chunk are done with its stage: fetch chunk c + 2
+        if (!wait(bar + CB_D, par)) { ok = 0; break; }
+        ld_pend &= ~(1u << st);
+        if (c + 2 < nchunks) issue(c + 2, st);
+        if (to) bulk_wait_read_all();
+        mbar_arrive(bar + CB_OB);
+      }
+      bulk_wait_all();
+    }
+  }
+
+  ok = __syncthreads_and(ok);
+  if (ok) {
+    if (warp < 8) {
+      const int q4 = warp & 3;
+      const int half = warp >> 2;
+      const int srow = 32 * q4 + lane;
+      if (summary) {
+        float* dst = summ + (((size_t)n * seg_launch + seg) * H + h) * DK * (DK + DV) +
+                     (size_t)srow * (DK + DV) + j0 + CPT * half;
+#pragma unroll
+        for (int e = 0; e < CPT; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+      } else if (S_final != nullptr && seg == seg_n - 1) {
+        float* dst = S_final + (((size_t)n * H + h) * DK + srow) * DV + j0 + CPT * half;
+#pragma unroll
+        for (int e = 0; e < CPT; e += 4)
+          *reinterpret_cast<float4*>(dst + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+      }
+    }
+  } else {
+    if (tid == 0) set_status(status, CKDA_ERR_DEVICE_TIMEOUT);
+    // every copy and MMA this CTA issued completes before its memory goes
+    if (warp == 8 && lane == 0 && mma_pend) mbar_wait_bounded(mma_bar, mma_par, kWaitNs);
+    if (warp == 9 && lane == 0) {
+      for (int s2 = 0; s2 < 2; ++s2)
+        if ((ld_pend >> s2) & 1u)
+          mbar_wait_bounded(bar + CB_FULL + 8 * s2, (ld_par >> s2) & 1u, kWaitNs);
     }
   }
   tc_fence_before();
@@ -1845,7 +1828,7 @@ cudaError_t launch_t(int phases, const void* q, const void* k, const void* v, co
       attr2[narrow] = true;
     }
     dim3 grid(cols / (narrow ? 32 : BV), H, n_seqs * segs.launch);
-    k2<<<grid, NT, kSmem2Bytes, stream>>>(mwq, mkh, mip, mvin, mout, ws_g, wg, S0, cu,
+    k2<<<grid, kCarryThreads, kSmem2Bytes, stream>>>(mwq, mkh, mip, mvin, mout, ws_g, wg, S0, cu,
                                           static_cast<Tout*>(out), S_final, n_seqs, T, H, DV,
                                           nch, status, segs.n, segs.launch, segs.start,
                                           segs.summ);
