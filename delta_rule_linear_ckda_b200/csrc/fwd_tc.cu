@@ -21,13 +21,16 @@
 //       Q' = Q * Gamma - A W
 //     and writes [-W; Q'], K * rho, [Inv diag(beta); P] (fp16) and gamma
 //     (fp32) of the unit to a workspace.
-//  2. carry_kernel -- one CTA per (sequence, head, 64-column d_v slice)
-//     walks its chunks in order with two dependent tensor-core products each:
+//  2. carry_kernel -- one CTA per (sequence, head, 64- or 32-column d_v
+//     slice) walks its chunks in order with two dependent tensor-core
+//     products each:
 //       [U; O] = [Inv diag(beta); P] V + [-W; Q'] S0    (carry MMA 1)
 //       D  = (K * rho)^T U,  S_C = Diag(gamma) S0 + D   (carry MMA 2)
 //     since U = U~ - W S0 and O = A U~ + Q' S0 with [U~; A U~] =
-//     [Inv diag(beta); P] V, while TMA streams the next chunk's factors (and
-//     its bf16 V tile) in.
+//     [Inv diag(beta); P] V.  Its warps have fixed roles (state and
+//     read-outs, MMA issue, TMA copies) and pass each chunk on through
+//     mbarriers, while TMA streams the next chunk's factors (and its bf16 V
+//     tile) in.
 //
 // Division-free score blocks: every pair s < r is split at the anchor m of
 // the highest bit in which r and s differ ("level" h, block size b = 2^h):
@@ -76,7 +79,6 @@ using namespace sm100;
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int BV = 64;  // d_v columns of one carry CTA
-constexpr int NT = 256;   // carry kernel threads
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per wait
 
 // Level operands of the factor kernel: levels are paired (2, 3) and (4, 5),
@@ -114,9 +116,10 @@ constexpr uint32_t CB_FULL = 0;   // stage s loaded (TMA transaction), + 8 s
 constexpr uint32_t CB_VRDY = 16;  // stage s's V converted to fp16 (compute threads), + 8 s
 constexpr uint32_t CB_SRDY = 32;  // the state's fp16 operand written (compute threads)
 constexpr uint32_t CB_X = 40;     // carry 1 ([U; O]) complete (tensor-core commit)
-constexpr uint32_t CB_U = 48;     // U in its operand tile, O staged or stored (compute threads)
+constexpr uint32_t CB_U = 48;     // U in its operand tile (the compute threads of rows 0..63)
 constexpr uint32_t CB_D = 56;     // carry 2 (D) complete (tensor-core commit)
 constexpr uint32_t CB_OB = 64;    // the output staging free again (store warp)
+constexpr uint32_t CB_O = 72;     // O read out, staged or stored (the threads of rows 64..127)
 constexpr int kCarryCompute = 256;              // state / epilogue threads (8 warps)
 constexpr int kCarryThreads = kCarryCompute + 64;  // + one MMA warp, one copy warp
 constexpr uint32_t kSmem2Used = OFF2_TMEMPTR + 16;
@@ -1210,9 +1213,10 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     mbar_init(bar + CB_VRDY + 8, kCarryCompute);
     mbar_init(bar + CB_SRDY, kCarryCompute);
     mbar_init(bar + CB_X, 1);
-    mbar_init(bar + CB_U, kCarryCompute);
+    mbar_init(bar + CB_U, kCarryCompute / 2);
     mbar_init(bar + CB_D, 1);
     mbar_init(bar + CB_OB, 1);
+    mbar_init(bar + CB_O, kCarryCompute / 2);
     fence_mbar_init();
     prefetch_tmap(&tm_wq);
     prefetch_tmap(&tm_kh);
@@ -1316,8 +1320,12 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       const int len = chunk_len(c);
       const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
       uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
-      for (int e = tid; e < C * 8; e += kCarryCompute) {
-        uint4 raw = vt[e];
+      static_assert(C * 8 == 2 * kCarryCompute, "two 16-byte chunks of V per thread");
+      uint4 raws[2] = {vt[tid], vt[tid + kCarryCompute]};
+#pragma unroll
+      for (int it = 0; it < 2; ++it) {
+        const int e = tid + it * kCarryCompute;
+        uint4 raw = raws[it];
         const int row = e >> 3;
         if (row < len) {
           const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -1406,9 +1414,11 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
           }
         }
       }
+      // (rows 0..63 release carry 2, rows 64..127 the output store and the
+      // accumulator)
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar + CB_U);
+      mbar_arrive(bar + (q4 < 2 ? CB_U : CB_O));
 
       // ---- while carry 2 runs: the next chunk's V ---------------------------------
       if (has_v && c + 1 < nchunks) {
@@ -1468,10 +1478,12 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const uint64_t so = st ? (uint64_t)(kStageBytes >> 4) : 0ull;
         // the stage's factors have landed
         if (!wait(bar + CB_FULL + 8 * st, spar)) { ok = 0; break; }
+        // the previous chunk's O rows of the accumulator have been read out
+        if (c > 0 && !wait(bar + CB_O, par ^ 1u)) { ok = 0; break; }
         if (has_v) {
           // carry 1's V term, [Inv diag(beta); P] V: independent of S, in as
-          // soon as V is fp16 (the accumulator was read out before carry 2
-          // of the previous chunk was issued)
+          // soon as V is fp16 (the U rows of the accumulator were read out
+          // before carry 2 of the previous chunk was issued)
           if (!wait(bar + CB_VRDY + 8 * st, spar)) { ok = 0; break; }
           tc_fence_after();
 #pragma unroll
@@ -1523,7 +1535,7 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const uint32_t par = (uint32_t)c & 1u;
         const bool to = tma_out(c);
         // O of the chunk staged: store it
-        if (!wait(bar + CB_U, par)) { ok = 0; break; }
+        if (!wait(bar + CB_O, par)) { ok = 0; break; }
         if (to) {
           // fixed-length batch: [T, H * d_v] per sequence, rows past T are
           // clipped; packed batch: only whole chunks come here
