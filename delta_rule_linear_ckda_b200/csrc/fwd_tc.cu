@@ -112,16 +112,19 @@ constexpr uint32_t OFF2_OB = OFF2_UB + 8192;  // O staging for its TMA store: fp
 constexpr uint32_t OFF2_BAR = OFF2_OB + 16384;  // mbarriers (below)
 constexpr uint32_t OFF2_TMEMPTR = OFF2_BAR + 128;
 // carry mbarriers, byte offsets from OFF2_BAR
-constexpr uint32_t CB_FULL = 0;   // stage s loaded (TMA transaction), + 8 s
-constexpr uint32_t CB_VRDY = 16;  // stage s's V converted to fp16 (compute threads), + 8 s
-constexpr uint32_t CB_SRDY = 32;  // the state's fp16 operand written (compute threads)
-constexpr uint32_t CB_X = 40;     // carry 1 ([U; O]) complete (tensor-core commit)
-constexpr uint32_t CB_U = 48;     // U in its operand tile (the compute threads of rows 0..63)
-constexpr uint32_t CB_D = 56;     // carry 2 (D) complete (tensor-core commit)
-constexpr uint32_t CB_OB = 64;    // the output staging free again (store warp)
-constexpr uint32_t CB_O = 72;     // O read out, staged or stored (the threads of rows 64..127)
-constexpr int kCarryCompute = 256;              // state / epilogue threads (8 warps)
-constexpr int kCarryThreads = kCarryCompute + 64;  // + one MMA warp, one copy warp
+constexpr uint32_t CB_FULLA = 0;  // stage s: [-W; Q'], [Inv diag(beta); P], V loaded, + 8 s
+constexpr uint32_t CB_FULLB = 16; // stage s: K * rho loaded, + 8 s
+constexpr uint32_t CB_VRDY = 32;  // stage s's V converted to fp16 (conversion threads), + 8 s
+constexpr uint32_t CB_SRDY = 48;  // the state's fp16 operand written (compute threads)
+constexpr uint32_t CB_X = 56;     // carry 1 ([U; O]) complete (tensor-core commit)
+constexpr uint32_t CB_U = 64;     // U in its operand tile (the compute threads of rows 0..63)
+constexpr uint32_t CB_D = 72;     // carry 2 (D) complete (tensor-core commit)
+constexpr uint32_t CB_OB = 80;    // the output staging free again (copy thread)
+constexpr uint32_t CB_O = 88;     // O read out, staged or stored (the threads of rows 64..127)
+constexpr uint32_t kStageBytesA = 73728 - 16384;  // a stage less K * rho
+constexpr int kCarryCompute = 256;  // state / epilogue threads (8 warps)
+constexpr int kCarryConvert = 128;  // V conversion threads (4 warps)
+constexpr int kCarryThreads = kCarryCompute + 64 + kCarryConvert;  // + MMA warp, copy warp
 constexpr uint32_t kSmem2Used = OFF2_TMEMPTR + 16;
 constexpr size_t kSmem2Bytes = kSmem2Used + 1024;
 
@@ -1207,10 +1210,12 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
 
   const uint32_t bar = sb + OFF2_BAR;
   if (tid == 0) {
-    mbar_init(bar + CB_FULL, 1);
-    mbar_init(bar + CB_FULL + 8, 1);
-    mbar_init(bar + CB_VRDY, kCarryCompute);
-    mbar_init(bar + CB_VRDY + 8, kCarryCompute);
+    mbar_init(bar + CB_FULLA, 1);
+    mbar_init(bar + CB_FULLA + 8, 1);
+    mbar_init(bar + CB_FULLB, 1);
+    mbar_init(bar + CB_FULLB + 8, 1);
+    mbar_init(bar + CB_VRDY, kCarryConvert);
+    mbar_init(bar + CB_VRDY + 8, kCarryConvert);
     mbar_init(bar + CB_SRDY, kCarryCompute);
     mbar_init(bar + CB_X, 1);
     mbar_init(bar + CB_U, kCarryCompute / 2);
@@ -1256,21 +1261,25 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
   };
   int ok = 1;
 
-  // Three roles hand each chunk to one another through mbarriers, so that
+  // Four roles hand each chunk to one another through mbarriers, so that
   // no block-wide barrier stands between the steps of the chunk-to-chunk
   // chain (S -> carry 1 -> U -> carry 2 -> S):
   //  * warps 0..7 (compute): the state slice in registers, the read-outs of
   //    both tensor-memory products, U into its operand tile, O staged or
-  //    stored, V of the next chunk converted to fp16;
+  //    stored;
   //  * warp 8 (one thread): every tcgen05 MMA;
   //  * warp 9 (one thread): the stage loads and the output stores by TMA.
+  //    A stage is loaded in two parts: what carry 1 reads ([-W; Q'],
+  //    [Inv diag(beta); P], V) is fetched again as soon as carry 1 is done
+  //    with it, K * rho once carry 2 is;
+  //  * warps 10..13 (conversion): each chunk's V to fp16 as soon as it lands.
   // Each barrier completes once per chunk (the stage barriers once per two),
   // so the parity waited for follows from the chunk index.
   float S[CPT];
   int mma_pend = 0;            // MMA thread: a commit not yet seen complete
   uint32_t mma_bar = 0, mma_par = 0;
-  uint32_t ld_pend = 0;        // copy thread: bit s, a load into stage s not yet seen complete
-  uint32_t ld_par = 0;         //   bit s, the parity of that load's phase
+  uint32_t ld_pend = 0;        // copy thread: bit 2 s + part, a load not yet seen complete
+  uint32_t ld_par = 0;         //   the same bit, the parity of that load's phase
 
   if (warp < 8) {
     // ---- compute warps ----------------------------------------------------------------
@@ -1313,76 +1322,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       const float* gp = ws_g + unit_of(c) * DK + grow;
       return SF ? *reinterpret_cast<const float2*>(gp) : make_float2(*gp, 0.f);
     };
-    // bf16 V (as loaded) -> fp16 in place in stage `s` (WG: times the write
-    // gate), rows past the chunk's `len` tokens -> 0.  Each 16-byte chunk
-    // stays within its 128-byte row under the swizzle.
-    auto convert_v = [&](int s, int c) {
-      const int len = chunk_len(c);
-      const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
-      uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
-      static_assert(C * 8 == 2 * kCarryCompute, "two 16-byte chunks of V per thread");
-      uint4 raws[2] = {vt[tid], vt[tid + kCarryCompute]};
-#pragma unroll
-      for (int it = 0; it < 2; ++it) {
-        const int e = tid + it * kCarryCompute;
-        uint4 raw = raws[it];
-        const int row = e >> 3;
-        if (row < len) {
-          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-          float f[8];
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 x2 = __bfloat1622float2(p2[t]);
-            f[2 * t] = x2.x;
-            f[2 * t + 1] = x2.y;
-          }
-          if constexpr (WG) {
-            // logical columns of this 16-byte chunk: 8 * (chunk ^ (row % 8));
-            // only the slice's own NBV columns are used (and read)
-            const int col = 8 * ((e & 7) ^ (row & 7));
-            if (col < NBV) {
-              const float* wp = wg + ((size_t)(t0c + row) * H + h) * DV + jv + col;
-              const float4 w0 = __ldg(reinterpret_cast<const float4*>(wp));
-              const float4 w1 = __ldg(reinterpret_cast<const float4*>(wp + 4));
-              f[0] *= w0.x; f[1] *= w0.y; f[2] *= w0.z; f[3] *= w0.w;
-              f[4] *= w1.x; f[5] *= w1.y; f[6] *= w1.z; f[7] *= w1.w;
-            }
-          }
-          raw = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]),
-                           pack_f16x2(f[4], f[5]), pack_f16x2(f[6], f[7]));
-        } else {
-          raw = make_uint4(0u, 0u, 0u, 0u);
-        }
-        vt[e] = raw;
-      }
-    };
-    // WG: the write-gate rows of chunk c pulled into L2 (one 128-byte line
-    // per thread) a chunk before its conversion reads them
-    auto prefetch_w = [&](int c) {
-      if constexpr (WG) {
-        constexpr int LPR = NBV / 32;  // 128-byte lines per row
-        const int r = tid / LPR;
-        if (has_v && c < nchunks && r < chunk_len(c))
-          prefetch_l2(wg + ((size_t)(tok0 + (int64_t)(cbeg + c) * C + r) * H + h) * DV + jv +
-                      32 * (tid % LPR));
-      }
-    };
-    // V of `c` into stage `s`, once the stage has landed; then tell the MMA thread
-    auto ready_v = [&](int s, int c) -> bool {
-      if (!wait(bar + CB_FULL + 8 * s, (uint32_t)(c >> 1) & 1u)) return false;
-      convert_v(s, c);
-      fence_proxy_async_smem();
-      mbar_arrive(bar + CB_VRDY + 8 * s);
-      return true;
-    };
-
-    if (has_v && nchunks > 0) {
-      prefetch_w(1);
-      ok = ready_v(0, 0);
-    }
     float2 gm = load_gamma(0);
     for (int c = 0; ok && c < nchunks; ++c) {
-      const int st = c & 1;
       const uint32_t par = (uint32_t)c & 1u;
       const int64_t t0 = tok0 + (int64_t)(cbeg + c) * C;
       const int Lc = chunk_len(c);
@@ -1419,12 +1360,6 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar + (q4 < 2 ? CB_U : CB_O));
-
-      // ---- while carry 2 runs: the next chunk's V ---------------------------------
-      if (has_v && c + 1 < nchunks) {
-        prefetch_w(c + 2);
-        if (!ready_v(st ^ 1, c + 1)) { ok = 0; break; }
-      }
 
       // ---- carry 2 done: S <- Diag(gamma) S + D, its fp16 copy for the next chunk --
       if (!wait(bar + CB_D, par)) { ok = 0; break; }
@@ -1476,20 +1411,22 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         const uint32_t par = (uint32_t)c & 1u;
         const uint32_t spar = (uint32_t)(c >> 1) & 1u;
         const uint64_t so = st ? (uint64_t)(kStageBytes >> 4) : 0ull;
-        // the stage's factors have landed
-        if (!wait(bar + CB_FULL + 8 * st, spar)) { ok = 0; break; }
         // the previous chunk's O rows of the accumulator have been read out
         if (c > 0 && !wait(bar + CB_O, par ^ 1u)) { ok = 0; break; }
         if (has_v) {
           // carry 1's V term, [Inv diag(beta); P] V: independent of S, in as
           // soon as V is fp16 (the U rows of the accumulator were read out
           // before carry 2 of the previous chunk was issued)
+          // (V converted implies the stage's first part has landed)
           if (!wait(bar + CB_VRDY + 8 * st, spar)) { ok = 0; break; }
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_f16(tmem + TM2_X, d_ip0 + so + 2 * kk, d_v0 + so + 128 * kk, id_c1,
                     kk > 0 ? 1u : 0u);
+        } else if (!wait(bar + CB_FULLA + 8 * st, spar)) {
+          ok = 0;
+          break;
         }
         // carry 1's S term, [-W; Q'] S
         if (!wait(bar + CB_SRDY, par)) { ok = 0; break; }
@@ -1500,8 +1437,8 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
                   id_c1, (kk > 0 || has_v) ? 1u : 0u);
         mma_commit(bar + CB_X);
         mma_pend = 1; mma_bar = bar + CB_X; mma_par = par;
-        // carry 2, D = (K rho)^T U, once U is in its tile
-        if (!wait(bar + CB_U, par)) { ok = 0; break; }
+        // carry 2, D = (K rho)^T U, once U is in its tile and K rho has landed
+        if (!wait(bar + CB_U, par) || !wait(bar + CB_FULLB + 8 * st, spar)) { ok = 0; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -1510,30 +1447,43 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
         mma_bar = bar + CB_D;
       }
     }
-  } else {
+  } else if (warp == 9) {
     // ---- copy thread: stage loads and output stores by TMA ----------------------------
     if (lane == 0) {
-      auto issue = [&](int c, int st) {
-        const uint32_t b = bar + CB_FULL + 8 * st;
+      // part 0 of chunk c into stage st: [-W; Q'], [Inv diag(beta); P], V;
+      // part 1: K * rho
+      auto issue = [&](int c, int st, int part) {
+        const uint32_t b = bar + (part ? CB_FULLB : CB_FULLA) + 8 * st;
         const uint32_t base = sb + st * kStageBytes;
         const int64_t uidx = unit_of(c);
-        mbar_expect_tx(b, kStageBytes);
-        tma_load_2d(base + CS_WQ, &tm_wq, 0, (int)(uidx * 2 * C), b);
-        tma_load_2d(base + CS_WQ + 16384, &tm_wq, 64, (int)(uidx * 2 * C), b);
-        tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), b);
-        tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), b);
-        tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), b);
-        tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
-                    (int)(tok0 + (int64_t)(cbeg + c) * C), b);
-        ld_pend |= 1u << st;
-        ld_par = (ld_par & ~(1u << st)) | (((uint32_t)(c >> 1) & 1u) << st);
+        if (part == 0) {
+          mbar_expect_tx(b, kStageBytesA);
+          tma_load_2d(base + CS_WQ, &tm_wq, 0, (int)(uidx * 2 * C), b);
+          tma_load_2d(base + CS_WQ + 16384, &tm_wq, 64, (int)(uidx * 2 * C), b);
+          tma_load_2d(base + CS_IP, &tm_ip, 0, (int)(uidx * 2 * C), b);
+          tma_load_2d(base + CS_V, &tm_v16, h * DV + (mcols ? 0 : jv),
+                      (int)(tok0 + (int64_t)(cbeg + c) * C), b);
+        } else {
+          mbar_expect_tx(b, kStageBytes - kStageBytesA);
+          tma_load_2d(base + CS_KH, &tm_kh, 0, (int)(uidx * C), b);
+          tma_load_2d(base + CS_KH + 8192, &tm_kh, 64, (int)(uidx * C), b);
+        }
+        const int bit = 2 * st + part;
+        ld_pend |= 1u << bit;
+        ld_par = (ld_par & ~(1u << bit)) | (((uint32_t)(c >> 1) & 1u) << bit);
       };
-      if (nchunks > 0) issue(0, 0);
-      if (nchunks > 1) issue(1, 1);
+      for (int c = 0; c < 2 && c < nchunks; ++c) {
+        issue(c, c, 0);
+        issue(c, c, 1);
+      }
       for (int c = 0; c < nchunks; ++c) {
         const int st = c & 1;
         const uint32_t par = (uint32_t)c & 1u;
         const bool to = tma_out(c);
+        // carry 1 is done with the stage's first part: fetch chunk c + 2's
+        if (!wait(bar + CB_X, par)) { ok = 0; break; }
+        ld_pend &= ~(1u << (2 * st));
+        if (c + 2 < nchunks) issue(c + 2, st, 0);
         // O of the chunk staged: store it
         if (!wait(bar + CB_O, par)) { ok = 0; break; }
         if (to) {
@@ -1553,14 +1503,95 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
           }
           bulk_commit();
         }
-        // both products of the chunk are done with its stage: fetch chunk c + 2
+        // carry 2 is done with K * rho: fetch chunk c + 2's
         if (!wait(bar + CB_D, par)) { ok = 0; break; }
-        ld_pend &= ~(1u << st);
-        if (c + 2 < nchunks) issue(c + 2, st);
+        ld_pend &= ~(1u << (2 * st + 1));
+        if (c + 2 < nchunks) issue(c + 2, st, 1);
         if (to) bulk_wait_read_all();
         mbar_arrive(bar + CB_OB);
       }
       bulk_wait_all();
+    }
+  } else if (has_v) {
+    // ---- conversion warps ---------------------------------------------------------------
+    const int ct = tid - (kCarryCompute + 64);  // 0 .. kCarryConvert - 1
+    // bf16 V (as loaded) -> fp16 in place in stage `s` (WG: times the write
+    // gate), rows past the chunk's `len` tokens -> 0.  Each 16-byte chunk
+    // stays within its 128-byte row under the swizzle.
+    auto convert_v = [&](int s, int c) {
+      const int len = chunk_len(c);
+      const int64_t t0c = tok0 + (int64_t)(cbeg + c) * C;
+      uint4* vt = reinterpret_cast<uint4*>(sm + s * kStageBytes + CS_V);
+      constexpr int kPer = C * 8 / kCarryConvert;  // 16-byte chunks of V per thread
+      static_assert(C * 8 == kPer * kCarryConvert, "V chunks per thread");
+      // every load of the thread first (V from shared memory; WG: the write
+      // gate from global memory), then the arithmetic
+      uint4 raws[kPer];
+      float4 wa[WG ? kPer : 1], wb[WG ? kPer : 1];
+#pragma unroll
+      for (int it = 0; it < kPer; ++it) {
+        const int e = ct + it * kCarryConvert;
+        raws[it] = vt[e];
+        if constexpr (WG) {
+          // logical columns of this 16-byte chunk: 8 * (chunk ^ (row % 8));
+          // only the slice's own NBV columns are used (and read)
+          const int row = e >> 3;
+          const int col = 8 * ((e & 7) ^ (row & 7));
+          wa[it] = wb[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (row < len && col < NBV) {
+            const float* wp = wg + ((size_t)(t0c + row) * H + h) * DV + jv + col;
+            wa[it] = __ldg(reinterpret_cast<const float4*>(wp));
+            wb[it] = __ldg(reinterpret_cast<const float4*>(wp + 4));
+          }
+        }
+      }
+#pragma unroll
+      for (int it = 0; it < kPer; ++it) {
+        const int e = ct + it * kCarryConvert;
+        const int row = e >> 3;
+        uint4 raw = raws[it];
+        if (row < len) {
+          const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+          float f[8];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 x2 = __bfloat1622float2(p2[t]);
+            f[2 * t] = x2.x;
+            f[2 * t + 1] = x2.y;
+          }
+          if constexpr (WG) {
+            f[0] *= wa[it].x; f[1] *= wa[it].y; f[2] *= wa[it].z; f[3] *= wa[it].w;
+            f[4] *= wb[it].x; f[5] *= wb[it].y; f[6] *= wb[it].z; f[7] *= wb[it].w;
+          }
+          raw = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]),
+                           pack_f16x2(f[4], f[5]), pack_f16x2(f[6], f[7]));
+        } else {
+          raw = make_uint4(0u, 0u, 0u, 0u);
+        }
+        vt[e] = raw;
+      }
+    };
+    // WG: the write-gate rows of chunk c pulled into L2 (128-byte lines
+    // spread over the conversion threads) a chunk before its conversion
+    // reads them
+    auto prefetch_w = [&](int c) {
+      if constexpr (WG) {
+        constexpr int LPR = NBV / 32;  // 128-byte lines per row
+        for (int e = ct; e < C * LPR; e += kCarryConvert) {
+          const int r = e / LPR;
+          if (c < nchunks && r < chunk_len(c))
+            prefetch_l2(wg + ((size_t)(tok0 + (int64_t)(cbeg + c) * C + r) * H + h) * DV + jv +
+                        32 * (e % LPR));
+        }
+      }
+    };
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c & 1;
+      prefetch_w(c + 1);
+      if (!wait(bar + CB_FULLA + 8 * st, (uint32_t)(c >> 1) & 1u)) { ok = 0; break; }
+      convert_v(st, c);
+      fence_proxy_async_smem();
+      mbar_arrive(bar + CB_VRDY + 8 * st);
     }
   }
 
@@ -1588,9 +1619,10 @@ carry_kernel(const __grid_constant__ CUtensorMap tm_wq, const __grid_constant__ 
     // every copy and MMA this CTA issued completes before its memory goes
     if (warp == 8 && lane == 0 && mma_pend) mbar_wait_bounded(mma_bar, mma_par, kWaitNs);
     if (warp == 9 && lane == 0) {
-      for (int s2 = 0; s2 < 2; ++s2)
-        if ((ld_pend >> s2) & 1u)
-          mbar_wait_bounded(bar + CB_FULL + 8 * s2, (ld_par >> s2) & 1u, kWaitNs);
+      for (int b2 = 0; b2 < 4; ++b2)
+        if ((ld_pend >> b2) & 1u)
+          mbar_wait_bounded(bar + ((b2 & 1) ? CB_FULLB : CB_FULLA) + 8 * (b2 >> 1),
+                            (ld_par >> b2) & 1u, kWaitNs);
     }
   }
   tc_fence_before();
