@@ -360,7 +360,8 @@ CKDA_API int ckda_fwd_chunked_fp32core(const void* q, const void* k, const void*
  * parameters, without launching anything: 1 = the tcgen05 tensor-core
  * kernels (bf16 inputs, d_k = 128, d_v in {64, 128}, chunk 64; fp16 operands
  * with fp32 accumulation; a per-chunk factor kernel over all chunks in
- * parallel, then a carry kernel per sequence, head and 64 columns of d_v),
+ * parallel, then a carry kernel per sequence, head and 64 (or 32) columns
+ * of d_v),
  * 0 = the fp32 CUDA-core kernel, or the negative
  * status an actual call with these sizes would return.  `varlen` is nonzero
  * for a packed batch (cu_seqlens given); B and T have the same meaning as in
