@@ -420,6 +420,27 @@ struct NextIn {
   int valid;  // 0: nothing to fetch
 };
 
+// sin and cos of a phase for the fp16 operands of the SFDA factor kernel.
+// Cody-Waite reduction to r = theta - n 2 pi, n = rint(theta / 2 pi), |r| <=
+// pi: 2 pi is split into 6.28125 (eight significant bits, so n * 6.28125 is
+// exact for |n| < 2^16) and the remainder, each subtracted with an fma; then
+// the hardware sine and cosine, whose absolute error on [-pi, pi] is a few
+// units of 2^-22, far below the fp16 rounding (2^-11) the values go through
+// next.  Phases beyond 1e5 take the accurate library path instead.
+__device__ __forceinline__ void phase_sincos(float th, float* s, float* c) {
+  if (fabsf(th) > 1e5f) {
+    sincosf(th, s, c);
+    return;
+  }
+  constexpr float kTwoPiHi = 6.28125f;
+  constexpr float kTwoPiLo = (float)(6.283185307179586 - 6.28125);
+  constexpr float kInvTwoPi = (float)(1.0 / 6.283185307179586);
+  const float n = rintf(th * kInvTwoPi);
+  float r = fmaf(-n, kTwoPiHi, th);
+  r = fmaf(-n, kTwoPiLo, r);
+  __sincosf(r, s, c);
+}
+
 // SFDA: turn the (alpha, theta) tiles of one quarter (alpha at F2_INA,
 // theta at F2_INA + 4096, fp32 [64 pos][16 pairs] each) into the gate tile
 // the gate pass reads, fp32 [64 pos][32] with (re, im) = alpha (cos theta,
@@ -430,10 +451,10 @@ __device__ __forceinline__ void phase_to_gates_q(uint32_t in, int tid) {
   const float4 a = lds_f4(in + F2_INA + p * 64 + 16 * j);
   const float4 th = lds_f4(in + F2_INA + 4096 + p * 64 + 16 * j);
   float s0, c0, s1, c1, s2, c2, s3, c3;
-  sincosf(th.x, &s0, &c0);
-  sincosf(th.y, &s1, &c1);
-  sincosf(th.z, &s2, &c2);
-  sincosf(th.w, &s3, &c3);
+  phase_sincos(th.x, &s0, &c0);
+  phase_sincos(th.y, &s1, &c1);
+  phase_sincos(th.z, &s2, &c2);
+  phase_sincos(th.w, &s3, &c3);
   __syncthreads();
   sts_f4(in + F2_INA + p * 128 + 32 * j, make_float4(a.x * c0, a.x * s0, a.y * c1, a.y * s1));
   sts_f4(in + F2_INA + p * 128 + 32 * j + 16, make_float4(a.z * c2, a.z * s2, a.w * c3, a.w * s3));

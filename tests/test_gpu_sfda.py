@@ -218,3 +218,24 @@ def test_tensor_core_agrees_with_the_fp32_kernel(ck):
     assert rel_max_err(o2, ro) <= TOL_F32 * 10 and rel_max_err(S2, rS) <= TOL_F32 * 10
     assert rel_max_err(o1, ro) <= TOL_BF16 and rel_max_err(S1, rS) <= TOL_BF16
     assert rel_max_err(o1, o2.double().cpu().numpy()) <= TOL_BF16
+
+
+def test_tensor_core_large_phases(ck):
+    """Phases far outside [-pi, pi]: |theta| up to about 5e3, and a quarter of
+    the channel pairs beyond 1e5.  The factor kernel reduces each phase to
+    [-pi, pi] before taking its sine and cosine (beyond 1e5 it uses the
+    accurate library routine); the oracle evaluates cos and sin of the same
+    fp32 phases in fp64."""
+    c = inputs.sfda_prefill(2, 200, 3, 128, 128, dtype=torch.bfloat16, s0_std=0.02, chunk=64,
+                            seed=71, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(72)
+    th = c.extra["theta"]
+    turns = torch.randint(-800, 800, th.shape, generator=g, device=DEV).float()
+    far = torch.randint(16000, 40000, th.shape, generator=g, device=DEV).float()
+    beyond = torch.rand(th.shape, generator=g, device=DEV) < 0.25
+    c.extra["theta"] = torch.where(beyond, th + 2 * math.pi * far,
+                                   th + 2 * math.pi * turns).contiguous()
+    assert float(c.extra["theta"].abs().max()) > 1e5
+    out, S = _run(ck, c)
+    ro, rS = _oracle(c)
+    assert rel_max_err(out, ro) <= TOL_BF16 and rel_max_err(S, rS) <= TOL_BF16
