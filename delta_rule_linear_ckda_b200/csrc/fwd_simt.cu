@@ -40,10 +40,14 @@
 //
 // One CTA owns one (sequence, head, d_v slice of width BV) and walks its
 // chunks in order; the slice of the state stays in shared memory in fp32.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace ckda {
 namespace simt {
+
+namespace cg = cooperative_groups;
 
 constexpr int kThreads = 256;
 constexpr int kMaxC = 64;
@@ -166,6 +170,25 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
   const SeqRange sr = seq_range(cu, n, n_seqs, T, status);
   if (!sr.ok) return;
 
+  // The two d_v halves of one (sequence, head) run as a cluster of two CTAs
+  // when C = 64 (see the launch): the S-independent score blocks T and A are
+  // then split between them, each computing half of the columns and writing
+  // them into both its own tiles and its partner's (distributed shared
+  // memory).  Cluster barriers replace the block barriers at the start of a
+  // chunk (neither CTA still reads the tiles the other is about to write)
+  // and after the score blocks (both halves present in both CTAs).
+  cg::cluster_group cluster = cg::this_cluster();
+  const bool pair = cluster.num_blocks() == 2;
+  const int prank = pair ? (int)cluster.block_rank() : 0;
+  float* Tm_peer = pair ? cluster.map_shared_rank(Tm, prank ^ 1) : Tm;
+  float* Am_peer = pair ? cluster.map_shared_rank(Am, prank ^ 1) : Am;
+  auto chunk_sync = [&]() {
+    if (pair)
+      cluster.sync();
+    else
+      __syncthreads();
+  };
+
   const size_t sbase = ((size_t)n * H + h) * DK * DV + j0;
   for (int e = tid; e < DK * BV / 4; e += kThreads) {
     const int i = e / (BV / 4), c4 = e % (BV / 4);
@@ -176,7 +199,7 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
 
   for (int64_t t0 = sr.begin; t0 < sr.end; t0 += C) {
     const int Lc = (sr.end - t0 < (int64_t)C) ? (int)(sr.end - t0) : C;
-    __syncthreads();  // previous chunk finished with every buffer
+    chunk_sync();  // previous chunk finished with every buffer (in both CTAs of a pair)
 
     // ---- stage inputs (fp32), identity transitions past the end ---------
     for (int e = tid; e < C * DK / 4; e += kThreads) {
@@ -266,7 +289,22 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
           for (int c = 0; c < CPL; ++c) x[c] *= a[c];
         }
       };
-      for (int s0 = warp; s0 < C; s0 += 32) {
+      // a pair splits the sixteen column quads so that each CTA's warps take
+      // one quad each with the same number of rows in total: quads s0 =
+      // 2w + r (warps 0..3) and 32 + 2 (w - 4) + 1 - r (warps 4..7) in CTA r
+      const int s_first = pair ? ((warp < 4) ? 2 * warp + prank : 32 + 2 * (warp - 4) + 1 - prank)
+                               : warp;
+      const int s_step = pair ? C : 32;
+      // a score-block entry into this CTA's tiles and, in a pair, the partner's
+      auto put = [&](int r, int s, float t, float a) {
+        Tm[r * CS + s] = t;
+        Am[r * CS + s] = a;
+        if (pair) {
+          Tm_peer[r * CS + s] = t;
+          Am_peer[r * CS + s] = a;
+        }
+      };
+      for (int s0 = s_first; s0 < C; s0 += s_step) {
         float x[4][CPL];
         // columns of this quad: diagonal of A, zeros above the diagonal
 #pragma unroll
@@ -282,8 +320,8 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
             for (int c = 0; c < CPL; ++c) d = fmaf(qs[c], x[m][c], d);
 #pragma unroll
             for (int off = 16; off >= 1; off >>= 1) d += __shfl_xor_sync(0xffffffffu, d, off);
-            if (lane == 0) { Am[s * CS + s] = d; Tm[s * CS + s] = 0.f; }
-            for (int r = lane; r < s; r += 32) { Tm[r * CS + s] = 0.f; Am[r * CS + s] = 0.f; }
+            if (lane == 0) put(s, s, 0.f, d);
+            for (int r = lane; r < s; r += 32) put(r, s, 0.f, 0.f);
           }
         }
         for (int blk = 0; s0 + 1 + 8 * blk < C; ++blk) {
@@ -325,16 +363,13 @@ fwd_simt_kernel(const Tin* __restrict__ q, const Tin* __restrict__ k, const Tin*
               reduce_scatter8(pk[m], lane);
               reduce_scatter8(pq[m], lane);
               const int s = s0 + 8 * m;
-              if (lane < 8 && r < C) {
-                Tm[r * CS + s] = G2 ? pk[m][0] : bs[r] * pk[m][0];
-                Am[r * CS + s] = pq[m][0];
-              }
+              if (lane < 8 && r < C) put(r, s, G2 ? pk[m][0] : bs[r] * pk[m][0], pq[m][0]);
             }
           }
         }
       }
     }
-    __syncthreads();
+    chunk_sync();  // (a pair: both halves of T and A in both CTAs)
 
     // ---- gate products: one thread per channel ------------------------
     // forward: Gamma_r (inclusive prefix); W rhs = beta K Gamma (G2: E Gamma);
@@ -553,11 +588,23 @@ static cudaError_t launch_t(const void* q, const void* k, const void* v, const f
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)L::kBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(DV / BV, H, n_seqs);
-  kern<<<grid, kThreads, L::kBytes, stream>>>(
-      static_cast<const Tin*>(q), static_cast<const Tin*>(k), static_cast<const Tin*>(v), alpha,
-      gt.beta, gt.b, gt.w, gt.theta, S0, cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
-  return cudaGetLastError();
+  // two d_v slices at C = 64: a cluster of the pair, which splits the score
+  // blocks (see the kernel)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(DV / BV, H, n_seqs);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (DV / BV == 2 && C == kMaxC) ? 2 : 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = attr[0].val.clusterDim.x > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<const Tin*>(q), static_cast<const Tin*>(k),
+                            static_cast<const Tin*>(v), alpha, gt.beta, gt.b, gt.w, gt.theta, S0,
+                            cu, static_cast<Tout*>(out), S_final, n_seqs, T, H, DV, C, status);
 }
 
 template <int DK, typename Tin, typename Tout, int GK>
